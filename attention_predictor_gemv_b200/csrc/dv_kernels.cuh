@@ -1,0 +1,731 @@
+// Decode-step kernels: LayerNorm, row GEMVs (dense and gathered), selection,
+// split-K decode attention and gather-axpy accumulation.
+//
+// Everything here is HBM-bound GEMV work at small batch: each weight byte is
+// used for B multiply-adds. The kernels stream whole rows with 16-byte loads,
+// keep 8 loads in flight per lane, reduce with warp shuffles, and never wait
+// on another CTA (cross-CTA steps use a last-CTA-done ticket).
+#pragma once
+
+#include "dv_common.cuh"
+
+namespace dv {
+
+// ----------------------------------------------------------------------------
+// LayerNorm: y = (x - mean) / sqrt(var + eps) * g + b, biased variance, one CTA
+// per batch row.
+// ----------------------------------------------------------------------------
+constexpr int LN_THREADS = 512;
+
+__global__ void __launch_bounds__(LN_THREADS)
+    layernorm_kernel(const float* __restrict__ x, float* __restrict__ y, int d, const float* __restrict__ g,
+                     const float* __restrict__ bta, float eps) {
+  __shared__ float red[LN_THREADS / 32];
+  griddep_launch();
+  griddep_wait();
+  const int b = blockIdx.x;
+  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)b * d);
+  float4* yr = reinterpret_cast<float4*>(y + (size_t)b * d);
+  const int n4 = d >> 2;
+  float s = 0.f;
+  for (int i = threadIdx.x; i < n4; i += LN_THREADS) {
+    float4 v = xr[i];
+    s += (v.x + v.y) + (v.z + v.w);
+  }
+  const float mean = block_sum<LN_THREADS>(s, red) / (float)d;
+  float q = 0.f;
+  for (int i = threadIdx.x; i < n4; i += LN_THREADS) {
+    float4 v = xr[i];
+    float a = v.x - mean, c = v.y - mean, e = v.z - mean, f = v.w - mean;
+    q += (a * a + c * c) + (e * e + f * f);
+  }
+  const float var = block_sum<LN_THREADS>(q, red) / (float)d;
+  const float rstd = rsqrtf(var + eps);
+  for (int i = threadIdx.x; i < n4; i += LN_THREADS) {
+    float4 v = xr[i];
+    float4 o = make_float4((v.x - mean) * rstd, (v.y - mean) * rstd, (v.z - mean) * rstd, (v.w - mean) * rstd);
+    if (g) {
+      float4 gg = reinterpret_cast<const float4*>(g)[i];
+      o.x *= gg.x; o.y *= gg.y; o.z *= gg.z; o.w *= gg.w;
+    }
+    if (bta) {
+      float4 bb = reinterpret_cast<const float4*>(bta)[i];
+      o.x += bb.x; o.y += bb.y; o.z += bb.z; o.w += bb.w;
+    }
+    yr[i] = o;
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Warp row-dot: one warp forms the dot products of RPW weight rows (K elements
+// each, 16-byte aligned) with nb <= NB fp32 input vectors X[b][0..K). U column
+// steps of RPW loads each are issued before any use: RPW * U = 8 loads of 16
+// bytes in flight per lane. On return every lane holds the full sums.
+// ----------------------------------------------------------------------------
+template <typename T, int NB, int RPW, int U>
+__device__ __forceinline__ void warp_rows_dot(const T* const (&rowp)[RPW], const bool (&valid)[RPW], int K,
+                                              const float* __restrict__ X, int ldx, int nb,
+                                              float (&acc)[RPW][NB]) {
+  constexpr int E = WT<T>::E;
+  const int lane = threadIdx.x & 31;
+  const int nvec = K / E;
+#pragma unroll
+  for (int r = 0; r < RPW; ++r)
+#pragma unroll
+    for (int b = 0; b < NB; ++b) acc[r][b] = 0.f;
+  for (int v0 = lane; v0 < nvec; v0 += 32 * U) {
+    uint4 w[U][RPW];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int v = v0 + u * 32;
+#pragma unroll
+      for (int r = 0; r < RPW; ++r) {
+        if (valid[r] && v < nvec) w[u][r] = ld_stream(rowp[r] + (size_t)v * E);
+        else w[u][r] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int v = v0 + u * 32;
+      if (v < nvec) {
+        float wf[RPW][E];
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) WT<T>::unpack(w[u][r], wf[r]);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          if (b < nb) {
+            float xv[E];
+            const float4* xp = reinterpret_cast<const float4*>(X + (size_t)b * ldx + (size_t)v * E);
+#pragma unroll
+            for (int e4 = 0; e4 < E / 4; ++e4) {
+              float4 t = __ldg(xp + e4);
+              xv[4 * e4 + 0] = t.x;
+              xv[4 * e4 + 1] = t.y;
+              xv[4 * e4 + 2] = t.z;
+              xv[4 * e4 + 3] = t.w;
+            }
+#pragma unroll
+            for (int r = 0; r < RPW; ++r)
+#pragma unroll
+              for (int e = 0; e < E; ++e) acc[r][b] = fmaf(wf[r][e], xv[e], acc[r][b]);
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < RPW; ++r)
+#pragma unroll
+    for (int b = 0; b < NB; ++b) acc[r][b] = warp_sum(acc[r][b]);
+}
+
+constexpr int GEMV_WARPS = 8;
+constexpr int GEMV_THREADS = GEMV_WARPS * 32;
+
+// Dense GEMV over rows 0..nrows-1 of W [nrows][K]: out[b][i] = W[i] . X[b] + bias[i].
+template <typename T, int NB, int RPW, int U>
+__global__ void __launch_bounds__(GEMV_THREADS)
+    dense_gemv_kernel(const T* __restrict__ W, int nrows, int K, const float* __restrict__ X, int ldx, int nb,
+                      const float* __restrict__ bias, float* __restrict__ out, int ldo) {
+  griddep_launch();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row0 = (blockIdx.x * GEMV_WARPS + warp) * RPW;
+  const T* rowp[RPW];
+  bool valid[RPW];
+#pragma unroll
+  for (int r = 0; r < RPW; ++r) {
+    valid[r] = row0 + r < nrows;
+    rowp[r] = W + (size_t)(valid[r] ? row0 + r : 0) * K;
+  }
+  griddep_wait();  // X comes from the previous kernel
+  float acc[RPW][NB];
+  warp_rows_dot<T, NB, RPW, U>(rowp, valid, K, X, ldx, nb, acc);
+#pragma unroll
+  for (int r = 0; r < RPW; ++r)
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+      if (lane == ((r * NB + b) & 31) && valid[r] && b < nb)
+        out[(size_t)b * ldo + row0 + r] = acc[r][b] + (bias ? bias[row0 + r] : 0.f);
+}
+
+// ----------------------------------------------------------------------------
+// Sparse W1 GEMV + b1 + ReLU + compaction (eq. (1), first factor).
+// CTA c owns selection slots [c*SEG, (c+1)*SEG), SEG = GEMV_WARPS * RPW. It
+// writes the slots whose activation is nonzero in some batch row, in slot
+// order, to seg_idx / seg_a at the segment's base and their number to
+// seg_cnt[c]. Compaction is thus deterministic: the consumer forms the
+// prefix sum over seg_cnt.
+// ----------------------------------------------------------------------------
+template <typename T, int NB, int RPW, int U>
+__global__ void __launch_bounds__(GEMV_THREADS)
+    mlp_up_kernel(const T* __restrict__ W1t, int d, int N, const float* __restrict__ X, int nb,
+                  const float* __restrict__ b1, const int32_t* __restrict__ idx, const int32_t* __restrict__ count_dev,
+                  int k_max, int32_t* __restrict__ seg_idx, float* __restrict__ seg_a, int32_t* __restrict__ seg_cnt,
+                  int* __restrict__ status) {
+  constexpr int SEG = GEMV_WARPS * RPW;
+  __shared__ float s_a[SEG][NB];
+  __shared__ int s_row[SEG];
+  __shared__ int s_nz[SEG];
+  griddep_launch();
+  griddep_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int cnt = *count_dev;
+  if (cnt > k_max || cnt < 0) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(status, 1);
+    cnt = cnt < 0 ? 0 : k_max;
+  }
+  const int slot0 = blockIdx.x * SEG + warp * RPW;
+  const T* rowp[RPW];
+  bool valid[RPW];
+  int rows[RPW];
+#pragma unroll
+  for (int r = 0; r < RPW; ++r) {
+    const int slot = slot0 + r;
+    int row = slot < cnt ? idx[slot] : -1;
+    if (slot < cnt && (row < 0 || row >= N)) {
+      if (lane == 0) raise_status(status, 2);
+      row = -1;
+    }
+    rows[r] = row;
+    valid[r] = row >= 0;
+    rowp[r] = W1t + (size_t)(row >= 0 ? row : 0) * d;
+  }
+  float acc[RPW][NB];
+  warp_rows_dot<T, NB, RPW, U>(rowp, valid, d, X, d, nb, acc);
+  if (lane == 0) {
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+      int nz = 0;
+      const float bias = valid[r] ? b1[rows[r]] : 0.f;
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const float a = (valid[r] && b < nb) ? fmaxf(acc[r][b] + bias, 0.f) : 0.f;
+        s_a[warp * RPW + r][b] = a;
+        nz |= a > 0.f;
+      }
+      s_nz[warp * RPW + r] = nz;
+      s_row[warp * RPW + r] = rows[r];
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int base = 0;
+#pragma unroll
+    for (int c0 = 0; c0 < SEG; c0 += 32) {
+      const int j = c0 + lane;
+      const int nz = (j < SEG) ? s_nz[j] : 0;
+      const unsigned bal = __ballot_sync(0xffffffffu, nz);
+      if (nz) {
+        const int p = blockIdx.x * SEG + base + __popc(bal & ((1u << lane) - 1u));
+        seg_idx[p] = s_row[j];
+        for (int b = 0; b < nb; ++b) seg_a[(size_t)p * nb + b] = s_a[j][b];
+      }
+      base += __popc(bal);
+    }
+    if (lane == 0) seg_cnt[blockIdx.x] = base;
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Sparse-head Q/K/V projection + KV append (eq. (2); the itpub KV-cache figure).
+// Slot s in [0, hc*3*dh): p = s / (3 dh) indexes head_idx, m = (s / dh) % 3
+// picks q/k/v, c = s % dh the channel. q goes to the workspace (fp32); k and v
+// are rounded to the cache dtype and written at slot `pos`.
+// ----------------------------------------------------------------------------
+template <typename T, int NB, int RPW, int U>
+__global__ void __launch_bounds__(GEMV_THREADS)
+    qkv_kernel(const T* __restrict__ Wqkv, int d, int h, int dh, const float* __restrict__ X, int nb,
+               const float* __restrict__ bqkv, const int32_t* __restrict__ head_idx,
+               const int32_t* __restrict__ head_count, int kh_max, float* __restrict__ q, T* __restrict__ Kc,
+               T* __restrict__ Vc, int cap, int pos, int* __restrict__ status) {
+  griddep_launch();
+  griddep_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int hc = *head_count;
+  if (hc > kh_max || hc < 0) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(status, 1);
+    hc = hc < 0 ? 0 : kh_max;
+  }
+  const int per = 3 * dh;
+  const int nslot = hc * per;
+  const int slot0 = (blockIdx.x * GEMV_WARPS + warp) * RPW;
+  const T* rowp[RPW];
+  bool valid[RPW];
+  int heads[RPW];
+#pragma unroll
+  for (int r = 0; r < RPW; ++r) {
+    const int slot = slot0 + r;
+    int head = -1;
+    if (slot < nslot) {
+      head = head_idx[slot / per];
+      if (head < 0 || head >= h) {
+        if (lane == 0) raise_status(status, 2);
+        head = -1;
+      }
+    }
+    heads[r] = head;
+    valid[r] = head >= 0;
+    rowp[r] = Wqkv + ((size_t)(head >= 0 ? head : 0) * per + (slot % per)) * d;
+  }
+  float acc[RPW][NB];
+  warp_rows_dot<T, NB, RPW, U>(rowp, valid, d, X, d, nb, acc);
+#pragma unroll
+  for (int r = 0; r < RPW; ++r) {
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (lane == ((r * NB + b) & 31) && valid[r] && b < nb) {
+        const int slot = slot0 + r;
+        const int p = slot / per, rem = slot % per, m = rem / dh, c = rem % dh;
+        float v = acc[r][b];
+        if (bqkv) v += bqkv[(size_t)heads[r] * per + rem];
+        if (m == 0) {
+          q[((size_t)b * kh_max + p) * dh + c] = v;
+        } else {
+          T* cache = (m == 1) ? Kc : Vc;
+          cache[(((size_t)b * h + heads[r]) * cap + pos) * dh + c] = WT<T>::store_cvt(v);
+        }
+      }
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Selection: per-row top-k by radix select on order-preserving keys, or a
+// strict threshold; the union over rows, compacted to ascending indices.
+// One CTA per score row writes its selection bitmap; the last CTA to finish
+// (ticket) ORs the bitmaps and writes idx / count, then resets the ticket.
+// ----------------------------------------------------------------------------
+constexpr int SEL_THREADS = 1024;
+constexpr int SEL_SMEM_KEYS = 49152;  // rows up to this length keep keys in shared memory
+
+// Order-preserving map float -> uint32: larger float, larger key. -0.0 maps
+// like +0.0; every NaN maps to 0, below -inf (0x007fffff).
+__device__ __forceinline__ uint32_t ord_key(float s) {
+  uint32_t u = __float_as_uint(s);
+  if (s != s) return 0u;
+  if ((u << 1) == 0u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+template <bool KEYS_IN_SMEM>
+__global__ void __launch_bounds__(SEL_THREADS)
+    select_kernel(const float* __restrict__ scores, int n, int nrows, int k, float tau, int mode,
+                  uint32_t* __restrict__ bitmaps, unsigned* __restrict__ ticket, int32_t* __restrict__ idx,
+                  int32_t* __restrict__ count) {
+  extern __shared__ uint32_t s_keys[];
+  __shared__ unsigned hist[256];
+  __shared__ unsigned sc[SEL_THREADS / 32 + 1];
+  __shared__ unsigned s_digit, s_kk, s_last;
+  griddep_launch();
+  griddep_wait();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b = blockIdx.x;
+  const float* row = scores + (size_t)b * n;
+  const int nw = (n + 31) >> 5;
+  uint32_t* bm = bitmaps + (size_t)b * nw;
+  const int wpt = (nw + SEL_THREADS - 1) / SEL_THREADS;  // bitmap words per thread
+  const int w0 = tid * wpt, w1 = min(nw, w0 + wpt);
+
+  if (mode == 1) {  // threshold: s > tau (NaN fails)
+    for (int w = w0; w < w1; ++w) {
+      uint32_t word = 0;
+      for (int j = 0; j < 32; ++j) {
+        const int i = w * 32 + j;
+        if (i < n && row[i] > tau) word |= 1u << j;
+      }
+      bm[w] = word;
+    }
+  } else if (k >= n || k <= 0) {
+    for (int w = w0; w < w1; ++w) {
+      uint32_t word = 0;
+      if (k > 0) {
+        const int rem = n - w * 32;
+        word = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
+      }
+      bm[w] = word;
+    }
+  } else {
+    if (KEYS_IN_SMEM) {
+      for (int i = tid; i < n; i += SEL_THREADS) s_keys[i] = ord_key(row[i]);
+    }
+    __syncthreads();
+    uint32_t prefix = 0, mask = 0;
+    unsigned kk = (unsigned)k;
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      for (int i = tid; i < 256; i += SEL_THREADS) hist[i] = 0;
+      __syncthreads();
+      for (int base = 0; base < n; base += SEL_THREADS) {
+        const int i = base + tid;
+        unsigned dig = 256u;
+        if (i < n) {
+          const uint32_t key = KEYS_IN_SMEM ? s_keys[i] : ord_key(row[i]);
+          if ((key & mask) == prefix) dig = (key >> shift) & 255u;
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, dig);
+        if (dig < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[dig], (unsigned)__popc(peers));
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // lane l scans digits 255-8l down to 248-8l
+        unsigned c[8], tot = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          c[j] = hist[255 - 8 * lane - j];
+          tot += c[j];
+        }
+        unsigned incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        const unsigned excl = incl - tot;
+        if (excl < kk && kk <= incl) {
+          unsigned cum = excl;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (cum + c[j] >= kk) {
+              s_digit = 255u - 8u * lane - j;
+              s_kk = kk - cum;
+              break;
+            }
+            cum += c[j];
+          }
+        }
+      }
+      __syncthreads();
+      prefix |= s_digit << shift;
+      mask |= 255u << shift;
+      kk = s_kk;
+      __syncthreads();
+    }
+    // prefix is the k-th largest key; kk of its copies are taken, lowest
+    // indices first. Ranks among equal keys come from a block scan in index
+    // order (thread t owns words [w0, w1)).
+    unsigned eq = 0;
+    for (int i = w0 * 32; i < min(n, w1 * 32); ++i) {
+      const uint32_t key = KEYS_IN_SMEM ? s_keys[i] : ord_key(row[i]);
+      eq += key == prefix;
+    }
+    unsigned tot;
+    unsigned rank = block_exclusive_scan<SEL_THREADS>(eq, sc, &tot);
+    for (int w = w0; w < w1; ++w) {
+      uint32_t word = 0;
+      for (int j = 0; j < 32; ++j) {
+        const int i = w * 32 + j;
+        if (i < n) {
+          const uint32_t key = KEYS_IN_SMEM ? s_keys[i] : ord_key(row[i]);
+          if (key > prefix || (key == prefix && rank++ < kk)) word |= 1u << j;
+        }
+      }
+      bm[w] = word;
+    }
+  }
+  // union over rows by the last CTA
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(ticket, 1u) == (unsigned)nrows - 1u);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  unsigned pc = 0;
+  for (int w = w0; w < w1; ++w) {
+    uint32_t u = 0;
+    for (int rr = 0; rr < nrows; ++rr) u |= __ldcg(bitmaps + (size_t)rr * nw + w);
+    pc += __popc(u);
+  }
+  unsigned total;
+  unsigned off = block_exclusive_scan<SEL_THREADS>(pc, sc, &total);
+  for (int w = w0; w < w1; ++w) {
+    uint32_t u = 0;
+    for (int rr = 0; rr < nrows; ++rr) u |= __ldcg(bitmaps + (size_t)rr * nw + w);
+    while (u) {
+      const int j = __ffs(u) - 1;
+      u &= u - 1u;
+      idx[off++] = w * 32 + j;
+    }
+  }
+  if (tid == 0) {
+    *count = (int32_t)total;
+    *ticket = 0u;
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Split-K decode attention over the selected heads (eq. (2), D_i normalised,
+// max-subtracted). CTA (s, p, b) handles keys [s*S, min(s*S+S, pos+1)) of
+// head head_idx[p], batch row b: it stages its K and V tiles in shared memory
+// with cp.async (all loads in flight at once), forms the scores, and writes
+// the partial (m, l, acc[dh]). The last split to finish for (b, p) combines
+// the partials into H[b][p][:].
+// ----------------------------------------------------------------------------
+constexpr int ATTN_THREADS = 128;
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+template <typename KT, int DH, int S>
+__global__ void __launch_bounds__(ATTN_THREADS)
+    attn_split_kernel(const float* __restrict__ q, const KT* __restrict__ Kc, const KT* __restrict__ Vc, int h, int cap,
+                      int pos, float scale, const int32_t* __restrict__ head_idx,
+                      const int32_t* __restrict__ head_count, int kh_max, int nsplit, float* __restrict__ part,
+                      unsigned* __restrict__ ctr, float* __restrict__ H, int* __restrict__ status) {
+  constexpr int E = WT<KT>::E;        // elements per 16-byte vector
+  constexpr int G = DH / E;           // lanes per key row
+  constexpr int KPP = ATTN_THREADS / G;  // keys per pass
+  __shared__ __align__(16) KT sK[S * DH];
+  __shared__ __align__(16) KT sV[S * DH];
+  __shared__ float sE[S];
+  __shared__ float sRed[KPP * DH];
+  __shared__ float red[ATTN_THREADS / 32];
+  __shared__ unsigned s_last;
+  griddep_launch();
+  griddep_wait();
+  const int s = blockIdx.x, p = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  int hc = *head_count;
+  hc = hc < 0 ? 0 : (hc > kh_max ? kh_max : hc);
+  if (p >= hc) return;
+  const int head = head_idx[p];
+  if (head < 0 || head >= h) {
+    if (tid == 0 && s == 0) raise_status(status, 2);
+    return;
+  }
+  const int t0 = s * S;
+  const int nk = min(S, pos + 1 - t0);
+  const size_t base = (((size_t)b * h + head) * cap + t0) * DH;
+  {
+    const int nvec = nk * DH / E;
+    for (int v = tid; v < nvec; v += ATTN_THREADS) {
+      cp_async16(sK + v * E, Kc + base + (size_t)v * E);
+      cp_async16(sV + v * E, Vc + base + (size_t)v * E);
+    }
+  }
+  const int g = tid % G, j = tid / G;
+  float qv[E];
+  {
+    const float* qp = q + ((size_t)b * kh_max + p) * DH + g * E;
+#pragma unroll
+    for (int e = 0; e < E; ++e) qv[e] = qp[e] * scale;
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  // scores
+  for (int t = j; t < nk; t += KPP) {
+    float kf[E];
+    WT<KT>::unpack(*reinterpret_cast<const uint4*>(sK + t * DH + g * E), kf);
+    float dot = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) dot = fmaf(qv[e], kf[e], dot);
+#pragma unroll
+    for (int o = G / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    if (g == 0) sE[t] = dot;
+  }
+  __syncthreads();
+  float m = -INFINITY;
+  for (int t = tid; t < nk; t += ATTN_THREADS) m = fmaxf(m, sE[t]);
+  m = block_max<ATTN_THREADS>(m, red);
+  float l = 0.f;
+  for (int t = tid; t < nk; t += ATTN_THREADS) {
+    const float pe = __expf(sE[t] - m);
+    sE[t] = pe;
+    l += pe;
+  }
+  l = block_sum<ATTN_THREADS>(l, red);  // ends with a barrier: sE is final
+  float acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  for (int t = j; t < nk; t += KPP) {
+    float vf[E];
+    WT<KT>::unpack(*reinterpret_cast<const uint4*>(sV + t * DH + g * E), vf);
+    const float pe = sE[t];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = fmaf(pe, vf[e], acc[e]);
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) sRed[j * DH + g * E + e] = acc[e];
+  __syncthreads();
+  float* pp = part + (((size_t)b * kh_max + p) * nsplit + s) * (DH + 2);
+  for (int c = tid; c < DH; c += ATTN_THREADS) {
+    float a = 0.f;
+#pragma unroll
+    for (int jj = 0; jj < KPP; ++jj) a += sRed[jj * DH + c];
+    pp[2 + c] = a;
+  }
+  if (tid == 0) {
+    pp[0] = m;
+    pp[1] = l;
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(ctr + (size_t)b * kh_max + p, 1u) == (unsigned)nsplit - 1u);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const float* p0 = part + ((size_t)b * kh_max + p) * nsplit * (DH + 2);
+  float M = -INFINITY;
+  for (int ss = 0; ss < nsplit; ++ss) M = fmaxf(M, __ldcg(p0 + (size_t)ss * (DH + 2)));
+  float den = 0.f;
+  for (int ss = 0; ss < nsplit; ++ss) {
+    const float* ps = p0 + (size_t)ss * (DH + 2);
+    den += __expf(__ldcg(ps) - M) * __ldcg(ps + 1);
+  }
+  for (int c = tid; c < DH; c += ATTN_THREADS) {
+    float num = 0.f;
+    for (int ss = 0; ss < nsplit; ++ss) {
+      const float* ps = p0 + (size_t)ss * (DH + 2);
+      num += __expf(__ldcg(ps) - M) * __ldcg(ps + 2 + c);
+    }
+    H[((size_t)b * kh_max + p) * DH + c] = num / den;
+  }
+  if (tid == 0) ctr[(size_t)b * kh_max + p] = 0u;
+}
+
+// ----------------------------------------------------------------------------
+// Gather-axpy: out[b][:] += sum_p coef[p][b] * W[row(p)][:] over a device-sized
+// list of rows. Grid (column tiles, G): CTA (x, y) owns columns
+// [x*AX_THREADS*E, ...) and list positions [total*y/G, total*(y+1)/G). Rows are
+// streamed with U 16-byte loads in flight per thread; the CTA's partial sums
+// are added to out with vector float atomics. The CTA with y == 0 adds bias.
+//
+// Row sources: RowsMlp (compacted neurons from mlp_up_kernel's segments; eq.
+// (1), second factor) and RowsHeads (rows c of W_i^O for i in S_A; eq. (2)).
+// ----------------------------------------------------------------------------
+constexpr int AX_THREADS = 128;
+constexpr int AX_CHUNK = 256;
+constexpr int AX_U = 8;
+
+struct RowsMlp {
+  const int32_t* seg_idx;
+  const float* seg_a;
+  const int32_t* seg_cnt;
+  int nseg, SEG;
+  // Builds the prefix sums of the segment counts in s_off[0..nseg]; returns the total.
+  __device__ int prologue(int* s_off, unsigned* sc) const {
+    unsigned run = 0;
+    for (int base = 0; base < nseg; base += AX_THREADS) {
+      const int i = base + threadIdx.x;
+      const unsigned c = i < nseg ? (unsigned)seg_cnt[i] : 0u;
+      unsigned tot;
+      const unsigned ex = block_exclusive_scan<AX_THREADS>(c, sc, &tot);
+      if (i < nseg) s_off[i] = (int)(run + ex);
+      run += tot;
+    }
+    if (threadIdx.x == 0) s_off[nseg] = (int)run;
+    __syncthreads();
+    return (int)run;
+  }
+  __device__ int row(int pidx, const int* s_off) const {
+    int lo = 0, hi = nseg - 1;  // last segment with s_off[seg] <= pidx
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_off[mid] <= pidx) lo = mid;
+      else hi = mid - 1;
+    }
+    return lo * SEG + (pidx - s_off[lo]);  // slot
+  }
+  __device__ int row_of_slot(int slot) const { return seg_idx[slot]; }
+  __device__ float coef(int slot, int b, int nb) const { return seg_a[(size_t)slot * nb + b]; }
+};
+
+struct RowsHeads {
+  const int32_t* head_idx;
+  const int32_t* head_count;
+  const float* Hbuf;  // [B][kh_max][dh]
+  int kh_max, dh, h;
+  __device__ int prologue(int*, unsigned*) const {
+    int hc = *head_count;
+    hc = hc < 0 ? 0 : (hc > kh_max ? kh_max : hc);
+    return hc * dh;
+  }
+  __device__ int row(int pidx, const int*) const { return pidx; }
+  __device__ int row_of_slot(int slot) const {
+    const int head = head_idx[slot / dh];
+    return (head < 0 || head >= h) ? -1 : head * dh + slot % dh;
+  }
+  __device__ float coef(int slot, int b, int) const {
+    return Hbuf[((size_t)b * kh_max + slot / dh) * dh + slot % dh];
+  }
+};
+
+template <typename T, int NB, class Src>
+__global__ void __launch_bounds__(AX_THREADS)
+    axpy_rows_kernel(const T* __restrict__ W, int d, int nrows_w, Src src, const float* __restrict__ bias,
+                     float* __restrict__ out, int nb, int G, int* __restrict__ status) {
+  constexpr int E = WT<T>::E;
+  extern __shared__ int s_off[];
+  __shared__ int s_rows[AX_CHUNK];
+  __shared__ float s_coef[AX_CHUNK][NB];
+  __shared__ unsigned sc[AX_THREADS / 32 + 1];
+  griddep_launch();
+  griddep_wait();
+  const int tid = threadIdx.x;
+  const int total = src.prologue(s_off, sc);
+  const int p0 = (int)(((long long)total * blockIdx.y) / G);
+  const int p1 = (int)(((long long)total * (blockIdx.y + 1)) / G);
+  const int col = (blockIdx.x * AX_THREADS + tid) * E;
+  const bool colok = col < d;
+  float acc[NB][E];
+#pragma unroll
+  for (int b = 0; b < NB; ++b)
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[b][e] = (bias && blockIdx.y == 0 && colok && b < nb) ? bias[col + e] : 0.f;
+  for (int c0 = p0; c0 < p1; c0 += AX_CHUNK) {
+    const int n = min(AX_CHUNK, p1 - c0);
+    for (int i = tid; i < n; i += AX_THREADS) {
+      const int slot = src.row(c0 + i, s_off);
+      int row = src.row_of_slot(slot);
+      if (row < 0 || row >= nrows_w) {
+        raise_status(status, 2);
+        row = -1;
+      }
+      s_rows[i] = row;
+#pragma unroll
+      for (int b = 0; b < NB; ++b) s_coef[i][b] = (row >= 0 && b < nb) ? src.coef(slot, b, nb) : 0.f;
+    }
+    __syncthreads();
+    for (int i0 = 0; i0 < n; i0 += AX_U) {
+      uint4 w[AX_U];
+#pragma unroll
+      for (int u = 0; u < AX_U; ++u) {
+        const int i = i0 + u;
+        const int row = (i < n) ? s_rows[i] : -1;
+        w[u] = (colok && row >= 0) ? ld_stream(W + (size_t)row * d + col) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < AX_U; ++u) {
+        const int i = i0 + u;
+        if (i < n) {
+          float wf[E];
+          WT<T>::unpack(w[u], wf);
+#pragma unroll
+          for (int b = 0; b < NB; ++b) {
+            const float cb = s_coef[i][b];
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc[b][e] = fmaf(cb, wf[e], acc[b][e]);
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
+  if (colok && (p1 > p0 || (bias && blockIdx.y == 0))) {
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (b < nb) {
+#pragma unroll
+        for (int e4 = 0; e4 < E / 4; ++e4) {
+          float4 v = make_float4(acc[b][4 * e4], acc[b][4 * e4 + 1], acc[b][4 * e4 + 2], acc[b][4 * e4 + 3]);
+          atomicAdd(reinterpret_cast<float4*>(out + (size_t)b * d + col + 4 * e4), v);
+        }
+      }
+    }
+  }
+}
+
+}  // namespace dv

@@ -121,7 +121,7 @@ def svd_predictor(W1t_f32: torch.Tensor, r: int):
     Returns At = (U_r S_r)^T [r][d] and Bm = V_r [N][r]."""
     W1 = W1t_f32.t()  # d x N
     d, N = W1.shape
-    if W1.is_cuda and r < min(d, N) // 2:
+    if r < min(d, N) // 2:
         U, S, V = torch.svd_lowrank(W1, q=min(r + 32, min(d, N)), niter=3)
         U, S, V = U[:, :r], S[:r], V[:, :r]
     else:

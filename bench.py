@@ -1,0 +1,419 @@
+"""Benchmark: one decode step of an OPT-1.3B-shaped decoder (24 layers of the
+d=2048, N=8192, h=32, dh=64 layer, KV length 512, batch 1, bf16 weights,
+fp32 accumulation) with contextual sparsity: the look-ahead predictors, top-k
+selection, sparse MHA over the selected heads and sparse MLP over the
+selected neurons, through the C ABI.
+
+Metric: microseconds per decode step per layer (lower is better), with the
+effective HBM bandwidth on the selected bytes. The 24 layers hold 2.6 GB of
+weights, more than L2 (126 MB), so every step streams its selected bytes
+from HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+For N > 1 (torchrun) every rank runs an independent replica (the path has
+no exchange step); the time is the maximum over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from attention_predictor_gemv_b200 import accounting as acct  # noqa: E402
+from attention_predictor_gemv_b200 import workload as wl  # noqa: E402
+
+METRIC = "us/decode-step/layer"
+CONFIG = "opt-1.3b"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--layers", type=int, default=24)
+    ap.add_argument("--k-frac", type=float, default=0.10)
+    ap.add_argument("--kh-frac", type=float, default=0.25)
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--no-lookahead", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas only: barrier and max-over-ranks timing)
+# ---------------------------------------------------------------------------
+
+
+def dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws <= 1:
+        return 0, 1, None
+    import datetime
+
+    import torch.distributed as dist
+
+    rank = int(os.environ["RANK"])
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    return rank, ws, dist
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(v, dist):
+    if dist is None:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_index: int):
+        self.dev = dev_index
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "100"], stdout=subprocess.PIPE,
+                                      stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.p = None
+        time.sleep(0.25)
+        return self
+
+    def __exit__(self, *a):
+        time.sleep(0.15)
+        self.out = ""
+        if self.p is not None:
+            self.p.terminate()
+            try:
+                self.out, _ = self.p.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.p.kill()
+                self.out = ""
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+
+
+def build_stack(shape, nlayers, B, k, k_h, lookahead, seed0=1000, layers=None):
+    from attention_predictor_gemv_b200.stack import DecoderStack
+
+    if layers is None:
+        layers = [wl.make_layer(shape, seed0 + l, "cuda") for l in range(nlayers)]
+    stk = DecoderStack(layers, B, k, k_h, 1.0 / float(np.sqrt(shape.dh)), lookahead=lookahead)
+    return stk, layers
+
+
+def capture(stk, x, pos):
+    from attention_predictor_gemv_b200 import binding as bd
+
+    stk.step(x, pos)  # eager warm-up (sets attributes, loads modules)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    n0 = bd.dv_launch_count()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            stk.step(x, pos)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    return g, bd.dv_launch_count() - n0
+
+
+def time_graph(g, steps, warmup, dist):
+    for _ in range(warmup):
+        g.replay()
+    barrier(dist)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        g.replay()
+    e1.record()
+    e1.synchronize()
+    barrier(dist)
+    return e0.elapsed_time(e1) / steps  # ms per step
+
+
+def selected_counts(stk):
+    """Mean k (selected neurons), k' (nonzero activations) and k_h over layers."""
+    ks, khs = [], []
+    for l in range(len(stk.layers)):
+        ks.append(int(stk.count[l].item()))
+        khs.append(int(stk.head_count[l].item()))
+    return float(np.mean(ks)), float(np.mean(khs))
+
+
+def nonzero_neurons(stk):
+    """k' per layer: selected neurons with a nonzero activation, read from the
+    workspace-independent recomputation y_M . W1 + b1 on the device (torch)."""
+    kp = []
+    for l, L in enumerate(stk.layers):
+        c = int(stk.count[l].item())
+        idx = stk.idx[l][:c].long()
+        pre = stk.yM[l] @ L.t["W1t"][idx].float().t() + L.t["b1"][idx]
+        kp.append(int((pre > 0).any(dim=0).sum().item()))
+    return float(np.mean(kp))
+
+
+def layer_bytes(shape, k, kp, kh, B):
+    return acct.layer_bytes(shape.d, shape.N, shape.r, shape.h, shape.dh, int(round(k)), int(round(kp)),
+                            int(round(kh)), B, shape.L + 1)
+
+
+def op_roofline(stk, shape, B, pos, peak_gbs):
+    """Times each library call of one layer-step over all layers with CUDA
+    events on the launching stream (weights of 24 layers: HBM-cold), and
+    returns the per-op average duration and effective bandwidth."""
+    from attention_predictor_gemv_b200 import binding as bd
+
+    st = torch.cuda.current_stream()
+    nL = len(stk.layers)
+    res = {}
+    x = torch.randn(B, shape.d, device="cuda")
+    ws = stk.ws_main
+    out = torch.empty(B, shape.d, device="cuda")
+
+    def timed(name, fn, nbytes):
+        for _ in range(2):
+            for l in range(nL):
+                fn(l)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        reps = 5
+        for _ in range(reps):
+            for l in range(nL):
+                fn(l)
+        e1.record(st)
+        e1.synchronize()
+        us = e0.elapsed_time(e1) * 1000.0 / (reps * nL)
+        res[name] = {"us": us, "bytes": nbytes, "gbs": nbytes / us / 1e3, "frac": nbytes / us / 1e3 / peak_gbs}
+
+    kp = nonzero_neurons(stk)
+    k, kh = selected_counts(stk)
+    lb = layer_bytes(shape, k, kp, kh, B)
+    p = stk.p
+    timed("dv_predict_heads", lambda l: bd.dv_predict_heads(stk.yA[l], stk.layers[l].t["PA"], p.k_h, stk.scores_h[l],
+                                                            stk.head_idx[l], stk.head_count[l], ws), lb.head_predictor)
+    timed("dv_predict_mlp", lambda l: bd.dv_predict_mlp(stk.yM[l], stk.layers[l].t["At"], stk.layers[l].t["Bm"],
+                                                        stk.layers[l].t["b1"], p.k, stk.scores[l], stk.idx[l],
+                                                        stk.count[l], ws), lb.mlp_predictor)
+    timed("dv_sparse_mha", lambda l: bd.dv_sparse_mha(stk.yA[l], stk.layers[l].t["Wqkv"], None,
+                                                      stk.layers[l].t["WOt"], None, stk.layers[l].t["K"],
+                                                      stk.layers[l].t["V"], pos, p.scale, stk.head_idx[l],
+                                                      stk.head_count[l], stk.kh_max, out, ws),
+          lb.qkv + lb.wo + lb.kv)
+    timed("dv_sparse_mlp", lambda l: bd.dv_sparse_mlp(stk.yM[l], stk.layers[l].t["W1t"], stk.layers[l].t["b1"],
+                                                      stk.layers[l].t["W2t"], None, stk.idx[l], stk.count[l],
+                                                      stk.k_max, out, ws), lb.w1 + lb.w2)
+    return res, lb, k, kp, kh
+
+
+def cpu_baseline(shape, B, k, k_h, seconds, seed=1000):
+    """The oracle (float64 numpy) on a bounded sample: repeated layer-steps of
+    one layer of the same shape, on the host cores."""
+    from threadpoolctl import threadpool_info
+
+    from oracle import dejavu_oracle as O
+
+    t = wl.make_layer(shape, seed, "cpu")
+    f = lambda a: O.bf16_bits_to_f64(a.contiguous().view(torch.int16).numpy().view(np.uint16)) \
+        if a.dtype == torch.bfloat16 else a.double().numpy()  # noqa: E731
+    L = O.LayerF64(PA=f(t["PA"]), Wqkv=f(t["Wqkv"]), bqkv=None, WOt=f(t["WOt"]), bO=None, K=f(t["K"]), V=f(t["V"]),
+                   At=f(t["At"]), Bm=f(t["Bm"]), b1=f(t["b1"]), W1t=f(t["W1t"]), W2t=f(t["W2t"]))
+    P = O.LayerParams(k=k, k_h=k_h, scale=1.0 / float(np.sqrt(shape.dh)))
+    x = wl.make_input(shape, 0, "cpu").double().numpy()
+    n, t0 = 0, time.perf_counter()
+    while True:
+        O.decode_layer(x, L, P, shape.L)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return {"value": el * 1e6 / n, "unit": "us/layer-step", "cores": int(threads), "kind": "oracle",
+            "sample": f"{n} layer-steps of one {CONFIG}-shaped layer (d={shape.d}, N={shape.N}, h={shape.h}, "
+                      f"dh={shape.dh}, KV {shape.L}+1, B={B}, k={k}, k_h={k_h}), float64 numpy, full layer "
+                      f"(LN, predictors, selection, sparse MHA, sparse MLP)"}
+
+
+def run_reference(args, rank, dist):
+    shape = wl.CONFIGS[CONFIG].with_(B=args.batch)
+    k, k_h = wl.k_for(args.k_frac, shape.N), wl.k_for(args.kh_frac, shape.h)
+    if rank != 0:
+        return
+    per_step = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+    cb = cpu_baseline(shape, args.batch, k, k_h, min(per_step, 10.0))
+    v = cb["value"]
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "us", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v * args.layers / 1e3,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{CONFIG}-shaped decoder layer, batch {args.batch}, KV {shape.L}, "
+                                   f"k={k}/{shape.N}, k_h={k_h}/{shape.h}", "layers": args.layers},
+            "cpu_baseline": cb, "e2e": {"value": v, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world, dist = dist_init()
+    if args.impl == "reference":
+        run_reference(args, rank, dist)
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+    from attention_predictor_gemv_b200 import binding as bd
+
+    dev = torch.cuda.current_device()
+    peaks = {}
+    pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pk):
+        with open(pk) as f:
+            peaks = json.load(f)
+    peak_gbs = float(peaks.get("hbm_gbs", 6650.0))
+    peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
+
+    B = args.batch
+    shape = wl.CONFIGS[CONFIG].with_(B=B)
+    k, k_h = wl.k_for(args.k_frac, shape.N), wl.k_for(args.kh_frac, shape.h)
+    pos = shape.L
+    torch.manual_seed(rank)
+    stk, layers = build_stack(shape, args.layers, B, k, k_h, not args.no_lookahead, seed0=1000 + 100 * rank)
+    x0 = wl.make_input(shape, 7 + rank, "cuda")
+    x = x0.clone()
+    g, launches_per_step = capture(stk, x, pos)
+
+    with Clocks(dev) as clk:
+        ms = time_graph(g, args.steps, args.warmup, dist)
+    ms = max_over_ranks(ms, dist)
+    clocks = clk.summary()
+
+    # end to end: pinned host input -> device, step, device -> host result
+    xh = torch.empty(B, shape.d, dtype=torch.float32, pin_memory=True)
+    xh.copy_(x0.cpu())
+    oh = torch.empty_like(xh).pin_memory()
+    for _ in range(max(1, args.warmup)):
+        x.copy_(xh, non_blocking=True)
+        g.replay()
+        oh.copy_(x, non_blocking=True)
+    barrier(dist)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        x.copy_(xh, non_blocking=True)
+        g.replay()
+        oh.copy_(x, non_blocking=True)
+    e1.record()
+    e1.synchronize()
+    barrier(dist)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist)
+
+    ops, lb, kmean, kp, kh = op_roofline(stk, shape, B, pos, peak_gbs)
+    dom = max(ops, key=lambda n: ops[n]["us"])
+    total_layer_bytes = lb.total
+    us_layer = ms * 1e3 / args.layers
+    value = ms * 1e3 / (args.layers * world)  # whole job: all ranks' layer-steps in the max-over-ranks time
+
+    sweep = []
+    if not args.no_sweep:
+        for kf in (0.05, 0.10, 0.20, 1.00):
+            for hf in (0.25, 0.50, 1.00):
+                kk, hh = wl.k_for(kf, shape.N), wl.k_for(hf, shape.h)
+                s2, _ = build_stack(shape, args.layers, B, kk, hh, not args.no_lookahead, layers=layers)
+                g2, _ = capture(s2, x, pos)
+                m2 = time_graph(g2, max(10, args.steps // 2), 3, dist)
+                kk_m, hh_m = selected_counts(s2)
+                b2 = layer_bytes(shape, kk_m, nonzero_neurons(s2), hh_m, B).total
+                sweep.append({"k_frac": kf, "kh_frac": hf, "k": kk, "k_h": hh, "us_per_layer": m2 * 1e3 / args.layers,
+                              "bytes_per_layer": b2, "gbs": b2 / (m2 * 1e3 / args.layers) / 1e3})
+                del g2, s2
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "us", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{CONFIG}-shaped decoder: {args.layers} layers of d={shape.d}, N={shape.N}, "
+                               f"r={shape.r}, h={shape.h}, dh={shape.dh}, KV length {shape.L}, batch {B}, "
+                               f"k={k} ({args.k_frac:.0%}), k_h={k_h} ({args.kh_frac:.0%}), "
+                               f"{'look-ahead' if not args.no_lookahead else 'synchronous'} prediction",
+                   "global_batch": B * world, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2: 24 layers, 2.6 GB of weights streamed per step"},
+        "tokens_per_s": B * world * 1e3 / ms,
+        "us_per_layer_step": us_layer,
+        "selected": {"k": kmean, "k_eff": kp, "k_h": kh},
+        "bytes_per_layer": total_layer_bytes,
+        "effective_gbs": total_layer_bytes / us_layer / 1e3,
+        "effective_frac": total_layer_bytes / us_layer / 1e3 / peak_gbs,
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": ops[dom]["gbs"], "peak": peak_gbs, "unit": "GB/s",
+                     "frac": ops[dom]["frac"], "traffic": None, "peak_source": peak_src, "per_op": ops},
+        "e2e": {"value": e2e_ms * 1e3 / (args.layers * world), "unit": "us", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": xh.numel() * 4, "d2h_bytes_per_step": oh.numel() * 4},
+        "gpu_launches": int(launches_per_step * args.steps),
+        "launches_per_step": int(launches_per_step),
+        "clocks": clocks,
+        "sweep": sweep,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(shape, B, k, k_h, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del g
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
