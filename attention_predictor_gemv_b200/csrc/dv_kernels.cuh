@@ -515,16 +515,20 @@ __global__ void __launch_bounds__(ATTN_THREADS)
   }
   cp_async_wait_all();
   __syncthreads();
-  // scores
-  for (int t = j; t < nk; t += KPP) {
-    float kf[E];
-    WT<KT>::unpack(*reinterpret_cast<const uint4*>(sK + t * DH + g * E), kf);
+  // scores; every thread runs the same trip count so the group shuffles
+  // below always see all 32 lanes of the warp
+  for (int tb = 0; tb < nk; tb += KPP) {
+    const int t = tb + j;
     float dot = 0.f;
+    if (t < nk) {
+      float kf[E];
+      WT<KT>::unpack(*reinterpret_cast<const uint4*>(sK + t * DH + g * E), kf);
 #pragma unroll
-    for (int e = 0; e < E; ++e) dot = fmaf(qv[e], kf[e], dot);
+      for (int e = 0; e < E; ++e) dot = fmaf(qv[e], kf[e], dot);
+    }
 #pragma unroll
     for (int o = G / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-    if (g == 0) sE[t] = dot;
+    if (g == 0 && t < nk) sE[t] = dot;
   }
   __syncthreads();
   float m = -INFINITY;

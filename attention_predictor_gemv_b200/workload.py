@@ -110,7 +110,12 @@ def make_layer(shape: LayerShape, seed: int, device="cpu", with_predictor=True) 
     shift = NormalDist().inv_cdf(1.0 - shape.p_active)
     t["b1"] = (-shift * W1f.norm(dim=1)).contiguous()  # fp32 [N]
     if with_predictor:
-        At, Bm = svd_predictor(W1f, r)
+        devs = [torch.device(device)] if torch.device(device).type == "cuda" else []
+        with torch.random.fork_rng(devices=devs):  # the randomized SVD draws from the global generator
+            torch.manual_seed(int(seed) + 104729)
+            if devs:
+                torch.cuda.manual_seed(int(seed) + 104729)
+            At, Bm = svd_predictor(W1f, r)
         t["At"] = At.to(wdt).contiguous()
         t["Bm"] = Bm.to(wdt).contiguous()
     return t
