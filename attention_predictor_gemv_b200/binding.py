@@ -90,6 +90,7 @@ _lib_dv_predict_layer = _sig("dv_predict_layer", _c_int,
                              [ctypes.POINTER(LayerWeightsC), ctypes.POINTER(Dims), ctypes.POINTER(LayerParamsC), _p,
                               ctypes.POINTER(LayerIOC), _p, _c_size, _p])
 _lib_dv_layernorm = _sig("dv_layernorm", _c_int, [_p, _c_int, _c_int, _p, _p, _c_float, _p, _p])
+_lib_dv_topk_static = _sig("dv_topk_static", _c_int, [_p, _c_int, _c_int, _c_int, _c_float, _c_int, _p, _p, _p])
 _lib_dv_launch_count = _sig("dv_launch_count", ctypes.c_uint64, [])
 
 
@@ -198,6 +199,15 @@ def dv_topk(scores, k, idx, count, ws, tau=0.0, mode=DV_TOPK, stream=None):
     _check(_lib_dv_topk(_ptr(scores, torch.float32, "scores"), B, n, int(k), float(tau), int(mode),
                         _ptr(idx, torch.int32, "idx"), _ptr(count, torch.int32, "count"), _ptr(ws, torch.uint8, "ws"),
                         ws.numel(), _stream(stream)), "dv_topk")
+
+
+def dv_topk_static(scores, k, idx, count, tau=0.0, mode=DV_TOPK, stream=None):
+    """dv_topk without a workspace: the scratch is the library's file-scope
+    device array (at most 16 rows of 65536 scores)."""
+    B, n = scores.shape
+    _check(_lib_dv_topk_static(_ptr(scores, torch.float32, "scores"), B, n, int(k), float(tau), int(mode),
+                               _ptr(idx, torch.int32, "idx"), _ptr(count, torch.int32, "count"), _stream(stream)),
+           "dv_topk_static")
 
 
 def dv_sparse_mlp(y, W1t, b1, W2t, b2, idx, count, k_max, out, ws, accumulate=False, stream=None):

@@ -3,6 +3,7 @@
 #include <atomic>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/dejavu.h"
 #include "dv_kernels.cuh"
@@ -623,3 +624,49 @@ dv_status dv_predict_layer(const dv_layer_weights* w, const dv_dims* dims, const
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// Selection with file-scope scratch, for callers that cannot allocate
+// (dv_topk_static). Layout of the array: the ticket in the first 256 bytes,
+// then the per-row selection bitmaps [rows][n/32].
+// ===========================================================================
+
+static __device__ __align__(256) unsigned char g_topk_static_scratch[DV_TOPK_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_addr[kMaxDevices] = {};
+
+// Device address of g_topk_static_scratch on the current device, looked up
+// once per device (the host-side name is only a stand-in for it).
+dv_status static_scratch_address(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DV_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return DV_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_topk_static_scratch) != cudaSuccess || !p) return DV_ERR_CUDA;
+    g_static_addr[dev] = p;
+  }
+  *out = g_static_addr[dev];
+  return DV_OK;
+}
+
+}  // namespace
+
+extern "C" dv_status dv_topk_static(const float* scores, int B, int n, int k, float tau, int mode, int32_t* idx,
+                                    int32_t* count, dv_stream_t stream) {
+  if (!mode_ok(mode) || !scores || !idx || !count || n < 1 || B < 1) return DV_ERR_ARG;
+  if (!ok_ptr(scores)) return DV_ERR_ALIGN;
+  if (B > DV_TOPK_STATIC_MAX_ROWS || n > DV_TOPK_STATIC_MAX_N) return DV_ERR_UNSUPPORTED;
+  void* base = nullptr;
+  DV_CHECK(static_scratch_address(&base));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned* ticket = static_cast<unsigned*>(base);
+  uint32_t* bitmaps = reinterpret_cast<uint32_t*>(static_cast<char*>(base) + 256);
+  DV_TRY(cudaMemsetAsync(ticket, 0, sizeof(unsigned), st));  // the last-CTA ticket starts at zero
+  return cuda_status(run_select(scores, B, n, k, tau, mode, bitmaps, ticket, idx, count, st));
+}

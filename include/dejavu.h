@@ -246,6 +246,31 @@ DV_API dv_status dv_predict_layer(const dv_layer_weights* w, const dv_dims* dims
                            const float* y, const dv_layer_io* out, void* ws, size_t ws_bytes,
                            dv_stream_t stream);
 
+/* Selection without a caller workspace. The paper has no counterpart: this
+ * is a variant of dv_topk (same rules, same kernel, same results) for callers
+ * that cannot allocate device memory, such as a plugin that runs inside a
+ * host framework which owns all device memory and hands it no allocator, or
+ * a caller whose memory budget is fixed before the decode loop starts.
+ *
+ * Its scratch (one selection bitmap per score row and a ticket) lives in a
+ * file-scope device array of DV_TOPK_STATIC_SCRATCH_BYTES bytes that every
+ * GPU which loads the library holds until the process exits. It therefore
+ * accepts at most DV_TOPK_STATIC_MAX_ROWS score rows of at most
+ * DV_TOPK_STATIC_MAX_N scores; larger sizes return DV_ERR_UNSUPPORTED and
+ * launch nothing. It calls no cudaMalloc / cudaFree.
+ *
+ * The first call on a device looks up the array's device address (one
+ * cudaGetSymbolAddress per device, with that device current); make that first
+ * call before any stream capture. Every call shares the one array per device:
+ * the ticket is cleared on the caller's stream before each launch, and calls
+ * that overlap on the GPU (other streams, other threads) race on it.
+ * Arguments and outputs are those of dv_topk. */
+#define DV_TOPK_STATIC_MAX_ROWS 16
+#define DV_TOPK_STATIC_MAX_N 65536
+#define DV_TOPK_STATIC_SCRATCH_BYTES (256 + 4 * DV_TOPK_STATIC_MAX_ROWS * (DV_TOPK_STATIC_MAX_N / 32))
+DV_API dv_status dv_topk_static(const float* scores, int B, int n, int k, float tau, int mode, int32_t* idx,
+                                int32_t* count, dv_stream_t stream);
+
 /* Number of kernels this library has launched in this process (host-side
  * counter, for reporting). */
 DV_API uint64_t dv_launch_count(void);
