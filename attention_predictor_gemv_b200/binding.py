@@ -86,11 +86,20 @@ _lib_dv_sparse_mha = _sig("dv_sparse_mha", _c_int,
 _lib_dv_decode_layer = _sig("dv_decode_layer", _c_int,
                             [ctypes.POINTER(LayerWeightsC), ctypes.POINTER(Dims), ctypes.POINTER(LayerParamsC), _p,
                              _c_int, ctypes.POINTER(LayerIOC), ctypes.POINTER(LayerIOC), _p, _c_size, _p])
+_lib_dv_decode_layer_begin = _sig("dv_decode_layer_begin", _c_int,
+                                  [ctypes.POINTER(LayerWeightsC), ctypes.POINTER(Dims), ctypes.POINTER(LayerParamsC),
+                                   _p, _c_int, ctypes.POINTER(LayerIOC), ctypes.POINTER(LayerIOC), _p, _c_size, _p])
+_lib_dv_decode_layer_end = _sig("dv_decode_layer_end", _c_int,
+                                [ctypes.POINTER(LayerWeightsC), ctypes.POINTER(Dims), ctypes.POINTER(LayerParamsC),
+                                 _p, _c_int, ctypes.POINTER(LayerIOC), ctypes.POINTER(LayerIOC), _p, _c_size, _p])
 _lib_dv_predict_layer = _sig("dv_predict_layer", _c_int,
                              [ctypes.POINTER(LayerWeightsC), ctypes.POINTER(Dims), ctypes.POINTER(LayerParamsC), _p,
                               ctypes.POINTER(LayerIOC), _p, _c_size, _p])
 _lib_dv_layernorm = _sig("dv_layernorm", _c_int, [_p, _c_int, _c_int, _p, _p, _c_float, _p, _p])
 _lib_dv_topk_static = _sig("dv_topk_static", _c_int, [_p, _c_int, _c_int, _c_int, _c_float, _c_int, _p, _p, _p])
+_lib_dv_prefetch_layer = _sig("dv_prefetch_layer", _c_int,
+                              [ctypes.POINTER(LayerWeightsC), ctypes.POINTER(Dims), ctypes.POINTER(LayerIOC), _c_int,
+                               _c_int, _p])
 _lib_dv_launch_count = _sig("dv_launch_count", ctypes.c_uint64, [])
 
 
@@ -278,7 +287,28 @@ def dv_decode_layer(layer: Layer, p: LayerParamsC, x, pos, ws, sel: Optional[Lay
                                 ws.numel(), _stream(stream)), "dv_decode_layer")
 
 
+def _layer_call(fn, name, layer, p, x, pos, ws, sel, trace, stream):
+    _check(fn(ctypes.byref(layer.c), ctypes.byref(layer.dims), ctypes.byref(p), _ptr(x, torch.float32, "x"), int(pos),
+              ctypes.byref(sel) if sel is not None else None, ctypes.byref(trace) if trace is not None else None,
+              _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)), name)
+
+
+def dv_decode_layer_begin(layer: Layer, p: LayerParamsC, x, pos, ws, sel: Optional[LayerIOC] = None,
+                          trace: Optional[LayerIOC] = None, stream=None):
+    _layer_call(_lib_dv_decode_layer_begin, "dv_decode_layer_begin", layer, p, x, pos, ws, sel, trace, stream)
+
+
+def dv_decode_layer_end(layer: Layer, p: LayerParamsC, x, pos, ws, sel: Optional[LayerIOC] = None,
+                        trace: Optional[LayerIOC] = None, stream=None):
+    _layer_call(_lib_dv_decode_layer_end, "dv_decode_layer_end", layer, p, x, pos, ws, sel, trace, stream)
+
+
 def dv_predict_layer(layer: Layer, p: LayerParamsC, y, out: LayerIOC, ws, stream=None):
     _check(_lib_dv_predict_layer(ctypes.byref(layer.c), ctypes.byref(layer.dims), ctypes.byref(p),
                                  _ptr(y, torch.float32, "y"), ctypes.byref(out), _ptr(ws, torch.uint8, "ws"),
                                  ws.numel(), _stream(stream)), "dv_predict_layer")
+
+
+def dv_prefetch_layer(layer: Layer, sel: LayerIOC, pos, with_w2=True, stream=None):
+    _check(_lib_dv_prefetch_layer(ctypes.byref(layer.c), ctypes.byref(layer.dims), ctypes.byref(sel), int(pos),
+                                  int(bool(with_w2)), _stream(stream)), "dv_prefetch_layer")

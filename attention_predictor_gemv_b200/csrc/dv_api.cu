@@ -2,11 +2,12 @@
 // Declarations and argument contracts: include/dejavu.h.
 #include <atomic>
 #include <cstdlib>
+#include <map>
 #include <cstring>
 #include <mutex>
 
 #include "../../include/dejavu.h"
-#include "dv_kernels.cuh"
+#include "dv_colowner.cuh"
 
 using namespace dv;
 using bf16 = __nv_bfloat16;
@@ -23,6 +24,24 @@ bool pdl_enabled() {
   return on;
 }
 
+// Every kernel asks for the largest shared-memory carveout, so that CTAs of
+// different kernels (consecutive ones overlapping under programmatic launch,
+// and the two streams of the look-ahead) can share an SM without the SM
+// having to drain and reconfigure its L1 / shared split. Cached per kernel.
+std::mutex g_carve_mu;
+std::map<std::pair<const void*, int>, bool> g_carve_set;
+
+template <typename K>
+void prefer_max_shared(K kern) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return;
+  const auto key = std::make_pair(reinterpret_cast<const void*>(kern), dev);
+  std::lock_guard<std::mutex> lock(g_carve_mu);
+  if (g_carve_set.count(key)) return;
+  cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+  g_carve_set[key] = true;
+}
+
 // Launch with programmatic stream serialisation, so a kernel's launch and
 // prologue overlap the tail of the previous kernel on the stream.
 template <typename... KArgs, typename... Args>
@@ -37,8 +56,58 @@ cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, c
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  prefer_max_shared(kern);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+// Launch as thread-block clusters of `cluster_x` CTAs (plus programmatic
+// stream serialisation).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster_x,
+                           Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cluster_x;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
+  prefer_max_shared(kern);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+// Raises a kernel's dynamic shared memory limit to `bytes` when needed (the
+// default 48 KB covers static plus dynamic). Cached per kernel and device.
+std::mutex g_smem_mu;
+struct SmemKey {
+  const void* fn;
+  int dev;
+  bool operator<(const SmemKey& o) const { return fn < o.fn || (fn == o.fn && dev < o.dev); }
+};
+std::map<SmemKey, size_t> g_smem_set;
+
+template <typename K>
+cudaError_t allow_smem(K kern, size_t bytes) {
+  if (bytes == 0) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const SmemKey key{reinterpret_cast<const void*>(kern), dev};
+  std::lock_guard<std::mutex> lock(g_smem_mu);
+  auto it = g_smem_set.find(key);
+  if (it != g_smem_set.end() && it->second >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) g_smem_set[key] = bytes;
+  return e;
 }
 
 int sm_count() {
@@ -67,14 +136,15 @@ int rpw_for(int K, int E) {
 constexpr int ATTN_S_MIN = 32;
 // Every layout starts with the same fixed header that holds the counters, so
 // calls of different operations may share one workspace: the status word at
-// 0, the two selection tickets at 16 and 32, and the attention split counters
-// [B][kh_max] from 1024.
-constexpr size_t WS_HEADER = 64 * 1024;
+// 0, the selection tickets at 16, 32, 48 and 64, the attention split counters
+// [B][kh_max] from 1024, and the neuron-score histograms from 64 KB.
+constexpr size_t WS_HEADER = 192 * 1024;
+constexpr size_t WS_HIST = 64 * 1024;  // [16][2048] digit histograms of the fused neuron predictor
 constexpr int KH_LIMIT = 1000;  // B * kh_max counters must fit the header
 
 // Workspace layout. Offsets in bytes from the workspace base.
 struct Layout {
-  size_t status, sel_ticket_h, sel_ticket_m, attn_ctr;
+  size_t status, sel_ticket_h, sel_ticket_m, pa_ticket, pb_ticket, attn_ctr, hist, t1;
   size_t yA, yM, z, scores_h, bm_h, head_idx, head_count, scores, bm_m, idx, count;
   size_t q, part, H, seg_idx, seg_a, seg_cnt, total;
   int nseg, SEG, nsplit_max;
@@ -98,7 +168,11 @@ Layout layout(const dv_dims& D, int wbytes) {
   L.status = take(WS_HEADER);
   L.sel_ticket_h = L.status + 16;
   L.sel_ticket_m = L.status + 32;
+  L.pa_ticket = L.status + 48;
+  L.pb_ticket = L.status + 64;
   L.attn_ctr = L.status + 1024;
+  L.hist = L.status + WS_HIST;
+  L.t1 = take(4ull * B * D.d);
   L.yA = take(4ull * B * D.d);
   L.yM = take(4ull * B * D.d);
   L.z = take(4ull * B * D.r);
@@ -178,16 +252,10 @@ cudaError_t run_gemv(dv_dtype dt, const void* W, int nrows, int K, const float* 
 
 cudaError_t run_select(const float* scores, int nrows, int n, int k, float tau, int mode, uint32_t* bm,
                        unsigned* ticket, int32_t* idx, int32_t* count, cudaStream_t st) {
-  const bool need_keys = (mode == DV_TOPK) && k > 0 && k < n;
-  if (need_keys && n <= SEL_SMEM_KEYS) {
+  if (n <= SEL_SMEM_KEYS) {  // keys (top-k) and the union bitmap in shared memory
     const size_t smem = 4ull * n;
-    static bool attr_set = false;
-    if (!attr_set) {
-      cudaError_t e = cudaFuncSetAttribute(select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           4 * SEL_SMEM_KEYS);
-      if (e != cudaSuccess) return e;
-      attr_set = true;
-    }
+    cudaError_t e = allow_smem(select_kernel<true>, smem);
+    if (e != cudaSuccess) return e;
     return launch(select_kernel<true>, dim3(nrows), SEL_THREADS, smem, st, scores, n, nrows, k, tau, mode, bm, ticket,
                   idx, count);
   }
@@ -218,11 +286,8 @@ cudaError_t run_axpy_st(const void* W, int d, int nrows_w, Src src, const float*
   const int gmax = (k_max + 3) / 4;
   if (G > gmax) G = gmax;
   if (G < 1) G = 1;
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(axpy_rows_kernel<T, NB, Src>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-  }
+  cudaError_t e = allow_smem(axpy_rows_kernel<T, NB, Src>, smem);
+  if (e != cudaSuccess) return e;
   return launch(axpy_rows_kernel<T, NB, Src>, dim3(tiles, G), AX_THREADS, smem, st, static_cast<const T*>(W), d,
                 nrows_w, src, bias, out, nb, G, status);
 }
@@ -408,6 +473,460 @@ dv_status check_ws(const Layout& L, void* ws, size_t ws_bytes) {
   return DV_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Fused layer path (dv_fused.cuh)
+// ---------------------------------------------------------------------------
+
+constexpr int ATTN_CS = 8;  // CTAs per cluster (per selected head) in attn_out_kernel
+
+int attn_out_S(int pos) { return (pos + 1 + ATTN_CS - 1) / ATTN_CS; }
+size_t attn_out_smem(int S, int dh, int kvbytes) { return 2ull * S * dh * kvbytes + 4ull * S; }
+
+bool fused_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("DV_FUSED");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+// Shapes the fused kernels take: column slices of W^O whole 16-byte vectors,
+// the normalised input and the K/V tiles within shared memory.
+bool fused_ok(const dv_dims& D, dv_dtype wdt) {
+  if (!fused_enabled()) return false;
+  const int wb = wbytes_of(wdt), E = 16 / wb;
+  if (D.d % (ATTN_CS * E) != 0) return false;
+  if ((size_t)D.B * D.d * 4 > 160 * 1024) return false;
+  if (attn_out_smem(attn_out_S(D.cap - 1), D.dh, wb) > 190 * 1024) return false;
+  if (D.N > SEL_SMEM_KEYS || D.h > HSEL_MAX) return false;
+  return true;
+}
+
+template <typename K, typename A>
+cudaError_t launch_fused(K kern, dim3 grid, size_t smem, cudaStream_t st, const A& a) {
+  cudaError_t e = allow_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  return launch(kern, grid, FUSED_THREADS, smem, st, a);
+}
+
+template <typename T, int NB>
+cudaError_t run_attn_in_nb(const AttnInArgs& a, cudaStream_t st) {
+  const int rpw = rpw_for(a.d, WT<T>::E);
+  const int slots = a.kh_max * 3 * a.dh, per = FUSED_WARPS * rpw;
+  const dim3 grid(slots > 0 ? (slots + per - 1) / per : 1);
+  const size_t smem = 4ull * a.nb * a.d;
+  switch (rpw) {
+    case 1: return launch_fused(attn_in_kernel<T, NB, 1, 8>, grid, smem, st, a);
+    case 2: return launch_fused(attn_in_kernel<T, NB, 2, 4>, grid, smem, st, a);
+    case 4: return launch_fused(attn_in_kernel<T, NB, 4, 2>, grid, smem, st, a);
+    default: return launch_fused(attn_in_kernel<T, NB, 8, 1>, grid, smem, st, a);
+  }
+}
+
+template <typename T>
+cudaError_t run_attn_in(const AttnInArgs& a, cudaStream_t st) {
+  switch (nb_bucket(a.nb)) {
+    case 1: return run_attn_in_nb<T, 1>(a, st);
+    case 2: return run_attn_in_nb<T, 2>(a, st);
+    case 4: return run_attn_in_nb<T, 4>(a, st);
+    case 8: return run_attn_in_nb<T, 8>(a, st);
+    default: return run_attn_in_nb<T, 16>(a, st);
+  }
+}
+
+template <typename KT, int DH, int NB>
+cudaError_t run_attn_out_nb(const AttnOutArgs& a, cudaStream_t st) {
+  const size_t smem = attn_out_smem(a.S, DH, sizeof(KT));
+  auto kern = attn_out_kernel<KT, DH, ATTN_CS, NB>;
+  cudaError_t e = allow_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  return launch_cluster(kern, dim3(ATTN_CS, a.kh_max > 0 ? a.kh_max : 1), FUSED_THREADS, smem, st, ATTN_CS, a);
+}
+
+template <typename KT, int DH>
+cudaError_t run_attn_out_dh(const AttnOutArgs& a, cudaStream_t st) {
+  switch (nb_bucket(a.nb)) {
+    case 1: return run_attn_out_nb<KT, DH, 1>(a, st);
+    case 2: return run_attn_out_nb<KT, DH, 2>(a, st);
+    case 4: return run_attn_out_nb<KT, DH, 4>(a, st);
+    case 8: return run_attn_out_nb<KT, DH, 8>(a, st);
+    default: return run_attn_out_nb<KT, DH, 16>(a, st);
+  }
+}
+
+template <typename KT>
+cudaError_t run_attn_out(const AttnOutArgs& a, cudaStream_t st) {
+  return a.dh == 64 ? run_attn_out_dh<KT, 64>(a, st) : run_attn_out_dh<KT, 128>(a, st);
+}
+
+int mlp_block_grid(int k_max) {
+  const int g = (k_max + 7) / 8;
+  return g < 1 ? 1 : (g > sm_count() ? sm_count() : g);
+}
+
+template <typename T, int NB>
+cudaError_t run_mlp_block_nb(const MlpBlockArgs& a, cudaStream_t st) {
+  const int rpw = rpw_for(a.d, WT<T>::E);
+  const dim3 grid(a.G);
+  const size_t smem = 4ull * a.nb * a.d;
+  switch (rpw) {
+    case 1: return launch_fused(mlp_block_kernel<T, NB, 1, 8>, grid, smem, st, a);
+    case 2: return launch_fused(mlp_block_kernel<T, NB, 2, 4>, grid, smem, st, a);
+    case 4: return launch_fused(mlp_block_kernel<T, NB, 4, 2>, grid, smem, st, a);
+    default: return launch_fused(mlp_block_kernel<T, NB, 8, 1>, grid, smem, st, a);
+  }
+}
+
+template <typename T>
+cudaError_t run_mlp_block(const MlpBlockArgs& a, cudaStream_t st) {
+  switch (nb_bucket(a.nb)) {
+    case 1: return run_mlp_block_nb<T, 1>(a, st);
+    case 2: return run_mlp_block_nb<T, 2>(a, st);
+    case 4: return run_mlp_block_nb<T, 4>(a, st);
+    case 8: return run_mlp_block_nb<T, 8>(a, st);
+    default: return run_mlp_block_nb<T, 16>(a, st);
+  }
+}
+
+template <typename T, int NB>
+cudaError_t run_predict_a_nb(const PredictAArgs& a, cudaStream_t st) {
+  const int rows = (a.PA ? a.h : 0) + (a.At ? a.r : 0);
+  const int rpw = rpw_for(a.d, WT<T>::E), per = FUSED_WARPS * rpw;
+  const dim3 grid(rows > 0 ? (rows + per - 1) / per : 1);
+  switch (rpw) {
+    case 1: return launch(predict_a_kernel<T, NB, 1, 8>, grid, FUSED_THREADS, 0, st, a);
+    case 2: return launch(predict_a_kernel<T, NB, 2, 4>, grid, FUSED_THREADS, 0, st, a);
+    case 4: return launch(predict_a_kernel<T, NB, 4, 2>, grid, FUSED_THREADS, 0, st, a);
+    default: return launch(predict_a_kernel<T, NB, 8, 1>, grid, FUSED_THREADS, 0, st, a);
+  }
+}
+
+template <typename T>
+cudaError_t run_predict_a(const PredictAArgs& a, cudaStream_t st) {
+  switch (nb_bucket(a.nb)) {
+    case 1: return run_predict_a_nb<T, 1>(a, st);
+    case 2: return run_predict_a_nb<T, 2>(a, st);
+    case 4: return run_predict_a_nb<T, 4>(a, st);
+    case 8: return run_predict_a_nb<T, 8>(a, st);
+    default: return run_predict_a_nb<T, 16>(a, st);
+  }
+}
+
+template <typename T, int NB>
+cudaError_t run_predict_b_nb(const PredictBArgs& a, cudaStream_t st) {
+  const int rpw = rpw_for(a.r, WT<T>::E), per = FUSED_WARPS * rpw;
+  const dim3 grid((a.N + per - 1) / per);
+  switch (rpw) {
+    case 1: return launch(predict_b_kernel<T, NB, 1, 8>, grid, FUSED_THREADS, 0, st, a);
+    case 2: return launch(predict_b_kernel<T, NB, 2, 4>, grid, FUSED_THREADS, 0, st, a);
+    case 4: return launch(predict_b_kernel<T, NB, 4, 2>, grid, FUSED_THREADS, 0, st, a);
+    default: return launch(predict_b_kernel<T, NB, 8, 1>, grid, FUSED_THREADS, 0, st, a);
+  }
+}
+
+template <typename T>
+cudaError_t run_predict_b(const PredictBArgs& a, cudaStream_t st) {
+  switch (nb_bucket(a.nb)) {
+    case 1: return run_predict_b_nb<T, 1>(a, st);
+    case 2: return run_predict_b_nb<T, 2>(a, st);
+    case 4: return run_predict_b_nb<T, 4>(a, st);
+    case 8: return run_predict_b_nb<T, 8>(a, st);
+    default: return run_predict_b_nb<T, 16>(a, st);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Column-owner kernels (dv_colowner.cuh) for batch 1-2
+// ---------------------------------------------------------------------------
+
+int co_nv(int d, int E) { return (d + CO_THREADS * E - 1) / (CO_THREADS * E); }
+int co_r(int nv) { return nv == 1 ? 8 : nv == 2 ? 4 : nv == 3 ? 3 : 2; }
+bool co_ok(int nb, int d, int E) { return nb <= 2 && co_nv(d, E) <= 6; }
+int co_grid(long long groups) {
+  const long long cap = 2ll * sm_count();
+  return (int)(groups < 1 ? 1 : (groups > cap ? cap : groups));
+}
+
+#define DV_CO_SWITCH(KERN, NB, grid, st, a)                                   \
+  switch (nv) {                                                              \
+    case 1: return launch(KERN<T, NB, 1, 8>, grid, CO_THREADS, 0, st, a);    \
+    case 2: return launch(KERN<T, NB, 2, 4>, grid, CO_THREADS, 0, st, a);    \
+    case 3: return launch(KERN<T, NB, 3, 3>, grid, CO_THREADS, 0, st, a);    \
+    case 4: return launch(KERN<T, NB, 4, 2>, grid, CO_THREADS, 0, st, a);    \
+    case 5: return launch(KERN<T, NB, 5, 2>, grid, CO_THREADS, 0, st, a);    \
+    default: return launch(KERN<T, NB, 6, 2>, grid, CO_THREADS, 0, st, a);   \
+  }
+
+template <typename T, int NB>
+cudaError_t run_attn_in_co_nb(const AttnInArgs& a, cudaStream_t st) {
+  const int nv = co_nv(a.d, WT<T>::E), R = co_r(nv);
+  const dim3 grid(co_grid(((long long)a.kh_max * 3 * a.dh + R - 1) / R));
+  DV_CO_SWITCH(attn_in_co_kernel, NB, grid, st, a)
+}
+
+template <typename T, int NB>
+cudaError_t run_mlp_block_co_nb(MlpBlockArgs a, cudaStream_t st) {
+  const int nv = co_nv(a.d, WT<T>::E), R = co_r(nv);
+  a.G = co_grid(((long long)a.k_max + R - 1) / R);
+  const dim3 grid(a.G);
+  DV_CO_SWITCH(mlp_block_co_kernel, NB, grid, st, a)
+}
+
+template <typename T, int NB>
+cudaError_t run_predict_a_co_nb(const PredictAArgs& a, cudaStream_t st) {
+  const int nv = co_nv(a.d, WT<T>::E), R = co_r(nv);
+  const int rows = (a.PA ? a.h : 0) + (a.At ? a.r : 0);
+  const dim3 grid(co_grid((rows + R - 1) / R));
+  DV_CO_SWITCH(predict_a_co_kernel, NB, grid, st, a)
+}
+#undef DV_CO_SWITCH
+
+template <typename T>
+cudaError_t run_attn_in_any(const AttnInArgs& a, cudaStream_t st) {
+  if (co_ok(a.nb, a.d, WT<T>::E))
+    return a.nb == 1 ? run_attn_in_co_nb<T, 1>(a, st) : run_attn_in_co_nb<T, 2>(a, st);
+  return run_attn_in<T>(a, st);
+}
+
+template <typename T>
+cudaError_t run_mlp_block_any(const MlpBlockArgs& a, cudaStream_t st) {
+  if (co_ok(a.nb, a.d, WT<T>::E))
+    return a.nb == 1 ? run_mlp_block_co_nb<T, 1>(a, st) : run_mlp_block_co_nb<T, 2>(a, st);
+  return run_mlp_block<T>(a, st);
+}
+
+template <typename T>
+cudaError_t run_predict_a_any(const PredictAArgs& a, cudaStream_t st) {
+  if (co_ok(a.nb, a.d, WT<T>::E))
+    return a.nb == 1 ? run_predict_a_co_nb<T, 1>(a, st) : run_predict_a_co_nb<T, 2>(a, st);
+  return run_predict_a<T>(a, st);
+}
+
+// The head set (heads) and/or the neuron set (neurons) predicted from y:
+// predict_a (head scores, z = y A), predict_b (neuron scores + first digit
+// histogram), select_finish (exact top-k / threshold of both).
+dv_status fused_predict(const Layout& L, void* ws, const dv_layer_weights* w, const dv_dims& D,
+                        const dv_layer_params* p, const float* y, bool heads, bool neurons, float* sh, int32_t* hidx,
+                        int32_t* hcnt, float* sm, int32_t* midx, int32_t* mcnt, cudaStream_t st) {
+  PredictAArgs a = {};
+  a.y = y;
+  a.PA = heads ? w->PA : nullptr;
+  a.At = neurons ? w->At : nullptr;
+  a.h = D.h;
+  a.r = D.r;
+  a.d = D.d;
+  a.nb = D.B;
+  a.scores_h = sh;
+  a.z = at<float>(ws, L.z);
+  DV_TRY(w->wdtype == DV_BF16 ? run_predict_a_any<bf16>(a, st) : run_predict_a_any<float>(a, st));
+  const bool hist_mode = p->mode == DV_TOPK && p->k > 0 && p->k < D.N;
+  if (neurons) {
+    PredictBArgs b = {};
+    b.z = a.z;
+    b.Bm = w->Bm;
+    b.b1 = w->b1;
+    b.N = D.N;
+    b.r = D.r;
+    b.nb = D.B;
+    b.hist_mode = hist_mode ? 1 : 0;
+    b.scores = sm;
+    b.hist = at<unsigned>(ws, L.hist);
+    DV_TRY(w->wdtype == DV_BF16 ? run_predict_b<bf16>(b, st) : run_predict_b<float>(b, st));
+  }
+  SelectFinishArgs f = {};
+  f.scores = sm;
+  f.hist = at<unsigned>(ws, L.hist);
+  f.bitmaps = at<uint32_t>(ws, L.bm_m);
+  f.ticket = at<unsigned>(ws, L.pb_ticket);
+  f.neuron_rows = neurons ? D.B : 0;
+  f.N = D.N;
+  f.nb = D.B;
+  f.k = p->k;
+  f.mode = p->mode;
+  f.tau = p->tau;
+  f.idx = midx;
+  f.count = mcnt;
+  f.scores_h = heads ? sh : nullptr;
+  f.h = D.h;
+  f.k_h = p->k_h;
+  f.mode_h = p->mode_h;
+  f.tau_h = p->tau_h;
+  f.head_idx = hidx;
+  f.head_count = hcnt;
+  const int grid = (neurons ? D.B : 0) + (heads ? 1 : 0);
+  const size_t smem = 4ull * (neurons && hist_mode ? (D.N > D.h ? D.N : D.h) : D.h);
+  DV_TRY(allow_smem(select_finish_kernel, smem));
+  DV_TRY(launch(select_finish_kernel, dim3(grid), dim3(SEL_THREADS), smem, st, f));
+  return DV_OK;
+}
+
+// Pointers a layer call writes: the trace buffers when given, else workspace.
+struct LayerBufs {
+  float *yA, *yM, *sh, *sm;
+  int32_t *hidx, *hcnt, *midx, *mcnt;
+  const int32_t *use_hidx, *use_hcnt, *use_midx, *use_mcnt;
+};
+
+LayerBufs layer_bufs(const Layout& L, void* ws, const dv_layer_io* sel, const dv_layer_io* trace) {
+  const dv_layer_io none = {};
+  const dv_layer_io& t = trace ? *trace : none;
+  LayerBufs r;
+  r.yA = t.yA ? t.yA : at<float>(ws, L.yA);
+  r.yM = t.yM ? t.yM : at<float>(ws, L.yM);
+  r.sh = t.scores_h ? t.scores_h : at<float>(ws, L.scores_h);
+  r.hidx = t.head_idx ? t.head_idx : at<int32_t>(ws, L.head_idx);
+  r.hcnt = t.head_count ? t.head_count : at<int32_t>(ws, L.head_count);
+  r.sm = t.scores ? t.scores : at<float>(ws, L.scores);
+  r.midx = t.idx ? t.idx : at<int32_t>(ws, L.idx);
+  r.mcnt = t.count ? t.count : at<int32_t>(ws, L.count);
+  r.use_hidx = sel ? sel->head_idx : r.hidx;
+  r.use_hcnt = sel ? sel->head_count : r.hcnt;
+  r.use_midx = sel ? sel->idx : r.midx;
+  r.use_mcnt = sel ? sel->count : r.mcnt;
+  return r;
+}
+
+// First half of a layer: LN1, the head set unless given, Q/K/V + KV append.
+dv_status layer_begin(const Layout& L, void* ws, const dv_layer_weights* w, const dv_dims& D, const dv_layer_params* p,
+                      float* x, int pos, const dv_layer_io* sel, const dv_layer_io* trace, cudaStream_t st) {
+  const LayerBufs r = layer_bufs(L, ws, sel, trace);
+  int* status = at<int>(ws, L.status);
+  if (fused_ok(D, w->wdtype)) {
+    if (!sel) {
+      DV_TRY(launch(layernorm_kernel, dim3(D.B), LN_THREADS, 0, st, (const float*)x, r.yA, D.d, w->ln1_g, w->ln1_b,
+                    p->eps));
+      DV_CHECK(fused_predict(L, ws, w, D, p, r.yA, true, false, r.sh, r.hidx, r.hcnt, nullptr, nullptr, nullptr, st));
+    }
+    AttnInArgs a = {};
+    a.x = x;
+    a.t1 = at<float>(ws, L.t1);
+    a.yA_out = sel ? (trace ? trace->yA : nullptr) : nullptr;
+    a.ln_g = w->ln1_g;
+    a.ln_b = w->ln1_b;
+    a.eps = p->eps;
+    a.Wqkv = w->Wqkv;
+    a.bqkv = w->bqkv;
+    a.head_idx = r.use_hidx;
+    a.head_count = r.use_hcnt;
+    a.kh_max = D.kh_max;
+    a.q = at<float>(ws, L.q);
+    a.Kc = w->Kc;
+    a.Vc = w->Vc;
+    a.h = D.h;
+    a.dh = D.dh;
+    a.d = D.d;
+    a.cap = D.cap;
+    a.pos = pos;
+    a.nb = D.B;
+    a.sets_ready = sel ? 1 : 0;
+    a.status = status;
+    return cuda_status(w->wdtype == DV_BF16 ? run_attn_in_any<bf16>(a, st) : run_attn_in_any<float>(a, st));
+  }
+  // kernel-per-step path
+  float* yA = r.yA;
+  if (sel && sel->yA) {
+    yA = sel->yA;  // LN1(x) computed by the caller
+  } else {
+    DV_TRY(launch(layernorm_kernel, dim3(D.B), LN_THREADS, 0, st, (const float*)x, yA, D.d, w->ln1_g, w->ln1_b,
+                  p->eps));
+  }
+  if (!sel)
+    DV_CHECK(do_predict_heads(L, ws, yA, D.B, D.d, D.h, w->PA, w->wdtype, p->k_h, p->tau_h, p->mode_h, r.sh, r.hidx,
+                              r.hcnt, st));
+  if (D.kh_max == 0) return DV_OK;
+  float* q = at<float>(ws, L.q);
+  return cuda_status(w->wdtype == DV_BF16
+                         ? run_qkv<bf16>(w->Wqkv, D.d, D.h, D.dh, yA, D.B, w->bqkv, r.use_hidx, r.use_hcnt, D.kh_max,
+                                         q, w->Kc, w->Vc, D.cap, pos, status, st)
+                         : run_qkv<float>(w->Wqkv, D.d, D.h, D.dh, yA, D.B, w->bqkv, r.use_hidx, r.use_hcnt,
+                                          D.kh_max, q, w->Kc, w->Vc, D.cap, pos, status, st));
+}
+
+// Second half: attention + W^O + residual, LN2, the neuron set unless given,
+// the sparse MLP + residual.
+dv_status layer_end(const Layout& L, void* ws, const dv_layer_weights* w, const dv_dims& D, const dv_layer_params* p,
+                    float* x, int pos, const dv_layer_io* sel, const dv_layer_io* trace, cudaStream_t st) {
+  const LayerBufs r = layer_bufs(L, ws, sel, trace);
+  int* status = at<int>(ws, L.status);
+  if (fused_ok(D, w->wdtype)) {
+    float* t1 = at<float>(ws, L.t1);
+    AttnOutArgs b = {};
+    b.q = at<float>(ws, L.q);
+    b.Kc = w->Kc;
+    b.Vc = w->Vc;
+    b.WOt = w->WOt;
+    b.bO = w->bO;
+    b.head_idx = r.use_hidx;
+    b.head_count = r.use_hcnt;
+    b.kh_max = D.kh_max;
+    b.x = x;
+    b.t1 = t1;
+    b.h = D.h;
+    b.dh = D.dh;
+    b.d = D.d;
+    b.cap = D.cap;
+    b.pos = pos;
+    b.nb = D.B;
+    b.S = attn_out_S(pos);
+    b.sets_ready = sel ? 1 : 0;
+    b.scale = p->scale;
+    b.status = status;
+    DV_TRY(w->kvdtype == DV_BF16 ? run_attn_out<bf16>(b, st) : run_attn_out<float>(b, st));
+    if (!sel) {
+      DV_TRY(launch(layernorm_kernel, dim3(D.B), LN_THREADS, 0, st, (const float*)t1, r.yM, D.d, w->ln2_g, w->ln2_b,
+                    p->eps));
+      DV_CHECK(fused_predict(L, ws, w, D, p, r.yM, false, true, nullptr, nullptr, nullptr, r.sm, r.midx, r.mcnt, st));
+    }
+    MlpBlockArgs c = {};
+    c.t1 = t1;
+    c.x = x;
+    c.ln_g = w->ln2_g;
+    c.ln_b = w->ln2_b;
+    c.eps = p->eps;
+    c.W1t = w->W1t;
+    c.b1 = w->b1;
+    c.W2t = w->W2t;
+    c.b2 = w->b2;
+    c.idx = r.use_midx;
+    c.count = r.use_mcnt;
+    c.k_max = D.k_max;
+    c.d = D.d;
+    c.N = D.N;
+    c.nb = D.B;
+    c.G = mlp_block_grid(D.k_max);
+    c.sets_ready = sel ? 1 : 0;
+    c.yM_out = sel ? (trace ? trace->yM : nullptr) : nullptr;
+    c.status = status;
+    return cuda_status(w->wdtype == DV_BF16 ? run_mlp_block_any<bf16>(c, st) : run_mlp_block_any<float>(c, st));
+  }
+  // kernel-per-step path
+  if (D.kh_max > 0) {
+    float* H = at<float>(ws, L.H);
+    const float* q = at<float>(ws, L.q);
+    DV_TRY(w->kvdtype == DV_BF16
+               ? run_attn<bf16>(D.dh, q, w->Kc, w->Vc, D.B, D.h, D.cap, pos, p->scale, r.use_hidx, r.use_hcnt,
+                                D.kh_max, at<float>(ws, L.part), at<unsigned>(ws, L.attn_ctr), H, status, st)
+               : run_attn<float>(D.dh, q, w->Kc, w->Vc, D.B, D.h, D.cap, pos, p->scale, r.use_hidx, r.use_hcnt,
+                                 D.kh_max, at<float>(ws, L.part), at<unsigned>(ws, L.attn_ctr), H, status, st));
+    RowsHeads src{r.use_hidx, r.use_hcnt, H, D.kh_max, D.dh, D.h};
+    DV_TRY(w->wdtype == DV_BF16 ? run_axpy<bf16>(w->WOt, D.d, D.h * D.dh, src, w->bO, x, D.B, D.kh_max * D.dh, 0,
+                                                 status, st)
+                                : run_axpy<float>(w->WOt, D.d, D.h * D.dh, src, w->bO, x, D.B, D.kh_max * D.dh, 0,
+                                                  status, st));
+  } else if (w->bO) {
+    RowsHeads none{r.use_hidx, r.use_hcnt, nullptr, 0, D.dh, D.h};
+    DV_TRY(w->wdtype == DV_BF16 ? run_axpy<bf16>(w->WOt, D.d, D.h * D.dh, none, w->bO, x, D.B, 1, 0, status, st)
+                                : run_axpy<float>(w->WOt, D.d, D.h * D.dh, none, w->bO, x, D.B, 1, 0, status, st));
+  }
+  DV_TRY(launch(layernorm_kernel, dim3(D.B), LN_THREADS, 0, st, (const float*)x, r.yM, D.d, w->ln2_g, w->ln2_b,
+                p->eps));
+  if (!sel)
+    DV_CHECK(do_predict_mlp(L, ws, r.yM, D.B, D.d, D.r, D.N, w->At, w->Bm, w->b1, w->wdtype, p->k, p->tau, p->mode,
+                            r.sm, r.midx, r.mcnt, st));
+  return do_sparse_mlp(L, ws, r.yM, D.B, D.d, D.N, w->W1t, w->b1, w->W2t, w->b2, w->wdtype, r.use_midx, r.use_mcnt,
+                       D.k_max, x, 1, st);
+}
+
 }  // namespace
 
 // ===========================================================================
@@ -549,53 +1068,81 @@ static dv_status check_layer(const dv_layer_weights* w, const dv_dims* dims, con
   return DV_OK;
 }
 
-dv_status dv_decode_layer(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p, float* x, int pos,
-                          const dv_layer_io* sel, const dv_layer_io* trace, void* ws, size_t ws_bytes,
-                          dv_stream_t stream) {
+static dv_status check_layer_call(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p, float* x,
+                                  int pos, const dv_layer_io* sel, const dv_layer_io* trace, void* ws,
+                                  size_t ws_bytes, Layout* L) {
   DV_CHECK(check_layer(w, dims, p));
   const dv_dims& D = *dims;
   if (!x) return DV_ERR_ARG;
   if (!ok_ptr(x)) return DV_ERR_ALIGN;
   if (pos < 0 || pos >= D.cap) return DV_ERR_ARG;
   if (sel && (!sel->head_idx || !sel->head_count || !sel->idx || !sel->count)) return DV_ERR_ARG;
-  const Layout L = layout(D, wbytes_of(w->wdtype));
-  DV_CHECK(check_ws(L, ws, ws_bytes));
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const dv_layer_io none = {};
-  const dv_layer_io& t = trace ? *trace : none;
-  float* yA = t.yA ? t.yA : at<float>(ws, L.yA);
-  float* yM = t.yM ? t.yM : at<float>(ws, L.yM);
-  if (!ok_ptr(yA) || !ok_ptr(yM)) return DV_ERR_ALIGN;
-  float* sh = t.scores_h ? t.scores_h : at<float>(ws, L.scores_h);
-  int32_t* hidx = t.head_idx ? t.head_idx : at<int32_t>(ws, L.head_idx);
-  int32_t* hcnt = t.head_count ? t.head_count : at<int32_t>(ws, L.head_count);
-  float* sm = t.scores ? t.scores : at<float>(ws, L.scores);
-  int32_t* midx = t.idx ? t.idx : at<int32_t>(ws, L.idx);
-  int32_t* mcnt = t.count ? t.count : at<int32_t>(ws, L.count);
-  const int32_t* use_hidx = sel ? sel->head_idx : hidx;
-  const int32_t* use_hcnt = sel ? sel->head_count : hcnt;
-  const int32_t* use_midx = sel ? sel->idx : midx;
-  const int32_t* use_mcnt = sel ? sel->count : mcnt;
+  if (sel && !ok_opt(sel->yA)) return DV_ERR_ALIGN;
+  if (trace && (!ok_opt(trace->yA) || !ok_opt(trace->yM) || !ok_opt(trace->scores) || !ok_opt(trace->scores_h)))
+    return DV_ERR_ALIGN;
+  *L = layout(D, wbytes_of(w->wdtype));
+  return check_ws(*L, ws, ws_bytes);
+}
 
-  if (sel && sel->yA) {
-    if (!ok_ptr(sel->yA)) return DV_ERR_ALIGN;
-    yA = sel->yA;  // LN1(x) computed by the caller
-  } else {
-    DV_TRY(launch(layernorm_kernel, dim3(D.B), LN_THREADS, 0, st, (const float*)x, yA, D.d, w->ln1_g, w->ln1_b,
-                  p->eps));
-  }
-  if (!sel)
-    DV_CHECK(do_predict_heads(L, ws, yA, D.B, D.d, D.h, w->PA, w->wdtype, p->k_h, p->tau_h, p->mode_h, sh, hidx, hcnt,
-                              st));
-  DV_CHECK(do_sparse_mha(L, ws, yA, D.B, D.d, D.h, D.dh, w->Wqkv, w->bqkv, w->WOt, w->bO, w->wdtype, w->Kc, w->Vc,
-                         D.cap, pos, p->scale, use_hidx, use_hcnt, D.kh_max, x, 1, st));
-  DV_TRY(launch(layernorm_kernel, dim3(D.B), LN_THREADS, 0, st, (const float*)x, yM, D.d, w->ln2_g, w->ln2_b, p->eps));
-  if (!sel)
-    DV_CHECK(do_predict_mlp(L, ws, yM, D.B, D.d, D.r, D.N, w->At, w->Bm, w->b1, w->wdtype, p->k, p->tau, p->mode, sm,
-                            midx, mcnt, st));
-  DV_CHECK(do_sparse_mlp(L, ws, yM, D.B, D.d, D.N, w->W1t, w->b1, w->W2t, w->b2, w->wdtype, use_midx, use_mcnt,
-                         D.k_max, x, 1, st));
-  return DV_OK;
+dv_status dv_decode_layer_begin(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p, float* x,
+                                int pos, const dv_layer_io* sel, const dv_layer_io* trace, void* ws, size_t ws_bytes,
+                                dv_stream_t stream) {
+  Layout L;
+  DV_CHECK(check_layer_call(w, dims, p, x, pos, sel, trace, ws, ws_bytes, &L));
+  return layer_begin(L, ws, w, *dims, p, x, pos, sel, trace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dv_status dv_decode_layer_end(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p, float* x,
+                              int pos, const dv_layer_io* sel, const dv_layer_io* trace, void* ws, size_t ws_bytes,
+                              dv_stream_t stream) {
+  Layout L;
+  DV_CHECK(check_layer_call(w, dims, p, x, pos, sel, trace, ws, ws_bytes, &L));
+  return layer_end(L, ws, w, *dims, p, x, pos, sel, trace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dv_status dv_decode_layer(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p, float* x, int pos,
+                          const dv_layer_io* sel, const dv_layer_io* trace, void* ws, size_t ws_bytes,
+                          dv_stream_t stream) {
+  Layout L;
+  DV_CHECK(check_layer_call(w, dims, p, x, pos, sel, trace, ws, ws_bytes, &L));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  DV_CHECK(layer_begin(L, ws, w, *dims, p, x, pos, sel, trace, st));
+  return layer_end(L, ws, w, *dims, p, x, pos, sel, trace, st);
+}
+
+dv_status dv_prefetch_layer(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_io* sel, int pos,
+                            int with_w2, dv_stream_t stream) {
+  if (!w || !dims || !sel || !sel->head_idx || !sel->head_count || !sel->idx || !sel->count) return DV_ERR_ARG;
+  const dv_dims& D = *dims;
+  if (!dims_ok(D) || D.h < 1 || pos < 0 || pos >= D.cap) return DV_ERR_ARG;
+  if (!dtype_ok(w->wdtype) || !dtype_ok(w->kvdtype)) return DV_ERR_ARG;
+  if (!ok_ptr(w->Wqkv) || !ok_ptr(w->WOt) || !ok_ptr(w->Kc) || !ok_ptr(w->Vc) || !ok_ptr(w->W1t) ||
+      !ok_ptr(w->W2t))
+    return DV_ERR_ALIGN;
+  PrefetchArgs a;
+  a.Wqkv = static_cast<const char*>(w->Wqkv);
+  a.WOt = static_cast<const char*>(w->WOt);
+  a.Kc = static_cast<const char*>(w->Kc);
+  a.Vc = static_cast<const char*>(w->Vc);
+  a.W1t = static_cast<const char*>(w->W1t);
+  a.W2t = static_cast<const char*>(w->W2t);
+  a.head_idx = sel->head_idx;
+  a.head_count = sel->head_count;
+  a.idx = sel->idx;
+  a.count = sel->count;
+  a.kh_max = D.kh_max;
+  a.k_max = D.k_max;
+  a.B = D.B;
+  a.h = D.h;
+  a.dh = D.dh;
+  a.d = D.d;
+  a.N = D.N;
+  a.cap = D.cap;
+  a.pos = pos;
+  a.wbytes = wbytes_of(w->wdtype);
+  a.kvbytes = wbytes_of(w->kvdtype);
+  a.with_w2 = with_w2 ? 1 : 0;
+  return cuda_status(launch(prefetch_layer_kernel, dim3(64), 256, 0, reinterpret_cast<cudaStream_t>(stream), a));
 }
 
 dv_status dv_layernorm(const float* x, int B, int d, const float* g, const float* beta, float eps, float* y,
@@ -616,11 +1163,18 @@ dv_status dv_predict_layer(const dv_layer_weights* w, const dv_dims* dims, const
   const Layout L = layout(D, wbytes_of(w->wdtype));
   DV_CHECK(check_ws(L, ws, ws_bytes));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  DV_CHECK(do_predict_heads(L, ws, y, D.B, D.d, D.h, w->PA, w->wdtype, p->k_h, p->tau_h, p->mode_h, out->scores_h,
-                            out->head_idx, out->head_count, st));
-  DV_CHECK(do_predict_mlp(L, ws, y, D.B, D.d, D.r, D.N, w->At, w->Bm, w->b1, w->wdtype, p->k, p->tau, p->mode,
-                          out->scores, out->idx, out->count, st));
-  return DV_OK;
+  if (fused_ok(D, w->wdtype)) {
+    DV_CHECK(fused_predict(L, ws, w, D, p, y, true, true, out->scores_h, out->head_idx, out->head_count, out->scores,
+                           out->idx, out->count, st));
+  } else {
+    DV_CHECK(do_predict_heads(L, ws, y, D.B, D.d, D.h, w->PA, w->wdtype, p->k_h, p->tau_h, p->mode_h, out->scores_h,
+                              out->head_idx, out->head_count, st));
+    DV_CHECK(do_predict_mlp(L, ws, y, D.B, D.d, D.r, D.N, w->At, w->Bm, w->b1, w->wdtype, p->k, p->tau, p->mode,
+                            out->scores, out->idx, out->count, st));
+  }
+  // consumers on other streams read the sets before their own dependency
+  // wait; the gate makes every such consumer start after the sets are done
+  return cuda_status(launch(gate_kernel, dim3(1), dim3(32), 0, st));
 }
 
 }  // extern "C"

@@ -1,0 +1,1123 @@
+// Fused per-layer kernels of the decode step.
+//
+// One layer runs as three kernels on the main stream:
+//   attn_in_kernel    LN1(x), Q/K/V of the selected heads, KV append
+//   attn_out_kernel   split attention + combine + W^O, one thread-block
+//                     cluster per selected head (DSMEM combine)
+//   mlp_block_kernel  LN2, W1 gather + b1 + ReLU, W2 gather-axpy
+// and the look-ahead predictor as two kernels on a side stream:
+//   predict_a_kernel  head scores and z = y A (+ head selection, last CTA)
+//   predict_b_kernel  neuron scores z B^T + b1 with a digit histogram
+//                     (+ exact top-k finish, last CTA)
+//
+// The residual stream moves x -> t1 -> x through the three main kernels:
+// attn_in zeroes t1, attn_out adds x + MHA(yA) into t1 and zeroes x, and
+// mlp_block adds t1 + MLP(yM) into x. Every block output is accumulated with
+// vector float atomics; the one CTA that owns a column slice adds the
+// residual (and the bias) exactly once.
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include "dv_kernels.cuh"
+
+namespace dv {
+
+namespace cg = cooperative_groups;
+
+constexpr int FUSED_THREADS = 256;
+constexpr int FUSED_WARPS = FUSED_THREADS / 32;
+constexpr int HSEL_MAX = 1024;  // heads handled by the in-kernel head selection
+
+// LayerNorm of every batch row of x [nb][d] into dst [nb][d] (shared
+// memory): one pass of 16-byte loads brings x in (all loads in flight, one
+// global round trip), then mean and biased variance are reduced from shared
+// memory and dst is normalised in place: (x - mean) / sqrt(var + eps) * g + beta.
+template <int NB>
+__device__ __forceinline__ void ln_to_smem(const float* __restrict__ x, int d, int nb, float eps,
+                                           const float* __restrict__ g, const float* __restrict__ beta,
+                                           float* __restrict__ dst, float* red) {
+  const int n4 = (nb * d) >> 2, d4 = d >> 2;
+  const float4* xs = reinterpret_cast<const float4*>(x);
+  float4* ds = reinterpret_cast<float4*>(dst);
+  constexpr int UNR = 4;
+  for (int i0 = threadIdx.x; i0 < n4; i0 += FUSED_THREADS * UNR) {
+    float4 v[UNR];
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) {
+      const int i = i0 + u * FUSED_THREADS;
+      if (i < n4) v[u] = __ldcg(xs + i);
+    }
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) {
+      const int i = i0 + u * FUSED_THREADS;
+      if (i < n4) ds[i] = v[u];
+    }
+  }
+  __syncthreads();
+  for (int b = 0; b < nb && b < NB; ++b) {
+    const float4* xr = ds + (size_t)b * d4;
+    float s = 0.f;
+    for (int i = threadIdx.x; i < d4; i += FUSED_THREADS) {
+      const float4 v = xr[i];
+      s += (v.x + v.y) + (v.z + v.w);
+    }
+    const float m = block_sum<FUSED_THREADS>(s, red) / (float)d;
+    float q = 0.f;
+    for (int i = threadIdx.x; i < d4; i += FUSED_THREADS) {
+      const float4 v = xr[i];
+      const float a = v.x - m, c = v.y - m, e = v.z - m, f = v.w - m;
+      q += (a * a + c * c) + (e * e + f * f);
+    }
+    const float rs = rsqrtf(block_sum<FUSED_THREADS>(q, red) / (float)d + eps);
+    float4* yr = ds + (size_t)b * d4;
+    for (int i = threadIdx.x; i < d4; i += FUSED_THREADS) {
+      const float4 v = yr[i];
+      float4 o = make_float4((v.x - m) * rs, (v.y - m) * rs, (v.z - m) * rs, (v.w - m) * rs);
+      if (g) {
+        const float4 gg = __ldg(reinterpret_cast<const float4*>(g) + i);
+        o.x *= gg.x; o.y *= gg.y; o.z *= gg.z; o.w *= gg.w;
+      }
+      if (beta) {
+        const float4 bb = __ldg(reinterpret_cast<const float4*>(beta) + i);
+        o.x += bb.x; o.y += bb.y; o.z += bb.z; o.w += bb.w;
+      }
+      yr[i] = o;
+    }
+  }
+  __syncthreads();
+}
+
+// ----------------------------------------------------------------------------
+// Row dots against a normalised input held in shared memory. Same load
+// pattern as warp_rows_dot (RPW rows, U column steps, 8 loads in flight per
+// lane), with the first column step optionally issued before the caller's
+// griddep_wait (its rows do not depend on the previous kernel).
+// ----------------------------------------------------------------------------
+template <typename T, int RPW, int U>
+struct RowLoads {
+  uint4 w[U][RPW];
+};
+
+template <typename T, int RPW, int U>
+__device__ __forceinline__ void issue_row_loads(RowLoads<T, RPW, U>& L, const T* const (&rowp)[RPW],
+                                                const bool (&valid)[RPW], int nvec, int v0) {
+  constexpr int E = WT<T>::E;
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int v = v0 + u * 32;
+#pragma unroll
+    for (int r = 0; r < RPW; ++r)
+      L.w[u][r] = (valid[r] && v < nvec) ? ld_stream(rowp[r] + (size_t)v * E) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+template <typename T, int NB, int RPW, int U>
+__device__ __forceinline__ void consume_row_loads(const RowLoads<T, RPW, U>& L, const float* __restrict__ ys, int d,
+                                                  int nb, int nvec, int v0, float (&acc)[RPW][NB]) {
+  constexpr int E = WT<T>::E;
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int v = v0 + u * 32;
+    if (v < nvec) {
+      float wf[RPW][E];
+#pragma unroll
+      for (int r = 0; r < RPW; ++r) WT<T>::unpack(L.w[u][r], wf[r]);
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        if (b < nb) {
+          float xv[E];
+          const float4* xp = reinterpret_cast<const float4*>(ys + (size_t)b * d + (size_t)v * E);
+#pragma unroll
+          for (int e4 = 0; e4 < E / 4; ++e4) {
+            const float4 t = xp[e4];
+            xv[4 * e4 + 0] = t.x;
+            xv[4 * e4 + 1] = t.y;
+            xv[4 * e4 + 2] = t.z;
+            xv[4 * e4 + 3] = t.w;
+          }
+#pragma unroll
+          for (int r = 0; r < RPW; ++r)
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc[r][b] = fmaf(wf[r][e], xv[e], acc[r][b]);
+        }
+      }
+    }
+  }
+}
+
+// Full dot of RPW rows with ys, where the loads of the first column step
+// (v0 = lane) were already issued into L.
+template <typename T, int NB, int RPW, int U>
+__device__ __forceinline__ void finish_rows_dot(RowLoads<T, RPW, U>& L, const T* const (&rowp)[RPW],
+                                                const bool (&valid)[RPW], const float* __restrict__ ys, int d,
+                                                int nb, float (&acc)[RPW][NB]) {
+  constexpr int E = WT<T>::E;
+  const int lane = threadIdx.x & 31;
+  const int nvec = d / E;
+#pragma unroll
+  for (int r = 0; r < RPW; ++r)
+#pragma unroll
+    for (int b = 0; b < NB; ++b) acc[r][b] = 0.f;
+  consume_row_loads<T, NB, RPW, U>(L, ys, d, nb, nvec, lane, acc);
+  for (int v0 = lane + 32 * U; v0 < nvec; v0 += 32 * U) {
+    issue_row_loads<T, RPW, U>(L, rowp, valid, nvec, v0);
+    consume_row_loads<T, NB, RPW, U>(L, ys, d, nb, nvec, v0, acc);
+  }
+#pragma unroll
+  for (int r = 0; r < RPW; ++r)
+#pragma unroll
+    for (int b = 0; b < NB; ++b) acc[r][b] = warp_sum(acc[r][b]);
+}
+
+// ----------------------------------------------------------------------------
+// mlp_block_kernel: x (+)= t1 + sum_j relu(yM . W1t[idx_j] + b1[idx_j]) W2t[idx_j]
+// (+ b2), yM = LN2(t1) (eq. (1)). CTA g owns selection slots
+// [g*cnt/G, (g+1)*cnt/G): it forms their activations (warp per row), keeps
+// the nonzero ones, streams their W2 rows over all d columns and adds its
+// partial sums to x. CTA 0 also adds t1 and b2. x must be zero on entry.
+// ----------------------------------------------------------------------------
+struct MlpBlockArgs {
+  const float* t1;  // [B][d] block input (residual after attention)
+  float* x;         // [B][d] output, zero on entry
+  const float* ln_g;
+  const float* ln_b;
+  float eps;
+  const void* W1t;
+  const float* b1;
+  const void* W2t;
+  const float* b2;
+  const int32_t* idx;
+  const int32_t* count;
+  int k_max, d, N, nb, G, sets_ready;
+  float* yM_out;  // optional copy of LN2(t1), written by CTA 0
+  int* status;
+};
+
+constexpr int MLP_MAX_ROWS = 64;  // selection slots per CTA held in shared memory at once
+
+template <typename T, int NB, int RPW, int U>
+__global__ void __launch_bounds__(FUSED_THREADS) mlp_block_kernel(MlpBlockArgs a) {
+  constexpr int E = WT<T>::E;
+  extern __shared__ __align__(16) float s_y[];  // [nb][d] normalised input
+  __shared__ float red[FUSED_WARPS];
+  __shared__ float s_act[MLP_MAX_ROWS][NB];
+  __shared__ int s_row[MLP_MAX_ROWS];
+  __shared__ int s_nz[MLP_MAX_ROWS];
+  __shared__ int s_list[MLP_MAX_ROWS];
+  __shared__ int s_nlist;
+  const T* W1t = static_cast<const T*>(a.W1t);
+  const T* W2t = static_cast<const T*>(a.W2t);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nvec = a.d / E;
+  griddep_launch();
+
+  int cnt = 0, j0 = 0, j1 = 0;
+  auto slot_range = [&]() {
+    cnt = *a.count;
+    if (cnt > a.k_max || cnt < 0) {
+      if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(a.status, 1);
+      cnt = cnt < 0 ? 0 : a.k_max;
+    }
+    j0 = (int)(((long long)cnt * blockIdx.x) / a.G);
+    j1 = (int)(((long long)cnt * (blockIdx.x + 1)) / a.G);
+  };
+  // rows of the first chunk handled by this warp
+  const T* rowp[RPW];
+  bool valid[RPW];
+  int rows[RPW];
+  float bias[RPW];
+  auto setup_rows = [&](int base, int limit) {
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+      const int j = base + warp * RPW + r;
+      int row = j < limit ? a.idx[j] : -1;
+      if (j < limit && (row < 0 || row >= a.N)) {
+        if (lane == 0) raise_status(a.status, 2);
+        row = -1;
+      }
+      rows[r] = row;
+      valid[r] = row >= 0;
+      rowp[r] = W1t + (size_t)(row >= 0 ? row : 0) * a.d;
+      bias[r] = row >= 0 ? a.b1[row] : 0.f;
+    }
+  };
+  RowLoads<T, RPW, U> L;
+  if (a.sets_ready) {  // the sets were made before the previous kernel: start streaming W1 now
+    slot_range();
+    setup_rows(j0, min(j1, j0 + MLP_MAX_ROWS));
+    issue_row_loads<T, RPW, U>(L, rowp, valid, nvec, lane);
+  }
+  griddep_wait();
+  if (!a.sets_ready) {
+    slot_range();
+    setup_rows(j0, min(j1, j0 + MLP_MAX_ROWS));
+    issue_row_loads<T, RPW, U>(L, rowp, valid, nvec, lane);
+  }
+  ln_to_smem<NB>(a.t1, a.d, a.nb, a.eps, a.ln_g, a.ln_b, s_y, red);
+  if (blockIdx.x == 0 && a.yM_out) {
+    const int n4 = (a.nb * a.d) >> 2;
+    for (int i = threadIdx.x; i < n4; i += FUSED_THREADS)
+      reinterpret_cast<float4*>(a.yM_out)[i] = reinterpret_cast<const float4*>(s_y)[i];
+  }
+
+  const int col = threadIdx.x * E;  // first column of this thread in each 256*E tile
+  for (int c0 = j0; c0 < j1 || (c0 == j0 && blockIdx.x == 0); c0 += MLP_MAX_ROWS) {
+    const int nrows = max(0, min(MLP_MAX_ROWS, j1 - c0));
+    // activations of this chunk: warp w handles slots w*RPW .. (then strided)
+    for (int base = 0; base < nrows; base += FUSED_WARPS * RPW) {
+      if (!(c0 == j0 && base == 0)) {
+        setup_rows(c0 + base, c0 + nrows);
+        issue_row_loads<T, RPW, U>(L, rowp, valid, nvec, lane);
+      }
+      float acc[RPW][NB];
+      finish_rows_dot<T, NB, RPW, U>(L, rowp, valid, s_y, a.d, a.nb, acc);
+      if (lane == 0) {
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) {
+          const int s = base + warp * RPW + r;
+          if (s < nrows) {
+            int nz = 0;
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+              const float v = (valid[r] && b < a.nb) ? fmaxf(acc[r][b] + bias[r], 0.f) : 0.f;
+              s_act[s][b] = v;
+              nz |= v > 0.f;
+            }
+            s_nz[s] = nz;
+            s_row[s] = rows[r];
+          }
+        }
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {  // compact the nonzero slots, in slot order
+      int base = 0;
+      for (int s0 = 0; s0 < nrows; s0 += 32) {
+        const int s = s0 + lane;
+        const int nz = s < nrows ? s_nz[s] : 0;
+        const unsigned bal = __ballot_sync(0xffffffffu, nz);
+        if (nz) s_list[base + __popc(bal & ((1u << lane) - 1u))] = s;
+        base += __popc(bal);
+      }
+      if (lane == 0) s_nlist = base;
+    }
+    __syncthreads();
+    const int nl = s_nlist;
+    const bool add_residual = blockIdx.x == 0 && c0 == j0;
+    // W2 rows of the nonzero slots, accumulated over all d columns
+    for (int t0 = 0; t0 < a.d; t0 += FUSED_THREADS * E) {
+      const int c = t0 + col;
+      const bool colok = c < a.d;
+      float acc[NB][E];
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[b][e] = 0.f;
+      if (add_residual && colok) {
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          if (b < a.nb) {
+#pragma unroll
+            for (int e4 = 0; e4 < E / 4; ++e4) {
+              const float4 t = __ldcg(reinterpret_cast<const float4*>(a.t1 + (size_t)b * a.d + c) + e4);
+              float4 bb = make_float4(0.f, 0.f, 0.f, 0.f);
+              if (a.b2) bb = __ldg(reinterpret_cast<const float4*>(a.b2 + c) + e4);
+              acc[b][4 * e4 + 0] = t.x + bb.x;
+              acc[b][4 * e4 + 1] = t.y + bb.y;
+              acc[b][4 * e4 + 2] = t.z + bb.z;
+              acc[b][4 * e4 + 3] = t.w + bb.w;
+            }
+          }
+        }
+      }
+      for (int i0 = 0; i0 < nl; i0 += AX_U) {
+        uint4 w[AX_U];
+#pragma unroll
+        for (int u = 0; u < AX_U; ++u) {
+          const int i = i0 + u;
+          w[u] = (colok && i < nl) ? ld_stream(W2t + (size_t)s_row[s_list[i]] * a.d + c) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < AX_U; ++u) {
+          const int i = i0 + u;
+          if (i < nl) {
+            float wf[E];
+            WT<T>::unpack(w[u], wf);
+            const int s = s_list[i];
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+              const float cb = s_act[s][b];
+#pragma unroll
+              for (int e = 0; e < E; ++e) acc[b][e] = fmaf(cb, wf[e], acc[b][e]);
+            }
+          }
+        }
+      }
+      if (colok && (nl > 0 || add_residual)) {
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          if (b < a.nb) {
+#pragma unroll
+            for (int e4 = 0; e4 < E / 4; ++e4)
+              atomicAdd(reinterpret_cast<float4*>(a.x + (size_t)b * a.d + c + 4 * e4),
+                        make_float4(acc[b][4 * e4], acc[b][4 * e4 + 1], acc[b][4 * e4 + 2], acc[b][4 * e4 + 3]));
+          }
+        }
+      }
+    }
+    __syncthreads();
+    if (nrows == 0) break;
+  }
+}
+
+// ----------------------------------------------------------------------------
+// attn_in_kernel: yA = LN1(x); for the selected heads q, k, v = yA Wqkv[i]^T
+// (+ bqkv); q -> workspace, k and v -> KV cache slot pos (eq. (2); KV-cache
+// figure (b)). Warp per output row, as qkv_kernel. CTA 0 also writes yA (for
+// the look-ahead predictor) and zeroes t1 (the next kernel accumulates into
+// it).
+// ----------------------------------------------------------------------------
+struct AttnInArgs {
+  const float* x;
+  float* t1;
+  float* yA_out;
+  const float* ln_g;
+  const float* ln_b;
+  float eps;
+  const void* Wqkv;
+  const float* bqkv;
+  const int32_t* head_idx;
+  const int32_t* head_count;
+  int kh_max;
+  float* q;
+  void* Kc;
+  void* Vc;
+  int h, dh, d, cap, pos, nb, sets_ready;
+  int* status;
+};
+
+template <typename T, int NB, int RPW, int U>
+__global__ void __launch_bounds__(FUSED_THREADS) attn_in_kernel(AttnInArgs a) {
+  constexpr int E = WT<T>::E;
+  extern __shared__ __align__(16) float s_y[];
+  __shared__ float red[FUSED_WARPS];
+  const T* Wqkv = static_cast<const T*>(a.Wqkv);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int per = 3 * a.dh;
+  const int nvec = a.d / E;
+  const int slot0 = (blockIdx.x * FUSED_WARPS + warp) * RPW;
+  griddep_launch();
+  const T* rowp[RPW];
+  bool valid[RPW];
+  int heads[RPW];
+  auto setup = [&]() {
+    int hc = *a.head_count;
+    if (hc > a.kh_max || hc < 0) {
+      if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(a.status, 1);
+      hc = hc < 0 ? 0 : a.kh_max;
+    }
+    const int nslot = hc * per;
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+      const int slot = slot0 + r;
+      int head = -1;
+      if (slot < nslot) {
+        head = a.head_idx[slot / per];
+        if (head < 0 || head >= a.h) {
+          if (lane == 0) raise_status(a.status, 2);
+          head = -1;
+        }
+      }
+      heads[r] = head;
+      valid[r] = head >= 0;
+      rowp[r] = Wqkv + ((size_t)(head >= 0 ? head : 0) * per + (slot % per)) * a.d;
+    }
+  };
+  RowLoads<T, RPW, U> L;
+  if (a.sets_ready) {
+    setup();
+    issue_row_loads<T, RPW, U>(L, rowp, valid, nvec, lane);
+  }
+  griddep_wait();
+  if (!a.sets_ready) {
+    setup();
+    issue_row_loads<T, RPW, U>(L, rowp, valid, nvec, lane);
+  }
+  ln_to_smem<NB>(a.x, a.d, a.nb, a.eps, a.ln_g, a.ln_b, s_y, red);
+  if (blockIdx.x == 0) {
+    const int n4 = (a.nb * a.d) >> 2;
+    for (int i = threadIdx.x; i < n4; i += FUSED_THREADS) {
+      reinterpret_cast<float4*>(a.t1)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (a.yA_out) reinterpret_cast<float4*>(a.yA_out)[i] = reinterpret_cast<const float4*>(s_y)[i];
+    }
+  }
+  float acc[RPW][NB];
+  finish_rows_dot<T, NB, RPW, U>(L, rowp, valid, s_y, a.d, a.nb, acc);
+  T* Kc = static_cast<T*>(a.Kc);
+  T* Vc = static_cast<T*>(a.Vc);
+#pragma unroll
+  for (int r = 0; r < RPW; ++r) {
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (lane == ((r * NB + b) & 31) && valid[r] && b < a.nb) {
+        const int slot = slot0 + r;
+        const int p = slot / per, rem = slot % per, m = rem / a.dh, c = rem % a.dh;
+        float v = acc[r][b];
+        if (a.bqkv) v += a.bqkv[(size_t)heads[r] * per + rem];
+        if (m == 0) {
+          a.q[((size_t)b * a.kh_max + p) * a.dh + c] = v;
+        } else {
+          T* cache = (m == 1) ? Kc : Vc;
+          cache[(((size_t)b * a.h + heads[r]) * a.cap + a.pos) * a.dh + c] = WT<T>::store_cvt(v);
+        }
+      }
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// attn_out_kernel: for selected head slot p (grid y) a cluster of CS CTAs
+// splits the keys 0..pos: each CTA stages its K/V range in shared memory
+// (slots below pos before griddep_wait: they do not depend on attn_in), forms
+// the partial (m, l, acc) of the max-subtracted softmax, and after a cluster
+// barrier every CTA combines the CS partials through distributed shared
+// memory into H (eq. (2): D_i^{-1} exp(.) X W_i^V). CTA c then multiplies H
+// by its column slice of W_i^O and adds the result to t1. The cluster of
+// slot 0 also moves the residual: t1 += x (+ bO) on its slices, then x = 0.
+// ----------------------------------------------------------------------------
+struct AttnOutArgs {
+  const float* q;
+  const void* Kc;
+  const void* Vc;
+  const void* WOt;
+  const float* bO;
+  const int32_t* head_idx;
+  const int32_t* head_count;
+  int kh_max;
+  float* x;
+  float* t1;
+  int h, dh, d, cap, pos, nb, S, sets_ready;
+  float scale;
+  int* status;
+};
+
+template <typename KT, int DH, int CS, int NB>
+__global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) {
+  constexpr int E = WT<KT>::E;
+  constexpr int G = DH / E;                 // lanes per key row
+  constexpr int KPP = FUSED_THREADS / G;    // keys per pass
+  extern __shared__ __align__(16) unsigned char s_dyn[];
+  KT* sK = reinterpret_cast<KT*>(s_dyn);                       // [S][DH]
+  KT* sV = sK + (size_t)a.S * DH;                              // [S][DH]
+  float* sE = reinterpret_cast<float*>(sV + (size_t)a.S * DH); // [S]
+  __shared__ __align__(16) float s_part[NB][DH + 2];  // this CTA's partial (m, l, acc)
+  __shared__ __align__(16) float s_H[NB][DH];
+  __shared__ float s_red[KPP * DH > FUSED_THREADS * E ? KPP * DH : FUSED_THREADS * E];
+  __shared__ float red[FUSED_WARPS];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int crank = (int)cluster.block_rank();
+  const int p = blockIdx.y;
+  const int tid = threadIdx.x;
+  const KT* Kc = static_cast<const KT*>(a.Kc);
+  const KT* Vc = static_cast<const KT*>(a.Vc);
+  const int nkeys = a.pos + 1;
+  const int t0 = crank * a.S;
+  const int nk = max(0, min(a.S, nkeys - t0));
+  griddep_launch();
+
+  int hc = 0, head = -1;
+  auto read_head = [&]() {
+    hc = *a.head_count;
+    hc = hc < 0 ? 0 : (hc > a.kh_max ? a.kh_max : hc);
+    head = p < hc ? a.head_idx[p] : -1;
+    if (p < hc && (head < 0 || head >= a.h)) {
+      if (tid == 0 && crank == 0) raise_status(a.status, 2);
+      head = -1;
+    }
+  };
+  // stage K/V of batch row b, keys [t0, t0+nk) except slot pos when `old_only`
+  auto stage = [&](int b, bool old_only, bool new_only) {
+    const int lo = new_only ? (a.pos - t0) : 0;
+    const int hi = old_only ? min(nk, a.pos - t0) : nk;
+    if (hi <= lo) return;
+    const size_t base = (((size_t)b * a.h + head) * a.cap + t0) * DH;
+    const int v0 = lo * DH / E, v1 = hi * DH / E;
+    for (int v = v0 + tid; v < v1; v += FUSED_THREADS) {
+      cp_async16(sK + v * E, Kc + base + (size_t)v * E);
+      cp_async16(sV + v * E, Vc + base + (size_t)v * E);
+    }
+  };
+  const bool pos_in_chunk = a.pos >= t0 && a.pos < t0 + nk;
+  // this CTA's column slice of W_head^O: DH rows of d/CS columns
+  auto prefetch_wo = [&]() {
+    const int cols = a.d / CS;
+    const char* base = static_cast<const char*>(a.WOt) +
+                       ((size_t)head * DH * a.d + (size_t)crank * cols) * sizeof(KT);
+    for (int i = tid; i < DH; i += FUSED_THREADS) prefetch_l2(base + (size_t)i * a.d * sizeof(KT), cols * sizeof(KT));
+  };
+  if (a.sets_ready) {
+    read_head();
+    if (head >= 0) {
+      stage(0, true, false);
+      prefetch_wo();
+    }
+  }
+  griddep_wait();
+  if (!a.sets_ready) {
+    read_head();
+    if (head >= 0) stage(0, true, false);
+  }
+  const bool active = head >= 0;
+  // ---- partial attention over this CTA's keys, per batch row ----
+  if (active) {
+    for (int b = 0; b < a.nb; ++b) {
+      if (b > 0) {
+        __syncthreads();  // previous row's tiles are consumed
+        stage(b, false, false);
+      } else if (pos_in_chunk) {
+        stage(0, false, true);  // slot pos, written by attn_in
+      }
+      const int g = tid % G, j = tid / G;
+      float qv[E];
+      const float* qp = a.q + ((size_t)b * a.kh_max + p) * DH + g * E;
+#pragma unroll
+      for (int e = 0; e < E; ++e) qv[e] = __ldcg(qp + e) * a.scale;
+      cp_async_wait_all();
+      __syncthreads();
+      for (int tb = 0; tb < nk; tb += KPP) {
+        const int t = tb + j;
+        float dot = 0.f;
+        if (t < nk) {
+          float kf[E];
+          WT<KT>::unpack(*reinterpret_cast<const uint4*>(sK + t * DH + g * E), kf);
+#pragma unroll
+          for (int e = 0; e < E; ++e) dot = fmaf(qv[e], kf[e], dot);
+        }
+#pragma unroll
+        for (int o = G / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        if (g == 0 && t < nk) sE[t] = dot;
+      }
+      __syncthreads();
+      float m = -INFINITY;
+      for (int t = tid; t < nk; t += FUSED_THREADS) m = fmaxf(m, sE[t]);
+      m = block_max<FUSED_THREADS>(m, red);
+      float l = 0.f;
+      for (int t = tid; t < nk; t += FUSED_THREADS) {
+        const float pe = __expf(sE[t] - m);
+        sE[t] = pe;
+        l += pe;
+      }
+      l = block_sum<FUSED_THREADS>(l, red);
+      float acc[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = 0.f;
+      for (int t = j; t < nk; t += KPP) {
+        float vf[E];
+        WT<KT>::unpack(*reinterpret_cast<const uint4*>(sV + t * DH + g * E), vf);
+        const float pe = sE[t];
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] = fmaf(pe, vf[e], acc[e]);
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) s_red[j * DH + g * E + e] = acc[e];
+      __syncthreads();
+      for (int c = tid; c < DH; c += FUSED_THREADS) {
+        float s = 0.f;
+#pragma unroll 4
+        for (int jj = 0; jj < KPP; ++jj) s += s_red[jj * DH + c];
+        s_part[b][2 + c] = s;
+      }
+      if (tid == 0) {
+        s_part[b][0] = nk > 0 ? m : -INFINITY;
+        s_part[b][1] = l;
+      }
+    }
+  }
+  cluster.sync();  // every CTA's partial is complete
+  if (active) {
+    // ---- combine the CS partials of each batch row (distributed smem) ----
+    for (int b = 0; b < a.nb; ++b) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < CS; ++r) {
+        const float* rp = cluster.map_shared_rank(&s_part[0][0], r);
+        M = fmaxf(M, rp[b * (DH + 2)]);
+      }
+      float den = 0.f;
+#pragma unroll
+      for (int r = 0; r < CS; ++r) {
+        const float* rp = cluster.map_shared_rank(&s_part[0][0], r);
+        const float mr = rp[b * (DH + 2)];
+        den += (mr == -INFINITY) ? 0.f : __expf(mr - M) * rp[b * (DH + 2) + 1];
+      }
+      for (int c = tid; c < DH; c += FUSED_THREADS) {
+        float num = 0.f;
+#pragma unroll
+        for (int r = 0; r < CS; ++r) {
+          const float* rp = cluster.map_shared_rank(&s_part[0][0], r);
+          const float mr = rp[b * (DH + 2)];
+          num += (mr == -INFINITY) ? 0.f : __expf(mr - M) * rp[b * (DH + 2) + 2 + c];
+        }
+        s_H[b][c] = num / den;
+      }
+    }
+  }
+  cluster.sync();  // remote partials are no longer read; s_H complete
+  // ---- W^O slice: columns [c_lo, c_hi) of this CTA ----
+  const int cols = a.d / CS;  // d % (8 CS) == 0 is checked on the host
+  const int c_lo = crank * cols;
+  const int ncg = cols / E;   // column groups of E columns
+  const bool residual = (p == 0);
+  if (!active && !residual) return;
+  const KT* WO = static_cast<const KT*>(a.WOt);
+  for (int cg0 = 0; cg0 < ncg; cg0 += FUSED_THREADS) {
+    const int ngrp = min(FUSED_THREADS, ncg - cg0);
+    const int nrg = max(1, FUSED_THREADS / ngrp);  // row groups
+    const int cgi = tid % ngrp, rg = tid / ngrp;
+    const bool thr_ok = rg < nrg && tid < ngrp * nrg;
+    const int c = c_lo + (cg0 + cgi) * E;
+    float acc[NB][E];
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[b][e] = 0.f;
+    if (active && thr_ok) {
+      const KT* Wh = WO + (size_t)head * DH * a.d + c;
+      for (int i0 = rg; i0 < DH; i0 += nrg * AX_U) {
+        uint4 w[AX_U];
+#pragma unroll
+        for (int u = 0; u < AX_U; ++u) {
+          const int i = i0 + u * nrg;
+          w[u] = i < DH ? ld_stream(Wh + (size_t)i * a.d) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < AX_U; ++u) {
+          const int i = i0 + u * nrg;
+          if (i < DH) {
+            float wf[E];
+            WT<KT>::unpack(w[u], wf);
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+              if (b < a.nb) {
+                const float hv = s_H[b][i];
+#pragma unroll
+                for (int e = 0; e < E; ++e) acc[b][e] = fmaf(hv, wf[e], acc[b][e]);
+              }
+            }
+          }
+        }
+      }
+    }
+    // reduce the row groups, one batch row at a time
+    for (int b = 0; b < a.nb && b < NB; ++b) {
+      if (nrg > 1) {
+        __syncthreads();
+        if (thr_ok) {
+#pragma unroll
+          for (int e = 0; e < E; ++e) s_red[(rg * ngrp + cgi) * E + e] = acc[b][e];
+        }
+        __syncthreads();
+      }
+      if (rg == 0 && thr_ok) {
+        float o[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          float sum = acc[b][e];
+          for (int r2 = 1; r2 < nrg; ++r2) sum += s_red[(r2 * ngrp + cgi) * E + e];
+          o[e] = sum;
+        }
+        if (residual) {
+          float* xr = a.x + (size_t)b * a.d + c;
+#pragma unroll
+          for (int e4 = 0; e4 < E / 4; ++e4) {
+            const float4 xv = __ldcg(reinterpret_cast<const float4*>(xr) + e4);
+            float4 bb = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (a.bO) bb = __ldg(reinterpret_cast<const float4*>(a.bO + c) + e4);
+            o[4 * e4 + 0] += xv.x + bb.x;
+            o[4 * e4 + 1] += xv.y + bb.y;
+            o[4 * e4 + 2] += xv.z + bb.z;
+            o[4 * e4 + 3] += xv.w + bb.w;
+            reinterpret_cast<float4*>(xr)[e4] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+#pragma unroll
+        for (int e4 = 0; e4 < E / 4; ++e4)
+          atomicAdd(reinterpret_cast<float4*>(a.t1 + (size_t)b * a.d + c + 4 * e4),
+                    make_float4(o[4 * e4], o[4 * e4 + 1], o[4 * e4 + 2], o[4 * e4 + 3]));
+      }
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Look-ahead predictor, first kernel: rows [0, h) of PA give the head scores
+// s_A[b][i] = y[b] . PA[i]; rows [h, h + r) of At give z[b][c] = y[b] . At[c]
+// (the first factor of the neuron predictor). The weight rows do not depend
+// on the previous kernel, so their first loads go out before griddep_wait.
+// ----------------------------------------------------------------------------
+struct PredictAArgs {
+  const float* y;  // [B][d]
+  const void* PA;  // [h][d] (null when heads are not predicted)
+  const void* At;  // [r][d] (null when z is not needed)
+  int h, r, d, nb;
+  float* scores_h;  // [B][h]
+  float* z;         // [B][r]
+};
+
+template <typename T, int NB, int RPW, int U>
+__global__ void __launch_bounds__(FUSED_THREADS) predict_a_kernel(PredictAArgs a) {
+  griddep_launch();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int heads = a.PA ? a.h : 0;
+  const int nrows = heads + (a.At ? a.r : 0);
+  const int row0 = (blockIdx.x * FUSED_WARPS + warp) * RPW;
+  const T* rowp[RPW];
+  bool valid[RPW];
+#pragma unroll
+  for (int r = 0; r < RPW; ++r) {
+    const int row = row0 + r;
+    valid[r] = row < nrows;
+    const T* base = row < heads ? static_cast<const T*>(a.PA) + (size_t)row * a.d
+                                : static_cast<const T*>(a.At) + (size_t)(valid[r] ? row - heads : 0) * a.d;
+    rowp[r] = valid[r] ? base : static_cast<const T*>(heads ? a.PA : a.At);
+  }
+  RowLoads<T, RPW, U> L;
+  issue_row_loads<T, RPW, U>(L, rowp, valid, a.d / WT<T>::E, lane);
+  griddep_wait();  // y comes from the previous kernel
+  float acc[RPW][NB];
+  finish_rows_dot<T, NB, RPW, U>(L, rowp, valid, a.y, a.d, a.nb, acc);
+#pragma unroll
+  for (int r = 0; r < RPW; ++r)
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+      if (lane == ((r * NB + b) & 31) && valid[r] && b < a.nb) {
+        const int row = row0 + r;
+        if (row < heads) a.scores_h[(size_t)b * a.h + row] = acc[r][b];
+        else a.z[(size_t)b * a.r + row - heads] = acc[r][b];
+      }
+}
+
+// ----------------------------------------------------------------------------
+// Look-ahead predictor, second kernel: neuron scores s[b][i] = z[b] . Bm[i] +
+// b1[i] (rows of length r); in top-k mode each score also adds one to a
+// global histogram of the top 11 bits of its order-preserving key (the first
+// digit pass of the selection, spread over the whole grid).
+// ----------------------------------------------------------------------------
+constexpr int PB_MAX_N = 65536;
+
+struct PredictBArgs {
+  const float* z;  // [B][r]
+  const void* Bm;  // [N][r]
+  const float* b1; // [N]
+  int N, r, nb, hist_mode;
+  float* scores;   // [B][N]
+  unsigned* hist;  // [B][2048], zero on entry
+};
+
+template <typename T, int NB, int RPW, int U>
+__global__ void __launch_bounds__(FUSED_THREADS) predict_b_kernel(PredictBArgs a) {
+  griddep_launch();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row0 = (blockIdx.x * FUSED_WARPS + warp) * RPW;
+  const T* rowp[RPW];
+  bool valid[RPW];
+  float bias[RPW];
+#pragma unroll
+  for (int r = 0; r < RPW; ++r) {
+    valid[r] = row0 + r < a.N;
+    rowp[r] = static_cast<const T*>(a.Bm) + (size_t)(valid[r] ? row0 + r : 0) * a.r;
+    bias[r] = valid[r] ? a.b1[row0 + r] : 0.f;
+  }
+  RowLoads<T, RPW, U> L;
+  issue_row_loads<T, RPW, U>(L, rowp, valid, a.r / WT<T>::E, lane);
+  griddep_wait();  // z comes from the previous kernel
+  float acc[RPW][NB];
+  finish_rows_dot<T, NB, RPW, U>(L, rowp, valid, a.z, a.r, a.nb, acc);
+  // lane (r * NB + b) % 32 owns score (r, b); lanes with equal histogram
+  // bins are merged before the global atomic (one per distinct bin)
+#pragma unroll
+  for (int c0 = 0; c0 < RPW * NB; c0 += 32) {
+    unsigned bin = 0xffffffffu;
+#pragma unroll
+    for (int r = 0; r < RPW; ++r)
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+        if (r * NB + b >= c0 && r * NB + b < c0 + 32 && lane == r * NB + b - c0 && valid[r] && b < a.nb) {
+          const float v = acc[r][b] + bias[r];
+          a.scores[(size_t)b * a.N + row0 + r] = v;
+          bin = (unsigned)b * SEL_BINS + (ord_key(v) >> 21);
+        }
+    if (a.hist_mode) {
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (bin != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(a.hist + bin, (unsigned)__popc(peers));
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Exact selection after predict_b_kernel. CTAs 0..B-1 take one neuron score
+// row each (1024 threads, keys in shared memory): the bin of the k-th largest
+// key comes from the global histogram (which this kernel clears), the keys in
+// that bin are collected and refined by two more digit passes, and a
+// warp-ordered pass takes every key above the threshold plus the lowest-index
+// copies of the threshold key. The last neuron CTA unites the rows' bitmaps
+// and writes idx / count. CTA B (when heads are predicted) selects the heads
+// from their scores by rank (few heads: direct comparison).
+// ----------------------------------------------------------------------------
+constexpr int SF_CAND = 4096;
+
+struct SelectFinishArgs {
+  const float* scores;  // [B][N]
+  unsigned* hist;       // [B][2048]
+  uint32_t* bitmaps;    // [B][N/32]
+  unsigned* ticket;
+  int neuron_rows;      // B when the neuron set is selected, else 0
+  int N, nb, k, mode;
+  float tau;
+  int32_t* idx;
+  int32_t* count;
+  const float* scores_h;  // [B][h] or null
+  int h, k_h, mode_h;
+  float tau_h;
+  int32_t* head_idx;
+  int32_t* head_count;
+};
+
+__global__ void __launch_bounds__(SEL_THREADS) select_finish_kernel(SelectFinishArgs a) {
+  extern __shared__ uint32_t s_keys[];  // [N] for a neuron row, [h] for the head row
+  __shared__ unsigned s_h[SEL_BINS];
+  __shared__ uint32_t s_cand[SF_CAND];
+  __shared__ uint32_t s_hsel[HSEL_MAX / 32];
+  __shared__ uint32_t s_bm[SEL_SMEM_KEYS / 32];
+  __shared__ unsigned sc[SEL_WARPS + 1];
+  __shared__ unsigned s_digit, s_kk, s_ncand, s_last;
+  griddep_launch();
+  griddep_wait();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  if ((int)blockIdx.x == a.neuron_rows) {
+    // ---- heads: the union over rows of each row's k_h best (or > tau) ----
+    const int h = a.h, nw = (h + 31) >> 5;
+    for (int w = tid; w < nw; w += SEL_THREADS) s_hsel[w] = 0u;
+    for (int b = 0; b < a.nb; ++b) {
+      __syncthreads();
+      for (int i = tid; i < h; i += SEL_THREADS) s_keys[i] = ord_key(a.scores_h[(size_t)b * h + i]);
+      __syncthreads();
+      for (int i = tid; i < h; i += SEL_THREADS) {
+        bool take;
+        if (a.mode_h == 1) {
+          take = a.scores_h[(size_t)b * h + i] > a.tau_h;
+        } else {
+          const uint32_t ki = s_keys[i];
+          int rank = 0;
+          for (int j = 0; j < h; ++j) {
+            const uint32_t kj = s_keys[j];
+            rank += (kj > ki) || (kj == ki && j < i);
+          }
+          take = rank < a.k_h;
+        }
+        if (take) atomicOr(&s_hsel[i >> 5], 1u << (i & 31));
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      unsigned base = 0;
+      for (int w0 = 0; w0 < nw; w0 += 32) {
+        const int w = w0 + lane;
+        const uint32_t u = w < nw ? s_hsel[w] : 0u;
+        const unsigned c = __popc(u);
+        unsigned incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        unsigned off = base + incl - c;
+        uint32_t v = u;
+        while (v) {
+          const int jb = __ffs(v) - 1;
+          v &= v - 1u;
+          a.head_idx[off++] = w * 32 + jb;
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) *a.head_count = (int32_t)base;
+    }
+    return;
+  }
+
+  // ---- one neuron score row ----
+  const int b = blockIdx.x, n = a.N;
+  const float* row = a.scores + (size_t)b * n;
+  const int nw = (n + 31) >> 5;
+  uint32_t* bm = a.bitmaps + (size_t)b * nw;
+  const int wpw = (nw + SEL_WARPS - 1) / SEL_WARPS;
+  const int w0 = warp * wpw, w1 = min(nw, w0 + wpw);
+  const bool hist_mode = a.mode == 0 && a.k > 0 && a.k < n;
+  if (!hist_mode) {
+    for (int w = w0; w < w1; ++w) {
+      const int i = w * 32 + lane;
+      const bool take = i < n && (a.mode == 1 ? row[i] > a.tau : a.k > 0);
+      const unsigned word = __ballot_sync(0xffffffffu, take);
+      if (lane == 0) s_bm[w] = word;
+    }
+  } else {
+    {  // keys into shared memory, 8 loads in flight per thread
+      constexpr int UNR = 8;
+      for (int i0 = tid; i0 < n; i0 += SEL_THREADS * UNR) {
+        float v[UNR];
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+          const int i = i0 + u * SEL_THREADS;
+          v[u] = i < n ? row[i] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+          const int i = i0 + u * SEL_THREADS;
+          if (i < n) s_keys[i] = ord_key(v[u]);
+        }
+      }
+    }
+    unsigned* gh = a.hist + (size_t)b * SEL_BINS;
+    for (int i = tid; i < SEL_BINS; i += SEL_THREADS) {
+      s_h[i] = gh[i];
+      gh[i] = 0u;  // cleared for the next call
+    }
+    __syncthreads();
+    uint32_t prefix = 0, mask = 0;
+    unsigned kk = (unsigned)a.k;
+    bool use_cand = true;
+#pragma unroll 1
+    for (int pass = 0; pass < 3; ++pass) {
+      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+      const unsigned dmask = pass == 2 ? 0x3ffu : 0x7ffu;
+      if (pass > 0) {
+        for (int i = tid; i < SEL_BINS; i += SEL_THREADS) s_h[i] = 0u;
+        __syncthreads();
+        const int nc = use_cand ? (int)s_ncand : n;
+        const uint32_t* src = use_cand ? s_cand : s_keys;
+        for (int i = tid; i < nc; i += SEL_THREADS) {
+          const uint32_t key = src[i];
+          if ((key & mask) == prefix) atomicAdd(&s_h[(key >> shift) & dmask], 1u);
+        }
+        __syncthreads();
+      }
+      const unsigned c0 = s_h[SEL_BINS - 1 - 2 * tid], c1 = s_h[SEL_BINS - 2 - 2 * tid];
+      unsigned tot;
+      const unsigned above = block_exclusive_scan<SEL_THREADS>(c0 + c1, sc, &tot);
+      if (above < kk && kk <= above + c0 + c1) {
+        if (kk <= above + c0) {
+          s_digit = SEL_BINS - 1 - 2 * tid;
+          s_kk = kk - above;
+        } else {
+          s_digit = SEL_BINS - 2 - 2 * tid;
+          s_kk = kk - above - c0;
+        }
+      }
+      __syncthreads();
+      prefix |= s_digit << shift;
+      mask |= dmask << shift;
+      kk = s_kk;
+      if (pass == 0) {  // the keys of the boundary bin
+        if (tid == 0) s_ncand = 0u;
+        __syncthreads();
+        for (int i = tid; i < n; i += SEL_THREADS) {
+          const uint32_t key = s_keys[i];
+          if ((key & mask) == prefix) {
+            const unsigned at = atomicAdd(&s_ncand, 1u);
+            if (at < SF_CAND) s_cand[at] = key;
+          }
+        }
+        __syncthreads();
+        use_cand = s_ncand <= SF_CAND;
+      }
+    }
+    unsigned eq = 0;
+    for (int w = w0; w < w1; ++w) {
+      const int i = w * 32 + lane;
+      eq += __popc(__ballot_sync(0xffffffffu, i < n && s_keys[i] == prefix));
+    }
+    if (lane == 0) sc[warp] = eq;
+    __syncthreads();
+    if (warp == 0) {
+      const unsigned v = sc[lane];
+      unsigned incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      sc[lane] = incl - v;
+    }
+    __syncthreads();
+    unsigned rank = sc[warp];
+    for (int w = w0; w < w1; ++w) {
+      const int i = w * 32 + lane;
+      const bool ok = i < n;
+      const uint32_t key = ok ? s_keys[i] : 0u;
+      const bool e = ok && key == prefix;
+      const unsigned em = __ballot_sync(0xffffffffu, e);
+      const unsigned rk = rank + __popc(em & ((1u << lane) - 1u));
+      const unsigned word = __ballot_sync(0xffffffffu, ok && (key > prefix || (e && rk < kk)));
+      if (lane == 0) s_bm[w] = word;
+      rank += __popc(em);
+    }
+  }
+  __syncthreads();
+  // union over the neuron rows: with one row the CTA's own bitmap is the
+  // union; otherwise the rows' bitmaps meet in global memory and the last
+  // CTA (ticket) ORs them, loading every word at once
+  if (a.neuron_rows > 1) {
+    for (int w = tid; w < nw; w += SEL_THREADS) bm[w] = s_bm[w];
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = (atomicAdd(a.ticket, 1u) == (unsigned)a.neuron_rows - 1u);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int w = tid; w < nw; w += SEL_THREADS) {
+      uint32_t u = 0;
+      for (int rr = 0; rr < a.neuron_rows; ++rr) u |= __ldcg(a.bitmaps + (size_t)rr * nw + w);
+      s_bm[w] = u;
+    }
+    __syncthreads();
+    if (tid == 0) *a.ticket = 0u;
+  }
+  unsigned pc = 0;
+  for (int w = w0; w < w1; ++w) pc += __popc(s_bm[w]);
+  if (lane == 0) sc[warp] = pc;
+  __syncthreads();
+  if (warp == 0) {
+    const unsigned v = sc[lane];
+    unsigned incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    sc[lane] = incl - v;
+    if (lane == 31) sc[SEL_WARPS] = incl;
+  }
+  __syncthreads();
+  unsigned off = sc[warp];
+  for (int w = w0; w < w1; ++w) {
+    const uint32_t u = s_bm[w];
+    if ((u >> lane) & 1u) a.idx[off + __popc(u & ((1u << lane) - 1u))] = w * 32 + lane;
+    off += __popc(u);
+  }
+  if (tid == 0) *a.count = (int32_t)sc[SEL_WARPS];
+}
+
+// ----------------------------------------------------------------------------
+// Gate: returns once the previous kernel on its stream has completed and its
+// writes are visible. Ends the look-ahead predictor so that a kernel on
+// another stream that depends on it through an event, and that may be
+// launched early by programmatic dependent launch (stream capture can give
+// such a cross-stream edge the programmatic type), cannot start before the
+// predicted sets are complete: it starts at the earliest when the gate has
+// exited.
+// ----------------------------------------------------------------------------
+__global__ void gate_kernel() { griddep_wait(); }
+
+}  // namespace dv

@@ -294,9 +294,18 @@ __global__ void __launch_bounds__(GEMV_THREADS)
 // strict threshold; the union over rows, compacted to ascending indices.
 // One CTA per score row writes its selection bitmap; the last CTA to finish
 // (ticket) ORs the bitmaps and writes idx / count, then resets the ticket.
+//
+// The k-th largest key is found in three digit passes (11, 11, 10 bits): a
+// shared-memory histogram of the digits of the keys that still match the
+// prefix, then a block-wide suffix scan over the bins. The flag and
+// compaction passes are warp-cooperative (one ballot per 32 indices), so the
+// result comes out in index order: keys above the threshold, then the
+// lowest-index copies of the threshold key.
 // ----------------------------------------------------------------------------
 constexpr int SEL_THREADS = 1024;
+constexpr int SEL_WARPS = SEL_THREADS / 32;
 constexpr int SEL_SMEM_KEYS = 49152;  // rows up to this length keep keys in shared memory
+constexpr int SEL_BINS = 2048;
 
 // Order-preserving map float -> uint32: larger float, larger key. -0.0 maps
 // like +0.0; every NaN maps to 0, below -inf (0x007fffff).
@@ -308,13 +317,18 @@ __device__ __forceinline__ uint32_t ord_key(float s) {
 }
 
 template <bool KEYS_IN_SMEM>
+__device__ __forceinline__ uint32_t sel_key(const uint32_t* s_keys, const float* row, int i) {
+  return KEYS_IN_SMEM ? s_keys[i] : ord_key(__ldcg(row + i));
+}
+
+template <bool KEYS_IN_SMEM>
 __global__ void __launch_bounds__(SEL_THREADS)
     select_kernel(const float* __restrict__ scores, int n, int nrows, int k, float tau, int mode,
                   uint32_t* __restrict__ bitmaps, unsigned* __restrict__ ticket, int32_t* __restrict__ idx,
                   int32_t* __restrict__ count) {
   extern __shared__ uint32_t s_keys[];
-  __shared__ unsigned hist[256];
-  __shared__ unsigned sc[SEL_THREADS / 32 + 1];
+  __shared__ unsigned hist[SEL_BINS];
+  __shared__ unsigned sc[SEL_WARPS + 1];
   __shared__ unsigned s_digit, s_kk, s_last;
   griddep_launch();
   griddep_wait();
@@ -323,103 +337,89 @@ __global__ void __launch_bounds__(SEL_THREADS)
   const float* row = scores + (size_t)b * n;
   const int nw = (n + 31) >> 5;
   uint32_t* bm = bitmaps + (size_t)b * nw;
-  const int wpt = (nw + SEL_THREADS - 1) / SEL_THREADS;  // bitmap words per thread
-  const int w0 = tid * wpt, w1 = min(nw, w0 + wpt);
+  const int wpw = (nw + SEL_WARPS - 1) / SEL_WARPS;  // bitmap words per warp
+  const int w0 = warp * wpw, w1 = min(nw, w0 + wpw);
 
-  if (mode == 1) {  // threshold: s > tau (NaN fails)
+  if (mode == 1 || k >= n || k <= 0) {
+    // threshold s > tau (NaN fails), or all / none
     for (int w = w0; w < w1; ++w) {
-      uint32_t word = 0;
-      for (int j = 0; j < 32; ++j) {
-        const int i = w * 32 + j;
-        if (i < n && row[i] > tau) word |= 1u << j;
-      }
-      bm[w] = word;
-    }
-  } else if (k >= n || k <= 0) {
-    for (int w = w0; w < w1; ++w) {
-      uint32_t word = 0;
-      if (k > 0) {
-        const int rem = n - w * 32;
-        word = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
-      }
-      bm[w] = word;
+      const int i = w * 32 + lane;
+      bool sel;
+      if (mode == 1) sel = i < n && row[i] > tau;
+      else sel = i < n && k > 0;
+      const unsigned word = __ballot_sync(0xffffffffu, sel);
+      if (lane == 0) bm[w] = word;
     }
   } else {
     if (KEYS_IN_SMEM) {
       for (int i = tid; i < n; i += SEL_THREADS) s_keys[i] = ord_key(row[i]);
     }
-    __syncthreads();
     uint32_t prefix = 0, mask = 0;
     unsigned kk = (unsigned)k;
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      for (int i = tid; i < 256; i += SEL_THREADS) hist[i] = 0;
+#pragma unroll 1
+    for (int pass = 0; pass < 3; ++pass) {
+      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);  // digits: bits 31..21, 20..10, 9..0
+      const unsigned dmask = pass == 2 ? 0x3ffu : 0x7ffu;
+      for (int i = tid; i < SEL_BINS; i += SEL_THREADS) hist[i] = 0;
       __syncthreads();
-      for (int base = 0; base < n; base += SEL_THREADS) {
-        const int i = base + tid;
-        unsigned dig = 256u;
-        if (i < n) {
-          const uint32_t key = KEYS_IN_SMEM ? s_keys[i] : ord_key(row[i]);
-          if ((key & mask) == prefix) dig = (key >> shift) & 255u;
-        }
-        const unsigned peers = __match_any_sync(0xffffffffu, dig);
-        if (dig < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[dig], (unsigned)__popc(peers));
+      for (int i = tid; i < n; i += SEL_THREADS) {
+        const uint32_t key = sel_key<KEYS_IN_SMEM>(s_keys, row, i);
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
       }
       __syncthreads();
-      if (warp == 0) {
-        // lane l scans digits 255-8l down to 248-8l
-        unsigned c[8], tot = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          c[j] = hist[255 - 8 * lane - j];
-          tot += c[j];
-        }
-        unsigned incl = tot;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += t;
-        }
-        const unsigned excl = incl - tot;
-        if (excl < kk && kk <= incl) {
-          unsigned cum = excl;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (cum + c[j] >= kk) {
-              s_digit = 255u - 8u * lane - j;
-              s_kk = kk - cum;
-              break;
-            }
-            cum += c[j];
-          }
+      // thread t owns bins 2047-2t and 2046-2t (descending); an exclusive scan
+      // in thread order counts the keys in higher bins
+      const unsigned c0 = hist[SEL_BINS - 1 - 2 * tid], c1 = hist[SEL_BINS - 2 - 2 * tid];
+      unsigned tot;
+      const unsigned above = block_exclusive_scan<SEL_THREADS>(c0 + c1, sc, &tot);
+      if (above < kk && kk <= above + c0 + c1) {
+        if (kk <= above + c0) {
+          s_digit = SEL_BINS - 1 - 2 * tid;
+          s_kk = kk - above;
+        } else {
+          s_digit = SEL_BINS - 2 - 2 * tid;
+          s_kk = kk - above - c0;
         }
       }
       __syncthreads();
       prefix |= s_digit << shift;
-      mask |= 255u << shift;
+      mask |= dmask << shift;
       kk = s_kk;
-      __syncthreads();
     }
     // prefix is the k-th largest key; kk of its copies are taken, lowest
-    // indices first. Ranks among equal keys come from a block scan in index
-    // order (thread t owns words [w0, w1)).
+    // indices first
     unsigned eq = 0;
-    for (int i = w0 * 32; i < min(n, w1 * 32); ++i) {
-      const uint32_t key = KEYS_IN_SMEM ? s_keys[i] : ord_key(row[i]);
-      eq += key == prefix;
-    }
-    unsigned tot;
-    unsigned rank = block_exclusive_scan<SEL_THREADS>(eq, sc, &tot);
     for (int w = w0; w < w1; ++w) {
-      uint32_t word = 0;
-      for (int j = 0; j < 32; ++j) {
-        const int i = w * 32 + j;
-        if (i < n) {
-          const uint32_t key = KEYS_IN_SMEM ? s_keys[i] : ord_key(row[i]);
-          if (key > prefix || (key == prefix && rank++ < kk)) word |= 1u << j;
-        }
+      const int i = w * 32 + lane;
+      const bool e = i < n && sel_key<KEYS_IN_SMEM>(s_keys, row, i) == prefix;
+      eq += __popc(__ballot_sync(0xffffffffu, e));
+    }
+    if (lane == 0) sc[warp] = eq;
+    __syncthreads();
+    if (warp == 0) {
+      const unsigned v = sc[lane];
+      unsigned incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
       }
-      bm[w] = word;
+      sc[lane] = incl - v;
+    }
+    __syncthreads();
+    unsigned rank = sc[warp];
+    for (int w = w0; w < w1; ++w) {
+      const int i = w * 32 + lane;
+      uint32_t key = 0;
+      bool valid = i < n;
+      if (valid) key = sel_key<KEYS_IN_SMEM>(s_keys, row, i);
+      const bool e = valid && key == prefix;
+      const unsigned em = __ballot_sync(0xffffffffu, e);
+      const unsigned r = rank + __popc(em & ((1u << lane) - 1u));
+      const bool sel = valid && (key > prefix || (e && r < kk));
+      const unsigned word = __ballot_sync(0xffffffffu, sel);
+      if (lane == 0) bm[w] = word;
+      rank += __popc(em);
     }
   }
   // union over rows by the last CTA
@@ -429,25 +429,54 @@ __global__ void __launch_bounds__(SEL_THREADS)
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  // the union of the rows' bitmaps, every word loaded at once, kept in the
+  // (now free) key buffer or, for long rows, re-read below
+  uint32_t* s_u = s_keys;
+  const bool u_in_smem = KEYS_IN_SMEM || nw <= 0;
   unsigned pc = 0;
-  for (int w = w0; w < w1; ++w) {
-    uint32_t u = 0;
-    for (int rr = 0; rr < nrows; ++rr) u |= __ldcg(bitmaps + (size_t)rr * nw + w);
-    pc += __popc(u);
-  }
-  unsigned total;
-  unsigned off = block_exclusive_scan<SEL_THREADS>(pc, sc, &total);
-  for (int w = w0; w < w1; ++w) {
-    uint32_t u = 0;
-    for (int rr = 0; rr < nrows; ++rr) u |= __ldcg(bitmaps + (size_t)rr * nw + w);
-    while (u) {
-      const int j = __ffs(u) - 1;
-      u &= u - 1u;
-      idx[off++] = w * 32 + j;
+  if (u_in_smem) {
+    for (int w = tid; w < nw; w += SEL_THREADS) {
+      uint32_t u = 0;
+      for (int rr = 0; rr < nrows; ++rr) u |= __ldcg(bitmaps + (size_t)rr * nw + w);
+      s_u[w] = u;
+    }
+    __syncthreads();
+    for (int w = w0; w < w1; ++w) pc += __popc(s_u[w]);
+  } else {
+    for (int w = w0; w < w1; ++w) {
+      uint32_t u = 0;
+      for (int rr = lane; rr < nrows; rr += 32) u |= __ldcg(bitmaps + (size_t)rr * nw + w);
+      pc += __popc(__reduce_or_sync(0xffffffffu, u));
     }
   }
+  if (lane == 0) sc[warp] = pc;
+  __syncthreads();
+  if (warp == 0) {
+    const unsigned v = sc[lane];
+    unsigned incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    sc[lane] = incl - v;
+    if (lane == 31) sc[SEL_WARPS] = incl;
+  }
+  __syncthreads();
+  unsigned off = sc[warp];
+  for (int w = w0; w < w1; ++w) {
+    uint32_t u = 0;
+    if (u_in_smem) {
+      u = s_u[w];
+    } else {
+      for (int rr = lane; rr < nrows; rr += 32) u |= __ldcg(bitmaps + (size_t)rr * nw + w);
+      u = __reduce_or_sync(0xffffffffu, u);
+    }
+    if ((u >> lane) & 1u) idx[off + __popc(u & ((1u << lane) - 1u))] = w * 32 + lane;
+    off += __popc(u);
+  }
   if (tid == 0) {
-    *count = (int32_t)total;
+    *count = (int32_t)sc[SEL_WARPS];
     *ticket = 0u;
   }
 }
@@ -728,6 +757,82 @@ __global__ void __launch_bounds__(AX_THREADS)
           atomicAdd(reinterpret_cast<float4*>(out + (size_t)b * d + col + 4 * e4), v);
         }
       }
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// L2 prefetch of one layer's selected parameters. With the look-ahead
+// predictor the sets of layer l+1 are known while layer l runs; this kernel
+// (on the side stream) asks the bulk-copy engine to bring layer l+1's
+// selected Q/K/V and W^O blocks, the selected heads' KV entries and the
+// selected W1 (and optionally W2) rows into L2, so layer l+1's kernels read
+// them from L2. Fire-and-forget: no data moves through the SMs.
+// ----------------------------------------------------------------------------
+constexpr uint32_t PF_CHUNK = 16384;  // bytes per prefetch request
+
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+struct PrefetchArgs {
+  const char* Wqkv;
+  const char* WOt;
+  const char* Kc;
+  const char* Vc;
+  const char* W1t;
+  const char* W2t;
+  const int32_t* head_idx;
+  const int32_t* head_count;
+  const int32_t* idx;
+  const int32_t* count;
+  int kh_max, k_max, B, h, dh, d, N, cap, pos, wbytes, kvbytes, with_w2;
+};
+
+__device__ __forceinline__ void prefetch_range(const char* base, size_t bytes, int chunk) {
+  const size_t off = (size_t)chunk * PF_CHUNK;
+  if (off < bytes) prefetch_l2(base + off, (uint32_t)min((size_t)PF_CHUNK, bytes - off));
+}
+
+__global__ void __launch_bounds__(256) prefetch_layer_kernel(PrefetchArgs a) {
+  griddep_launch();
+  griddep_wait();
+  int hc = *a.head_count, cnt = *a.count;
+  hc = hc < 0 ? 0 : (hc > a.kh_max ? a.kh_max : hc);
+  cnt = cnt < 0 ? 0 : (cnt > a.k_max ? a.k_max : cnt);
+  const size_t qkv = (size_t)3 * a.dh * a.d * a.wbytes, wo = (size_t)a.dh * a.d * a.wbytes;
+  const size_t kv = (size_t)a.pos * a.dh * a.kvbytes, row = (size_t)a.d * a.wbytes;
+  const int nq = (int)((qkv + PF_CHUNK - 1) / PF_CHUNK), nwo = (int)((wo + PF_CHUNK - 1) / PF_CHUNK);
+  const int nkv = (int)((kv + PF_CHUNK - 1) / PF_CHUNK), nrow = (int)((row + PF_CHUNK - 1) / PF_CHUNK);
+  const int per_head = nq + nwo + 2 * a.B * nkv;
+  const int per_neuron = nrow * (a.with_w2 ? 2 : 1);
+  const long long total = (long long)hc * per_head + (long long)cnt * per_neuron;
+  for (long long it = blockIdx.x * 256ll + threadIdx.x; it < total; it += (long long)gridDim.x * 256) {
+    if (it < (long long)hc * per_head) {
+      const int p = (int)(it / per_head);
+      int c = (int)(it % per_head);
+      const int head = a.head_idx[p];
+      if (head < 0 || head >= a.h) continue;
+      if (c < nq) {
+        prefetch_range(a.Wqkv + (size_t)head * qkv, qkv, c);
+      } else if ((c -= nq) < nwo) {
+        prefetch_range(a.WOt + (size_t)head * wo, wo, c);
+      } else {
+        c -= nwo;
+        const int which = c / (a.B * nkv);  // 0: K, 1: V
+        c %= a.B * nkv;
+        const int b = c / nkv;
+        const size_t cache_off = (((size_t)b * a.h + head) * a.cap) * a.dh * a.kvbytes;
+        prefetch_range((which ? a.Vc : a.Kc) + cache_off, kv, c % nkv);
+      }
+    } else {
+      const long long r = it - (long long)hc * per_head;
+      const int j = (int)(r / per_neuron);
+      int c = (int)(r % per_neuron);
+      const int neuron = a.idx[j];
+      if (neuron < 0 || neuron >= a.N) continue;
+      const char* base = (c < nrow ? a.W1t : a.W2t) + (size_t)neuron * row;
+      prefetch_range(base, row, c % nrow);
     }
   }
 }

@@ -25,7 +25,7 @@ class DecoderStack:
     def __init__(self, layers: List[Dict[str, torch.Tensor]], B: int, k: int, k_h: int, scale: float,
                  lookahead: bool = True, eps: float = 1e-5, mode: int = bd.DV_TOPK, tau: float = 0.0,
                  mode_h: int = bd.DV_TOPK, tau_h: float = 0.0, k_max: Optional[int] = None,
-                 kh_max: Optional[int] = None):
+                 kh_max: Optional[int] = None, prefetch: bool = False, prefetch_w2: bool = True):
         t0 = layers[0]
         N, d = t0["W1t"].shape
         h = t0["Wqkv"].shape[0]
@@ -36,6 +36,8 @@ class DecoderStack:
         self.layers = [bd.Layer(t, B, self.k_max, self.kh_max) for t in layers]
         self.p = bd.params(k, k_h, scale, eps, tau, mode, tau_h, mode_h)
         self.lookahead = lookahead
+        self.prefetch = prefetch and lookahead
+        self.prefetch_w2 = prefetch_w2
         D = self.layers[0].dims
         self.ws_main = bd.workspace(bd.DV_OP_DECODE_LAYER, D, dev)
         self.ws_side = bd.workspace(bd.DV_OP_DECODE_LAYER, D, dev)
@@ -51,49 +53,53 @@ class DecoderStack:
         self.idx = [torch.zeros(N, **i32) for _ in range(nL)]
         self.count = [torch.zeros(1, **i32) for _ in range(nL)]
         self.yM = [torch.empty(B, d, **f32) for _ in range(nL)]
-        self.io_sets = [bd.layer_io(yA=self.yA[l], scores_h=self.scores_h[l], head_idx=self.head_idx[l],
+        # the side stream writes a layer's sets here
+        self.io_sets = [bd.layer_io(scores_h=self.scores_h[l], head_idx=self.head_idx[l],
                                     head_count=self.head_count[l], scores=self.scores[l], idx=self.idx[l],
                                     count=self.count[l]) for l in range(nL)]
+        # a layer that predicts its own sets writes them (and yA, yM) here
         self.io_trace = [bd.layer_io(yA=self.yA[l], scores_h=self.scores_h[l], head_idx=self.head_idx[l],
                                      head_count=self.head_count[l], yM=self.yM[l], scores=self.scores[l],
                                      idx=self.idx[l], count=self.count[l]) for l in range(nL)]
-        self.io_given = [bd.layer_io(yA=self.yA[l], head_idx=self.head_idx[l], head_count=self.head_count[l],
-                                     idx=self.idx[l], count=self.count[l]) for l in range(nL)]
-        self.io_trace_yM = [bd.layer_io(yM=self.yM[l]) for l in range(nL)]
-        # layer 0 under look-ahead: the side stream reads yA[0] while layer 0
-        # runs, so layer 0 keeps its own LN1 output in the workspace
-        self.io_trace_no_yA = [bd.layer_io(scores_h=self.scores_h[l], head_idx=self.head_idx[l],
-                                           head_count=self.head_count[l], yM=self.yM[l], scores=self.scores[l],
-                                           idx=self.idx[l], count=self.count[l]) for l in range(nL)]
+        # a layer whose sets were predicted ahead reads them from here ...
+        self.io_given = [bd.layer_io(head_idx=self.head_idx[l], head_count=self.head_count[l], idx=self.idx[l],
+                                     count=self.count[l]) for l in range(nL)]
+        # ... and writes its normalised block inputs here
+        self.io_trace_y = [bd.layer_io(yA=self.yA[l], yM=self.yM[l]) for l in range(nL)]
         self.side = torch.cuda.Stream(device=dev)
         self.ev_yA = [torch.cuda.Event() for _ in range(nL)]
         self.ev_sel = [torch.cuda.Event() for _ in range(nL)]
+        self.ev_join = torch.cuda.Event()
 
     def step(self, x: torch.Tensor, pos: int):
         """One token through every layer, in place on the residual x [B][d]."""
         main = torch.cuda.current_stream()
         nL = len(self.layers)
+        la = self.lookahead and nL > 1
         for l, L in enumerate(self.layers):
-            if not self.lookahead or l == 0:
-                if self.lookahead and nL > 1:
-                    bd.dv_layernorm(x, self.yA[l], L.t.get("ln1_g"), L.t.get("ln1_b"), self.p.eps)
-                    self.ev_yA[l].record(main)
-                    self._predict_next(l)
-                    bd.dv_decode_layer(L, self.p, x, pos, self.ws_main, trace=self.io_trace_no_yA[l])
-                else:
-                    bd.dv_decode_layer(L, self.p, x, pos, self.ws_main, trace=self.io_trace[l])
+            if la and l > 0:
+                main.wait_event(self.ev_sel[l])  # sets of layer l, predicted from layer l-1
+                sel, trace = self.io_given[l], self.io_trace_y[l]
             else:
-                bd.dv_layernorm(x, self.yA[l], L.t.get("ln1_g"), L.t.get("ln1_b"), self.p.eps)
-                if l + 1 < nL:
-                    self.ev_yA[l].record(main)
-                    self._predict_next(l)
-                main.wait_event(self.ev_sel[l])
-                bd.dv_decode_layer(L, self.p, x, pos, self.ws_main, sel=self.io_given[l],
-                                   trace=self.io_trace_yM[l])
+                sel, trace = None, self.io_trace[l]
+            bd.dv_decode_layer_begin(L, self.p, x, pos, self.ws_main, sel=sel, trace=trace)
+            if la and l + 1 < nL:
+                self.ev_yA[l].record(main)  # yA[l] is written by the work just issued
+                self._predict_next(l, pos)
+            bd.dv_decode_layer_end(L, self.p, x, pos, self.ws_main, sel=sel, trace=trace)
+        if la:
+            # join the side stream back into the main stream
+            self.ev_join.record(self.side)
+            main.wait_event(self.ev_join)
 
-    def _predict_next(self, l: int):
-        """Side stream: the sets of layer l+1 from layer l's yA."""
+    def _predict_next(self, l: int, pos: int):
+        """Side stream: the sets of layer l+1 from layer l's yA, then an L2
+        prefetch of the parameters those sets select (layer l+1 runs after
+        layer l on the main stream, and finds them in L2)."""
         self.side.wait_event(self.ev_yA[l])
         bd.dv_predict_layer(self.layers[l + 1], self.p, self.yA[l], self.io_sets[l + 1], self.ws_side,
                             stream=self.side)
         self.ev_sel[l + 1].record(self.side)
+        if self.prefetch:
+            bd.dv_prefetch_layer(self.layers[l + 1], self.io_sets[l + 1], pos, with_w2=self.prefetch_w2,
+                                 stream=self.side)

@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--no-lookahead", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--prefetch", action="store_true", help="L2-prefetch each layer's selected rows on the side stream")
+    ap.add_argument("--no-prefetch-w2", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args()
@@ -147,12 +149,13 @@ class Clocks:
 # ---------------------------------------------------------------------------
 
 
-def build_stack(shape, nlayers, B, k, k_h, lookahead, seed0=1000, layers=None):
+def build_stack(shape, nlayers, B, k, k_h, lookahead, seed0=1000, layers=None, prefetch=False, prefetch_w2=True):
     from attention_predictor_gemv_b200.stack import DecoderStack
 
     if layers is None:
         layers = [wl.make_layer(shape, seed0 + l, "cuda") for l in range(nlayers)]
-    stk = DecoderStack(layers, B, k, k_h, 1.0 / float(np.sqrt(shape.dh)), lookahead=lookahead)
+    stk = DecoderStack(layers, B, k, k_h, 1.0 / float(np.sqrt(shape.dh)), lookahead=lookahead, prefetch=prefetch,
+                       prefetch_w2=prefetch_w2)
     return stk, layers
 
 
@@ -331,7 +334,8 @@ def main():
     k, k_h = wl.k_for(args.k_frac, shape.N), wl.k_for(args.kh_frac, shape.h)
     pos = shape.L
     torch.manual_seed(rank)
-    stk, layers = build_stack(shape, args.layers, B, k, k_h, not args.no_lookahead, seed0=1000 + 100 * rank)
+    pf = dict(prefetch=args.prefetch, prefetch_w2=not args.no_prefetch_w2)
+    stk, layers = build_stack(shape, args.layers, B, k, k_h, not args.no_lookahead, seed0=1000 + 100 * rank, **pf)
     x0 = wl.make_input(shape, 7 + rank, "cuda")
     x = x0.clone()
     g, launches_per_step = capture(stk, x, pos)
@@ -372,7 +376,7 @@ def main():
         for kf in (0.05, 0.10, 0.20, 1.00):
             for hf in (0.25, 0.50, 1.00):
                 kk, hh = wl.k_for(kf, shape.N), wl.k_for(hf, shape.h)
-                s2, _ = build_stack(shape, args.layers, B, kk, hh, not args.no_lookahead, layers=layers)
+                s2, _ = build_stack(shape, args.layers, B, kk, hh, not args.no_lookahead, layers=layers, **pf)
                 g2, _ = capture(s2, x, pos)
                 m2 = time_graph(g2, max(10, args.steps // 2), 3, dist)
                 kk_m, hh_m = selected_counts(s2)

@@ -237,14 +237,43 @@ DV_API dv_status dv_decode_layer(const dv_layer_weights* w, const dv_dims* dims,
                           float* x, int pos, const dv_layer_io* sel, const dv_layer_io* trace, void* ws,
                           size_t ws_bytes, dv_stream_t stream);
 
+/* dv_decode_layer in two calls, so that a caller can start work on another
+ * stream between them (the look-ahead predictor of the next layer reads
+ * trace->yA, complete when _begin's work is): _begin computes LN1, the head
+ * set unless `sel` gives it, and the selected heads' q, k, v (k and v into the
+ * cache at pos); _end computes the attention, W^O, LN2, the neuron set unless
+ * given, and the MLP, updating x. Both take the arguments of dv_decode_layer;
+ * _end must follow _begin on the same stream with the same workspace, x and
+ * pos, and nothing else may use that workspace in between. */
+DV_API dv_status dv_decode_layer_begin(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p,
+                                       float* x, int pos, const dv_layer_io* sel, const dv_layer_io* trace, void* ws,
+                                       size_t ws_bytes, dv_stream_t stream);
+DV_API dv_status dv_decode_layer_end(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p,
+                                     float* x, int pos, const dv_layer_io* sel, const dv_layer_io* trace, void* ws,
+                                     size_t ws_bytes, dv_stream_t stream);
+
 /* Look-ahead prediction (§1): the head set and neuron set of a layer
  * computed from another layer's input y (in the stack, from layer l's yA for
  * layer l+1). Writes out->scores_h, head_idx, head_count, scores, idx,
  * count (all required). Uses its own workspace so it can run on a side
- * stream concurrently with the layer that reads the other workspace. */
+ * stream concurrently with the layer that reads the other workspace. Its last
+ * launch only waits for the others to complete, so that work on another
+ * stream ordered after this call by an event never starts before the sets
+ * are written, even when launched with programmatic dependent launch. */
 DV_API dv_status dv_predict_layer(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p,
                            const float* y, const dv_layer_io* out, void* ws, size_t ws_bytes,
                            dv_stream_t stream);
+
+/* L2 prefetch of one layer's selected parameters (§1: for the next layer
+ * the look-ahead predictor picks the heads / neurons and only those
+ * parameters are loaded). Given the sets `sel` (head_idx/head_count and
+ * idx/count, device), asks the GPU's bulk-copy engine to bring into L2: the
+ * selected heads' Wqkv and WOt blocks, their K and V entries in slots
+ * 0..pos-1 for every batch row, the selected neurons' W1t rows and, when
+ * with_w2 != 0, their W2t rows. Nothing is computed or written; the call only
+ * warms L2 for a layer that runs later on another stream. */
+DV_API dv_status dv_prefetch_layer(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_io* sel, int pos,
+                                   int with_w2, dv_stream_t stream);
 
 /* Selection without a caller workspace. The paper has no counterpart: this
  * is a variant of dv_topk (same rules, same kernel, same results) for callers

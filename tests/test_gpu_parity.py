@@ -29,7 +29,12 @@ SHAPES = {
     "ragged": dict(d=1032, N=1000, r=40, h=6, dh=128, L=99, cap=100, wdtype="bf16", kvdtype="bf16", p_active=0.2),
     "opt-like": dict(d=2048, N=8192, r=256, h=32, dh=64, L=512, cap=520, wdtype="bf16", kvdtype="bf16",
                      p_active=0.10),
+    # dh = 128, a key count that does not split evenly over the attention cluster
+    "fused128": dict(d=1024, N=4096, r=64, h=8, dh=128, L=300, cap=310, wdtype="bf16", kvdtype="bf16",
+                     p_active=0.15),
 }
+# "ragged" runs the kernel-per-step layer path (d is not a multiple of the
+# W^O column slices); the other shapes run the fused layer kernels.
 
 
 def shape(name, B=1, **kw):
@@ -322,7 +327,8 @@ def _trace_bufs(s):
                 idx=torch.zeros(s.N, **i), count=torch.zeros(1, **i))
 
 
-@pytest.mark.parametrize("name,B", [("tiny", 1), ("ragged", 3), ("opt-like", 1), ("opt-like", 4)])
+@pytest.mark.parametrize("name,B", [("tiny", 1), ("ragged", 3), ("opt-like", 1), ("opt-like", 4), ("fused128", 1),
+                                    ("fused128", 3), ("tiny", 2)])
 def test_decode_layer(name, B):
     s, t = layer(name, B, seed=11)
     t["ln1_g"] = 1.0 + 0.1 * torch.randn(s.d, device=DEV)
@@ -357,10 +363,11 @@ def test_decode_layer(name, B):
     no_device_errors(ws)
 
 
-@pytest.mark.parametrize("lookahead", [True, False])
-def test_lookahead_stack(lookahead):
-    nL, B = 3, 1
-    s = shape("ragged", B)
+@pytest.mark.parametrize("name,lookahead,B", [("ragged", True, 1), ("ragged", False, 1), ("fused128", True, 1),
+                                              ("fused128", False, 2), ("opt-like", True, 1)])
+def test_lookahead_stack(name, lookahead, B):
+    nL = 3
+    s = shape(name, B)
     layers = [wl.make_layer(s, 100 + l, DEV) for l in range(nL)]
     K0 = [(f64(t["K"]), f64(t["V"])) for t in layers]
     k, k_h = wl.k_for(0.1, s.N), 2
@@ -394,9 +401,10 @@ def test_lookahead_stack(lookahead):
     no_device_errors(stk.ws_side)
 
 
-def test_stack_step_in_cuda_graph_matches_eager():
+@pytest.mark.parametrize("name", ["ragged", "fused128"])
+def test_stack_step_in_cuda_graph_matches_eager(name):
     nL, B = 3, 2
-    s = shape("ragged", B)
+    s = shape(name, B)
     layers_a = [wl.make_layer(s, 200 + l, DEV) for l in range(nL)]
     layers_b = [{kk: v.clone() for kk, v in t.items()} for t in layers_a]
     k, k_h = wl.k_for(0.1, s.N), 2
@@ -416,3 +424,44 @@ def test_stack_step_in_cuda_graph_matches_eager():
     g.replay()
     torch.cuda.synchronize()
     assert_out((xb - x).cpu().numpy(), (xa - x).cpu().numpy())
+
+
+@pytest.mark.parametrize("name", ["fused128", "ragged"])
+def test_decode_layer_with_empty_sets(name):
+    """k = 0 and k_h = 0: the layer adds only the output biases."""
+    s, t = layer(name, 1, seed=12)
+    t["bO"] = torch.randn(s.d, device=DEV) * 0.1
+    t["b2"] = torch.randn(s.d, device=DEV) * 0.1
+    x = wl.make_input(s, 22, DEV)
+    x0 = x.clone()
+    L = bd.Layer(t, 1, 0, 0)
+    p = bd.params(0, 0, 0.1)
+    ws = bd.workspace(bd.DV_OP_DECODE_LAYER, L.dims)
+    bd.dv_decode_layer(L, p, x, s.L, ws)
+    torch.cuda.synchronize()
+    assert torch.allclose(x, x0 + t["bO"] + t["b2"], rtol=1e-6, atol=1e-6)
+    no_device_errors(ws)
+
+
+@pytest.mark.parametrize("name", ["fused128", "opt-like", "tiny"])
+def test_predict_layer_matches_oracle(name):
+    """The look-ahead call (both sets from one input) on the fused predictor."""
+    B = 2
+    s, t = layer(name, B, seed=13)
+    k, k_h = wl.k_for(0.1, s.N), 2
+    L = bd.Layer(t, B, min(s.N, B * k), min(s.h, B * k_h))
+    p = bd.params(k, k_h, 0.1)
+    ws = bd.workspace(bd.DV_OP_DECODE_LAYER, L.dims)
+    y = wl.make_input(s, 23, DEV)
+    tb = _trace_bufs(s)
+    out = bd.layer_io(scores_h=tb["scores_h"], head_idx=tb["head_idx"], head_count=tb["head_count"],
+                      scores=tb["scores"], idx=tb["idx"], count=tb["count"])
+    for _ in range(2):  # twice: the in-kernel histogram and tickets must be left clean
+        bd.dv_predict_layer(L, p, y, out, ws)
+        torch.cuda.synchronize()
+        sh, sm = tb["scores_h"].cpu().numpy(), tb["scores"].cpu().numpy()
+        assert_scores(sh, O.head_predictor_scores(f64(y), f64(t["PA"])))
+        assert_scores(sm, O.mlp_predictor_scores(f64(y), f64(t["At"]), f64(t["Bm"]), f64(t["b1"])))
+        assert np.array_equal(selected(tb["head_idx"], tb["head_count"]), O.select(sh, k=k_h))
+        assert np.array_equal(selected(tb["idx"], tb["count"]), O.select(sm, k=k))
+    no_device_errors(ws)
