@@ -92,6 +92,12 @@ _lib_dv_decode_layer_begin = _sig("dv_decode_layer_begin", _c_int,
 _lib_dv_decode_layer_end = _sig("dv_decode_layer_end", _c_int,
                                 [ctypes.POINTER(LayerWeightsC), ctypes.POINTER(Dims), ctypes.POINTER(LayerParamsC),
                                  _p, _c_int, ctypes.POINTER(LayerIOC), ctypes.POINTER(LayerIOC), _p, _c_size, _p])
+_lib_dv_decode_layer_attn = _sig("dv_decode_layer_attn", _c_int,
+                                 [ctypes.POINTER(LayerWeightsC), ctypes.POINTER(Dims), ctypes.POINTER(LayerParamsC),
+                                  _p, _c_int, ctypes.POINTER(LayerIOC), ctypes.POINTER(LayerIOC), _p, _c_size, _p])
+_lib_dv_decode_layer_mlp = _sig("dv_decode_layer_mlp", _c_int,
+                                [ctypes.POINTER(LayerWeightsC), ctypes.POINTER(Dims), ctypes.POINTER(LayerParamsC),
+                                 _p, ctypes.POINTER(LayerIOC), ctypes.POINTER(LayerIOC), _p, _c_size, _p])
 _lib_dv_predict_layer = _sig("dv_predict_layer", _c_int,
                              [ctypes.POINTER(LayerWeightsC), ctypes.POINTER(Dims), ctypes.POINTER(LayerParamsC), _p,
                               ctypes.POINTER(LayerIOC), _p, _c_size, _p])
@@ -301,6 +307,19 @@ def dv_decode_layer_begin(layer: Layer, p: LayerParamsC, x, pos, ws, sel: Option
 def dv_decode_layer_end(layer: Layer, p: LayerParamsC, x, pos, ws, sel: Optional[LayerIOC] = None,
                         trace: Optional[LayerIOC] = None, stream=None):
     _layer_call(_lib_dv_decode_layer_end, "dv_decode_layer_end", layer, p, x, pos, ws, sel, trace, stream)
+
+
+def dv_decode_layer_attn(layer: Layer, p: LayerParamsC, x, pos, ws, sel: Optional[LayerIOC] = None,
+                         trace: Optional[LayerIOC] = None, stream=None):
+    _layer_call(_lib_dv_decode_layer_attn, "dv_decode_layer_attn", layer, p, x, pos, ws, sel, trace, stream)
+
+
+def dv_decode_layer_mlp(layer: Layer, p: LayerParamsC, x, ws, sel: Optional[LayerIOC] = None,
+                        trace: Optional[LayerIOC] = None, stream=None):
+    _check(_lib_dv_decode_layer_mlp(ctypes.byref(layer.c), ctypes.byref(layer.dims), ctypes.byref(p),
+                                    _ptr(x, torch.float32, "x"), ctypes.byref(sel) if sel is not None else None,
+                                    ctypes.byref(trace) if trace is not None else None, _ptr(ws, torch.uint8, "ws"),
+                                    ws.numel(), _stream(stream)), "dv_decode_layer_mlp")
 
 
 def dv_predict_layer(layer: Layer, p: LayerParamsC, y, out: LayerIOC, ws, stream=None):

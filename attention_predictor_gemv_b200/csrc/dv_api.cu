@@ -640,7 +640,10 @@ cudaError_t run_predict_b(const PredictBArgs& a, cudaStream_t st) {
 // ---------------------------------------------------------------------------
 
 int co_nv(int d, int E) { return (d + CO_THREADS * E - 1) / (CO_THREADS * E); }
-int co_r(int nv) { return nv == 1 ? 8 : nv == 2 ? 4 : nv == 3 ? 3 : 2; }
+// Rows per group: 8 or more 16-byte loads in flight per thread. The MLP
+// kernel also holds the W2 rows and its output slice, so it keeps fewer.
+int co_r(int nv) { return nv == 1 ? 8 : nv == 2 ? 4 : nv == 3 ? 3 : 4; }
+int co_r_mlp(int nv) { return nv == 1 ? 8 : nv == 2 ? 4 : nv == 3 ? 3 : 2; }
 bool co_ok(int nb, int d, int E) { return nb <= 2 && co_nv(d, E) <= 6; }
 int co_grid(long long groups) {
   const long long cap = 2ll * sm_count();
@@ -648,6 +651,15 @@ int co_grid(long long groups) {
 }
 
 #define DV_CO_SWITCH(KERN, NB, grid, st, a)                                   \
+  switch (nv) {                                                              \
+    case 1: return launch(KERN<T, NB, 1, 8>, grid, CO_THREADS, 0, st, a);    \
+    case 2: return launch(KERN<T, NB, 2, 4>, grid, CO_THREADS, 0, st, a);    \
+    case 3: return launch(KERN<T, NB, 3, 3>, grid, CO_THREADS, 0, st, a);    \
+    case 4: return launch(KERN<T, NB, 4, 4>, grid, CO_THREADS, 0, st, a);    \
+    case 5: return launch(KERN<T, NB, 5, 4>, grid, CO_THREADS, 0, st, a);    \
+    default: return launch(KERN<T, NB, 6, 4>, grid, CO_THREADS, 0, st, a);   \
+  }
+#define DV_CO_SWITCH_MLP(KERN, NB, grid, st, a)                               \
   switch (nv) {                                                              \
     case 1: return launch(KERN<T, NB, 1, 8>, grid, CO_THREADS, 0, st, a);    \
     case 2: return launch(KERN<T, NB, 2, 4>, grid, CO_THREADS, 0, st, a);    \
@@ -666,10 +678,10 @@ cudaError_t run_attn_in_co_nb(const AttnInArgs& a, cudaStream_t st) {
 
 template <typename T, int NB>
 cudaError_t run_mlp_block_co_nb(MlpBlockArgs a, cudaStream_t st) {
-  const int nv = co_nv(a.d, WT<T>::E), R = co_r(nv);
+  const int nv = co_nv(a.d, WT<T>::E), R = co_r_mlp(nv);
   a.G = co_grid(((long long)a.k_max + R - 1) / R);
   const dim3 grid(a.G);
-  DV_CO_SWITCH(mlp_block_co_kernel, NB, grid, st, a)
+  DV_CO_SWITCH_MLP(mlp_block_co_kernel, NB, grid, st, a)
 }
 
 template <typename T, int NB>
@@ -680,6 +692,7 @@ cudaError_t run_predict_a_co_nb(const PredictAArgs& a, cudaStream_t st) {
   DV_CO_SWITCH(predict_a_co_kernel, NB, grid, st, a)
 }
 #undef DV_CO_SWITCH
+#undef DV_CO_SWITCH_MLP
 
 template <typename T>
 cudaError_t run_attn_in_any(const AttnInArgs& a, cudaStream_t st) {
@@ -842,14 +855,12 @@ dv_status layer_begin(const Layout& L, void* ws, const dv_layer_weights* w, cons
                                           D.kh_max, q, w->Kc, w->Vc, D.cap, pos, status, st));
 }
 
-// Second half: attention + W^O + residual, LN2, the neuron set unless given,
-// the sparse MLP + residual.
-dv_status layer_end(const Layout& L, void* ws, const dv_layer_weights* w, const dv_dims& D, const dv_layer_params* p,
-                    float* x, int pos, const dv_layer_io* sel, const dv_layer_io* trace, cudaStream_t st) {
+// Attention half: split attention over the selected heads, W^O, residual.
+dv_status layer_attn(const Layout& L, void* ws, const dv_layer_weights* w, const dv_dims& D, const dv_layer_params* p,
+                     float* x, int pos, const dv_layer_io* sel, const dv_layer_io* trace, cudaStream_t st) {
   const LayerBufs r = layer_bufs(L, ws, sel, trace);
   int* status = at<int>(ws, L.status);
   if (fused_ok(D, w->wdtype)) {
-    float* t1 = at<float>(ws, L.t1);
     AttnOutArgs b = {};
     b.q = at<float>(ws, L.q);
     b.Kc = w->Kc;
@@ -860,7 +871,7 @@ dv_status layer_end(const Layout& L, void* ws, const dv_layer_weights* w, const 
     b.head_count = r.use_hcnt;
     b.kh_max = D.kh_max;
     b.x = x;
-    b.t1 = t1;
+    b.t1 = at<float>(ws, L.t1);
     b.h = D.h;
     b.dh = D.dh;
     b.d = D.d;
@@ -871,7 +882,38 @@ dv_status layer_end(const Layout& L, void* ws, const dv_layer_weights* w, const 
     b.sets_ready = sel ? 1 : 0;
     b.scale = p->scale;
     b.status = status;
-    DV_TRY(w->kvdtype == DV_BF16 ? run_attn_out<bf16>(b, st) : run_attn_out<float>(b, st));
+    return cuda_status(w->kvdtype == DV_BF16 ? run_attn_out<bf16>(b, st) : run_attn_out<float>(b, st));
+  }
+  if (D.kh_max > 0) {
+    float* H = at<float>(ws, L.H);
+    const float* q = at<float>(ws, L.q);
+    DV_TRY(w->kvdtype == DV_BF16
+               ? run_attn<bf16>(D.dh, q, w->Kc, w->Vc, D.B, D.h, D.cap, pos, p->scale, r.use_hidx, r.use_hcnt,
+                                D.kh_max, at<float>(ws, L.part), at<unsigned>(ws, L.attn_ctr), H, status, st)
+               : run_attn<float>(D.dh, q, w->Kc, w->Vc, D.B, D.h, D.cap, pos, p->scale, r.use_hidx, r.use_hcnt,
+                                 D.kh_max, at<float>(ws, L.part), at<unsigned>(ws, L.attn_ctr), H, status, st));
+    RowsHeads src{r.use_hidx, r.use_hcnt, H, D.kh_max, D.dh, D.h};
+    return cuda_status(w->wdtype == DV_BF16 ? run_axpy<bf16>(w->WOt, D.d, D.h * D.dh, src, w->bO, x, D.B,
+                                                             D.kh_max * D.dh, 0, status, st)
+                                            : run_axpy<float>(w->WOt, D.d, D.h * D.dh, src, w->bO, x, D.B,
+                                                              D.kh_max * D.dh, 0, status, st));
+  }
+  if (w->bO) {
+    RowsHeads none{r.use_hidx, r.use_hcnt, nullptr, 0, D.dh, D.h};
+    return cuda_status(w->wdtype == DV_BF16
+                           ? run_axpy<bf16>(w->WOt, D.d, D.h * D.dh, none, w->bO, x, D.B, 1, 0, status, st)
+                           : run_axpy<float>(w->WOt, D.d, D.h * D.dh, none, w->bO, x, D.B, 1, 0, status, st));
+  }
+  return DV_OK;
+}
+
+// MLP half: LN2, the neuron set unless given, the sparse MLP + residual.
+dv_status layer_mlp(const Layout& L, void* ws, const dv_layer_weights* w, const dv_dims& D, const dv_layer_params* p,
+                    float* x, const dv_layer_io* sel, const dv_layer_io* trace, cudaStream_t st) {
+  const LayerBufs r = layer_bufs(L, ws, sel, trace);
+  int* status = at<int>(ws, L.status);
+  if (fused_ok(D, w->wdtype)) {
+    float* t1 = at<float>(ws, L.t1);
     if (!sel) {
       DV_TRY(launch(layernorm_kernel, dim3(D.B), LN_THREADS, 0, st, (const float*)t1, r.yM, D.d, w->ln2_g, w->ln2_b,
                     p->eps));
@@ -899,25 +941,6 @@ dv_status layer_end(const Layout& L, void* ws, const dv_layer_weights* w, const 
     c.status = status;
     return cuda_status(w->wdtype == DV_BF16 ? run_mlp_block_any<bf16>(c, st) : run_mlp_block_any<float>(c, st));
   }
-  // kernel-per-step path
-  if (D.kh_max > 0) {
-    float* H = at<float>(ws, L.H);
-    const float* q = at<float>(ws, L.q);
-    DV_TRY(w->kvdtype == DV_BF16
-               ? run_attn<bf16>(D.dh, q, w->Kc, w->Vc, D.B, D.h, D.cap, pos, p->scale, r.use_hidx, r.use_hcnt,
-                                D.kh_max, at<float>(ws, L.part), at<unsigned>(ws, L.attn_ctr), H, status, st)
-               : run_attn<float>(D.dh, q, w->Kc, w->Vc, D.B, D.h, D.cap, pos, p->scale, r.use_hidx, r.use_hcnt,
-                                 D.kh_max, at<float>(ws, L.part), at<unsigned>(ws, L.attn_ctr), H, status, st));
-    RowsHeads src{r.use_hidx, r.use_hcnt, H, D.kh_max, D.dh, D.h};
-    DV_TRY(w->wdtype == DV_BF16 ? run_axpy<bf16>(w->WOt, D.d, D.h * D.dh, src, w->bO, x, D.B, D.kh_max * D.dh, 0,
-                                                 status, st)
-                                : run_axpy<float>(w->WOt, D.d, D.h * D.dh, src, w->bO, x, D.B, D.kh_max * D.dh, 0,
-                                                  status, st));
-  } else if (w->bO) {
-    RowsHeads none{r.use_hidx, r.use_hcnt, nullptr, 0, D.dh, D.h};
-    DV_TRY(w->wdtype == DV_BF16 ? run_axpy<bf16>(w->WOt, D.d, D.h * D.dh, none, w->bO, x, D.B, 1, 0, status, st)
-                                : run_axpy<float>(w->WOt, D.d, D.h * D.dh, none, w->bO, x, D.B, 1, 0, status, st));
-  }
   DV_TRY(launch(layernorm_kernel, dim3(D.B), LN_THREADS, 0, st, (const float*)x, r.yM, D.d, w->ln2_g, w->ln2_b,
                 p->eps));
   if (!sel)
@@ -925,6 +948,12 @@ dv_status layer_end(const Layout& L, void* ws, const dv_layer_weights* w, const 
                             r.sm, r.midx, r.mcnt, st));
   return do_sparse_mlp(L, ws, r.yM, D.B, D.d, D.N, w->W1t, w->b1, w->W2t, w->b2, w->wdtype, r.use_midx, r.use_mcnt,
                        D.k_max, x, 1, st);
+}
+
+dv_status layer_end(const Layout& L, void* ws, const dv_layer_weights* w, const dv_dims& D, const dv_layer_params* p,
+                    float* x, int pos, const dv_layer_io* sel, const dv_layer_io* trace, cudaStream_t st) {
+  DV_CHECK(layer_attn(L, ws, w, D, p, x, pos, sel, trace, st));
+  return layer_mlp(L, ws, w, D, p, x, sel, trace, st);
 }
 
 }  // namespace
@@ -1098,6 +1127,22 @@ dv_status dv_decode_layer_end(const dv_layer_weights* w, const dv_dims* dims, co
   Layout L;
   DV_CHECK(check_layer_call(w, dims, p, x, pos, sel, trace, ws, ws_bytes, &L));
   return layer_end(L, ws, w, *dims, p, x, pos, sel, trace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dv_status dv_decode_layer_attn(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p, float* x,
+                               int pos, const dv_layer_io* sel, const dv_layer_io* trace, void* ws, size_t ws_bytes,
+                               dv_stream_t stream) {
+  Layout L;
+  DV_CHECK(check_layer_call(w, dims, p, x, pos, sel, trace, ws, ws_bytes, &L));
+  return layer_attn(L, ws, w, *dims, p, x, pos, sel, trace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dv_status dv_decode_layer_mlp(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p, float* x,
+                              const dv_layer_io* sel, const dv_layer_io* trace, void* ws, size_t ws_bytes,
+                              dv_stream_t stream) {
+  Layout L;
+  DV_CHECK(check_layer_call(w, dims, p, x, 0, sel, trace, ws, ws_bytes, &L));
+  return layer_mlp(L, ws, w, *dims, p, x, sel, trace, reinterpret_cast<cudaStream_t>(stream));
 }
 
 dv_status dv_decode_layer(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p, float* x, int pos,

@@ -444,7 +444,7 @@ __global__ void __launch_bounds__(CO_THREADS) mlp_block_co_kernel(MlpBlockArgs a
       }
 #pragma unroll
       for (int e4 = 0; e4 < E / 4; ++e4)
-        atomicAdd(reinterpret_cast<float4*>(a.x + (size_t)b * a.d + c) + e4,
+        red_add4(a.x + (size_t)b * a.d + c + 4 * e4,
                   make_float4(o[4 * e4], o[4 * e4 + 1], o[4 * e4 + 2], o[4 * e4 + 3]));
     }
   }

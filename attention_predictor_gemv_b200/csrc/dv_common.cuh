@@ -137,4 +137,11 @@ __device__ __forceinline__ unsigned block_exclusive_scan(unsigned v, unsigned* s
 
 __device__ __forceinline__ void raise_status(int* st, int bit) { atomicOr(st, bit); }
 
+// out[0..3] += v without returning the old values (a fire-and-forget vector
+// reduction in L2, so the issuing thread does not wait for it).
+__device__ __forceinline__ void red_add4(float* out, float4 v) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(out), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
+
 }  // namespace dv

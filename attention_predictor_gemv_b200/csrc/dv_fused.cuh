@@ -360,7 +360,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) mlp_block_kernel(MlpBlockArgs a
           if (b < a.nb) {
 #pragma unroll
             for (int e4 = 0; e4 < E / 4; ++e4)
-              atomicAdd(reinterpret_cast<float4*>(a.x + (size_t)b * a.d + c + 4 * e4),
+              red_add4(a.x + (size_t)b * a.d + c + 4 * e4,
                         make_float4(acc[b][4 * e4], acc[b][4 * e4 + 1], acc[b][4 * e4 + 2], acc[b][4 * e4 + 3]));
           }
         }
@@ -683,16 +683,17 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
 #pragma unroll
       for (int e = 0; e < E; ++e) acc[b][e] = 0.f;
     if (active && thr_ok) {
+      constexpr int WO_U = 16;  // rows of W^O in flight per thread
       const KT* Wh = WO + (size_t)head * DH * a.d + c;
-      for (int i0 = rg; i0 < DH; i0 += nrg * AX_U) {
-        uint4 w[AX_U];
+      for (int i0 = rg; i0 < DH; i0 += nrg * WO_U) {
+        uint4 w[WO_U];
 #pragma unroll
-        for (int u = 0; u < AX_U; ++u) {
+        for (int u = 0; u < WO_U; ++u) {
           const int i = i0 + u * nrg;
           w[u] = i < DH ? ld_stream(Wh + (size_t)i * a.d) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
-        for (int u = 0; u < AX_U; ++u) {
+        for (int u = 0; u < WO_U; ++u) {
           const int i = i0 + u * nrg;
           if (i < DH) {
             float wf[E];
@@ -743,7 +744,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
         }
 #pragma unroll
         for (int e4 = 0; e4 < E / 4; ++e4)
-          atomicAdd(reinterpret_cast<float4*>(a.t1 + (size_t)b * a.d + c + 4 * e4),
+          red_add4(a.t1 + (size_t)b * a.d + c + 4 * e4,
                     make_float4(o[4 * e4], o[4 * e4 + 1], o[4 * e4 + 2], o[4 * e4 + 3]));
       }
     }
@@ -865,7 +866,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) predict_b_kernel(PredictBArgs a
 // and writes idx / count. CTA B (when heads are predicted) selects the heads
 // from their scores by rank (few heads: direct comparison).
 // ----------------------------------------------------------------------------
-constexpr int SF_CAND = 4096;
+constexpr int SF_CAND = 2048;  // keeps static + dynamic shared memory within 227 KB at N = 49152
 
 struct SelectFinishArgs {
   const float* scores;  // [B][N]

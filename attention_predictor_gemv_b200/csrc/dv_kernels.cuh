@@ -754,7 +754,7 @@ __global__ void __launch_bounds__(AX_THREADS)
 #pragma unroll
         for (int e4 = 0; e4 < E / 4; ++e4) {
           float4 v = make_float4(acc[b][4 * e4], acc[b][4 * e4 + 1], acc[b][4 * e4 + 2], acc[b][4 * e4 + 3]);
-          atomicAdd(reinterpret_cast<float4*>(out + (size_t)b * d + col + 4 * e4), v);
+          red_add4(out + (size_t)b * d + col + 4 * e4, v);
         }
       }
     }

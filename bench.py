@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--no-lookahead", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-big", action="store_true", help="skip the OPT-175B-shaped measurement")
+    ap.add_argument("--big-layers", type=int, default=4)
     ap.add_argument("--prefetch", action="store_true", help="L2-prefetch each layer's selected rows on the side stream")
     ap.add_argument("--no-prefetch-w2", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -160,20 +162,15 @@ def build_stack(shape, nlayers, B, k, k_h, lookahead, seed0=1000, layers=None, p
 
 
 def capture(stk, x, pos):
+    """The decode step as a CUDA graph, and how many library kernels it holds."""
     from attention_predictor_gemv_b200 import binding as bd
 
-    stk.step(x, pos)  # eager warm-up (sets attributes, loads modules)
+    stk.step(x, pos)  # eager warm-up
     torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    s = torch.cuda.Stream()
-    s.wait_stream(torch.cuda.current_stream())
     n0 = bd.dv_launch_count()
-    with torch.cuda.stream(s):
-        with torch.cuda.graph(g, stream=s):
-            stk.step(x, pos)
-    torch.cuda.current_stream().wait_stream(s)
-    torch.cuda.synchronize()
-    return g, bd.dv_launch_count() - n0
+    g = graph_of(lambda: stk.step(x, pos))
+    n1 = bd.dv_launch_count()
+    return g, (n1 - n0) // 2  # graph_of runs fn once eagerly, then captures it
 
 
 def time_graph(g, steps, warmup, dist):
@@ -216,53 +213,85 @@ def layer_bytes(shape, k, kp, kh, B):
                             int(round(kh)), B, shape.L + 1)
 
 
-def op_roofline(stk, shape, B, pos, peak_gbs):
-    """Times each library call of one layer-step over all layers with CUDA
-    events on the launching stream (weights of 24 layers: HBM-cold), and
-    returns the per-op average duration and effective bandwidth."""
+def graph_of(fn):
+    """Captures fn (library launches on the current stream) into a CUDA graph."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    return g
+
+
+def kernel_roofline(stk, shape, B, pos, peak_gbs, reps=20):
+    """Average duration of each main-path kernel in the look-ahead steady
+    state (sets given): one CUDA graph per kernel with that kernel's call for
+    every layer, timed with CUDA events on the launching stream; each
+    kernel's algorithmic bytes per launch divided by its average duration.
+    The residual state is restored afterwards."""
     from attention_predictor_gemv_b200 import binding as bd
 
-    st = torch.cuda.current_stream()
     nL = len(stk.layers)
-    res = {}
     x = torch.randn(B, shape.d, device="cuda")
-    ws = stk.ws_main
-    out = torch.empty(B, shape.d, device="cuda")
-
-    def timed(name, fn, nbytes):
-        for _ in range(2):
-            for l in range(nL):
-                fn(l)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(st)
-        reps = 5
-        for _ in range(reps):
-            for l in range(nL):
-                fn(l)
-        e1.record(st)
-        e1.synchronize()
-        us = e0.elapsed_time(e1) * 1000.0 / (reps * nL)
-        res[name] = {"us": us, "bytes": nbytes, "gbs": nbytes / us / 1e3, "frac": nbytes / us / 1e3 / peak_gbs}
-
+    snap = [(t["K"].clone(), t["V"].clone()) for t in (L.t for L in stk.layers)]
     kp = nonzero_neurons(stk)
     k, kh = selected_counts(stk)
     lb = layer_bytes(shape, k, kp, kh, B)
-    p = stk.p
-    timed("dv_predict_heads", lambda l: bd.dv_predict_heads(stk.yA[l], stk.layers[l].t["PA"], p.k_h, stk.scores_h[l],
-                                                            stk.head_idx[l], stk.head_count[l], ws), lb.head_predictor)
-    timed("dv_predict_mlp", lambda l: bd.dv_predict_mlp(stk.yM[l], stk.layers[l].t["At"], stk.layers[l].t["Bm"],
-                                                        stk.layers[l].t["b1"], p.k, stk.scores[l], stk.idx[l],
-                                                        stk.count[l], ws), lb.mlp_predictor)
-    timed("dv_sparse_mha", lambda l: bd.dv_sparse_mha(stk.yA[l], stk.layers[l].t["Wqkv"], None,
-                                                      stk.layers[l].t["WOt"], None, stk.layers[l].t["K"],
-                                                      stk.layers[l].t["V"], pos, p.scale, stk.head_idx[l],
-                                                      stk.head_count[l], stk.kh_max, out, ws),
-          lb.qkv + lb.wo + lb.kv)
-    timed("dv_sparse_mlp", lambda l: bd.dv_sparse_mlp(stk.yM[l], stk.layers[l].t["W1t"], stk.layers[l].t["b1"],
-                                                      stk.layers[l].t["W2t"], None, stk.idx[l], stk.count[l],
-                                                      stk.k_max, out, ws), lb.w1 + lb.w2)
+    p, ws = stk.p, stk.ws_main
+    calls = {
+        "attn_in": (lambda l: bd.dv_decode_layer_begin(stk.layers[l], p, x, pos, ws, sel=stk.io_given[l],
+                                                       trace=stk.io_trace_y[l]), lb.qkv),
+        "attn_out": (lambda l: bd.dv_decode_layer_attn(stk.layers[l], p, x, pos, ws, sel=stk.io_given[l],
+                                                       trace=stk.io_trace_y[l]), lb.kv + lb.wo),
+        "mlp_block": (lambda l: bd.dv_decode_layer_mlp(stk.layers[l], p, x, ws, sel=stk.io_given[l],
+                                                       trace=stk.io_trace_y[l]), lb.w1 + lb.w2),
+    }
+    res = {}
+    for name, (fn, nbytes) in calls.items():
+        g = graph_of(lambda: [fn(l) for l in range(nL)])
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        e1.synchronize()
+        us = e0.elapsed_time(e1) * 1000.0 / (reps * nL)
+        res[name] = {"us": us, "bytes": nbytes, "gbs": nbytes / us / 1e3, "frac": nbytes / us / 1e3 / peak_gbs}
+        del g
+    for t, (K, V) in zip((L.t for L in stk.layers), snap):
+        t["K"].copy_(K)
+        t["V"].copy_(V)
     return res, lb, k, kp, kh
+
+
+def big_config(args, peak_gbs, dist):
+    """OPT-175B-shaped layers (d=12288, N=49152, h=96, dh=128, KV 2048) at
+    85% sparsity on neurons and heads, batch 1: the regime where the selected
+    bytes (about 0.65 GB per layer) rather than latency bound the step."""
+    shape = wl.CONFIGS["opt-175b"].with_(B=1)
+    k, k_h = wl.k_for(0.15, shape.N), wl.k_for(0.15, shape.h)
+    stk, layers = build_stack(shape, args.big_layers, 1, k, k_h, True, seed0=5000)
+    x = wl.make_input(shape, 11, "cuda")
+    g, _ = capture(stk, x, shape.L)
+    ms = time_graph(g, 10, 3, dist)
+    kern, lb, km, kp, kh = kernel_roofline(stk, shape, 1, shape.L, peak_gbs, reps=5)
+    us_layer = ms * 1e3 / args.big_layers
+    out = {"workload": f"{args.big_layers} OPT-175B-shaped layers: d={shape.d}, N={shape.N}, r={shape.r}, "
+                       f"h={shape.h}, dh={shape.dh}, KV length {shape.L}, batch 1, k={k} (15%), k_h={k_h} (15%), "
+                       "look-ahead", "us_per_layer_step": us_layer, "bytes_per_layer": lb.total,
+           "effective_gbs": lb.total / us_layer / 1e3, "effective_frac": lb.total / us_layer / 1e3 / peak_gbs,
+           "selected": {"k": km, "k_eff": kp, "k_h": kh}, "kernels": kern}
+    del g, stk, layers
+    torch.cuda.empty_cache()
+    return out
 
 
 def cpu_baseline(shape, B, k, k_h, seconds, seed=1000):
@@ -365,7 +394,7 @@ def main():
     barrier(dist)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist)
 
-    ops, lb, kmean, kp, kh = op_roofline(stk, shape, B, pos, peak_gbs)
+    ops, lb, kmean, kp, kh = kernel_roofline(stk, shape, B, pos, peak_gbs)
     dom = max(ops, key=lambda n: ops[n]["us"])
     total_layer_bytes = lb.total
     us_layer = ms * 1e3 / args.layers
@@ -384,6 +413,10 @@ def main():
                 sweep.append({"k_frac": kf, "kh_frac": hf, "k": kk, "k_h": hh, "us_per_layer": m2 * 1e3 / args.layers,
                               "bytes_per_layer": b2, "gbs": b2 / (m2 * 1e3 / args.layers) / 1e3})
                 del g2, s2
+
+    big = None
+    if not args.no_big:
+        big = big_config(args, peak_gbs, dist)
 
     line = {
         "metric": METRIC, "value": value, "unit": "us", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -409,6 +442,7 @@ def main():
         "launches_per_step": int(launches_per_step),
         "clocks": clocks,
         "sweep": sweep,
+        "opt175b_shaped": big,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(shape, B, k, k_h, args.cpu_seconds)

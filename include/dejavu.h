@@ -252,6 +252,20 @@ DV_API dv_status dv_decode_layer_end(const dv_layer_weights* w, const dv_dims* d
                                      float* x, int pos, const dv_layer_io* sel, const dv_layer_io* trace, void* ws,
                                      size_t ws_bytes, dv_stream_t stream);
 
+/* The two parts of dv_decode_layer_end, for callers that order or time them
+ * separately: _attn computes the selected heads' attention (eq. (2)) over
+ * slots 0..pos, multiplies by W^O and adds the result and bO to the residual
+ * (kept in the workspace until _mlp); _mlp applies LN2, predicts the neuron
+ * set unless `sel` gives it, and computes the sparse MLP (eq. (1)) into x.
+ * They must follow dv_decode_layer_begin in this order, on one stream, with
+ * the same workspace and x. */
+DV_API dv_status dv_decode_layer_attn(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p,
+                                      float* x, int pos, const dv_layer_io* sel, const dv_layer_io* trace, void* ws,
+                                      size_t ws_bytes, dv_stream_t stream);
+DV_API dv_status dv_decode_layer_mlp(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p,
+                                     float* x, const dv_layer_io* sel, const dv_layer_io* trace, void* ws,
+                                     size_t ws_bytes, dv_stream_t stream);
+
 /* Look-ahead prediction (§1): the head set and neuron set of a layer
  * computed from another layer's input y (in the stack, from layer l's yA for
  * layer l+1). Writes out->scores_h, head_idx, head_count, scores, idx,

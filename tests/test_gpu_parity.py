@@ -465,3 +465,30 @@ def test_predict_layer_matches_oracle(name):
         assert np.array_equal(selected(tb["head_idx"], tb["head_count"]), O.select(sh, k=k_h))
         assert np.array_equal(selected(tb["idx"], tb["count"]), O.select(sm, k=k))
     no_device_errors(ws)
+
+
+@pytest.mark.parametrize("name", ["fused128", "ragged"])
+def test_layer_in_three_calls_equals_one(name):
+    """begin + attn + mlp (look-ahead sets given) == dv_decode_layer with the same sets."""
+    B = 2
+    s, t = layer(name, B, seed=14)
+    t2 = {kk: v.clone() for kk, v in t.items()}
+    k, k_h = wl.k_for(0.1, s.N), 2
+    hidx = torch.from_numpy(_subset(s.h, 3, 5)).to(DEV)
+    hcnt = torch.tensor([3], dtype=torch.int32, device=DEV)
+    midx = torch.from_numpy(_subset(s.N, 2 * k, 6)).to(DEV)
+    mcnt = torch.tensor([2 * k], dtype=torch.int32, device=DEV)
+    sel = bd.layer_io(head_idx=hidx, head_count=hcnt, idx=midx, count=mcnt)
+    x = wl.make_input(s, 24, DEV)
+    xa, xb = x.clone(), x.clone()
+    La, Lb = bd.Layer(t, B, 2 * k, 3), bd.Layer(t2, B, 2 * k, 3)
+    p = bd.params(k, 1, 0.1)  # the sets are given; k and k_h only bound them
+    wsa, wsb = bd.workspace(bd.DV_OP_DECODE_LAYER, La.dims), bd.workspace(bd.DV_OP_DECODE_LAYER, Lb.dims)
+    bd.dv_decode_layer(La, p, xa, s.L, wsa, sel=sel)
+    bd.dv_decode_layer_begin(Lb, p, xb, s.L, wsb, sel=sel)
+    bd.dv_decode_layer_attn(Lb, p, xb, s.L, wsb, sel=sel)
+    bd.dv_decode_layer_mlp(Lb, p, xb, wsb, sel=sel)
+    torch.cuda.synchronize()
+    assert_out((xb - x).cpu().numpy(), (xa - x).cpu().numpy())
+    no_device_errors(wsa)
+    no_device_errors(wsb)
