@@ -17,10 +17,13 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdejavu.so")
-SOURCES = ["dv_api.cu"]
-HEADERS = ["dv_common.cuh", "dv_kernels.cuh"]
+# One translation unit per kernel family, compiled in parallel, then linked.
+SOURCES = ["dv_api.cu", "dv_inst_legacy.cu", "dv_inst_legacy_attn.cu", "dv_inst_attn_in.cu", "dv_inst_attn_out.cu",
+           "dv_inst_mlp.cu", "dv_inst_pred.cu"]
+HEADERS = ["dv_common.cuh", "dv_kernels.cuh", "dv_fused.cuh", "dv_colowner.cuh", "dv_launch.cuh", "dv_launchers.cuh",
+           "dv_api_kernels.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared", "-Xcompiler", "-fvisibility=hidden",
+FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr"]
 
 
@@ -44,20 +47,36 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and up_to_date():
-        return LIB
-    cmd = [nvcc_path(), *ARCH, *FLAGS, *extra, "-I", os.path.join(ROOT, "include"), "-o", LIB + ".tmp",
-           *[os.path.join(CSRC, s) for s in SOURCES]]
-    if verbose:
-        print(" ".join(cmd), flush=True)
+def build(force: bool = False, verbose: bool = False, extra=(), csrc: str = CSRC, out: str = LIB) -> str:
+    if not force and out == LIB and up_to_date():
+        return out
+    nvcc = nvcc_path()
+    objdir = out + ".objs"
+    os.makedirs(objdir, exist_ok=True)
+    procs = []
+    for src in SOURCES:
+        obj = os.path.join(objdir, src.replace(".cu", ".o"))
+        cmd = [nvcc, *ARCH, *FLAGS, *extra, "-I", os.path.join(ROOT, "include"), "-c", "-o", obj,
+               os.path.join(csrc, src)]
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        procs.append((obj, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)))
+    errors = []
+    for obj, p in procs:
+        log = p.communicate()[0]
+        if p.returncode != 0:
+            errors.append(log)
+        elif verbose and log:
+            print(log)
+    if errors:
+        raise RuntimeError("nvcc failed:\n" + "\n".join(errors))
+    cmd = [nvcc, *ARCH, "-shared", "-o", out + ".tmp", *[o for o, _ in procs]]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
-        raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)
-    if verbose and (r.stdout or r.stderr):
-        print(r.stdout + r.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+        raise RuntimeError("nvcc link failed:\n" + r.stdout + r.stderr)
+    os.replace(out + ".tmp", out)
+    shutil.rmtree(objdir, ignore_errors=True)
+    return out
 
 
 if __name__ == "__main__":

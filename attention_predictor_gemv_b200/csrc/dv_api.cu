@@ -7,131 +7,14 @@
 #include <mutex>
 
 #include "../../include/dejavu.h"
-#include "dv_colowner.cuh"
+#include "dv_api_kernels.cuh"
+#include "dv_launchers.cuh"
 
 using namespace dv;
 using bf16 = __nv_bfloat16;
 
 namespace {
 
-std::atomic<uint64_t> g_launches{0};
-
-bool pdl_enabled() {
-  static const bool on = [] {
-    const char* e = std::getenv("DV_PDL");
-    return !(e && e[0] == '0');
-  }();
-  return on;
-}
-
-// Every kernel asks for the largest shared-memory carveout, so that CTAs of
-// different kernels (consecutive ones overlapping under programmatic launch,
-// and the two streams of the look-ahead) can share an SM without the SM
-// having to drain and reconfigure its L1 / shared split. Cached per kernel.
-std::mutex g_carve_mu;
-std::map<std::pair<const void*, int>, bool> g_carve_set;
-
-template <typename K>
-void prefer_max_shared(K kern) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return;
-  const auto key = std::make_pair(reinterpret_cast<const void*>(kern), dev);
-  std::lock_guard<std::mutex> lock(g_carve_mu);
-  if (g_carve_set.count(key)) return;
-  cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
-  g_carve_set[key] = true;
-}
-
-// Launch with programmatic stream serialisation, so a kernel's launch and
-// prologue overlap the tail of the previous kernel on the stream.
-template <typename... KArgs, typename... Args>
-cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl_enabled() ? 1 : 0;
-  prefer_max_shared(kern);
-  g_launches.fetch_add(1, std::memory_order_relaxed);
-  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
-}
-
-// Launch as thread-block clusters of `cluster_x` CTAs (plus programmatic
-// stream serialisation).
-template <typename... KArgs, typename... Args>
-cudaError_t launch_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster_x,
-                           Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cluster_x;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl_enabled() ? 2 : 1;
-  prefer_max_shared(kern);
-  g_launches.fetch_add(1, std::memory_order_relaxed);
-  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
-}
-
-// Raises a kernel's dynamic shared memory limit to `bytes` when needed (the
-// default 48 KB covers static plus dynamic). Cached per kernel and device.
-std::mutex g_smem_mu;
-struct SmemKey {
-  const void* fn;
-  int dev;
-  bool operator<(const SmemKey& o) const { return fn < o.fn || (fn == o.fn && dev < o.dev); }
-};
-std::map<SmemKey, size_t> g_smem_set;
-
-template <typename K>
-cudaError_t allow_smem(K kern, size_t bytes) {
-  if (bytes == 0) return cudaSuccess;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  const SmemKey key{reinterpret_cast<const void*>(kern), dev};
-  std::lock_guard<std::mutex> lock(g_smem_mu);
-  auto it = g_smem_set.find(key);
-  if (it != g_smem_set.end() && it->second >= bytes) return cudaSuccess;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e == cudaSuccess) g_smem_set[key] = bytes;
-  return e;
-}
-
-int sm_count() {
-  static int n = [] {
-    int dev = 0, v = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    return v > 0 ? v : 148;
-  }();
-  return n;
-}
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
-bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
-
-size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
-
-int nb_bucket(int B) { return B <= 1 ? 1 : B <= 2 ? 2 : B <= 4 ? 4 : B <= 8 ? 8 : 16; }
-
-// RPW rows per warp and U column steps so that RPW * U = 8 loads per lane.
-int rpw_for(int K, int E) {
-  const int vpl = (K / E + 31) / 32;
-  return vpl >= 8 ? 1 : vpl >= 4 ? 2 : vpl >= 2 ? 4 : 8;
-}
 
 constexpr int ATTN_S_MIN = 32;
 // Every layout starts with the same fixed header that holds the counters, so
@@ -214,176 +97,6 @@ dv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DV_OK : DV_ERR_
   } while (0)
 
 // ---------------------------------------------------------------------------
-// Launchers (arguments already checked)
-// ---------------------------------------------------------------------------
-
-template <typename T, int NB>
-cudaError_t run_dense_gemv_nb(const void* W, int nrows, int K, const float* X, int ldx, int nb, const float* bias,
-                              float* out, int ldo, cudaStream_t st) {
-  const T* w = static_cast<const T*>(W);
-  const int rpw = rpw_for(K, WT<T>::E);
-  const int rows_per_cta = GEMV_WARPS * rpw;
-  dim3 grid((nrows + rows_per_cta - 1) / rows_per_cta);
-  switch (rpw) {
-    case 1: return launch(dense_gemv_kernel<T, NB, 1, 8>, grid, GEMV_THREADS, 0, st, w, nrows, K, X, ldx, nb, bias, out, ldo);
-    case 2: return launch(dense_gemv_kernel<T, NB, 2, 4>, grid, GEMV_THREADS, 0, st, w, nrows, K, X, ldx, nb, bias, out, ldo);
-    case 4: return launch(dense_gemv_kernel<T, NB, 4, 2>, grid, GEMV_THREADS, 0, st, w, nrows, K, X, ldx, nb, bias, out, ldo);
-    default: return launch(dense_gemv_kernel<T, NB, 8, 1>, grid, GEMV_THREADS, 0, st, w, nrows, K, X, ldx, nb, bias, out, ldo);
-  }
-}
-
-template <typename T>
-cudaError_t run_dense_gemv(const void* W, int nrows, int K, const float* X, int ldx, int nb, const float* bias,
-                           float* out, int ldo, cudaStream_t st) {
-  switch (nb_bucket(nb)) {
-    case 1: return run_dense_gemv_nb<T, 1>(W, nrows, K, X, ldx, nb, bias, out, ldo, st);
-    case 2: return run_dense_gemv_nb<T, 2>(W, nrows, K, X, ldx, nb, bias, out, ldo, st);
-    case 4: return run_dense_gemv_nb<T, 4>(W, nrows, K, X, ldx, nb, bias, out, ldo, st);
-    case 8: return run_dense_gemv_nb<T, 8>(W, nrows, K, X, ldx, nb, bias, out, ldo, st);
-    default: return run_dense_gemv_nb<T, 16>(W, nrows, K, X, ldx, nb, bias, out, ldo, st);
-  }
-}
-
-cudaError_t run_gemv(dv_dtype dt, const void* W, int nrows, int K, const float* X, int ldx, int nb, const float* bias,
-                     float* out, int ldo, cudaStream_t st) {
-  return dt == DV_BF16 ? run_dense_gemv<bf16>(W, nrows, K, X, ldx, nb, bias, out, ldo, st)
-                       : run_dense_gemv<float>(W, nrows, K, X, ldx, nb, bias, out, ldo, st);
-}
-
-cudaError_t run_select(const float* scores, int nrows, int n, int k, float tau, int mode, uint32_t* bm,
-                       unsigned* ticket, int32_t* idx, int32_t* count, cudaStream_t st) {
-  if (n <= SEL_SMEM_KEYS) {  // keys (top-k) and the union bitmap in shared memory
-    const size_t smem = 4ull * n;
-    cudaError_t e = allow_smem(select_kernel<true>, smem);
-    if (e != cudaSuccess) return e;
-    return launch(select_kernel<true>, dim3(nrows), SEL_THREADS, smem, st, scores, n, nrows, k, tau, mode, bm, ticket,
-                  idx, count);
-  }
-  return launch(select_kernel<false>, dim3(nrows), SEL_THREADS, 0, st, scores, n, nrows, k, tau, mode, bm, ticket, idx,
-                count);
-}
-
-template <typename T, int NB>
-cudaError_t run_mlp_up_nb(const void* W1t, int d, int N, const float* y, int nb, const float* b1, const int32_t* idx,
-                          const int32_t* count, int k_max, int32_t* seg_idx, float* seg_a, int32_t* seg_cnt,
-                          int* status, int nseg, cudaStream_t st) {
-  const T* w = static_cast<const T*>(W1t);
-  dim3 grid(nseg > 0 ? nseg : 1);
-  switch (rpw_for(d, WT<T>::E)) {
-    case 1: return launch(mlp_up_kernel<T, NB, 1, 8>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status);
-    case 2: return launch(mlp_up_kernel<T, NB, 2, 4>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status);
-    case 4: return launch(mlp_up_kernel<T, NB, 4, 2>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status);
-    default: return launch(mlp_up_kernel<T, NB, 8, 1>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status);
-  }
-}
-
-template <typename T, int NB, class Src>
-cudaError_t run_axpy_st(const void* W, int d, int nrows_w, Src src, const float* bias, float* out, int nb, int k_max,
-                        size_t smem, int* status, cudaStream_t st) {
-  constexpr int E = WT<T>::E;
-  const int tiles = (d + AX_THREADS * E - 1) / (AX_THREADS * E);
-  int G = (2 * sm_count() + tiles - 1) / tiles;
-  const int gmax = (k_max + 3) / 4;
-  if (G > gmax) G = gmax;
-  if (G < 1) G = 1;
-  cudaError_t e = allow_smem(axpy_rows_kernel<T, NB, Src>, smem);
-  if (e != cudaSuccess) return e;
-  return launch(axpy_rows_kernel<T, NB, Src>, dim3(tiles, G), AX_THREADS, smem, st, static_cast<const T*>(W), d,
-                nrows_w, src, bias, out, nb, G, status);
-}
-
-template <typename T, class Src>
-cudaError_t run_axpy(const void* W, int d, int nrows_w, Src src, const float* bias, float* out, int nb, int k_max,
-                     size_t smem, int* status, cudaStream_t st) {
-  switch (nb_bucket(nb)) {
-    case 1: return run_axpy_st<T, 1>(W, d, nrows_w, src, bias, out, nb, k_max, smem, status, st);
-    case 2: return run_axpy_st<T, 2>(W, d, nrows_w, src, bias, out, nb, k_max, smem, status, st);
-    case 4: return run_axpy_st<T, 4>(W, d, nrows_w, src, bias, out, nb, k_max, smem, status, st);
-    case 8: return run_axpy_st<T, 8>(W, d, nrows_w, src, bias, out, nb, k_max, smem, status, st);
-    default: return run_axpy_st<T, 16>(W, d, nrows_w, src, bias, out, nb, k_max, smem, status, st);
-  }
-}
-
-template <typename T>
-cudaError_t run_mlp_up(const void* W1t, int d, int N, const float* y, int nb, const float* b1, const int32_t* idx,
-                       const int32_t* count, int k_max, int32_t* seg_idx, float* seg_a, int32_t* seg_cnt, int* status,
-                       int nseg, cudaStream_t st) {
-  switch (nb_bucket(nb)) {
-    case 1: return run_mlp_up_nb<T, 1>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, st);
-    case 2: return run_mlp_up_nb<T, 2>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, st);
-    case 4: return run_mlp_up_nb<T, 4>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, st);
-    case 8: return run_mlp_up_nb<T, 8>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, st);
-    default: return run_mlp_up_nb<T, 16>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, st);
-  }
-}
-
-template <typename T, int NB>
-cudaError_t run_qkv_nb(const void* Wqkv, int d, int h, int dh, const float* y, int nb, const float* bqkv,
-                       const int32_t* head_idx, const int32_t* head_count, int kh_max, float* q, void* Kc, void* Vc,
-                       int cap, int pos, int* status, cudaStream_t st) {
-  const T* w = static_cast<const T*>(Wqkv);
-  const int rpw = rpw_for(d, WT<T>::E);
-  const int slots = kh_max * 3 * dh;
-  const int per_cta = GEMV_WARPS * rpw;
-  dim3 grid((slots + per_cta - 1) / per_cta > 0 ? (slots + per_cta - 1) / per_cta : 1);
-  T* K = static_cast<T*>(Kc);
-  T* V = static_cast<T*>(Vc);
-  switch (rpw) {
-    case 1: return launch(qkv_kernel<T, NB, 1, 8>, grid, GEMV_THREADS, 0, st, w, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, K, V, cap, pos, status);
-    case 2: return launch(qkv_kernel<T, NB, 2, 4>, grid, GEMV_THREADS, 0, st, w, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, K, V, cap, pos, status);
-    case 4: return launch(qkv_kernel<T, NB, 4, 2>, grid, GEMV_THREADS, 0, st, w, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, K, V, cap, pos, status);
-    default: return launch(qkv_kernel<T, NB, 8, 1>, grid, GEMV_THREADS, 0, st, w, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, K, V, cap, pos, status);
-  }
-}
-
-template <typename T>
-cudaError_t run_qkv(const void* Wqkv, int d, int h, int dh, const float* y, int nb, const float* bqkv,
-                    const int32_t* head_idx, const int32_t* head_count, int kh_max, float* q, void* Kc, void* Vc,
-                    int cap, int pos, int* status, cudaStream_t st) {
-  switch (nb_bucket(nb)) {
-    case 1: return run_qkv_nb<T, 1>(Wqkv, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, Kc, Vc, cap, pos, status, st);
-    case 2: return run_qkv_nb<T, 2>(Wqkv, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, Kc, Vc, cap, pos, status, st);
-    case 4: return run_qkv_nb<T, 4>(Wqkv, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, Kc, Vc, cap, pos, status, st);
-    case 8: return run_qkv_nb<T, 8>(Wqkv, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, Kc, Vc, cap, pos, status, st);
-    default: return run_qkv_nb<T, 16>(Wqkv, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, Kc, Vc, cap, pos, status, st);
-  }
-}
-
-// Keys per split: the largest of 64 / 32 that still gives >= 2 CTAs per SM.
-int attn_split_len(int B, int kh_max, int pos) {
-  const int want = 2 * sm_count();
-  if ((long long)B * kh_max * ((pos + 1 + 63) / 64) >= want) return 64;
-  return 32;
-}
-
-template <typename KT, int DH>
-cudaError_t run_attn_dh(const float* q, const void* Kc, const void* Vc, int B, int h, int cap, int pos, float scale,
-                        const int32_t* head_idx, const int32_t* head_count, int kh_max, float* part, unsigned* ctr,
-                        float* H, int* status, cudaStream_t st) {
-  const int S = (sizeof(KT) * DH * 64 * 2 <= 32768) ? attn_split_len(B, kh_max, pos) : 32;
-  const int nsplit = (pos + 1 + S - 1) / S;
-  dim3 grid(nsplit, kh_max, B);
-  const KT* K = static_cast<const KT*>(Kc);
-  const KT* V = static_cast<const KT*>(Vc);
-  if constexpr (sizeof(KT) * DH * 64 * 2 <= 32768) {  // K and V tiles in static shared memory
-    if (S == 64)
-      return launch(attn_split_kernel<KT, DH, 64>, grid, ATTN_THREADS, 0, st, q, K, V, h, cap, pos, scale, head_idx,
-                    head_count, kh_max, nsplit, part, ctr, H, status);
-  }
-  return launch(attn_split_kernel<KT, DH, 32>, grid, ATTN_THREADS, 0, st, q, K, V, h, cap, pos, scale, head_idx,
-                head_count, kh_max, nsplit, part, ctr, H, status);
-}
-
-template <typename KT>
-cudaError_t run_attn(int dh, const float* q, const void* Kc, const void* Vc, int B, int h, int cap, int pos,
-                     float scale, const int32_t* head_idx, const int32_t* head_count, int kh_max, float* part,
-                     unsigned* ctr, float* H, int* status, cudaStream_t st) {
-  if (dh == 64)
-    return run_attn_dh<KT, 64>(q, Kc, Vc, B, h, cap, pos, scale, head_idx, head_count, kh_max, part, ctr, H, status, st);
-  return run_attn_dh<KT, 128>(q, Kc, Vc, B, h, cap, pos, scale, head_idx, head_count, kh_max, part, ctr, H, status, st);
-}
-
-// ---------------------------------------------------------------------------
 // Operation bodies shared by the public entry points
 // ---------------------------------------------------------------------------
 
@@ -418,19 +131,14 @@ dv_status do_sparse_mlp(const Layout& L, void* ws, const float* y, int B, int d,
   if (L.nseg == 0) {
     if (b2) {  // nothing selected: out (+)= b2 only
       RowsHeads none{idx, count, nullptr, 0, 1, 0};
-      return cuda_status(dt == DV_BF16 ? run_axpy<bf16>(W2t, d, N, none, b2, out, B, 1, 0, status, st)
-                                       : run_axpy<float>(W2t, d, N, none, b2, out, B, 1, 0, status, st));
+      return cuda_status(run_axpy_dt(dt, W2t, d, N, none, b2, out, B, 1, 0, status, st));
     }
     return DV_OK;
   }
-  if (dt == DV_BF16)
-    DV_TRY(run_mlp_up<bf16>(W1t, d, N, y, B, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, L.nseg, st));
-  else
-    DV_TRY(run_mlp_up<float>(W1t, d, N, y, B, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, L.nseg, st));
+  DV_TRY(run_mlp_up_dt(dt, W1t, d, N, y, B, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, L.nseg, st));
   RowsMlp src{seg_idx, seg_a, seg_cnt, L.nseg, L.SEG};
   const size_t smem = 4ull * (L.nseg + 1);
-  return cuda_status(dt == DV_BF16 ? run_axpy<bf16>(W2t, d, N, src, b2, out, B, k_max, smem, status, st)
-                                   : run_axpy<float>(W2t, d, N, src, b2, out, B, k_max, smem, status, st));
+  return cuda_status(run_axpy_dt(dt, W2t, d, N, src, b2, out, B, k_max, smem, status, st));
 }
 
 dv_status do_sparse_mha(const Layout& L, void* ws, const float* y, int B, int d, int h, int dh, const void* Wqkv,
@@ -442,25 +150,17 @@ dv_status do_sparse_mha(const Layout& L, void* ws, const float* y, int B, int d,
   if (kh_max == 0) {
     if (bO) {
       RowsHeads none{head_idx, head_count, nullptr, 0, dh, h};
-      return cuda_status(dt == DV_BF16 ? run_axpy<bf16>(WOt, d, h * dh, none, bO, out, B, 1, 0, status, st)
-                                       : run_axpy<float>(WOt, d, h * dh, none, bO, out, B, 1, 0, status, st));
+      return cuda_status(run_axpy_dt(dt, WOt, d, h * dh, none, bO, out, B, 1, 0, status, st));
     }
     return DV_OK;
   }
   float* q = at<float>(ws, L.q);
   float* H = at<float>(ws, L.H);
-  if (dt == DV_BF16) {
-    DV_TRY(run_qkv<bf16>(Wqkv, d, h, dh, y, B, bqkv, head_idx, head_count, kh_max, q, Kc, Vc, cap, pos, status, st));
-    DV_TRY(run_attn<bf16>(dh, q, Kc, Vc, B, h, cap, pos, scale, head_idx, head_count, kh_max, at<float>(ws, L.part),
-                          at<unsigned>(ws, L.attn_ctr), H, status, st));
-  } else {
-    DV_TRY(run_qkv<float>(Wqkv, d, h, dh, y, B, bqkv, head_idx, head_count, kh_max, q, Kc, Vc, cap, pos, status, st));
-    DV_TRY(run_attn<float>(dh, q, Kc, Vc, B, h, cap, pos, scale, head_idx, head_count, kh_max, at<float>(ws, L.part),
-                           at<unsigned>(ws, L.attn_ctr), H, status, st));
-  }
+  DV_TRY(run_qkv_dt(dt, Wqkv, d, h, dh, y, B, bqkv, head_idx, head_count, kh_max, q, Kc, Vc, cap, pos, status, st));
+  DV_TRY(run_attn_dt(dt, dh, q, Kc, Vc, B, h, cap, pos, scale, head_idx, head_count, kh_max, at<float>(ws, L.part),
+                     at<unsigned>(ws, L.attn_ctr), H, status, st));
   RowsHeads src{head_idx, head_count, H, kh_max, dh, h};
-  return cuda_status(dt == DV_BF16 ? run_axpy<bf16>(WOt, d, h * dh, src, bO, out, B, kh_max * dh, 0, status, st)
-                                   : run_axpy<float>(WOt, d, h * dh, src, bO, out, B, kh_max * dh, 0, status, st));
+  return cuda_status(run_axpy_dt(dt, WOt, d, h * dh, src, bO, out, B, kh_max * dh, 0, status, st));
 }
 
 int wbytes_of(dv_dtype t) { return t == DV_BF16 ? 2 : 4; }
@@ -477,10 +177,6 @@ dv_status check_ws(const Layout& L, void* ws, size_t ws_bytes) {
 // Fused layer path (dv_fused.cuh)
 // ---------------------------------------------------------------------------
 
-constexpr int ATTN_CS = 8;  // CTAs per cluster (per selected head) in attn_out_kernel
-
-int attn_out_S(int pos) { return (pos + 1 + ATTN_CS - 1) / ATTN_CS; }
-size_t attn_out_smem(int S, int dh, int kvbytes) { return 2ull * S * dh * kvbytes + 4ull * S; }
 
 bool fused_enabled() {
   static const bool on = [] {
@@ -502,218 +198,6 @@ bool fused_ok(const dv_dims& D, dv_dtype wdt) {
   return true;
 }
 
-template <typename K, typename A>
-cudaError_t launch_fused(K kern, dim3 grid, size_t smem, cudaStream_t st, const A& a) {
-  cudaError_t e = allow_smem(kern, smem);
-  if (e != cudaSuccess) return e;
-  return launch(kern, grid, FUSED_THREADS, smem, st, a);
-}
-
-template <typename T, int NB>
-cudaError_t run_attn_in_nb(const AttnInArgs& a, cudaStream_t st) {
-  const int rpw = rpw_for(a.d, WT<T>::E);
-  const int slots = a.kh_max * 3 * a.dh, per = FUSED_WARPS * rpw;
-  const dim3 grid(slots > 0 ? (slots + per - 1) / per : 1);
-  const size_t smem = 4ull * a.nb * a.d;
-  switch (rpw) {
-    case 1: return launch_fused(attn_in_kernel<T, NB, 1, 8>, grid, smem, st, a);
-    case 2: return launch_fused(attn_in_kernel<T, NB, 2, 4>, grid, smem, st, a);
-    case 4: return launch_fused(attn_in_kernel<T, NB, 4, 2>, grid, smem, st, a);
-    default: return launch_fused(attn_in_kernel<T, NB, 8, 1>, grid, smem, st, a);
-  }
-}
-
-template <typename T>
-cudaError_t run_attn_in(const AttnInArgs& a, cudaStream_t st) {
-  switch (nb_bucket(a.nb)) {
-    case 1: return run_attn_in_nb<T, 1>(a, st);
-    case 2: return run_attn_in_nb<T, 2>(a, st);
-    case 4: return run_attn_in_nb<T, 4>(a, st);
-    case 8: return run_attn_in_nb<T, 8>(a, st);
-    default: return run_attn_in_nb<T, 16>(a, st);
-  }
-}
-
-template <typename KT, int DH, int NB>
-cudaError_t run_attn_out_nb(const AttnOutArgs& a, cudaStream_t st) {
-  const size_t smem = attn_out_smem(a.S, DH, sizeof(KT));
-  auto kern = attn_out_kernel<KT, DH, ATTN_CS, NB>;
-  cudaError_t e = allow_smem(kern, smem);
-  if (e != cudaSuccess) return e;
-  return launch_cluster(kern, dim3(ATTN_CS, a.kh_max > 0 ? a.kh_max : 1), FUSED_THREADS, smem, st, ATTN_CS, a);
-}
-
-template <typename KT, int DH>
-cudaError_t run_attn_out_dh(const AttnOutArgs& a, cudaStream_t st) {
-  switch (nb_bucket(a.nb)) {
-    case 1: return run_attn_out_nb<KT, DH, 1>(a, st);
-    case 2: return run_attn_out_nb<KT, DH, 2>(a, st);
-    case 4: return run_attn_out_nb<KT, DH, 4>(a, st);
-    case 8: return run_attn_out_nb<KT, DH, 8>(a, st);
-    default: return run_attn_out_nb<KT, DH, 16>(a, st);
-  }
-}
-
-template <typename KT>
-cudaError_t run_attn_out(const AttnOutArgs& a, cudaStream_t st) {
-  return a.dh == 64 ? run_attn_out_dh<KT, 64>(a, st) : run_attn_out_dh<KT, 128>(a, st);
-}
-
-int mlp_block_grid(int k_max) {
-  const int g = (k_max + 7) / 8;
-  return g < 1 ? 1 : (g > sm_count() ? sm_count() : g);
-}
-
-template <typename T, int NB>
-cudaError_t run_mlp_block_nb(const MlpBlockArgs& a, cudaStream_t st) {
-  const int rpw = rpw_for(a.d, WT<T>::E);
-  const dim3 grid(a.G);
-  const size_t smem = 4ull * a.nb * a.d;
-  switch (rpw) {
-    case 1: return launch_fused(mlp_block_kernel<T, NB, 1, 8>, grid, smem, st, a);
-    case 2: return launch_fused(mlp_block_kernel<T, NB, 2, 4>, grid, smem, st, a);
-    case 4: return launch_fused(mlp_block_kernel<T, NB, 4, 2>, grid, smem, st, a);
-    default: return launch_fused(mlp_block_kernel<T, NB, 8, 1>, grid, smem, st, a);
-  }
-}
-
-template <typename T>
-cudaError_t run_mlp_block(const MlpBlockArgs& a, cudaStream_t st) {
-  switch (nb_bucket(a.nb)) {
-    case 1: return run_mlp_block_nb<T, 1>(a, st);
-    case 2: return run_mlp_block_nb<T, 2>(a, st);
-    case 4: return run_mlp_block_nb<T, 4>(a, st);
-    case 8: return run_mlp_block_nb<T, 8>(a, st);
-    default: return run_mlp_block_nb<T, 16>(a, st);
-  }
-}
-
-template <typename T, int NB>
-cudaError_t run_predict_a_nb(const PredictAArgs& a, cudaStream_t st) {
-  const int rows = (a.PA ? a.h : 0) + (a.At ? a.r : 0);
-  const int rpw = rpw_for(a.d, WT<T>::E), per = FUSED_WARPS * rpw;
-  const dim3 grid(rows > 0 ? (rows + per - 1) / per : 1);
-  switch (rpw) {
-    case 1: return launch(predict_a_kernel<T, NB, 1, 8>, grid, FUSED_THREADS, 0, st, a);
-    case 2: return launch(predict_a_kernel<T, NB, 2, 4>, grid, FUSED_THREADS, 0, st, a);
-    case 4: return launch(predict_a_kernel<T, NB, 4, 2>, grid, FUSED_THREADS, 0, st, a);
-    default: return launch(predict_a_kernel<T, NB, 8, 1>, grid, FUSED_THREADS, 0, st, a);
-  }
-}
-
-template <typename T>
-cudaError_t run_predict_a(const PredictAArgs& a, cudaStream_t st) {
-  switch (nb_bucket(a.nb)) {
-    case 1: return run_predict_a_nb<T, 1>(a, st);
-    case 2: return run_predict_a_nb<T, 2>(a, st);
-    case 4: return run_predict_a_nb<T, 4>(a, st);
-    case 8: return run_predict_a_nb<T, 8>(a, st);
-    default: return run_predict_a_nb<T, 16>(a, st);
-  }
-}
-
-template <typename T, int NB>
-cudaError_t run_predict_b_nb(const PredictBArgs& a, cudaStream_t st) {
-  const int rpw = rpw_for(a.r, WT<T>::E), per = FUSED_WARPS * rpw;
-  const dim3 grid((a.N + per - 1) / per);
-  switch (rpw) {
-    case 1: return launch(predict_b_kernel<T, NB, 1, 8>, grid, FUSED_THREADS, 0, st, a);
-    case 2: return launch(predict_b_kernel<T, NB, 2, 4>, grid, FUSED_THREADS, 0, st, a);
-    case 4: return launch(predict_b_kernel<T, NB, 4, 2>, grid, FUSED_THREADS, 0, st, a);
-    default: return launch(predict_b_kernel<T, NB, 8, 1>, grid, FUSED_THREADS, 0, st, a);
-  }
-}
-
-template <typename T>
-cudaError_t run_predict_b(const PredictBArgs& a, cudaStream_t st) {
-  switch (nb_bucket(a.nb)) {
-    case 1: return run_predict_b_nb<T, 1>(a, st);
-    case 2: return run_predict_b_nb<T, 2>(a, st);
-    case 4: return run_predict_b_nb<T, 4>(a, st);
-    case 8: return run_predict_b_nb<T, 8>(a, st);
-    default: return run_predict_b_nb<T, 16>(a, st);
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Column-owner kernels (dv_colowner.cuh) for batch 1-2
-// ---------------------------------------------------------------------------
-
-int co_nv(int d, int E) { return (d + CO_THREADS * E - 1) / (CO_THREADS * E); }
-// Rows per group: 8 or more 16-byte loads in flight per thread. The MLP
-// kernel also holds the W2 rows and its output slice, so it keeps fewer.
-int co_r(int nv) { return nv == 1 ? 8 : nv == 2 ? 4 : nv == 3 ? 3 : 4; }
-int co_r_mlp(int nv) { return nv == 1 ? 8 : nv == 2 ? 4 : nv == 3 ? 3 : 2; }
-bool co_ok(int nb, int d, int E) { return nb <= 2 && co_nv(d, E) <= 6; }
-int co_grid(long long groups) {
-  const long long cap = 2ll * sm_count();
-  return (int)(groups < 1 ? 1 : (groups > cap ? cap : groups));
-}
-
-#define DV_CO_SWITCH(KERN, NB, grid, st, a)                                   \
-  switch (nv) {                                                              \
-    case 1: return launch(KERN<T, NB, 1, 8>, grid, CO_THREADS, 0, st, a);    \
-    case 2: return launch(KERN<T, NB, 2, 4>, grid, CO_THREADS, 0, st, a);    \
-    case 3: return launch(KERN<T, NB, 3, 3>, grid, CO_THREADS, 0, st, a);    \
-    case 4: return launch(KERN<T, NB, 4, 4>, grid, CO_THREADS, 0, st, a);    \
-    case 5: return launch(KERN<T, NB, 5, 4>, grid, CO_THREADS, 0, st, a);    \
-    default: return launch(KERN<T, NB, 6, 4>, grid, CO_THREADS, 0, st, a);   \
-  }
-#define DV_CO_SWITCH_MLP(KERN, NB, grid, st, a)                               \
-  switch (nv) {                                                              \
-    case 1: return launch(KERN<T, NB, 1, 8>, grid, CO_THREADS, 0, st, a);    \
-    case 2: return launch(KERN<T, NB, 2, 4>, grid, CO_THREADS, 0, st, a);    \
-    case 3: return launch(KERN<T, NB, 3, 3>, grid, CO_THREADS, 0, st, a);    \
-    case 4: return launch(KERN<T, NB, 4, 2>, grid, CO_THREADS, 0, st, a);    \
-    case 5: return launch(KERN<T, NB, 5, 2>, grid, CO_THREADS, 0, st, a);    \
-    default: return launch(KERN<T, NB, 6, 2>, grid, CO_THREADS, 0, st, a);   \
-  }
-
-template <typename T, int NB>
-cudaError_t run_attn_in_co_nb(const AttnInArgs& a, cudaStream_t st) {
-  const int nv = co_nv(a.d, WT<T>::E), R = co_r(nv);
-  const dim3 grid(co_grid(((long long)a.kh_max * 3 * a.dh + R - 1) / R));
-  DV_CO_SWITCH(attn_in_co_kernel, NB, grid, st, a)
-}
-
-template <typename T, int NB>
-cudaError_t run_mlp_block_co_nb(MlpBlockArgs a, cudaStream_t st) {
-  const int nv = co_nv(a.d, WT<T>::E), R = co_r_mlp(nv);
-  a.G = co_grid(((long long)a.k_max + R - 1) / R);
-  const dim3 grid(a.G);
-  DV_CO_SWITCH_MLP(mlp_block_co_kernel, NB, grid, st, a)
-}
-
-template <typename T, int NB>
-cudaError_t run_predict_a_co_nb(const PredictAArgs& a, cudaStream_t st) {
-  const int nv = co_nv(a.d, WT<T>::E), R = co_r(nv);
-  const int rows = (a.PA ? a.h : 0) + (a.At ? a.r : 0);
-  const dim3 grid(co_grid((rows + R - 1) / R));
-  DV_CO_SWITCH(predict_a_co_kernel, NB, grid, st, a)
-}
-#undef DV_CO_SWITCH
-#undef DV_CO_SWITCH_MLP
-
-template <typename T>
-cudaError_t run_attn_in_any(const AttnInArgs& a, cudaStream_t st) {
-  if (co_ok(a.nb, a.d, WT<T>::E))
-    return a.nb == 1 ? run_attn_in_co_nb<T, 1>(a, st) : run_attn_in_co_nb<T, 2>(a, st);
-  return run_attn_in<T>(a, st);
-}
-
-template <typename T>
-cudaError_t run_mlp_block_any(const MlpBlockArgs& a, cudaStream_t st) {
-  if (co_ok(a.nb, a.d, WT<T>::E))
-    return a.nb == 1 ? run_mlp_block_co_nb<T, 1>(a, st) : run_mlp_block_co_nb<T, 2>(a, st);
-  return run_mlp_block<T>(a, st);
-}
-
-template <typename T>
-cudaError_t run_predict_a_any(const PredictAArgs& a, cudaStream_t st) {
-  if (co_ok(a.nb, a.d, WT<T>::E))
-    return a.nb == 1 ? run_predict_a_co_nb<T, 1>(a, st) : run_predict_a_co_nb<T, 2>(a, st);
-  return run_predict_a<T>(a, st);
-}
 
 // The head set (heads) and/or the neuron set (neurons) predicted from y:
 // predict_a (head scores, z = y A), predict_b (neuron scores + first digit
@@ -731,7 +215,7 @@ dv_status fused_predict(const Layout& L, void* ws, const dv_layer_weights* w, co
   a.nb = D.B;
   a.scores_h = sh;
   a.z = at<float>(ws, L.z);
-  DV_TRY(w->wdtype == DV_BF16 ? run_predict_a_any<bf16>(a, st) : run_predict_a_any<float>(a, st));
+  DV_TRY(run_predict_a_any_dt(w->wdtype, a, st));
   const bool hist_mode = p->mode == DV_TOPK && p->k > 0 && p->k < D.N;
   if (neurons) {
     PredictBArgs b = {};
@@ -744,7 +228,7 @@ dv_status fused_predict(const Layout& L, void* ws, const dv_layer_weights* w, co
     b.hist_mode = hist_mode ? 1 : 0;
     b.scores = sm;
     b.hist = at<unsigned>(ws, L.hist);
-    DV_TRY(w->wdtype == DV_BF16 ? run_predict_b<bf16>(b, st) : run_predict_b<float>(b, st));
+    DV_TRY(run_predict_b_dt(w->wdtype, b, st));
   }
   SelectFinishArgs f = {};
   f.scores = sm;
@@ -833,7 +317,7 @@ dv_status layer_begin(const Layout& L, void* ws, const dv_layer_weights* w, cons
     a.nb = D.B;
     a.sets_ready = sel ? 1 : 0;
     a.status = status;
-    return cuda_status(w->wdtype == DV_BF16 ? run_attn_in_any<bf16>(a, st) : run_attn_in_any<float>(a, st));
+    return cuda_status(run_attn_in_any_dt(w->wdtype, a, st));
   }
   // kernel-per-step path
   float* yA = r.yA;
@@ -848,11 +332,7 @@ dv_status layer_begin(const Layout& L, void* ws, const dv_layer_weights* w, cons
                               r.hcnt, st));
   if (D.kh_max == 0) return DV_OK;
   float* q = at<float>(ws, L.q);
-  return cuda_status(w->wdtype == DV_BF16
-                         ? run_qkv<bf16>(w->Wqkv, D.d, D.h, D.dh, yA, D.B, w->bqkv, r.use_hidx, r.use_hcnt, D.kh_max,
-                                         q, w->Kc, w->Vc, D.cap, pos, status, st)
-                         : run_qkv<float>(w->Wqkv, D.d, D.h, D.dh, yA, D.B, w->bqkv, r.use_hidx, r.use_hcnt,
-                                          D.kh_max, q, w->Kc, w->Vc, D.cap, pos, status, st));
+  return cuda_status(run_qkv_dt(w->wdtype, w->Wqkv, D.d, D.h, D.dh, yA, D.B, w->bqkv, r.use_hidx, r.use_hcnt, D.kh_max, q, w->Kc, w->Vc, D.cap, pos, status, st));
 }
 
 // Attention half: split attention over the selected heads, W^O, residual.
@@ -882,27 +362,18 @@ dv_status layer_attn(const Layout& L, void* ws, const dv_layer_weights* w, const
     b.sets_ready = sel ? 1 : 0;
     b.scale = p->scale;
     b.status = status;
-    return cuda_status(w->kvdtype == DV_BF16 ? run_attn_out<bf16>(b, st) : run_attn_out<float>(b, st));
+    return cuda_status(run_attn_out_dt(w->kvdtype, b, st));
   }
   if (D.kh_max > 0) {
     float* H = at<float>(ws, L.H);
     const float* q = at<float>(ws, L.q);
-    DV_TRY(w->kvdtype == DV_BF16
-               ? run_attn<bf16>(D.dh, q, w->Kc, w->Vc, D.B, D.h, D.cap, pos, p->scale, r.use_hidx, r.use_hcnt,
-                                D.kh_max, at<float>(ws, L.part), at<unsigned>(ws, L.attn_ctr), H, status, st)
-               : run_attn<float>(D.dh, q, w->Kc, w->Vc, D.B, D.h, D.cap, pos, p->scale, r.use_hidx, r.use_hcnt,
-                                 D.kh_max, at<float>(ws, L.part), at<unsigned>(ws, L.attn_ctr), H, status, st));
+    DV_TRY(run_attn_dt(w->kvdtype, D.dh, q, w->Kc, w->Vc, D.B, D.h, D.cap, pos, p->scale, r.use_hidx, r.use_hcnt, D.kh_max, at<float>(ws, L.part), at<unsigned>(ws, L.attn_ctr), H, status, st));
     RowsHeads src{r.use_hidx, r.use_hcnt, H, D.kh_max, D.dh, D.h};
-    return cuda_status(w->wdtype == DV_BF16 ? run_axpy<bf16>(w->WOt, D.d, D.h * D.dh, src, w->bO, x, D.B,
-                                                             D.kh_max * D.dh, 0, status, st)
-                                            : run_axpy<float>(w->WOt, D.d, D.h * D.dh, src, w->bO, x, D.B,
-                                                              D.kh_max * D.dh, 0, status, st));
+    return cuda_status(run_axpy_dt(w->wdtype, w->WOt, D.d, D.h * D.dh, src, w->bO, x, D.B, D.kh_max * D.dh, 0, status, st));
   }
   if (w->bO) {
     RowsHeads none{r.use_hidx, r.use_hcnt, nullptr, 0, D.dh, D.h};
-    return cuda_status(w->wdtype == DV_BF16
-                           ? run_axpy<bf16>(w->WOt, D.d, D.h * D.dh, none, w->bO, x, D.B, 1, 0, status, st)
-                           : run_axpy<float>(w->WOt, D.d, D.h * D.dh, none, w->bO, x, D.B, 1, 0, status, st));
+    return cuda_status(run_axpy_dt(w->wdtype, w->WOt, D.d, D.h * D.dh, none, w->bO, x, D.B, 1, 0, status, st));
   }
   return DV_OK;
 }
@@ -939,7 +410,7 @@ dv_status layer_mlp(const Layout& L, void* ws, const dv_layer_weights* w, const 
     c.sets_ready = sel ? 1 : 0;
     c.yM_out = sel ? (trace ? trace->yM : nullptr) : nullptr;
     c.status = status;
-    return cuda_status(w->wdtype == DV_BF16 ? run_mlp_block_any<bf16>(c, st) : run_mlp_block_any<float>(c, st));
+    return cuda_status(run_mlp_block_any_dt(w->wdtype, c, st));
   }
   DV_TRY(launch(layernorm_kernel, dim3(D.B), LN_THREADS, 0, st, (const float*)x, r.yM, D.d, w->ln2_g, w->ln2_b,
                 p->eps));

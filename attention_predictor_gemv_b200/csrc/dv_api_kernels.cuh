@@ -1,0 +1,390 @@
+// Kernels that the C ABI layer launches itself: LayerNorm, the exact
+// selection that ends the look-ahead predictor, its gate, and the L2
+// prefetch of a layer's selected rows. Included by one translation unit.
+#pragma once
+
+#include "dv_fused.cuh"
+
+namespace dv {
+
+// ----------------------------------------------------------------------------
+// LayerNorm: y = (x - mean) / sqrt(var + eps) * g + b, biased variance, one CTA
+// per batch row.
+// ----------------------------------------------------------------------------
+constexpr int LN_THREADS = 512;
+
+__global__ void __launch_bounds__(LN_THREADS)
+    layernorm_kernel(const float* __restrict__ x, float* __restrict__ y, int d, const float* __restrict__ g,
+                     const float* __restrict__ bta, float eps) {
+  __shared__ float red[LN_THREADS / 32];
+  griddep_launch();
+  griddep_wait();
+  const int b = blockIdx.x;
+  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)b * d);
+  float4* yr = reinterpret_cast<float4*>(y + (size_t)b * d);
+  const int n4 = d >> 2;
+  float s = 0.f;
+  for (int i = threadIdx.x; i < n4; i += LN_THREADS) {
+    float4 v = xr[i];
+    s += (v.x + v.y) + (v.z + v.w);
+  }
+  const float mean = block_sum<LN_THREADS>(s, red) / (float)d;
+  float q = 0.f;
+  for (int i = threadIdx.x; i < n4; i += LN_THREADS) {
+    float4 v = xr[i];
+    float a = v.x - mean, c = v.y - mean, e = v.z - mean, f = v.w - mean;
+    q += (a * a + c * c) + (e * e + f * f);
+  }
+  const float var = block_sum<LN_THREADS>(q, red) / (float)d;
+  const float rstd = rsqrtf(var + eps);
+  for (int i = threadIdx.x; i < n4; i += LN_THREADS) {
+    float4 v = xr[i];
+    float4 o = make_float4((v.x - mean) * rstd, (v.y - mean) * rstd, (v.z - mean) * rstd, (v.w - mean) * rstd);
+    if (g) {
+      float4 gg = reinterpret_cast<const float4*>(g)[i];
+      o.x *= gg.x; o.y *= gg.y; o.z *= gg.z; o.w *= gg.w;
+    }
+    if (bta) {
+      float4 bb = reinterpret_cast<const float4*>(bta)[i];
+      o.x += bb.x; o.y += bb.y; o.z += bb.z; o.w += bb.w;
+    }
+    yr[i] = o;
+  }
+}
+
+// ----------------------------------------------------------------------------
+// L2 prefetch of one layer's selected parameters. With the look-ahead
+// predictor the sets of layer l+1 are known while layer l runs; this kernel
+// (on the side stream) asks the bulk-copy engine to bring layer l+1's
+// selected Q/K/V and W^O blocks, the selected heads' KV entries and the
+// selected W1 (and optionally W2) rows into L2, so layer l+1's kernels read
+// them from L2. Fire-and-forget: no data moves through the SMs.
+// ----------------------------------------------------------------------------
+struct PrefetchArgs {
+  const char* Wqkv;
+  const char* WOt;
+  const char* Kc;
+  const char* Vc;
+  const char* W1t;
+  const char* W2t;
+  const int32_t* head_idx;
+  const int32_t* head_count;
+  const int32_t* idx;
+  const int32_t* count;
+  int kh_max, k_max, B, h, dh, d, N, cap, pos, wbytes, kvbytes, with_w2;
+};
+
+__device__ __forceinline__ void prefetch_range(const char* base, size_t bytes, int chunk) {
+  const size_t off = (size_t)chunk * PF_CHUNK;
+  if (off < bytes) prefetch_l2(base + off, (uint32_t)min((size_t)PF_CHUNK, bytes - off));
+}
+
+__global__ void __launch_bounds__(256) prefetch_layer_kernel(PrefetchArgs a) {
+  griddep_launch();
+  griddep_wait();
+  int hc = *a.head_count, cnt = *a.count;
+  hc = hc < 0 ? 0 : (hc > a.kh_max ? a.kh_max : hc);
+  cnt = cnt < 0 ? 0 : (cnt > a.k_max ? a.k_max : cnt);
+  const size_t qkv = (size_t)3 * a.dh * a.d * a.wbytes, wo = (size_t)a.dh * a.d * a.wbytes;
+  const size_t kv = (size_t)a.pos * a.dh * a.kvbytes, row = (size_t)a.d * a.wbytes;
+  const int nq = (int)((qkv + PF_CHUNK - 1) / PF_CHUNK), nwo = (int)((wo + PF_CHUNK - 1) / PF_CHUNK);
+  const int nkv = (int)((kv + PF_CHUNK - 1) / PF_CHUNK), nrow = (int)((row + PF_CHUNK - 1) / PF_CHUNK);
+  const int per_head = nq + nwo + 2 * a.B * nkv;
+  const int per_neuron = nrow * (a.with_w2 ? 2 : 1);
+  const long long total = (long long)hc * per_head + (long long)cnt * per_neuron;
+  for (long long it = blockIdx.x * 256ll + threadIdx.x; it < total; it += (long long)gridDim.x * 256) {
+    if (it < (long long)hc * per_head) {
+      const int p = (int)(it / per_head);
+      int c = (int)(it % per_head);
+      const int head = a.head_idx[p];
+      if (head < 0 || head >= a.h) continue;
+      if (c < nq) {
+        prefetch_range(a.Wqkv + (size_t)head * qkv, qkv, c);
+      } else if ((c -= nq) < nwo) {
+        prefetch_range(a.WOt + (size_t)head * wo, wo, c);
+      } else {
+        c -= nwo;
+        const int which = c / (a.B * nkv);  // 0: K, 1: V
+        c %= a.B * nkv;
+        const int b = c / nkv;
+        const size_t cache_off = (((size_t)b * a.h + head) * a.cap) * a.dh * a.kvbytes;
+        prefetch_range((which ? a.Vc : a.Kc) + cache_off, kv, c % nkv);
+      }
+    } else {
+      const long long r = it - (long long)hc * per_head;
+      const int j = (int)(r / per_neuron);
+      int c = (int)(r % per_neuron);
+      const int neuron = a.idx[j];
+      if (neuron < 0 || neuron >= a.N) continue;
+      const char* base = (c < nrow ? a.W1t : a.W2t) + (size_t)neuron * row;
+      prefetch_range(base, row, c % nrow);
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Exact selection after predict_b_kernel. CTAs 0..B-1 take one neuron score
+// row each (1024 threads, keys in shared memory): the bin of the k-th largest
+// key comes from the global histogram (which this kernel clears), the keys in
+// that bin are collected and refined by two more digit passes, and a
+// warp-ordered pass takes every key above the threshold plus the lowest-index
+// copies of the threshold key. The last neuron CTA unites the rows' bitmaps
+// and writes idx / count. CTA B (when heads are predicted) selects the heads
+// from their scores by rank (few heads: direct comparison).
+// ----------------------------------------------------------------------------
+constexpr int SF_CAND = 2048;  // keeps static + dynamic shared memory within 227 KB at N = 49152
+
+struct SelectFinishArgs {
+  const float* scores;  // [B][N]
+  unsigned* hist;       // [B][2048]
+  uint32_t* bitmaps;    // [B][N/32]
+  unsigned* ticket;
+  int neuron_rows;      // B when the neuron set is selected, else 0
+  int N, nb, k, mode;
+  float tau;
+  int32_t* idx;
+  int32_t* count;
+  const float* scores_h;  // [B][h] or null
+  int h, k_h, mode_h;
+  float tau_h;
+  int32_t* head_idx;
+  int32_t* head_count;
+};
+
+__global__ void __launch_bounds__(SEL_THREADS) select_finish_kernel(SelectFinishArgs a) {
+  extern __shared__ uint32_t s_keys[];  // [N] for a neuron row, [h] for the head row
+  __shared__ unsigned s_h[SEL_BINS];
+  __shared__ uint32_t s_cand[SF_CAND];
+  __shared__ uint32_t s_hsel[HSEL_MAX / 32];
+  __shared__ uint32_t s_bm[SEL_SMEM_KEYS / 32];
+  __shared__ unsigned sc[SEL_WARPS + 1];
+  __shared__ unsigned s_digit, s_kk, s_ncand, s_last;
+  griddep_launch();
+  griddep_wait();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  if ((int)blockIdx.x == a.neuron_rows) {
+    // ---- heads: the union over rows of each row's k_h best (or > tau) ----
+    const int h = a.h, nw = (h + 31) >> 5;
+    for (int w = tid; w < nw; w += SEL_THREADS) s_hsel[w] = 0u;
+    for (int b = 0; b < a.nb; ++b) {
+      __syncthreads();
+      for (int i = tid; i < h; i += SEL_THREADS) s_keys[i] = ord_key(a.scores_h[(size_t)b * h + i]);
+      __syncthreads();
+      for (int i = tid; i < h; i += SEL_THREADS) {
+        bool take;
+        if (a.mode_h == 1) {
+          take = a.scores_h[(size_t)b * h + i] > a.tau_h;
+        } else {
+          const uint32_t ki = s_keys[i];
+          int rank = 0;
+          for (int j = 0; j < h; ++j) {
+            const uint32_t kj = s_keys[j];
+            rank += (kj > ki) || (kj == ki && j < i);
+          }
+          take = rank < a.k_h;
+        }
+        if (take) atomicOr(&s_hsel[i >> 5], 1u << (i & 31));
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      unsigned base = 0;
+      for (int w0 = 0; w0 < nw; w0 += 32) {
+        const int w = w0 + lane;
+        const uint32_t u = w < nw ? s_hsel[w] : 0u;
+        const unsigned c = __popc(u);
+        unsigned incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        unsigned off = base + incl - c;
+        uint32_t v = u;
+        while (v) {
+          const int jb = __ffs(v) - 1;
+          v &= v - 1u;
+          a.head_idx[off++] = w * 32 + jb;
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) *a.head_count = (int32_t)base;
+    }
+    return;
+  }
+
+  // ---- one neuron score row ----
+  const int b = blockIdx.x, n = a.N;
+  const float* row = a.scores + (size_t)b * n;
+  const int nw = (n + 31) >> 5;
+  uint32_t* bm = a.bitmaps + (size_t)b * nw;
+  const int wpw = (nw + SEL_WARPS - 1) / SEL_WARPS;
+  const int w0 = warp * wpw, w1 = min(nw, w0 + wpw);
+  const bool hist_mode = a.mode == 0 && a.k > 0 && a.k < n;
+  if (!hist_mode) {
+    for (int w = w0; w < w1; ++w) {
+      const int i = w * 32 + lane;
+      const bool take = i < n && (a.mode == 1 ? row[i] > a.tau : a.k > 0);
+      const unsigned word = __ballot_sync(0xffffffffu, take);
+      if (lane == 0) s_bm[w] = word;
+    }
+  } else {
+    {  // keys into shared memory, 8 loads in flight per thread
+      constexpr int UNR = 8;
+      for (int i0 = tid; i0 < n; i0 += SEL_THREADS * UNR) {
+        float v[UNR];
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+          const int i = i0 + u * SEL_THREADS;
+          v[u] = i < n ? row[i] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+          const int i = i0 + u * SEL_THREADS;
+          if (i < n) s_keys[i] = ord_key(v[u]);
+        }
+      }
+    }
+    unsigned* gh = a.hist + (size_t)b * SEL_BINS;
+    for (int i = tid; i < SEL_BINS; i += SEL_THREADS) {
+      s_h[i] = gh[i];
+      gh[i] = 0u;  // cleared for the next call
+    }
+    __syncthreads();
+    uint32_t prefix = 0, mask = 0;
+    unsigned kk = (unsigned)a.k;
+    bool use_cand = true;
+#pragma unroll 1
+    for (int pass = 0; pass < 3; ++pass) {
+      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+      const unsigned dmask = pass == 2 ? 0x3ffu : 0x7ffu;
+      if (pass > 0) {
+        for (int i = tid; i < SEL_BINS; i += SEL_THREADS) s_h[i] = 0u;
+        __syncthreads();
+        const int nc = use_cand ? (int)s_ncand : n;
+        const uint32_t* src = use_cand ? s_cand : s_keys;
+        for (int i = tid; i < nc; i += SEL_THREADS) {
+          const uint32_t key = src[i];
+          if ((key & mask) == prefix) atomicAdd(&s_h[(key >> shift) & dmask], 1u);
+        }
+        __syncthreads();
+      }
+      const unsigned c0 = s_h[SEL_BINS - 1 - 2 * tid], c1 = s_h[SEL_BINS - 2 - 2 * tid];
+      unsigned tot;
+      const unsigned above = block_exclusive_scan<SEL_THREADS>(c0 + c1, sc, &tot);
+      if (above < kk && kk <= above + c0 + c1) {
+        if (kk <= above + c0) {
+          s_digit = SEL_BINS - 1 - 2 * tid;
+          s_kk = kk - above;
+        } else {
+          s_digit = SEL_BINS - 2 - 2 * tid;
+          s_kk = kk - above - c0;
+        }
+      }
+      __syncthreads();
+      prefix |= s_digit << shift;
+      mask |= dmask << shift;
+      kk = s_kk;
+      if (pass == 0) {  // the keys of the boundary bin
+        if (tid == 0) s_ncand = 0u;
+        __syncthreads();
+        for (int i = tid; i < n; i += SEL_THREADS) {
+          const uint32_t key = s_keys[i];
+          if ((key & mask) == prefix) {
+            const unsigned at = atomicAdd(&s_ncand, 1u);
+            if (at < SF_CAND) s_cand[at] = key;
+          }
+        }
+        __syncthreads();
+        use_cand = s_ncand <= SF_CAND;
+      }
+    }
+    unsigned eq = 0;
+    for (int w = w0; w < w1; ++w) {
+      const int i = w * 32 + lane;
+      eq += __popc(__ballot_sync(0xffffffffu, i < n && s_keys[i] == prefix));
+    }
+    if (lane == 0) sc[warp] = eq;
+    __syncthreads();
+    if (warp == 0) {
+      const unsigned v = sc[lane];
+      unsigned incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      sc[lane] = incl - v;
+    }
+    __syncthreads();
+    unsigned rank = sc[warp];
+    for (int w = w0; w < w1; ++w) {
+      const int i = w * 32 + lane;
+      const bool ok = i < n;
+      const uint32_t key = ok ? s_keys[i] : 0u;
+      const bool e = ok && key == prefix;
+      const unsigned em = __ballot_sync(0xffffffffu, e);
+      const unsigned rk = rank + __popc(em & ((1u << lane) - 1u));
+      const unsigned word = __ballot_sync(0xffffffffu, ok && (key > prefix || (e && rk < kk)));
+      if (lane == 0) s_bm[w] = word;
+      rank += __popc(em);
+    }
+  }
+  __syncthreads();
+  // union over the neuron rows: with one row the CTA's own bitmap is the
+  // union; otherwise the rows' bitmaps meet in global memory and the last
+  // CTA (ticket) ORs them, loading every word at once
+  if (a.neuron_rows > 1) {
+    for (int w = tid; w < nw; w += SEL_THREADS) bm[w] = s_bm[w];
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = (atomicAdd(a.ticket, 1u) == (unsigned)a.neuron_rows - 1u);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int w = tid; w < nw; w += SEL_THREADS) {
+      uint32_t u = 0;
+      for (int rr = 0; rr < a.neuron_rows; ++rr) u |= __ldcg(a.bitmaps + (size_t)rr * nw + w);
+      s_bm[w] = u;
+    }
+    __syncthreads();
+    if (tid == 0) *a.ticket = 0u;
+  }
+  unsigned pc = 0;
+  for (int w = w0; w < w1; ++w) pc += __popc(s_bm[w]);
+  if (lane == 0) sc[warp] = pc;
+  __syncthreads();
+  if (warp == 0) {
+    const unsigned v = sc[lane];
+    unsigned incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    sc[lane] = incl - v;
+    if (lane == 31) sc[SEL_WARPS] = incl;
+  }
+  __syncthreads();
+  unsigned off = sc[warp];
+  for (int w = w0; w < w1; ++w) {
+    const uint32_t u = s_bm[w];
+    if ((u >> lane) & 1u) a.idx[off + __popc(u & ((1u << lane) - 1u))] = w * 32 + lane;
+    off += __popc(u);
+  }
+  if (tid == 0) *a.count = (int32_t)sc[SEL_WARPS];
+}
+
+// ----------------------------------------------------------------------------
+// Gate: returns once the previous kernel on its stream has completed and its
+// writes are visible. Ends the look-ahead predictor so that a kernel on
+// another stream that depends on it through an event, and that may be
+// launched early by programmatic dependent launch (stream capture can give
+// such a cross-stream edge the programmatic type), cannot start before the
+// predicted sets are complete: it starts at the earliest when the gate has
+// exited.
+// ----------------------------------------------------------------------------
+__global__ void gate_kernel() { griddep_wait(); }
+
+}  // namespace dv

@@ -856,269 +856,5 @@ __global__ void __launch_bounds__(FUSED_THREADS) predict_b_kernel(PredictBArgs a
   }
 }
 
-// ----------------------------------------------------------------------------
-// Exact selection after predict_b_kernel. CTAs 0..B-1 take one neuron score
-// row each (1024 threads, keys in shared memory): the bin of the k-th largest
-// key comes from the global histogram (which this kernel clears), the keys in
-// that bin are collected and refined by two more digit passes, and a
-// warp-ordered pass takes every key above the threshold plus the lowest-index
-// copies of the threshold key. The last neuron CTA unites the rows' bitmaps
-// and writes idx / count. CTA B (when heads are predicted) selects the heads
-// from their scores by rank (few heads: direct comparison).
-// ----------------------------------------------------------------------------
-constexpr int SF_CAND = 2048;  // keeps static + dynamic shared memory within 227 KB at N = 49152
-
-struct SelectFinishArgs {
-  const float* scores;  // [B][N]
-  unsigned* hist;       // [B][2048]
-  uint32_t* bitmaps;    // [B][N/32]
-  unsigned* ticket;
-  int neuron_rows;      // B when the neuron set is selected, else 0
-  int N, nb, k, mode;
-  float tau;
-  int32_t* idx;
-  int32_t* count;
-  const float* scores_h;  // [B][h] or null
-  int h, k_h, mode_h;
-  float tau_h;
-  int32_t* head_idx;
-  int32_t* head_count;
-};
-
-__global__ void __launch_bounds__(SEL_THREADS) select_finish_kernel(SelectFinishArgs a) {
-  extern __shared__ uint32_t s_keys[];  // [N] for a neuron row, [h] for the head row
-  __shared__ unsigned s_h[SEL_BINS];
-  __shared__ uint32_t s_cand[SF_CAND];
-  __shared__ uint32_t s_hsel[HSEL_MAX / 32];
-  __shared__ uint32_t s_bm[SEL_SMEM_KEYS / 32];
-  __shared__ unsigned sc[SEL_WARPS + 1];
-  __shared__ unsigned s_digit, s_kk, s_ncand, s_last;
-  griddep_launch();
-  griddep_wait();
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
-  if ((int)blockIdx.x == a.neuron_rows) {
-    // ---- heads: the union over rows of each row's k_h best (or > tau) ----
-    const int h = a.h, nw = (h + 31) >> 5;
-    for (int w = tid; w < nw; w += SEL_THREADS) s_hsel[w] = 0u;
-    for (int b = 0; b < a.nb; ++b) {
-      __syncthreads();
-      for (int i = tid; i < h; i += SEL_THREADS) s_keys[i] = ord_key(a.scores_h[(size_t)b * h + i]);
-      __syncthreads();
-      for (int i = tid; i < h; i += SEL_THREADS) {
-        bool take;
-        if (a.mode_h == 1) {
-          take = a.scores_h[(size_t)b * h + i] > a.tau_h;
-        } else {
-          const uint32_t ki = s_keys[i];
-          int rank = 0;
-          for (int j = 0; j < h; ++j) {
-            const uint32_t kj = s_keys[j];
-            rank += (kj > ki) || (kj == ki && j < i);
-          }
-          take = rank < a.k_h;
-        }
-        if (take) atomicOr(&s_hsel[i >> 5], 1u << (i & 31));
-      }
-    }
-    __syncthreads();
-    if (warp == 0) {
-      unsigned base = 0;
-      for (int w0 = 0; w0 < nw; w0 += 32) {
-        const int w = w0 + lane;
-        const uint32_t u = w < nw ? s_hsel[w] : 0u;
-        const unsigned c = __popc(u);
-        unsigned incl = c;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += t;
-        }
-        unsigned off = base + incl - c;
-        uint32_t v = u;
-        while (v) {
-          const int jb = __ffs(v) - 1;
-          v &= v - 1u;
-          a.head_idx[off++] = w * 32 + jb;
-        }
-        base += __shfl_sync(0xffffffffu, incl, 31);
-      }
-      if (lane == 0) *a.head_count = (int32_t)base;
-    }
-    return;
-  }
-
-  // ---- one neuron score row ----
-  const int b = blockIdx.x, n = a.N;
-  const float* row = a.scores + (size_t)b * n;
-  const int nw = (n + 31) >> 5;
-  uint32_t* bm = a.bitmaps + (size_t)b * nw;
-  const int wpw = (nw + SEL_WARPS - 1) / SEL_WARPS;
-  const int w0 = warp * wpw, w1 = min(nw, w0 + wpw);
-  const bool hist_mode = a.mode == 0 && a.k > 0 && a.k < n;
-  if (!hist_mode) {
-    for (int w = w0; w < w1; ++w) {
-      const int i = w * 32 + lane;
-      const bool take = i < n && (a.mode == 1 ? row[i] > a.tau : a.k > 0);
-      const unsigned word = __ballot_sync(0xffffffffu, take);
-      if (lane == 0) s_bm[w] = word;
-    }
-  } else {
-    {  // keys into shared memory, 8 loads in flight per thread
-      constexpr int UNR = 8;
-      for (int i0 = tid; i0 < n; i0 += SEL_THREADS * UNR) {
-        float v[UNR];
-#pragma unroll
-        for (int u = 0; u < UNR; ++u) {
-          const int i = i0 + u * SEL_THREADS;
-          v[u] = i < n ? row[i] : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < UNR; ++u) {
-          const int i = i0 + u * SEL_THREADS;
-          if (i < n) s_keys[i] = ord_key(v[u]);
-        }
-      }
-    }
-    unsigned* gh = a.hist + (size_t)b * SEL_BINS;
-    for (int i = tid; i < SEL_BINS; i += SEL_THREADS) {
-      s_h[i] = gh[i];
-      gh[i] = 0u;  // cleared for the next call
-    }
-    __syncthreads();
-    uint32_t prefix = 0, mask = 0;
-    unsigned kk = (unsigned)a.k;
-    bool use_cand = true;
-#pragma unroll 1
-    for (int pass = 0; pass < 3; ++pass) {
-      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-      const unsigned dmask = pass == 2 ? 0x3ffu : 0x7ffu;
-      if (pass > 0) {
-        for (int i = tid; i < SEL_BINS; i += SEL_THREADS) s_h[i] = 0u;
-        __syncthreads();
-        const int nc = use_cand ? (int)s_ncand : n;
-        const uint32_t* src = use_cand ? s_cand : s_keys;
-        for (int i = tid; i < nc; i += SEL_THREADS) {
-          const uint32_t key = src[i];
-          if ((key & mask) == prefix) atomicAdd(&s_h[(key >> shift) & dmask], 1u);
-        }
-        __syncthreads();
-      }
-      const unsigned c0 = s_h[SEL_BINS - 1 - 2 * tid], c1 = s_h[SEL_BINS - 2 - 2 * tid];
-      unsigned tot;
-      const unsigned above = block_exclusive_scan<SEL_THREADS>(c0 + c1, sc, &tot);
-      if (above < kk && kk <= above + c0 + c1) {
-        if (kk <= above + c0) {
-          s_digit = SEL_BINS - 1 - 2 * tid;
-          s_kk = kk - above;
-        } else {
-          s_digit = SEL_BINS - 2 - 2 * tid;
-          s_kk = kk - above - c0;
-        }
-      }
-      __syncthreads();
-      prefix |= s_digit << shift;
-      mask |= dmask << shift;
-      kk = s_kk;
-      if (pass == 0) {  // the keys of the boundary bin
-        if (tid == 0) s_ncand = 0u;
-        __syncthreads();
-        for (int i = tid; i < n; i += SEL_THREADS) {
-          const uint32_t key = s_keys[i];
-          if ((key & mask) == prefix) {
-            const unsigned at = atomicAdd(&s_ncand, 1u);
-            if (at < SF_CAND) s_cand[at] = key;
-          }
-        }
-        __syncthreads();
-        use_cand = s_ncand <= SF_CAND;
-      }
-    }
-    unsigned eq = 0;
-    for (int w = w0; w < w1; ++w) {
-      const int i = w * 32 + lane;
-      eq += __popc(__ballot_sync(0xffffffffu, i < n && s_keys[i] == prefix));
-    }
-    if (lane == 0) sc[warp] = eq;
-    __syncthreads();
-    if (warp == 0) {
-      const unsigned v = sc[lane];
-      unsigned incl = v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-      }
-      sc[lane] = incl - v;
-    }
-    __syncthreads();
-    unsigned rank = sc[warp];
-    for (int w = w0; w < w1; ++w) {
-      const int i = w * 32 + lane;
-      const bool ok = i < n;
-      const uint32_t key = ok ? s_keys[i] : 0u;
-      const bool e = ok && key == prefix;
-      const unsigned em = __ballot_sync(0xffffffffu, e);
-      const unsigned rk = rank + __popc(em & ((1u << lane) - 1u));
-      const unsigned word = __ballot_sync(0xffffffffu, ok && (key > prefix || (e && rk < kk)));
-      if (lane == 0) s_bm[w] = word;
-      rank += __popc(em);
-    }
-  }
-  __syncthreads();
-  // union over the neuron rows: with one row the CTA's own bitmap is the
-  // union; otherwise the rows' bitmaps meet in global memory and the last
-  // CTA (ticket) ORs them, loading every word at once
-  if (a.neuron_rows > 1) {
-    for (int w = tid; w < nw; w += SEL_THREADS) bm[w] = s_bm[w];
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = (atomicAdd(a.ticket, 1u) == (unsigned)a.neuron_rows - 1u);
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    for (int w = tid; w < nw; w += SEL_THREADS) {
-      uint32_t u = 0;
-      for (int rr = 0; rr < a.neuron_rows; ++rr) u |= __ldcg(a.bitmaps + (size_t)rr * nw + w);
-      s_bm[w] = u;
-    }
-    __syncthreads();
-    if (tid == 0) *a.ticket = 0u;
-  }
-  unsigned pc = 0;
-  for (int w = w0; w < w1; ++w) pc += __popc(s_bm[w]);
-  if (lane == 0) sc[warp] = pc;
-  __syncthreads();
-  if (warp == 0) {
-    const unsigned v = sc[lane];
-    unsigned incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    sc[lane] = incl - v;
-    if (lane == 31) sc[SEL_WARPS] = incl;
-  }
-  __syncthreads();
-  unsigned off = sc[warp];
-  for (int w = w0; w < w1; ++w) {
-    const uint32_t u = s_bm[w];
-    if ((u >> lane) & 1u) a.idx[off + __popc(u & ((1u << lane) - 1u))] = w * 32 + lane;
-    off += __popc(u);
-  }
-  if (tid == 0) *a.count = (int32_t)sc[SEL_WARPS];
-}
-
-// ----------------------------------------------------------------------------
-// Gate: returns once the previous kernel on its stream has completed and its
-// writes are visible. Ends the look-ahead predictor so that a kernel on
-// another stream that depends on it through an event, and that may be
-// launched early by programmatic dependent launch (stream capture can give
-// such a cross-stream edge the programmatic type), cannot start before the
-// predicted sets are complete: it starts at the earliest when the gate has
-// exited.
-// ----------------------------------------------------------------------------
-__global__ void gate_kernel() { griddep_wait(); }
 
 }  // namespace dv

@@ -1,0 +1,10 @@
+// Instantiates the launchers of attn_out (split attention + W^O).
+#include "dv_launchers.cuh"
+
+namespace dv {
+
+cudaError_t run_attn_out_dt(dv_dtype kvdt, const AttnOutArgs& a, cudaStream_t st) {
+  return kvdt == DV_BF16 ? run_attn_out<bf16>(a, st) : run_attn_out<float>(a, st);
+}
+
+}  // namespace dv

@@ -12,51 +12,6 @@
 namespace dv {
 
 // ----------------------------------------------------------------------------
-// LayerNorm: y = (x - mean) / sqrt(var + eps) * g + b, biased variance, one CTA
-// per batch row.
-// ----------------------------------------------------------------------------
-constexpr int LN_THREADS = 512;
-
-__global__ void __launch_bounds__(LN_THREADS)
-    layernorm_kernel(const float* __restrict__ x, float* __restrict__ y, int d, const float* __restrict__ g,
-                     const float* __restrict__ bta, float eps) {
-  __shared__ float red[LN_THREADS / 32];
-  griddep_launch();
-  griddep_wait();
-  const int b = blockIdx.x;
-  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)b * d);
-  float4* yr = reinterpret_cast<float4*>(y + (size_t)b * d);
-  const int n4 = d >> 2;
-  float s = 0.f;
-  for (int i = threadIdx.x; i < n4; i += LN_THREADS) {
-    float4 v = xr[i];
-    s += (v.x + v.y) + (v.z + v.w);
-  }
-  const float mean = block_sum<LN_THREADS>(s, red) / (float)d;
-  float q = 0.f;
-  for (int i = threadIdx.x; i < n4; i += LN_THREADS) {
-    float4 v = xr[i];
-    float a = v.x - mean, c = v.y - mean, e = v.z - mean, f = v.w - mean;
-    q += (a * a + c * c) + (e * e + f * f);
-  }
-  const float var = block_sum<LN_THREADS>(q, red) / (float)d;
-  const float rstd = rsqrtf(var + eps);
-  for (int i = threadIdx.x; i < n4; i += LN_THREADS) {
-    float4 v = xr[i];
-    float4 o = make_float4((v.x - mean) * rstd, (v.y - mean) * rstd, (v.z - mean) * rstd, (v.w - mean) * rstd);
-    if (g) {
-      float4 gg = reinterpret_cast<const float4*>(g)[i];
-      o.x *= gg.x; o.y *= gg.y; o.z *= gg.z; o.w *= gg.w;
-    }
-    if (bta) {
-      float4 bb = reinterpret_cast<const float4*>(bta)[i];
-      o.x += bb.x; o.y += bb.y; o.z += bb.z; o.w += bb.w;
-    }
-    yr[i] = o;
-  }
-}
-
-// ----------------------------------------------------------------------------
 // Warp row-dot: one warp forms the dot products of RPW weight rows (K elements
 // each, 16-byte aligned) with nb <= NB fp32 input vectors X[b][0..K). U column
 // steps of RPW loads each are issued before any use: RPW * U = 8 loads of 16
@@ -761,80 +716,12 @@ __global__ void __launch_bounds__(AX_THREADS)
   }
 }
 
-// ----------------------------------------------------------------------------
-// L2 prefetch of one layer's selected parameters. With the look-ahead
-// predictor the sets of layer l+1 are known while layer l runs; this kernel
-// (on the side stream) asks the bulk-copy engine to bring layer l+1's
-// selected Q/K/V and W^O blocks, the selected heads' KV entries and the
-// selected W1 (and optionally W2) rows into L2, so layer l+1's kernels read
-// them from L2. Fire-and-forget: no data moves through the SMs.
-// ----------------------------------------------------------------------------
+// Asks the bulk-copy engine to bring [p, p + bytes) into L2; no data moves
+// through the SM.
 constexpr uint32_t PF_CHUNK = 16384;  // bytes per prefetch request
 
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
-struct PrefetchArgs {
-  const char* Wqkv;
-  const char* WOt;
-  const char* Kc;
-  const char* Vc;
-  const char* W1t;
-  const char* W2t;
-  const int32_t* head_idx;
-  const int32_t* head_count;
-  const int32_t* idx;
-  const int32_t* count;
-  int kh_max, k_max, B, h, dh, d, N, cap, pos, wbytes, kvbytes, with_w2;
-};
-
-__device__ __forceinline__ void prefetch_range(const char* base, size_t bytes, int chunk) {
-  const size_t off = (size_t)chunk * PF_CHUNK;
-  if (off < bytes) prefetch_l2(base + off, (uint32_t)min((size_t)PF_CHUNK, bytes - off));
-}
-
-__global__ void __launch_bounds__(256) prefetch_layer_kernel(PrefetchArgs a) {
-  griddep_launch();
-  griddep_wait();
-  int hc = *a.head_count, cnt = *a.count;
-  hc = hc < 0 ? 0 : (hc > a.kh_max ? a.kh_max : hc);
-  cnt = cnt < 0 ? 0 : (cnt > a.k_max ? a.k_max : cnt);
-  const size_t qkv = (size_t)3 * a.dh * a.d * a.wbytes, wo = (size_t)a.dh * a.d * a.wbytes;
-  const size_t kv = (size_t)a.pos * a.dh * a.kvbytes, row = (size_t)a.d * a.wbytes;
-  const int nq = (int)((qkv + PF_CHUNK - 1) / PF_CHUNK), nwo = (int)((wo + PF_CHUNK - 1) / PF_CHUNK);
-  const int nkv = (int)((kv + PF_CHUNK - 1) / PF_CHUNK), nrow = (int)((row + PF_CHUNK - 1) / PF_CHUNK);
-  const int per_head = nq + nwo + 2 * a.B * nkv;
-  const int per_neuron = nrow * (a.with_w2 ? 2 : 1);
-  const long long total = (long long)hc * per_head + (long long)cnt * per_neuron;
-  for (long long it = blockIdx.x * 256ll + threadIdx.x; it < total; it += (long long)gridDim.x * 256) {
-    if (it < (long long)hc * per_head) {
-      const int p = (int)(it / per_head);
-      int c = (int)(it % per_head);
-      const int head = a.head_idx[p];
-      if (head < 0 || head >= a.h) continue;
-      if (c < nq) {
-        prefetch_range(a.Wqkv + (size_t)head * qkv, qkv, c);
-      } else if ((c -= nq) < nwo) {
-        prefetch_range(a.WOt + (size_t)head * wo, wo, c);
-      } else {
-        c -= nwo;
-        const int which = c / (a.B * nkv);  // 0: K, 1: V
-        c %= a.B * nkv;
-        const int b = c / nkv;
-        const size_t cache_off = (((size_t)b * a.h + head) * a.cap) * a.dh * a.kvbytes;
-        prefetch_range((which ? a.Vc : a.Kc) + cache_off, kv, c % nkv);
-      }
-    } else {
-      const long long r = it - (long long)hc * per_head;
-      const int j = (int)(r / per_neuron);
-      int c = (int)(r % per_neuron);
-      const int neuron = a.idx[j];
-      if (neuron < 0 || neuron >= a.N) continue;
-      const char* base = (c < nrow ? a.W1t : a.W2t) + (size_t)neuron * row;
-      prefetch_range(base, row, c % nrow);
-    }
-  }
 }
 
 }  // namespace dv

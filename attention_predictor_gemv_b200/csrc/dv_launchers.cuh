@@ -1,0 +1,413 @@
+// Kernel launchers: grid shapes and template dispatch. The function
+// templates named at the end are instantiated once, each in its own
+// translation unit (dv_inst_*.cu), so the kernels compile in parallel.
+#pragma once
+
+#include "../../include/dejavu.h"
+#include "dv_colowner.cuh"
+#include "dv_launch.cuh"
+
+namespace dv {
+
+using bf16 = __nv_bfloat16;
+
+// ---------------------------------------------------------------------------
+// Launchers (arguments already checked)
+// ---------------------------------------------------------------------------
+
+template <typename T, int NB>
+cudaError_t run_dense_gemv_nb(const void* W, int nrows, int K, const float* X, int ldx, int nb, const float* bias,
+                              float* out, int ldo, cudaStream_t st) {
+  const T* w = static_cast<const T*>(W);
+  const int rpw = rpw_for(K, WT<T>::E);
+  const int rows_per_cta = GEMV_WARPS * rpw;
+  dim3 grid((nrows + rows_per_cta - 1) / rows_per_cta);
+  switch (rpw) {
+    case 1: return launch(dense_gemv_kernel<T, NB, 1, 8>, grid, GEMV_THREADS, 0, st, w, nrows, K, X, ldx, nb, bias, out, ldo);
+    case 2: return launch(dense_gemv_kernel<T, NB, 2, 4>, grid, GEMV_THREADS, 0, st, w, nrows, K, X, ldx, nb, bias, out, ldo);
+    case 4: return launch(dense_gemv_kernel<T, NB, 4, 2>, grid, GEMV_THREADS, 0, st, w, nrows, K, X, ldx, nb, bias, out, ldo);
+    default: return launch(dense_gemv_kernel<T, NB, 8, 1>, grid, GEMV_THREADS, 0, st, w, nrows, K, X, ldx, nb, bias, out, ldo);
+  }
+}
+
+template <typename T>
+cudaError_t run_dense_gemv(const void* W, int nrows, int K, const float* X, int ldx, int nb, const float* bias,
+                           float* out, int ldo, cudaStream_t st) {
+  switch (nb_bucket(nb)) {
+    case 1: return run_dense_gemv_nb<T, 1>(W, nrows, K, X, ldx, nb, bias, out, ldo, st);
+    case 2: return run_dense_gemv_nb<T, 2>(W, nrows, K, X, ldx, nb, bias, out, ldo, st);
+    case 4: return run_dense_gemv_nb<T, 4>(W, nrows, K, X, ldx, nb, bias, out, ldo, st);
+    case 8: return run_dense_gemv_nb<T, 8>(W, nrows, K, X, ldx, nb, bias, out, ldo, st);
+    default: return run_dense_gemv_nb<T, 16>(W, nrows, K, X, ldx, nb, bias, out, ldo, st);
+  }
+}
+
+cudaError_t run_gemv(dv_dtype dt, const void* W, int nrows, int K, const float* X, int ldx, int nb, const float* bias,
+                     float* out, int ldo, cudaStream_t st);
+
+cudaError_t run_select(const float* scores, int nrows, int n, int k, float tau, int mode, uint32_t* bm,
+                       unsigned* ticket, int32_t* idx, int32_t* count, cudaStream_t st);
+
+template <typename T, int NB>
+cudaError_t run_mlp_up_nb(const void* W1t, int d, int N, const float* y, int nb, const float* b1, const int32_t* idx,
+                          const int32_t* count, int k_max, int32_t* seg_idx, float* seg_a, int32_t* seg_cnt,
+                          int* status, int nseg, cudaStream_t st) {
+  const T* w = static_cast<const T*>(W1t);
+  dim3 grid(nseg > 0 ? nseg : 1);
+  switch (rpw_for(d, WT<T>::E)) {
+    case 1: return launch(mlp_up_kernel<T, NB, 1, 8>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status);
+    case 2: return launch(mlp_up_kernel<T, NB, 2, 4>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status);
+    case 4: return launch(mlp_up_kernel<T, NB, 4, 2>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status);
+    default: return launch(mlp_up_kernel<T, NB, 8, 1>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status);
+  }
+}
+
+template <typename T, int NB, class Src>
+cudaError_t run_axpy_st(const void* W, int d, int nrows_w, Src src, const float* bias, float* out, int nb, int k_max,
+                        size_t smem, int* status, cudaStream_t st) {
+  constexpr int E = WT<T>::E;
+  const int tiles = (d + AX_THREADS * E - 1) / (AX_THREADS * E);
+  int G = (2 * sm_count() + tiles - 1) / tiles;
+  const int gmax = (k_max + 3) / 4;
+  if (G > gmax) G = gmax;
+  if (G < 1) G = 1;
+  cudaError_t e = allow_smem(axpy_rows_kernel<T, NB, Src>, smem);
+  if (e != cudaSuccess) return e;
+  return launch(axpy_rows_kernel<T, NB, Src>, dim3(tiles, G), AX_THREADS, smem, st, static_cast<const T*>(W), d,
+                nrows_w, src, bias, out, nb, G, status);
+}
+
+template <typename T, class Src>
+cudaError_t run_axpy(const void* W, int d, int nrows_w, Src src, const float* bias, float* out, int nb, int k_max,
+                     size_t smem, int* status, cudaStream_t st) {
+  switch (nb_bucket(nb)) {
+    case 1: return run_axpy_st<T, 1>(W, d, nrows_w, src, bias, out, nb, k_max, smem, status, st);
+    case 2: return run_axpy_st<T, 2>(W, d, nrows_w, src, bias, out, nb, k_max, smem, status, st);
+    case 4: return run_axpy_st<T, 4>(W, d, nrows_w, src, bias, out, nb, k_max, smem, status, st);
+    case 8: return run_axpy_st<T, 8>(W, d, nrows_w, src, bias, out, nb, k_max, smem, status, st);
+    default: return run_axpy_st<T, 16>(W, d, nrows_w, src, bias, out, nb, k_max, smem, status, st);
+  }
+}
+
+template <typename T>
+cudaError_t run_mlp_up(const void* W1t, int d, int N, const float* y, int nb, const float* b1, const int32_t* idx,
+                       const int32_t* count, int k_max, int32_t* seg_idx, float* seg_a, int32_t* seg_cnt, int* status,
+                       int nseg, cudaStream_t st) {
+  switch (nb_bucket(nb)) {
+    case 1: return run_mlp_up_nb<T, 1>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, st);
+    case 2: return run_mlp_up_nb<T, 2>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, st);
+    case 4: return run_mlp_up_nb<T, 4>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, st);
+    case 8: return run_mlp_up_nb<T, 8>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, st);
+    default: return run_mlp_up_nb<T, 16>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, st);
+  }
+}
+
+template <typename T, int NB>
+cudaError_t run_qkv_nb(const void* Wqkv, int d, int h, int dh, const float* y, int nb, const float* bqkv,
+                       const int32_t* head_idx, const int32_t* head_count, int kh_max, float* q, void* Kc, void* Vc,
+                       int cap, int pos, int* status, cudaStream_t st) {
+  const T* w = static_cast<const T*>(Wqkv);
+  const int rpw = rpw_for(d, WT<T>::E);
+  const int slots = kh_max * 3 * dh;
+  const int per_cta = GEMV_WARPS * rpw;
+  dim3 grid((slots + per_cta - 1) / per_cta > 0 ? (slots + per_cta - 1) / per_cta : 1);
+  T* K = static_cast<T*>(Kc);
+  T* V = static_cast<T*>(Vc);
+  switch (rpw) {
+    case 1: return launch(qkv_kernel<T, NB, 1, 8>, grid, GEMV_THREADS, 0, st, w, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, K, V, cap, pos, status);
+    case 2: return launch(qkv_kernel<T, NB, 2, 4>, grid, GEMV_THREADS, 0, st, w, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, K, V, cap, pos, status);
+    case 4: return launch(qkv_kernel<T, NB, 4, 2>, grid, GEMV_THREADS, 0, st, w, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, K, V, cap, pos, status);
+    default: return launch(qkv_kernel<T, NB, 8, 1>, grid, GEMV_THREADS, 0, st, w, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, K, V, cap, pos, status);
+  }
+}
+
+template <typename T>
+cudaError_t run_qkv(const void* Wqkv, int d, int h, int dh, const float* y, int nb, const float* bqkv,
+                    const int32_t* head_idx, const int32_t* head_count, int kh_max, float* q, void* Kc, void* Vc,
+                    int cap, int pos, int* status, cudaStream_t st) {
+  switch (nb_bucket(nb)) {
+    case 1: return run_qkv_nb<T, 1>(Wqkv, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, Kc, Vc, cap, pos, status, st);
+    case 2: return run_qkv_nb<T, 2>(Wqkv, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, Kc, Vc, cap, pos, status, st);
+    case 4: return run_qkv_nb<T, 4>(Wqkv, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, Kc, Vc, cap, pos, status, st);
+    case 8: return run_qkv_nb<T, 8>(Wqkv, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, Kc, Vc, cap, pos, status, st);
+    default: return run_qkv_nb<T, 16>(Wqkv, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, Kc, Vc, cap, pos, status, st);
+  }
+}
+
+// Keys per split: the largest of 64 / 32 that still gives >= 2 CTAs per SM.
+inline int attn_split_len(int B, int kh_max, int pos) {
+  const int want = 2 * sm_count();
+  if ((long long)B * kh_max * ((pos + 1 + 63) / 64) >= want) return 64;
+  return 32;
+}
+
+template <typename KT, int DH>
+cudaError_t run_attn_dh(const float* q, const void* Kc, const void* Vc, int B, int h, int cap, int pos, float scale,
+                        const int32_t* head_idx, const int32_t* head_count, int kh_max, float* part, unsigned* ctr,
+                        float* H, int* status, cudaStream_t st) {
+  const int S = (sizeof(KT) * DH * 64 * 2 <= 32768) ? attn_split_len(B, kh_max, pos) : 32;
+  const int nsplit = (pos + 1 + S - 1) / S;
+  dim3 grid(nsplit, kh_max, B);
+  const KT* K = static_cast<const KT*>(Kc);
+  const KT* V = static_cast<const KT*>(Vc);
+  if constexpr (sizeof(KT) * DH * 64 * 2 <= 32768) {  // K and V tiles in static shared memory
+    if (S == 64)
+      return launch(attn_split_kernel<KT, DH, 64>, grid, ATTN_THREADS, 0, st, q, K, V, h, cap, pos, scale, head_idx,
+                    head_count, kh_max, nsplit, part, ctr, H, status);
+  }
+  return launch(attn_split_kernel<KT, DH, 32>, grid, ATTN_THREADS, 0, st, q, K, V, h, cap, pos, scale, head_idx,
+                head_count, kh_max, nsplit, part, ctr, H, status);
+}
+
+template <typename KT>
+cudaError_t run_attn(int dh, const float* q, const void* Kc, const void* Vc, int B, int h, int cap, int pos,
+                     float scale, const int32_t* head_idx, const int32_t* head_count, int kh_max, float* part,
+                     unsigned* ctr, float* H, int* status, cudaStream_t st) {
+  if (dh == 64)
+    return run_attn_dh<KT, 64>(q, Kc, Vc, B, h, cap, pos, scale, head_idx, head_count, kh_max, part, ctr, H, status, st);
+  return run_attn_dh<KT, 128>(q, Kc, Vc, B, h, cap, pos, scale, head_idx, head_count, kh_max, part, ctr, H, status, st);
+}
+
+
+constexpr int ATTN_CS = 8;  // CTAs per cluster (per selected head) in attn_out_kernel
+
+inline int attn_out_S(int pos) { return (pos + 1 + ATTN_CS - 1) / ATTN_CS; }
+inline size_t attn_out_smem(int S, int dh, int kvbytes) { return 2ull * S * dh * kvbytes + 4ull * S; }
+
+template <typename K, typename A>
+cudaError_t launch_fused(K kern, dim3 grid, size_t smem, cudaStream_t st, const A& a) {
+  cudaError_t e = allow_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  return launch(kern, grid, FUSED_THREADS, smem, st, a);
+}
+
+template <typename T, int NB>
+cudaError_t run_attn_in_nb(const AttnInArgs& a, cudaStream_t st) {
+  const int rpw = rpw_for(a.d, WT<T>::E);
+  const int slots = a.kh_max * 3 * a.dh, per = FUSED_WARPS * rpw;
+  const dim3 grid(slots > 0 ? (slots + per - 1) / per : 1);
+  const size_t smem = 4ull * a.nb * a.d;
+  switch (rpw) {
+    case 1: return launch_fused(attn_in_kernel<T, NB, 1, 8>, grid, smem, st, a);
+    case 2: return launch_fused(attn_in_kernel<T, NB, 2, 4>, grid, smem, st, a);
+    case 4: return launch_fused(attn_in_kernel<T, NB, 4, 2>, grid, smem, st, a);
+    default: return launch_fused(attn_in_kernel<T, NB, 8, 1>, grid, smem, st, a);
+  }
+}
+
+template <typename T>
+cudaError_t run_attn_in(const AttnInArgs& a, cudaStream_t st) {
+  switch (nb_bucket(a.nb)) {
+    case 1: return run_attn_in_nb<T, 1>(a, st);
+    case 2: return run_attn_in_nb<T, 2>(a, st);
+    case 4: return run_attn_in_nb<T, 4>(a, st);
+    case 8: return run_attn_in_nb<T, 8>(a, st);
+    default: return run_attn_in_nb<T, 16>(a, st);
+  }
+}
+
+template <typename KT, int DH, int NB>
+cudaError_t run_attn_out_nb(const AttnOutArgs& a, cudaStream_t st) {
+  const size_t smem = attn_out_smem(a.S, DH, sizeof(KT));
+  auto kern = attn_out_kernel<KT, DH, ATTN_CS, NB>;
+  cudaError_t e = allow_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  return launch_cluster(kern, dim3(ATTN_CS, a.kh_max > 0 ? a.kh_max : 1), FUSED_THREADS, smem, st, ATTN_CS, a);
+}
+
+template <typename KT, int DH>
+cudaError_t run_attn_out_dh(const AttnOutArgs& a, cudaStream_t st) {
+  switch (nb_bucket(a.nb)) {
+    case 1: return run_attn_out_nb<KT, DH, 1>(a, st);
+    case 2: return run_attn_out_nb<KT, DH, 2>(a, st);
+    case 4: return run_attn_out_nb<KT, DH, 4>(a, st);
+    case 8: return run_attn_out_nb<KT, DH, 8>(a, st);
+    default: return run_attn_out_nb<KT, DH, 16>(a, st);
+  }
+}
+
+template <typename KT>
+cudaError_t run_attn_out(const AttnOutArgs& a, cudaStream_t st) {
+  return a.dh == 64 ? run_attn_out_dh<KT, 64>(a, st) : run_attn_out_dh<KT, 128>(a, st);
+}
+
+inline int mlp_block_grid(int k_max) {
+  const int g = (k_max + 7) / 8;
+  return g < 1 ? 1 : (g > sm_count() ? sm_count() : g);
+}
+
+template <typename T, int NB>
+cudaError_t run_mlp_block_nb(const MlpBlockArgs& a, cudaStream_t st) {
+  const int rpw = rpw_for(a.d, WT<T>::E);
+  const dim3 grid(a.G);
+  const size_t smem = 4ull * a.nb * a.d;
+  switch (rpw) {
+    case 1: return launch_fused(mlp_block_kernel<T, NB, 1, 8>, grid, smem, st, a);
+    case 2: return launch_fused(mlp_block_kernel<T, NB, 2, 4>, grid, smem, st, a);
+    case 4: return launch_fused(mlp_block_kernel<T, NB, 4, 2>, grid, smem, st, a);
+    default: return launch_fused(mlp_block_kernel<T, NB, 8, 1>, grid, smem, st, a);
+  }
+}
+
+template <typename T>
+cudaError_t run_mlp_block(const MlpBlockArgs& a, cudaStream_t st) {
+  switch (nb_bucket(a.nb)) {
+    case 1: return run_mlp_block_nb<T, 1>(a, st);
+    case 2: return run_mlp_block_nb<T, 2>(a, st);
+    case 4: return run_mlp_block_nb<T, 4>(a, st);
+    case 8: return run_mlp_block_nb<T, 8>(a, st);
+    default: return run_mlp_block_nb<T, 16>(a, st);
+  }
+}
+
+template <typename T, int NB>
+cudaError_t run_predict_a_nb(const PredictAArgs& a, cudaStream_t st) {
+  const int rows = (a.PA ? a.h : 0) + (a.At ? a.r : 0);
+  const int rpw = rpw_for(a.d, WT<T>::E), per = FUSED_WARPS * rpw;
+  const dim3 grid(rows > 0 ? (rows + per - 1) / per : 1);
+  switch (rpw) {
+    case 1: return launch(predict_a_kernel<T, NB, 1, 8>, grid, FUSED_THREADS, 0, st, a);
+    case 2: return launch(predict_a_kernel<T, NB, 2, 4>, grid, FUSED_THREADS, 0, st, a);
+    case 4: return launch(predict_a_kernel<T, NB, 4, 2>, grid, FUSED_THREADS, 0, st, a);
+    default: return launch(predict_a_kernel<T, NB, 8, 1>, grid, FUSED_THREADS, 0, st, a);
+  }
+}
+
+template <typename T>
+cudaError_t run_predict_a(const PredictAArgs& a, cudaStream_t st) {
+  switch (nb_bucket(a.nb)) {
+    case 1: return run_predict_a_nb<T, 1>(a, st);
+    case 2: return run_predict_a_nb<T, 2>(a, st);
+    case 4: return run_predict_a_nb<T, 4>(a, st);
+    case 8: return run_predict_a_nb<T, 8>(a, st);
+    default: return run_predict_a_nb<T, 16>(a, st);
+  }
+}
+
+template <typename T, int NB>
+cudaError_t run_predict_b_nb(const PredictBArgs& a, cudaStream_t st) {
+  const int rpw = rpw_for(a.r, WT<T>::E), per = FUSED_WARPS * rpw;
+  const dim3 grid((a.N + per - 1) / per);
+  switch (rpw) {
+    case 1: return launch(predict_b_kernel<T, NB, 1, 8>, grid, FUSED_THREADS, 0, st, a);
+    case 2: return launch(predict_b_kernel<T, NB, 2, 4>, grid, FUSED_THREADS, 0, st, a);
+    case 4: return launch(predict_b_kernel<T, NB, 4, 2>, grid, FUSED_THREADS, 0, st, a);
+    default: return launch(predict_b_kernel<T, NB, 8, 1>, grid, FUSED_THREADS, 0, st, a);
+  }
+}
+
+template <typename T>
+cudaError_t run_predict_b(const PredictBArgs& a, cudaStream_t st) {
+  switch (nb_bucket(a.nb)) {
+    case 1: return run_predict_b_nb<T, 1>(a, st);
+    case 2: return run_predict_b_nb<T, 2>(a, st);
+    case 4: return run_predict_b_nb<T, 4>(a, st);
+    case 8: return run_predict_b_nb<T, 8>(a, st);
+    default: return run_predict_b_nb<T, 16>(a, st);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Column-owner kernels (dv_colowner.cuh) for batch 1-2
+// ---------------------------------------------------------------------------
+
+inline int co_nv(int d, int E) { return (d + CO_THREADS * E - 1) / (CO_THREADS * E); }
+// Rows per group: 8 or more 16-byte loads in flight per thread. The MLP
+// kernel also holds the W2 rows and its output slice, so it keeps fewer.
+inline int co_r(int nv) { return nv == 1 ? 8 : nv == 2 ? 4 : nv == 3 ? 3 : 4; }
+inline int co_r_mlp(int nv) { return nv == 1 ? 8 : nv == 2 ? 4 : nv == 3 ? 3 : 2; }
+inline bool co_ok(int nb, int d, int E) { return nb <= 2 && co_nv(d, E) <= 6; }
+inline int co_grid(long long groups) {
+  const long long cap = 2ll * sm_count();
+  return (int)(groups < 1 ? 1 : (groups > cap ? cap : groups));
+}
+
+#define DV_CO_SWITCH(KERN, NB, grid, st, a)                                   \
+  switch (nv) {                                                              \
+    case 1: return launch(KERN<T, NB, 1, 8>, grid, CO_THREADS, 0, st, a);    \
+    case 2: return launch(KERN<T, NB, 2, 4>, grid, CO_THREADS, 0, st, a);    \
+    case 3: return launch(KERN<T, NB, 3, 3>, grid, CO_THREADS, 0, st, a);    \
+    case 4: return launch(KERN<T, NB, 4, 4>, grid, CO_THREADS, 0, st, a);    \
+    case 5: return launch(KERN<T, NB, 5, 4>, grid, CO_THREADS, 0, st, a);    \
+    default: return launch(KERN<T, NB, 6, 4>, grid, CO_THREADS, 0, st, a);   \
+  }
+#define DV_CO_SWITCH_MLP(KERN, NB, grid, st, a)                               \
+  switch (nv) {                                                              \
+    case 1: return launch(KERN<T, NB, 1, 8>, grid, CO_THREADS, 0, st, a);    \
+    case 2: return launch(KERN<T, NB, 2, 4>, grid, CO_THREADS, 0, st, a);    \
+    case 3: return launch(KERN<T, NB, 3, 3>, grid, CO_THREADS, 0, st, a);    \
+    case 4: return launch(KERN<T, NB, 4, 2>, grid, CO_THREADS, 0, st, a);    \
+    case 5: return launch(KERN<T, NB, 5, 2>, grid, CO_THREADS, 0, st, a);    \
+    default: return launch(KERN<T, NB, 6, 2>, grid, CO_THREADS, 0, st, a);   \
+  }
+
+template <typename T, int NB>
+cudaError_t run_attn_in_co_nb(const AttnInArgs& a, cudaStream_t st) {
+  const int nv = co_nv(a.d, WT<T>::E), R = co_r(nv);
+  const dim3 grid(co_grid(((long long)a.kh_max * 3 * a.dh + R - 1) / R));
+  DV_CO_SWITCH(attn_in_co_kernel, NB, grid, st, a)
+}
+
+template <typename T, int NB>
+cudaError_t run_mlp_block_co_nb(MlpBlockArgs a, cudaStream_t st) {
+  const int nv = co_nv(a.d, WT<T>::E), R = co_r_mlp(nv);
+  a.G = co_grid(((long long)a.k_max + R - 1) / R);
+  const dim3 grid(a.G);
+  DV_CO_SWITCH_MLP(mlp_block_co_kernel, NB, grid, st, a)
+}
+
+template <typename T, int NB>
+cudaError_t run_predict_a_co_nb(const PredictAArgs& a, cudaStream_t st) {
+  const int nv = co_nv(a.d, WT<T>::E), R = co_r(nv);
+  const int rows = (a.PA ? a.h : 0) + (a.At ? a.r : 0);
+  const dim3 grid(co_grid((rows + R - 1) / R));
+  DV_CO_SWITCH(predict_a_co_kernel, NB, grid, st, a)
+}
+#undef DV_CO_SWITCH
+#undef DV_CO_SWITCH_MLP
+
+template <typename T>
+cudaError_t run_attn_in_any(const AttnInArgs& a, cudaStream_t st) {
+  if (co_ok(a.nb, a.d, WT<T>::E))
+    return a.nb == 1 ? run_attn_in_co_nb<T, 1>(a, st) : run_attn_in_co_nb<T, 2>(a, st);
+  return run_attn_in<T>(a, st);
+}
+
+template <typename T>
+cudaError_t run_mlp_block_any(const MlpBlockArgs& a, cudaStream_t st) {
+  if (co_ok(a.nb, a.d, WT<T>::E))
+    return a.nb == 1 ? run_mlp_block_co_nb<T, 1>(a, st) : run_mlp_block_co_nb<T, 2>(a, st);
+  return run_mlp_block<T>(a, st);
+}
+
+template <typename T>
+cudaError_t run_predict_a_any(const PredictAArgs& a, cudaStream_t st) {
+  if (co_ok(a.nb, a.d, WT<T>::E))
+    return a.nb == 1 ? run_predict_a_co_nb<T, 1>(a, st) : run_predict_a_co_nb<T, 2>(a, st);
+  return run_predict_a<T>(a, st);
+}
+
+// ---------------------------------------------------------------------------
+// Entry points of the per-family translation units: element-type dispatch.
+// ---------------------------------------------------------------------------
+
+cudaError_t run_mlp_up_dt(dv_dtype dt, const void* W1t, int d, int N, const float* y, int nb, const float* b1,
+                          const int32_t* idx, const int32_t* count, int k_max, int32_t* seg_idx, float* seg_a,
+                          int32_t* seg_cnt, int* status, int nseg, cudaStream_t st);
+cudaError_t run_axpy_dt(dv_dtype dt, const void* W, int d, int nrows_w, RowsHeads src, const float* bias, float* out,
+                        int nb, int k_max, size_t smem, int* status, cudaStream_t st);
+cudaError_t run_axpy_dt(dv_dtype dt, const void* W, int d, int nrows_w, RowsMlp src, const float* bias, float* out,
+                        int nb, int k_max, size_t smem, int* status, cudaStream_t st);
+cudaError_t run_qkv_dt(dv_dtype dt, const void* Wqkv, int d, int h, int dh, const float* y, int nb, const float* bqkv,
+                       const int32_t* head_idx, const int32_t* head_count, int kh_max, float* q, void* Kc, void* Vc,
+                       int cap, int pos, int* status, cudaStream_t st);
+cudaError_t run_attn_dt(dv_dtype kvdt, int dh, const float* q, const void* Kc, const void* Vc, int B, int h, int cap,
+                        int pos, float scale, const int32_t* head_idx, const int32_t* head_count, int kh_max,
+                        float* part, unsigned* ctr, float* H, int* status, cudaStream_t st);
+cudaError_t run_attn_in_any_dt(dv_dtype wdt, const AttnInArgs& a, cudaStream_t st);
+cudaError_t run_attn_out_dt(dv_dtype kvdt, const AttnOutArgs& a, cudaStream_t st);
+cudaError_t run_mlp_block_any_dt(dv_dtype wdt, const MlpBlockArgs& a, cudaStream_t st);
+cudaError_t run_predict_a_any_dt(dv_dtype wdt, const PredictAArgs& a, cudaStream_t st);
+cudaError_t run_predict_b_dt(dv_dtype wdt, const PredictBArgs& a, cudaStream_t st);
+
+}  // namespace dv
