@@ -193,7 +193,7 @@ bool fused_ok(const dv_dims& D, dv_dtype wdt) {
   const int wb = wbytes_of(wdt), E = 16 / wb;
   if (D.d % (ATTN_CS * E) != 0) return false;
   if ((size_t)D.B * D.d * 4 > 160 * 1024) return false;
-  if (attn_out_smem(attn_out_S(D.cap - 1), D.dh, wb) > 190 * 1024) return false;
+  if (attn_out_smem(attn_out_S(D.cap - 1), D.dh, wb, D.B) > ATTN_SMEM_MAX) return false;
   if (D.N > SEL_SMEM_KEYS || D.h > HSEL_MAX) return false;
   return true;
 }

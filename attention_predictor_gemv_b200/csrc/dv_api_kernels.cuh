@@ -264,9 +264,13 @@ __global__ void __launch_bounds__(SEL_THREADS) select_finish_kernel(SelectFinish
         __syncthreads();
         const int nc = use_cand ? (int)s_ncand : n;
         const uint32_t* src = use_cand ? s_cand : s_keys;
-        for (int i = tid; i < nc; i += SEL_THREADS) {
-          const uint32_t key = src[i];
-          if ((key & mask) == prefix) atomicAdd(&s_h[(key >> shift) & dmask], 1u);
+        for (int i0 = 0; i0 < nc; i0 += SEL_THREADS) {
+          const int i = i0 + tid;
+          const uint32_t key = i < nc ? src[i] : 0u;
+          const bool in = i < nc && (key & mask) == prefix;
+          const unsigned bin = in ? (key >> shift) & dmask : 0xffffffffu;
+          const unsigned peers = __match_any_sync(0xffffffffu, bin);
+          if (in && (__ffs(peers) - 1) == lane) atomicAdd(&s_h[bin], (unsigned)__popc(peers));
         }
         __syncthreads();
       }
@@ -289,10 +293,18 @@ __global__ void __launch_bounds__(SEL_THREADS) select_finish_kernel(SelectFinish
       if (pass == 0) {  // the keys of the boundary bin
         if (tid == 0) s_ncand = 0u;
         __syncthreads();
-        for (int i = tid; i < n; i += SEL_THREADS) {
-          const uint32_t key = s_keys[i];
-          if ((key & mask) == prefix) {
-            const unsigned at = atomicAdd(&s_ncand, 1u);
+        // one shared-memory atomic per warp and step (a per-key atomic on the
+        // one counter serialises the hundreds of keys in the boundary bin)
+        for (int i0 = 0; i0 < n; i0 += SEL_THREADS) {
+          const int i = i0 + tid;
+          const uint32_t key = i < n ? s_keys[i] : 0u;
+          const bool c = i < n && (key & mask) == prefix;
+          const unsigned bal = __ballot_sync(0xffffffffu, c);
+          unsigned base = 0u;
+          if (lane == 0 && bal) base = atomicAdd(&s_ncand, (unsigned)__popc(bal));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          if (c) {
+            const unsigned at = base + __popc(bal & ((1u << lane) - 1u));
             if (at < SF_CAND) s_cand[at] = key;
           }
         }

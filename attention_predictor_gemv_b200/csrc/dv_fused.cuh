@@ -478,13 +478,18 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_in_kernel(AttnInArgs a) {
 
 // ----------------------------------------------------------------------------
 // attn_out_kernel: for selected head slot p (grid y) a cluster of CS CTAs
-// splits the keys 0..pos: each CTA stages its K/V range in shared memory
-// (slots below pos before griddep_wait: they do not depend on attn_in), forms
-// the partial (m, l, acc) of the max-subtracted softmax, and after a cluster
-// barrier every CTA combines the CS partials through distributed shared
-// memory into H (eq. (2): D_i^{-1} exp(.) X W_i^V). CTA c then multiplies H
-// by its column slice of W_i^O and adds the result to t1. The cluster of
-// slot 0 also moves the residual: t1 += x (+ bO) on its slices, then x = 0.
+// splits the keys 0..pos: CTA c stages its K/V range in shared memory (slots
+// below pos before griddep_wait: they do not depend on attn_in) and forms
+// the partial (m, l, acc) of the max-subtracted softmax (eq. (2):
+// D_i^{-1} exp(.) X W_i^V), each warp over its own keys with a running max,
+// then merged across the CTA's warps. Every CTA stores its partial into the
+// shared memory of all CS CTAs of the cluster (distributed shared memory), so
+// after one cluster barrier each CTA combines the CS partials into H locally.
+// CTA c then multiplies H by its column slice of W_i^O and adds the result to
+// t1. With WV > 0 the slice (WV 16-byte vectors per thread) is loaded into
+// registers before griddep_wait; with WV = 0 it is streamed afterwards. The
+// cluster of slot 0 also moves the residual: t1 += x (+ bO) on its slices,
+// then x = 0.
 // ----------------------------------------------------------------------------
 struct AttnOutArgs {
   const float* q;
@@ -502,29 +507,52 @@ struct AttnOutArgs {
   int* status;
 };
 
-template <typename KT, int DH, int CS, int NB>
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
+// Merges the softmax partial (mo, lo, ao) into (m, l, acc).
+template <int E>
+__device__ __forceinline__ void softmax_merge(float& m, float& l, float (&acc)[E], float mo, float lo,
+                                              const float (&ao)[E]) {
+  const float M = fmaxf(m, mo);
+  if (M == -INFINITY) return;  // both empty
+  const float c1 = __expf(m - M), c2 = __expf(mo - M);
+  l = l * c1 + lo * c2;
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = acc[e] * c1 + ao[e] * c2;
+  m = M;
+}
+
+template <typename KT, int DH, int CS, int NB, int WV>
 __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) {
   constexpr int E = WT<KT>::E;
-  constexpr int G = DH / E;                 // lanes per key row
-  constexpr int KPP = FUSED_THREADS / G;    // keys per pass
+  constexpr int G = DH / E;    // lanes per key row
+  constexpr int KPW = 32 / G;  // keys per warp step
+  constexpr int PW = DH + 2;   // partial: m, l, acc[DH]
+  constexpr int RG = WV > 0 ? DH / WV : 1;  // W^O row groups (register path)
   extern __shared__ __align__(16) unsigned char s_dyn[];
-  KT* sK = reinterpret_cast<KT*>(s_dyn);                       // [S][DH]
-  KT* sV = sK + (size_t)a.S * DH;                              // [S][DH]
-  float* sE = reinterpret_cast<float*>(sV + (size_t)a.S * DH); // [S]
-  __shared__ __align__(16) float s_part[NB][DH + 2];  // this CTA's partial (m, l, acc)
+  KT* sK = reinterpret_cast<KT*>(s_dyn);                          // [S][DH]
+  KT* sV = sK + (size_t)a.S * DH;                                 // [S][DH]
+  float* s_all = reinterpret_cast<float*>(sV + (size_t)a.S * DH);  // [nb][CS][PW]
+  __shared__ __align__(16) float s_w[FUSED_WARPS][PW];
   __shared__ __align__(16) float s_H[NB][DH];
-  __shared__ float s_red[KPP * DH > FUSED_THREADS * E ? KPP * DH : FUSED_THREADS * E];
-  __shared__ float red[FUSED_WARPS];
+  __shared__ float s_red[WV > 0 ? 1 : FUSED_THREADS * E];
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = (int)cluster.block_rank();
   const int p = blockIdx.y;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const KT* Kc = static_cast<const KT*>(a.Kc);
   const KT* Vc = static_cast<const KT*>(a.Vc);
+  const KT* WO = static_cast<const KT*>(a.WOt);
   const int nkeys = a.pos + 1;
   const int t0 = crank * a.S;
   const int nk = max(0, min(a.S, nkeys - t0));
+  const int cols = a.d / CS;  // d % (8 CS) == 0 is checked on the host
+  const int c_lo = crank * cols;
   griddep_launch();
+  cluster_arrive_relaxed();  // waited on before the first store into another CTA
 
   int hc = 0, head = -1;
   auto read_head = [&]() {
@@ -549,46 +577,66 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
     }
   };
   const bool pos_in_chunk = a.pos >= t0 && a.pos < t0 + nk;
-  // this CTA's column slice of W_head^O: DH rows of d/CS columns
+  // register path: thread (cgi, rg) holds rows rg + i RG of column vector cgi
+  const int cgi = tid / RG, rg = tid % RG;
+  uint4 wo[WV > 0 ? WV : 1];
+  auto load_wo = [&]() {
+    if constexpr (WV > 0) {
+      const KT* Wh = WO + (size_t)head * DH * a.d + c_lo + cgi * E;
+#pragma unroll
+      for (int i = 0; i < WV; ++i) wo[i] = ld_stream(Wh + (size_t)(rg + i * RG) * a.d);
+    }
+  };
   auto prefetch_wo = [&]() {
-    const int cols = a.d / CS;
-    const char* base = static_cast<const char*>(a.WOt) +
-                       ((size_t)head * DH * a.d + (size_t)crank * cols) * sizeof(KT);
-    for (int i = tid; i < DH; i += FUSED_THREADS) prefetch_l2(base + (size_t)i * a.d * sizeof(KT), cols * sizeof(KT));
+    if constexpr (WV == 0) {
+      const char* base = reinterpret_cast<const char*>(WO + (size_t)head * DH * a.d + c_lo);
+      for (int i = tid; i < DH; i += FUSED_THREADS) prefetch_l2(base + (size_t)i * a.d * sizeof(KT), cols * sizeof(KT));
+    }
   };
   if (a.sets_ready) {
     read_head();
     if (head >= 0) {
       stage(0, true, false);
+      load_wo();
       prefetch_wo();
     }
   }
   griddep_wait();
   if (!a.sets_ready) {
     read_head();
-    if (head >= 0) stage(0, true, false);
+    if (head >= 0) {
+      stage(0, true, false);
+      load_wo();
+    }
   }
   const bool active = head >= 0;
+  cluster_wait();  // every CTA of the cluster runs: its shared memory may be written
   // ---- partial attention over this CTA's keys, per batch row ----
   if (active) {
+    const int g = lane % G, kq = lane / G;
+    const int KW = (nk + FUSED_WARPS - 1) / FUSED_WARPS;
+    const int kw0 = min(nk, warp * KW), kw1 = min(nk, kw0 + KW);
     for (int b = 0; b < a.nb; ++b) {
       if (b > 0) {
-        __syncthreads();  // previous row's tiles are consumed
+        __syncthreads();  // previous row's tiles and s_w are consumed
         stage(b, false, false);
       } else if (pos_in_chunk) {
         stage(0, false, true);  // slot pos, written by attn_in
       }
-      const int g = tid % G, j = tid / G;
       float qv[E];
       const float* qp = a.q + ((size_t)b * a.kh_max + p) * DH + g * E;
 #pragma unroll
       for (int e = 0; e < E; ++e) qv[e] = __ldcg(qp + e) * a.scale;
       cp_async_wait_all();
       __syncthreads();
-      for (int tb = 0; tb < nk; tb += KPP) {
-        const int t = tb + j;
+      float m = -INFINITY, l = 0.f, acc[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = 0.f;
+      for (int tb = kw0; tb < kw1; tb += KPW) {  // warp-uniform trip count
+        const int t = tb + kq;
+        const bool ok = t < kw1;
         float dot = 0.f;
-        if (t < nk) {
+        if (ok) {
           float kf[E];
           WT<KT>::unpack(*reinterpret_cast<const uint4*>(sK + t * DH + g * E), kf);
 #pragma unroll
@@ -596,156 +644,202 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
         }
 #pragma unroll
         for (int o = G / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-        if (g == 0 && t < nk) sE[t] = dot;
+        if (ok) {
+          float vf[E];
+          WT<KT>::unpack(*reinterpret_cast<const uint4*>(sV + t * DH + g * E), vf);
+          const float mn = fmaxf(m, dot);
+          const float c = __expf(m - mn), pe = __expf(dot - mn);
+          l = l * c + pe;
+#pragma unroll
+          for (int e = 0; e < E; ++e) acc[e] = fmaf(pe, vf[e], acc[e] * c);
+          m = mn;
+        }
+      }
+      // merge the warp's KPW key groups (lanes g, g + G, ... hold the same dims)
+#pragma unroll
+      for (int o = G; o < 32; o <<= 1) {
+        const float mo = __shfl_xor_sync(0xffffffffu, m, o), lo = __shfl_xor_sync(0xffffffffu, l, o);
+        float ao[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) ao[e] = __shfl_xor_sync(0xffffffffu, acc[e], o);
+        softmax_merge<E>(m, l, acc, mo, lo, ao);
+      }
+      if (kq == 0) {
+        if (g == 0) {
+          s_w[warp][0] = m;
+          s_w[warp][1] = l;
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) s_w[warp][2 + g * E + e] = acc[e];
       }
       __syncthreads();
-      float m = -INFINITY;
-      for (int t = tid; t < nk; t += FUSED_THREADS) m = fmaxf(m, sE[t]);
-      m = block_max<FUSED_THREADS>(m, red);
-      float l = 0.f;
-      for (int t = tid; t < nk; t += FUSED_THREADS) {
-        const float pe = __expf(sE[t] - m);
-        sE[t] = pe;
-        l += pe;
-      }
-      l = block_sum<FUSED_THREADS>(l, red);
-      float acc[E];
+      // this CTA's partial, stored into every CTA of the cluster
+      for (int c = tid; c < PW; c += FUSED_THREADS) {
+        float M = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < E; ++e) acc[e] = 0.f;
-      for (int t = j; t < nk; t += KPP) {
-        float vf[E];
-        WT<KT>::unpack(*reinterpret_cast<const uint4*>(sV + t * DH + g * E), vf);
-        const float pe = sE[t];
+        for (int w = 0; w < FUSED_WARPS; ++w) M = fmaxf(M, s_w[w][0]);
+        float v = 0.f;
+        if (M != -INFINITY) {
+          if (c == 0) {
+            v = M;
+          } else {
 #pragma unroll
-        for (int e = 0; e < E; ++e) acc[e] = fmaf(pe, vf[e], acc[e]);
-      }
+            for (int w = 0; w < FUSED_WARPS; ++w) {
+              const float mw = s_w[w][0];
+              v += (mw == -INFINITY) ? 0.f : __expf(mw - M) * s_w[w][c];
+            }
+          }
+        } else {
+          v = (c == 0) ? -INFINITY : 0.f;
+        }
+        const int off = (b * CS + crank) * PW + c;
 #pragma unroll
-      for (int e = 0; e < E; ++e) s_red[j * DH + g * E + e] = acc[e];
-      __syncthreads();
-      for (int c = tid; c < DH; c += FUSED_THREADS) {
-        float s = 0.f;
-#pragma unroll 4
-        for (int jj = 0; jj < KPP; ++jj) s += s_red[jj * DH + c];
-        s_part[b][2 + c] = s;
-      }
-      if (tid == 0) {
-        s_part[b][0] = nk > 0 ? m : -INFINITY;
-        s_part[b][1] = l;
+        for (int r = 0; r < CS; ++r) cluster.map_shared_rank(s_all, r)[off] = v;
       }
     }
   }
-  cluster.sync();  // every CTA's partial is complete
+  cluster.sync();  // every partial has reached every CTA
   if (active) {
-    // ---- combine the CS partials of each batch row (distributed smem) ----
-    for (int b = 0; b < a.nb; ++b) {
+    // ---- combine the CS partials of each batch row (local shared memory) ----
+    for (int i = tid; i < a.nb * DH; i += FUSED_THREADS) {
+      const int b = i / DH, c = i % DH;
+      const float* pb = s_all + (size_t)b * CS * PW;
       float M = -INFINITY;
 #pragma unroll
-      for (int r = 0; r < CS; ++r) {
-        const float* rp = cluster.map_shared_rank(&s_part[0][0], r);
-        M = fmaxf(M, rp[b * (DH + 2)]);
-      }
-      float den = 0.f;
+      for (int r = 0; r < CS; ++r) M = fmaxf(M, pb[r * PW]);
+      float den = 0.f, num = 0.f;
 #pragma unroll
       for (int r = 0; r < CS; ++r) {
-        const float* rp = cluster.map_shared_rank(&s_part[0][0], r);
-        const float mr = rp[b * (DH + 2)];
-        den += (mr == -INFINITY) ? 0.f : __expf(mr - M) * rp[b * (DH + 2) + 1];
+        const float mr = pb[r * PW];
+        const float f = (mr == -INFINITY) ? 0.f : __expf(mr - M);
+        den += f * pb[r * PW + 1];
+        num += f * pb[r * PW + 2 + c];
       }
-      for (int c = tid; c < DH; c += FUSED_THREADS) {
-        float num = 0.f;
-#pragma unroll
-        for (int r = 0; r < CS; ++r) {
-          const float* rp = cluster.map_shared_rank(&s_part[0][0], r);
-          const float mr = rp[b * (DH + 2)];
-          num += (mr == -INFINITY) ? 0.f : __expf(mr - M) * rp[b * (DH + 2) + 2 + c];
-        }
-        s_H[b][c] = num / den;
-      }
+      s_H[b][c] = num / den;
     }
   }
-  cluster.sync();  // remote partials are no longer read; s_H complete
-  // ---- W^O slice: columns [c_lo, c_hi) of this CTA ----
-  const int cols = a.d / CS;  // d % (8 CS) == 0 is checked on the host
-  const int c_lo = crank * cols;
-  const int ncg = cols / E;   // column groups of E columns
+  __syncthreads();
   const bool residual = (p == 0);
   if (!active && !residual) return;
-  const KT* WO = static_cast<const KT*>(a.WOt);
-  for (int cg0 = 0; cg0 < ncg; cg0 += FUSED_THREADS) {
-    const int ngrp = min(FUSED_THREADS, ncg - cg0);
-    const int nrg = max(1, FUSED_THREADS / ngrp);  // row groups
-    const int cgi = tid % ngrp, rg = tid / ngrp;
-    const bool thr_ok = rg < nrg && tid < ngrp * nrg;
-    const int c = c_lo + (cg0 + cgi) * E;
-    float acc[NB][E];
+  // residual (slot 0's cluster): o += x + bO at columns c..c+E-1, then x = 0
+  auto add_residual = [&](float (&o)[E], int b, int c) {
+    float* xr = a.x + (size_t)b * a.d + c;
+#pragma unroll
+    for (int e4 = 0; e4 < E / 4; ++e4) {
+      const float4 xv = __ldcg(reinterpret_cast<const float4*>(xr) + e4);
+      float4 bb = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (a.bO) bb = __ldg(reinterpret_cast<const float4*>(a.bO + c) + e4);
+      o[4 * e4 + 0] += xv.x + bb.x;
+      o[4 * e4 + 1] += xv.y + bb.y;
+      o[4 * e4 + 2] += xv.z + bb.z;
+      o[4 * e4 + 3] += xv.w + bb.w;
+      reinterpret_cast<float4*>(xr)[e4] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  if constexpr (WV > 0) {
+    // ---- W^O slice from registers; row groups reduced across RG lanes ----
+    float o[NB][E];
 #pragma unroll
     for (int b = 0; b < NB; ++b)
 #pragma unroll
-      for (int e = 0; e < E; ++e) acc[b][e] = 0.f;
-    if (active && thr_ok) {
-      constexpr int WO_U = 16;  // rows of W^O in flight per thread
-      const KT* Wh = WO + (size_t)head * DH * a.d + c;
-      for (int i0 = rg; i0 < DH; i0 += nrg * WO_U) {
-        uint4 w[WO_U];
+      for (int e = 0; e < E; ++e) o[b][e] = 0.f;
+    if (active) {
 #pragma unroll
-        for (int u = 0; u < WO_U; ++u) {
-          const int i = i0 + u * nrg;
-          w[u] = i < DH ? ld_stream(Wh + (size_t)i * a.d) : make_uint4(0u, 0u, 0u, 0u);
+      for (int i = 0; i < WV; ++i) {
+        float wf[E];
+        WT<KT>::unpack(wo[i], wf);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          const float hv = b < a.nb ? s_H[b][rg + i * RG] : 0.f;
+#pragma unroll
+          for (int e = 0; e < E; ++e) o[b][e] = fmaf(hv, wf[e], o[b][e]);
         }
+      }
+    }
 #pragma unroll
-        for (int u = 0; u < WO_U; ++u) {
-          const int i = i0 + u * nrg;
-          if (i < DH) {
-            float wf[E];
-            WT<KT>::unpack(w[u], wf);
+    for (int sh = RG / 2; sh > 0; sh >>= 1)
 #pragma unroll
-            for (int b = 0; b < NB; ++b) {
-              if (b < a.nb) {
-                const float hv = s_H[b][i];
+      for (int b = 0; b < NB; ++b)
 #pragma unroll
-                for (int e = 0; e < E; ++e) acc[b][e] = fmaf(hv, wf[e], acc[b][e]);
+        for (int e = 0; e < E; ++e) o[b][e] += __shfl_xor_sync(0xffffffffu, o[b][e], sh);
+    if (rg == 0) {
+      const int c = c_lo + cgi * E;
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        if (b >= a.nb) break;
+        if (residual) add_residual(o[b], b, c);
+#pragma unroll
+        for (int e4 = 0; e4 < E / 4; ++e4)
+          red_add4(a.t1 + (size_t)b * a.d + c + 4 * e4,
+                   make_float4(o[b][4 * e4], o[b][4 * e4 + 1], o[b][4 * e4 + 2], o[b][4 * e4 + 3]));
+      }
+    }
+  } else {
+    // ---- W^O slice streamed: columns [c_lo, c_lo + cols) ----
+    const int ncg = cols / E;
+    for (int cg0 = 0; cg0 < ncg; cg0 += FUSED_THREADS) {
+      const int ngrp = min(FUSED_THREADS, ncg - cg0);
+      const int nrg = max(1, FUSED_THREADS / ngrp);  // row groups
+      const int cgj = tid % ngrp, rgj = tid / ngrp;
+      const bool thr_ok = rgj < nrg && tid < ngrp * nrg;
+      const int c = c_lo + (cg0 + cgj) * E;
+      float acc[NB][E];
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[b][e] = 0.f;
+      if (active && thr_ok) {
+        constexpr int WO_U = 16;  // rows of W^O in flight per thread
+        const KT* Wh = WO + (size_t)head * DH * a.d + c;
+        for (int i0 = rgj; i0 < DH; i0 += nrg * WO_U) {
+          uint4 w[WO_U];
+#pragma unroll
+          for (int u = 0; u < WO_U; ++u) {
+            const int i = i0 + u * nrg;
+            w[u] = i < DH ? ld_stream(Wh + (size_t)i * a.d) : make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+          for (int u = 0; u < WO_U; ++u) {
+            const int i = i0 + u * nrg;
+            if (i < DH) {
+              float wf[E];
+              WT<KT>::unpack(w[u], wf);
+#pragma unroll
+              for (int b = 0; b < NB; ++b) {
+                if (b < a.nb) {
+                  const float hv = s_H[b][i];
+#pragma unroll
+                  for (int e = 0; e < E; ++e) acc[b][e] = fmaf(hv, wf[e], acc[b][e]);
+                }
               }
             }
           }
         }
       }
-    }
-    // reduce the row groups, one batch row at a time
-    for (int b = 0; b < a.nb && b < NB; ++b) {
-      if (nrg > 1) {
-        __syncthreads();
-        if (thr_ok) {
+      // reduce the row groups, one batch row at a time
+      for (int b = 0; b < a.nb && b < NB; ++b) {
+        if (nrg > 1) {
+          __syncthreads();
+          if (thr_ok) {
 #pragma unroll
-          for (int e = 0; e < E; ++e) s_red[(rg * ngrp + cgi) * E + e] = acc[b][e];
-        }
-        __syncthreads();
-      }
-      if (rg == 0 && thr_ok) {
-        float o[E];
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          float sum = acc[b][e];
-          for (int r2 = 1; r2 < nrg; ++r2) sum += s_red[(r2 * ngrp + cgi) * E + e];
-          o[e] = sum;
-        }
-        if (residual) {
-          float* xr = a.x + (size_t)b * a.d + c;
-#pragma unroll
-          for (int e4 = 0; e4 < E / 4; ++e4) {
-            const float4 xv = __ldcg(reinterpret_cast<const float4*>(xr) + e4);
-            float4 bb = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (a.bO) bb = __ldg(reinterpret_cast<const float4*>(a.bO + c) + e4);
-            o[4 * e4 + 0] += xv.x + bb.x;
-            o[4 * e4 + 1] += xv.y + bb.y;
-            o[4 * e4 + 2] += xv.z + bb.z;
-            o[4 * e4 + 3] += xv.w + bb.w;
-            reinterpret_cast<float4*>(xr)[e4] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int e = 0; e < E; ++e) s_red[(rgj * ngrp + cgj) * E + e] = acc[b][e];
           }
+          __syncthreads();
         }
+        if (rgj == 0 && thr_ok) {
+          float o[E];
 #pragma unroll
-        for (int e4 = 0; e4 < E / 4; ++e4)
-          red_add4(a.t1 + (size_t)b * a.d + c + 4 * e4,
-                    make_float4(o[4 * e4], o[4 * e4 + 1], o[4 * e4 + 2], o[4 * e4 + 3]));
+          for (int e = 0; e < E; ++e) {
+            float sum = acc[b][e];
+            for (int r2 = 1; r2 < nrg; ++r2) sum += s_red[(r2 * ngrp + cgj) * E + e];
+            o[e] = sum;
+          }
+          if (residual) add_residual(o, b, c);
+#pragma unroll
+          for (int e4 = 0; e4 < E / 4; ++e4)
+            red_add4(a.t1 + (size_t)b * a.d + c + 4 * e4,
+                     make_float4(o[4 * e4], o[4 * e4 + 1], o[4 * e4 + 2], o[4 * e4 + 3]));
+        }
       }
     }
   }

@@ -1,10 +1,12 @@
-// Instantiates the launchers of attn_out (split attention + W^O).
+// Instantiates the launchers of attn_out (split attention + W^O), bf16.
 #include "dv_launchers.cuh"
 
 namespace dv {
 
 cudaError_t run_attn_out_dt(dv_dtype kvdt, const AttnOutArgs& a, cudaStream_t st) {
-  return kvdt == DV_BF16 ? run_attn_out<bf16>(a, st) : run_attn_out<float>(a, st);
+  return kvdt == DV_BF16 ? run_attn_out_bf16(a, st) : run_attn_out_f32(a, st);
 }
+
+cudaError_t run_attn_out_bf16(const AttnOutArgs& a, cudaStream_t st) { return run_attn_out<bf16>(a, st); }
 
 }  // namespace dv

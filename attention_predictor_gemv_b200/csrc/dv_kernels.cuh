@@ -317,9 +317,15 @@ __global__ void __launch_bounds__(SEL_THREADS)
       const unsigned dmask = pass == 2 ? 0x3ffu : 0x7ffu;
       for (int i = tid; i < SEL_BINS; i += SEL_THREADS) hist[i] = 0;
       __syncthreads();
-      for (int i = tid; i < n; i += SEL_THREADS) {
-        const uint32_t key = sel_key<KEYS_IN_SMEM>(s_keys, row, i);
-        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
+      // keys of a warp that share a bin add once (scores crowd into few
+      // top-digit bins, where per-key atomics would serialise)
+      for (int i0 = 0; i0 < n; i0 += SEL_THREADS) {
+        const int i = i0 + tid;
+        const uint32_t key = i < n ? sel_key<KEYS_IN_SMEM>(s_keys, row, i) : 0u;
+        const bool in = i < n && (key & mask) == prefix;
+        const unsigned bin = in ? (key >> shift) & dmask : 0xffffffffu;
+        const unsigned peers = __match_any_sync(0xffffffffu, bin);
+        if (in && (__ffs(peers) - 1) == lane) atomicAdd(&hist[bin], (unsigned)__popc(peers));
       }
       __syncthreads();
       // thread t owns bins 2047-2t and 2046-2t (descending); an exclusive scan

@@ -4,7 +4,7 @@
 #pragma once
 
 #include "../../include/dejavu.h"
-#include "dv_colowner.cuh"
+#include "dv_stream.cuh"
 #include "dv_launch.cuh"
 
 namespace dv {
@@ -172,7 +172,22 @@ cudaError_t run_attn(int dh, const float* q, const void* Kc, const void* Vc, int
 constexpr int ATTN_CS = 8;  // CTAs per cluster (per selected head) in attn_out_kernel
 
 inline int attn_out_S(int pos) { return (pos + 1 + ATTN_CS - 1) / ATTN_CS; }
-inline size_t attn_out_smem(int S, int dh, int kvbytes) { return 2ull * S * dh * kvbytes + 4ull * S; }
+// K/V tiles of S keys plus the cluster's partials (m, l, acc[dh]) of nb rows.
+inline size_t attn_out_smem(int S, int dh, int kvbytes, int nb) {
+  return 2ull * S * dh * kvbytes + 4ull * nb * ATTN_CS * (dh + 2);
+}
+constexpr size_t ATTN_SMEM_MAX = 200 * 1024;  // dynamic part; the static part stays below 24 KB
+
+// W^O vectors per thread when a CTA's W^O slice (dh rows of d / ATTN_CS
+// columns) fits in registers: dh / (256 / column vectors); 0 streams it.
+inline int attn_out_wv(int d, int dh, int E, int nb) {
+  const int ncg = d / ATTN_CS / E;
+  if (nb > 4 || ncg < 8 || ncg > 256 || 256 % ncg != 0) return 0;
+  const int rg = 256 / ncg;
+  if (dh % rg != 0) return 0;
+  const int wv = dh / rg;
+  return (wv == 8 || wv == 16) ? wv : 0;
+}
 
 template <typename K, typename A>
 cudaError_t launch_fused(K kern, dim3 grid, size_t smem, cudaStream_t st, const A& a) {
@@ -206,13 +221,25 @@ cudaError_t run_attn_in(const AttnInArgs& a, cudaStream_t st) {
   }
 }
 
-template <typename KT, int DH, int NB>
-cudaError_t run_attn_out_nb(const AttnOutArgs& a, cudaStream_t st) {
-  const size_t smem = attn_out_smem(a.S, DH, sizeof(KT));
-  auto kern = attn_out_kernel<KT, DH, ATTN_CS, NB>;
+template <typename KT, int DH, int NB, int WV>
+cudaError_t run_attn_out_nbw(const AttnOutArgs& a, cudaStream_t st) {
+  const size_t smem = attn_out_smem(a.S, DH, sizeof(KT), a.nb);
+  auto kern = attn_out_kernel<KT, DH, ATTN_CS, NB, WV>;
   cudaError_t e = allow_smem(kern, smem);
   if (e != cudaSuccess) return e;
   return launch_cluster(kern, dim3(ATTN_CS, a.kh_max > 0 ? a.kh_max : 1), FUSED_THREADS, smem, st, ATTN_CS, a);
+}
+
+template <typename KT, int DH, int NB>
+cudaError_t run_attn_out_nb(const AttnOutArgs& a, cudaStream_t st) {
+  if constexpr (NB <= 4) {
+    switch (attn_out_wv(a.d, DH, WT<KT>::E, a.nb)) {
+      case 8: return run_attn_out_nbw<KT, DH, NB, 8>(a, st);
+      case 16: return run_attn_out_nbw<KT, DH, NB, 16>(a, st);
+      default: break;
+    }
+  }
+  return run_attn_out_nbw<KT, DH, NB, 0>(a, st);
 }
 
 template <typename KT, int DH>
@@ -366,8 +393,68 @@ cudaError_t run_predict_a_co_nb(const PredictAArgs& a, cudaStream_t st) {
 #undef DV_CO_SWITCH
 #undef DV_CO_SWITCH_MLP
 
+// ---------------------------------------------------------------------------
+// Streaming kernels (dv_stream.cuh) for rows of 16 KB and more, batch 1-2
+// ---------------------------------------------------------------------------
+
+inline bool stream_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("DV_STREAM");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+inline bool st_ok(int nb, int d, int E) {
+  const int nv = co_nv(d, E);
+  return stream_enabled() && nb <= 2 && nv >= 4 && nv <= 6;
+}
+inline size_t st_smem(int nv) { return (size_t)ST_SLOTS * nv * CO_THREADS * 16; }
+inline int st_grid(long long rows) {
+  const long long cap = sm_count();
+  return (int)(rows < 1 ? 1 : (rows > cap ? cap : rows));
+}
+
+#define DV_ST_SWITCH(KERN, NB, grid, st, a)                                         \
+  switch (nv) {                                                                    \
+    case 4: return launch_fused_co(KERN<T, NB, 4>, grid, st_smem(4), st, a);        \
+    case 5: return launch_fused_co(KERN<T, NB, 5>, grid, st_smem(5), st, a);        \
+    default: return launch_fused_co(KERN<T, NB, 6>, grid, st_smem(6), st, a);       \
+  }
+
+template <typename K, typename A>
+cudaError_t launch_fused_co(K kern, dim3 grid, size_t smem, cudaStream_t st, const A& a) {
+  cudaError_t e = allow_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  return launch(kern, grid, CO_THREADS, smem, st, a);
+}
+
+template <typename T, int NB>
+cudaError_t run_attn_in_st_nb(const AttnInArgs& a, cudaStream_t st) {
+  const int nv = co_nv(a.d, WT<T>::E);
+  const dim3 grid(st_grid((long long)a.kh_max * 3 * a.dh));
+  DV_ST_SWITCH(attn_in_stream_kernel, NB, grid, st, a)
+}
+
+template <typename T, int NB>
+cudaError_t run_mlp_block_st_nb(MlpBlockArgs a, cudaStream_t st) {
+  const int nv = co_nv(a.d, WT<T>::E);
+  a.G = st_grid(a.k_max);
+  const dim3 grid(a.G);
+  DV_ST_SWITCH(mlp_stream_kernel, NB, grid, st, a)
+}
+
+template <typename T, int NB>
+cudaError_t run_predict_a_st_nb(const PredictAArgs& a, cudaStream_t st) {
+  const int nv = co_nv(a.d, WT<T>::E);
+  const dim3 grid(st_grid((a.PA ? a.h : 0) + (a.At ? a.r : 0)));
+  DV_ST_SWITCH(predict_a_stream_kernel, NB, grid, st, a)
+}
+#undef DV_ST_SWITCH
+
 template <typename T>
 cudaError_t run_attn_in_any(const AttnInArgs& a, cudaStream_t st) {
+  if (st_ok(a.nb, a.d, WT<T>::E))
+    return a.nb == 1 ? run_attn_in_st_nb<T, 1>(a, st) : run_attn_in_st_nb<T, 2>(a, st);
   if (co_ok(a.nb, a.d, WT<T>::E))
     return a.nb == 1 ? run_attn_in_co_nb<T, 1>(a, st) : run_attn_in_co_nb<T, 2>(a, st);
   return run_attn_in<T>(a, st);
@@ -375,6 +462,8 @@ cudaError_t run_attn_in_any(const AttnInArgs& a, cudaStream_t st) {
 
 template <typename T>
 cudaError_t run_mlp_block_any(const MlpBlockArgs& a, cudaStream_t st) {
+  if (st_ok(a.nb, a.d, WT<T>::E))
+    return a.nb == 1 ? run_mlp_block_st_nb<T, 1>(a, st) : run_mlp_block_st_nb<T, 2>(a, st);
   if (co_ok(a.nb, a.d, WT<T>::E))
     return a.nb == 1 ? run_mlp_block_co_nb<T, 1>(a, st) : run_mlp_block_co_nb<T, 2>(a, st);
   return run_mlp_block<T>(a, st);
@@ -382,6 +471,8 @@ cudaError_t run_mlp_block_any(const MlpBlockArgs& a, cudaStream_t st) {
 
 template <typename T>
 cudaError_t run_predict_a_any(const PredictAArgs& a, cudaStream_t st) {
+  if (st_ok(a.nb, a.d, WT<T>::E))
+    return a.nb == 1 ? run_predict_a_st_nb<T, 1>(a, st) : run_predict_a_st_nb<T, 2>(a, st);
   if (co_ok(a.nb, a.d, WT<T>::E))
     return a.nb == 1 ? run_predict_a_co_nb<T, 1>(a, st) : run_predict_a_co_nb<T, 2>(a, st);
   return run_predict_a<T>(a, st);
@@ -406,6 +497,8 @@ cudaError_t run_attn_dt(dv_dtype kvdt, int dh, const float* q, const void* Kc, c
                         float* part, unsigned* ctr, float* H, int* status, cudaStream_t st);
 cudaError_t run_attn_in_any_dt(dv_dtype wdt, const AttnInArgs& a, cudaStream_t st);
 cudaError_t run_attn_out_dt(dv_dtype kvdt, const AttnOutArgs& a, cudaStream_t st);
+cudaError_t run_attn_out_bf16(const AttnOutArgs& a, cudaStream_t st);
+cudaError_t run_attn_out_f32(const AttnOutArgs& a, cudaStream_t st);
 cudaError_t run_mlp_block_any_dt(dv_dtype wdt, const MlpBlockArgs& a, cudaStream_t st);
 cudaError_t run_predict_a_any_dt(dv_dtype wdt, const PredictAArgs& a, cudaStream_t st);
 cudaError_t run_predict_b_dt(dv_dtype wdt, const PredictBArgs& a, cudaStream_t st);

@@ -1,0 +1,412 @@
+// Streaming variants of the column-owner kernels for long rows (16 KB and
+// more: d >= 8192 in bf16), where a CTA streams tens of rows and the
+// register-resident loads of dv_colowner.cuh leave the memory pipe idle
+// between row groups.
+//
+// Rows pass through a ring of ST_SLOTS row slots in shared memory. Each of the
+// CTA's 256 threads copies its own 16-byte column vectors of upcoming rows into
+// the ring (cp.async, 16 bytes, through L2 only) and later reads back only what
+// it copied itself, so the ring needs no CTA barrier: a thread's
+// cp.async.wait_group orders its own copies. ST_SLOTS - 1 rows are in flight
+// while the CTA consumes one. The partial dot products of each warp collect in
+// shared memory and are summed across the CTA once per ST_RB rows.
+#pragma once
+
+#include "dv_colowner.cuh"
+
+namespace dv {
+
+constexpr int ST_SLOTS = 8;  // row slots of the ring
+constexpr int ST_RB = 16;    // rows per CTA reduction
+constexpr int ST_CH = 64;    // MLP: selection slots per chunk (W1 pass, then their W2 rows)
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Ring layout: [ST_SLOTS][NV][CO_THREADS] 16-byte vectors.
+template <int NV>
+__device__ __forceinline__ uint4* st_vec(uint4* ring, int slot, int j) {
+  return ring + ((size_t)(slot % ST_SLOTS) * NV + j) * CO_THREADS + threadIdx.x;
+}
+
+// Copies this thread's vectors of `row` (null: nothing) into `slot` and
+// closes one cp.async group (empty when row is null).
+template <typename T, int NV>
+__device__ __forceinline__ void st_issue(uint4* ring, int slot, const T* row, int nvec) {
+  constexpr int E = WT<T>::E;
+  if (row) {
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const int v = j * CO_THREADS + threadIdx.x;
+      if (v < nvec) cp_async16(st_vec<NV>(ring, slot, j), row + (size_t)v * E);
+    }
+  }
+  cp_async_commit();
+}
+
+// This thread's vectors of the row in `slot` (zero past the row's end).
+template <int NV>
+__device__ __forceinline__ void st_read(uint4* ring, int slot, int nvec, uint4 (&w)[NV]) {
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int v = j * CO_THREADS + threadIdx.x;
+    w[j] = v < nvec ? *st_vec<NV>(ring, slot, j) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// Issues the first ST_SLOTS - 1 rows of [r0, r1) (always ST_SLOTS - 1 groups).
+template <typename T, int NV, class RowFn>
+__device__ __forceinline__ void st_prologue(uint4* ring, int r0, int r1, int nvec, RowFn row) {
+#pragma unroll 1
+  for (int s = 0; s < ST_SLOTS - 1; ++s) st_issue<T, NV>(ring, s, r0 + s < r1 ? row(r0 + s) : nullptr, nvec);
+}
+
+// Streams rows [r0, r1) whose first ST_SLOTS - 1 were issued by st_prologue;
+// row(i) gives row i's pointer (null: skipped). For every row and batch row
+// out(i, b, s) receives the CTA-wide dot product s of the row with the input
+// slices xr, called by one thread. red: [2][ST_RB][NB][CO_WARPS].
+template <typename T, int NB, int NV, class RowFn, class OutFn>
+__device__ __forceinline__ void st_rows_dot(uint4* ring, int r0, int r1, int nvec,
+                                            const float (&xr)[NB][NV][WT<T>::E], float* red, RowFn row,
+                                            OutFn out) {
+  constexpr int E = WT<T>::E;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n = r1 - r0;
+#pragma unroll 1
+  for (int i = 0; i < n; ++i) {
+    const int ahead = i + ST_SLOTS - 1;
+    st_issue<T, NV>(ring, ahead, ahead < n ? row(r0 + ahead) : nullptr, nvec);
+    cp_async_wait<ST_SLOTS - 1>();
+    uint4 w[NV];
+    st_read<NV>(ring, i, nvec, w);
+    float acc[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) acc[b] = 0.f;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      float wf[E];
+      WT<T>::unpack(w[j], wf);
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[b] = fmaf(wf[e], xr[b][j][e], acc[b]);
+    }
+    const int buf = (i / ST_RB) & 1, ri = i % ST_RB;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      const float s = warp_sum(acc[b]);
+      if (lane == 0) red[((buf * ST_RB + ri) * NB + b) * CO_WARPS + warp] = s;
+    }
+    if (ri == ST_RB - 1 || i == n - 1) {
+      __syncthreads();
+      const int nr = ri + 1;
+      for (int t = threadIdx.x; t < nr * NB; t += CO_THREADS) {
+        const int rr = t / NB, b = t % NB;
+        float s = 0.f;
+#pragma unroll
+        for (int q = 0; q < CO_WARPS; ++q) s += red[((buf * ST_RB + rr) * NB + b) * CO_WARPS + q];
+        out(r0 + i - ri + rr, b, s);
+      }
+      // the other buffer is written next; this one again only after the
+      // next reduction's barrier, which every reader above reaches first
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// attn_in_stream_kernel: attn_in_kernel for long rows. CTA g streams the rows
+// [g n / G, (g + 1) n / G) of the n = |S_A| * 3 dh selected Q/K/V rows.
+// ----------------------------------------------------------------------------
+template <typename T, int NB, int NV>
+__global__ void __launch_bounds__(CO_THREADS, 1) attn_in_stream_kernel(AttnInArgs a) {
+  constexpr int E = WT<T>::E;
+  extern __shared__ __align__(16) uint4 s_ring[];
+  __shared__ float red[2 * ST_RB * NB * CO_WARPS];
+  __shared__ float lnred[2 * NB * CO_WARPS];
+  const T* Wqkv = static_cast<const T*>(a.Wqkv);
+  const int per = 3 * a.dh, nvec = a.d / E;
+  griddep_launch();
+  int r0 = 0, r1 = 0;
+  auto setup = [&]() {
+    int hc = *a.head_count;
+    if (hc > a.kh_max || hc < 0) {
+      if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(a.status, 1);
+      hc = hc < 0 ? 0 : a.kh_max;
+    }
+    const long long n = (long long)hc * per;
+    r0 = (int)(n * blockIdx.x / gridDim.x);
+    r1 = (int)(n * (blockIdx.x + 1) / gridDim.x);
+  };
+  auto head_of = [&](int slot) {
+    const int head = a.head_idx[slot / per];
+    return (head < 0 || head >= a.h) ? -1 : head;
+  };
+  auto row = [&](int slot) -> const T* {
+    const int head = head_of(slot);
+    return head < 0 ? nullptr : Wqkv + ((size_t)head * per + slot % per) * a.d;
+  };
+  if (a.sets_ready) {
+    setup();
+    st_prologue<T, NV>(s_ring, r0, r1, nvec, row);
+  }
+  griddep_wait();
+  if (!a.sets_ready) {
+    setup();
+    st_prologue<T, NV>(s_ring, r0, r1, nvec, row);
+  }
+  float xr[NB][NV][E];
+  x_slice_load<T, NB, NV>(a.x, a.d, a.nb, xr);
+  x_slice_ln<T, NB, NV>(xr, a.d, a.eps, a.ln_g, a.ln_b, lnred);
+  if (blockIdx.x == 0) {
+    if (a.yA_out) x_slice_store<T, NB, NV>(xr, a.d, a.nb, a.yA_out);
+    const int n4 = (a.nb * a.d) >> 2;
+    for (int i = threadIdx.x; i < n4; i += CO_THREADS)
+      reinterpret_cast<float4*>(a.t1)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  T* Kc = static_cast<T*>(a.Kc);
+  T* Vc = static_cast<T*>(a.Vc);
+  st_rows_dot<T, NB, NV>(s_ring, r0, r1, nvec, xr, red, row, [&](int slot, int b, float v) {
+    if (b >= a.nb) return;
+    const int head = head_of(slot);
+    if (head < 0) {
+      if (threadIdx.x == 0) raise_status(a.status, 2);
+      return;
+    }
+    const int p = slot / per, rem = slot % per, m = rem / a.dh, c = rem % a.dh;
+    if (a.bqkv) v += a.bqkv[(size_t)head * per + rem];
+    if (m == 0) {
+      a.q[((size_t)b * a.kh_max + p) * a.dh + c] = v;
+    } else {
+      T* cache = (m == 1) ? Kc : Vc;
+      cache[(((size_t)b * a.h + head) * a.cap + a.pos) * a.dh + c] = WT<T>::store_cvt(v);
+    }
+  });
+}
+
+// ----------------------------------------------------------------------------
+// predict_a_stream_kernel: predict_a_kernel for long rows (rows [0, h) of PA,
+// then rows [0, r) of At).
+// ----------------------------------------------------------------------------
+template <typename T, int NB, int NV>
+__global__ void __launch_bounds__(CO_THREADS, 1) predict_a_stream_kernel(PredictAArgs a) {
+  constexpr int E = WT<T>::E;
+  extern __shared__ __align__(16) uint4 s_ring[];
+  __shared__ float red[2 * ST_RB * NB * CO_WARPS];
+  const int nvec = a.d / E;
+  const int heads = a.PA ? a.h : 0;
+  const long long n = heads + (a.At ? a.r : 0);
+  const int r0 = (int)(n * blockIdx.x / gridDim.x), r1 = (int)(n * (blockIdx.x + 1) / gridDim.x);
+  auto row = [&](int i) -> const T* {
+    return i < heads ? static_cast<const T*>(a.PA) + (size_t)i * a.d
+                     : static_cast<const T*>(a.At) + (size_t)(i - heads) * a.d;
+  };
+  griddep_launch();
+  st_prologue<T, NV>(s_ring, r0, r1, nvec, row);
+  griddep_wait();  // y comes from the previous kernel
+  float xr[NB][NV][E];
+  x_slice_load<T, NB, NV>(a.y, a.d, a.nb, xr);
+  st_rows_dot<T, NB, NV>(s_ring, r0, r1, nvec, xr, red, row, [&](int i, int b, float v) {
+    if (b >= a.nb) return;
+    if (i < heads) a.scores_h[(size_t)b * a.h + i] = v;
+    else a.z[(size_t)b * a.r + i - heads] = v;
+  });
+}
+
+// ----------------------------------------------------------------------------
+// mlp_stream_kernel: mlp_block_kernel for long rows. CTA g owns selection slots
+// [g cnt / G, (g + 1) cnt / G), taken ST_CH at a time: the chunk's W1 rows
+// stream through the ring (dot products with LN2(t1)), one CTA reduction gives
+// the activations relu(. + b1), the nonzero ones are compacted, and their W2
+// rows stream through the ring into the thread's own output columns, which
+// are added to x once at the end (CTA 0 also adds t1 and b2).
+// ----------------------------------------------------------------------------
+template <typename T, int NB, int NV>
+__global__ void __launch_bounds__(CO_THREADS, 1) mlp_stream_kernel(MlpBlockArgs a) {
+  constexpr int E = WT<T>::E;
+  extern __shared__ __align__(16) uint4 s_ring[];
+  __shared__ float red[ST_CH * NB * CO_WARPS];
+  __shared__ float lnred[2 * NB * CO_WARPS];
+  __shared__ int s_row[ST_CH];     // W1 rows of the chunk (-1: invalid index)
+  __shared__ float s_bias[ST_CH];
+  __shared__ int s_row2[ST_CH];    // W2 rows with a nonzero activation
+  __shared__ float s_act2[ST_CH][NB];
+  __shared__ int s_nz;
+  const T* W1t = static_cast<const T*>(a.W1t);
+  const T* W2t = static_cast<const T*>(a.W2t);
+  const int nvec = a.d / E;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  griddep_launch();
+  int j0 = 0, j1 = 0;
+  auto slot_range = [&]() {
+    int cnt = *a.count;
+    if (cnt > a.k_max || cnt < 0) {
+      if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(a.status, 1);
+      cnt = cnt < 0 ? 0 : a.k_max;
+    }
+    j0 = (int)(((long long)cnt * blockIdx.x) / gridDim.x);
+    j1 = (int)(((long long)cnt * (blockIdx.x + 1)) / gridDim.x);
+  };
+  // the chunk's row indices and biases into shared memory, then its first rows
+  auto chunk_begin = [&](int c0, int cn) {
+    if ((int)threadIdx.x < cn) {
+      int rw = a.idx[c0 + threadIdx.x];
+      if (rw < 0 || rw >= a.N) {
+        raise_status(a.status, 2);
+        rw = -1;
+      }
+      s_row[threadIdx.x] = rw;
+      s_bias[threadIdx.x] = rw >= 0 ? a.b1[rw] : 0.f;
+    }
+    __syncthreads();
+    st_prologue<T, NV>(s_ring, 0, cn, nvec, [&](int i) -> const T* {
+      const int rw = s_row[i];
+      return rw >= 0 ? W1t + (size_t)rw * a.d : nullptr;
+    });
+  };
+  if (a.sets_ready) {
+    slot_range();
+    if (j1 > j0) chunk_begin(j0, min(ST_CH, j1 - j0));
+  }
+  griddep_wait();
+  if (!a.sets_ready) {
+    slot_range();
+    if (j1 > j0) chunk_begin(j0, min(ST_CH, j1 - j0));
+  }
+  float xr[NB][NV][E];
+  x_slice_load<T, NB, NV>(a.t1, a.d, a.nb, xr);
+  x_slice_ln<T, NB, NV>(xr, a.d, a.eps, a.ln_g, a.ln_b, lnred);
+  if (blockIdx.x == 0 && a.yM_out) x_slice_store<T, NB, NV>(xr, a.d, a.nb, a.yM_out);
+
+  float acc[NB][NV][E];
+#pragma unroll
+  for (int b = 0; b < NB; ++b)
+#pragma unroll
+    for (int j = 0; j < NV; ++j)
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[b][j][e] = 0.f;
+#pragma unroll 1
+  for (int c0 = j0; c0 < j1; c0 += ST_CH) {
+    const int cn = min(ST_CH, j1 - c0);
+    if (c0 != j0) chunk_begin(c0, cn);
+    // ---- W1: partial dots of the chunk's rows ----
+#pragma unroll 1
+    for (int i = 0; i < cn; ++i) {
+      const int ahead = i + ST_SLOTS - 1;
+      const int rw = ahead < cn ? s_row[ahead] : -1;
+      st_issue<T, NV>(s_ring, ahead, rw >= 0 ? W1t + (size_t)rw * a.d : nullptr, nvec);
+      cp_async_wait<ST_SLOTS - 1>();
+      uint4 w[NV];
+      st_read<NV>(s_ring, i, nvec, w);
+      float d1[NB];
+#pragma unroll
+      for (int b = 0; b < NB; ++b) d1[b] = 0.f;
+#pragma unroll
+      for (int j = 0; j < NV; ++j) {
+        float wf[E];
+        WT<T>::unpack(w[j], wf);
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+          for (int e = 0; e < E; ++e) d1[b] = fmaf(wf[e], xr[b][j][e], d1[b]);
+      }
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const float s = warp_sum(d1[b]);
+        if (lane == 0) red[(i * NB + b) * CO_WARPS + warp] = s;
+      }
+    }
+    __syncthreads();
+    // ---- activations, nonzero ones compacted in slot order ----
+    if (warp == 0) {
+      int base = 0;
+#pragma unroll 1
+      for (int i0 = 0; i0 < cn; i0 += 32) {
+        const int i = i0 + lane;
+        float act[NB];
+        bool nz = false;
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          float s = 0.f;
+          if (i < cn && b < a.nb && s_row[i] >= 0) {
+#pragma unroll
+            for (int q = 0; q < CO_WARPS; ++q) s += red[(i * NB + b) * CO_WARPS + q];
+            s = fmaxf(s + s_bias[i], 0.f);
+          }
+          act[b] = s;
+          nz |= s > 0.f;
+        }
+        const unsigned bal = __ballot_sync(0xffffffffu, nz);
+        if (nz) {
+          const int at = base + __popc(bal & ((1u << lane) - 1u));
+          s_row2[at] = s_row[i];
+#pragma unroll
+          for (int b = 0; b < NB; ++b) s_act2[at][b] = act[b];
+        }
+        base += __popc(bal);
+      }
+      if (lane == 0) s_nz = base;
+    }
+    __syncthreads();
+    // ---- W2: the nonzero rows into this thread's columns ----
+    const int nl = s_nz;
+    auto row2 = [&](int i) -> const T* { return W2t + (size_t)s_row2[i] * a.d; };
+    st_prologue<T, NV>(s_ring, 0, nl, nvec, row2);
+#pragma unroll 1
+    for (int i = 0; i < nl; ++i) {
+      const int ahead = i + ST_SLOTS - 1;
+      st_issue<T, NV>(s_ring, ahead, ahead < nl ? row2(ahead) : nullptr, nvec);
+      cp_async_wait<ST_SLOTS - 1>();
+      uint4 w[NV];
+      st_read<NV>(s_ring, i, nvec, w);
+      float cb[NB];
+#pragma unroll
+      for (int b = 0; b < NB; ++b) cb[b] = s_act2[i][b];
+#pragma unroll
+      for (int j = 0; j < NV; ++j) {
+        float wf[E];
+        WT<T>::unpack(w[j], wf);
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+          for (int e = 0; e < E; ++e) acc[b][j][e] = fmaf(cb[b], wf[e], acc[b][j][e]);
+      }
+    }
+    __syncthreads();  // s_row / s_row2 / s_act2 are rewritten by the next chunk
+  }
+  const bool residual = blockIdx.x == 0;
+  if (j1 == j0 && !residual) return;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int c = (j * CO_THREADS + threadIdx.x) * E;
+    if (c >= a.d) continue;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (b >= a.nb) continue;
+      float o[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) o[e] = acc[b][j][e];
+      if (residual) {
+#pragma unroll
+        for (int e4 = 0; e4 < E / 4; ++e4) {
+          const float4 t = __ldcg(reinterpret_cast<const float4*>(a.t1 + (size_t)b * a.d + c) + e4);
+          float4 bb = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (a.b2) bb = *(reinterpret_cast<const float4*>(a.b2 + c) + e4);
+          o[4 * e4 + 0] += t.x + bb.x;
+          o[4 * e4 + 1] += t.y + bb.y;
+          o[4 * e4 + 2] += t.z + bb.z;
+          o[4 * e4 + 3] += t.w + bb.w;
+        }
+      }
+#pragma unroll
+      for (int e4 = 0; e4 < E / 4; ++e4)
+        red_add4(a.x + (size_t)b * a.d + c + 4 * e4,
+                 make_float4(o[4 * e4], o[4 * e4 + 1], o[4 * e4 + 2], o[4 * e4 + 3]));
+    }
+  }
+}
+
+}  // namespace dv

@@ -32,6 +32,9 @@ SHAPES = {
     # dh = 128, a key count that does not split evenly over the attention cluster
     "fused128": dict(d=1024, N=4096, r=64, h=8, dh=128, L=300, cap=310, wdtype="bf16", kvdtype="bf16",
                      p_active=0.15),
+    # rows of 16 KB (bf16, d = 8192): the shared-memory ring kernels
+    "wide": dict(d=8192, N=12288, r=64, h=8, dh=128, L=200, cap=210, wdtype="bf16", kvdtype="bf16",
+                 p_active=0.10),
 }
 # "ragged" runs the kernel-per-step layer path (d is not a multiple of the
 # W^O column slices); the other shapes run the fused layer kernels.
@@ -363,6 +366,36 @@ def test_decode_layer(name, B):
     no_device_errors(ws)
 
 
+@pytest.mark.parametrize("name,B,kf,khf", [("wide", 1, 0.1, 0.25), ("wide", 1, 1.0, 1.0), ("wide", 2, 0.05, 0.5),
+                                          ("wide", 1, 0.0005, 0.125)])
+def test_decode_layer_selected_fractions(name, B, kf, khf):
+    """Layer output vs the oracle across selection sizes: from a few rows per
+    CTA (most CTAs idle) to every neuron and head (several chunks per CTA)."""
+    s, t = layer(name, B, seed=15)
+    x = wl.make_input(s, 24, DEV)
+    k = max(1, wl.k_for(kf, s.N))
+    k_h = max(1, wl.k_for(khf, s.h))
+    L = bd.Layer(t, B, min(s.N, B * k), min(s.h, B * k_h))
+    p = bd.params(k, k_h, 1.0 / np.sqrt(s.dh))
+    ws = bd.workspace(bd.DV_OP_DECODE_LAYER, L.dims)
+    tb = _trace_bufs(s)
+    x0 = x.clone()
+    OL = oracle_layer(t)
+    OL.K, OL.V = f64(t["K"]), f64(t["V"])
+    bd.dv_decode_layer(L, p, x, s.L, ws, trace=bd.layer_io(**tb))
+    torch.cuda.synchronize()
+    P = O.LayerParams(k=k, k_h=k_h, scale=1.0 / np.sqrt(s.dh))
+    sh, sm = tb["scores_h"].cpu().numpy(), tb["scores"].cpu().numpy()
+    hsel, msel = O.select(sh, k=k_h), O.select(sm, k=k)
+    assert np.array_equal(selected(tb["head_idx"], tb["head_count"]), hsel)
+    assert np.array_equal(selected(tb["idx"], tb["count"]), msel)
+    tr = O.decode_layer(f64(x0), OL, P, s.L, head_idx=hsel, idx=msel)
+    assert_out(tb["yA"].cpu().numpy(), tr.yA, "yA")
+    assert_out(tb["yM"].cpu().numpy(), tr.yM, "yM")
+    assert_out((x - x0).cpu().numpy(), tr.x_out - f64(x0), "x_out - x")
+    no_device_errors(ws)
+
+
 @pytest.mark.parametrize("name,lookahead,B", [("ragged", True, 1), ("ragged", False, 1), ("fused128", True, 1),
                                               ("fused128", False, 2), ("opt-like", True, 1)])
 def test_lookahead_stack(name, lookahead, B):
@@ -443,7 +476,7 @@ def test_decode_layer_with_empty_sets(name):
     no_device_errors(ws)
 
 
-@pytest.mark.parametrize("name", ["fused128", "opt-like", "tiny"])
+@pytest.mark.parametrize("name", ["fused128", "opt-like", "tiny", "wide"])
 def test_predict_layer_matches_oracle(name):
     """The look-ahead call (both sets from one input) on the fused predictor."""
     B = 2
@@ -467,7 +500,7 @@ def test_predict_layer_matches_oracle(name):
     no_device_errors(ws)
 
 
-@pytest.mark.parametrize("name", ["fused128", "ragged"])
+@pytest.mark.parametrize("name", ["fused128", "ragged", "wide"])
 def test_layer_in_three_calls_equals_one(name):
     """begin + attn + mlp (look-ahead sets given) == dv_decode_layer with the same sets."""
     B = 2
