@@ -158,6 +158,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_finish_kernel(SelectFinish
   __shared__ uint32_t s_hsel[HSEL_MAX / 32];
   __shared__ uint32_t s_bm[SEL_SMEM_KEYS / 32];
   __shared__ unsigned sc[SEL_WARPS + 1];
+  __shared__ unsigned s_h8[256];
   __shared__ unsigned s_digit, s_kk, s_ncand, s_last;
   griddep_launch();
   griddep_wait();
@@ -230,6 +231,9 @@ __global__ void __launch_bounds__(SEL_THREADS) select_finish_kernel(SelectFinish
       if (lane == 0) s_bm[w] = word;
     }
   } else {
+    unsigned* gh = a.hist + (size_t)b * SEL_BINS;
+    static_assert(SEL_BINS == 2 * SEL_THREADS, "two histogram bins per thread");
+    const unsigned h0 = gh[tid], h1 = gh[tid + SEL_THREADS];
     {  // keys into shared memory, 8 loads in flight per thread
       constexpr int UNR = 8;
       for (int i0 = tid; i0 < n; i0 += SEL_THREADS * UNR) {
@@ -246,17 +250,79 @@ __global__ void __launch_bounds__(SEL_THREADS) select_finish_kernel(SelectFinish
         }
       }
     }
-    unsigned* gh = a.hist + (size_t)b * SEL_BINS;
-    for (int i = tid; i < SEL_BINS; i += SEL_THREADS) {
-      s_h[i] = gh[i];
-      gh[i] = 0u;  // cleared for the next call
-    }
+    s_h[tid] = h0;
+    s_h[tid + SEL_THREADS] = h1;
+    gh[tid] = 0u;  // cleared for the next call
+    gh[tid + SEL_THREADS] = 0u;
     __syncthreads();
     uint32_t prefix = 0, mask = 0;
     unsigned kk = (unsigned)a.k;
-    bool use_cand = true;
+    bool use_cand = true, take_all_eq = false;
 #pragma unroll 1
     for (int pass = 0; pass < 3; ++pass) {
+      if (pass == 1 && use_cand) {
+        // the boundary bin's keys (few) refined by warp 0 alone in 8-bit
+        // digits (bits 20..13, 12..5, 4..0): no CTA barrier per digit
+        if (warp == 0) {
+          const int nc = (int)s_ncand;
+          unsigned cnt_eq = 0u;
+#pragma unroll 1
+          for (int ps = 0; ps < 3; ++ps) {
+            const int sh = ps == 0 ? 13 : (ps == 1 ? 5 : 0);
+            const unsigned dm = ps == 2 ? 0x1fu : 0xffu;
+            for (int i = lane; i < 256; i += 32) s_h8[i] = 0u;
+            __syncwarp();
+            for (int i = lane; i < nc; i += 32) {
+              const uint32_t key = s_cand[i];
+              if ((key & mask) == prefix) atomicAdd(&s_h8[(key >> sh) & dm], 1u);
+            }
+            __syncwarp();
+            // lane l owns bins 255 - 8l down to 248 - 8l
+            unsigned c[8], sum = 0u;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              c[j] = s_h8[255 - 8 * lane - j];
+              sum += c[j];
+            }
+            unsigned incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+              const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
+              if (lane >= o) incl += t;
+            }
+            const unsigned excl = incl - sum;
+            const bool mine = excl < kk && kk <= incl;
+            unsigned dig = 0u, knew = 0u, cnt = 0u, acc = excl;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              if (mine && dig == 0u && knew == 0u && acc + c[j] >= kk) {
+                dig = 255u - 8u * lane - j;
+                knew = kk - acc;
+                cnt = c[j];
+              }
+              acc += c[j];
+            }
+            const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+            dig = __shfl_sync(0xffffffffu, dig, src);
+            kk = __shfl_sync(0xffffffffu, knew, src);
+            cnt_eq = __shfl_sync(0xffffffffu, cnt, src);
+            prefix |= dig << sh;
+            mask |= dm << sh;
+            __syncwarp();
+          }
+          if (lane == 0) {
+            s_digit = prefix;
+            s_kk = kk;
+            s_ncand = cnt_eq;
+          }
+        }
+        __syncthreads();
+        prefix = s_digit;
+        mask = 0xffffffffu;
+        kk = s_kk;
+        take_all_eq = (kk == s_ncand);  // every key equal to the threshold is taken
+        break;
+      }
       const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
       const unsigned dmask = pass == 2 ? 0x3ffu : 0x7ffu;
       if (pass > 0) {
@@ -312,6 +378,13 @@ __global__ void __launch_bounds__(SEL_THREADS) select_finish_kernel(SelectFinish
         use_cand = s_ncand <= SF_CAND;
       }
     }
+    if (take_all_eq) {
+      for (int w = w0; w < w1; ++w) {
+        const int i = w * 32 + lane;
+        const unsigned word = __ballot_sync(0xffffffffu, i < n && s_keys[i] >= prefix);
+        if (lane == 0) s_bm[w] = word;
+      }
+    } else {
     unsigned eq = 0;
     for (int w = w0; w < w1; ++w) {
       const int i = w * 32 + lane;
@@ -341,6 +414,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_finish_kernel(SelectFinish
       const unsigned word = __ballot_sync(0xffffffffu, ok && (key > prefix || (e && rk < kk)));
       if (lane == 0) s_bm[w] = word;
       rank += __popc(em);
+    }
     }
   }
   __syncthreads();

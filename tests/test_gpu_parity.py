@@ -500,6 +500,37 @@ def test_predict_layer_matches_oracle(name):
     no_device_errors(ws)
 
 
+@pytest.mark.parametrize("name,group", [("opt-like", 8), ("opt-like", 0), ("ragged", 0), ("wide", 7)])
+def test_predict_layer_ties_at_threshold(name, group):
+    """Neuron scores with many exact ties at the k-th value (Bm rows and b1
+    repeated in groups; group 0: every score equal): the selection takes the
+    keys above the threshold and the lowest-index copies of the threshold."""
+    B = 1
+    s, t = layer(name, B, seed=16)
+    if group:
+        rep = torch.arange(s.N, device=DEV) // group * group
+        t["Bm"] = t["Bm"][rep].contiguous()
+        t["b1"] = t["b1"][rep].contiguous()
+    else:
+        t["Bm"] = torch.zeros_like(t["Bm"])
+        t["b1"] = torch.full_like(t["b1"], -0.5)
+    k, k_h = wl.k_for(0.1, s.N) + 1, 1
+    L = bd.Layer(t, B, min(s.N, B * k), min(s.h, B * k_h))
+    p = bd.params(k, k_h, 0.1)
+    ws = bd.workspace(bd.DV_OP_DECODE_LAYER, L.dims)
+    y = wl.make_input(s, 25, DEV)
+    tb = _trace_bufs(s)
+    out = bd.layer_io(scores_h=tb["scores_h"], head_idx=tb["head_idx"], head_count=tb["head_count"],
+                      scores=tb["scores"], idx=tb["idx"], count=tb["count"])
+    bd.dv_predict_layer(L, p, y, out, ws)
+    torch.cuda.synchronize()
+    sm = tb["scores"].cpu().numpy()
+    kth = np.sort(sm[0])[::-1][k - 1]
+    assert (sm[0] == kth).sum() > 1  # the threshold value is tied
+    assert np.array_equal(selected(tb["idx"], tb["count"]), O.select(sm, k=k))
+    no_device_errors(ws)
+
+
 @pytest.mark.parametrize("name", ["fused128", "ragged", "wide"])
 def test_layer_in_three_calls_equals_one(name):
     """begin + attn + mlp (look-ahead sets given) == dv_decode_layer with the same sets."""
