@@ -101,6 +101,14 @@ _lib_dv_decode_layer_mlp = _sig("dv_decode_layer_mlp", _c_int,
 _lib_dv_predict_layer = _sig("dv_predict_layer", _c_int,
                              [ctypes.POINTER(LayerWeightsC), ctypes.POINTER(Dims), ctypes.POINTER(LayerParamsC), _p,
                               ctypes.POINTER(LayerIOC), _p, _c_size, _p])
+_lib_dv_decode_layer_begin_ahead = _sig("dv_decode_layer_begin_ahead", _c_int,
+                                        [ctypes.POINTER(LayerWeightsC), ctypes.POINTER(Dims),
+                                         ctypes.POINTER(LayerParamsC), _p, _c_int, ctypes.POINTER(LayerIOC),
+                                         ctypes.POINTER(LayerIOC), _p, _c_size, ctypes.POINTER(LayerWeightsC), _p, _p,
+                                         _c_size, _p])
+_lib_dv_predict_layer_tail = _sig("dv_predict_layer_tail", _c_int,
+                                  [ctypes.POINTER(LayerWeightsC), ctypes.POINTER(Dims), ctypes.POINTER(LayerParamsC),
+                                   ctypes.POINTER(LayerIOC), _p, _c_size, _p])
 _lib_dv_layernorm = _sig("dv_layernorm", _c_int, [_p, _c_int, _c_int, _p, _p, _c_float, _p, _p])
 _lib_dv_topk_static = _sig("dv_topk_static", _c_int, [_p, _c_int, _c_int, _c_int, _c_float, _c_int, _p, _p, _p])
 _lib_dv_prefetch_layer = _sig("dv_prefetch_layer", _c_int,
@@ -326,6 +334,21 @@ def dv_predict_layer(layer: Layer, p: LayerParamsC, y, out: LayerIOC, ws, stream
     _check(_lib_dv_predict_layer(ctypes.byref(layer.c), ctypes.byref(layer.dims), ctypes.byref(p),
                                  _ptr(y, torch.float32, "y"), ctypes.byref(out), _ptr(ws, torch.uint8, "ws"),
                                  ws.numel(), _stream(stream)), "dv_predict_layer")
+
+
+def dv_decode_layer_begin_ahead(layer: Layer, p: LayerParamsC, x, pos, ws, nxt: Layer, next_scores_h, next_ws,
+                                sel: Optional[LayerIOC] = None, trace: Optional[LayerIOC] = None, stream=None):
+    _check(_lib_dv_decode_layer_begin_ahead(
+        ctypes.byref(layer.c), ctypes.byref(layer.dims), ctypes.byref(p), _ptr(x, torch.float32, "x"), int(pos),
+        ctypes.byref(sel) if sel is not None else None, ctypes.byref(trace) if trace is not None else None,
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), ctypes.byref(nxt.c), _ptr(next_scores_h, torch.float32, "scores_h"),
+        _ptr(next_ws, torch.uint8, "next_ws"), next_ws.numel(), _stream(stream)), "dv_decode_layer_begin_ahead")
+
+
+def dv_predict_layer_tail(layer: Layer, p: LayerParamsC, out: LayerIOC, ws, stream=None):
+    _check(_lib_dv_predict_layer_tail(ctypes.byref(layer.c), ctypes.byref(layer.dims), ctypes.byref(p),
+                                      ctypes.byref(out), _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)),
+           "dv_predict_layer_tail")
 
 
 def dv_prefetch_layer(layer: Layer, sel: LayerIOC, pos, with_w2=True, stream=None):

@@ -199,27 +199,15 @@ bool fused_ok(const dv_dims& D, dv_dtype wdt) {
 }
 
 
-// The head set (heads) and/or the neuron set (neurons) predicted from y:
-// predict_a (head scores, z = y A), predict_b (neuron scores + first digit
-// histogram), select_finish (exact top-k / threshold of both).
-dv_status fused_predict(const Layout& L, void* ws, const dv_layer_weights* w, const dv_dims& D,
-                        const dv_layer_params* p, const float* y, bool heads, bool neurons, float* sh, int32_t* hidx,
-                        int32_t* hcnt, float* sm, int32_t* midx, int32_t* mcnt, cudaStream_t st) {
-  PredictAArgs a = {};
-  a.y = y;
-  a.PA = heads ? w->PA : nullptr;
-  a.At = neurons ? w->At : nullptr;
-  a.h = D.h;
-  a.r = D.r;
-  a.d = D.d;
-  a.nb = D.B;
-  a.scores_h = sh;
-  a.z = at<float>(ws, L.z);
-  DV_TRY(run_predict_a_any_dt(w->wdtype, a, st));
+// Second half of the fused predictor: neuron scores from z (in ws) and the
+// selections; the head scores sh must be complete when heads is set.
+dv_status fused_predict_rest(const Layout& L, void* ws, const dv_layer_weights* w, const dv_dims& D,
+                             const dv_layer_params* p, bool heads, bool neurons, float* sh, int32_t* hidx,
+                             int32_t* hcnt, float* sm, int32_t* midx, int32_t* mcnt, cudaStream_t st) {
   const bool hist_mode = p->mode == DV_TOPK && p->k > 0 && p->k < D.N;
   if (neurons) {
     PredictBArgs b = {};
-    b.z = a.z;
+    b.z = at<float>(ws, L.z);
     b.Bm = w->Bm;
     b.b1 = w->b1;
     b.N = D.N;
@@ -257,6 +245,26 @@ dv_status fused_predict(const Layout& L, void* ws, const dv_layer_weights* w, co
   return DV_OK;
 }
 
+// The head set (heads) and/or the neuron set (neurons) predicted from y:
+// predict_a (head scores, z = y A), predict_b (neuron scores + first digit
+// histogram), select_finish (exact top-k / threshold of both).
+dv_status fused_predict(const Layout& L, void* ws, const dv_layer_weights* w, const dv_dims& D,
+                        const dv_layer_params* p, const float* y, bool heads, bool neurons, float* sh, int32_t* hidx,
+                        int32_t* hcnt, float* sm, int32_t* midx, int32_t* mcnt, cudaStream_t st) {
+  PredictAArgs a = {};
+  a.y = y;
+  a.PA = heads ? w->PA : nullptr;
+  a.At = neurons ? w->At : nullptr;
+  a.h = D.h;
+  a.r = D.r;
+  a.d = D.d;
+  a.nb = D.B;
+  a.scores_h = sh;
+  a.z = at<float>(ws, L.z);
+  DV_TRY(run_predict_a_any_dt(w->wdtype, a, st));
+  return fused_predict_rest(L, ws, w, D, p, heads, neurons, sh, hidx, hcnt, sm, midx, mcnt, st);
+}
+
 // Pointers a layer call writes: the trace buffers when given, else workspace.
 struct LayerBufs {
   float *yA, *yM, *sh, *sm;
@@ -284,10 +292,28 @@ LayerBufs layer_bufs(const Layout& L, void* ws, const dv_layer_io* sel, const dv
 }
 
 // First half of a layer: LN1, the head set unless given, Q/K/V + KV append.
+// The first half of the next layer's look-ahead predictor, computed with a
+// layer's q, k, v: head scores into sh, z into z.
+struct Ahead {
+  const dv_layer_weights* w;
+  float* sh;
+  float* z;
+};
+
 dv_status layer_begin(const Layout& L, void* ws, const dv_layer_weights* w, const dv_dims& D, const dv_layer_params* p,
-                      float* x, int pos, const dv_layer_io* sel, const dv_layer_io* trace, cudaStream_t st) {
+                      float* x, int pos, const dv_layer_io* sel, const dv_layer_io* trace, cudaStream_t st,
+                      const Ahead* ahead = nullptr) {
   const LayerBufs r = layer_bufs(L, ws, sel, trace);
   int* status = at<int>(ws, L.status);
+  if (ahead && !fused_ok(D, w->wdtype)) {
+    // kernel-per-step path: the layer, then the two predictor GEMVs from yA
+    float* yA = (sel && sel->yA) ? sel->yA : r.yA;
+    dv_layer_io tr = trace ? *trace : dv_layer_io{};
+    if (!(sel && sel->yA)) tr.yA = yA;
+    DV_CHECK(layer_begin(L, ws, w, D, p, x, pos, sel, &tr, st));
+    DV_TRY(run_gemv(w->wdtype, ahead->w->PA, D.h, D.d, yA, D.d, D.B, nullptr, ahead->sh, D.h, st));
+    return cuda_status(run_gemv(w->wdtype, ahead->w->At, D.r, D.d, yA, D.d, D.B, nullptr, ahead->z, D.r, st));
+  }
   if (fused_ok(D, w->wdtype)) {
     if (!sel) {
       DV_TRY(launch(layernorm_kernel, dim3(D.B), LN_THREADS, 0, st, (const float*)x, r.yA, D.d, w->ln1_g, w->ln1_b,
@@ -317,6 +343,30 @@ dv_status layer_begin(const Layout& L, void* ws, const dv_layer_weights* w, cons
     a.nb = D.B;
     a.sets_ready = sel ? 1 : 0;
     a.status = status;
+    if (ahead && attn_in_takes_rows(D.B, D.d, w->wdtype == DV_BF16 ? 8 : 4)) {
+      a.PA2 = ahead->w->PA;
+      a.At2 = ahead->w->At;
+      a.sh2 = ahead->sh;
+      a.z2 = ahead->z;
+      a.n2h = D.h;
+      a.n2r = D.r;
+      return cuda_status(run_attn_in_any_dt(w->wdtype, a, st));
+    }
+    if (ahead) {  // the row kernel: the predictor's first stage as its own launch, from yA
+      if (!a.yA_out) a.yA_out = r.yA;
+      DV_TRY(run_attn_in_any_dt(w->wdtype, a, st));
+      PredictAArgs pa = {};
+      pa.y = a.yA_out;
+      pa.PA = ahead->w->PA;
+      pa.At = ahead->w->At;
+      pa.h = D.h;
+      pa.r = D.r;
+      pa.d = D.d;
+      pa.nb = D.B;
+      pa.scores_h = ahead->sh;
+      pa.z = ahead->z;
+      return cuda_status(run_predict_a_any_dt(w->wdtype, pa, st));
+    }
     return cuda_status(run_attn_in_any_dt(w->wdtype, a, st));
   }
   // kernel-per-step path
@@ -590,6 +640,45 @@ dv_status dv_decode_layer_begin(const dv_layer_weights* w, const dv_dims* dims, 
   Layout L;
   DV_CHECK(check_layer_call(w, dims, p, x, pos, sel, trace, ws, ws_bytes, &L));
   return layer_begin(L, ws, w, *dims, p, x, pos, sel, trace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dv_status dv_decode_layer_begin_ahead(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p,
+                                      float* x, int pos, const dv_layer_io* sel, const dv_layer_io* trace, void* ws,
+                                      size_t ws_bytes, const dv_layer_weights* next, float* next_scores_h,
+                                      void* next_ws, size_t next_ws_bytes, dv_stream_t stream) {
+  Layout L;
+  DV_CHECK(check_layer_call(w, dims, p, x, pos, sel, trace, ws, ws_bytes, &L));
+  DV_CHECK(check_layer(next, dims, p));
+  if (next->wdtype != w->wdtype) return DV_ERR_UNSUPPORTED;
+  if (!next_scores_h || !next_ws) return DV_ERR_ARG;
+  if (!ok_ptr(next_scores_h)) return DV_ERR_ALIGN;
+  DV_CHECK(check_ws(L, next_ws, next_ws_bytes));
+  if (next_ws == ws) return DV_ERR_ARG;
+  const Ahead ahead{next, next_scores_h, at<float>(next_ws, L.z)};
+  return layer_begin(L, ws, w, *dims, p, x, pos, sel, trace, reinterpret_cast<cudaStream_t>(stream), &ahead);
+}
+
+dv_status dv_predict_layer_tail(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p,
+                                const dv_layer_io* out, void* ws, size_t ws_bytes, dv_stream_t stream) {
+  DV_CHECK(check_layer(w, dims, p));
+  const dv_dims& D = *dims;
+  if (!out || !out->scores_h || !out->head_idx || !out->head_count || !out->scores || !out->idx || !out->count)
+    return DV_ERR_ARG;
+  if (!ok_ptr(out->scores) || !ok_ptr(out->scores_h)) return DV_ERR_ALIGN;
+  const Layout L = layout(D, wbytes_of(w->wdtype));
+  DV_CHECK(check_ws(L, ws, ws_bytes));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (fused_ok(D, w->wdtype)) {
+    DV_CHECK(fused_predict_rest(L, ws, w, D, p, true, true, out->scores_h, out->head_idx, out->head_count,
+                                out->scores, out->idx, out->count, st));
+  } else {
+    DV_TRY(run_select(out->scores_h, D.B, D.h, p->k_h, p->tau_h, p->mode_h, at<uint32_t>(ws, L.bm_h),
+                      at<unsigned>(ws, L.sel_ticket_h), out->head_idx, out->head_count, st));
+    DV_TRY(run_gemv(w->wdtype, w->Bm, D.N, D.r, at<float>(ws, L.z), D.r, D.B, w->b1, out->scores, D.N, st));
+    DV_TRY(run_select(out->scores, D.B, D.N, p->k, p->tau, p->mode, at<uint32_t>(ws, L.bm_m),
+                      at<unsigned>(ws, L.sel_ticket_m), out->idx, out->count, st));
+  }
+  return cuda_status(launch(gate_kernel, dim3(1), dim3(32), 0, st));
 }
 
 dv_status dv_decode_layer_end(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p, float* x,

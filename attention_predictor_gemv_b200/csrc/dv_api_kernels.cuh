@@ -356,23 +356,39 @@ __global__ void __launch_bounds__(SEL_THREADS) select_finish_kernel(SelectFinish
       prefix |= s_digit << shift;
       mask |= dmask << shift;
       kk = s_kk;
-      if (pass == 0) {  // the keys of the boundary bin
-        if (tid == 0) s_ncand = 0u;
+      if (pass == 0) {  // the keys of the boundary bin, in index order
+        // each warp counts its words' candidates, a scan over the warps gives
+        // the offsets, then each warp writes its own (no shared counter: one
+        // address hit by every warp serialises)
+        unsigned cnt = 0u;
+        for (int w = w0; w < w1; ++w) {
+          const int i = w * 32 + lane;
+          const bool c = i < n && (s_keys[i] & mask) == prefix;
+          cnt += __popc(__ballot_sync(0xffffffffu, c));
+        }
+        if (lane == 0) sc[warp] = cnt;
         __syncthreads();
-        // one shared-memory atomic per warp and step (a per-key atomic on the
-        // one counter serialises the hundreds of keys in the boundary bin)
-        for (int i0 = 0; i0 < n; i0 += SEL_THREADS) {
-          const int i = i0 + tid;
+        if (warp == 0) {
+          const unsigned v = sc[lane];
+          unsigned incl = v;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+          }
+          sc[lane] = incl - v;
+          if (lane == 31) s_ncand = incl;
+        }
+        __syncthreads();
+        unsigned at = sc[warp];
+        for (int w = w0; w < w1; ++w) {
+          const int i = w * 32 + lane;
           const uint32_t key = i < n ? s_keys[i] : 0u;
           const bool c = i < n && (key & mask) == prefix;
           const unsigned bal = __ballot_sync(0xffffffffu, c);
-          unsigned base = 0u;
-          if (lane == 0 && bal) base = atomicAdd(&s_ncand, (unsigned)__popc(bal));
-          base = __shfl_sync(0xffffffffu, base, 0);
-          if (c) {
-            const unsigned at = base + __popc(bal & ((1u << lane) - 1u));
-            if (at < SF_CAND) s_cand[at] = key;
-          }
+          const unsigned mine = at + __popc(bal & ((1u << lane) - 1u));
+          if (c && mine < SF_CAND) s_cand[mine] = key;
+          at += __popc(bal);
         }
         __syncthreads();
         use_cand = s_ncand <= SF_CAND;

@@ -188,7 +188,9 @@ __device__ __forceinline__ void co_dot(const uint4 (&w)[R][NV], const float (&xr
 
 // ----------------------------------------------------------------------------
 // attn_in_co_kernel: attn_in_kernel (LN1, selected heads' q/k/v, KV append)
-// with R output rows per CTA, column-owner layout.
+// with R output rows per CTA, column-owner layout. Slots [0, kh_max 3 dh) are
+// the Q/K/V rows of the selected heads (those past the count idle), slots
+// after them the optional rows of the next layer's predictor.
 // ----------------------------------------------------------------------------
 template <typename T, int NB, int NV, int R>
 __global__ void __launch_bounds__(CO_THREADS) attn_in_co_kernel(AttnInArgs a) {
@@ -198,7 +200,8 @@ __global__ void __launch_bounds__(CO_THREADS) attn_in_co_kernel(AttnInArgs a) {
   const T* Wqkv = static_cast<const T*>(a.Wqkv);
   const int per = 3 * a.dh;
   const int nvec = a.d / E;
-  const int ngroups = (a.kh_max * per + R - 1) / R;
+  const int qrows = a.kh_max * per, n2 = a.n2h + a.n2r;
+  const int ngroups = (qrows + n2 + R - 1) / R;
   int slot0 = blockIdx.x * R;
   griddep_launch();
   const T* rowp[R];
@@ -217,17 +220,25 @@ __global__ void __launch_bounds__(CO_THREADS) attn_in_co_kernel(AttnInArgs a) {
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const int slot = slot0 + r;
-      int head = -1;
+      int head = -1;  // >= 0: a Q/K/V row of that head; <= -2: predictor row -2 - head
+      const T* rp = Wqkv;
       if (slot < nslot) {
         head = a.head_idx[slot / per];
         if (head < 0 || head >= a.h) {
           if (threadIdx.x == 0) raise_status(a.status, 2);
           head = -1;
+        } else {
+          rp = Wqkv + ((size_t)head * per + (slot % per)) * a.d;
         }
+      } else if (slot >= qrows && slot < qrows + n2) {
+        const int i2 = slot - qrows;
+        head = -2 - i2;
+        rp = i2 < a.n2h ? static_cast<const T*>(a.PA2) + (size_t)i2 * a.d
+                        : static_cast<const T*>(a.At2) + (size_t)(i2 - a.n2h) * a.d;
       }
       heads[r] = head;
-      valid[r] = head >= 0;
-      rowp[r] = Wqkv + ((size_t)(head >= 0 ? head : 0) * per + (slot % per)) * a.d;
+      valid[r] = head != -1;
+      rowp[r] = rp;
     }
   };
   uint4 w[R][NV];
@@ -271,9 +282,15 @@ __global__ void __launch_bounds__(CO_THREADS) attn_in_co_kernel(AttnInArgs a) {
           head = heads[rr];
         }
       if (!ok || b >= a.nb) continue;
+      float v = s_out[i];
+      if (head <= -2) {
+        const int i2 = -2 - head;
+        if (i2 < a.n2h) a.sh2[(size_t)b * a.n2h + i2] = v;
+        else a.z2[(size_t)b * a.n2r + i2 - a.n2h] = v;
+        continue;
+      }
       const int slot = slot0 + r;
       const int p = slot / per, rem = slot % per, m = rem / a.dh, c = rem % a.dh;
-      float v = s_out[i];
       if (a.bqkv) v += a.bqkv[(size_t)head * per + rem];
       if (m == 0) {
         a.q[((size_t)b * a.kh_max + p) * a.dh + c] = v;

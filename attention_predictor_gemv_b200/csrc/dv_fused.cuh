@@ -395,6 +395,14 @@ struct AttnInArgs {
   void* Vc;
   int h, dh, d, cap, pos, nb, sets_ready;
   int* status;
+  // optional rows of the next layer's predictor, dotted with the same yA
+  // (column-owner and streaming kernels): PA2 [n2h][d] -> sh2 [nb][n2h],
+  // At2 [n2r][d] -> z2 [nb][n2r]
+  const void* PA2;
+  const void* At2;
+  float* sh2;
+  float* z2;
+  int n2h, n2r;
 };
 
 template <typename T, int NB, int RPW, int U>

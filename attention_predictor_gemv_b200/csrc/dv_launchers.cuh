@@ -371,7 +371,7 @@ inline int co_grid(long long groups) {
 template <typename T, int NB>
 cudaError_t run_attn_in_co_nb(const AttnInArgs& a, cudaStream_t st) {
   const int nv = co_nv(a.d, WT<T>::E), R = co_r(nv);
-  const dim3 grid(co_grid(((long long)a.kh_max * 3 * a.dh + R - 1) / R));
+  const dim3 grid(co_grid(((long long)a.kh_max * 3 * a.dh + a.n2h + a.n2r + R - 1) / R));
   DV_CO_SWITCH(attn_in_co_kernel, NB, grid, st, a)
 }
 
@@ -431,7 +431,7 @@ cudaError_t launch_fused_co(K kern, dim3 grid, size_t smem, cudaStream_t st, con
 template <typename T, int NB>
 cudaError_t run_attn_in_st_nb(const AttnInArgs& a, cudaStream_t st) {
   const int nv = co_nv(a.d, WT<T>::E);
-  const dim3 grid(st_grid((long long)a.kh_max * 3 * a.dh));
+  const dim3 grid(st_grid((long long)a.kh_max * 3 * a.dh + a.n2h + a.n2r));
   DV_ST_SWITCH(attn_in_stream_kernel, NB, grid, st, a)
 }
 
@@ -450,6 +450,10 @@ cudaError_t run_predict_a_st_nb(const PredictAArgs& a, cudaStream_t st) {
   DV_ST_SWITCH(predict_a_stream_kernel, NB, grid, st, a)
 }
 #undef DV_ST_SWITCH
+
+// Whether run_attn_in_any picks a kernel that also takes the next layer's
+// predictor rows (the column-owner and streaming kernels).
+inline bool attn_in_takes_rows(int nb, int d, int E) { return st_ok(nb, d, E) || co_ok(nb, d, E); }
 
 template <typename T>
 cudaError_t run_attn_in_any(const AttnInArgs& a, cudaStream_t st) {

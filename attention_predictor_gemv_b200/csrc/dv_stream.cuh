@@ -119,7 +119,8 @@ __device__ __forceinline__ void st_rows_dot(uint4* ring, int r0, int r1, int nve
 
 // ----------------------------------------------------------------------------
 // attn_in_stream_kernel: attn_in_kernel for long rows. CTA g streams the rows
-// [g n / G, (g + 1) n / G) of the n = |S_A| * 3 dh selected Q/K/V rows.
+// [g n / G, (g + 1) n / G) of the n = |S_A| * 3 dh selected Q/K/V rows
+// followed by the optional rows of the next layer's predictor.
 // ----------------------------------------------------------------------------
 template <typename T, int NB, int NV>
 __global__ void __launch_bounds__(CO_THREADS, 1) attn_in_stream_kernel(AttnInArgs a) {
@@ -130,14 +131,15 @@ __global__ void __launch_bounds__(CO_THREADS, 1) attn_in_stream_kernel(AttnInArg
   const T* Wqkv = static_cast<const T*>(a.Wqkv);
   const int per = 3 * a.dh, nvec = a.d / E;
   griddep_launch();
-  int r0 = 0, r1 = 0;
+  int r0 = 0, r1 = 0, nq = 0;  // rows [0, nq): Q/K/V; [nq, nq + n2h + n2r): next layer's predictor
   auto setup = [&]() {
     int hc = *a.head_count;
     if (hc > a.kh_max || hc < 0) {
       if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(a.status, 1);
       hc = hc < 0 ? 0 : a.kh_max;
     }
-    const long long n = (long long)hc * per;
+    nq = hc * per;
+    const long long n = (long long)nq + a.n2h + a.n2r;
     r0 = (int)(n * blockIdx.x / gridDim.x);
     r1 = (int)(n * (blockIdx.x + 1) / gridDim.x);
   };
@@ -146,6 +148,11 @@ __global__ void __launch_bounds__(CO_THREADS, 1) attn_in_stream_kernel(AttnInArg
     return (head < 0 || head >= a.h) ? -1 : head;
   };
   auto row = [&](int slot) -> const T* {
+    if (slot >= nq) {
+      const int i2 = slot - nq;
+      return i2 < a.n2h ? static_cast<const T*>(a.PA2) + (size_t)i2 * a.d
+                        : static_cast<const T*>(a.At2) + (size_t)(i2 - a.n2h) * a.d;
+    }
     const int head = head_of(slot);
     return head < 0 ? nullptr : Wqkv + ((size_t)head * per + slot % per) * a.d;
   };
@@ -171,6 +178,12 @@ __global__ void __launch_bounds__(CO_THREADS, 1) attn_in_stream_kernel(AttnInArg
   T* Vc = static_cast<T*>(a.Vc);
   st_rows_dot<T, NB, NV>(s_ring, r0, r1, nvec, xr, red, row, [&](int slot, int b, float v) {
     if (b >= a.nb) return;
+    if (slot >= nq) {
+      const int i2 = slot - nq;
+      if (i2 < a.n2h) a.sh2[(size_t)b * a.n2h + i2] = v;
+      else a.z2[(size_t)b * a.n2r + i2 - a.n2h] = v;
+      return;
+    }
     const int head = head_of(slot);
     if (head < 0) {
       if (threadIdx.x == 0) raise_status(a.status, 2);

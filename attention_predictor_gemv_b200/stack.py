@@ -25,7 +25,8 @@ class DecoderStack:
     def __init__(self, layers: List[Dict[str, torch.Tensor]], B: int, k: int, k_h: int, scale: float,
                  lookahead: bool = True, eps: float = 1e-5, mode: int = bd.DV_TOPK, tau: float = 0.0,
                  mode_h: int = bd.DV_TOPK, tau_h: float = 0.0, k_max: Optional[int] = None,
-                 kh_max: Optional[int] = None, prefetch: bool = False, prefetch_w2: bool = True):
+                 kh_max: Optional[int] = None, prefetch: bool = False, prefetch_w2: bool = True,
+                 fuse_ahead: bool = True):
         t0 = layers[0]
         N, d = t0["W1t"].shape
         h = t0["Wqkv"].shape[0]
@@ -38,6 +39,8 @@ class DecoderStack:
         self.lookahead = lookahead
         self.prefetch = prefetch and lookahead
         self.prefetch_w2 = prefetch_w2
+        # the predictor's first stage for layer l+1 inside layer l's q/k/v kernel
+        self.fuse_ahead = fuse_ahead
         D = self.layers[0].dims
         self.ws_main = bd.workspace(bd.DV_OP_DECODE_LAYER, D, dev)
         self.ws_side = bd.workspace(bd.DV_OP_DECODE_LAYER, D, dev)
@@ -82,9 +85,14 @@ class DecoderStack:
                 sel, trace = self.io_given[l], self.io_trace_y[l]
             else:
                 sel, trace = None, self.io_trace[l]
-            bd.dv_decode_layer_begin(L, self.p, x, pos, self.ws_main, sel=sel, trace=trace)
-            if la and l + 1 < nL:
-                self.ev_yA[l].record(main)  # yA[l] is written by the work just issued
+            ahead = la and l + 1 < nL
+            if ahead and self.fuse_ahead:
+                bd.dv_decode_layer_begin_ahead(L, self.p, x, pos, self.ws_main, self.layers[l + 1],
+                                               self.scores_h[l + 1], self.ws_side, sel=sel, trace=trace)
+            else:
+                bd.dv_decode_layer_begin(L, self.p, x, pos, self.ws_main, sel=sel, trace=trace)
+            if ahead:
+                self.ev_yA[l].record(main)  # yA[l] (and the first stage for l+1) written by the work just issued
                 self._predict_next(l, pos)
             bd.dv_decode_layer_end(L, self.p, x, pos, self.ws_main, sel=sel, trace=trace)
         if la:
@@ -97,8 +105,12 @@ class DecoderStack:
         prefetch of the parameters those sets select (layer l+1 runs after
         layer l on the main stream, and finds them in L2)."""
         self.side.wait_event(self.ev_yA[l])
-        bd.dv_predict_layer(self.layers[l + 1], self.p, self.yA[l], self.io_sets[l + 1], self.ws_side,
-                            stream=self.side)
+        if self.fuse_ahead:
+            bd.dv_predict_layer_tail(self.layers[l + 1], self.p, self.io_sets[l + 1], self.ws_side,
+                                     stream=self.side)
+        else:
+            bd.dv_predict_layer(self.layers[l + 1], self.p, self.yA[l], self.io_sets[l + 1], self.ws_side,
+                                stream=self.side)
         self.ev_sel[l + 1].record(self.side)
         if self.prefetch:
             bd.dv_prefetch_layer(self.layers[l + 1], self.io_sets[l + 1], pos, with_w2=self.prefetch_w2,

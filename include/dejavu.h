@@ -278,6 +278,31 @@ DV_API dv_status dv_predict_layer(const dv_layer_weights* w, const dv_dims* dims
                            const float* y, const dv_layer_io* out, void* ws, size_t ws_bytes,
                            dv_stream_t stream);
 
+/* Look-ahead prediction split across the two streams (§1). The predictor's
+ * first stage for the next layer -- head scores y P_A'^T and z = y A' -- reads
+ * the same normalised input y = LN1(x) as this layer's q, k, v, so it runs in
+ * the same kernel:
+ *
+ * dv_decode_layer_begin_ahead is dv_decode_layer_begin (same arguments,
+ * same results) that also writes, for the layer `next` (same dims and
+ * weight dtype as w), the head scores into next_scores_h [B][h] (fp32,
+ * device, 16-byte aligned) and z [B][r] into the workspace next_ws (sized
+ * for DV_OP_DECODE_LAYER with the same dims; it must not be ws).
+ *
+ * dv_predict_layer_tail then completes the prediction for that layer on any
+ * stream ordered after the begin_ahead call: neuron scores z B^T + b1 and
+ * both selections, written like dv_predict_layer; out->scores_h must be the
+ * next_scores_h given to begin_ahead and ws its next_ws. Together the two
+ * calls give the same scores and sets as dv_predict_layer(next, y). Its last
+ * launch is the same gate as dv_predict_layer's. */
+DV_API dv_status dv_decode_layer_begin_ahead(const dv_layer_weights* w, const dv_dims* dims,
+                                             const dv_layer_params* p, float* x, int pos, const dv_layer_io* sel,
+                                             const dv_layer_io* trace, void* ws, size_t ws_bytes,
+                                             const dv_layer_weights* next, float* next_scores_h, void* next_ws,
+                                             size_t next_ws_bytes, dv_stream_t stream);
+DV_API dv_status dv_predict_layer_tail(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p,
+                                       const dv_layer_io* out, void* ws, size_t ws_bytes, dv_stream_t stream);
+
 /* L2 prefetch of one layer's selected parameters (§1: for the next layer
  * the look-ahead predictor picks the heads / neurons and only those
  * parameters are loaded). Given the sets `sel` (head_idx/head_count and

@@ -396,15 +396,19 @@ def test_decode_layer_selected_fractions(name, B, kf, khf):
     no_device_errors(ws)
 
 
-@pytest.mark.parametrize("name,lookahead,B", [("ragged", True, 1), ("ragged", False, 1), ("fused128", True, 1),
-                                              ("fused128", False, 2), ("opt-like", True, 1)])
-def test_lookahead_stack(name, lookahead, B):
+@pytest.mark.parametrize("name,lookahead,B,fuse", [("ragged", True, 1, True), ("ragged", False, 1, True),
+                                                   ("fused128", True, 1, True), ("fused128", False, 2, True),
+                                                   ("opt-like", True, 1, True), ("opt-like", True, 1, False),
+                                                   ("ragged", True, 2, False), ("fused128", True, 2, True)])
+def test_lookahead_stack(name, lookahead, B, fuse):
+    """fuse: the next layer's predictor first stage inside the q/k/v kernel
+    (begin_ahead + predict_layer_tail) rather than dv_predict_layer."""
     nL = 3
     s = shape(name, B)
     layers = [wl.make_layer(s, 100 + l, DEV) for l in range(nL)]
     K0 = [(f64(t["K"]), f64(t["V"])) for t in layers]
     k, k_h = wl.k_for(0.1, s.N), 2
-    stk = DecoderStack(layers, B, k, k_h, 1.0 / np.sqrt(s.dh), lookahead=lookahead)
+    stk = DecoderStack(layers, B, k, k_h, 1.0 / np.sqrt(s.dh), lookahead=lookahead, fuse_ahead=fuse)
     x = wl.make_input(s, 31, DEV)
     x0 = f64(x)
     pos = s.L
@@ -529,6 +533,49 @@ def test_predict_layer_ties_at_threshold(name, group):
     assert (sm[0] == kth).sum() > 1  # the threshold value is tied
     assert np.array_equal(selected(tb["idx"], tb["count"]), O.select(sm, k=k))
     no_device_errors(ws)
+
+
+@pytest.mark.parametrize("name,B", [("opt-like", 1), ("fused128", 2), ("ragged", 1), ("wide", 1), ("tiny", 3)])
+def test_begin_ahead_and_tail_predict_next_layer(name, B):
+    """The next layer's predictor split over begin_ahead (its first stage in
+    this layer's q/k/v kernel) and predict_layer_tail: scores of layer 2 from
+    layer 1's yA, sets = the oracle's selection of those scores, and layer 1's
+    own q/k/v work unchanged (the KV slot it writes)."""
+    s, t = layer(name, B, seed=17)
+    t2 = wl.make_layer(s, 18, DEV)
+    k, k_h = wl.k_for(0.1, s.N), 2
+    L1 = bd.Layer(t, B, min(s.N, B * k), min(s.h, B * k_h))
+    L2 = bd.Layer(t2, B, min(s.N, B * k), min(s.h, B * k_h))
+    p = bd.params(k, k_h, 0.1)
+    ws1 = bd.workspace(bd.DV_OP_DECODE_LAYER, L1.dims)
+    ws2 = bd.workspace(bd.DV_OP_DECODE_LAYER, L1.dims)
+    x = wl.make_input(s, 26, DEV)
+    tb1, tb2 = _trace_bufs(s), _trace_bufs(s)
+    Kref, Vref = t["K"].clone(), t["V"].clone()
+    x_ref = x.clone()
+    ws_ref = bd.workspace(bd.DV_OP_DECODE_LAYER, L1.dims)
+    tr_ref = _trace_bufs(s)
+    t_ref = {kk: v for kk, v in t.items()}
+    t_ref["K"], t_ref["V"] = Kref, Vref
+    bd.dv_decode_layer_begin(bd.Layer(t_ref, B, L1.dims.k_max, L1.dims.kh_max), p, x_ref, s.L, ws_ref,
+                             trace=bd.layer_io(**tr_ref))
+    bd.dv_decode_layer_begin_ahead(L1, p, x, s.L, ws1, L2, tb2["scores_h"], ws2, trace=bd.layer_io(**tb1))
+    out2 = bd.layer_io(scores_h=tb2["scores_h"], head_idx=tb2["head_idx"], head_count=tb2["head_count"],
+                       scores=tb2["scores"], idx=tb2["idx"], count=tb2["count"])
+    bd.dv_predict_layer_tail(L2, p, out2, ws2)
+    torch.cuda.synchronize()
+    yA = f64(tb1["yA"])
+    sh, sm = tb2["scores_h"].cpu().numpy(), tb2["scores"].cpu().numpy()
+    assert_scores(sh, O.head_predictor_scores(yA, f64(t2["PA"])))
+    assert_scores(sm, O.mlp_predictor_scores(yA, f64(t2["At"]), f64(t2["Bm"]), f64(t2["b1"])))
+    assert np.array_equal(selected(tb2["head_idx"], tb2["head_count"]), O.select(sh, k=k_h))
+    assert np.array_equal(selected(tb2["idx"], tb2["count"]), O.select(sm, k=k))
+    # layer 1's own begin: same sets and the same KV slot as the plain call
+    assert np.array_equal(selected(tb1["head_idx"], tb1["head_count"]),
+                          selected(tr_ref["head_idx"], tr_ref["head_count"]))
+    assert torch.equal(t["K"][:, :, s.L], Kref[:, :, s.L]) and torch.equal(t["V"][:, :, s.L], Vref[:, :, s.L])
+    no_device_errors(ws1)
+    no_device_errors(ws2)
 
 
 @pytest.mark.parametrize("name", ["fused128", "ragged", "wide"])
