@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_finish_kernel(SelectFinish
   __shared__ uint32_t s_hsel[HSEL_MAX / 32];
   __shared__ uint32_t s_bm[SEL_SMEM_KEYS / 32];
   __shared__ unsigned sc[SEL_WARPS + 1];
-  __shared__ unsigned s_h8[256];
+  __shared__ unsigned s_wcnt[SEL_WARPS];
   __shared__ unsigned s_digit, s_kk, s_ncand, s_last;
   griddep_launch();
   griddep_wait();
@@ -220,8 +220,22 @@ __global__ void __launch_bounds__(SEL_THREADS) select_finish_kernel(SelectFinish
   const float* row = a.scores + (size_t)b * n;
   const int nw = (n + 31) >> 5;
   uint32_t* bm = a.bitmaps + (size_t)b * nw;
-  const int wpw = (nw + SEL_WARPS - 1) / SEL_WARPS;
+  const int wpw = (nw + SEL_WARPS - 1) / SEL_WARPS;  // warp w owns the words [w wpw, (w+1) wpw)
   const int w0 = warp * wpw, w1 = min(nw, w0 + wpw);
+  const unsigned lt = (1u << lane) - 1u;
+  // exclusive offset of this warp's count among the CTA's warps, and the
+  // total: every warp scans the SEL_WARPS counts itself (no second barrier)
+  auto warp_offsets = [&](unsigned& off, unsigned& total) {
+    const unsigned v = s_wcnt[lane];
+    unsigned incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    off = __shfl_sync(0xffffffffu, incl - v, warp);
+    total = __shfl_sync(0xffffffffu, incl, 31);
+  };
   const bool hist_mode = a.mode == 0 && a.k > 0 && a.k < n;
   if (!hist_mode) {
     for (int w = w0; w < w1; ++w) {
@@ -233,6 +247,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_finish_kernel(SelectFinish
   } else {
     unsigned* gh = a.hist + (size_t)b * SEL_BINS;
     static_assert(SEL_BINS == 2 * SEL_THREADS, "two histogram bins per thread");
+    static_assert(SEL_WARPS == 32, "one count per lane of a warp");
     const unsigned h0 = gh[tid], h1 = gh[tid + SEL_THREADS];
     {  // keys into shared memory, 8 loads in flight per thread
       constexpr int UNR = 8;
@@ -255,145 +270,136 @@ __global__ void __launch_bounds__(SEL_THREADS) select_finish_kernel(SelectFinish
     gh[tid] = 0u;  // cleared for the next call
     gh[tid + SEL_THREADS] = 0u;
     __syncthreads();
-    uint32_t prefix = 0, mask = 0;
-    unsigned kk = (unsigned)a.k;
-    bool use_cand = true, take_all_eq = false;
-#pragma unroll 1
-    for (int pass = 0; pass < 3; ++pass) {
-      if (pass == 1 && use_cand) {
-        // the boundary bin's keys (few) refined by warp 0 alone in 8-bit
-        // digits (bits 20..13, 12..5, 4..0): no CTA barrier per digit
-        if (warp == 0) {
-          const int nc = (int)s_ncand;
-          unsigned cnt_eq = 0u;
-#pragma unroll 1
-          for (int ps = 0; ps < 3; ++ps) {
-            const int sh = ps == 0 ? 13 : (ps == 1 ? 5 : 0);
-            const unsigned dm = ps == 2 ? 0x1fu : 0xffu;
-            for (int i = lane; i < 256; i += 32) s_h8[i] = 0u;
-            __syncwarp();
-            for (int i = lane; i < nc; i += 32) {
-              const uint32_t key = s_cand[i];
-              if ((key & mask) == prefix) atomicAdd(&s_h8[(key >> sh) & dm], 1u);
-            }
-            __syncwarp();
-            // lane l owns bins 255 - 8l down to 248 - 8l
-            unsigned c[8], sum = 0u;
+    // ---- top digit (bits 31..21) of the k-th largest key: warp 0 walks the
+    // histogram from the top, 64 bins per lane ----
+    if (warp == 0) {
+      const int hi = SEL_BINS - 1 - 64 * lane;  // lane's bins hi, hi-1, ..., hi-63
+      unsigned sum = 0u;
+#pragma unroll 8
+      for (int j = 0; j < 64; ++j) sum += s_h[hi - j];
+      unsigned incl = sum;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              c[j] = s_h8[255 - 8 * lane - j];
-              sum += c[j];
-            }
-            unsigned incl = sum;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-              const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
-              if (lane >= o) incl += t;
-            }
-            const unsigned excl = incl - sum;
-            const bool mine = excl < kk && kk <= incl;
-            unsigned dig = 0u, knew = 0u, cnt = 0u, acc = excl;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              if (mine && dig == 0u && knew == 0u && acc + c[j] >= kk) {
-                dig = 255u - 8u * lane - j;
-                knew = kk - acc;
-                cnt = c[j];
-              }
-              acc += c[j];
-            }
-            const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
-            dig = __shfl_sync(0xffffffffu, dig, src);
-            kk = __shfl_sync(0xffffffffu, knew, src);
-            cnt_eq = __shfl_sync(0xffffffffu, cnt, src);
-            prefix |= dig << sh;
-            mask |= dm << sh;
-            __syncwarp();
-          }
-          if (lane == 0) {
-            s_digit = prefix;
-            s_kk = kk;
-            s_ncand = cnt_eq;
-          }
-        }
-        __syncthreads();
-        prefix = s_digit;
-        mask = 0xffffffffu;
-        kk = s_kk;
-        take_all_eq = (kk == s_ncand);  // every key equal to the threshold is taken
-        break;
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
       }
-      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-      const unsigned dmask = pass == 2 ? 0x3ffu : 0x7ffu;
-      if (pass > 0) {
+      const unsigned kk0 = (unsigned)a.k;
+      if (incl - sum < kk0 && kk0 <= incl) {
+        unsigned acc = incl - sum;
+        for (int j = 0; j < 64; ++j) {
+          const unsigned c = s_h[hi - j];
+          if (acc + c >= kk0) {
+            s_digit = (unsigned)(hi - j);
+            s_kk = kk0 - acc;
+            break;
+          }
+          acc += c;
+        }
+      }
+    }
+    __syncthreads();
+    uint32_t prefix = s_digit << 21, mask = 0x7ffu << 21;
+    unsigned kk = s_kk;
+    bool take_all_eq = false;
+    // ---- the keys of the boundary bin, compacted in index order ----
+    {
+      unsigned cnt = 0u;
+      for (int w = w0; w < w1; ++w) {
+        const int i = w * 32 + lane;
+        cnt += __popc(__ballot_sync(0xffffffffu, i < n && (s_keys[i] & mask) == prefix));
+      }
+      if (lane == 0) s_wcnt[warp] = cnt;
+    }
+    __syncthreads();
+    unsigned off, nc;
+    warp_offsets(off, nc);
+    if (nc <= SF_CAND) {
+      for (int w = w0; w < w1; ++w) {
+        const int i = w * 32 + lane;
+        const uint32_t key = i < n ? s_keys[i] : 0u;
+        const bool c = i < n && (key & mask) == prefix;
+        const unsigned bal = __ballot_sync(0xffffffffu, c);
+        if (c) s_cand[off + __popc(bal & lt)] = key;
+        off += __popc(bal);
+      }
+      __syncthreads();
+      // ---- warp 0: the kk-th largest candidate by bisection on the low 21
+      // bits (count of candidates >= a trial key, one warp reduction each) ----
+      if (warp == 0) {
+        constexpr int KR = 16;  // candidates per lane held in registers
+        uint32_t ck[KR];
+        const bool in_regs = nc <= 32u * KR;
+#pragma unroll
+        for (int q = 0; q < KR; ++q) {
+          const unsigned i = q * 32u + lane;
+          ck[q] = (in_regs && i < nc) ? s_cand[i] : 0u;
+        }
+        auto count_ge = [&](uint32_t t) {
+          unsigned c = 0u;
+          if (in_regs) {
+#pragma unroll
+            for (int q = 0; q < KR; ++q) c += (q * 32u + lane < nc) && ck[q] >= t;
+          } else {
+            for (unsigned i = lane; i < nc; i += 32u) c += s_cand[i] >= t;
+          }
+          return __reduce_add_sync(0xffffffffu, c);
+        };
+        uint32_t T = prefix;
+#pragma unroll 1
+        for (int bit = 20; bit >= 0; --bit) {
+          const uint32_t t = T | (1u << bit);
+          if (count_ge(t) >= kk) T = t;
+        }
+        // T is the kk-th largest candidate key; c_gt keys above it
+        const unsigned c_ge = count_ge(T), c_gt = (T == 0xffffffffu) ? 0u : count_ge(T + 1u);
+        if (lane == 0) {
+          s_digit = T;
+          s_kk = kk - c_gt;
+          s_ncand = c_ge - c_gt;  // keys equal to T
+        }
+      }
+      __syncthreads();
+      prefix = s_digit;
+      mask = 0xffffffffu;
+      kk = s_kk;
+      take_all_eq = (kk == s_ncand);
+    } else {
+      // many keys in the boundary bin: two more digit passes over all keys
+#pragma unroll 1
+      for (int pass = 1; pass < 3; ++pass) {
+        const int shift = pass == 1 ? 10 : 0;
+        const unsigned dmask = pass == 2 ? 0x3ffu : 0x7ffu;
         for (int i = tid; i < SEL_BINS; i += SEL_THREADS) s_h[i] = 0u;
         __syncthreads();
-        const int nc = use_cand ? (int)s_ncand : n;
-        const uint32_t* src = use_cand ? s_cand : s_keys;
-        for (int i0 = 0; i0 < nc; i0 += SEL_THREADS) {
+        for (int i0 = 0; i0 < n; i0 += SEL_THREADS) {
           const int i = i0 + tid;
-          const uint32_t key = i < nc ? src[i] : 0u;
-          const bool in = i < nc && (key & mask) == prefix;
+          const uint32_t key = i < n ? s_keys[i] : 0u;
+          const bool in = i < n && (key & mask) == prefix;
           const unsigned bin = in ? (key >> shift) & dmask : 0xffffffffu;
           const unsigned peers = __match_any_sync(0xffffffffu, bin);
           if (in && (__ffs(peers) - 1) == lane) atomicAdd(&s_h[bin], (unsigned)__popc(peers));
         }
         __syncthreads();
-      }
-      const unsigned c0 = s_h[SEL_BINS - 1 - 2 * tid], c1 = s_h[SEL_BINS - 2 - 2 * tid];
-      unsigned tot;
-      const unsigned above = block_exclusive_scan<SEL_THREADS>(c0 + c1, sc, &tot);
-      if (above < kk && kk <= above + c0 + c1) {
-        if (kk <= above + c0) {
-          s_digit = SEL_BINS - 1 - 2 * tid;
-          s_kk = kk - above;
-        } else {
-          s_digit = SEL_BINS - 2 - 2 * tid;
-          s_kk = kk - above - c0;
-        }
-      }
-      __syncthreads();
-      prefix |= s_digit << shift;
-      mask |= dmask << shift;
-      kk = s_kk;
-      if (pass == 0) {  // the keys of the boundary bin, in index order
-        // each warp counts its words' candidates, a scan over the warps gives
-        // the offsets, then each warp writes its own (no shared counter: one
-        // address hit by every warp serialises)
-        unsigned cnt = 0u;
-        for (int w = w0; w < w1; ++w) {
-          const int i = w * 32 + lane;
-          const bool c = i < n && (s_keys[i] & mask) == prefix;
-          cnt += __popc(__ballot_sync(0xffffffffu, c));
-        }
-        if (lane == 0) sc[warp] = cnt;
-        __syncthreads();
-        if (warp == 0) {
-          const unsigned v = sc[lane];
-          unsigned incl = v;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += t;
+        const unsigned c0 = s_h[SEL_BINS - 1 - 2 * tid], c1 = s_h[SEL_BINS - 2 - 2 * tid];
+        unsigned tot;
+        const unsigned above = block_exclusive_scan<SEL_THREADS>(c0 + c1, sc, &tot);
+        if (above < kk && kk <= above + c0 + c1) {
+          if (kk <= above + c0) {
+            s_digit = SEL_BINS - 1 - 2 * tid;
+            s_kk = kk - above;
+          } else {
+            s_digit = SEL_BINS - 2 - 2 * tid;
+            s_kk = kk - above - c0;
           }
-          sc[lane] = incl - v;
-          if (lane == 31) s_ncand = incl;
         }
         __syncthreads();
-        unsigned at = sc[warp];
-        for (int w = w0; w < w1; ++w) {
-          const int i = w * 32 + lane;
-          const uint32_t key = i < n ? s_keys[i] : 0u;
-          const bool c = i < n && (key & mask) == prefix;
-          const unsigned bal = __ballot_sync(0xffffffffu, c);
-          const unsigned mine = at + __popc(bal & ((1u << lane) - 1u));
-          if (c && mine < SF_CAND) s_cand[mine] = key;
-          at += __popc(bal);
-        }
-        __syncthreads();
-        use_cand = s_ncand <= SF_CAND;
+        prefix |= s_digit << shift;
+        mask |= dmask << shift;
+        kk = s_kk;
       }
     }
+    // ---- the row's bitmap: keys above the threshold key T = prefix, plus the
+    // kk lowest-index keys equal to it ----
     if (take_all_eq) {
       for (int w = w0; w < w1; ++w) {
         const int i = w * 32 + lane;
@@ -401,43 +407,34 @@ __global__ void __launch_bounds__(SEL_THREADS) select_finish_kernel(SelectFinish
         if (lane == 0) s_bm[w] = word;
       }
     } else {
-    unsigned eq = 0;
-    for (int w = w0; w < w1; ++w) {
-      const int i = w * 32 + lane;
-      eq += __popc(__ballot_sync(0xffffffffu, i < n && s_keys[i] == prefix));
-    }
-    if (lane == 0) sc[warp] = eq;
-    __syncthreads();
-    if (warp == 0) {
-      const unsigned v = sc[lane];
-      unsigned incl = v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
+      unsigned eq = 0u;
+      for (int w = w0; w < w1; ++w) {
+        const int i = w * 32 + lane;
+        eq += __popc(__ballot_sync(0xffffffffu, i < n && s_keys[i] == prefix));
       }
-      sc[lane] = incl - v;
-    }
-    __syncthreads();
-    unsigned rank = sc[warp];
-    for (int w = w0; w < w1; ++w) {
-      const int i = w * 32 + lane;
-      const bool ok = i < n;
-      const uint32_t key = ok ? s_keys[i] : 0u;
-      const bool e = ok && key == prefix;
-      const unsigned em = __ballot_sync(0xffffffffu, e);
-      const unsigned rk = rank + __popc(em & ((1u << lane) - 1u));
-      const unsigned word = __ballot_sync(0xffffffffu, ok && (key > prefix || (e && rk < kk)));
-      if (lane == 0) s_bm[w] = word;
-      rank += __popc(em);
-    }
+      __syncthreads();  // s_wcnt is rewritten
+      if (lane == 0) s_wcnt[warp] = eq;
+      __syncthreads();
+      unsigned rank, tot_eq;
+      warp_offsets(rank, tot_eq);
+      for (int w = w0; w < w1; ++w) {
+        const int i = w * 32 + lane;
+        const bool ok = i < n;
+        const uint32_t key = ok ? s_keys[i] : 0u;
+        const bool e = ok && key == prefix;
+        const unsigned em = __ballot_sync(0xffffffffu, e);
+        const unsigned rk = rank + __popc(em & lt);
+        const unsigned word = __ballot_sync(0xffffffffu, ok && (key > prefix || (e && rk < kk)));
+        if (lane == 0) s_bm[w] = word;
+        rank += __popc(em);
+      }
     }
   }
-  __syncthreads();
   // union over the neuron rows: with one row the CTA's own bitmap is the
   // union; otherwise the rows' bitmaps meet in global memory and the last
   // CTA (ticket) ORs them, loading every word at once
   if (a.neuron_rows > 1) {
+    __syncthreads();
     for (int w = tid; w < nw; w += SEL_THREADS) bm[w] = s_bm[w];
     __threadfence();
     __syncthreads();
@@ -453,30 +450,23 @@ __global__ void __launch_bounds__(SEL_THREADS) select_finish_kernel(SelectFinish
     __syncthreads();
     if (tid == 0) *a.ticket = 0u;
   }
-  unsigned pc = 0;
+  // idx: each warp writes the set bits of its own words in ascending order
+  __syncwarp();
+  unsigned pc = 0u;
   for (int w = w0; w < w1; ++w) pc += __popc(s_bm[w]);
-  if (lane == 0) sc[warp] = pc;
+  __syncthreads();  // s_wcnt is rewritten
+  if (lane == 0) s_wcnt[warp] = pc;
   __syncthreads();
-  if (warp == 0) {
-    const unsigned v = sc[lane];
-    unsigned incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    sc[lane] = incl - v;
-    if (lane == 31) sc[SEL_WARPS] = incl;
-  }
-  __syncthreads();
-  unsigned off = sc[warp];
+  unsigned out_off, total;
+  warp_offsets(out_off, total);
   for (int w = w0; w < w1; ++w) {
     const uint32_t u = s_bm[w];
-    if ((u >> lane) & 1u) a.idx[off + __popc(u & ((1u << lane) - 1u))] = w * 32 + lane;
-    off += __popc(u);
+    if ((u >> lane) & 1u) a.idx[out_off + __popc(u & lt)] = w * 32 + lane;
+    out_off += __popc(u);
   }
-  if (tid == 0) *a.count = (int32_t)sc[SEL_WARPS];
+  if (tid == 0) *a.count = (int32_t)total;
 }
+
 
 // ----------------------------------------------------------------------------
 // Gate: returns once the previous kernel on its stream has completed and its

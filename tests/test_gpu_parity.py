@@ -504,7 +504,7 @@ def test_predict_layer_matches_oracle(name):
     no_device_errors(ws)
 
 
-@pytest.mark.parametrize("name,group", [("opt-like", 8), ("opt-like", 0), ("ragged", 0), ("wide", 7)])
+@pytest.mark.parametrize("name,group", [("opt-like", 8), ("opt-like", 2), ("opt-like", 0), ("ragged", 0), ("wide", 7)])
 def test_predict_layer_ties_at_threshold(name, group):
     """Neuron scores with many exact ties at the k-th value (Bm rows and b1
     repeated in groups; group 0: every score equal): the selection takes the
