@@ -108,7 +108,8 @@ _lib_dv_decode_layer_begin_ahead = _sig("dv_decode_layer_begin_ahead", _c_int,
                                          _c_size, _p])
 _lib_dv_predict_layer_tail = _sig("dv_predict_layer_tail", _c_int,
                                   [ctypes.POINTER(LayerWeightsC), ctypes.POINTER(Dims), ctypes.POINTER(LayerParamsC),
-                                   ctypes.POINTER(LayerIOC), _p, _c_size, _p])
+                                   ctypes.POINTER(LayerIOC), _c_int, _p, _c_size, _p])
+DV_SET_HEADS, DV_SET_NEURONS = 1, 2
 _lib_dv_layernorm = _sig("dv_layernorm", _c_int, [_p, _c_int, _c_int, _p, _p, _c_float, _p, _p])
 _lib_dv_topk_static = _sig("dv_topk_static", _c_int, [_p, _c_int, _c_int, _c_int, _c_float, _c_int, _p, _p, _p])
 _lib_dv_prefetch_layer = _sig("dv_prefetch_layer", _c_int,
@@ -345,10 +346,11 @@ def dv_decode_layer_begin_ahead(layer: Layer, p: LayerParamsC, x, pos, ws, nxt: 
         _ptr(next_ws, torch.uint8, "next_ws"), next_ws.numel(), _stream(stream)), "dv_decode_layer_begin_ahead")
 
 
-def dv_predict_layer_tail(layer: Layer, p: LayerParamsC, out: LayerIOC, ws, stream=None):
+def dv_predict_layer_tail(layer: Layer, p: LayerParamsC, out: LayerIOC, ws, sets=DV_SET_HEADS | DV_SET_NEURONS,
+                          stream=None):
     _check(_lib_dv_predict_layer_tail(ctypes.byref(layer.c), ctypes.byref(layer.dims), ctypes.byref(p),
-                                      ctypes.byref(out), _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)),
-           "dv_predict_layer_tail")
+                                      ctypes.byref(out), int(sets), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+                                      _stream(stream)), "dv_predict_layer_tail")
 
 
 def dv_prefetch_layer(layer: Layer, sel: LayerIOC, pos, with_w2=True, stream=None):

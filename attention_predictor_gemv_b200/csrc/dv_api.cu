@@ -659,24 +659,29 @@ dv_status dv_decode_layer_begin_ahead(const dv_layer_weights* w, const dv_dims* 
 }
 
 dv_status dv_predict_layer_tail(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p,
-                                const dv_layer_io* out, void* ws, size_t ws_bytes, dv_stream_t stream) {
+                                const dv_layer_io* out, int sets, void* ws, size_t ws_bytes, dv_stream_t stream) {
   DV_CHECK(check_layer(w, dims, p));
   const dv_dims& D = *dims;
-  if (!out || !out->scores_h || !out->head_idx || !out->head_count || !out->scores || !out->idx || !out->count)
-    return DV_ERR_ARG;
-  if (!ok_ptr(out->scores) || !ok_ptr(out->scores_h)) return DV_ERR_ALIGN;
+  const bool heads = (sets & DV_SET_HEADS) != 0, neurons = (sets & DV_SET_NEURONS) != 0;
+  if (!out || sets < 1 || sets > (DV_SET_HEADS | DV_SET_NEURONS)) return DV_ERR_ARG;
+  if (heads && (!out->scores_h || !out->head_idx || !out->head_count)) return DV_ERR_ARG;
+  if (neurons && (!out->scores || !out->idx || !out->count)) return DV_ERR_ARG;
+  if ((heads && !ok_ptr(out->scores_h)) || (neurons && !ok_ptr(out->scores))) return DV_ERR_ALIGN;
   const Layout L = layout(D, wbytes_of(w->wdtype));
   DV_CHECK(check_ws(L, ws, ws_bytes));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (fused_ok(D, w->wdtype)) {
-    DV_CHECK(fused_predict_rest(L, ws, w, D, p, true, true, out->scores_h, out->head_idx, out->head_count,
+    DV_CHECK(fused_predict_rest(L, ws, w, D, p, heads, neurons, out->scores_h, out->head_idx, out->head_count,
                                 out->scores, out->idx, out->count, st));
   } else {
-    DV_TRY(run_select(out->scores_h, D.B, D.h, p->k_h, p->tau_h, p->mode_h, at<uint32_t>(ws, L.bm_h),
-                      at<unsigned>(ws, L.sel_ticket_h), out->head_idx, out->head_count, st));
-    DV_TRY(run_gemv(w->wdtype, w->Bm, D.N, D.r, at<float>(ws, L.z), D.r, D.B, w->b1, out->scores, D.N, st));
-    DV_TRY(run_select(out->scores, D.B, D.N, p->k, p->tau, p->mode, at<uint32_t>(ws, L.bm_m),
-                      at<unsigned>(ws, L.sel_ticket_m), out->idx, out->count, st));
+    if (heads)
+      DV_TRY(run_select(out->scores_h, D.B, D.h, p->k_h, p->tau_h, p->mode_h, at<uint32_t>(ws, L.bm_h),
+                        at<unsigned>(ws, L.sel_ticket_h), out->head_idx, out->head_count, st));
+    if (neurons) {
+      DV_TRY(run_gemv(w->wdtype, w->Bm, D.N, D.r, at<float>(ws, L.z), D.r, D.B, w->b1, out->scores, D.N, st));
+      DV_TRY(run_select(out->scores, D.B, D.N, p->k, p->tau, p->mode, at<uint32_t>(ws, L.bm_m),
+                        at<unsigned>(ws, L.sel_ticket_m), out->idx, out->count, st));
+    }
   }
   return cuda_status(launch(gate_kernel, dim3(1), dim3(32), 0, st));
 }

@@ -3,9 +3,12 @@
 "Deja Vu: 利用上下文稀疏性提升大语言模型推理效率", §1: consecutive layers see
 similar inputs (residual connections), so the sets of layer l+1 are predicted
 from layer l's input, asynchronously, off the critical path. Here the
-predictor of layer l+1 runs on a side CUDA stream from layer l's normalised
-attention input yA_l while the main stream runs layer l's sparse blocks; layer
-l+1 waits on an event for its sets. Layer 0 predicts its own sets.
+predictor of layer l+1 reads layer l's normalised attention input yA_l: its
+first stage (head scores and z = yA_l A) runs inside layer l's q/k/v kernel,
+the head selection on one side stream and the neuron scores and selection on
+another, while the main stream runs layer l's sparse blocks; layer l+1 waits
+on one event for its head set before its q/k/v and on another for its neuron
+set before its MLP. Layer 0 predicts its own sets.
 
 This module only orders library calls on streams (events, waits); every
 arithmetic step runs in libdejavu's kernels. A step can be captured into a
@@ -40,10 +43,15 @@ class DecoderStack:
         self.prefetch = prefetch and lookahead
         self.prefetch_w2 = prefetch_w2
         # the predictor's first stage for layer l+1 inside layer l's q/k/v kernel
-        self.fuse_ahead = fuse_ahead
+        # (the L2 prefetch option keeps the one-call predictor on one side stream)
+        self.fuse_ahead = fuse_ahead and not self.prefetch
         D = self.layers[0].dims
         self.ws_main = bd.workspace(bd.DV_OP_DECODE_LAYER, D, dev)
         self.ws_side = bd.workspace(bd.DV_OP_DECODE_LAYER, D, dev)
+        # fused look-ahead: layer l+1's z and selection scratch live in the
+        # side workspace of l+1's parity, so layer l+1's q/k/v kernel (which
+        # writes z for l+2) never overwrites a z that is still being read
+        self.ws_ahead = [self.ws_side, bd.workspace(bd.DV_OP_DECODE_LAYER, D, dev)] if self.fuse_ahead else []
         nL = len(layers)
         i32 = dict(dtype=torch.int32, device=dev)
         f32 = dict(dtype=torch.float32, device=dev)
@@ -70,12 +78,18 @@ class DecoderStack:
         # ... and writes its normalised block inputs here
         self.io_trace_y = [bd.layer_io(yA=self.yA[l], yM=self.yM[l]) for l in range(nL)]
         self.side = torch.cuda.Stream(device=dev)
+        self.side_m = torch.cuda.Stream(device=dev)  # fused look-ahead: the neuron sets
+        self.ev_heads = [torch.cuda.Event() for _ in range(nL)]
+        self.ev_neurons = [torch.cuda.Event() for _ in range(nL)]
+        self.ev_join_m = torch.cuda.Event()
         self.ev_yA = [torch.cuda.Event() for _ in range(nL)]
         self.ev_sel = [torch.cuda.Event() for _ in range(nL)]
         self.ev_join = torch.cuda.Event()
 
     def step(self, x: torch.Tensor, pos: int):
         """One token through every layer, in place on the residual x [B][d]."""
+        if self.lookahead and self.fuse_ahead and len(self.layers) > 1:
+            return self._step_fused(x, pos)
         main = torch.cuda.current_stream()
         nL = len(self.layers)
         la = self.lookahead and nL > 1
@@ -85,14 +99,9 @@ class DecoderStack:
                 sel, trace = self.io_given[l], self.io_trace_y[l]
             else:
                 sel, trace = None, self.io_trace[l]
-            ahead = la and l + 1 < nL
-            if ahead and self.fuse_ahead:
-                bd.dv_decode_layer_begin_ahead(L, self.p, x, pos, self.ws_main, self.layers[l + 1],
-                                               self.scores_h[l + 1], self.ws_side, sel=sel, trace=trace)
-            else:
-                bd.dv_decode_layer_begin(L, self.p, x, pos, self.ws_main, sel=sel, trace=trace)
-            if ahead:
-                self.ev_yA[l].record(main)  # yA[l] (and the first stage for l+1) written by the work just issued
+            bd.dv_decode_layer_begin(L, self.p, x, pos, self.ws_main, sel=sel, trace=trace)
+            if la and l + 1 < nL:
+                self.ev_yA[l].record(main)  # yA[l] is written by the work just issued
                 self._predict_next(l, pos)
             bd.dv_decode_layer_end(L, self.p, x, pos, self.ws_main, sel=sel, trace=trace)
         if la:
@@ -100,17 +109,51 @@ class DecoderStack:
             self.ev_join.record(self.side)
             main.wait_event(self.ev_join)
 
+    def _step_fused(self, x: torch.Tensor, pos: int):
+        """Look-ahead with the predictor's first stage for layer l+1 inside
+        layer l's q/k/v kernel. Layer l+1 needs its head set before its own
+        q/k/v but its neuron set only before its MLP, so the two selections
+        run on two side streams and the main stream waits for each just
+        before the kernel that reads it."""
+        main = torch.cuda.current_stream()
+        nL = len(self.layers)
+        for l, L in enumerate(self.layers):
+            if l > 0:
+                main.wait_event(self.ev_heads[l])
+                sel, trace = self.io_given[l], self.io_trace_y[l]
+            else:
+                sel, trace = None, self.io_trace[l]
+            if l + 1 < nL:
+                ws_next = self.ws_ahead[(l + 1) % 2]
+                bd.dv_decode_layer_begin_ahead(L, self.p, x, pos, self.ws_main, self.layers[l + 1],
+                                               self.scores_h[l + 1], ws_next, sel=sel, trace=trace)
+                self.ev_yA[l].record(main)  # the first stage for l+1 is written by the work just issued
+                self.side.wait_event(self.ev_yA[l])
+                bd.dv_predict_layer_tail(self.layers[l + 1], self.p, self.io_sets[l + 1], ws_next,
+                                         sets=bd.DV_SET_HEADS, stream=self.side)
+                self.ev_heads[l + 1].record(self.side)
+                self.side_m.wait_event(self.ev_yA[l])
+                bd.dv_predict_layer_tail(self.layers[l + 1], self.p, self.io_sets[l + 1], ws_next,
+                                         sets=bd.DV_SET_NEURONS, stream=self.side_m)
+                self.ev_neurons[l + 1].record(self.side_m)
+            else:
+                bd.dv_decode_layer_begin(L, self.p, x, pos, self.ws_main, sel=sel, trace=trace)
+            bd.dv_decode_layer_attn(L, self.p, x, pos, self.ws_main, sel=sel, trace=trace)
+            if l > 0:
+                main.wait_event(self.ev_neurons[l])
+            bd.dv_decode_layer_mlp(L, self.p, x, self.ws_main, sel=sel, trace=trace)
+        self.ev_join.record(self.side)
+        main.wait_event(self.ev_join)
+        self.ev_join_m.record(self.side_m)
+        main.wait_event(self.ev_join_m)
+
     def _predict_next(self, l: int, pos: int):
         """Side stream: the sets of layer l+1 from layer l's yA, then an L2
         prefetch of the parameters those sets select (layer l+1 runs after
         layer l on the main stream, and finds them in L2)."""
         self.side.wait_event(self.ev_yA[l])
-        if self.fuse_ahead:
-            bd.dv_predict_layer_tail(self.layers[l + 1], self.p, self.io_sets[l + 1], self.ws_side,
-                                     stream=self.side)
-        else:
-            bd.dv_predict_layer(self.layers[l + 1], self.p, self.yA[l], self.io_sets[l + 1], self.ws_side,
-                                stream=self.side)
+        bd.dv_predict_layer(self.layers[l + 1], self.p, self.yA[l], self.io_sets[l + 1], self.ws_side,
+                            stream=self.side)
         self.ev_sel[l + 1].record(self.side)
         if self.prefetch:
             bd.dv_prefetch_layer(self.layers[l + 1], self.io_sets[l + 1], pos, with_w2=self.prefetch_w2,

@@ -290,18 +290,26 @@ DV_API dv_status dv_predict_layer(const dv_layer_weights* w, const dv_dims* dims
  * for DV_OP_DECODE_LAYER with the same dims; it must not be ws).
  *
  * dv_predict_layer_tail then completes the prediction for that layer on any
- * stream ordered after the begin_ahead call: neuron scores z B^T + b1 and
- * both selections, written like dv_predict_layer; out->scores_h must be the
- * next_scores_h given to begin_ahead and ws its next_ws. Together the two
- * calls give the same scores and sets as dv_predict_layer(next, y). Its last
- * launch is the same gate as dv_predict_layer's. */
+ * stream ordered after the begin_ahead call: `sets` = DV_SET_HEADS, the head
+ * selection from next_scores_h; DV_SET_NEURONS, the neuron scores
+ * z B^T + b1 and their selection; or both. It writes the chosen sets' fields
+ * of `out` like dv_predict_layer (out->scores_h must be the next_scores_h
+ * given to begin_ahead, ws its next_ws). The head part and the neuron part
+ * may run as two calls on two streams (they use disjoint parts of ws): the
+ * next layer needs its head set before its q, k, v but its neuron set only
+ * before its MLP. Together the calls give the same scores and sets as
+ * dv_predict_layer(next, y). Each call ends with the same gate as
+ * dv_predict_layer. Until the neuron part has completed, ws must not be
+ * given to another begin_ahead call. */
 DV_API dv_status dv_decode_layer_begin_ahead(const dv_layer_weights* w, const dv_dims* dims,
                                              const dv_layer_params* p, float* x, int pos, const dv_layer_io* sel,
                                              const dv_layer_io* trace, void* ws, size_t ws_bytes,
                                              const dv_layer_weights* next, float* next_scores_h, void* next_ws,
                                              size_t next_ws_bytes, dv_stream_t stream);
+enum { DV_SET_HEADS = 1, DV_SET_NEURONS = 2 };
 DV_API dv_status dv_predict_layer_tail(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p,
-                                       const dv_layer_io* out, void* ws, size_t ws_bytes, dv_stream_t stream);
+                                       const dv_layer_io* out, int sets, void* ws, size_t ws_bytes,
+                                       dv_stream_t stream);
 
 /* L2 prefetch of one layer's selected parameters (§1: for the next layer
  * the look-ahead predictor picks the heads / neurons and only those

@@ -535,8 +535,9 @@ def test_predict_layer_ties_at_threshold(name, group):
     no_device_errors(ws)
 
 
-@pytest.mark.parametrize("name,B", [("opt-like", 1), ("fused128", 2), ("ragged", 1), ("wide", 1), ("tiny", 3)])
-def test_begin_ahead_and_tail_predict_next_layer(name, B):
+@pytest.mark.parametrize("name,B,split", [("opt-like", 1, True), ("opt-like", 1, False), ("fused128", 2, True),
+                                          ("ragged", 1, True), ("wide", 1, True), ("tiny", 3, False)])
+def test_begin_ahead_and_tail_predict_next_layer(name, B, split):
     """The next layer's predictor split over begin_ahead (its first stage in
     this layer's q/k/v kernel) and predict_layer_tail: scores of layer 2 from
     layer 1's yA, sets = the oracle's selection of those scores, and layer 1's
@@ -562,7 +563,14 @@ def test_begin_ahead_and_tail_predict_next_layer(name, B):
     bd.dv_decode_layer_begin_ahead(L1, p, x, s.L, ws1, L2, tb2["scores_h"], ws2, trace=bd.layer_io(**tb1))
     out2 = bd.layer_io(scores_h=tb2["scores_h"], head_idx=tb2["head_idx"], head_count=tb2["head_count"],
                        scores=tb2["scores"], idx=tb2["idx"], count=tb2["count"])
-    bd.dv_predict_layer_tail(L2, p, out2, ws2)
+    if split:  # the head part and the neuron part on two streams, as the stack runs them
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        bd.dv_predict_layer_tail(L2, p, out2, ws2, sets=bd.DV_SET_HEADS)
+        bd.dv_predict_layer_tail(L2, p, out2, ws2, sets=bd.DV_SET_NEURONS, stream=side)
+        torch.cuda.current_stream().wait_stream(side)
+    else:
+        bd.dv_predict_layer_tail(L2, p, out2, ws2)
     torch.cuda.synchronize()
     yA = f64(tb1["yA"])
     sh, sm = tb2["scores_h"].cpu().numpy(), tb2["scores"].cpu().numpy()
