@@ -111,15 +111,17 @@ class DecoderStack:
 
     def _step_fused(self, x: torch.Tensor, pos: int):
         """Look-ahead with the predictor's first stage for layer l+1 inside
-        layer l's q/k/v kernel. Layer l+1 needs its head set before its own
-        q/k/v but its neuron set only before its MLP, so the two selections
-        run on two side streams and the main stream waits for each just
-        before the kernel that reads it."""
+        layer l's q/k/v kernel. The head selection runs on one side stream and
+        the neuron scores and selection on another. Both waits of the main
+        stream sit just before layer l's MLP kernel: the neuron set of layer l
+        is read there, and the head set of layer l+1 is read by layer l+1's
+        q/k/v kernel, which follows the MLP kernel with programmatic launch
+        (a kernel after a cross-stream wait cannot launch early, so no wait
+        sits in front of the q/k/v or attention kernels)."""
         main = torch.cuda.current_stream()
         nL = len(self.layers)
         for l, L in enumerate(self.layers):
             if l > 0:
-                main.wait_event(self.ev_heads[l])
                 sel, trace = self.io_given[l], self.io_trace_y[l]
             else:
                 sel, trace = None, self.io_trace[l]
@@ -141,6 +143,8 @@ class DecoderStack:
             bd.dv_decode_layer_attn(L, self.p, x, pos, self.ws_main, sel=sel, trace=trace)
             if l > 0:
                 main.wait_event(self.ev_neurons[l])
+            if l + 1 < nL:
+                main.wait_event(self.ev_heads[l + 1])
             bd.dv_decode_layer_mlp(L, self.p, x, self.ws_main, sel=sel, trace=trace)
         self.ev_join.record(self.side)
         main.wait_event(self.ev_join)
