@@ -132,7 +132,10 @@ __global__ void __launch_bounds__(256) prefetch_layer_kernel(PrefetchArgs a) {
 // and writes idx / count. CTA B (when heads are predicted) selects the heads
 // from their scores by rank (few heads: direct comparison).
 // ----------------------------------------------------------------------------
-constexpr int SF_CAND = 2048;  // keeps static + dynamic shared memory within 227 KB at N = 49152
+// Boundary-bin keys held in shared memory. They share one array with the
+// digit histogram, which is no longer read once they are written, so that
+// static plus dynamic shared memory stays within 227 KB at N = 49152.
+constexpr int SF_CAND = 4096;
 
 struct SelectFinishArgs {
   const float* scores;  // [B][N]
@@ -153,8 +156,9 @@ struct SelectFinishArgs {
 
 __global__ void __launch_bounds__(SEL_THREADS) select_finish_kernel(SelectFinishArgs a) {
   extern __shared__ uint32_t s_keys[];  // [N] for a neuron row, [h] for the head row
-  __shared__ unsigned s_h[SEL_BINS];
-  __shared__ uint32_t s_cand[SF_CAND];
+  __shared__ uint32_t s_hc[SF_CAND > SEL_BINS ? SF_CAND : SEL_BINS];
+  unsigned* s_h = s_hc;      // [SEL_BINS] digit histogram
+  uint32_t* s_cand = s_hc;   // [SF_CAND] boundary-bin keys (after the top digit is known)
   __shared__ uint32_t s_hsel[HSEL_MAX / 32];
   __shared__ uint32_t s_bm[SEL_SMEM_KEYS / 32];
   __shared__ unsigned sc[SEL_WARPS + 1];

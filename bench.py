@@ -228,6 +228,37 @@ def graph_of(fn):
     return g
 
 
+# Source headers of each main-path kernel, for matching a committed ncu
+# capture to the code that runs now.
+KERNEL_HEADERS = {
+    "attn_in": ("dv_common.cuh", "dv_fused.cuh", "dv_colowner.cuh"),
+    "mlp_block": ("dv_common.cuh", "dv_fused.cuh", "dv_colowner.cuh"),
+    "attn_out": ("dv_common.cuh", "dv_kernels.cuh", "dv_fused.cuh"),
+}
+
+
+def measured_traffic(op):
+    """Per-launch DRAM bytes (read + write) of `op`'s kernel from the ncu
+    summary under profiles/ (lines `traffic <op> <bytes> <sha256 prefix>`),
+    or None when no capture exists or the kernel's headers changed since."""
+    import glob
+    import hashlib
+
+    csrc = os.path.join(ROOT, "attention_predictor_gemv_b200", "csrc")
+    h = hashlib.sha256()
+    for f in KERNEL_HEADERS.get(op, ()):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    digest = h.hexdigest()[:16]
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        with open(path) as fh:
+            for line in fh:
+                parts = line.split()
+                if len(parts) == 4 and parts[0] == "traffic" and parts[1] == op and parts[3] == digest:
+                    return {"bytes": int(parts[2]), "source": os.path.relpath(path, ROOT)}
+    return None
+
+
 def kernel_roofline(stk, shape, B, pos, peak_gbs, reps=20):
     """Average duration of each main-path kernel in the look-ahead steady
     state (sets given): one CUDA graph per kernel with that kernel's call for
@@ -396,6 +427,7 @@ def main():
 
     ops, lb, kmean, kp, kh = kernel_roofline(stk, shape, B, pos, peak_gbs)
     dom = max(ops, key=lambda n: ops[n]["us"])
+    traffic = measured_traffic(dom)
     total_layer_bytes = lb.total
     us_layer = ms * 1e3 / args.layers
     value = ms * 1e3 / (args.layers * world)  # whole job: all ranks' layer-steps in the max-over-ranks time
@@ -435,7 +467,9 @@ def main():
         "effective_gbs": total_layer_bytes / us_layer / 1e3,
         "effective_frac": total_layer_bytes / us_layer / 1e3 / peak_gbs,
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": ops[dom]["gbs"], "peak": peak_gbs, "unit": "GB/s",
-                     "frac": ops[dom]["frac"], "traffic": None, "peak_source": peak_src, "per_op": ops},
+                     "frac": ops[dom]["frac"], "traffic": traffic["bytes"] if traffic else None,
+                     "traffic_source": traffic["source"] if traffic else None,
+                     "algorithmic_bytes": ops[dom]["bytes"], "peak_source": peak_src, "per_op": ops},
         "e2e": {"value": e2e_ms * 1e3 / (args.layers * world), "unit": "us", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": xh.numel() * 4, "d2h_bytes_per_step": oh.numel() * 4},
         "gpu_launches": int(launches_per_step * args.steps),
