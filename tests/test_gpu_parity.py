@@ -331,7 +331,7 @@ def _trace_bufs(s):
 
 
 @pytest.mark.parametrize("name,B", [("tiny", 1), ("ragged", 3), ("opt-like", 1), ("opt-like", 4), ("fused128", 1),
-                                    ("fused128", 3), ("tiny", 2)])
+                                    ("fused128", 3), ("tiny", 2), ("fused128", 6)])
 def test_decode_layer(name, B):
     s, t = layer(name, B, seed=11)
     t["ln1_g"] = 1.0 + 0.1 * torch.randn(s.d, device=DEV)
