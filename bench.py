@@ -73,21 +73,28 @@ def dist_init():
 
     rank = int(os.environ["RANK"])
     local = int(os.environ.get("LOCAL_RANK", rank))
-    torch.cuda.set_device(local)
-    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:  # host-only ranks (the reference arm, tests): gloo
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
     return rank, ws, dist
 
 
 def barrier(dist):
     if dist is not None:
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def max_over_ranks(v, dist):
+    """The largest of the ranks' values (every rank gets it)."""
     if dist is None:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -359,7 +366,7 @@ def run_reference(args, rank, dist):
     if rank != 0:
         return
     per_step = max(1.0, 60.0 / max(1, args.steps + args.warmup))
-    cb = cpu_baseline(shape, args.batch, k, k_h, min(per_step, 10.0))
+    cb = cpu_baseline(shape, args.batch, k, k_h, min(per_step, args.cpu_seconds))
     v = cb["value"]
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "us", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": v * args.layers / 1e3,
