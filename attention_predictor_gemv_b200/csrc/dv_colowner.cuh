@@ -62,38 +62,36 @@ __device__ __forceinline__ void x_slice_load(const float* __restrict__ x, int d,
 }
 
 // LayerNorm of the slices in place: (x - mean) / sqrt(var + eps) * g + beta,
-// mean and biased variance over the d columns of each batch row. Columns
-// outside the row stay zero.
+// mean and biased variance over the d columns of each batch row, both from
+// one CTA reduction of the sums of x and x^2 (var = E[x^2] - mean^2 in fp32:
+// the block inputs have |mean| of the order of their spread, far from the
+// cancellation regime). Columns outside the row stay zero. red holds
+// 2 NB CO_WARPS floats.
 template <typename T, int NB, int NV>
 __device__ __forceinline__ void x_slice_ln(float (&xr)[NB][NV][WT<T>::E], int d, float eps, const float* g,
                                            const float* beta, float* red) {
   constexpr int E = WT<T>::E;
-  float s[NB];
+  float sq[2 * NB];
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
-    s[b] = 0.f;
+    float s1 = 0.f, s2 = 0.f;
 #pragma unroll
     for (int j = 0; j < NV; ++j)
 #pragma unroll
-      for (int e = 0; e < E; ++e) s[b] += xr[b][j][e];
+      for (int e = 0; e < E; ++e) {
+        s1 += xr[b][j][e];
+        s2 = fmaf(xr[b][j][e], xr[b][j][e], s2);
+      }
+    sq[b] = s1;
+    sq[NB + b] = s2;
   }
-  block_sum_n<NB>(s, red);
-  float q[NB];
+  block_sum_n<2 * NB>(sq, red);
+  float s[NB], q[NB];
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
-    s[b] /= (float)d;
-    q[b] = 0.f;
-#pragma unroll
-    for (int j = 0; j < NV; ++j) {
-      const bool ok = (j * CO_THREADS + (int)threadIdx.x) * E < d;
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const float t = xr[b][j][e] - s[b];
-        q[b] += ok ? t * t : 0.f;
-      }
-    }
+    s[b] = sq[b] / (float)d;
+    q[b] = fmaxf(sq[NB + b] / (float)d - s[b] * s[b], 0.f) * (float)d;
   }
-  block_sum_n<NB>(q, red);
 #pragma unroll
   for (int j = 0; j < NV; ++j) {
     const int c = (j * CO_THREADS + threadIdx.x) * E;
@@ -305,9 +303,14 @@ __global__ void __launch_bounds__(CO_THREADS) attn_in_co_kernel(AttnInArgs a) {
 // ----------------------------------------------------------------------------
 // mlp_block_co_kernel: mlp_block_kernel (LN2, W1 + b1 + ReLU, W2 gather-axpy,
 // residual) in the column-owner layout. CTA g owns selection slots
-// [g*cnt/G, (g+1)*cnt/G), taken R at a time; the W2 rows of the nonzero
-// activations accumulate into the thread's own columns across all chunks and
-// are added to x once at the end. CTA 0 also adds t1 and b2.
+// [g*cnt/G, (g+1)*cnt/G), taken R at a time. A chunk's W2 rows are loaded
+// together with its W1 rows (before griddep_wait for the first chunk), not
+// after the activations are known: the predictor selects the neurons it
+// expects to be active, so their W2 rows are needed, and at these row
+// lengths the kernel is bound by the latency of dependent loads, not by
+// bytes. The W2 rows of nonzero activations accumulate into the thread's own
+// columns across all chunks and are added to x once at the end; CTA 0 also
+// adds t1 and b2.
 // ----------------------------------------------------------------------------
 template <typename T, int NB, int NV, int R>
 __global__ void __launch_bounds__(CO_THREADS) mlp_block_co_kernel(MlpBlockArgs a) {
@@ -315,9 +318,6 @@ __global__ void __launch_bounds__(CO_THREADS) mlp_block_co_kernel(MlpBlockArgs a
   __shared__ float red[(R * NB > 2 * NB ? R * NB : 2 * NB) * CO_WARPS];
   __shared__ float s_out[R * NB];
   __shared__ float s_act[R][NB];
-  __shared__ int s_row[R];
-  __shared__ int s_list[R];
-  __shared__ int s_nlist;
   const T* W1t = static_cast<const T*>(a.W1t);
   const T* W2t = static_cast<const T*>(a.W2t);
   const int nvec = a.d / E;
@@ -333,8 +333,8 @@ __global__ void __launch_bounds__(CO_THREADS) mlp_block_co_kernel(MlpBlockArgs a
     j1 = (int)(((long long)cnt * (blockIdx.x + 1)) / a.G);
   };
   const T* rowp[R];
+  const T* rowp2[R];
   bool valid[R];
-  int rows[R];
   float bias[R];
   auto setup_rows = [&](int base) {
 #pragma unroll
@@ -345,23 +345,27 @@ __global__ void __launch_bounds__(CO_THREADS) mlp_block_co_kernel(MlpBlockArgs a
         if (threadIdx.x == 0) raise_status(a.status, 2);
         row = -1;
       }
-      rows[r] = row;
       valid[r] = row >= 0;
       rowp[r] = W1t + (size_t)(row >= 0 ? row : 0) * a.d;
+      rowp2[r] = W2t + (size_t)(row >= 0 ? row : 0) * a.d;
       bias[r] = row >= 0 ? a.b1[row] : 0.f;
     }
   };
-  uint4 w[R][NV];
+  uint4 w[R][NV], w2[R][NV];
+  auto issue = [&]() {
+    co_issue<T, NV, R>(w, rowp, valid, nvec);
+    co_issue<T, NV, R>(w2, rowp2, valid, nvec);
+  };
   if (a.sets_ready) {
     slot_range();
     setup_rows(j0);
-    co_issue<T, NV, R>(w, rowp, valid, nvec);
+    issue();
   }
   griddep_wait();
   if (!a.sets_ready) {
     slot_range();
     setup_rows(j0);
-    co_issue<T, NV, R>(w, rowp, valid, nvec);
+    issue();
   }
   float xr[NB][NV][E];
   x_slice_load<T, NB, NV>(a.t1, a.d, a.nb, xr);
@@ -378,62 +382,38 @@ __global__ void __launch_bounds__(CO_THREADS) mlp_block_co_kernel(MlpBlockArgs a
   for (int c0 = j0; c0 < j1; c0 += R) {
     if (c0 != j0) {
       setup_rows(c0);
-      co_issue<T, NV, R>(w, rowp, valid, nvec);
+      issue();
     }
     co_dot<T, NB, NV, R>(w, xr, red, s_out);
-    if (threadIdx.x < 32) {
-      const int lane = threadIdx.x;
-      int nz = 0;
-      if (lane < R) {
-        const int r = lane;
+    if (threadIdx.x < R * NB) {
+      const int r = threadIdx.x / NB, b = threadIdx.x % NB;
+      float v = 0.f;
 #pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          float v = 0.f;
-          if (b < a.nb) {
-#pragma unroll
-            for (int rr = 0; rr < R; ++rr)
-              if (rr == r) v = valid[rr] ? fmaxf(s_out[r * NB + b] + bias[rr], 0.f) : 0.f;
-          }
-          s_act[r][b] = v;
-          nz |= v > 0.f;
-        }
-#pragma unroll
-        for (int rr = 0; rr < R; ++rr)
-          if (rr == r) s_row[r] = rows[rr];
-      }
-      const unsigned bal = __ballot_sync(0xffffffffu, nz);
-      if (nz) s_list[__popc(bal & ((1u << lane) - 1u))] = lane;
-      if (lane == 0) s_nlist = __popc(bal);
+      for (int rr = 0; rr < R; ++rr)
+        if (rr == r) v = (valid[rr] && b < a.nb) ? fmaxf(s_out[r * NB + b] + bias[rr], 0.f) : 0.f;
+      s_act[r][b] = v;
     }
     __syncthreads();
-    const int nl = s_nlist;
-    uint4 w2[R][NV];
 #pragma unroll
-    for (int i = 0; i < R; ++i)
+    for (int r = 0; r < R; ++r) {
+      bool nz = false;
 #pragma unroll
-      for (int j = 0; j < NV; ++j) {
-        const int v = j * CO_THREADS + threadIdx.x;
-        w2[i][j] = (i < nl && v < nvec) ? ld_stream(W2t + (size_t)s_row[s_list[i]] * a.d + (size_t)v * E)
-                                        : make_uint4(0u, 0u, 0u, 0u);
-      }
-#pragma unroll
-    for (int i = 0; i < R; ++i) {
-      if (i < nl) {
-        const int s = s_list[i];
+      for (int b = 0; b < NB; ++b) nz |= s_act[r][b] > 0.f;
+      if (nz) {  // the same for every thread: zero activations add nothing
 #pragma unroll
         for (int j = 0; j < NV; ++j) {
           float wf[E];
-          WT<T>::unpack(w2[i][j], wf);
+          WT<T>::unpack(w2[r][j], wf);
 #pragma unroll
           for (int b = 0; b < NB; ++b) {
-            const float cb = s_act[s][b];
+            const float cb = s_act[r][b];
 #pragma unroll
             for (int e = 0; e < E; ++e) acc[b][j][e] = fmaf(cb, wf[e], acc[b][j][e]);
           }
         }
       }
     }
-    __syncthreads();  // s_act / s_list are rewritten by the next chunk
+    __syncthreads();  // s_act is rewritten by the next chunk
   }
   const bool residual = blockIdx.x == 0;
   if (j1 == j0 && !residual) return;
