@@ -497,7 +497,12 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_in_kernel(AttnInArgs a) {
 // t1. With WV > 0 the slice (WV 16-byte vectors per thread) is loaded into
 // registers before griddep_wait; with WV = 0 it is streamed afterwards. The
 // cluster of slot 0 also moves the residual: t1 += x (+ bO) on its slices,
-// then x = 0.
+// then x = 0. With WV < 0 (long rows, batch 1-2) CTA c instead multiplies H
+// by whole rows c, c + CS, ... of W_i^O (each thread -WV 16-byte vectors of a
+// row) and adds its full-width partial to t1: on B200 a CTA streaming whole
+// 16-24 KB rows reaches about three times the bandwidth of CTAs that each
+// read a 2-3 KB column slice of every row. CTA 0 of slot 0's cluster then
+// moves the residual over all columns.
 // ----------------------------------------------------------------------------
 struct AttnOutArgs {
   const float* q;
@@ -599,6 +604,10 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
     if constexpr (WV == 0) {
       const char* base = reinterpret_cast<const char*>(WO + (size_t)head * DH * a.d + c_lo);
       for (int i = tid; i < DH; i += FUSED_THREADS) prefetch_l2(base + (size_t)i * a.d * sizeof(KT), cols * sizeof(KT));
+    } else if constexpr (WV < 0) {
+      const char* base = reinterpret_cast<const char*>(WO + (size_t)head * DH * a.d);
+      for (int i = crank + tid * CS; i < DH; i += FUSED_THREADS * CS)
+        prefetch_l2(base + (size_t)i * a.d * sizeof(KT), a.d * sizeof(KT));
     }
   };
   if (a.sets_ready) {
@@ -727,7 +736,9 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
     }
   }
   __syncthreads();
-  const bool residual = (p == 0);
+  // slot 0's cluster moves the residual: every CTA on its own column slice,
+  // or CTA 0 on all columns when CTAs take whole rows
+  const bool residual = (p == 0) && (WV >= 0 || crank == 0);
   if (!active && !residual) return;
   // residual (slot 0's cluster): o += x + bO at columns c..c+E-1, then x = 0
   auto add_residual = [&](float (&o)[E], int b, int c) {
@@ -744,7 +755,64 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
       reinterpret_cast<float4*>(xr)[e4] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
   };
-  if constexpr (WV > 0) {
+  if constexpr (WV < 0) {
+    // ---- whole rows crank, crank + CS, ... of W_i^O; this thread's vectors
+    // tid + 256 j of each row; U rows in flight ----
+    constexpr int NVO = -WV, U = 2;
+    const KT* Wh = WO + (size_t)head * DH * a.d;
+    float o[NB][NVO][E];
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+      for (int j = 0; j < NVO; ++j)
+#pragma unroll
+        for (int e = 0; e < E; ++e) o[b][j][e] = 0.f;
+    if (active) {
+#pragma unroll 1
+      for (int r0 = crank; r0 < DH; r0 += CS * U) {
+        uint4 w[U][NVO];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+          for (int j = 0; j < NVO; ++j) {
+            const int r = r0 + u * CS, v = tid + j * FUSED_THREADS;
+            w[u][j] = (r < DH && v * E < a.d) ? ld_stream(Wh + (size_t)r * a.d + (size_t)v * E)
+                                              : make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int r = r0 + u * CS;
+          if (r < DH) {
+#pragma unroll
+            for (int j = 0; j < NVO; ++j) {
+              float wf[E];
+              WT<KT>::unpack(w[u][j], wf);
+#pragma unroll
+              for (int b = 0; b < NB; ++b) {
+                const float hv = b < a.nb ? s_H[b][r] : 0.f;
+#pragma unroll
+                for (int e = 0; e < E; ++e) o[b][j][e] = fmaf(hv, wf[e], o[b][j][e]);
+              }
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < NVO; ++j) {
+      const int c = (tid + j * FUSED_THREADS) * E;
+      if (c >= a.d) continue;
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        if (b >= a.nb) break;
+        if (residual) add_residual(o[b][j], b, c);
+#pragma unroll
+        for (int e4 = 0; e4 < E / 4; ++e4)
+          red_add4(a.t1 + (size_t)b * a.d + c + 4 * e4,
+                   make_float4(o[b][j][4 * e4], o[b][j][4 * e4 + 1], o[b][j][4 * e4 + 2], o[b][j][4 * e4 + 3]));
+      }
+    }
+  } else if constexpr (WV > 0) {
     // ---- W^O slice from registers; row groups reduced across RG lanes ----
     float o[NB][E];
 #pragma unroll

@@ -230,8 +230,24 @@ cudaError_t run_attn_out_nbw(const AttnOutArgs& a, cudaStream_t st) {
   return launch_cluster(kern, dim3(ATTN_CS, a.kh_max > 0 ? a.kh_max : 1), FUSED_THREADS, smem, st, ATTN_CS, a);
 }
 
+// Whole-row W^O (long rows, bf16, batch 1-2): 16-byte vectors per thread
+// per row, 4-6 (d = 8192-12288); 0 when the path does not apply.
+inline int attn_out_whole_rows(int d, int E, int kvbytes, int nb) {
+  if (nb > 2 || kvbytes != 2 || d % (256 * E) != 0) return 0;
+  const int nvo = d / (256 * E);
+  return (nvo >= 4 && nvo <= 6) ? nvo : 0;
+}
+
 template <typename KT, int DH, int NB>
 cudaError_t run_attn_out_nb(const AttnOutArgs& a, cudaStream_t st) {
+  if constexpr (NB <= 2 && sizeof(KT) == 2) {
+    switch (attn_out_whole_rows(a.d, WT<KT>::E, sizeof(KT), a.nb)) {
+      case 4: return run_attn_out_nbw<KT, DH, NB, -4>(a, st);
+      case 5: return run_attn_out_nbw<KT, DH, NB, -5>(a, st);
+      case 6: return run_attn_out_nbw<KT, DH, NB, -6>(a, st);
+      default: break;
+    }
+  }
   if constexpr (NB <= 4) {
     switch (attn_out_wv(a.d, DH, WT<KT>::E, a.nb)) {
       case 8: return run_attn_out_nbw<KT, DH, NB, 8>(a, st);
