@@ -518,6 +518,7 @@ struct AttnOutArgs {
   int h, dh, d, cap, pos, nb, S, sets_ready;
   float scale;
   int* status;
+  int stage_rows;  // batch rows whose K/V tiles fit in shared memory at once: nb, or 1
 };
 
 __device__ __forceinline__ void cluster_arrive_relaxed() {
@@ -546,9 +547,10 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
   constexpr int PW = DH + 2;   // partial: m, l, acc[DH]
   constexpr int RG = WV > 0 ? DH / WV : 1;  // W^O row groups (register path)
   extern __shared__ __align__(16) unsigned char s_dyn[];
-  KT* sK = reinterpret_cast<KT*>(s_dyn);                          // [S][DH]
-  KT* sV = sK + (size_t)a.S * DH;                                 // [S][DH]
-  float* s_all = reinterpret_cast<float*>(sV + (size_t)a.S * DH);  // [nb][CS][PW]
+  const int SR = a.stage_rows;
+  KT* sK = reinterpret_cast<KT*>(s_dyn);                               // [SR][S][DH]
+  KT* sV = sK + (size_t)SR * a.S * DH;                                 // [SR][S][DH]
+  float* s_all = reinterpret_cast<float*>(sV + (size_t)SR * a.S * DH);  // [nb][CS][PW]
   __shared__ __align__(16) float s_w[FUSED_WARPS][PW];
   __shared__ __align__(16) float s_H[NB][DH];
   __shared__ float s_red[WV > 0 ? 1 : FUSED_THREADS * E];
@@ -583,10 +585,11 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
     const int hi = old_only ? min(nk, a.pos - t0) : nk;
     if (hi <= lo) return;
     const size_t base = (((size_t)b * a.h + head) * a.cap + t0) * DH;
+    const size_t tile = (size_t)(b % SR) * a.S * DH;
     const int v0 = lo * DH / E, v1 = hi * DH / E;
     for (int v = v0 + tid; v < v1; v += FUSED_THREADS) {
-      cp_async16(sK + v * E, Kc + base + (size_t)v * E);
-      cp_async16(sV + v * E, Vc + base + (size_t)v * E);
+      cp_async16(sK + tile + v * E, Kc + base + (size_t)v * E);
+      cp_async16(sV + tile + v * E, Vc + base + (size_t)v * E);
     }
   };
   const bool pos_in_chunk = a.pos >= t0 && a.pos < t0 + nk;
@@ -610,10 +613,14 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
         prefetch_l2(base + (size_t)i * a.d * sizeof(KT), a.d * sizeof(KT));
     }
   };
+  // the slots below pos of every batch row whose tiles fit (all rows, or row 0)
+  auto stage_old = [&]() {
+    for (int b = 0; b < (SR == a.nb ? a.nb : 1); ++b) stage(b, true, false);
+  };
   if (a.sets_ready) {
     read_head();
     if (head >= 0) {
-      stage(0, true, false);
+      stage_old();
       load_wo();
       prefetch_wo();
     }
@@ -622,7 +629,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
   if (!a.sets_ready) {
     read_head();
     if (head >= 0) {
-      stage(0, true, false);
+      stage_old();
       load_wo();
     }
   }
@@ -633,13 +640,16 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
     const int g = lane % G, kq = lane / G;
     const int KW = (nk + FUSED_WARPS - 1) / FUSED_WARPS;
     const int kw0 = min(nk, warp * KW), kw1 = min(nk, kw0 + KW);
+    if (SR == a.nb && pos_in_chunk)
+      for (int b = 0; b < a.nb; ++b) stage(b, false, true);  // slot pos of every row, written by attn_in
     for (int b = 0; b < a.nb; ++b) {
-      if (b > 0) {
-        __syncthreads();  // previous row's tiles and s_w are consumed
-        stage(b, false, false);
-      } else if (pos_in_chunk) {
-        stage(0, false, true);  // slot pos, written by attn_in
+      if (b > 0) __syncthreads();  // previous row's s_w (and tiles, when staged row by row) are consumed
+      if (SR == 1) {
+        if (b > 0) stage(b, false, false);
+        else if (pos_in_chunk) stage(0, false, true);  // slot pos, written by attn_in
       }
+      const KT* tK = sK + (size_t)(b % SR) * a.S * DH;
+      const KT* tV = sV + (size_t)(b % SR) * a.S * DH;
       float qv[E];
       const float* qp = a.q + ((size_t)b * a.kh_max + p) * DH + g * E;
 #pragma unroll
@@ -655,7 +665,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
         float dot = 0.f;
         if (ok) {
           float kf[E];
-          WT<KT>::unpack(*reinterpret_cast<const uint4*>(sK + t * DH + g * E), kf);
+          WT<KT>::unpack(*reinterpret_cast<const uint4*>(tK + t * DH + g * E), kf);
 #pragma unroll
           for (int e = 0; e < E; ++e) dot = fmaf(qv[e], kf[e], dot);
         }
@@ -663,7 +673,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
         for (int o = G / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
         if (ok) {
           float vf[E];
-          WT<KT>::unpack(*reinterpret_cast<const uint4*>(sV + t * DH + g * E), vf);
+          WT<KT>::unpack(*reinterpret_cast<const uint4*>(tV + t * DH + g * E), vf);
           const float mn = fmaxf(m, dot);
           const float c = __expf(m - mn), pe = __expf(dot - mn);
           l = l * c + pe;

@@ -222,8 +222,11 @@ cudaError_t run_attn_in(const AttnInArgs& a, cudaStream_t st) {
 }
 
 template <typename KT, int DH, int NB, int WV>
-cudaError_t run_attn_out_nbw(const AttnOutArgs& a, cudaStream_t st) {
-  const size_t smem = attn_out_smem(a.S, DH, sizeof(KT), a.nb);
+cudaError_t run_attn_out_nbw(AttnOutArgs a, cudaStream_t st) {
+  // K/V tiles of every batch row at once when they fit, else row by row
+  const size_t tiles = 2ull * a.S * DH * sizeof(KT);
+  a.stage_rows = attn_out_smem(a.S, DH, sizeof(KT), a.nb) + (a.nb - 1) * tiles <= ATTN_SMEM_MAX ? a.nb : 1;
+  const size_t smem = attn_out_smem(a.S, DH, sizeof(KT), a.nb) + (a.stage_rows - 1) * tiles;
   auto kern = attn_out_kernel<KT, DH, ATTN_CS, NB, WV>;
   cudaError_t e = allow_smem(kern, smem);
   if (e != cudaSuccess) return e;
@@ -351,7 +354,7 @@ cudaError_t run_predict_b(const PredictBArgs& a, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------------------
-// Column-owner kernels (dv_colowner.cuh) for batch 1-2
+// Column-owner kernels (dv_colowner.cuh) for batch 1-4
 // ---------------------------------------------------------------------------
 
 inline int co_nv(int d, int E) { return (d + CO_THREADS * E - 1) / (CO_THREADS * E); }
@@ -359,7 +362,13 @@ inline int co_nv(int d, int E) { return (d + CO_THREADS * E - 1) / (CO_THREADS *
 // kernel also holds the W2 rows and its output slice, so it keeps fewer.
 inline int co_r(int nv) { return nv == 1 ? 8 : nv == 2 ? 4 : nv == 3 ? 3 : 4; }
 inline int co_r_mlp(int nv) { return nv == 1 ? 8 : nv == 2 ? 4 : nv == 3 ? 3 : 2; }
-inline bool co_ok(int nb, int d, int E) { return nb <= 2 && co_nv(d, E) <= 6; }
+// batch 1-2 up to 6 vectors per thread per row (d <= 12288 bf16); batch 3-4
+// up to 2 (the input slices and the MLP's output columns of 4 rows stay in
+// registers)
+inline bool co_ok(int nb, int d, int E) {
+  const int nv = co_nv(d, E);
+  return (nb <= 2 && nv <= 6) || (nb <= 4 && nv <= 2);
+}
 inline int co_grid(long long groups) {
   const long long cap = 2ll * sm_count();
   return (int)(groups < 1 ? 1 : (groups > cap ? cap : groups));
@@ -384,11 +393,20 @@ inline int co_grid(long long groups) {
     default: return launch(KERN<T, NB, 6, 2>, grid, CO_THREADS, 0, st, a);   \
   }
 
+// batch 3-4: vectors per thread 1 or 2 only
+#define DV_CO_SWITCH4(KERN, grid, st, a)                                      \
+  if (nv == 1) return launch(KERN<T, 4, 1, 8>, grid, CO_THREADS, 0, st, a);  \
+  return launch(KERN<T, 4, 2, 4>, grid, CO_THREADS, 0, st, a);
+
 template <typename T, int NB>
 cudaError_t run_attn_in_co_nb(const AttnInArgs& a, cudaStream_t st) {
   const int nv = co_nv(a.d, WT<T>::E), R = co_r(nv);
   const dim3 grid(co_grid(((long long)a.kh_max * 3 * a.dh + a.n2h + a.n2r + R - 1) / R));
-  DV_CO_SWITCH(attn_in_co_kernel, NB, grid, st, a)
+  if constexpr (NB == 4) {
+    DV_CO_SWITCH4(attn_in_co_kernel, grid, st, a)
+  } else {
+    DV_CO_SWITCH(attn_in_co_kernel, NB, grid, st, a)
+  }
 }
 
 template <typename T, int NB>
@@ -396,7 +414,11 @@ cudaError_t run_mlp_block_co_nb(MlpBlockArgs a, cudaStream_t st) {
   const int nv = co_nv(a.d, WT<T>::E), R = co_r_mlp(nv);
   a.G = co_grid(((long long)a.k_max + R - 1) / R);
   const dim3 grid(a.G);
-  DV_CO_SWITCH_MLP(mlp_block_co_kernel, NB, grid, st, a)
+  if constexpr (NB == 4) {
+    DV_CO_SWITCH4(mlp_block_co_kernel, grid, st, a)
+  } else {
+    DV_CO_SWITCH_MLP(mlp_block_co_kernel, NB, grid, st, a)
+  }
 }
 
 template <typename T, int NB>
@@ -404,10 +426,15 @@ cudaError_t run_predict_a_co_nb(const PredictAArgs& a, cudaStream_t st) {
   const int nv = co_nv(a.d, WT<T>::E), R = co_r(nv);
   const int rows = (a.PA ? a.h : 0) + (a.At ? a.r : 0);
   const dim3 grid(co_grid((rows + R - 1) / R));
-  DV_CO_SWITCH(predict_a_co_kernel, NB, grid, st, a)
+  if constexpr (NB == 4) {
+    DV_CO_SWITCH4(predict_a_co_kernel, grid, st, a)
+  } else {
+    DV_CO_SWITCH(predict_a_co_kernel, NB, grid, st, a)
+  }
 }
 #undef DV_CO_SWITCH
 #undef DV_CO_SWITCH_MLP
+#undef DV_CO_SWITCH4
 
 // ---------------------------------------------------------------------------
 // Streaming kernels (dv_stream.cuh) for rows of 16 KB and more, batch 1-2
@@ -476,7 +503,7 @@ cudaError_t run_attn_in_any(const AttnInArgs& a, cudaStream_t st) {
   if (st_ok(a.nb, a.d, WT<T>::E))
     return a.nb == 1 ? run_attn_in_st_nb<T, 1>(a, st) : run_attn_in_st_nb<T, 2>(a, st);
   if (co_ok(a.nb, a.d, WT<T>::E))
-    return a.nb == 1 ? run_attn_in_co_nb<T, 1>(a, st) : run_attn_in_co_nb<T, 2>(a, st);
+    return a.nb == 1 ? run_attn_in_co_nb<T, 1>(a, st) : a.nb == 2 ? run_attn_in_co_nb<T, 2>(a, st) : run_attn_in_co_nb<T, 4>(a, st);
   return run_attn_in<T>(a, st);
 }
 
@@ -484,7 +511,10 @@ template <typename T>
 cudaError_t run_mlp_block_any(const MlpBlockArgs& a, cudaStream_t st) {
   if (st_ok(a.nb, a.d, WT<T>::E))
     return a.nb == 1 ? run_mlp_block_st_nb<T, 1>(a, st) : run_mlp_block_st_nb<T, 2>(a, st);
-  if (co_ok(a.nb, a.d, WT<T>::E))
+  // batch 3-4: the union set spans several row groups per CTA, which the
+  // column-owner MLP kernel takes one after the other (measured slower than
+  // the row kernel there), so only batch 1-2 use it
+  if (a.nb <= 2 && co_ok(a.nb, a.d, WT<T>::E))
     return a.nb == 1 ? run_mlp_block_co_nb<T, 1>(a, st) : run_mlp_block_co_nb<T, 2>(a, st);
   return run_mlp_block<T>(a, st);
 }
@@ -494,7 +524,7 @@ cudaError_t run_predict_a_any(const PredictAArgs& a, cudaStream_t st) {
   if (st_ok(a.nb, a.d, WT<T>::E))
     return a.nb == 1 ? run_predict_a_st_nb<T, 1>(a, st) : run_predict_a_st_nb<T, 2>(a, st);
   if (co_ok(a.nb, a.d, WT<T>::E))
-    return a.nb == 1 ? run_predict_a_co_nb<T, 1>(a, st) : run_predict_a_co_nb<T, 2>(a, st);
+    return a.nb == 1 ? run_predict_a_co_nb<T, 1>(a, st) : a.nb == 2 ? run_predict_a_co_nb<T, 2>(a, st) : run_predict_a_co_nb<T, 4>(a, st);
   return run_predict_a<T>(a, st);
 }
 
