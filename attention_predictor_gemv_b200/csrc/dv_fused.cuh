@@ -551,6 +551,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
   KT* sK = reinterpret_cast<KT*>(s_dyn);                               // [SR][S][DH]
   KT* sV = sK + (size_t)SR * a.S * DH;                                 // [SR][S][DH]
   float* s_all = reinterpret_cast<float*>(sV + (size_t)SR * a.S * DH);  // [nb][CS][PW]
+  float* s_q = s_all + (size_t)a.nb * CS * PW;                          // [nb][DH], scaled q
   __shared__ __align__(16) float s_w[FUSED_WARPS][PW];
   __shared__ __align__(16) float s_H[NB][DH];
   __shared__ float s_red[WV > 0 ? 1 : FUSED_THREADS * E];
@@ -642,6 +643,13 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
     const int kw0 = min(nk, warp * KW), kw1 = min(nk, kw0 + KW);
     if (SR == a.nb && pos_in_chunk)
       for (int b = 0; b < a.nb; ++b) stage(b, false, true);  // slot pos of every row, written by attn_in
+    // q of every batch row (written by attn_in) in one round of loads
+    for (int i = tid; i < a.nb * DH / 4; i += FUSED_THREADS) {
+      const int b = i / (DH / 4), c4 = i % (DH / 4);
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(a.q + ((size_t)b * a.kh_max + p) * DH) + c4);
+      reinterpret_cast<float4*>(s_q + (size_t)b * DH)[c4] =
+          make_float4(v.x * a.scale, v.y * a.scale, v.z * a.scale, v.w * a.scale);
+    }
     for (int b = 0; b < a.nb; ++b) {
       if (b > 0) __syncthreads();  // previous row's s_w (and tiles, when staged row by row) are consumed
       if (SR == 1) {
@@ -650,12 +658,11 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
       }
       const KT* tK = sK + (size_t)(b % SR) * a.S * DH;
       const KT* tV = sV + (size_t)(b % SR) * a.S * DH;
-      float qv[E];
-      const float* qp = a.q + ((size_t)b * a.kh_max + p) * DH + g * E;
-#pragma unroll
-      for (int e = 0; e < E; ++e) qv[e] = __ldcg(qp + e) * a.scale;
       cp_async_wait_all();
-      __syncthreads();
+      __syncthreads();  // tiles and s_q complete
+      float qv[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) qv[e] = s_q[(size_t)b * DH + g * E + e];
       float m = -INFINITY, l = 0.f, acc[E];
 #pragma unroll
       for (int e = 0; e < E; ++e) acc[e] = 0.f;

@@ -172,11 +172,11 @@ cudaError_t run_attn(int dh, const float* q, const void* Kc, const void* Vc, int
 constexpr int ATTN_CS = 8;  // CTAs per cluster (per selected head) in attn_out_kernel
 
 inline int attn_out_S(int pos) { return (pos + 1 + ATTN_CS - 1) / ATTN_CS; }
-// K/V tiles of S keys plus the cluster's partials (m, l, acc[dh]) of nb rows.
+// K/V tiles of S keys, the cluster's partials (m, l, acc[dh]) and q of nb rows.
 inline size_t attn_out_smem(int S, int dh, int kvbytes, int nb) {
-  return 2ull * S * dh * kvbytes + 4ull * nb * ATTN_CS * (dh + 2);
+  return 2ull * S * dh * kvbytes + 4ull * nb * ATTN_CS * (dh + 2) + 4ull * nb * dh;
 }
-constexpr size_t ATTN_SMEM_MAX = 200 * 1024;  // dynamic part; the static part stays below 24 KB
+constexpr size_t ATTN_SMEM_MAX = 204 * 1024;  // dynamic part; the static part stays below 21 KB
 
 // W^O vectors per thread when a CTA's W^O slice (dh rows of d / ATTN_CS
 // columns) fits in registers: dh / (256 / column vectors); 0 streams it.
@@ -223,9 +223,14 @@ cudaError_t run_attn_in(const AttnInArgs& a, cudaStream_t st) {
 
 template <typename KT, int DH, int NB, int WV>
 cudaError_t run_attn_out_nbw(AttnOutArgs a, cudaStream_t st) {
-  // K/V tiles of every batch row at once when they fit, else row by row
+  // K/V tiles of every batch row at once when they fit, else row by row; and
+  // row by row too when the grid is larger than the SMs and holding every
+  // row would leave one CTA per SM (a second wave costs more than staging
+  // the rows one after the other)
   const size_t tiles = 2ull * a.S * DH * sizeof(KT);
-  a.stage_rows = attn_out_smem(a.S, DH, sizeof(KT), a.nb) + (a.nb - 1) * tiles <= ATTN_SMEM_MAX ? a.nb : 1;
+  const size_t all_rows = attn_out_smem(a.S, DH, sizeof(KT), a.nb) + (a.nb - 1) * tiles;
+  const bool waves = (long long)ATTN_CS * (a.kh_max > 0 ? a.kh_max : 1) > sm_count();
+  a.stage_rows = (all_rows <= ATTN_SMEM_MAX && !(waves && all_rows > 110 * 1024)) ? a.nb : 1;
   const size_t smem = attn_out_smem(a.S, DH, sizeof(KT), a.nb) + (a.stage_rows - 1) * tiles;
   auto kern = attn_out_kernel<KT, DH, ATTN_CS, NB, WV>;
   cudaError_t e = allow_smem(kern, smem);
