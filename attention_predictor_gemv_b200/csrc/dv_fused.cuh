@@ -659,7 +659,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
       const KT* tK = sK + (size_t)(b % SR) * a.S * DH;
       const KT* tV = sV + (size_t)(b % SR) * a.S * DH;
       cp_async_wait_all();
-      __syncthreads();  // tiles and s_q complete
+      if (b == 0 || SR == 1) __syncthreads();  // tiles and s_q complete (all rows' tiles land before row 0)
       float qv[E];
 #pragma unroll
       for (int e = 0; e < E; ++e) qv[e] = s_q[(size_t)b * DH + g * E + e];
@@ -909,8 +909,11 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
           }
         }
       }
-      // reduce the row groups, one batch row at a time
-      for (int b = 0; b < a.nb && b < NB; ++b) {
+      // reduce the row groups, one batch row at a time (unrolled, so that
+      // acc keeps static indices and stays in registers)
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        if (b >= a.nb) break;
         if (nrg > 1) {
           __syncthreads();
           if (thr_ok) {
