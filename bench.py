@@ -244,11 +244,8 @@ KERNEL_HEADERS = {
 }
 
 
-def measured_traffic(op):
-    """Per-launch DRAM bytes (read + write) of `op`'s kernel from the ncu
-    summary under profiles/ (lines `traffic <op> <bytes> <sha256 prefix>`),
-    or None when no capture exists or the kernel's headers changed since."""
-    import glob
+def kernel_sources_digest(op):
+    """SHA-256 prefix of `op`'s kernel source headers."""
     import hashlib
 
     csrc = os.path.join(ROOT, "attention_predictor_gemv_b200", "csrc")
@@ -256,8 +253,18 @@ def measured_traffic(op):
     for f in KERNEL_HEADERS.get(op, ()):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
-    digest = h.hexdigest()[:16]
-    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(op, profiles_dir=None):
+    """Per-launch DRAM bytes (read + write) of `op`'s kernel from the ncu
+    summary under profiles/ (lines `traffic <op> <bytes> <sha256 prefix>`),
+    or None when no capture exists or the kernel's headers changed since."""
+    import glob
+
+    digest = kernel_sources_digest(op)
+    pdir = profiles_dir or os.path.join(ROOT, "profiles")
+    for path in sorted(glob.glob(os.path.join(pdir, "*.md"))):
         with open(path) as fh:
             for line in fh:
                 parts = line.split()

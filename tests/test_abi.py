@@ -112,3 +112,43 @@ def test_decode_layer_argument_checks():
     w.W1t = A + 8
     assert f(ctypes.byref(w), ctypes.byref(D), ctypes.byref(p), A, 0, None, None, A, 1 << 30,
              None) == bd.DV_ERR_ALIGN
+
+
+def test_lookahead_split_argument_checks():
+    """dv_decode_layer_begin_ahead / dv_predict_layer_tail reject bad
+    arguments on the host (no GPU is touched: every pointer is fake)."""
+    w = bd.LayerWeightsC(bd.DV_BF16, bd.DV_BF16, None, None, A, A, None, A, None, A, A, None, None, A, A, A, A, A,
+                         None)
+    D = bd.dims(B=1, d=64, N=256, r=16, h=4, dh=64, cap=8, k_max=32, kh_max=2)
+    p = bd.params(32, 2, 0.125)
+    ws_bytes = bd.dv_workspace_size(bd.DV_OP_DECODE_LAYER, D)
+    W1 = 0x20000  # another fake aligned workspace
+    ahead = bd._lib_dv_decode_layer_begin_ahead
+    args = lambda **kw: dict(dict(x=A, pos=0, ws=A, nxt=ctypes.byref(w), sh=A, nws=W1), **kw)  # noqa: E731
+
+    def call(**kw):
+        a = args(**kw)
+        return ahead(ctypes.byref(w), ctypes.byref(D), ctypes.byref(p), a["x"], a["pos"], None, None, a["ws"],
+                     ws_bytes, a["nxt"], a["sh"], a["nws"], ws_bytes, None)
+
+    assert call(nws=A) == bd.DV_ERR_ARG  # the look-ahead workspace must not be the layer's
+    assert call(sh=None) == bd.DV_ERR_ARG
+    assert call(sh=A + 4) == bd.DV_ERR_ALIGN
+    assert call(pos=8) == bd.DV_ERR_ARG  # pos >= cap
+    assert call(nxt=None) == bd.DV_ERR_ARG
+    w16 = bd.LayerWeightsC(bd.DV_F32, bd.DV_F32, None, None, A, A, None, A, None, A, A, None, None, A, A, A, A, A,
+                           None)
+    assert call(nxt=ctypes.byref(w16)) == bd.DV_ERR_UNSUPPORTED  # next layer's dtype differs
+    tail = bd._lib_dv_predict_layer_tail
+    io = bd.LayerIOC(None, A, A, A, None, A, A, A)
+    for sets in (0, 4, -1):
+        assert tail(ctypes.byref(w), ctypes.byref(D), ctypes.byref(p), ctypes.byref(io), sets, W1, ws_bytes,
+                    None) == bd.DV_ERR_ARG
+    io_no_heads = bd.LayerIOC(None, None, None, None, None, A, A, A)
+    assert tail(ctypes.byref(w), ctypes.byref(D), ctypes.byref(p), ctypes.byref(io_no_heads), bd.DV_SET_HEADS, W1,
+                ws_bytes, None) == bd.DV_ERR_ARG
+    io_bad = bd.LayerIOC(None, A, A, A, None, A + 4, A, A)
+    assert tail(ctypes.byref(w), ctypes.byref(D), ctypes.byref(p), ctypes.byref(io_bad), bd.DV_SET_NEURONS, W1,
+                ws_bytes, None) == bd.DV_ERR_ALIGN
+    assert tail(ctypes.byref(w), ctypes.byref(D), ctypes.byref(p), ctypes.byref(io), bd.DV_SET_HEADS, W1, 16,
+                None) == bd.DV_ERR_WORKSPACE
