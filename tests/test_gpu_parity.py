@@ -504,6 +504,33 @@ def test_predict_layer_matches_oracle(name):
     no_device_errors(ws)
 
 
+@pytest.mark.parametrize("kf,equal", [(0.15, False), (0.05, False), (0.15, True)])
+def test_predict_layer_at_the_largest_neuron_count(kf, equal):
+    """The fused selection at N = 49152 (the OPT-175B neuron count, the most
+    the selection keeps in shared memory), batch 1: exact top-k of the
+    emitted scores, including all-equal scores (every key in one bin)."""
+    s = wl.LayerShape(B=1, d=256, N=49152, r=32, h=4, dh=64, L=64, cap=65, wdtype="bf16", kvdtype="bf16",
+                      p_active=0.1)
+    t = wl.make_layer(s, 19, DEV)
+    if equal:
+        t["Bm"] = torch.zeros_like(t["Bm"])
+        t["b1"] = torch.full_like(t["b1"], 0.25)
+    k, k_h = wl.k_for(kf, s.N), 1
+    L = bd.Layer(t, 1, k, k_h)
+    p = bd.params(k, k_h, 0.1)
+    ws = bd.workspace(bd.DV_OP_DECODE_LAYER, L.dims)
+    y = wl.make_input(s, 27, DEV)
+    tb = _trace_bufs(s)
+    out = bd.layer_io(scores_h=tb["scores_h"], head_idx=tb["head_idx"], head_count=tb["head_count"],
+                      scores=tb["scores"], idx=tb["idx"], count=tb["count"])
+    bd.dv_predict_layer(L, p, y, out, ws)
+    torch.cuda.synchronize()
+    sm = tb["scores"].cpu().numpy()
+    assert_scores(sm, O.mlp_predictor_scores(f64(y), f64(t["At"]), f64(t["Bm"]), f64(t["b1"])))
+    assert np.array_equal(selected(tb["idx"], tb["count"]), O.select(sm, k=k))
+    no_device_errors(ws)
+
+
 @pytest.mark.parametrize("name,group", [("opt-like", 8), ("opt-like", 2), ("opt-like", 0), ("ragged", 0), ("wide", 7)])
 def test_predict_layer_ties_at_threshold(name, group):
     """Neuron scores with many exact ties at the k-th value (Bm rows and b1
