@@ -466,9 +466,10 @@ def main():
 
     line = {
         "metric": METRIC, "value": value, "unit": "us", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "ms_per_step": ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": f"{CONFIG}-shaped decoder: {args.layers} layers of d={shape.d}, N={shape.N}, "
+        "config": {"workload": f"{CONFIG}-shaped decoder (bf16 weights and KV cache, fp32 arithmetic): "
+                               f"{args.layers} layers of d={shape.d}, N={shape.N}, "
                                f"r={shape.r}, h={shape.h}, dh={shape.dh}, KV length {shape.L}, batch {B}, "
                                f"k={k} ({args.k_frac:.0%}), k_h={k_h} ({args.kh_frac:.0%}), "
                                f"{'look-ahead' if not args.no_lookahead else 'synchronous'} prediction",
