@@ -2,19 +2,25 @@
 //
 // One layer runs as three kernels on the main stream:
 //   attn_in_kernel    LN1(x), Q/K/V of the selected heads, KV append
+//                     (column-owner and ring variants: dv_colowner.cuh,
+//                     dv_stream.cuh; they can also carry the next layer's
+//                     predictor first stage)
 //   attn_out_kernel   split attention + combine + W^O, one thread-block
 //                     cluster per selected head (DSMEM combine)
 //   mlp_block_kernel  LN2, W1 gather + b1 + ReLU, W2 gather-axpy
-// and the look-ahead predictor as two kernels on a side stream:
-//   predict_a_kernel  head scores and z = y A (+ head selection, last CTA)
+//                     (column-owner and ring variants as above)
+// and the look-ahead predictor as kernels on side streams:
+//   predict_a_kernel  head scores and z = y A (when not carried by attn_in)
 //   predict_b_kernel  neuron scores z B^T + b1 with a digit histogram
-//                     (+ exact top-k finish, last CTA)
+//   select_finish_kernel and gate_kernel (dv_api_kernels.cuh): the exact
+//                     head and neuron selections, and the ordering gate
 //
 // The residual stream moves x -> t1 -> x through the three main kernels:
 // attn_in zeroes t1, attn_out adds x + MHA(yA) into t1 and zeroes x, and
 // mlp_block adds t1 + MLP(yM) into x. Every block output is accumulated with
-// vector float atomics; the one CTA that owns a column slice adds the
-// residual (and the bias) exactly once.
+// vector float reductions; one CTA per column (a column slice's owner, or
+// CTA 0 when CTAs take whole rows) adds the residual (and the bias) exactly
+// once.
 #pragma once
 
 #include <cooperative_groups.h>

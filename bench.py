@@ -245,14 +245,20 @@ KERNEL_HEADERS = {
 
 
 def kernel_sources_digest(op):
-    """SHA-256 prefix of `op`'s kernel source headers."""
+    """SHA-256 prefix of `op`'s kernel source headers with comments and
+    blank lines removed (so an edited comment keeps a capture valid)."""
     import hashlib
+    import re
 
     csrc = os.path.join(ROOT, "attention_predictor_gemv_b200", "csrc")
     h = hashlib.sha256()
     for f in KERNEL_HEADERS.get(op, ()):
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(csrc, f)) as fh:
+            text = re.sub(r"/\*.*?\*/", "", fh.read(), flags=re.S)
+        for line in text.splitlines():
+            code = re.sub(r"//.*", "", line).rstrip()
+            if code.strip():
+                h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 
