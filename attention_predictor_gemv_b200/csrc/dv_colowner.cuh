@@ -5,10 +5,11 @@
 // 16-byte vectors j * 256 + t (j < NV). The thread keeps its slice of the
 // (normalised) input in registers for every row the CTA streams, so the input
 // is read from memory once per CTA and never from shared memory; LayerNorm
-// needs only two block-wide sums. A CTA streams R rows with R * NV 16-byte
+// needs one block-wide reduction. A CTA streams R rows with R * NV 16-byte
 // loads in flight per thread, fully coalesced (each row is read by the whole
 // CTA), and reduces the R partial dot products across the CTA at the end.
-// Used when NB * NV is small (batch 1-2): the slices then fit in registers.
+// Used when NB * NV is small (batch 1-2 up to NV = 6, batch 3-4 up to NV = 2):
+// the slices then fit in registers.
 #pragma once
 
 #include "dv_fused.cuh"
