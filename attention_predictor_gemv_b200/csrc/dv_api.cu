@@ -799,23 +799,15 @@ static __device__ __align__(256) unsigned char g_topk_static_scratch[DV_TOPK_STA
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_static_mu;
-void* g_static_addr[kMaxDevices] = {};
-
-// Device address of g_topk_static_scratch on the current device, looked up
-// once per device (the host-side name is only a stand-in for it).
+// Device address of g_topk_static_scratch in the current context, looked up
+// on every call: the host-side name is only a stand-in, and after a context
+// is torn down and rebuilt (cudaDeviceReset, a host framework resetting the
+// device) the module is loaded again and the array may sit elsewhere, so a
+// cached address could be stale. The lookup does no allocation.
 dv_status static_scratch_address(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return DV_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return DV_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_static_mu);
-  if (!g_static_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_topk_static_scratch) != cudaSuccess || !p) return DV_ERR_CUDA;
-    g_static_addr[dev] = p;
-  }
-  *out = g_static_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_topk_static_scratch) != cudaSuccess || !p) return DV_ERR_CUDA;
+  *out = p;
   return DV_OK;
 }
 

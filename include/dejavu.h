@@ -335,9 +335,11 @@ DV_API dv_status dv_prefetch_layer(const dv_layer_weights* w, const dv_dims* dim
  * DV_TOPK_STATIC_MAX_N scores; larger sizes return DV_ERR_UNSUPPORTED and
  * launch nothing. It calls no cudaMalloc / cudaFree.
  *
- * The first call on a device looks up the array's device address (one
- * cudaGetSymbolAddress per device, with that device current); make that first
- * call before any stream capture. Every call shares the one array per device:
+ * Every call looks up the array's device address on the current device
+ * (cudaGetSymbolAddress, which allocates nothing), so the address stays right
+ * after a context reset. The first call on a device also loads the library's
+ * device code there, which is set-up work: make that first call before any
+ * stream capture. Every call shares the one array per device:
  * the ticket is cleared on the caller's stream before each launch, and calls
  * that overlap on the GPU (other streams, other threads) race on it.
  * Arguments and outputs are those of dv_topk. */

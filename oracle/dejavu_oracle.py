@@ -28,7 +28,7 @@ Sources (page title, then section / equation):
 * "A Survey on Efficient Inference for Large Language Models" (reading note),
   Transformer section: head outputs are concatenated and projected by W^O.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent or garbled:
 
 * predictor: rank-r factors, s = (y A) B^T + b1, with A = At^T (the pages' §4.1
   is not part of the extraction); head predictor: one linear map P_A [h][d];

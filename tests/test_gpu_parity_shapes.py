@@ -1,0 +1,260 @@
+"""CUDA path vs the CPU oracle at the layer shapes of the large workloads.
+
+The fused layer kernels are instantiated per row length: column-owner kernels
+with 1-3 16-byte vectors per thread and row (d <= 6144 bf16), shared-memory
+ring kernels with 4, 5 or 6 (d = 8192, 10240 / 9216, 12288), and an attention
+kernel that reads whole W^O rows per CTA for d = 8192, 10240 and 12288. These
+tests reach every instantiation the OPT-6.7B, OPT-66B and OPT-175B-shaped
+workloads run, with their KV lengths (1024, 2048), at batch 1 and 2:
+
+* slices: d, dh and the KV length at full size, fewer neurons and heads, so
+  the float64 oracle holds every weight (one layer, and a 3-layer look-ahead
+  stack);
+* full size: the OPT-175B-shaped layer itself (d = 12288, N = 49152, h = 96,
+  KV 2048) with the sets the bench uses (15% of neurons and heads), run as the
+  bench runs it (look-ahead stack, CUDA graph), and checked on the selected
+  rows: the oracle needs only the gathered rows of W1, W2, Wqkv, W^O and the
+  selected heads' caches to evaluate eq. (1) and eq. (2) on given sets, and
+  the whole predictor to score every neuron and head.
+
+Tolerances as everywhere: index sets bit-exact (the oracle's selection of the
+scores the GPU emitted), scores within 1e-3, block outputs within relative L2
+5e-3 and max-abs 2e-2 ||out||_inf.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import dejavu_oracle as O
+from tests._helpers import assert_out, assert_scores, f64, oracle_layer, selected
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from attention_predictor_gemv_b200 import binding as bd
+    from attention_predictor_gemv_b200 import workload as wl
+    from attention_predictor_gemv_b200.stack import DecoderStack
+
+DEV = "cuda"
+
+SLICES = {
+    # OPT-175B row length: ring kernels with 6 vectors per thread, whole-row W^O (6)
+    "175b-slice": dict(d=12288, N=4096, r=64, h=8, dh=128, L=2048, cap=2056, p_active=0.05),
+    # OPT-66B row length: ring kernels with 5 vectors per thread (the last one
+    # partial), W^O streamed in column slices (d / 8 columns is not a multiple
+    # of 2048)
+    "66b-slice": dict(d=9216, N=4096, r=64, h=8, dh=128, L=1024, cap=1032, p_active=0.06),
+    # ring kernels with 5 whole vectors per thread, whole-row W^O (5)
+    "d10240": dict(d=10240, N=2048, r=64, h=6, dh=128, L=700, cap=710, p_active=0.1),
+    # OPT-6.7B layer at full size: column-owner kernels with 2 vectors per thread
+    "6.7b": dict(d=4096, N=16384, r=512, h=32, dh=128, L=2048, cap=2176, p_active=0.08),
+}
+
+
+def _shape(name, B):
+    return wl.LayerShape(B=B, wdtype="bf16", kvdtype="bf16", **SLICES[name])
+
+
+def _trace_bufs(s):
+    f = dict(device=DEV, dtype=torch.float32)
+    i = dict(device=DEV, dtype=torch.int32)
+    return dict(yA=torch.empty(s.B, s.d, **f), scores_h=torch.empty(s.B, s.h, **f), head_idx=torch.zeros(s.h, **i),
+                head_count=torch.zeros(1, **i), yM=torch.empty(s.B, s.d, **f), scores=torch.empty(s.B, s.N, **f),
+                idx=torch.zeros(s.N, **i), count=torch.zeros(1, **i))
+
+
+def _no_device_errors(ws):
+    assert bd.dv_read_device_status(ws) == 0
+
+
+@pytest.mark.parametrize("name,B,kf,khf", [("175b-slice", 1, 0.15, 0.25), ("175b-slice", 2, 0.15, 0.25),
+                                          ("66b-slice", 1, 0.06, 0.25), ("66b-slice", 2, 0.06, 0.5),
+                                          ("d10240", 1, 0.1, 0.34), ("6.7b", 1, 0.08, 0.2), ("6.7b", 2, 0.08, 0.2)])
+def test_decode_layer_at_large_row_lengths(name, B, kf, khf):
+    s = _shape(name, B)
+    t = wl.make_layer(s, 31, DEV)
+    t["ln2_g"] = 1.0 + 0.1 * torch.randn(s.d, device=DEV)
+    x = wl.make_input(s, 32, DEV)
+    k, k_h = max(1, wl.k_for(kf, s.N)), max(1, wl.k_for(khf, s.h))
+    L = bd.Layer(t, B, min(s.N, B * k), min(s.h, B * k_h))
+    p = bd.params(k, k_h, 1.0 / np.sqrt(s.dh))
+    ws = bd.workspace(bd.DV_OP_DECODE_LAYER, L.dims)
+    tb = _trace_bufs(s)
+    x0 = x.clone()
+    OL = oracle_layer(t)
+    bd.dv_decode_layer(L, p, x, s.L, ws, trace=bd.layer_io(**tb))
+    torch.cuda.synchronize()
+    P = O.LayerParams(k=k, k_h=k_h, scale=1.0 / np.sqrt(s.dh))
+    sh, sm = tb["scores_h"].cpu().numpy(), tb["scores"].cpu().numpy()
+    hsel, msel = O.select(sh, k=k_h), O.select(sm, k=k)
+    assert np.array_equal(selected(tb["head_idx"], tb["head_count"]), hsel)
+    assert np.array_equal(selected(tb["idx"], tb["count"]), msel)
+    tr = O.decode_layer(f64(x0), OL, P, s.L, head_idx=hsel, idx=msel)
+    assert_out(tb["yA"].cpu().numpy(), tr.yA, "yA")
+    assert_scores(sh, O.head_predictor_scores(f64(tb["yA"]), OL.PA))
+    assert_out(tb["yM"].cpu().numpy(), tr.yM, "yM")
+    assert_scores(sm, O.mlp_predictor_scores(f64(tb["yM"]), OL.At, OL.Bm, OL.b1))
+    assert_out((x - x0).cpu().numpy(), tr.x_out - f64(x0), "x_out - x")
+    # the KV slot of every selected head, in every batch row
+    for b in range(B):
+        for j, i in enumerate(hsel):
+            for cache, ref in ((t["K"], tr.mha.k_new), (t["V"], tr.mha.v_new)):
+                got = f64(cache[b, i, s.L])
+                assert np.all(np.abs(got - ref[b, j]) <= np.abs(ref[b, j]) * 2.0 ** -7 + 1e-6)
+    _no_device_errors(ws)
+
+
+@pytest.mark.parametrize("name,B", [("175b-slice", 1), ("175b-slice", 2), ("66b-slice", 2), ("6.7b", 1)])
+def test_lookahead_stack_at_large_row_lengths(name, B):
+    """Three layers with the look-ahead predictor (its first stage inside the
+    q/k/v kernel, the selections on side streams): every layer's sets are the
+    oracle's selection of the scores the GPU emitted from the previous
+    layer's attention input, and the stack output matches."""
+    nL = 3
+    s = _shape(name, B)
+    layers = [wl.make_layer(s, 300 + l, DEV) for l in range(nL)]
+    K0 = [(f64(t["K"]), f64(t["V"])) for t in layers]
+    k, k_h = wl.k_for(0.1, s.N), 2
+    stk = DecoderStack(layers, B, k, k_h, 1.0 / np.sqrt(s.dh), lookahead=True)
+    x = wl.make_input(s, 33, DEV)
+    x0 = f64(x)
+    stk.step(x, s.L)
+    torch.cuda.synchronize()
+    OLs = []
+    for l, t in enumerate(layers):
+        OL = oracle_layer(t)
+        OL.K, OL.V = K0[l]
+        OLs.append(OL)
+    P = O.LayerParams(k=k, k_h=k_h, scale=1.0 / np.sqrt(s.dh))
+    sel = []
+    for l in range(nL):
+        sh, sm = stk.scores_h[l].cpu().numpy(), stk.scores[l].cpu().numpy()
+        hs, ms = O.select(sh, k=k_h), O.select(sm, k=k)
+        assert np.array_equal(selected(stk.head_idx[l], stk.head_count[l]), hs), l
+        assert np.array_equal(selected(stk.idx[l], stk.count[l]), ms), l
+        if l > 0:
+            yprev = f64(stk.yA[l - 1])
+            assert_scores(sh, O.head_predictor_scores(yprev, OLs[l].PA))
+            assert_scores(sm, O.mlp_predictor_scores(yprev, OLs[l].At, OLs[l].Bm, OLs[l].b1))
+        sel.append((hs, ms))
+    xo, _ = O.decode_stack(x0, OLs, P, s.L, lookahead=True, sel_override=sel)
+    assert_out(x.cpu().numpy() - x0, xo - x0)
+    _no_device_errors(stk.ws_main)
+    _no_device_errors(stk.ws_side)
+
+
+@pytest.mark.parametrize("N,B,kf", [(49152, 1, 0.15), (49152, 2, 0.05), (36864, 2, 0.06), (36864, 4, 0.06)])
+def test_fused_layer_selection_at_the_largest_neuron_counts(N, B, kf):
+    """The OPT-175B and OPT-66B neuron counts through the fused layer call
+    (synchronous prediction, batch unions): exact sets and the layer output."""
+    s = wl.LayerShape(B=B, d=1024, N=N, r=64, h=8, dh=64, L=128, cap=130, wdtype="bf16", kvdtype="bf16",
+                      p_active=0.06)
+    t = wl.make_layer(s, 41, DEV)
+    x = wl.make_input(s, 42, DEV)
+    k, k_h = wl.k_for(kf, N), 2
+    L = bd.Layer(t, B, min(N, B * k), min(s.h, B * k_h))
+    p = bd.params(k, k_h, 1.0 / np.sqrt(s.dh))
+    ws = bd.workspace(bd.DV_OP_DECODE_LAYER, L.dims)
+    tb = _trace_bufs(s)
+    x0 = x.clone()
+    OL = oracle_layer(t)
+    bd.dv_decode_layer(L, p, x, s.L, ws, trace=bd.layer_io(**tb))
+    torch.cuda.synchronize()
+    sh, sm = tb["scores_h"].cpu().numpy(), tb["scores"].cpu().numpy()
+    hsel, msel = O.select(sh, k=k_h), O.select(sm, k=k)
+    assert np.array_equal(selected(tb["head_idx"], tb["head_count"]), hsel)
+    assert np.array_equal(selected(tb["idx"], tb["count"]), msel)
+    assert_scores(sm, O.mlp_predictor_scores(f64(tb["yM"]), OL.At, OL.Bm, OL.b1))
+    P = O.LayerParams(k=k, k_h=k_h, scale=1.0 / np.sqrt(s.dh))
+    tr = O.decode_layer(f64(x0), OL, P, s.L, head_idx=hsel, idx=msel)
+    assert_out((x - x0).cpu().numpy(), tr.x_out - f64(x0), "x_out - x")
+    _no_device_errors(ws)
+
+
+# ---------------------------------------------------------------------------
+# full size, checked on the gathered rows
+# ---------------------------------------------------------------------------
+
+
+def _oracle_layer_on_rows(x, t, hsel, msel, pos, scale, eps=1e-5):
+    """eq. (2) then eq. (1) for one pre-LN layer on the given sets, from the
+    selected rows only (gathered here by plain indexing): the oracle's
+    functions composed as in its decode_layer, with the weight arrays
+    replaced by their selected rows and the sets by 0..k-1. Returns
+    (yA, yM, x_out, k_new, v_new)."""
+    hs = torch.from_numpy(np.asarray(hsel, dtype=np.int64)).to(DEV)
+    ms = torch.from_numpy(np.asarray(msel, dtype=np.int64)).to(DEV)
+    yA = O.layernorm(x, eps)
+    Kh, Vh = f64(t["K"][:, hs]), f64(t["V"][:, hs])
+    mha = O.sparse_mha(yA, f64(t["Wqkv"][hs]), None, f64(t["WOt"][hs]), None, Kh, Vh, pos, scale,
+                       np.arange(len(hsel)), "bf16")
+    x1 = x + mha.out
+    yM = O.layernorm(x1, eps)
+    out_m = O.sparse_mlp(yM, f64(t["W1t"][ms]), f64(t["b1"][ms]), f64(t["W2t"][ms]), None, np.arange(len(msel)))
+    return yA, yM, x1 + out_m, mha.k_new, mha.v_new
+
+
+@pytest.mark.parametrize("B", [1, 2])
+def test_opt175b_shaped_stack_in_bench_configuration(B):
+    """Two full OPT-175B-shaped layers (d = 12288, N = 49152, r = 1024,
+    h = 96, dh = 128, KV length 2048) at 15% of neurons and heads, run as the
+    bench runs them: look-ahead stack captured in a CUDA graph and replayed.
+    Layer 0 predicts its own sets; layer 1 uses the sets predicted from layer
+    0's attention input. Checked: every score against the whole predictor,
+    the sets bit-exact, both layers' outputs and the written KV slots against
+    the oracle on the selected rows."""
+    s = wl.CONFIGS["opt-175b"].with_(B=B)
+    layers = [wl.make_layer(s, 5000 + l, DEV) for l in range(2)]
+    k, k_h = wl.k_for(0.15, s.N), wl.k_for(0.15, s.h)
+    scale = 1.0 / np.sqrt(s.dh)
+    stk = DecoderStack(layers, B, k, k_h, scale, lookahead=True)
+    x = wl.make_input(s, 11, DEV)
+    xin = x.clone()
+    Kpre = [(t["K"].clone(), t["V"].clone()) for t in layers]
+    pos = s.L
+    stk.step(x, pos)  # eager once (kernel set-up outside the capture), then back to the start state
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            stk.step(x, pos)
+    torch.cuda.current_stream().wait_stream(side)
+    for (K, V), t in zip(Kpre, layers):
+        t["K"].copy_(K)
+        t["V"].copy_(V)
+    x.copy_(xin)
+    g.replay()
+    torch.cuda.synchronize()
+    # the oracle works on copies of the pre-step caches
+    xcur = f64(xin)
+    for l, t in enumerate(layers):
+        tcache = dict(t)
+        tcache["K"], tcache["V"] = Kpre[l]
+        sh, sm = stk.scores_h[l].cpu().numpy(), stk.scores[l].cpu().numpy()
+        hs, ms = O.select(sh, k=k_h), O.select(sm, k=k)
+        assert np.array_equal(selected(stk.head_idx[l], stk.head_count[l]), hs), l
+        assert np.array_equal(selected(stk.idx[l], stk.count[l]), ms), l
+        ypred = f64(stk.yA[0]) if l == 1 else None
+        yA, yM, xout, k_new, v_new = _oracle_layer_on_rows(xcur, tcache, hs, ms, pos, scale)
+        assert_out(stk.yA[l].cpu().numpy(), yA, f"yA[{l}]")
+        assert_out(stk.yM[l].cpu().numpy(), yM, f"yM[{l}]")
+        if l == 0:
+            ysrc_h, ysrc_m = yA, yM
+        else:
+            ysrc_h = ysrc_m = ypred  # look-ahead: both sets from layer 0's yA
+        assert_scores(sh, O.head_predictor_scores(ysrc_h, f64(t["PA"])), f"scores_h[{l}]")
+        assert_scores(sm, O.mlp_predictor_scores(ysrc_m, f64(t["At"]), f64(t["Bm"]), f64(t["b1"])),
+                      f"scores[{l}]")
+        for b in range(B):
+            for j, i in enumerate(hs):
+                for cache, ref in ((t["K"], k_new), (t["V"], v_new)):
+                    got = f64(cache[b, i, pos])
+                    assert np.all(np.abs(got - ref[b, j]) <= np.abs(ref[b, j]) * 2.0 ** -7 + 1e-6)
+        xcur = xout
+    assert_out(x.cpu().numpy() - f64(xin), xcur - f64(xin), "stack out - x")
+    _no_device_errors(stk.ws_main)
+    _no_device_errors(stk.ws_side)
+    del g

@@ -373,3 +373,80 @@ def test_lookahead_with_full_sets_equals_synchronous():
     xs, _ = O.decode_stack(x, layers, P, pos, lookahead=False)
     xl, _ = O.decode_stack(x, la, P, pos, lookahead=True)
     assert np.allclose(xs, xl, rtol=1e-13, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# head predictor and GeLU (pins independent of the oracle's own expressions)
+# --------------------------------------------------------------------------
+
+
+def test_head_predictor_scores_against_library_and_closed_forms():
+    """s_A = y P_A^T, pinned four ways: torch's F.linear (another library's
+    matrix product), unit rows of P_A that pick single coordinates of y, a row
+    equal to y (its squared norm) and a row orthogonal to y (zero), and exact
+    rational brute force. h != d, so a transposed P_A cannot pass."""
+    r = rng(21)
+    B, d, h = 3, 10, 7
+    y = r.standard_normal((B, d))
+    PA = r.standard_normal((h, d))
+    got = O.head_predictor_scores(y, PA)
+    assert got.shape == (B, h)
+    want = F.linear(torch.from_numpy(y), torch.from_numpy(PA)).numpy()
+    assert np.allclose(got, want, rtol=1e-13, atol=1e-13)
+    # unit rows: head i scores coordinate j_i of y
+    cols = [4, 0, 9, 2, 2, 7, 5]
+    E = np.zeros((h, d))
+    E[np.arange(h), cols] = 1.0
+    assert np.array_equal(O.head_predictor_scores(y, E), y[:, cols])
+    # a row equal to y[0] scores ||y[0]||^2; a row orthogonal to it scores 0
+    u = y[0] / np.linalg.norm(y[0])
+    v = r.standard_normal(d)
+    v -= (v @ u) * u
+    P2 = np.stack([y[0], v])
+    s = O.head_predictor_scores(y[:1], P2)[0]
+    assert np.isclose(s[0], float(np.sum(y[0] ** 2)), rtol=1e-13)
+    assert abs(s[1]) <= 1e-12 * np.linalg.norm(v) * np.linalg.norm(y[0])
+    # permuting the heads permutes the scores
+    perm = r.permutation(h)
+    assert np.array_equal(O.head_predictor_scores(y, PA[perm]), got[:, perm])
+    # exact rationals on small integers / powers of two: the float64 result is exact
+    yi = r.integers(-8, 9, size=(2, d))
+    Pi = r.integers(-8, 9, size=(h, d))
+    exact = [[float(sum(Fraction(int(yi[b, j]), 4) * Fraction(int(Pi[i, j]), 8) for j in range(d)))
+              for i in range(h)] for b in range(2)]
+    assert np.array_equal(O.head_predictor_scores(yi / 4.0, Pi / 8.0), np.array(exact))
+
+
+def test_gelu_against_torch_and_limits():
+    """GeLU in the exact erf form v * Phi(v): torch's F.gelu (approximate='none'),
+    GeLU(0) = 0, GeLU(v) - GeLU(-v) = v (odd part), and the limits v -> +inf
+    (identity) and v -> -inf (zero)."""
+    v = np.concatenate([np.linspace(-8.0, 8.0, 401), rng(22).standard_normal(200) * 3.0])
+    got = O.gelu(v)
+    want = F.gelu(torch.from_numpy(v), approximate="none").numpy()
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-15)
+    assert O.gelu(np.array([0.0]))[0] == 0.0
+    assert np.allclose(O.gelu(v) - O.gelu(-v), v, rtol=1e-12, atol=1e-14)
+    assert np.isclose(O.gelu(np.array([40.0]))[0], 40.0) and abs(O.gelu(np.array([-40.0]))[0]) < 1e-300
+    # the tanh approximation differs: the oracle is the erf form
+    tanh_form = F.gelu(torch.from_numpy(v), approximate="tanh").numpy()
+    assert np.max(np.abs(got - tanh_form)) > 1e-6
+
+
+def test_sparse_mlp_gelu_all_neurons_is_dense_gelu_ffn():
+    """eq. (1) with sigma = GeLU: with S_M = every neuron the sparse MLP equals a
+    torch Linear -> GeLU -> Linear FFN; dropping a neuron changes it (GeLU has
+    no exact zeros, so no set smaller than all neurons is exact)."""
+    r = rng(23)
+    B, d, N = 2, 12, 40
+    y = r.standard_normal((B, d))
+    W1t = r.standard_normal((N, d)) / np.sqrt(d)
+    W2t = r.standard_normal((N, d)) / np.sqrt(d)
+    b1 = r.standard_normal(N) * 0.3
+    b2 = r.standard_normal(d) * 0.1
+    got = O.sparse_mlp(y, W1t, b1, W2t, b2, np.arange(N), act="gelu")
+    ty = torch.from_numpy(y)
+    hid = F.gelu(F.linear(ty, torch.from_numpy(W1t), torch.from_numpy(b1)), approximate="none")
+    want = F.linear(hid, torch.from_numpy(W2t).t().contiguous(), torch.from_numpy(b2)).numpy()
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-12)
+    assert not np.allclose(O.sparse_mlp(y, W1t, b1, W2t, b2, np.arange(1, N), act="gelu"), got, rtol=1e-9)

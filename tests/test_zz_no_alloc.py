@@ -3,15 +3,19 @@
 memory and gives it no allocator). It keeps its scratch in the library's
 file-scope device array instead of a caller workspace.
 
-Checked through the C ABI against dv_topk (the workspace version) on two
-calls in a row with different sizes: the index sets and counts must be
-identical. Collected last so that a failure here comes after every other
-test has run; it also passes alone in a fresh process.
+Checked through the C ABI against dv_topk (the workspace version) on
+consecutive calls with different sizes, up to the largest size the array
+holds (16 rows of 65,536 scores): the index sets and counts must be
+identical, and equal to the oracle's selection of the same scores. Collected
+last so that a failure here comes after every other test has run; it also
+passes alone in a fresh process.
 """
 
 import numpy as np
 import pytest
 import torch
+
+from oracle import dejavu_oracle as O
 
 pytestmark = pytest.mark.gpu
 
@@ -45,12 +49,18 @@ def test_topk_static_matches_workspace_version_on_consecutive_calls():
         (torch.randn(3, 5000, generator=g, device="cuda"), 123, bd.DV_TOPK, 0.0),
         (torch.randn(1, 65536, generator=g, device="cuda"), 6554, bd.DV_TOPK, 0.0),
         (torch.randn(16, 2048, generator=g, device="cuda"), 0, bd.DV_THRESHOLD, 1.5),
+        # the largest accepted size: every bitmap word of the array in use
+        (torch.randn(16, 65536, generator=g, device="cuda"), 3000, bd.DV_TOPK, 0.0),
+        (torch.randn(16, 65536, generator=g, device="cuda"), 0, bd.DV_THRESHOLD, 2.5),
+        (torch.randn(2, 777, generator=g, device="cuda"), 40, bd.DV_TOPK, 0.0),
     ]
     for scores, k, mode, tau in cases:  # consecutive calls share the one scratch array
         want_idx, want_cnt = _with_workspace(scores, k, mode, tau)
         got_idx, got_cnt = _static(scores, k, mode, tau)
         assert got_cnt == want_cnt
         assert np.array_equal(got_idx, want_idx)
+        ref = O.select(scores.cpu().numpy(), k=k, tau=tau, mode="topk" if mode == bd.DV_TOPK else "threshold")
+        assert np.array_equal(got_idx, ref)
 
 
 def test_topk_static_rejects_sizes_beyond_its_array():
