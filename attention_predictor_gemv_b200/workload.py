@@ -139,3 +139,13 @@ def svd_predictor(W1t_f32: torch.Tensor, r: int):
 def make_input(shape: LayerShape, seed: int, device="cpu") -> torch.Tensor:
     g = _gen(seed + 7919, device)
     return torch.randn(shape.B, shape.d, generator=g, device=device, dtype=torch.float32)
+
+
+def make_kv(shape: LayerShape, B: int, seed: int, device="cpu"):
+    """KV caches [B][h][cap][dh] ~ N(0, 1) for batch B (the same recipe as
+    make_layer's caches), for running one set of weights at several batches."""
+    g = _gen(seed + 15485863, device)
+    kvdt = _dt(shape.kvdtype)
+    K = _randn((B, shape.h, shape.cap, shape.dh), g, device, 1.0, kvdt)
+    V = _randn((B, shape.h, shape.cap, shape.dh), g, device, 1.0, kvdt)
+    return K, V

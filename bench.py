@@ -1,18 +1,28 @@
-"""Benchmark: one decode step of an OPT-1.3B-shaped decoder (24 layers of the
-d=2048, N=8192, h=32, dh=64 layer, KV length 512, batch 1, bf16 weights,
-fp32 accumulation) with contextual sparsity: the look-ahead predictors, top-k
-selection, sparse MHA over the selected heads and sparse MLP over the
-selected neurons, through the C ABI.
+"""Benchmark: decode steps of OPT-shaped decoder stacks with contextual
+sparsity (the look-ahead predictors, top-k selection, sparse MHA over the
+selected heads and sparse MLP over the selected neurons), through the C ABI,
+bf16 weights and KV cache, fp32 arithmetic.
 
-Metric: microseconds per decode step per layer (lower is better), with the
-effective HBM bandwidth on the selected bytes. The 24 layers hold 2.6 GB of
-weights, more than L2 (126 MB), so every step streams its selected bytes
-from HBM.
+Headline: 24 OPT-175B-shaped layers (d=12288, N=49152, r=1024, h=96, dh=128,
+KV length 2048; 87 GB of weights), batch 1, 85% sparsity on neurons and heads
+(k = 7373, k_h = 14), look-ahead on; one step = one token through the 24
+layers. Metric: microseconds per decode step per layer (lower is better), with
+the effective HBM bandwidth on the selected bytes.
+
+Also measured in the same run (each in the JSON line):
+  * the OPT-175B sweep: sparsity 50/75/85/95% x batch 1/2/4/8/16, plus the
+    dense path of the same kernels at each batch (sparse/dense crossover);
+  * OPT-6.7B-shaped stack, 32 layers, 128 generated tokens with the KV
+    position advancing, look-ahead on and off;
+  * OPT-66B-shaped stack, 64 layers, batch 1/2/4/8 (union sets);
+  * OPT-1.3B-shaped stack, 24 layers, neuron x head fraction sweep; the tiny
+    layer (latency only, L2-resident);
+  * the CPU oracle on the host cores (single thread and all cores).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
-For N > 1 (torchrun) every rank runs an independent replica (the path has
-no exchange step); the time is the maximum over ranks.
+For N > 1 (torchrun) every rank runs an independent replica of the headline
+stack (the path has no exchange step); the time is the maximum over ranks.
 """
 
 from __future__ import annotations
@@ -34,28 +44,27 @@ from attention_predictor_gemv_b200 import accounting as acct  # noqa: E402
 from attention_predictor_gemv_b200 import workload as wl  # noqa: E402
 
 METRIC = "us/decode-step/layer"
-CONFIG = "opt-1.3b"
+HEADLINE = "opt-175b"
+HEADLINE_SPARSITY = 0.85
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--layers", type=int, default=24)
-    ap.add_argument("--k-frac", type=float, default=0.10)
-    ap.add_argument("--kh-frac", type=float, default=0.25)
+    ap.add_argument("--config", default=HEADLINE, choices=sorted(wl.CONFIGS))
+    ap.add_argument("--layers", type=int, default=0, help="0: the workload's own layer count")
+    ap.add_argument("--sparsity", type=float, default=HEADLINE_SPARSITY,
+                    help="fraction of neurons and heads skipped at the headline point")
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--no-lookahead", action="store_true")
-    ap.add_argument("--no-sweep", action="store_true")
-    ap.add_argument("--no-big", action="store_true", help="skip the OPT-175B-shaped measurement")
-    ap.add_argument("--big-layers", type=int, default=4)
-    ap.add_argument("--prefetch", action="store_true", help="L2-prefetch each layer's selected rows on the side stream")
-    ap.add_argument("--no-prefetch-w2", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the sparsity x batch sweep")
+    ap.add_argument("--no-extra", action="store_true", help="skip the OPT-6.7B/66B/1.3B/tiny measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    return ap.parse_args()
+    ap.add_argument("--cpu-seconds", type=float, default=2.0, help="seconds per CPU oracle timing")
+    return ap.parse_args(argv)
 
 
 # ---------------------------------------------------------------------------
@@ -75,10 +84,10 @@ def dist_init():
     local = int(os.environ.get("LOCAL_RANK", rank))
     if torch.cuda.is_available():
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
     else:  # host-only ranks (the reference arm, tests): gloo
-        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=300))
     return rank, ws, dist
 
 
@@ -112,6 +121,7 @@ class Clocks:
     def __init__(self, dev_index: int):
         self.dev = dev_index
         self.p = None
+        self.out = ""
 
     def __enter__(self):
         try:
@@ -120,12 +130,11 @@ class Clocks:
                                       stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.p = None
-        time.sleep(0.25)
+        time.sleep(0.3)
         return self
 
     def __exit__(self, *a):
         time.sleep(0.15)
-        self.out = ""
         if self.p is not None:
             self.p.terminate()
             try:
@@ -154,30 +163,56 @@ class Clocks:
 
 
 # ---------------------------------------------------------------------------
-# the GPU arm
+# stacks, graphs and timing
 # ---------------------------------------------------------------------------
 
 
-def build_stack(shape, nlayers, B, k, k_h, lookahead, seed0=1000, layers=None, prefetch=False, prefetch_w2=True):
+def make_layers(shape, n, seed0):
+    """n layers of `shape` (weights, predictors, batch-1 KV caches) on the GPU."""
+    return [wl.make_layer(shape.with_(B=1), seed0 + l, "cuda") for l in range(n)]
+
+
+def with_kv(layers, shape, B, seed):
+    """The layers with fresh KV caches for batch B (weights shared)."""
+    out = []
+    for l, t in enumerate(layers):
+        K, V = wl.make_kv(shape, B, seed + l, "cuda")
+        out.append(dict(t, K=K, V=V))
+    return out
+
+
+def build_stack(layers, shape, B, k, k_h, lookahead):
     from attention_predictor_gemv_b200.stack import DecoderStack
 
-    if layers is None:
-        layers = [wl.make_layer(shape, seed0 + l, "cuda") for l in range(nlayers)]
-    stk = DecoderStack(layers, B, k, k_h, 1.0 / float(np.sqrt(shape.dh)), lookahead=lookahead, prefetch=prefetch,
-                       prefetch_w2=prefetch_w2)
-    return stk, layers
+    return DecoderStack(layers, B, k, k_h, 1.0 / float(np.sqrt(shape.dh)), lookahead=lookahead)
+
+
+def graph_of(fn):
+    """Captures fn (library launches on the current stream) into a CUDA graph
+    after one eager call (kernel set-up stays outside the capture)."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    return g
 
 
 def capture(stk, x, pos):
     """The decode step as a CUDA graph, and how many library kernels it holds."""
     from attention_predictor_gemv_b200 import binding as bd
 
-    stk.step(x, pos)  # eager warm-up
+    stk.step(x, pos)
     torch.cuda.synchronize()
     n0 = bd.dv_launch_count()
     g = graph_of(lambda: stk.step(x, pos))
     n1 = bd.dv_launch_count()
-    return g, (n1 - n0) // 2  # graph_of runs fn once eagerly, then captures it
+    return g, (n1 - n0) // 2  # graph_of calls fn twice (eager, then captured)
 
 
 def time_graph(g, steps, warmup, dist):
@@ -195,17 +230,15 @@ def time_graph(g, steps, warmup, dist):
 
 
 def selected_counts(stk):
-    """Mean k (selected neurons), k' (nonzero activations) and k_h over layers."""
-    ks, khs = [], []
-    for l in range(len(stk.layers)):
-        ks.append(int(stk.count[l].item()))
-        khs.append(int(stk.head_count[l].item()))
+    """Mean k (selected neurons) and k_h over the layers."""
+    ks = [int(stk.count[l].item()) for l in range(len(stk.layers))]
+    khs = [int(stk.head_count[l].item()) for l in range(len(stk.layers))]
     return float(np.mean(ks)), float(np.mean(khs))
 
 
 def nonzero_neurons(stk):
-    """k' per layer: selected neurons with a nonzero activation, read from the
-    workspace-independent recomputation y_M . W1 + b1 on the device (torch)."""
+    """k' per layer: selected neurons with a nonzero activation in some batch
+    row, recomputed from the layer's y_M on the device (torch, reporting only)."""
     kp = []
     for l, L in enumerate(stk.layers):
         c = int(stk.count[l].item())
@@ -217,30 +250,37 @@ def nonzero_neurons(stk):
 
 def layer_bytes(shape, k, kp, kh, B):
     return acct.layer_bytes(shape.d, shape.N, shape.r, shape.h, shape.dh, int(round(k)), int(round(kp)),
-                            int(round(kh)), B, shape.L + 1)
+                            int(round(kh)), B, shape.L + 1, wdtype=shape.wdtype, kvdtype=shape.kvdtype)
 
 
-def graph_of(fn):
-    """Captures fn (library launches on the current stream) into a CUDA graph."""
-    fn()
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    s = torch.cuda.Stream()
-    s.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(s):
-        with torch.cuda.graph(g, stream=s):
-            fn()
-    torch.cuda.current_stream().wait_stream(s)
-    torch.cuda.synchronize()
-    return g
+def point(layers, shape, B, sparsity, steps, warmup, dist, lookahead=True, kv_seed=None):
+    """One (batch, sparsity) point: the step of the whole stack as a CUDA
+    graph, timed; returns the measurement and the stack (for more timing)."""
+    keep = 1.0 - sparsity
+    k, k_h = wl.k_for(keep, shape.N), wl.k_for(keep, shape.h)
+    ls = with_kv(layers, shape, B, kv_seed) if kv_seed is not None else layers
+    stk = build_stack(ls, shape, B, k, k_h, lookahead)
+    x = wl.make_input(shape.with_(B=B), 7 + B, "cuda")
+    g, launches = capture(stk, x, shape.L)
+    ms = time_graph(g, steps, warmup, dist)
+    km, kh = selected_counts(stk)
+    kp = nonzero_neurons(stk)
+    lb = layer_bytes(shape, km, kp, kh, B)
+    n = len(layers)
+    us = ms * 1e3 / n
+    res = {"batch": B, "sparsity": sparsity, "k": k, "k_h": k_h, "k_union": km, "k_eff": kp, "k_h_union": kh,
+           "us_per_layer": us, "tokens_per_s": B * 1e3 / ms, "bytes_per_layer": lb.total,
+           "gbs": lb.total / us / 1e3, "launches_per_step": launches}
+    return res, stk, g, x, lb
 
 
 # Source headers of each main-path kernel, for matching a committed ncu
 # capture to the code that runs now.
 KERNEL_HEADERS = {
-    "attn_in": ("dv_common.cuh", "dv_fused.cuh", "dv_colowner.cuh"),
-    "mlp_block": ("dv_common.cuh", "dv_fused.cuh", "dv_colowner.cuh"),
+    "attn_in": ("dv_common.cuh", "dv_fused.cuh", "dv_colowner.cuh", "dv_stream.cuh"),
+    "mlp_block": ("dv_common.cuh", "dv_fused.cuh", "dv_colowner.cuh", "dv_stream.cuh"),
     "attn_out": ("dv_common.cuh", "dv_kernels.cuh", "dv_fused.cuh"),
+    "predict_neurons": ("dv_common.cuh", "dv_fused.cuh", "dv_api_kernels.cuh"),
 }
 
 
@@ -262,10 +302,11 @@ def kernel_sources_digest(op):
     return h.hexdigest()[:16]
 
 
-def measured_traffic(op, profiles_dir=None):
+def measured_traffic(op, profiles_dir=None, workload=None):
     """Per-launch DRAM bytes (read + write) of `op`'s kernel from the ncu
-    summary under profiles/ (lines `traffic <op> <bytes> <sha256 prefix>`),
-    or None when no capture exists or the kernel's headers changed since."""
+    summaries under profiles/ (lines `traffic <op> <bytes> <sha256 prefix>
+    [workload]`), or None when no capture exists or the kernel's headers
+    changed since. With `workload`, only lines naming it count."""
     import glob
 
     digest = kernel_sources_digest(op)
@@ -274,17 +315,19 @@ def measured_traffic(op, profiles_dir=None):
         with open(path) as fh:
             for line in fh:
                 parts = line.split()
-                if len(parts) == 4 and parts[0] == "traffic" and parts[1] == op and parts[3] == digest:
+                if len(parts) in (4, 5) and parts[0] == "traffic" and parts[1] == op and parts[3] == digest:
+                    if workload is not None and (len(parts) < 5 or parts[4] != workload):
+                        continue
                     return {"bytes": int(parts[2]), "source": os.path.relpath(path, ROOT)}
     return None
 
 
 def kernel_roofline(stk, shape, B, pos, peak_gbs, reps=20):
-    """Average duration of each main-path kernel in the look-ahead steady
+    """Average duration of each kernel of the step in the look-ahead steady
     state (sets given): one CUDA graph per kernel with that kernel's call for
     every layer, timed with CUDA events on the launching stream; each
     kernel's algorithmic bytes per launch divided by its average duration.
-    The residual state is restored afterwards."""
+    The residual state and caches are restored afterwards."""
     from attention_predictor_gemv_b200 import binding as bd
 
     nL = len(stk.layers)
@@ -293,18 +336,30 @@ def kernel_roofline(stk, shape, B, pos, peak_gbs, reps=20):
     kp = nonzero_neurons(stk)
     k, kh = selected_counts(stk)
     lb = layer_bytes(shape, k, kp, kh, B)
+    w = acct.ELEM[shape.wdtype]
     p, ws = stk.p, stk.ws_main
+    pred_bytes = shape.N * shape.r * w + 4 * shape.N + 2 * 4 * B * shape.N + 4 * int(round(k))
     calls = {
         "attn_in": (lambda l: bd.dv_decode_layer_begin(stk.layers[l], p, x, pos, ws, sel=stk.io_given[l],
-                                                       trace=stk.io_trace_y[l]), lb.qkv),
+                                                       trace=stk.io_trace_y[l]), lb.qkv, range(nL)),
         "attn_out": (lambda l: bd.dv_decode_layer_attn(stk.layers[l], p, x, pos, ws, sel=stk.io_given[l],
-                                                       trace=stk.io_trace_y[l]), lb.kv + lb.wo),
+                                                       trace=stk.io_trace_y[l]), lb.kv + lb.wo, range(nL)),
         "mlp_block": (lambda l: bd.dv_decode_layer_mlp(stk.layers[l], p, x, ws, sel=stk.io_given[l],
-                                                       trace=stk.io_trace_y[l]), lb.w1 + lb.w2),
+                                                       trace=stk.io_trace_y[l]), lb.w1 + lb.w2, range(nL)),
     }
+    if stk.fuse_ahead and nL > 1:
+        # the look-ahead tails on the main stream: neuron scores z B^T + b1 and
+        # their selection; the head selection
+        calls["predict_neurons"] = (
+            lambda l: bd.dv_predict_layer_tail(stk.layers[l], p, stk.io_sets[l], stk.ws_ahead[l % 2],
+                                               sets=bd.DV_SET_NEURONS), pred_bytes, range(1, nL))
+        calls["select_heads"] = (
+            lambda l: bd.dv_predict_layer_tail(stk.layers[l], p, stk.io_sets[l], stk.ws_ahead[l % 2],
+                                               sets=bd.DV_SET_HEADS), 2 * 4 * B * shape.h, range(1, nL))
     res = {}
-    for name, (fn, nbytes) in calls.items():
-        g = graph_of(lambda: [fn(l) for l in range(nL)])
+    for name, (fn, nbytes, ls) in calls.items():
+        ls = list(ls)
+        g = graph_of(lambda: [fn(l) for l in ls])
         for _ in range(3):
             g.replay()
         torch.cuda.synchronize()
@@ -314,7 +369,7 @@ def kernel_roofline(stk, shape, B, pos, peak_gbs, reps=20):
             g.replay()
         e1.record()
         e1.synchronize()
-        us = e0.elapsed_time(e1) * 1000.0 / (reps * nL)
+        us = e0.elapsed_time(e1) * 1000.0 / (reps * len(ls))
         res[name] = {"us": us, "bytes": nbytes, "gbs": nbytes / us / 1e3, "frac": nbytes / us / 1e3 / peak_gbs}
         del g
     for t, (K, V) in zip((L.t for L in stk.layers), snap):
@@ -323,71 +378,257 @@ def kernel_roofline(stk, shape, B, pos, peak_gbs, reps=20):
     return res, lb, k, kp, kh
 
 
-def big_config(args, peak_gbs, dist):
-    """OPT-175B-shaped layers (d=12288, N=49152, h=96, dh=128, KV 2048) at
-    85% sparsity on neurons and heads, batch 1: the regime where the selected
-    bytes (about 0.65 GB per layer) rather than latency bound the step."""
-    shape = wl.CONFIGS["opt-175b"].with_(B=1)
-    k, k_h = wl.k_for(0.15, shape.N), wl.k_for(0.15, shape.h)
-    stk, layers = build_stack(shape, args.big_layers, 1, k, k_h, True, seed0=5000)
-    x = wl.make_input(shape, 11, "cuda")
-    g, _ = capture(stk, x, shape.L)
-    ms = time_graph(g, 10, 3, dist)
-    kern, lb, km, kp, kh = kernel_roofline(stk, shape, 1, shape.L, peak_gbs, reps=5)
-    us_layer = ms * 1e3 / args.big_layers
-    out = {"workload": f"{args.big_layers} OPT-175B-shaped layers: d={shape.d}, N={shape.N}, r={shape.r}, "
-                       f"h={shape.h}, dh={shape.dh}, KV length {shape.L}, batch 1, k={k} (15%), k_h={k_h} (15%), "
-                       "look-ahead", "us_per_layer_step": us_layer, "bytes_per_layer": lb.total,
-           "effective_gbs": lb.total / us_layer / 1e3, "effective_frac": lb.total / us_layer / 1e3 / peak_gbs,
-           "selected": {"k": km, "k_eff": kp, "k_h": kh}, "kernels": kern}
-    del g, stk, layers
+def free_gpu():
+    import gc
+
+    gc.collect()
+    torch.cuda.synchronize()
     torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------------------
+# secondary workloads
+# ---------------------------------------------------------------------------
+
+
+def sweep_175b(layers, shape, args, dist):
+    """Sparsity 50/75/85/95% x batch 1/2/4/8/16 on the headline stack's
+    weights, and the dense path (every neuron and head) at each batch."""
+    out = []
+    for B in (1, 2, 4, 8, 16):
+        for s in (0.50, 0.75, 0.85, 0.95, 0.0):
+            res, stk, g, x, _ = point(layers, shape, B, s, 6, 2, dist, kv_seed=9000 + 100 * B)
+            res["dense"] = s == 0.0
+            out.append(res)
+            del stk, g, x
+        free_gpu()
     return out
 
 
-def cpu_baseline(shape, B, k, k_h, seconds, seed=1000):
-    """The oracle (float64 numpy) on a bounded sample: repeated layer-steps of
-    one layer of the same shape, on the host cores."""
-    from threadpoolctl import threadpool_info
+def generation(shape, nL, lookahead, tokens, dist):
+    """OPT-6.7B-shaped stack: `tokens` decode steps with the KV position
+    advancing (one CUDA graph per position), timed as one generation."""
+    layers = make_layers(shape, nL, 3000)
+    k, k_h = wl.DEFAULT_SELECTION["opt-6.7b"]
+    res = {}
+    for la in ((True, False) if lookahead else (False,)):
+        stk = build_stack(layers, shape, 1, k, k_h, la)
+        x = wl.make_input(shape, 3, "cuda")
+        graphs = [graph_of(lambda p=shape.L + i: stk.step(x, p)) for i in range(tokens)]
+        for g in graphs:  # warm-up generation
+            g.replay()
+        barrier(dist)
+        times = []
+        for _ in range(2):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for g in graphs:
+                g.replay()
+            e1.record()
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1))
+        barrier(dist)
+        ms = float(np.mean(times))
+        km, kh = selected_counts(stk)
+        kp = nonzero_neurons(stk)
+        lb = layer_bytes(shape, km, kp, kh, 1)  # bytes at the first position; KV grows by one slot per token
+        us = ms * 1e3 / (tokens * nL)
+        res["lookahead" if la else "synchronous"] = {
+            "us_per_layer": us, "tokens_per_s": tokens * 1e3 / ms, "ms_per_token": ms / tokens,
+            "k": k, "k_h": k_h, "k_eff": kp, "bytes_per_layer": lb.total, "gbs": lb.total / us / 1e3}
+        del graphs, stk, x
+        free_gpu()
+    del layers
+    free_gpu()
+    return {"workload": f"{nL} OPT-6.7B-shaped layers: d={shape.d}, N={shape.N}, r={shape.r}, h={shape.h}, "
+                        f"dh={shape.dh}, KV positions {shape.L}..{shape.L + tokens - 1}, batch 1, k={k} (8%), "
+                        f"k_h={k_h} (20%); {tokens} generated tokens, one graph per position", **res}
+
+
+def opt66b(shape, nL, dist):
+    """OPT-66B-shaped stack, 64 layers (about 139 GB of weights), batch
+    1/2/4/8 with union sets, 6% of neurons and 20% of heads per row."""
+    layers = make_layers(shape, nL, 4000)
+    k, k_h = wl.DEFAULT_SELECTION["opt-66b"]
+    out = []
+    for B in (1, 2, 4, 8):
+        ls = with_kv(layers, shape, B, 4500 + B) if B > 1 else layers
+        stk = build_stack(ls, shape, B, k, k_h, True)
+        x = wl.make_input(shape.with_(B=B), 5, "cuda")
+        g, launches = capture(stk, x, shape.L)
+        ms = time_graph(g, 6, 2, dist)
+        km, kh = selected_counts(stk)
+        kp = nonzero_neurons(stk)
+        lb = layer_bytes(shape, km, kp, kh, B)
+        us = ms * 1e3 / nL
+        out.append({"batch": B, "k": k, "k_h": k_h, "k_union": km, "k_eff": kp, "k_h_union": kh, "us_per_layer": us,
+                    "tokens_per_s": B * 1e3 / ms, "bytes_per_layer": lb.total, "gbs": lb.total / us / 1e3})
+        del g, stk, x, ls
+        free_gpu()
+    del layers
+    free_gpu()
+    return {"workload": f"{nL} OPT-66B-shaped layers: d={shape.d}, N={shape.N}, r={shape.r}, h={shape.h}, "
+                        f"dh={shape.dh}, KV length {shape.L}, k={k} (6%), k_h={k_h} (20%) per row, look-ahead",
+            "points": out}
+
+
+def opt13b(dist):
+    """OPT-1.3B-shaped stack (24 layers, 2.6 GB of weights), batch 1: the
+    neuron x head fraction sweep of the configuration."""
+    shape = wl.CONFIGS["opt-1.3b"]
+    layers = make_layers(shape, 24, 1000)
+    out = []
+    for kf in (0.05, 0.10, 0.20, 1.00):
+        for hf in (0.25, 0.50, 1.00):
+            k, k_h = wl.k_for(kf, shape.N), wl.k_for(hf, shape.h)
+            stk = build_stack(layers, shape, 1, k, k_h, True)
+            x = wl.make_input(shape, 7, "cuda")
+            g, _ = capture(stk, x, shape.L)
+            ms = time_graph(g, 20, 3, dist)
+            km, kh = selected_counts(stk)
+            lb = layer_bytes(shape, km, nonzero_neurons(stk), kh, 1)
+            us = ms * 1e3 / 24
+            out.append({"k_frac": kf, "kh_frac": hf, "k": k, "k_h": k_h, "us_per_layer": us,
+                        "bytes_per_layer": lb.total, "gbs": lb.total / us / 1e3})
+            del g, stk, x
+    del layers
+    free_gpu()
+    return {"workload": "24 OPT-1.3B-shaped layers: d=2048, N=8192, r=256, h=32, dh=64, KV length 512, batch 1, "
+                        "look-ahead; 2.6 GB of weights streamed per step", "points": out}
+
+
+def tiny_latency(dist):
+    """The tiny fp32 layer (L2-resident): latency of one layer-step."""
+    shape = wl.CONFIGS["tiny"]
+    layers = make_layers(shape, 1, 0)
+    k, k_h = wl.DEFAULT_SELECTION["tiny"]
+    stk = build_stack(layers, shape, 1, k, k_h, False)
+    x = wl.make_input(shape, 0, "cuda")
+    g, launches = capture(stk, x, shape.L)
+    ms = time_graph(g, 200, 20, dist)
+    del g, stk
+    return {"workload": "1 tiny fp32 layer: d=256, N=1024, r=32, h=4, dh=64, KV length 64, k=128, k_h=2, "
+                        "synchronous prediction (L2-resident: latency only)", "us_per_layer": ms * 1e3,
+            "launches_per_step": launches}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (reported baseline; also the reference arm)
+# ---------------------------------------------------------------------------
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_layer_from(t):
+    """The oracle's float64 layer from a layer's tensors (device or host)."""
+    from oracle import dejavu_oracle as O
+
+    def f(a):
+        a = a.detach().cpu().contiguous()
+        if a.dtype == torch.bfloat16:
+            return O.bf16_bits_to_f64(a.view(torch.int16).numpy().view(np.uint16))
+        return a.double().numpy()
+
+    return O.LayerF64(PA=f(t["PA"]), Wqkv=f(t["Wqkv"]), bqkv=None, WOt=f(t["WOt"]), bO=None, K=f(t["K"]),
+                      V=f(t["V"]), At=f(t["At"]), Bm=f(t["Bm"]), b1=f(t["b1"]), W1t=f(t["W1t"]), W2t=f(t["W2t"]),
+                      kv_round="bf16" if t["K"].dtype == torch.bfloat16 else None)
+
+
+def time_oracle(OL, shape, k, k_h, seconds, threads=None, max_steps=None):
+    """Repeated oracle layer-steps (float64 numpy: LN, predictors, selection,
+    sparse MHA, sparse MLP) for about `seconds`; `threads` limits the BLAS
+    threads (None: all). Returns (us per layer-step, steps)."""
+    from threadpoolctl import threadpool_limits
 
     from oracle import dejavu_oracle as O
 
-    t = wl.make_layer(shape, seed, "cpu")
-    f = lambda a: O.bf16_bits_to_f64(a.contiguous().view(torch.int16).numpy().view(np.uint16)) \
-        if a.dtype == torch.bfloat16 else a.double().numpy()  # noqa: E731
-    L = O.LayerF64(PA=f(t["PA"]), Wqkv=f(t["Wqkv"]), bqkv=None, WOt=f(t["WOt"]), bO=None, K=f(t["K"]), V=f(t["V"]),
-                   At=f(t["At"]), Bm=f(t["Bm"]), b1=f(t["b1"]), W1t=f(t["W1t"]), W2t=f(t["W2t"]))
     P = O.LayerParams(k=k, k_h=k_h, scale=1.0 / float(np.sqrt(shape.dh)))
-    x = wl.make_input(shape, 0, "cpu").double().numpy()
+    x = wl.make_input(shape.with_(B=1), 0, "cpu").double().numpy()
     n, t0 = 0, time.perf_counter()
-    while True:
-        O.decode_layer(x, L, P, shape.L)
-        n += 1
-        el = time.perf_counter() - t0
-        if el >= seconds:
-            break
-    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    return {"value": el * 1e6 / n, "unit": "us/layer-step", "cores": int(threads), "kind": "oracle",
-            "sample": f"{n} layer-steps of one {CONFIG}-shaped layer (d={shape.d}, N={shape.N}, h={shape.h}, "
-                      f"dh={shape.dh}, KV {shape.L}+1, B={B}, k={k}, k_h={k_h}), float64 numpy, full layer "
-                      f"(LN, predictors, selection, sparse MHA, sparse MLP)"}
+    with threadpool_limits(limits=threads):
+        while True:
+            O.decode_layer(x, OL, P, shape.L)
+            n += 1
+            el = time.perf_counter() - t0
+            if el >= seconds or (max_steps and n >= max_steps):
+                break
+    return el * 1e6 / n, n
+
+
+def cpu_baseline(headline_layer, shape, k, k_h, seconds):
+    """The oracle on the host cores: one headline-shaped layer-step (sparse),
+    single-threaded and on all cores; and configs tiny, OPT-1.3B and one
+    OPT-6.7B layer, sparse and dense, single-threaded and on all cores."""
+    cores = host_cores()
+    OL = oracle_layer_from(headline_layer)
+    v_all, n_all = time_oracle(OL, shape, k, k_h, 3 * seconds)
+    v_one, n_one = time_oracle(OL, shape, k, k_h, 3 * seconds, threads=1)
+    del OL
+    table = []
+    for name in ("tiny", "opt-1.3b", "opt-6.7b"):
+        s = wl.CONFIGS[name].with_(B=1)
+        t = wl.make_layer(s, 1000, "cpu")
+        OLs = oracle_layer_from(t)
+        ks, khs = wl.DEFAULT_SELECTION[name]
+        for mode, kk, hh in (("sparse", ks, khs), ("dense", s.N, s.h)):
+            for thr in (1, None):
+                us, n = time_oracle(OLs, s, kk, hh, seconds, threads=thr)
+                table.append({"workload": name, "mode": mode, "k": kk, "k_h": hh,
+                              "threads": 1 if thr == 1 else cores, "us_per_layer_step": us, "steps": n})
+        del OLs, t
+    return {"value": v_all, "unit": "us/layer-step", "cores": cores, "kind": "oracle",
+            "sample": f"{n_all} layer-steps of one OPT-175B-shaped layer (d={shape.d}, N={shape.N}, r={shape.r}, "
+                      f"h={shape.h}, dh={shape.dh}, KV {shape.L}+1, B=1, k={k}, k_h={k_h}), float64 numpy, full "
+                      f"layer (LN, predictors, selection, sparse MHA, sparse MLP), all {cores} host cores",
+            "single_thread": {"value": v_one, "steps": n_one}, "table": table}
 
 
 def run_reference(args, rank, dist):
-    shape = wl.CONFIGS[CONFIG].with_(B=args.batch)
-    k, k_h = wl.k_for(args.k_frac, shape.N), wl.k_for(args.kh_frac, shape.h)
+    """The reference arm: the oracle (float64 numpy, host cores) on the
+    headline workload, one layer-step per timed step (the layer built on the
+    host; the GPU is not used)."""
     if rank != 0:
         return
-    per_step = max(1.0, 60.0 / max(1, args.steps + args.warmup))
-    cb = cpu_baseline(shape, args.batch, k, k_h, min(per_step, args.cpu_seconds))
-    v = cb["value"]
+    shape = wl.CONFIGS[args.config]
+    keep = 1.0 - args.sparsity
+    k, k_h = wl.k_for(keep, shape.N), wl.k_for(keep, shape.h)
+    t = wl.make_layer(shape.with_(B=1), 5000, "cpu")
+    OL = oracle_layer_from(t)
+    del t
+    time_oracle(OL, shape, k, k_h, 0.0, max_steps=max(1, args.warmup))
+    v, n = time_oracle(OL, shape, k, k_h, 1e9, max_steps=max(1, args.steps))
+    cores = host_cores()
+    nL = args.layers or shape.layers
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "us", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v * args.layers / 1e3,
-            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{CONFIG}-shaped decoder layer, batch {args.batch}, KV {shape.L}, "
-                                   f"k={k}/{shape.N}, k_h={k_h}/{shape.h}", "layers": args.layers},
-            "cpu_baseline": cb, "e2e": {"value": v, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v * nL / 1e3, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(shape, nL, args.batch, k, k_h, not args.no_lookahead),
+            "cpu_baseline": {"value": v, "unit": "us/layer-step", "cores": cores, "kind": "oracle",
+                             "sample": f"{n} layer-steps of one {args.config}-shaped layer (B=1, k={k}, k_h={k_h}), "
+                                       f"float64 numpy on {cores} host cores, one layer-step per timed step"},
+            "e2e": {"value": v, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def config_of(shape, nL, B, k, k_h, lookahead):
+    name = {"opt-175b": "OPT-175B", "opt-66b": "OPT-66B", "opt-6.7b": "OPT-6.7B", "opt-1.3b": "OPT-1.3B",
+            "tiny": "tiny"}
+    key = [n for n, s in wl.CONFIGS.items() if s.d == shape.d and s.N == shape.N][0]
+    return {"workload": f"{nL} {name[key]}-shaped decoder layers (bf16 weights and KV cache, fp32 arithmetic): "
+                        f"d={shape.d}, N={shape.N}, r={shape.r}, h={shape.h}, dh={shape.dh}, KV length {shape.L}, "
+                        f"batch {B}, k={k} ({k / shape.N:.0%}), k_h={k_h} ({k_h / shape.h:.0%}), "
+                        f"{'look-ahead' if lookahead else 'synchronous'} prediction",
+            "global_batch": B, "seq_len": shape.L + 1}
+
+
+# ---------------------------------------------------------------------------
+# main
+# ---------------------------------------------------------------------------
 
 
 def main():
@@ -410,12 +651,15 @@ def main():
     peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
 
     B = args.batch
-    shape = wl.CONFIGS[CONFIG].with_(B=B)
-    k, k_h = wl.k_for(args.k_frac, shape.N), wl.k_for(args.kh_frac, shape.h)
+    shape = wl.CONFIGS[args.config].with_(B=B)
+    nL = args.layers or shape.layers
+    keep = 1.0 - args.sparsity
+    k, k_h = wl.k_for(keep, shape.N), wl.k_for(keep, shape.h)
     pos = shape.L
     torch.manual_seed(rank)
-    pf = dict(prefetch=args.prefetch, prefetch_w2=not args.no_prefetch_w2)
-    stk, layers = build_stack(shape, args.layers, B, k, k_h, not args.no_lookahead, seed0=1000 + 100 * rank, **pf)
+    layers = make_layers(shape, nL, 5000 + 100 * rank)
+    ls = with_kv(layers, shape, B, 6000 + rank) if B > 1 else layers
+    stk = build_stack(ls, shape, B, k, k_h, not args.no_lookahead)
     x0 = wl.make_input(shape, 7 + rank, "cuda")
     x = x0.clone()
     g, launches_per_step = capture(stk, x, pos)
@@ -446,66 +690,71 @@ def main():
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist)
 
     ops, lb, kmean, kp, kh = kernel_roofline(stk, shape, B, pos, peak_gbs)
-    dom = max(ops, key=lambda n: ops[n]["us"])
-    traffic = measured_traffic(dom)
-    total_layer_bytes = lb.total
-    us_layer = ms * 1e3 / args.layers
-    value = ms * 1e3 / (args.layers * world)  # whole job: all ranks' layer-steps in the max-over-ranks time
-
-    sweep = []
-    if not args.no_sweep:
-        for kf in (0.05, 0.10, 0.20, 1.00):
-            for hf in (0.25, 0.50, 1.00):
-                kk, hh = wl.k_for(kf, shape.N), wl.k_for(hf, shape.h)
-                s2, _ = build_stack(shape, args.layers, B, kk, hh, not args.no_lookahead, layers=layers, **pf)
-                g2, _ = capture(s2, x, pos)
-                m2 = time_graph(g2, max(10, args.steps // 2), 3, dist)
-                kk_m, hh_m = selected_counts(s2)
-                b2 = layer_bytes(shape, kk_m, nonzero_neurons(s2), hh_m, B).total
-                sweep.append({"k_frac": kf, "kh_frac": hf, "k": kk, "k_h": hh, "us_per_layer": m2 * 1e3 / args.layers,
-                              "bytes_per_layer": b2, "gbs": b2 / (m2 * 1e3 / args.layers) / 1e3})
-                del g2, s2
-
-    big = None
-    if not args.no_big:
-        big = big_config(args, peak_gbs, dist)
+    main_ops = [n for n in ("attn_in", "attn_out", "mlp_block") if n in ops]
+    dom = max(main_ops, key=lambda n: ops[n]["us"])
+    wl_tag = f"{args.config}-b{B}-s{int(round(args.sparsity * 100))}"
+    traffic = measured_traffic(dom, workload=wl_tag)
+    us_layer = ms * 1e3 / nL
+    value = ms * 1e3 / (nL * world)  # whole job: all ranks' layer-steps in the max-over-ranks time
+    del g
+    side = {}
+    if world == 1:
+        headline_layer0 = layers[0]
+        del stk
+        free_gpu()
+        if not args.no_sweep:
+            side["opt175b_sweep"] = sweep_175b(layers, shape.with_(B=1), args, dist)
+        cpu = None
+        if rank == 0 and not args.no_cpu_baseline:
+            cpu = cpu_baseline(headline_layer0, shape.with_(B=1), k, k_h, args.cpu_seconds)
+        del layers, ls, headline_layer0
+        free_gpu()
+        if not args.no_extra:
+            side["opt6.7b_generation"] = generation(wl.CONFIGS["opt-6.7b"], 32, True, 128, dist)
+            side["opt66b"] = opt66b(wl.CONFIGS["opt-66b"], 64, dist)
+            side["opt1.3b"] = opt13b(dist)
+            side["tiny"] = tiny_latency(dist)
+    else:
+        cpu = None
 
     line = {
         "metric": METRIC, "value": value, "unit": "us", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": f"{CONFIG}-shaped decoder (bf16 weights and KV cache, fp32 arithmetic): "
-                               f"{args.layers} layers of d={shape.d}, N={shape.N}, "
-                               f"r={shape.r}, h={shape.h}, dh={shape.dh}, KV length {shape.L}, batch {B}, "
-                               f"k={k} ({args.k_frac:.0%}), k_h={k_h} ({args.kh_frac:.0%}), "
-                               f"{'look-ahead' if not args.no_lookahead else 'synchronous'} prediction",
-                   "global_batch": B * world, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2: 24 layers, 2.6 GB of weights streamed per step"},
+        "config": dict(config_of(shape, nL, B, k, k_h, not args.no_lookahead),
+                       parallelism=f"replicas x{world}",
+                       l2=f"inputs larger than L2: {nL} layers, {weight_bytes(shape) * nL / 1e9:.0f} GB of "
+                          "weights streamed per step"),
         "tokens_per_s": B * world * 1e3 / ms,
         "us_per_layer_step": us_layer,
         "selected": {"k": kmean, "k_eff": kp, "k_h": kh},
-        "bytes_per_layer": total_layer_bytes,
-        "effective_gbs": total_layer_bytes / us_layer / 1e3,
-        "effective_frac": total_layer_bytes / us_layer / 1e3 / peak_gbs,
+        "bytes_per_layer": lb.total,
+        "effective_gbs": lb.total / us_layer / 1e3,
+        "effective_frac": lb.total / us_layer / 1e3 / peak_gbs,
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": ops[dom]["gbs"], "peak": peak_gbs, "unit": "GB/s",
                      "frac": ops[dom]["frac"], "traffic": traffic["bytes"] if traffic else None,
                      "traffic_source": traffic["source"] if traffic else None,
                      "algorithmic_bytes": ops[dom]["bytes"], "peak_source": peak_src, "per_op": ops},
-        "e2e": {"value": e2e_ms * 1e3 / (args.layers * world), "unit": "us", "ms_per_step": e2e_ms,
+        "e2e": {"value": e2e_ms * 1e3 / (nL * world), "unit": "us", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": xh.numel() * 4, "d2h_bytes_per_step": oh.numel() * 4},
         "gpu_launches": int(launches_per_step * args.steps),
         "launches_per_step": int(launches_per_step),
         "clocks": clocks,
-        "sweep": sweep,
-        "opt175b_shaped": big,
+        **side,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(shape, B, k, k_h, args.cpu_seconds)
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del g
     if dist is not None:
         dist.destroy_process_group()
+
+
+def weight_bytes(shape):
+    """Bytes of one layer's weights and predictors (bf16 / fp32)."""
+    w = acct.ELEM[shape.wdtype]
+    return (2 * shape.N * shape.d + 4 * shape.h * shape.dh * shape.d + shape.h * shape.d + shape.r * shape.d
+            + shape.N * shape.r) * w
 
 
 if __name__ == "__main__":
