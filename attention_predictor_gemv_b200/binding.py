@@ -23,6 +23,7 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "dejavu.h")
 DV_OK, DV_ERR_ARG, DV_ERR_ALIGN, DV_ERR_UNSUPPORTED, DV_ERR_CUDA, DV_ERR_DEVICE, DV_ERR_WORKSPACE = range(7)
 DV_F32, DV_BF16 = 0, 1
 DV_TOPK, DV_THRESHOLD = 0, 1
+DV_ACT_RELU, DV_ACT_GELU = 0, 1
 (DV_OP_PREDICT_MLP, DV_OP_PREDICT_HEADS, DV_OP_TOPK, DV_OP_SPARSE_MLP, DV_OP_SPARSE_MHA,
  DV_OP_DECODE_LAYER) = range(6)
 
@@ -52,7 +53,7 @@ class LayerWeightsC(ctypes.Structure):
 
 class LayerParamsC(ctypes.Structure):
     _fields_ = [("k", _c_int), ("tau", _c_float), ("mode", _c_int), ("k_h", _c_int), ("tau_h", _c_float),
-                ("mode_h", _c_int), ("scale", _c_float), ("eps", _c_float)]
+                ("mode_h", _c_int), ("scale", _c_float), ("eps", _c_float), ("act", _c_int), ("exact_kv", _c_int)]
 
 
 class LayerIOC(ctypes.Structure):
@@ -80,6 +81,9 @@ _lib_dv_topk = _sig("dv_topk", _c_int, [_p, _c_int, _c_int, _c_int, _c_float, _c
 _lib_dv_sparse_mlp = _sig("dv_sparse_mlp", _c_int,
                           [_p, _c_int, _c_int, _c_int, _p, _p, _p, _p, _c_int, _p, _p, _c_int, _p, _c_int, _p, _c_size,
                            _p])
+_lib_dv_sparse_mlp_act = _sig("dv_sparse_mlp_act", _c_int,
+                              [_p, _c_int, _c_int, _c_int, _p, _p, _p, _p, _c_int, _p, _p, _c_int, _p, _c_int, _c_int,
+                               _p, _c_size, _p])
 _lib_dv_sparse_mha = _sig("dv_sparse_mha", _c_int,
                           [_p, _c_int, _c_int, _c_int, _c_int, _p, _p, _p, _p, _c_int, _p, _p, _c_int, _c_int, _c_int,
                            _c_float, _p, _p, _c_int, _p, _c_int, _p, _c_size, _p])
@@ -234,14 +238,18 @@ def dv_topk_static(scores, k, idx, count, tau=0.0, mode=DV_TOPK, stream=None):
            "dv_topk_static")
 
 
-def dv_sparse_mlp(y, W1t, b1, W2t, b2, idx, count, k_max, out, ws, accumulate=False, stream=None):
+def dv_sparse_mlp(y, W1t, b1, W2t, b2, idx, count, k_max, out, ws, accumulate=False, stream=None, act=DV_ACT_RELU):
+    """dv_sparse_mlp (ReLU), or dv_sparse_mlp_act with another activation."""
     B, d = y.shape
     N = W1t.shape[0]
-    _check(_lib_dv_sparse_mlp(_ptr(y, torch.float32, "y"), B, d, N, _ptr(W1t, None, "W1t"),
-                              _ptr(b1, torch.float32, "b1"), _ptr(W2t, W1t.dtype, "W2t"), _ptr(b2, torch.float32, "b2"),
-                              _wdt(W1t), _ptr(idx, torch.int32, "idx"), _ptr(count, torch.int32, "count"), int(k_max),
-                              _ptr(out, torch.float32, "out"), int(bool(accumulate)), _ptr(ws, torch.uint8, "ws"),
-                              ws.numel(), _stream(stream)), "dv_sparse_mlp")
+    args = [_ptr(y, torch.float32, "y"), B, d, N, _ptr(W1t, None, "W1t"), _ptr(b1, torch.float32, "b1"),
+            _ptr(W2t, W1t.dtype, "W2t"), _ptr(b2, torch.float32, "b2"), _wdt(W1t), _ptr(idx, torch.int32, "idx"),
+            _ptr(count, torch.int32, "count"), int(k_max), _ptr(out, torch.float32, "out"), int(bool(accumulate))]
+    tail = [_ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)]
+    if act == DV_ACT_RELU:
+        _check(_lib_dv_sparse_mlp(*args, *tail), "dv_sparse_mlp")
+    else:
+        _check(_lib_dv_sparse_mlp_act(*args, int(act), *tail), "dv_sparse_mlp_act")
 
 
 def dv_sparse_mha(y, Wqkv, bqkv, WOt, bO, Kc, Vc, pos, scale, head_idx, head_count, kh_max, out, ws,
@@ -282,8 +290,10 @@ class Layer:
                                g("b1", torch.float32), g("W1t"), g("W2t"), g("b2", torch.float32))
 
 
-def params(k, k_h, scale, eps=1e-5, tau=0.0, mode=DV_TOPK, tau_h=0.0, mode_h=DV_TOPK) -> LayerParamsC:
-    return LayerParamsC(int(k), float(tau), int(mode), int(k_h), float(tau_h), int(mode_h), float(scale), float(eps))
+def params(k, k_h, scale, eps=1e-5, tau=0.0, mode=DV_TOPK, tau_h=0.0, mode_h=DV_TOPK, act=DV_ACT_RELU,
+           exact_kv=False) -> LayerParamsC:
+    return LayerParamsC(int(k), float(tau), int(mode), int(k_h), float(tau_h), int(mode_h), float(scale), float(eps),
+                        int(act), int(bool(exact_kv)))
 
 
 def layer_io(yA=None, scores_h=None, head_idx=None, head_count=None, yM=None, scores=None, idx=None,

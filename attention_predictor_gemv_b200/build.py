@@ -19,9 +19,10 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdejavu.so")
 # One translation unit per kernel family, compiled in parallel, then linked.
 SOURCES = ["dv_api.cu", "dv_inst_legacy.cu", "dv_inst_legacy_attn.cu", "dv_inst_attn_in.cu", "dv_inst_attn_out.cu", "dv_inst_attn_out_f32.cu",
-           "dv_inst_mlp.cu", "dv_inst_pred.cu"]
+           "dv_inst_mlp.cu", "dv_inst_pred.cu", "dv_inst_tc.cu"]
 HEADERS = ["dv_common.cuh", "dv_kernels.cuh", "dv_fused.cuh", "dv_colowner.cuh", "dv_launch.cuh", "dv_launchers.cuh",
-           "dv_api_kernels.cuh", "dv_stream.cuh"]
+           "dv_api_kernels.cuh", "dv_stream.cuh", "dv_tc.cuh", "dv_tc_args.h",
+           "dv_tc_launch.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr"]

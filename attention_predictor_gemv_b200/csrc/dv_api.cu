@@ -9,6 +9,7 @@
 #include "../../include/dejavu.h"
 #include "dv_api_kernels.cuh"
 #include "dv_launchers.cuh"
+#include "dv_tc_launch.h"
 
 using namespace dv;
 using bf16 = __nv_bfloat16;
@@ -29,8 +30,8 @@ constexpr int KH_LIMIT = 1000;  // B * kh_max counters must fit the header
 struct Layout {
   size_t status, sel_ticket_h, sel_ticket_m, pa_ticket, pb_ticket, attn_ctr, hist, t1;
   size_t yA, yM, z, scores_h, bm_h, head_idx, head_count, scores, bm_m, idx, count;
-  size_t q, part, H, seg_idx, seg_a, seg_cnt, total;
-  int nseg, SEG, nsplit_max;
+  size_t q, part, H, seg_idx, seg_a, seg_cnt, tc_act, tc_rowid, tc_tiles, total;
+  int nseg, SEG, nsplit_max, KC;
 };
 
 bool dims_ok(const dv_dims& D) {
@@ -73,6 +74,12 @@ Layout layout(const dv_dims& D, int wbytes) {
   L.seg_idx = take(4ull * L.nseg * L.SEG);
   L.seg_a = take(4ull * L.nseg * L.SEG * B);
   L.seg_cnt = take(4ull * (L.nseg > 0 ? L.nseg : 1));
+  // tensor-core MLP: activations compacted per tile of 128 selected neurons
+  const int tiles = tc_tiles(D.k_max);
+  L.KC = tiles * TC_M;
+  L.tc_act = take(4ull * TC_N * L.KC);
+  L.tc_rowid = take(4ull * (L.KC > 0 ? L.KC : 1));
+  L.tc_tiles = take(4ull * (tiles > 0 ? tiles : 1));
   L.total = o;
   return L;
 }
@@ -95,6 +102,17 @@ dv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DV_OK : DV_ERR_
     dv_status _s = (expr);        \
     if (_s != DV_OK) return _s;   \
   } while (0)
+
+// Tensor-core path for batch 5..16 (defined below)
+bool tc_ok(int B, dv_dtype wdt, int dh, int k_max);
+dv_status tc_mlp(const Layout& L, void* ws, const float* y, int B, int d, int N, const void* W1t, const float* b1,
+                 const void* W2t, const float* b2, const int32_t* idx, const int32_t* count, int k_max, float* out,
+                 int act, cudaStream_t st);
+dv_status tc_qkv(const Layout& L, void* ws, const float* y, int B, int d, int h, int dh, const void* Wqkv,
+                 const float* bqkv, void* Kc, void* Vc, int cap, int pos, const int32_t* head_idx,
+                 const int32_t* head_count, int kh_max, cudaStream_t st);
+dv_status tc_wo(const Layout& L, void* ws, int B, int d, int h, int dh, const void* WOt, const float* bO,
+                const int32_t* head_idx, const int32_t* head_count, int kh_max, float* out, cudaStream_t st);
 
 // ---------------------------------------------------------------------------
 // Operation bodies shared by the public entry points
@@ -122,8 +140,9 @@ dv_status do_predict_heads(const Layout& L, void* ws, const float* y, int B, int
 
 dv_status do_sparse_mlp(const Layout& L, void* ws, const float* y, int B, int d, int N, const void* W1t,
                         const float* b1, const void* W2t, const float* b2, dv_dtype dt, const int32_t* idx,
-                        const int32_t* count, int k_max, float* out, int accumulate, cudaStream_t st) {
+                        const int32_t* count, int k_max, float* out, int accumulate, int act, cudaStream_t st) {
   if (!accumulate) DV_TRY(cudaMemsetAsync(out, 0, 4ull * B * d, st));
+  if (tc_ok(B, dt, 64, k_max)) return tc_mlp(L, ws, y, B, d, N, W1t, b1, W2t, b2, idx, count, k_max, out, act, st);
   int* status = at<int>(ws, L.status);
   int32_t* seg_idx = at<int32_t>(ws, L.seg_idx);
   float* seg_a = at<float>(ws, L.seg_a);
@@ -135,7 +154,7 @@ dv_status do_sparse_mlp(const Layout& L, void* ws, const float* y, int B, int d,
     }
     return DV_OK;
   }
-  DV_TRY(run_mlp_up_dt(dt, W1t, d, N, y, B, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, L.nseg, st));
+  DV_TRY(run_mlp_up_dt(dt, W1t, d, N, y, B, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, L.nseg, act, st));
   RowsMlp src{seg_idx, seg_a, seg_cnt, L.nseg, L.SEG};
   const size_t smem = 4ull * (L.nseg + 1);
   return cuda_status(run_axpy_dt(dt, W2t, d, N, src, b2, out, B, k_max, smem, status, st));
@@ -147,6 +166,14 @@ dv_status do_sparse_mha(const Layout& L, void* ws, const float* y, int B, int d,
                         float* out, int accumulate, cudaStream_t st) {
   if (!accumulate) DV_TRY(cudaMemsetAsync(out, 0, 4ull * B * d, st));
   int* status = at<int>(ws, L.status);
+  if (tc_ok(B, dt, dh, 0)) {
+    if (kh_max > 0) {
+      DV_CHECK(tc_qkv(L, ws, y, B, d, h, dh, Wqkv, bqkv, Kc, Vc, cap, pos, head_idx, head_count, kh_max, st));
+      DV_TRY(run_attn_dt(dt, dh, at<float>(ws, L.q), Kc, Vc, B, h, cap, pos, scale, head_idx, head_count, kh_max,
+                         at<float>(ws, L.part), at<unsigned>(ws, L.attn_ctr), at<float>(ws, L.H), status, st));
+    }
+    return tc_wo(L, ws, B, d, h, dh, WOt, bO, head_idx, head_count, kh_max, out, st);
+  }
   if (kh_max == 0) {
     if (bO) {
       RowsHeads none{head_idx, head_count, nullptr, 0, dh, h};
@@ -166,11 +193,94 @@ dv_status do_sparse_mha(const Layout& L, void* ws, const float* y, int B, int d,
 int wbytes_of(dv_dtype t) { return t == DV_BF16 ? 2 : 4; }
 bool dtype_ok(int t) { return t == DV_F32 || t == DV_BF16; }
 bool mode_ok(int m) { return m == DV_TOPK || m == DV_THRESHOLD; }
+bool act_ok(int a) { return a == DV_ACT_RELU || a == DV_ACT_GELU; }
 
 dv_status check_ws(const Layout& L, void* ws, size_t ws_bytes) {
   if (!ok_ptr(ws)) return ws ? DV_ERR_ALIGN : DV_ERR_ARG;
   if (ws_bytes < L.total) return DV_ERR_WORKSPACE;
   return DV_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core path (dv_tc.cuh) for batch 5..16 with bf16 weights
+// ---------------------------------------------------------------------------
+
+bool tc_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("DV_TC");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+bool tc_ok(int B, dv_dtype wdt, int dh, int k_max) {
+  return tc_enabled() && B >= TC_MIN_B && tc_shape_ok(B, wbytes_of(wdt), dh > 0 ? dh : 64, k_max);
+}
+
+dv_status tc_mlp(const Layout& L, void* ws, const float* y, int B, int d, int N, const void* W1t, const float* b1,
+                 const void* W2t, const float* b2, const int32_t* idx, const int32_t* count, int k_max, float* out,
+                 int act, cudaStream_t st) {
+  TcMlpArgs a = {};
+  a.act = act;
+  a.W1t = static_cast<const bf16*>(W1t);
+  a.b1 = b1;
+  a.W2t = static_cast<const bf16*>(W2t);
+  a.b2 = b2;
+  a.y = y;
+  a.idx = idx;
+  a.count = count;
+  a.k_max = k_max;
+  a.d = d;
+  a.N = N;
+  a.nb = B;
+  a.KC = L.KC;
+  a.act_c = at<float>(ws, L.tc_act);
+  a.rowid_c = at<int32_t>(ws, L.tc_rowid);
+  a.tile_cnt = at<int32_t>(ws, L.tc_tiles);
+  a.out = out;
+  a.status = at<int>(ws, L.status);
+  return cuda_status(run_tc_mlp(a, st));
+}
+
+dv_status tc_qkv(const Layout& L, void* ws, const float* y, int B, int d, int h, int dh, const void* Wqkv,
+                 const float* bqkv, void* Kc, void* Vc, int cap, int pos, const int32_t* head_idx,
+                 const int32_t* head_count, int kh_max, cudaStream_t st) {
+  TcQkvArgs a = {};
+  a.Wqkv = static_cast<const bf16*>(Wqkv);
+  a.bqkv = bqkv;
+  a.y = y;
+  a.head_idx = head_idx;
+  a.head_count = head_count;
+  a.kh_max = kh_max;
+  a.h = h;
+  a.dh = dh;
+  a.d = d;
+  a.nb = B;
+  a.cap = cap;
+  a.pos = pos;
+  a.q = at<float>(ws, L.q);
+  a.Kc = static_cast<bf16*>(Kc);
+  a.Vc = static_cast<bf16*>(Vc);
+  a.status = at<int>(ws, L.status);
+  return cuda_status(run_tc_qkv(a, st));
+}
+
+dv_status tc_wo(const Layout& L, void* ws, int B, int d, int h, int dh, const void* WOt, const float* bO,
+                const int32_t* head_idx, const int32_t* head_count, int kh_max, float* out, cudaStream_t st) {
+  TcWoArgs a = {};
+  a.WOt = static_cast<const bf16*>(WOt);
+  a.bO = bO;
+  a.H = at<float>(ws, L.H);
+  a.head_idx = head_idx;
+  a.head_count = head_count;
+  a.kh_max = kh_max;
+  a.h = h;
+  a.dh = dh;
+  a.d = d;
+  a.nb = B;
+  a.out = out;
+  a.status = at<int>(ws, L.status);
+  return cuda_status(run_tc_wo(a, st));
 }
 
 // ---------------------------------------------------------------------------
@@ -190,6 +300,7 @@ bool fused_enabled() {
 // the normalised input and the K/V tiles within shared memory.
 bool fused_ok(const dv_dims& D, dv_dtype wdt) {
   if (!fused_enabled()) return false;
+  if (tc_ok(D.B, wdt, D.dh, D.k_max)) return false;  // batch 5..16, bf16: tensor-core kernels
   const int wb = wbytes_of(wdt), E = 16 / wb;
   if (D.d % (ATTN_CS * E) != 0) return false;
   if ((size_t)D.B * D.d * 4 > 160 * 1024) return false;
@@ -300,6 +411,9 @@ struct Ahead {
   float* z;
 };
 
+dv_status layer_begin_fused_qkv(const dv_layer_weights* w, const dv_dims& D, AttnInArgs a, const Ahead* ahead,
+                                float* yA_ws, cudaStream_t st);
+
 dv_status layer_begin(const Layout& L, void* ws, const dv_layer_weights* w, const dv_dims& D, const dv_layer_params* p,
                       float* x, int pos, const dv_layer_io* sel, const dv_layer_io* trace, cudaStream_t st,
                       const Ahead* ahead = nullptr) {
@@ -343,31 +457,12 @@ dv_status layer_begin(const Layout& L, void* ws, const dv_layer_weights* w, cons
     a.nb = D.B;
     a.sets_ready = sel ? 1 : 0;
     a.status = status;
-    if (ahead && attn_in_takes_rows(D.B, D.d, w->wdtype == DV_BF16 ? 8 : 4)) {
-      a.PA2 = ahead->w->PA;
-      a.At2 = ahead->w->At;
-      a.sh2 = ahead->sh;
-      a.z2 = ahead->z;
-      a.n2h = D.h;
-      a.n2r = D.r;
-      return cuda_status(run_attn_in_any_dt(w->wdtype, a, st));
-    }
-    if (ahead) {  // the row kernel: the predictor's first stage as its own launch, from yA
-      if (!a.yA_out) a.yA_out = r.yA;
-      DV_TRY(run_attn_in_any_dt(w->wdtype, a, st));
-      PredictAArgs pa = {};
-      pa.y = a.yA_out;
-      pa.PA = ahead->w->PA;
-      pa.At = ahead->w->At;
-      pa.h = D.h;
-      pa.r = D.r;
-      pa.d = D.d;
-      pa.nb = D.B;
-      pa.scores_h = ahead->sh;
-      pa.z = ahead->z;
-      return cuda_status(run_predict_a_any_dt(w->wdtype, pa, st));
-    }
-    return cuda_status(run_attn_in_any_dt(w->wdtype, a, st));
+    if (p->exact_kv && !a.yA_out) a.yA_out = r.yA;  // the other heads' k, v are formed from yA
+    DV_CHECK(layer_begin_fused_qkv(w, D, a, ahead, r.yA, st));
+    if (p->exact_kv)
+      DV_TRY(run_kv_rest_dt(w->wdtype, w->Wqkv, D.d, D.h, D.dh, a.yA_out, D.B, w->bqkv, r.use_hidx, r.use_hcnt,
+                            D.kh_max, w->Kc, w->Vc, D.cap, pos, status, st));
+    return DV_OK;
   }
   // kernel-per-step path
   float* yA = r.yA;
@@ -380,9 +475,51 @@ dv_status layer_begin(const Layout& L, void* ws, const dv_layer_weights* w, cons
   if (!sel)
     DV_CHECK(do_predict_heads(L, ws, yA, D.B, D.d, D.h, w->PA, w->wdtype, p->k_h, p->tau_h, p->mode_h, r.sh, r.hidx,
                               r.hcnt, st));
-  if (D.kh_max == 0) return DV_OK;
-  float* q = at<float>(ws, L.q);
-  return cuda_status(run_qkv_dt(w->wdtype, w->Wqkv, D.d, D.h, D.dh, yA, D.B, w->bqkv, r.use_hidx, r.use_hcnt, D.kh_max, q, w->Kc, w->Vc, D.cap, pos, status, st));
+  if (D.kh_max > 0) {
+    if (tc_ok(D.B, w->wdtype, D.dh, D.k_max)) {
+      DV_CHECK(tc_qkv(L, ws, yA, D.B, D.d, D.h, D.dh, w->Wqkv, w->bqkv, w->Kc, w->Vc, D.cap, pos, r.use_hidx,
+                      r.use_hcnt, D.kh_max, st));
+    } else {
+      DV_TRY(run_qkv_dt(w->wdtype, w->Wqkv, D.d, D.h, D.dh, yA, D.B, w->bqkv, r.use_hidx, r.use_hcnt, D.kh_max,
+                        at<float>(ws, L.q), w->Kc, w->Vc, D.cap, pos, status, st));
+    }
+  }
+  if (p->exact_kv)
+    DV_TRY(run_kv_rest_dt(w->wdtype, w->Wqkv, D.d, D.h, D.dh, yA, D.B, w->bqkv, r.use_hidx, r.use_hcnt, D.kh_max, w->Kc,
+                          w->Vc, D.cap, pos, status, st));
+  return DV_OK;
+}
+
+// The fused Q/K/V launch of layer_begin (a filled in), with the next
+// layer's predictor first stage when `ahead` is given; yA_ws receives LN1(x)
+// when the first stage needs its own launch.
+dv_status layer_begin_fused_qkv(const dv_layer_weights* w, const dv_dims& D, AttnInArgs a, const Ahead* ahead,
+                                float* yA_ws, cudaStream_t st) {
+  if (ahead && attn_in_takes_rows(D.B, D.d, w->wdtype == DV_BF16 ? 8 : 4)) {
+    a.PA2 = ahead->w->PA;
+    a.At2 = ahead->w->At;
+    a.sh2 = ahead->sh;
+    a.z2 = ahead->z;
+    a.n2h = D.h;
+    a.n2r = D.r;
+    return cuda_status(run_attn_in_any_dt(w->wdtype, a, st));
+  }
+  if (ahead) {  // the row kernel: the predictor's first stage as its own launch, from yA
+    if (!a.yA_out) a.yA_out = yA_ws;
+    DV_TRY(run_attn_in_any_dt(w->wdtype, a, st));
+    PredictAArgs pa = {};
+    pa.y = a.yA_out;
+    pa.PA = ahead->w->PA;
+    pa.At = ahead->w->At;
+    pa.h = D.h;
+    pa.r = D.r;
+    pa.d = D.d;
+    pa.nb = D.B;
+    pa.scores_h = ahead->sh;
+    pa.z = ahead->z;
+    return cuda_status(run_predict_a_any_dt(w->wdtype, pa, st));
+  }
+  return cuda_status(run_attn_in_any_dt(w->wdtype, a, st));
 }
 
 // Attention half: split attention over the selected heads, W^O, residual.
@@ -413,6 +550,13 @@ dv_status layer_attn(const Layout& L, void* ws, const dv_layer_weights* w, const
     b.scale = p->scale;
     b.status = status;
     return cuda_status(run_attn_out_dt(w->kvdtype, b, st));
+  }
+  if (tc_ok(D.B, w->wdtype, D.dh, D.k_max)) {
+    if (D.kh_max > 0)
+      DV_TRY(run_attn_dt(w->kvdtype, D.dh, at<float>(ws, L.q), w->Kc, w->Vc, D.B, D.h, D.cap, pos, p->scale,
+                         r.use_hidx, r.use_hcnt, D.kh_max, at<float>(ws, L.part), at<unsigned>(ws, L.attn_ctr),
+                         at<float>(ws, L.H), status, st));
+    return tc_wo(L, ws, D.B, D.d, D.h, D.dh, w->WOt, w->bO, r.use_hidx, r.use_hcnt, D.kh_max, x, st);
   }
   if (D.kh_max > 0) {
     float* H = at<float>(ws, L.H);
@@ -460,6 +604,7 @@ dv_status layer_mlp(const Layout& L, void* ws, const dv_layer_weights* w, const 
     c.sets_ready = sel ? 1 : 0;
     c.yM_out = sel ? (trace ? trace->yM : nullptr) : nullptr;
     c.status = status;
+    c.act = p->act;
     return cuda_status(run_mlp_block_any_dt(w->wdtype, c, st));
   }
   DV_TRY(launch(layernorm_kernel, dim3(D.B), LN_THREADS, 0, st, (const float*)x, r.yM, D.d, w->ln2_g, w->ln2_b,
@@ -468,7 +613,7 @@ dv_status layer_mlp(const Layout& L, void* ws, const dv_layer_weights* w, const 
     DV_CHECK(do_predict_mlp(L, ws, r.yM, D.B, D.d, D.r, D.N, w->At, w->Bm, w->b1, w->wdtype, p->k, p->tau, p->mode,
                             r.sm, r.midx, r.mcnt, st));
   return do_sparse_mlp(L, ws, r.yM, D.B, D.d, D.N, w->W1t, w->b1, w->W2t, w->b2, w->wdtype, r.use_midx, r.use_mcnt,
-                       D.k_max, x, 1, st);
+                       D.k_max, x, 1, p->act, st);
 }
 
 dv_status layer_end(const Layout& L, void* ws, const dv_layer_weights* w, const dv_dims& D, const dv_layer_params* p,
@@ -565,18 +710,25 @@ dv_status dv_topk(const float* scores, int B, int n, int k, float tau, int mode,
                                 idx, count, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-dv_status dv_sparse_mlp(const float* y, int B, int d, int N, const void* W1t, const float* b1, const void* W2t,
-                        const float* b2, dv_dtype wdtype, const int32_t* idx, const int32_t* count, int k_max,
-                        float* out, int accumulate, void* ws, size_t ws_bytes, dv_stream_t stream) {
-  if (!dtype_ok(wdtype)) return DV_ERR_ARG;
+dv_status dv_sparse_mlp_act(const float* y, int B, int d, int N, const void* W1t, const float* b1, const void* W2t,
+                            const float* b2, dv_dtype wdtype, const int32_t* idx, const int32_t* count, int k_max,
+                            float* out, int accumulate, int act, void* ws, size_t ws_bytes, dv_stream_t stream) {
+  if (!dtype_ok(wdtype) || !act_ok(act)) return DV_ERR_ARG;
   if (!y || !W1t || !b1 || !W2t || !idx || !count || !out) return DV_ERR_ARG;
   if (!ok_ptr(y) || !ok_ptr(W1t) || !ok_ptr(W2t) || !ok_ptr(out) || !ok_opt(b2)) return DV_ERR_ALIGN;
   dv_dims D = {B, d, N, 0, 0, 0, 0, k_max, 0};
   if (!dims_ok(D)) return DV_ERR_ARG;
   const Layout L = layout(D, wbytes_of(wdtype));
   DV_CHECK(check_ws(L, ws, ws_bytes));
-  return do_sparse_mlp(L, ws, y, B, d, N, W1t, b1, W2t, b2, wdtype, idx, count, k_max, out, accumulate,
+  return do_sparse_mlp(L, ws, y, B, d, N, W1t, b1, W2t, b2, wdtype, idx, count, k_max, out, accumulate, act,
                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+dv_status dv_sparse_mlp(const float* y, int B, int d, int N, const void* W1t, const float* b1, const void* W2t,
+                        const float* b2, dv_dtype wdtype, const int32_t* idx, const int32_t* count, int k_max,
+                        float* out, int accumulate, void* ws, size_t ws_bytes, dv_stream_t stream) {
+  return dv_sparse_mlp_act(y, B, d, N, W1t, b1, W2t, b2, wdtype, idx, count, k_max, out, accumulate, DV_ACT_RELU, ws,
+                           ws_bytes, stream);
 }
 
 dv_status dv_sparse_mha(const float* y, int B, int d, int h, int dh, const void* Wqkv, const float* bqkv,
@@ -601,7 +753,8 @@ dv_status dv_sparse_mha(const float* y, int B, int d, int h, int dh, const void*
 static dv_status check_layer(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p) {
   if (!w || !dims || !p) return DV_ERR_ARG;
   const dv_dims& D = *dims;
-  if (!dtype_ok(w->wdtype) || !dtype_ok(w->kvdtype) || !mode_ok(p->mode) || !mode_ok(p->mode_h)) return DV_ERR_ARG;
+  if (!dtype_ok(w->wdtype) || !dtype_ok(w->kvdtype) || !mode_ok(p->mode) || !mode_ok(p->mode_h) || !act_ok(p->act))
+    return DV_ERR_ARG;
   if (w->kvdtype != w->wdtype) return DV_ERR_UNSUPPORTED;
   if (!dims_ok(D) || D.h < 1 || D.r < 8 || D.cap < 1) return DV_ERR_ARG;
   if (D.dh != 64 && D.dh != 128) return DV_ERR_UNSUPPORTED;

@@ -391,7 +391,7 @@ __global__ void __launch_bounds__(CO_THREADS) mlp_block_co_kernel(MlpBlockArgs a
       float v = 0.f;
 #pragma unroll
       for (int rr = 0; rr < R; ++rr)
-        if (rr == r) v = (valid[rr] && b < a.nb) ? fmaxf(s_out[r * NB + b] + bias[rr], 0.f) : 0.f;
+        if (rr == r) v = (valid[rr] && b < a.nb) ? activate(s_out[r * NB + b] + bias[rr], a.act) : 0.f;
       s_act[r][b] = v;
     }
     __syncthreads();
@@ -399,7 +399,7 @@ __global__ void __launch_bounds__(CO_THREADS) mlp_block_co_kernel(MlpBlockArgs a
     for (int r = 0; r < R; ++r) {
       bool nz = false;
 #pragma unroll
-      for (int b = 0; b < NB; ++b) nz |= s_act[r][b] > 0.f;
+      for (int b = 0; b < NB; ++b) nz |= s_act[r][b] != 0.f;
       if (nz) {  // the same for every thread: zero activations add nothing
 #pragma unroll
         for (int j = 0; j < NV; ++j) {

@@ -137,6 +137,13 @@ __device__ __forceinline__ unsigned block_exclusive_scan(unsigned v, unsigned* s
 
 __device__ __forceinline__ void raise_status(int* st, int bit) { atomicOr(st, bit); }
 
+// The MLP's activation sigma of eq. (1): ReLU, or GeLU in its exact form
+// v Phi(v) = v (1 + erf(v / sqrt(2))) / 2 (erff is CUDA's error function).
+enum : int { ACT_RELU = 0, ACT_GELU = 1 };
+__device__ __forceinline__ float activate(float v, int act) {
+  return act == ACT_GELU ? 0.5f * v * (1.f + erff(v * 0.70710678118654752f)) : fmaxf(v, 0.f);
+}
+
 // out[0..3] += v without returning the old values (a fire-and-forget vector
 // reduction in L2, so the issuing thread does not wait for it).
 __device__ __forceinline__ void red_add4(float* out, float4 v) {

@@ -198,6 +198,7 @@ struct MlpBlockArgs {
   int k_max, d, N, nb, G, sets_ready;
   float* yM_out;  // optional copy of LN2(t1), written by CTA 0
   int* status;
+  int act;        // ACT_RELU or ACT_GELU
 };
 
 constexpr int MLP_MAX_ROWS = 64;  // selection slots per CTA held in shared memory at once
@@ -286,9 +287,9 @@ __global__ void __launch_bounds__(FUSED_THREADS) mlp_block_kernel(MlpBlockArgs a
             int nz = 0;
 #pragma unroll
             for (int b = 0; b < NB; ++b) {
-              const float v = (valid[r] && b < a.nb) ? fmaxf(acc[r][b] + bias[r], 0.f) : 0.f;
+              const float v = (valid[r] && b < a.nb) ? activate(acc[r][b] + bias[r], a.act) : 0.f;
               s_act[s][b] = v;
-              nz |= v > 0.f;
+              nz |= v != 0.f;
             }
             s_nz[s] = nz;
             s_row[s] = rows[r];

@@ -24,10 +24,11 @@ cudaError_t run_select(const float* scores, int nrows, int n, int k, float tau, 
 
 cudaError_t run_mlp_up_dt(dv_dtype dt, const void* W1t, int d, int N, const float* y, int nb, const float* b1,
                           const int32_t* idx, const int32_t* count, int k_max, int32_t* seg_idx, float* seg_a,
-                          int32_t* seg_cnt, int* status, int nseg, cudaStream_t st) {
+                          int32_t* seg_cnt, int* status, int nseg, int act, cudaStream_t st) {
   return dt == DV_BF16
-             ? run_mlp_up<bf16>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, st)
-             : run_mlp_up<float>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, st);
+             ? run_mlp_up<bf16>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, act, st)
+             : run_mlp_up<float>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, act,
+                                 st);
 }
 
 cudaError_t run_axpy_dt(dv_dtype dt, const void* W, int d, int nrows_w, RowsHeads src, const float* bias, float* out,

@@ -12,6 +12,15 @@ cudaError_t run_qkv_dt(dv_dtype dt, const void* Wqkv, int d, int h, int dh, cons
                                         status, st);
 }
 
+cudaError_t run_kv_rest_dt(dv_dtype dt, const void* Wqkv, int d, int h, int dh, const float* y, int nb,
+                           const float* bqkv, const int32_t* head_idx, const int32_t* head_count, int kh_max, void* Kc,
+                           void* Vc, int cap, int pos, int* status, cudaStream_t st) {
+  return dt == DV_BF16 ? run_kv_rest<bf16>(Wqkv, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, Kc, Vc, cap, pos,
+                                           status, st)
+                       : run_kv_rest<float>(Wqkv, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, Kc, Vc, cap,
+                                            pos, status, st);
+}
+
 cudaError_t run_attn_dt(dv_dtype kvdt, int dh, const float* q, const void* Kc, const void* Vc, int B, int h, int cap,
                         int pos, float scale, const int32_t* head_idx, const int32_t* head_count, int kh_max,
                         float* part, unsigned* ctr, float* H, int* status, cudaStream_t st) {

@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(GEMV_THREADS)
     mlp_up_kernel(const T* __restrict__ W1t, int d, int N, const float* __restrict__ X, int nb,
                   const float* __restrict__ b1, const int32_t* __restrict__ idx, const int32_t* __restrict__ count_dev,
                   int k_max, int32_t* __restrict__ seg_idx, float* __restrict__ seg_a, int32_t* __restrict__ seg_cnt,
-                  int* __restrict__ status) {
+                  int* __restrict__ status, int act) {
   constexpr int SEG = GEMV_WARPS * RPW;
   __shared__ float s_a[SEG][NB];
   __shared__ int s_row[SEG];
@@ -154,9 +154,9 @@ __global__ void __launch_bounds__(GEMV_THREADS)
       const float bias = valid[r] ? b1[rows[r]] : 0.f;
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
-        const float a = (valid[r] && b < nb) ? fmaxf(acc[r][b] + bias, 0.f) : 0.f;
+        const float a = (valid[r] && b < nb) ? activate(acc[r][b] + bias, act) : 0.f;
         s_a[warp * RPW + r][b] = a;
-        nz |= a > 0.f;
+        nz |= a != 0.f;
       }
       s_nz[warp * RPW + r] = nz;
       s_row[warp * RPW + r] = rows[r];
@@ -239,6 +239,83 @@ __global__ void __launch_bounds__(GEMV_THREADS)
           T* cache = (m == 1) ? Kc : Vc;
           cache[(((size_t)b * h + heads[r]) * cap + pos) * dh + c] = WT<T>::store_cvt(v);
         }
+      }
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Exact KV maintenance: k and v at slot `pos` for the heads NOT in the
+// selected set (the KV-cache figure (b): every step appends the new token's
+// key and value for every head), so later steps attend over true keys and
+// values. Every CTA rebuilds the ascending list of unselected heads from
+// head_idx in shared memory. Slot s in [0, (h - hc) * 2 dh): p = s / (2 dh)
+// indexes that list, m = 1 + (s / dh) % 2 picks k / v, c = s % dh.
+// ----------------------------------------------------------------------------
+constexpr int KV_REST_MAX_H = 1024;
+
+template <typename T, int NB, int RPW, int U>
+__global__ void __launch_bounds__(GEMV_THREADS)
+    kv_rest_kernel(const T* __restrict__ Wqkv, int d, int h, int dh, const float* __restrict__ X, int nb,
+                   const float* __restrict__ bqkv, const int32_t* __restrict__ head_idx,
+                   const int32_t* __restrict__ head_count, int kh_max, T* __restrict__ Kc, T* __restrict__ Vc, int cap,
+                   int pos, int* __restrict__ status) {
+  __shared__ int s_rest[KV_REST_MAX_H];
+  __shared__ unsigned char s_sel[KV_REST_MAX_H];
+  __shared__ int s_nrest;
+  griddep_launch();
+  griddep_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int hc = *head_count;
+  if (hc > kh_max || hc < 0) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(status, 1);
+    hc = hc < 0 ? 0 : kh_max;
+  }
+  for (int i = threadIdx.x; i < h; i += GEMV_THREADS) s_sel[i] = 0;
+  __syncthreads();
+  for (int p = threadIdx.x; p < hc; p += GEMV_THREADS) {
+    const int head = head_idx[p];
+    if (head >= 0 && head < h) s_sel[head] = 1;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int base = 0;
+    for (int i0 = 0; i0 < h; i0 += 32) {
+      const int i = i0 + lane;
+      const bool rest = i < h && !s_sel[i];
+      const unsigned bal = __ballot_sync(0xffffffffu, rest);
+      if (rest) s_rest[base + __popc(bal & ((1u << lane) - 1u))] = i;
+      base += __popc(bal);
+    }
+    if (lane == 0) s_nrest = base;
+  }
+  __syncthreads();
+  const int per = 2 * dh;
+  const int nslot = s_nrest * per;
+  const int slot0 = (blockIdx.x * GEMV_WARPS + warp) * RPW;
+  if (slot0 >= nslot) return;
+  const T* rowp[RPW];
+  bool valid[RPW];
+  int heads[RPW];
+#pragma unroll
+  for (int r = 0; r < RPW; ++r) {
+    const int slot = slot0 + r;
+    valid[r] = slot < nslot;
+    heads[r] = valid[r] ? s_rest[slot / per] : 0;
+    rowp[r] = Wqkv + ((size_t)heads[r] * 3 * dh + dh + (valid[r] ? slot % per : 0)) * d;
+  }
+  float acc[RPW][NB];
+  warp_rows_dot<T, NB, RPW, U>(rowp, valid, d, X, d, nb, acc);
+#pragma unroll
+  for (int r = 0; r < RPW; ++r) {
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (lane == ((r * NB + b) & 31) && valid[r] && b < nb) {
+        const int rem = (slot0 + r) % per, c = rem % dh;
+        float v = acc[r][b];
+        if (bqkv) v += bqkv[(size_t)heads[r] * 3 * dh + dh + rem];
+        T* cache = rem < dh ? Kc : Vc;
+        cache[(((size_t)b * h + heads[r]) * cap + pos) * dh + c] = WT<T>::store_cvt(v);
       }
     }
   }

@@ -51,14 +51,14 @@ cudaError_t run_select(const float* scores, int nrows, int n, int k, float tau, 
 template <typename T, int NB>
 cudaError_t run_mlp_up_nb(const void* W1t, int d, int N, const float* y, int nb, const float* b1, const int32_t* idx,
                           const int32_t* count, int k_max, int32_t* seg_idx, float* seg_a, int32_t* seg_cnt,
-                          int* status, int nseg, cudaStream_t st) {
+                          int* status, int nseg, int act, cudaStream_t st) {
   const T* w = static_cast<const T*>(W1t);
   dim3 grid(nseg > 0 ? nseg : 1);
   switch (rpw_for(d, WT<T>::E)) {
-    case 1: return launch(mlp_up_kernel<T, NB, 1, 8>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status);
-    case 2: return launch(mlp_up_kernel<T, NB, 2, 4>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status);
-    case 4: return launch(mlp_up_kernel<T, NB, 4, 2>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status);
-    default: return launch(mlp_up_kernel<T, NB, 8, 1>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status);
+    case 1: return launch(mlp_up_kernel<T, NB, 1, 8>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, act);
+    case 2: return launch(mlp_up_kernel<T, NB, 2, 4>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, act);
+    case 4: return launch(mlp_up_kernel<T, NB, 4, 2>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, act);
+    default: return launch(mlp_up_kernel<T, NB, 8, 1>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, act);
   }
 }
 
@@ -92,13 +92,13 @@ cudaError_t run_axpy(const void* W, int d, int nrows_w, Src src, const float* bi
 template <typename T>
 cudaError_t run_mlp_up(const void* W1t, int d, int N, const float* y, int nb, const float* b1, const int32_t* idx,
                        const int32_t* count, int k_max, int32_t* seg_idx, float* seg_a, int32_t* seg_cnt, int* status,
-                       int nseg, cudaStream_t st) {
+                       int nseg, int act, cudaStream_t st) {
   switch (nb_bucket(nb)) {
-    case 1: return run_mlp_up_nb<T, 1>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, st);
-    case 2: return run_mlp_up_nb<T, 2>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, st);
-    case 4: return run_mlp_up_nb<T, 4>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, st);
-    case 8: return run_mlp_up_nb<T, 8>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, st);
-    default: return run_mlp_up_nb<T, 16>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, st);
+    case 1: return run_mlp_up_nb<T, 1>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, act, st);
+    case 2: return run_mlp_up_nb<T, 2>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, act, st);
+    case 4: return run_mlp_up_nb<T, 4>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, act, st);
+    case 8: return run_mlp_up_nb<T, 8>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, act, st);
+    default: return run_mlp_up_nb<T, 16>(W1t, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, nseg, act, st);
   }
 }
 
@@ -131,6 +131,38 @@ cudaError_t run_qkv(const void* Wqkv, int d, int h, int dh, const float* y, int 
     case 4: return run_qkv_nb<T, 4>(Wqkv, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, Kc, Vc, cap, pos, status, st);
     case 8: return run_qkv_nb<T, 8>(Wqkv, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, Kc, Vc, cap, pos, status, st);
     default: return run_qkv_nb<T, 16>(Wqkv, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, Kc, Vc, cap, pos, status, st);
+  }
+}
+
+template <typename T, int NB>
+cudaError_t run_kv_rest_nb(const void* Wqkv, int d, int h, int dh, const float* y, int nb, const float* bqkv,
+                           const int32_t* head_idx, const int32_t* head_count, int kh_max, void* Kc, void* Vc, int cap,
+                           int pos, int* status, cudaStream_t st) {
+  const T* w = static_cast<const T*>(Wqkv);
+  const int rpw = rpw_for(d, WT<T>::E);
+  const int per_cta = GEMV_WARPS * rpw;
+  const int slots = h * 2 * dh;  // every head unselected, at most
+  dim3 grid((slots + per_cta - 1) / per_cta > 0 ? (slots + per_cta - 1) / per_cta : 1);
+  T* K = static_cast<T*>(Kc);
+  T* V = static_cast<T*>(Vc);
+  switch (rpw) {
+    case 1: return launch(kv_rest_kernel<T, NB, 1, 8>, grid, GEMV_THREADS, 0, st, w, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, K, V, cap, pos, status);
+    case 2: return launch(kv_rest_kernel<T, NB, 2, 4>, grid, GEMV_THREADS, 0, st, w, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, K, V, cap, pos, status);
+    case 4: return launch(kv_rest_kernel<T, NB, 4, 2>, grid, GEMV_THREADS, 0, st, w, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, K, V, cap, pos, status);
+    default: return launch(kv_rest_kernel<T, NB, 8, 1>, grid, GEMV_THREADS, 0, st, w, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, K, V, cap, pos, status);
+  }
+}
+
+template <typename T>
+cudaError_t run_kv_rest(const void* Wqkv, int d, int h, int dh, const float* y, int nb, const float* bqkv,
+                        const int32_t* head_idx, const int32_t* head_count, int kh_max, void* Kc, void* Vc, int cap,
+                        int pos, int* status, cudaStream_t st) {
+  switch (nb_bucket(nb)) {
+    case 1: return run_kv_rest_nb<T, 1>(Wqkv, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, Kc, Vc, cap, pos, status, st);
+    case 2: return run_kv_rest_nb<T, 2>(Wqkv, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, Kc, Vc, cap, pos, status, st);
+    case 4: return run_kv_rest_nb<T, 4>(Wqkv, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, Kc, Vc, cap, pos, status, st);
+    case 8: return run_kv_rest_nb<T, 8>(Wqkv, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, Kc, Vc, cap, pos, status, st);
+    default: return run_kv_rest_nb<T, 16>(Wqkv, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, Kc, Vc, cap, pos, status, st);
   }
 }
 
@@ -539,7 +571,7 @@ cudaError_t run_predict_a_any(const PredictAArgs& a, cudaStream_t st) {
 
 cudaError_t run_mlp_up_dt(dv_dtype dt, const void* W1t, int d, int N, const float* y, int nb, const float* b1,
                           const int32_t* idx, const int32_t* count, int k_max, int32_t* seg_idx, float* seg_a,
-                          int32_t* seg_cnt, int* status, int nseg, cudaStream_t st);
+                          int32_t* seg_cnt, int* status, int nseg, int act, cudaStream_t st);
 cudaError_t run_axpy_dt(dv_dtype dt, const void* W, int d, int nrows_w, RowsHeads src, const float* bias, float* out,
                         int nb, int k_max, size_t smem, int* status, cudaStream_t st);
 cudaError_t run_axpy_dt(dv_dtype dt, const void* W, int d, int nrows_w, RowsMlp src, const float* bias, float* out,
@@ -547,6 +579,9 @@ cudaError_t run_axpy_dt(dv_dtype dt, const void* W, int d, int nrows_w, RowsMlp 
 cudaError_t run_qkv_dt(dv_dtype dt, const void* Wqkv, int d, int h, int dh, const float* y, int nb, const float* bqkv,
                        const int32_t* head_idx, const int32_t* head_count, int kh_max, float* q, void* Kc, void* Vc,
                        int cap, int pos, int* status, cudaStream_t st);
+cudaError_t run_kv_rest_dt(dv_dtype dt, const void* Wqkv, int d, int h, int dh, const float* y, int nb,
+                           const float* bqkv, const int32_t* head_idx, const int32_t* head_count, int kh_max, void* Kc,
+                           void* Vc, int cap, int pos, int* status, cudaStream_t st);
 cudaError_t run_attn_dt(dv_dtype kvdt, int dh, const float* q, const void* Kc, const void* Vc, int B, int h, int cap,
                         int pos, float scale, const int32_t* head_idx, const int32_t* head_count, int kh_max,
                         float* part, unsigned* ctr, float* H, int* status, cudaStream_t st);

@@ -347,10 +347,10 @@ __global__ void __launch_bounds__(CO_THREADS, 1) mlp_stream_kernel(MlpBlockArgs 
           if (i < cn && b < a.nb && s_row[i] >= 0) {
 #pragma unroll
             for (int q = 0; q < CO_WARPS; ++q) s += red[(i * NB + b) * CO_WARPS + q];
-            s = fmaxf(s + s_bias[i], 0.f);
+            s = activate(s + s_bias[i], a.act);
           }
           act[b] = s;
-          nz |= s > 0.f;
+          nz |= s != 0.f;
         }
         const unsigned bal = __ballot_sync(0xffffffffu, nz);
         if (nz) {

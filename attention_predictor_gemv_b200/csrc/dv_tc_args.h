@@ -1,0 +1,60 @@
+// Argument blocks and sizes of the tensor-core gathered-row kernels
+// (dv_tc.cuh), shared by the kernels and the host code that launches them.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace dv {
+
+constexpr int TC_M = 128;         // tile rows (rowdot) / columns (rowaxpy)
+constexpr int TC_N = 16;          // batch rows, zero-padded
+constexpr int TC_MIN_B = 5;       // batch rows from which the layer calls use the tensor-core kernels
+constexpr int TC_MAX_TILES = 1024;  // tiles of 128 selected neurons (k_max <= 131072)
+constexpr int DV_DEV_TIMEOUT_BIT = 8;  // device status bit: a bounded wait ran out
+
+struct TcQkvArgs {
+  const __nv_bfloat16* Wqkv;  // [h][3][dh][d]
+  const float* bqkv;          // [h][3][dh] or null
+  const float* y;             // [nb][d] normalised input
+  const int32_t* head_idx;
+  const int32_t* head_count;
+  int kh_max, h, dh, d, nb, cap, pos;
+  float* q;                   // [nb][kh_max][dh]
+  __nv_bfloat16* Kc;          // [nb][h][cap][dh]
+  __nv_bfloat16* Vc;
+  int* status;
+};
+
+struct TcMlpArgs {
+  const __nv_bfloat16* W1t;  // [N][d]
+  const float* b1;           // [N]
+  const __nv_bfloat16* W2t;  // [N][d]
+  const float* b2;           // [d] or null
+  const float* y;            // [nb][d]
+  const int32_t* idx;
+  const int32_t* count;
+  int k_max, d, N, nb;
+  int KC;                    // slots per batch row of act_c: tiles_max x 128
+  int tiles_per_group;       // rowdot tiles per rowaxpy unit
+  float* act_c;              // [16][KC] activations, compacted per tile
+  int32_t* rowid_c;          // [KC] the neuron of each compacted slot
+  int32_t* tile_cnt;         // [tiles_max] nonzero neurons per tile
+  float* out;                // [nb][d], accumulated into
+  int* status;
+  int act;                   // ACT_RELU or ACT_GELU
+};
+
+struct TcWoArgs {
+  const __nv_bfloat16* WOt;  // [h][dh][d]
+  const float* bO;           // [d] or null
+  const float* H;            // [nb][kh_max][dh]
+  const int32_t* head_idx;
+  const int32_t* head_count;
+  int kh_max, h, dh, d, nb;
+  int heads_per_group;
+  float* out;                // [nb][d], accumulated into
+  int* status;
+};
+
+}  // namespace dv

@@ -1,0 +1,21 @@
+// Host-side declarations of the tensor-core kernel launchers (dv_inst_tc.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "dv_tc_args.h"
+
+namespace dv {
+
+// Shapes the tensor-core path takes: bf16 weights, at most 16 batch rows,
+// dh a multiple of 64, at most 1024 tiles of 128 selected neurons.
+bool tc_shape_ok(int B, int wbytes, int dh, int k_max);
+// Tiles of 128 selected neurons for a bound of k_max.
+int tc_tiles(int k_max);
+
+cudaError_t run_tc_qkv(const TcQkvArgs& a, cudaStream_t st);
+// W1 + bias + ReLU with per-tile compaction, then the W2 gather-axpy into out.
+cudaError_t run_tc_mlp(TcMlpArgs a, cudaStream_t st);
+cudaError_t run_tc_wo(TcWoArgs a, cudaStream_t st);
+
+}  // namespace dv

@@ -29,7 +29,7 @@ class DecoderStack:
                  lookahead: bool = True, eps: float = 1e-5, mode: int = bd.DV_TOPK, tau: float = 0.0,
                  mode_h: int = bd.DV_TOPK, tau_h: float = 0.0, k_max: Optional[int] = None,
                  kh_max: Optional[int] = None, prefetch: bool = False, prefetch_w2: bool = True,
-                 fuse_ahead: bool = True):
+                 fuse_ahead: bool = True, act: int = bd.DV_ACT_RELU, exact_kv: bool = False):
         t0 = layers[0]
         N, d = t0["W1t"].shape
         h = t0["Wqkv"].shape[0]
@@ -38,7 +38,7 @@ class DecoderStack:
         self.k_max = k_max if k_max is not None else (N if mode == bd.DV_THRESHOLD else min(N, B * k))
         self.kh_max = kh_max if kh_max is not None else (h if mode_h == bd.DV_THRESHOLD else min(h, B * k_h))
         self.layers = [bd.Layer(t, B, self.k_max, self.kh_max) for t in layers]
-        self.p = bd.params(k, k_h, scale, eps, tau, mode, tau_h, mode_h)
+        self.p = bd.params(k, k_h, scale, eps, tau, mode, tau_h, mode_h, act=act, exact_kv=exact_kv)
         self.lookahead = lookahead
         self.prefetch = prefetch and lookahead
         self.prefetch_w2 = prefetch_w2

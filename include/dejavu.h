@@ -71,11 +71,19 @@ typedef enum { DV_F32 = 0, DV_BF16 = 1 } dv_dtype;
  * +0.0, NaN below -inf), or every score strictly greater than tau. */
 typedef enum { DV_TOPK = 0, DV_THRESHOLD = 1 } dv_select_mode;
 
+/* The MLP's activation sigma in eq. (1) ("ReLU or GeLU", §2.3). With ReLU,
+ * neurons whose activation is zero in every batch row are dropped before
+ * their W2 rows are read; GeLU has no exact zeros, so every selected neuron's
+ * W2 row is read. GeLU is the exact form v Phi(v) = v (1 + erf(v/sqrt 2)) / 2. */
+typedef enum { DV_ACT_RELU = 0, DV_ACT_GELU = 1 } dv_activation;
+
 /* Device status word bits (dv_read_device_status). */
 enum {
   DV_DEV_COUNT_CLAMPED = 1, /* a device count exceeded its bound */
   DV_DEV_INDEX_RANGE = 2,   /* a selected index was outside [0, n); skipped */
-  DV_DEV_BAD_PARTIAL = 4    /* attention combine found no partial for a head */
+  DV_DEV_BAD_PARTIAL = 4,   /* attention combine found no partial for a head */
+  DV_DEV_TIMEOUT = 8        /* a bounded wait inside a kernel ran out (about 2 s); the kernel
+                               stopped early and its outputs are incomplete */
 };
 
 /* Opaque stream handle; pass a cudaStream_t. */
@@ -140,7 +148,8 @@ DV_API dv_status dv_predict_heads(const float* y, int B, int d, int h, const voi
 DV_API dv_status dv_topk(const float* scores, int B, int n, int k, float tau, int mode, int32_t* idx,
                   int32_t* count, void* ws, size_t ws_bytes, dv_stream_t stream);
 
-/* Sparsified MLP, eq. (1), with ReLU:
+/* Sparsified MLP, eq. (1), with ReLU (dv_sparse_mlp_act: with the activation
+ * `act`, a dv_activation; dv_sparse_mlp is dv_sparse_mlp_act with DV_ACT_RELU):
  *   out[b] (+)= sum_{j < count} relu(y[b] . W1t[idx[j]] + b1[idx[j]]) W2t[idx[j]] (+ b2)
  * y [B][d] fp32; W1t, W2t [N][d] in `wdtype` (neuron-major: row i is column
  * W1_i / W2_i); b1 [N] fp32; b2 [d] fp32 or NULL; idx / count: the selected
@@ -151,6 +160,10 @@ DV_API dv_status dv_sparse_mlp(const float* y, int B, int d, int N, const void* 
                         const void* W2t, const float* b2, dv_dtype wdtype, const int32_t* idx,
                         const int32_t* count, int k_max, float* out, int accumulate, void* ws,
                         size_t ws_bytes, dv_stream_t stream);
+DV_API dv_status dv_sparse_mlp_act(const float* y, int B, int d, int N, const void* W1t, const float* b1,
+                                   const void* W2t, const float* b2, dv_dtype wdtype, const int32_t* idx,
+                                   const int32_t* count, int k_max, float* out, int accumulate, int act, void* ws,
+                                   size_t ws_bytes, dv_stream_t stream);
 
 /* Sparsified MHA, eq. (2), over a KV cache, for the heads in head_idx:
  *   for i in S_A: q, k, v = y Wqkv[i][0..2]^T (+ bqkv[i]);
@@ -208,6 +221,11 @@ typedef struct {
   int mode_h;  /* dv_select_mode for heads */
   float scale; /* softmax scale on q.k */
   float eps;   /* LayerNorm epsilon */
+  int act;     /* dv_activation of the MLP (0 = ReLU) */
+  int exact_kv; /* nonzero: also compute k and v of the UNSELECTED heads and store them at
+                   slot pos (every head's cache then holds this token, as a dense model's
+                   would; 2 h_unselected dh d more weight bytes); 0: only the selected
+                   heads' slots are written, the others keep what they held */
 } dv_layer_params;
 
 /* Device buffers for the selected sets and the intermediates of a layer. In

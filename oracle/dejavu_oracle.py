@@ -293,6 +293,34 @@ def sparse_mha(y, Wqkv, bqkv, WOt, bO, Kc, Vc, pos: int, scale: float, head_idx,
     return MHAResult(out=out, H=H, q=Q, k_new=KN, v_new=VN)
 
 
+def unselected_kv(y, Wqkv, bqkv, Kc, Vc, pos: int, head_idx, kv_round: Optional[str] = "bf16"):
+    """Exact KV maintenance: the current token's key and value for every head
+    NOT in head_idx, rounded like the selected heads' (itpub blog on KV
+    caching, figure (b): each step appends the new token's K and V for every
+    head), written at slot ``pos`` of the given caches in place. With it a
+    head left out at one step still holds this token when it is selected at a
+    later step, as in the dense model."""
+    y = np.atleast_2d(np.asarray(y, dtype=np.float64))
+    W = np.asarray(Wqkv, dtype=np.float64)
+    chosen = set(int(i) for i in np.asarray(head_idx).ravel())
+    for i in range(W.shape[0]):
+        if i in chosen:
+            continue
+        for b in range(y.shape[0]):
+            k = W[i, 1] @ y[b]
+            v = W[i, 2] @ y[b]
+            if bqkv is not None:
+                bb = np.asarray(bqkv, dtype=np.float64)
+                k, v = k + bb[i, 1], v + bb[i, 2]
+            if kv_round == "bf16":
+                k, v = round_to_bf16(k), round_to_bf16(v)
+            else:
+                k = k.astype(np.float32).astype(np.float64)
+                v = v.astype(np.float32).astype(np.float64)
+            Kc[b, i, pos] = k
+            Vc[b, i, pos] = v
+
+
 # ----------------------------------------------------------------------------
 # One decoder layer and a stack with the look-ahead predictor
 # ----------------------------------------------------------------------------
@@ -334,6 +362,7 @@ class LayerParams:
     scale: float = 0.125
     eps: float = 1e-5
     act: str = "relu"
+    exact_kv: bool = False
 
 
 @dataclass
@@ -354,7 +383,8 @@ def decode_layer(x, L: LayerF64, P: LayerParams, pos: int, head_idx=None, idx=No
     """One decode step of one pre-LN decoder layer with contextual sparsity:
 
         yA = LN1(x);  S_A = select(y_A P_A^T)       (unless head_idx is given)
-        x1 = x + MHA_{S_A}(yA)                       (eq. (2), appends k, v at pos)
+        x1 = x + MHA_{S_A}(yA)                       (eq. (2), appends k, v at pos;
+                                                      with P.exact_kv every head's k, v)
         yM = LN2(x1); S_M = select((yM A) B^T + b1)  (unless idx is given)
         x2 = x1 + MLP_{S_M}(yM)                      (eq. (1))
     """
@@ -366,6 +396,8 @@ def decode_layer(x, L: LayerF64, P: LayerParams, pos: int, head_idx=None, idx=No
                   else np.asarray(head_idx, dtype=np.int64))
     t.mha = sparse_mha(t.yA, L.Wqkv, L.bqkv, L.WOt, L.bO, L.K, L.V, pos, P.scale,
                        t.head_idx, L.kv_round)
+    if P.exact_kv:
+        unselected_kv(t.yA, L.Wqkv, L.bqkv, L.K, L.V, pos, t.head_idx, L.kv_round)
     t.out_A = t.mha.out
     x1 = x + t.out_A
     t.yM = layernorm(x1, P.eps, L.ln2_g, L.ln2_b)

@@ -152,3 +152,10 @@ def test_lookahead_split_argument_checks():
                 ws_bytes, None) == bd.DV_ERR_ALIGN
     assert tail(ctypes.byref(w), ctypes.byref(D), ctypes.byref(p), ctypes.byref(io), bd.DV_SET_HEADS, W1, 16,
                 None) == bd.DV_ERR_WORKSPACE
+
+
+def test_sparse_mlp_act_rejects_unknown_activation():
+    f = bd._lib_dv_sparse_mlp_act
+    args = [A, 1, 64, 256, A, A, A, None, bd.DV_BF16, A, A, 16, A, 0]
+    assert f(*args, 2, A, 1 << 30, None) == bd.DV_ERR_ARG
+    assert f(*args, -1, A, 1 << 30, None) == bd.DV_ERR_ARG

@@ -450,3 +450,63 @@ def test_sparse_mlp_gelu_all_neurons_is_dense_gelu_ffn():
     want = F.linear(hid, torch.from_numpy(W2t).t().contiguous(), torch.from_numpy(b2)).numpy()
     assert np.allclose(got, want, rtol=1e-12, atol=1e-12)
     assert not np.allclose(O.sparse_mlp(y, W1t, b1, W2t, b2, np.arange(1, N), act="gelu"), got, rtol=1e-9)
+
+
+# --------------------------------------------------------------------------
+# exact KV maintenance for unselected heads
+# --------------------------------------------------------------------------
+
+
+def test_unselected_kv_against_torch_projection_and_bf16_rounding():
+    """Slot pos of every unselected head holds bf16(y W_i^K) and bf16(y W_i^V)
+    as torch's F.linear and its bfloat16 conversion (round to nearest even)
+    give them; selected heads and other slots are untouched."""
+    r = rng(31)
+    B, d, h, dh, cap, pos = 2, 24, 5, 8, 6, 3
+    y = r.standard_normal((B, d))
+    Wqkv = r.standard_normal((h, 3, dh, d)) / np.sqrt(d)
+    bqkv = r.standard_normal((h, 3, dh)) * 0.1
+    K0 = r.standard_normal((B, h, cap, dh))
+    V0 = r.standard_normal((B, h, cap, dh))
+    K, V = K0.copy(), V0.copy()
+    S = [1, 3]
+    O.unselected_kv(y, Wqkv, bqkv, K, V, pos, S, "bf16")
+    ty = torch.from_numpy(y)
+    for i in range(h):
+        if i in S:
+            assert np.array_equal(K[:, i], K0[:, i]) and np.array_equal(V[:, i], V0[:, i])
+            continue
+        for m, cache in ((1, K), (2, V)):
+            want = F.linear(ty, torch.from_numpy(Wqkv[i, m]), torch.from_numpy(bqkv[i, m]))
+            want = want.to(torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+            # float64 -> bf16 directly vs via float32 can differ only where a
+            # double rounding lands on a tie; allow one bf16 ulp there
+            assert np.all(np.abs(cache[:, i, pos] - want) <= np.abs(want) * 2.0 ** -7 + 1e-12)
+        mask = np.ones(cap, bool)
+        mask[pos] = False
+        assert np.array_equal(K[:, i][:, mask], K0[:, i][:, mask])
+
+
+def test_exact_kv_completes_the_dense_cache_and_leaves_outputs_unchanged():
+    """sparse_mha on S followed by unselected_kv writes at slot pos exactly
+    what sparse_mha over all heads writes (the dense cache), and the layer's
+    output is the same with and without exact KV at that step."""
+    r = rng(32)
+    B, d, h, dh, cap, pos = 2, 32, 6, 8, 9, 5
+    L = O.LayerF64(PA=r.standard_normal((h, d)), Wqkv=r.standard_normal((h, 3, dh, d)) / np.sqrt(d), bqkv=None,
+                   WOt=r.standard_normal((h, dh, d)) / np.sqrt(dh), bO=None, K=r.standard_normal((B, h, cap, dh)),
+                   V=r.standard_normal((B, h, cap, dh)), At=r.standard_normal((8, d)),
+                   Bm=r.standard_normal((64, 8)), b1=r.standard_normal(64) * 0.1,
+                   W1t=r.standard_normal((64, d)) / np.sqrt(d), W2t=r.standard_normal((64, d)) / np.sqrt(d))
+    x = r.standard_normal((B, d))
+    dense_K, dense_V = L.K.copy(), L.V.copy()
+    y = O.layernorm(x)
+    O.sparse_mha(y, L.Wqkv, None, L.WOt, None, dense_K, dense_V, pos, 0.3, list(range(h)), "bf16")
+    import copy
+    La, Lb = copy.deepcopy(L), copy.deepcopy(L)
+    ta = O.decode_layer(x, La, O.LayerParams(k=10, k_h=2, scale=0.3), pos)
+    tb = O.decode_layer(x, Lb, O.LayerParams(k=10, k_h=2, scale=0.3, exact_kv=True), pos)
+    assert np.array_equal(ta.x_out, tb.x_out)
+    assert np.array_equal(Lb.K[:, :, pos], dense_K[:, :, pos]) and np.array_equal(Lb.V[:, :, pos], dense_V[:, :, pos])
+    unsel = [i for i in range(h) if i not in set(ta.head_idx.tolist())]
+    assert unsel and np.array_equal(La.K[:, unsel, pos], L.K[:, unsel, pos])  # without: the old slot stays
