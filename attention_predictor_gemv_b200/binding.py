@@ -84,6 +84,12 @@ _lib_dv_sparse_mlp = _sig("dv_sparse_mlp", _c_int,
 _lib_dv_sparse_mlp_act = _sig("dv_sparse_mlp_act", _c_int,
                               [_p, _c_int, _c_int, _c_int, _p, _p, _p, _p, _c_int, _p, _p, _c_int, _p, _c_int, _c_int,
                                _p, _c_size, _p])
+_lib_dv_sparse_mlp_q8 = _sig("dv_sparse_mlp_q8", _c_int,
+                             [_p, _c_int, _c_int, _c_int, _p, _p, _p, _p, _p, _p, _p, _p, _c_int, _p, _c_int, _c_int,
+                              _p, _c_size, _p])
+_lib_dv_sparse_mha_q8 = _sig("dv_sparse_mha_q8", _c_int,
+                             [_p, _c_int, _c_int, _c_int, _c_int, _p, _p, _p, _p, _p, _p, _p, _p, _c_int, _c_int,
+                              _c_float, _p, _p, _c_int, _p, _c_int, _p, _c_size, _p])
 _lib_dv_sparse_mha = _sig("dv_sparse_mha", _c_int,
                           [_p, _c_int, _c_int, _c_int, _c_int, _p, _p, _p, _p, _c_int, _p, _p, _c_int, _c_int, _c_int,
                            _c_float, _p, _p, _c_int, _p, _c_int, _p, _c_size, _p])
@@ -250,6 +256,37 @@ def dv_sparse_mlp(y, W1t, b1, W2t, b2, idx, count, k_max, out, ws, accumulate=Fa
         _check(_lib_dv_sparse_mlp(*args, *tail), "dv_sparse_mlp")
     else:
         _check(_lib_dv_sparse_mlp_act(*args, int(act), *tail), "dv_sparse_mlp_act")
+
+
+def dv_sparse_mlp_q8(y, W1q, W1s, b1, W2q, W2s, b2, idx, count, k_max, out, ws, accumulate=False, act=DV_ACT_RELU,
+                     stream=None):
+    """dv_sparse_mlp_q8: int8 rows W1q, W2q [N][d] with fp32 row scales W1s, W2s [N]."""
+    B, d = y.shape
+    N = W1q.shape[0]
+    _check(_lib_dv_sparse_mlp_q8(_ptr(y, torch.float32, "y"), B, d, N, _ptr(W1q, torch.int8, "W1q"),
+                                 _ptr(W1s, torch.float32, "W1s"), _ptr(b1, torch.float32, "b1"),
+                                 _ptr(W2q, torch.int8, "W2q"), _ptr(W2s, torch.float32, "W2s"),
+                                 _ptr(b2, torch.float32, "b2"), _ptr(idx, torch.int32, "idx"),
+                                 _ptr(count, torch.int32, "count"), int(k_max), _ptr(out, torch.float32, "out"),
+                                 int(bool(accumulate)), int(act), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+                                 _stream(stream)), "dv_sparse_mlp_q8")
+
+
+def dv_sparse_mha_q8(y, Wqkvq, Wqkv_s, bqkv, WOq, WO_s, bO, Kc, Vc, pos, scale, head_idx, head_count, kh_max, out, ws,
+                     accumulate=False, stream=None):
+    """dv_sparse_mha_q8: int8 rows Wqkvq [h][3][dh][d], WOq [h][dh][d] with fp32 row scales
+    Wqkv_s [h][3][dh], WO_s [h][dh]; bf16 KV caches [B][h][cap][dh]."""
+    B, d = y.shape
+    h, _, dh, _ = Wqkvq.shape
+    cap = Kc.shape[2]
+    _check(_lib_dv_sparse_mha_q8(_ptr(y, torch.float32, "y"), B, d, h, dh, _ptr(Wqkvq, torch.int8, "Wqkvq"),
+                                 _ptr(Wqkv_s, torch.float32, "Wqkv_s"), _ptr(bqkv, torch.float32, "bqkv"),
+                                 _ptr(WOq, torch.int8, "WOq"), _ptr(WO_s, torch.float32, "WO_s"),
+                                 _ptr(bO, torch.float32, "bO"), _ptr(Kc, torch.bfloat16, "Kc"),
+                                 _ptr(Vc, torch.bfloat16, "Vc"), int(cap), int(pos), float(scale),
+                                 _ptr(head_idx, torch.int32, "head_idx"), _ptr(head_count, torch.int32, "head_count"),
+                                 int(kh_max), _ptr(out, torch.float32, "out"), int(bool(accumulate)),
+                                 _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)), "dv_sparse_mha_q8")
 
 
 def dv_sparse_mha(y, Wqkv, bqkv, WOt, bO, Kc, Vc, pos, scale, head_idx, head_count, kh_max, out, ws,

@@ -19,7 +19,8 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdejavu.so")
 # One translation unit per kernel family, compiled in parallel, then linked.
 SOURCES = ["dv_api.cu", "dv_inst_legacy.cu", "dv_inst_legacy_attn.cu", "dv_inst_attn_in.cu", "dv_inst_attn_out.cu", "dv_inst_attn_out_f32.cu",
-           "dv_inst_mlp.cu", "dv_inst_pred.cu", "dv_inst_tc.cu"]
+           "dv_inst_mlp.cu", "dv_inst_pred.cu", "dv_inst_tc.cu",
+           "dv_inst_q8.cu"]
 HEADERS = ["dv_common.cuh", "dv_kernels.cuh", "dv_fused.cuh", "dv_colowner.cuh", "dv_launch.cuh", "dv_launchers.cuh",
            "dv_api_kernels.cuh", "dv_stream.cuh", "dv_tc.cuh", "dv_tc_args.h",
            "dv_tc_launch.h"]

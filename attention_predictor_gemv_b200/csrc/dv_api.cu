@@ -657,7 +657,9 @@ size_t dv_workspace_size(int op, const dv_dims* dims) {
     D.kh_max = 0;
   }
   if (!dims_ok(D)) return 0;
-  return layout(D, 2).total > layout(D, 4).total ? layout(D, 2).total : layout(D, 4).total;
+  size_t n = 0;
+  for (int wb : {1, 2, 4}) n = layout(D, wb).total > n ? layout(D, wb).total : n;  // int8, bf16, fp32 weights
+  return n;
 }
 
 dv_status dv_read_device_status(void* ws, dv_stream_t stream, int* out) {
@@ -748,6 +750,72 @@ dv_status dv_sparse_mha(const float* y, int B, int d, int h, int dh, const void*
   DV_CHECK(check_ws(L, ws, ws_bytes));
   return do_sparse_mha(L, ws, y, B, d, h, dh, Wqkv, bqkv, WOt, bO, wdtype, Kc, Vc, cap, pos, scale, head_idx,
                        head_count, kh_max, out, accumulate, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dv_status dv_sparse_mlp_q8(const float* y, int B, int d, int N, const int8_t* W1q, const float* W1s, const float* b1,
+                           const int8_t* W2q, const float* W2s, const float* b2, const int32_t* idx,
+                           const int32_t* count, int k_max, float* out, int accumulate, int act, void* ws,
+                           size_t ws_bytes, dv_stream_t stream) {
+  if (!act_ok(act)) return DV_ERR_ARG;
+  if (!y || !W1q || !W1s || !b1 || !W2q || !W2s || !idx || !count || !out) return DV_ERR_ARG;
+  if (!ok_ptr(y) || !ok_ptr(W1q) || !ok_ptr(W2q) || !ok_ptr(W1s) || !ok_ptr(W2s) || !ok_ptr(out) || !ok_opt(b2))
+    return DV_ERR_ALIGN;
+  dv_dims D = {B, d, N, 0, 0, 0, 0, k_max, 0};
+  if (!dims_ok(D)) return DV_ERR_ARG;
+  if (B > 4 || d % 16 != 0) return DV_ERR_UNSUPPORTED;
+  const Layout L = layout(D, 1);
+  DV_CHECK(check_ws(L, ws, ws_bytes));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (!accumulate) DV_TRY(cudaMemsetAsync(out, 0, 4ull * B * d, st));
+  int* status = at<int>(ws, L.status);
+  if (L.nseg == 0) {
+    if (b2) {  // nothing selected: out (+)= b2 only
+      RowsHeads none{idx, count, nullptr, 0, 1, 0};
+      return cuda_status(run_axpy_q8(W2q, d, N, none, b2, out, B, 1, 0, status, st));
+    }
+    return DV_OK;
+  }
+  int32_t* seg_idx = at<int32_t>(ws, L.seg_idx);
+  float* seg_a = at<float>(ws, L.seg_a);
+  int32_t* seg_cnt = at<int32_t>(ws, L.seg_cnt);
+  DV_TRY(run_mlp_up_q8(W1q, W1s, d, N, y, B, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, L.nseg, act, st));
+  RowsMlp src{seg_idx, seg_a, seg_cnt, L.nseg, L.SEG, W2s};
+  return cuda_status(run_axpy_q8(W2q, d, N, src, b2, out, B, k_max, 4ull * (L.nseg + 1), status, st));
+}
+
+dv_status dv_sparse_mha_q8(const float* y, int B, int d, int h, int dh, const int8_t* Wqkvq, const float* Wqkv_s,
+                           const float* bqkv, const int8_t* WOq, const float* WO_s, const float* bO, void* Kc, void* Vc,
+                           int cap, int pos, float scale, const int32_t* head_idx, const int32_t* head_count,
+                           int kh_max, float* out, int accumulate, void* ws, size_t ws_bytes, dv_stream_t stream) {
+  if (!y || !Wqkvq || !Wqkv_s || !WOq || !WO_s || !Kc || !Vc || !head_idx || !head_count || !out) return DV_ERR_ARG;
+  if (!ok_ptr(y) || !ok_ptr(Wqkvq) || !ok_ptr(Wqkv_s) || !ok_ptr(WOq) || !ok_ptr(WO_s) || !ok_ptr(Kc) ||
+      !ok_ptr(Vc) || !ok_ptr(out) || !ok_opt(bO) || !ok_opt(bqkv))
+    return DV_ERR_ALIGN;
+  if (dh != 64 && dh != 128) return DV_ERR_UNSUPPORTED;
+  if (cap < 1 || pos < 0 || pos >= cap) return DV_ERR_ARG;
+  dv_dims D = {B, d, 1, 0, h, dh, cap, 0, kh_max};
+  if (!dims_ok(D) || h < 1) return DV_ERR_ARG;
+  if (B > 4 || d % 16 != 0) return DV_ERR_UNSUPPORTED;
+  const Layout L = layout(D, 1);
+  DV_CHECK(check_ws(L, ws, ws_bytes));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (!accumulate) DV_TRY(cudaMemsetAsync(out, 0, 4ull * B * d, st));
+  int* status = at<int>(ws, L.status);
+  if (kh_max == 0) {
+    if (bO) {
+      RowsHeads none{head_idx, head_count, nullptr, 0, dh, h};
+      return cuda_status(run_axpy_q8(WOq, d, h * dh, none, bO, out, B, 1, 0, status, st));
+    }
+    return DV_OK;
+  }
+  float* q = at<float>(ws, L.q);
+  float* H = at<float>(ws, L.H);
+  DV_TRY(run_qkv_q8(Wqkvq, Wqkv_s, d, h, dh, y, B, bqkv, head_idx, head_count, kh_max, q, Kc, Vc, cap, pos, status,
+                    st));
+  DV_TRY(run_attn_dt(DV_BF16, dh, q, Kc, Vc, B, h, cap, pos, scale, head_idx, head_count, kh_max, at<float>(ws, L.part),
+                     at<unsigned>(ws, L.attn_ctr), H, status, st));
+  RowsHeads src{head_idx, head_count, H, kh_max, dh, h, WO_s};
+  return cuda_status(run_axpy_q8(WOq, d, h * dh, src, bO, out, B, kh_max * dh, 0, status, st));
 }
 
 static dv_status check_layer(const dv_layer_weights* w, const dv_dims* dims, const dv_layer_params* p) {

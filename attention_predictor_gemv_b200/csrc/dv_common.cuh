@@ -66,6 +66,20 @@ struct WT<__nv_bfloat16> {
   __device__ static __forceinline__ __nv_bfloat16 store_cvt(float v) { return __float2bfloat16_rn(v); }
 };
 
+// Weight-only int8 rows (a per-row scale applied by the kernel): a 16-byte
+// vector holds 16 signed bytes, element i in byte i.
+template <>
+struct WT<int8_t> {
+  static constexpr int E = 16;
+  __device__ static __forceinline__ void unpack(const uint4& u, float (&f)[16]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) f[4 * i + j] = (float)(int8_t)(w[i] >> (8 * j));
+  }
+};
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -604,11 +604,27 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
   // register path: thread (cgi, rg) holds rows rg + i RG of column vector cgi
   const int cgi = tid / RG, rg = tid % RG;
   uint4 wo[WV > 0 ? WV : 1];
+  // whole-row path: rows crank + CS u, u < WU, of W_i^O are this CTA's first
+  // group; they are loaded into registers at the start, so they arrive while
+  // the attention runs
+  constexpr int WU = WV < 0 ? (NB == 1 ? 4 : 2) : 1;
+  constexpr int NVO = WV < 0 ? -WV : 1;
+  uint4 wfirst[WU][NVO];
   auto load_wo = [&]() {
     if constexpr (WV > 0) {
       const KT* Wh = WO + (size_t)head * DH * a.d + c_lo + cgi * E;
 #pragma unroll
       for (int i = 0; i < WV; ++i) wo[i] = ld_stream(Wh + (size_t)(rg + i * RG) * a.d);
+    } else if constexpr (WV < 0) {
+      const KT* Wh = WO + (size_t)head * DH * a.d;
+#pragma unroll
+      for (int u = 0; u < WU; ++u)
+#pragma unroll
+        for (int j = 0; j < NVO; ++j) {
+          const int r = crank + u * CS, v = tid + j * FUSED_THREADS;
+          wfirst[u][j] = (r < DH && v * E < a.d) ? ld_stream(Wh + (size_t)r * a.d + (size_t)v * E)
+                                                 : make_uint4(0u, 0u, 0u, 0u);
+        }
     }
   };
   auto prefetch_wo = [&]() {
@@ -781,8 +797,9 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
   };
   if constexpr (WV < 0) {
     // ---- whole rows crank, crank + CS, ... of W_i^O; this thread's vectors
-    // tid + 256 j of each row; U rows in flight ----
-    constexpr int NVO = -WV, U = 2;
+    // tid + 256 j of each row; U rows in flight, the first group loaded at
+    // the start of the kernel ----
+    constexpr int U = WU;
     const KT* Wh = WO + (size_t)head * DH * a.d;
     float o[NB][NVO][E];
 #pragma unroll
@@ -791,9 +808,29 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
       for (int j = 0; j < NVO; ++j)
 #pragma unroll
         for (int e = 0; e < E; ++e) o[b][j][e] = 0.f;
+    auto consume = [&](const uint4 (&w)[U][NVO], int r0) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int r = r0 + u * CS;
+        if (r < DH) {
+#pragma unroll
+          for (int j = 0; j < NVO; ++j) {
+            float wf[E];
+            WT<KT>::unpack(w[u][j], wf);
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+              const float hv = b < a.nb ? s_H[b][r] : 0.f;
+#pragma unroll
+              for (int e = 0; e < E; ++e) o[b][j][e] = fmaf(hv, wf[e], o[b][j][e]);
+            }
+          }
+        }
+      }
+    };
     if (active) {
+      consume(wfirst, crank);
 #pragma unroll 1
-      for (int r0 = crank; r0 < DH; r0 += CS * U) {
+      for (int r0 = crank + CS * U; r0 < DH; r0 += CS * U) {
         uint4 w[U][NVO];
 #pragma unroll
         for (int u = 0; u < U; ++u)
@@ -803,23 +840,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
             w[u][j] = (r < DH && v * E < a.d) ? ld_stream(Wh + (size_t)r * a.d + (size_t)v * E)
                                               : make_uint4(0u, 0u, 0u, 0u);
           }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int r = r0 + u * CS;
-          if (r < DH) {
-#pragma unroll
-            for (int j = 0; j < NVO; ++j) {
-              float wf[E];
-              WT<KT>::unpack(w[u][j], wf);
-#pragma unroll
-              for (int b = 0; b < NB; ++b) {
-                const float hv = b < a.nb ? s_H[b][r] : 0.f;
-#pragma unroll
-                for (int e = 0; e < E; ++e) o[b][j][e] = fmaf(hv, wf[e], o[b][j][e]);
-              }
-            }
-          }
-        }
+        consume(w, r0);
       }
     }
 #pragma unroll

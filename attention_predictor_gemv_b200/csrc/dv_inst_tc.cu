@@ -11,7 +11,7 @@ template <typename K, typename A>
 cudaError_t launch_tc(K kern, int grid, cudaStream_t st, const A& a) {
   cudaError_t e = allow_smem(kern, TC_SMEM);
   if (e != cudaSuccess) return e;
-  return launch(kern, dim3(grid < 1 ? 1 : grid), dim3(TC_THREADS), TC_SMEM, st, a);
+  return launch_main(kern, dim3(grid < 1 ? 1 : grid), dim3(TC_THREADS), TC_SMEM, st, a);
 }
 
 int clamp_grid(long long units) {

@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(GEMV_THREADS)
     mlp_up_kernel(const T* __restrict__ W1t, int d, int N, const float* __restrict__ X, int nb,
                   const float* __restrict__ b1, const int32_t* __restrict__ idx, const int32_t* __restrict__ count_dev,
                   int k_max, int32_t* __restrict__ seg_idx, float* __restrict__ seg_a, int32_t* __restrict__ seg_cnt,
-                  int* __restrict__ status, int act) {
+                  int* __restrict__ status, int act, const float* __restrict__ wscale) {
   constexpr int SEG = GEMV_WARPS * RPW;
   __shared__ float s_a[SEG][NB];
   __shared__ int s_row[SEG];
@@ -152,9 +152,10 @@ __global__ void __launch_bounds__(GEMV_THREADS)
     for (int r = 0; r < RPW; ++r) {
       int nz = 0;
       const float bias = valid[r] ? b1[rows[r]] : 0.f;
+      const float sc = (valid[r] && wscale) ? wscale[rows[r]] : 1.f;
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
-        const float a = (valid[r] && b < nb) ? activate(acc[r][b] + bias, act) : 0.f;
+        const float a = (valid[r] && b < nb) ? activate(acc[r][b] * sc + bias, act) : 0.f;
         s_a[warp * RPW + r][b] = a;
         nz |= a != 0.f;
       }
@@ -187,12 +188,12 @@ __global__ void __launch_bounds__(GEMV_THREADS)
 // picks q/k/v, c = s % dh the channel. q goes to the workspace (fp32); k and v
 // are rounded to the cache dtype and written at slot `pos`.
 // ----------------------------------------------------------------------------
-template <typename T, int NB, int RPW, int U>
+template <typename T, typename KT, int NB, int RPW, int U>
 __global__ void __launch_bounds__(GEMV_THREADS)
     qkv_kernel(const T* __restrict__ Wqkv, int d, int h, int dh, const float* __restrict__ X, int nb,
                const float* __restrict__ bqkv, const int32_t* __restrict__ head_idx,
-               const int32_t* __restrict__ head_count, int kh_max, float* __restrict__ q, T* __restrict__ Kc,
-               T* __restrict__ Vc, int cap, int pos, int* __restrict__ status) {
+               const int32_t* __restrict__ head_count, int kh_max, float* __restrict__ q, KT* __restrict__ Kc,
+               KT* __restrict__ Vc, int cap, int pos, int* __restrict__ status, const float* __restrict__ wscale) {
   griddep_launch();
   griddep_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -232,12 +233,13 @@ __global__ void __launch_bounds__(GEMV_THREADS)
         const int slot = slot0 + r;
         const int p = slot / per, rem = slot % per, m = rem / dh, c = rem % dh;
         float v = acc[r][b];
+        if (wscale) v *= wscale[(size_t)heads[r] * per + rem];
         if (bqkv) v += bqkv[(size_t)heads[r] * per + rem];
         if (m == 0) {
           q[((size_t)b * kh_max + p) * dh + c] = v;
         } else {
-          T* cache = (m == 1) ? Kc : Vc;
-          cache[(((size_t)b * h + heads[r]) * cap + pos) * dh + c] = WT<T>::store_cvt(v);
+          KT* cache = (m == 1) ? Kc : Vc;
+          cache[(((size_t)b * h + heads[r]) * cap + pos) * dh + c] = WT<KT>::store_cvt(v);
         }
       }
     }
@@ -676,6 +678,7 @@ struct RowsMlp {
   const float* seg_a;
   const int32_t* seg_cnt;
   int nseg, SEG;
+  const float* wscale = nullptr;  // per-row scale of int8 weights, or null
   // Builds the prefix sums of the segment counts in s_off[0..nseg]; returns the total.
   __device__ int prologue(int* s_off, unsigned* sc) const {
     unsigned run = 0;
@@ -709,6 +712,7 @@ struct RowsHeads {
   const int32_t* head_count;
   const float* Hbuf;  // [B][kh_max][dh]
   int kh_max, dh, h;
+  const float* wscale = nullptr;  // per-row scale of int8 weights, or null
   __device__ int prologue(int*, unsigned*) const {
     int hc = *head_count;
     hc = hc < 0 ? 0 : (hc > kh_max ? kh_max : hc);
@@ -756,8 +760,9 @@ __global__ void __launch_bounds__(AX_THREADS)
         row = -1;
       }
       s_rows[i] = row;
+      const float sc = (row >= 0 && src.wscale) ? src.wscale[row] : 1.f;
 #pragma unroll
-      for (int b = 0; b < NB; ++b) s_coef[i][b] = (row >= 0 && b < nb) ? src.coef(slot, b, nb) : 0.f;
+      for (int b = 0; b < NB; ++b) s_coef[i][b] = (row >= 0 && b < nb) ? src.coef(slot, b, nb) * sc : 0.f;
     }
     __syncthreads();
     for (int i0 = 0; i0 < n; i0 += AX_U) {

@@ -57,8 +57,58 @@ inline cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t 
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
+// The highest scheduling priority of the device, given to the kernels of the
+// layer's critical path (Q/K/V, attention + W^O, MLP) so that, when the
+// look-ahead predictor's kernels on the side streams compete for SMs, the
+// critical-path CTAs are placed first. DV_PRIO=0 turns it off. Cached per
+// device.
+inline int main_priority() {
+  static const bool on = [] {
+    const char* e = std::getenv("DV_PRIO");
+    return !(e && e[0] == '0');
+  }();
+  if (!on) return 0;
+  static int prio[64];
+  static bool have[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (!have[dev]) {
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) greatest = 0;
+    prio[dev] = greatest;
+    have[dev] = true;
+  }
+  return prio[dev];
+}
+
+// launch() with the critical-path priority.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_main(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                               Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributePriority;
+  attr[n].val.priority = main_priority();
+  ++n;
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  prefer_max_shared(kern);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Launch as thread-block clusters of `cluster_x` CTAs (plus programmatic
-// stream serialisation).
+// stream serialisation), with the critical-path priority.
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster_x,
                            Args... args) {
@@ -67,15 +117,17 @@ inline cudaError_t launch_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block,
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[3];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = cluster_x;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributePriority;
+  attr[1].val.priority = main_priority();
+  attr[2].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[2].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl_enabled() ? 2 : 1;
+  cfg.numAttrs = pdl_enabled() ? 3 : 2;
   prefer_max_shared(kern);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);

@@ -55,10 +55,10 @@ cudaError_t run_mlp_up_nb(const void* W1t, int d, int N, const float* y, int nb,
   const T* w = static_cast<const T*>(W1t);
   dim3 grid(nseg > 0 ? nseg : 1);
   switch (rpw_for(d, WT<T>::E)) {
-    case 1: return launch(mlp_up_kernel<T, NB, 1, 8>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, act);
-    case 2: return launch(mlp_up_kernel<T, NB, 2, 4>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, act);
-    case 4: return launch(mlp_up_kernel<T, NB, 4, 2>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, act);
-    default: return launch(mlp_up_kernel<T, NB, 8, 1>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, act);
+    case 1: return launch(mlp_up_kernel<T, NB, 1, 8>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, act, (const float*)nullptr);
+    case 2: return launch(mlp_up_kernel<T, NB, 2, 4>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, act, (const float*)nullptr);
+    case 4: return launch(mlp_up_kernel<T, NB, 4, 2>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, act, (const float*)nullptr);
+    default: return launch(mlp_up_kernel<T, NB, 8, 1>, grid, GEMV_THREADS, 0, st, w, d, N, y, nb, b1, idx, count, k_max, seg_idx, seg_a, seg_cnt, status, act, (const float*)nullptr);
   }
 }
 
@@ -114,10 +114,10 @@ cudaError_t run_qkv_nb(const void* Wqkv, int d, int h, int dh, const float* y, i
   T* K = static_cast<T*>(Kc);
   T* V = static_cast<T*>(Vc);
   switch (rpw) {
-    case 1: return launch(qkv_kernel<T, NB, 1, 8>, grid, GEMV_THREADS, 0, st, w, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, K, V, cap, pos, status);
-    case 2: return launch(qkv_kernel<T, NB, 2, 4>, grid, GEMV_THREADS, 0, st, w, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, K, V, cap, pos, status);
-    case 4: return launch(qkv_kernel<T, NB, 4, 2>, grid, GEMV_THREADS, 0, st, w, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, K, V, cap, pos, status);
-    default: return launch(qkv_kernel<T, NB, 8, 1>, grid, GEMV_THREADS, 0, st, w, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, K, V, cap, pos, status);
+    case 1: return launch(qkv_kernel<T, T, NB, 1, 8>, grid, GEMV_THREADS, 0, st, w, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, K, V, cap, pos, status, (const float*)nullptr);
+    case 2: return launch(qkv_kernel<T, T, NB, 2, 4>, grid, GEMV_THREADS, 0, st, w, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, K, V, cap, pos, status, (const float*)nullptr);
+    case 4: return launch(qkv_kernel<T, T, NB, 4, 2>, grid, GEMV_THREADS, 0, st, w, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, K, V, cap, pos, status, (const float*)nullptr);
+    default: return launch(qkv_kernel<T, T, NB, 8, 1>, grid, GEMV_THREADS, 0, st, w, d, h, dh, y, nb, bqkv, head_idx, head_count, kh_max, q, K, V, cap, pos, status, (const float*)nullptr);
   }
 }
 
@@ -225,7 +225,7 @@ template <typename K, typename A>
 cudaError_t launch_fused(K kern, dim3 grid, size_t smem, cudaStream_t st, const A& a) {
   cudaError_t e = allow_smem(kern, smem);
   if (e != cudaSuccess) return e;
-  return launch(kern, grid, FUSED_THREADS, smem, st, a);
+  return launch_main(kern, grid, FUSED_THREADS, smem, st, a);
 }
 
 template <typename T, int NB>
@@ -411,38 +411,38 @@ inline int co_grid(long long groups) {
   return (int)(groups < 1 ? 1 : (groups > cap ? cap : groups));
 }
 
-#define DV_CO_SWITCH(KERN, NB, grid, st, a)                                   \
+#define DV_CO_SWITCH(KERN, NB, grid, st, a, LAUNCH)                           \
   switch (nv) {                                                              \
-    case 1: return launch(KERN<T, NB, 1, 8>, grid, CO_THREADS, 0, st, a);    \
-    case 2: return launch(KERN<T, NB, 2, 4>, grid, CO_THREADS, 0, st, a);    \
-    case 3: return launch(KERN<T, NB, 3, 3>, grid, CO_THREADS, 0, st, a);    \
-    case 4: return launch(KERN<T, NB, 4, 4>, grid, CO_THREADS, 0, st, a);    \
-    case 5: return launch(KERN<T, NB, 5, 4>, grid, CO_THREADS, 0, st, a);    \
-    default: return launch(KERN<T, NB, 6, 4>, grid, CO_THREADS, 0, st, a);   \
+    case 1: return LAUNCH(KERN<T, NB, 1, 8>, grid, CO_THREADS, 0, st, a);    \
+    case 2: return LAUNCH(KERN<T, NB, 2, 4>, grid, CO_THREADS, 0, st, a);    \
+    case 3: return LAUNCH(KERN<T, NB, 3, 3>, grid, CO_THREADS, 0, st, a);    \
+    case 4: return LAUNCH(KERN<T, NB, 4, 4>, grid, CO_THREADS, 0, st, a);    \
+    case 5: return LAUNCH(KERN<T, NB, 5, 4>, grid, CO_THREADS, 0, st, a);    \
+    default: return LAUNCH(KERN<T, NB, 6, 4>, grid, CO_THREADS, 0, st, a);   \
   }
 #define DV_CO_SWITCH_MLP(KERN, NB, grid, st, a)                               \
   switch (nv) {                                                              \
-    case 1: return launch(KERN<T, NB, 1, 8>, grid, CO_THREADS, 0, st, a);    \
-    case 2: return launch(KERN<T, NB, 2, 4>, grid, CO_THREADS, 0, st, a);    \
-    case 3: return launch(KERN<T, NB, 3, 3>, grid, CO_THREADS, 0, st, a);    \
-    case 4: return launch(KERN<T, NB, 4, 2>, grid, CO_THREADS, 0, st, a);    \
-    case 5: return launch(KERN<T, NB, 5, 2>, grid, CO_THREADS, 0, st, a);    \
-    default: return launch(KERN<T, NB, 6, 2>, grid, CO_THREADS, 0, st, a);   \
+    case 1: return launch_main(KERN<T, NB, 1, 8>, grid, CO_THREADS, 0, st, a); \
+    case 2: return launch_main(KERN<T, NB, 2, 4>, grid, CO_THREADS, 0, st, a); \
+    case 3: return launch_main(KERN<T, NB, 3, 3>, grid, CO_THREADS, 0, st, a); \
+    case 4: return launch_main(KERN<T, NB, 4, 2>, grid, CO_THREADS, 0, st, a); \
+    case 5: return launch_main(KERN<T, NB, 5, 2>, grid, CO_THREADS, 0, st, a); \
+    default: return launch_main(KERN<T, NB, 6, 2>, grid, CO_THREADS, 0, st, a); \
   }
 
 // batch 3-4: vectors per thread 1 or 2 only
-#define DV_CO_SWITCH4(KERN, grid, st, a)                                      \
-  if (nv == 1) return launch(KERN<T, 4, 1, 8>, grid, CO_THREADS, 0, st, a);  \
-  return launch(KERN<T, 4, 2, 4>, grid, CO_THREADS, 0, st, a);
+#define DV_CO_SWITCH4(KERN, grid, st, a, LAUNCH)                              \
+  if (nv == 1) return LAUNCH(KERN<T, 4, 1, 8>, grid, CO_THREADS, 0, st, a);  \
+  return LAUNCH(KERN<T, 4, 2, 4>, grid, CO_THREADS, 0, st, a);
 
 template <typename T, int NB>
 cudaError_t run_attn_in_co_nb(const AttnInArgs& a, cudaStream_t st) {
   const int nv = co_nv(a.d, WT<T>::E), R = co_r(nv);
   const dim3 grid(co_grid(((long long)a.kh_max * 3 * a.dh + a.n2h + a.n2r + R - 1) / R));
   if constexpr (NB == 4) {
-    DV_CO_SWITCH4(attn_in_co_kernel, grid, st, a)
+    DV_CO_SWITCH4(attn_in_co_kernel, grid, st, a, launch_main)
   } else {
-    DV_CO_SWITCH(attn_in_co_kernel, NB, grid, st, a)
+    DV_CO_SWITCH(attn_in_co_kernel, NB, grid, st, a, launch_main)
   }
 }
 
@@ -452,7 +452,7 @@ cudaError_t run_mlp_block_co_nb(MlpBlockArgs a, cudaStream_t st) {
   a.G = co_grid(((long long)a.k_max + R - 1) / R);
   const dim3 grid(a.G);
   if constexpr (NB == 4) {
-    DV_CO_SWITCH4(mlp_block_co_kernel, grid, st, a)
+    DV_CO_SWITCH4(mlp_block_co_kernel, grid, st, a, launch_main)
   } else {
     DV_CO_SWITCH_MLP(mlp_block_co_kernel, NB, grid, st, a)
   }
@@ -464,9 +464,9 @@ cudaError_t run_predict_a_co_nb(const PredictAArgs& a, cudaStream_t st) {
   const int rows = (a.PA ? a.h : 0) + (a.At ? a.r : 0);
   const dim3 grid(co_grid((rows + R - 1) / R));
   if constexpr (NB == 4) {
-    DV_CO_SWITCH4(predict_a_co_kernel, grid, st, a)
+    DV_CO_SWITCH4(predict_a_co_kernel, grid, st, a, launch)
   } else {
-    DV_CO_SWITCH(predict_a_co_kernel, NB, grid, st, a)
+    DV_CO_SWITCH(predict_a_co_kernel, NB, grid, st, a, launch)
   }
 }
 #undef DV_CO_SWITCH
@@ -505,7 +505,7 @@ template <typename K, typename A>
 cudaError_t launch_fused_co(K kern, dim3 grid, size_t smem, cudaStream_t st, const A& a) {
   cudaError_t e = allow_smem(kern, smem);
   if (e != cudaSuccess) return e;
-  return launch(kern, grid, CO_THREADS, smem, st, a);
+  return launch_main(kern, grid, CO_THREADS, smem, st, a);
 }
 
 template <typename T, int NB>
@@ -586,6 +586,17 @@ cudaError_t run_attn_dt(dv_dtype kvdt, int dh, const float* q, const void* Kc, c
                         int pos, float scale, const int32_t* head_idx, const int32_t* head_count, int kh_max,
                         float* part, unsigned* ctr, float* H, int* status, cudaStream_t st);
 cudaError_t run_attn_in_any_dt(dv_dtype wdt, const AttnInArgs& a, cudaStream_t st);
+// weight-only int8 (dv_inst_q8.cu), batch 1-4
+cudaError_t run_mlp_up_q8(const int8_t* W1, const float* s1, int d, int N, const float* y, int nb, const float* b1,
+                          const int32_t* idx, const int32_t* count, int k_max, int32_t* seg_idx, float* seg_a,
+                          int32_t* seg_cnt, int* status, int nseg, int act, cudaStream_t st);
+cudaError_t run_qkv_q8(const int8_t* W, const float* s, int d, int h, int dh, const float* y, int nb, const float* bqkv,
+                       const int32_t* head_idx, const int32_t* head_count, int kh_max, float* q, void* Kc, void* Vc,
+                       int cap, int pos, int* status, cudaStream_t st);
+cudaError_t run_axpy_q8(const int8_t* W, int d, int nrows_w, RowsMlp src, const float* bias, float* out, int nb,
+                        int k_max, size_t smem, int* status, cudaStream_t st);
+cudaError_t run_axpy_q8(const int8_t* W, int d, int nrows_w, RowsHeads src, const float* bias, float* out, int nb,
+                        int k_max, size_t smem, int* status, cudaStream_t st);
 cudaError_t run_attn_out_dt(dv_dtype kvdt, const AttnOutArgs& a, cudaStream_t st);
 cudaError_t run_attn_out_bf16(const AttnOutArgs& a, cudaStream_t st);
 cudaError_t run_attn_out_f32(const AttnOutArgs& a, cudaStream_t st);

@@ -149,3 +149,26 @@ def make_kv(shape: LayerShape, B: int, seed: int, device="cpu"):
     K = _randn((B, shape.h, shape.cap, shape.dh), g, device, 1.0, kvdt)
     V = _randn((B, shape.h, shape.cap, shape.dh), g, device, 1.0, kvdt)
     return K, V
+
+
+def quantize_rows(W: torch.Tensor):
+    """Weight-only int8 encoding of a weight tensor whose rows run along the
+    last axis: one fp32 scale per row, s = max |W_row| / 127 (1 for an all-zero
+    row), q = round(W / s) clamped to [-127, 127]. Returns (q int8, s fp32)
+    with s shaped like W without its last axis. The decode path reads q and s;
+    the real row it stands for is q * s."""
+    Wf = W.float()
+    s = Wf.abs().amax(dim=-1) / 127.0
+    s = torch.where(s > 0, s, torch.ones_like(s))
+    q = torch.clamp(torch.round(Wf / s.unsqueeze(-1)), -127, 127).to(torch.int8)
+    return q.contiguous(), s.contiguous()
+
+
+def quantize_layer(t: Dict[str, torch.Tensor]) -> Dict[str, torch.Tensor]:
+    """int8 + row-scale versions of a layer's gathered weights (W1t, W2t,
+    Wqkv, WOt) under the keys W1q/W1s, W2q/W2s, Wqkvq/Wqkv_s, WOq/WO_s."""
+    out = {}
+    for name, qn, sn in (("W1t", "W1q", "W1s"), ("W2t", "W2q", "W2s"), ("Wqkv", "Wqkvq", "Wqkv_s"),
+                         ("WOt", "WOq", "WO_s")):
+        out[qn], out[sn] = quantize_rows(t[name])
+    return out

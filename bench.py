@@ -64,6 +64,9 @@ def parse(argv=None):
     ap.add_argument("--no-extra", action="store_true", help="skip the OPT-6.7B/66B/1.3B/tiny measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=2.0, help="seconds per CPU oracle timing")
+    ap.add_argument("--neurons", type=int, default=0,
+                    help="0: the workload's neuron count; else fewer neurons per layer, for profiler captures of a "
+                         "small case (k stays the headline's)")
     return ap.parse_args(argv)
 
 
@@ -607,7 +610,7 @@ def run_reference(args, rank, dist):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "us", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": v * nL / 1e3, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_of(shape, nL, args.batch, k, k_h, not args.no_lookahead),
+            "config": config_of(args.config, shape, nL, args.batch, k, k_h, not args.no_lookahead),
             "cpu_baseline": {"value": v, "unit": "us/layer-step", "cores": cores, "kind": "oracle",
                              "sample": f"{n} layer-steps of one {args.config}-shaped layer (B=1, k={k}, k_h={k_h}), "
                                        f"float64 numpy on {cores} host cores, one layer-step per timed step"},
@@ -615,10 +618,9 @@ def run_reference(args, rank, dist):
     print(json.dumps(line), flush=True)
 
 
-def config_of(shape, nL, B, k, k_h, lookahead):
+def config_of(key, shape, nL, B, k, k_h, lookahead):
     name = {"opt-175b": "OPT-175B", "opt-66b": "OPT-66B", "opt-6.7b": "OPT-6.7B", "opt-1.3b": "OPT-1.3B",
             "tiny": "tiny"}
-    key = [n for n, s in wl.CONFIGS.items() if s.d == shape.d and s.N == shape.N][0]
     return {"workload": f"{nL} {name[key]}-shaped decoder layers (bf16 weights and KV cache, fp32 arithmetic): "
                         f"d={shape.d}, N={shape.N}, r={shape.r}, h={shape.h}, dh={shape.dh}, KV length {shape.L}, "
                         f"batch {B}, k={k} ({k / shape.N:.0%}), k_h={k_h} ({k_h / shape.h:.0%}), "
@@ -655,6 +657,9 @@ def main():
     nL = args.layers or shape.layers
     keep = 1.0 - args.sparsity
     k, k_h = wl.k_for(keep, shape.N), wl.k_for(keep, shape.h)
+    if args.neurons:  # a small case for profiler captures: fewer neurons, the same k
+        shape = shape.with_(N=args.neurons)
+        k = min(k, args.neurons)
     pos = shape.L
     torch.manual_seed(rank)
     layers = make_layers(shape, nL, 5000 + 100 * rank)
@@ -721,7 +726,7 @@ def main():
         "metric": METRIC, "value": value, "unit": "us", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": dict(config_of(shape, nL, B, k, k_h, not args.no_lookahead),
+        "config": dict(config_of(args.config, shape, nL, B, k, k_h, not args.no_lookahead),
                        parallelism=f"replicas x{world}",
                        l2=f"inputs larger than L2: {nL} layers, {weight_bytes(shape) * nL / 1e9:.0f} GB of "
                           "weights streamed per step"),

@@ -165,6 +165,29 @@ DV_API dv_status dv_sparse_mlp_act(const float* y, int B, int d, int N, const vo
                                    const int32_t* count, int k_max, float* out, int accumulate, int act, void* ws,
                                    size_t ws_bytes, dv_stream_t stream);
 
+/* Weight-only int8 variants of dv_sparse_mlp_act and dv_sparse_mha (the
+ * gathered rows of W1, W2, W^{Q,K,V} and W^O stored as int8 with one fp32
+ * scale per row; the selected bytes halve against bf16. Deja Vu translation,
+ * §1: contextual sparsity is compatible with quantization; the reading note
+ * of "A Survey on Efficient Inference for LLMs": weight-only quantization
+ * speeds up decoding, which is bound by weight loading).
+ * Row i of a weight matrix stands for the real row W[i] = Wq[i] * Ws[i]:
+ *   W1q, W2q [N][d] int8 with W1s, W2s [N] fp32;
+ *   Wqkvq [h][3][dh][d] int8 with Wqkv_s [h][3][dh] fp32;
+ *   WOq [h][dh][d] int8 with WO_s [h][dh] fp32.
+ * Everything else as in the bf16 calls; the KV cache is bf16. Batch 1-4 and
+ * d a multiple of 16 (DV_ERR_UNSUPPORTED otherwise); W1s, W2s, Wqkv_s and
+ * WO_s must be 16-byte aligned like the other arrays. */
+DV_API dv_status dv_sparse_mlp_q8(const float* y, int B, int d, int N, const int8_t* W1q, const float* W1s,
+                                  const float* b1, const int8_t* W2q, const float* W2s, const float* b2,
+                                  const int32_t* idx, const int32_t* count, int k_max, float* out, int accumulate,
+                                  int act, void* ws, size_t ws_bytes, dv_stream_t stream);
+DV_API dv_status dv_sparse_mha_q8(const float* y, int B, int d, int h, int dh, const int8_t* Wqkvq,
+                                  const float* Wqkv_s, const float* bqkv, const int8_t* WOq, const float* WO_s,
+                                  const float* bO, void* Kc, void* Vc, int cap, int pos, float scale,
+                                  const int32_t* head_idx, const int32_t* head_count, int kh_max, float* out,
+                                  int accumulate, void* ws, size_t ws_bytes, dv_stream_t stream);
+
 /* Sparsified MHA, eq. (2), over a KV cache, for the heads in head_idx:
  *   for i in S_A: q, k, v = y Wqkv[i][0..2]^T (+ bqkv[i]);
  *                 K[b][i][pos] = k, V[b][i][pos] = v (rounded to kvdtype);

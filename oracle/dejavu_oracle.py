@@ -89,6 +89,15 @@ def f64_to_bf16_bits(x) -> np.ndarray:
     return (r.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
 
 
+def dequantize_rows(q, scale) -> np.ndarray:
+    """Weight-only int8 rows with one scale per row: the real weight row i is
+    q[i] * scale[i], rows running along the last axis of q (so scale has q's
+    shape without that axis). Exact in float64 (an int8 times a binary32)."""
+    q = np.asarray(q).astype(np.float64)
+    s = np.asarray(scale, dtype=np.float32).astype(np.float64)
+    return q * s[..., None]
+
+
 def as_f64(a, dtype: str) -> np.ndarray:
     """Decode a weight array given as float32 ('f32') or bf16 bits ('bf16')."""
     if dtype == "bf16":

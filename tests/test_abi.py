@@ -159,3 +159,29 @@ def test_sparse_mlp_act_rejects_unknown_activation():
     args = [A, 1, 64, 256, A, A, A, None, bd.DV_BF16, A, A, 16, A, 0]
     assert f(*args, 2, A, 1 << 30, None) == bd.DV_ERR_ARG
     assert f(*args, -1, A, 1 << 30, None) == bd.DV_ERR_ARG
+
+
+def test_q8_block_calls_check_arguments_on_the_host():
+    f = bd._lib_dv_sparse_mlp_q8
+    base = dict(y=A, B=1, d=64, N=256, W1q=A, W1s=A, b1=A, W2q=A, W2s=A, b2=None, idx=A, count=A, k_max=16, out=A,
+                acc=0, act=0, ws=A, wsb=1 << 30, st=None)
+
+    def call(**kw):
+        a = dict(base, **kw)
+        return f(*a.values())
+
+    assert call(W1s=None) == bd.DV_ERR_ARG
+    assert call(W2q=A + 8) == bd.DV_ERR_ALIGN
+    assert call(B=5) == bd.DV_ERR_UNSUPPORTED
+    assert call(d=72) == bd.DV_ERR_UNSUPPORTED  # d % 16
+    assert call(act=3) == bd.DV_ERR_ARG
+    assert call(wsb=16) == bd.DV_ERR_WORKSPACE
+    g = bd._lib_dv_sparse_mha_q8
+    args = [A, 1, 64, 4, 64, A, A, None, A, A, None, A, A, 8, 3, 0.125, A, A, 2, A, 0, A, 1 << 30, None]
+    assert g(*args[:5], None, *args[6:]) == bd.DV_ERR_ARG
+    bad = list(args)
+    bad[4] = 96
+    assert g(*bad) == bd.DV_ERR_UNSUPPORTED  # dh
+    bad = list(args)
+    bad[14] = 8
+    assert g(*bad) == bd.DV_ERR_ARG  # pos >= cap

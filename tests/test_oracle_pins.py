@@ -510,3 +510,23 @@ def test_exact_kv_completes_the_dense_cache_and_leaves_outputs_unchanged():
     assert np.array_equal(Lb.K[:, :, pos], dense_K[:, :, pos]) and np.array_equal(Lb.V[:, :, pos], dense_V[:, :, pos])
     unsel = [i for i in range(h) if i not in set(ta.head_idx.tolist())]
     assert unsel and np.array_equal(La.K[:, unsel, pos], L.K[:, unsel, pos])  # without: the old slot stays
+
+
+def test_dequantize_rows_is_q_times_row_scale():
+    """int8 rows with one scale per row, rows along the last axis: checked
+    element by element with explicit loops and exact rationals (power-of-two
+    scales), a scale of 1 giving the integers back, and a transposed scale
+    shape failing."""
+    r = rng(41)
+    q = r.integers(-127, 128, size=(2, 3, 4, 5)).astype(np.int8)
+    s = (2.0 ** r.integers(-8, 3, size=(2, 3, 4))).astype(np.float32)
+    W = O.dequantize_rows(q, s)
+    assert W.shape == q.shape
+    for a in range(2):
+        for b in range(3):
+            for c in range(4):
+                for e in range(5):
+                    assert W[a, b, c, e] == float(Fraction(int(q[a, b, c, e])) * Fraction(float(s[a, b, c])))
+    assert np.array_equal(O.dequantize_rows(q, np.ones((2, 3, 4), np.float32)), q.astype(np.float64))
+    with pytest.raises(ValueError):
+        O.dequantize_rows(q, np.ones((5, 4, 3, 2), np.float32)[..., 0])
