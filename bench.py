@@ -381,6 +381,59 @@ def kernel_roofline(stk, shape, B, pos, peak_gbs, reps=20):
     return res, lb, k, kp, kh
 
 
+def int8_blocks(stk, shape, pos, peak_gbs, reps=20):
+    """The sparse MLP and MHA blocks of the headline layer 0 (its own selected
+    sets, batch 1) through the block calls, bf16 rows (dv_sparse_mlp /
+    dv_sparse_mha) against weight-only int8 rows with per-row scales
+    (dv_sparse_mlp_q8 / dv_sparse_mha_q8): CUDA graph of one call, replayed;
+    the selected rows (0.2-0.4 GB) exceed L2, so each replay reads HBM."""
+    from attention_predictor_gemv_b200 import binding as bd
+
+    t = stk.layers[0].t
+    q = wl.quantize_layer(t)
+    yM, yA = stk.yM[0], stk.yA[0]
+    idx, cnt, hidx, hcnt = stk.idx[0], stk.count[0], stk.head_idx[0], stk.head_count[0]
+    k, kh = int(cnt.item()), int(hcnt.item())
+    rows = idx[:k].long()
+    kp = int((yM @ t["W1t"][rows].float().t() + t["b1"][rows] > 0).any(dim=0).sum().item())
+    d, dh = shape.d, shape.dh
+    out = torch.empty(1, d, device="cuda")
+    ws_m = bd.workspace(bd.DV_OP_SPARSE_MLP, bd.dims(B=1, d=d, N=shape.N, k_max=k))
+    ws_a = bd.workspace(bd.DV_OP_SPARSE_MHA, bd.dims(B=1, d=d, N=1, h=shape.h, dh=dh, cap=shape.cap, kh_max=kh))
+    K, V = t["K"].clone(), t["V"].clone()
+    sc = 1.0 / float(np.sqrt(dh))
+    kv = kh * (pos + 2) * 2 * dh * 2
+    calls = {
+        "mlp_bf16": (lambda: bd.dv_sparse_mlp(yM, t["W1t"], t["b1"], t["W2t"], None, idx, cnt, k, out, ws_m),
+                     k * (2 * d + 4) + kp * 2 * d),
+        "mlp_int8": (lambda: bd.dv_sparse_mlp_q8(yM, q["W1q"], q["W1s"], t["b1"], q["W2q"], q["W2s"], None, idx, cnt,
+                                                 k, out, ws_m), k * (d + 8) + kp * (d + 4)),
+        "mha_bf16": (lambda: bd.dv_sparse_mha(yA, t["Wqkv"], None, t["WOt"], None, K, V, pos, sc, hidx, hcnt, kh, out,
+                                              ws_a), kh * 4 * dh * d * 2 + kv),
+        "mha_int8": (lambda: bd.dv_sparse_mha_q8(yA, q["Wqkvq"], q["Wqkv_s"], None, q["WOq"], q["WO_s"], None, K, V,
+                                                 pos, sc, hidx, hcnt, kh, out, ws_a), kh * 4 * dh * (d + 4) + kv),
+    }
+    res = {}
+    for name, (fn, nbytes) in calls.items():
+        g = graph_of(fn)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        e1.synchronize()
+        us = e0.elapsed_time(e1) * 1000.0 / reps
+        res[name] = {"us": us, "bytes": nbytes, "gbs": nbytes / us / 1e3, "frac": nbytes / us / 1e3 / peak_gbs}
+        del g
+    del q
+    free_gpu()
+    return {"workload": f"one OPT-175B-shaped layer's sparse MLP (k={k}, k'={kp}) and MHA (k_h={kh}, KV {pos + 1}) "
+                        "blocks, batch 1, block calls (kernel per step)", **res}
+
+
 def free_gpu():
     import gc
 
@@ -399,11 +452,13 @@ def sweep_175b(layers, shape, args, dist):
     weights, and the dense path (every neuron and head) at each batch."""
     out = []
     for B in (1, 2, 4, 8, 16):
+        ls = with_kv(layers, shape, B, 9000 + 100 * B) if B > 1 else layers  # one set of caches per batch
         for s in (0.50, 0.75, 0.85, 0.95, 0.0):
-            res, stk, g, x, _ = point(layers, shape, B, s, 6, 2, dist, kv_seed=9000 + 100 * B)
+            res, stk, g, x, _ = point(ls, shape, B, s, 6, 2, dist)
             res["dense"] = s == 0.0
             out.append(res)
             del stk, g, x
+        del ls
         free_gpu()
     return out
 
@@ -705,6 +760,8 @@ def main():
     side = {}
     if world == 1:
         headline_layer0 = layers[0]
+        if not args.no_extra:
+            side["int8_blocks"] = int8_blocks(stk, shape, pos, peak_gbs)
         del stk
         free_gpu()
         if not args.no_sweep:
