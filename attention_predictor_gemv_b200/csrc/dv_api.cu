@@ -833,6 +833,7 @@ static dv_status check_layer(const dv_layer_weights* w, const dv_dims* dims, con
       !ok_opt(w->ln1_g) || !ok_opt(w->ln1_b) || !ok_opt(w->ln2_g) || !ok_opt(w->ln2_b))
     return DV_ERR_ALIGN;
   if (p->k < 0 || p->k_h < 0) return DV_ERR_ARG;
+  if (p->exact_kv && D.h > KV_REST_MAX_H) return DV_ERR_UNSUPPORTED;  // the unselected-head list lives in shared memory
   // top-k: the union over B rows has at most min(n, B k) members
   if (p->mode == DV_TOPK && (long long)p->k * D.B > D.k_max && D.N > D.k_max) return DV_ERR_ARG;
   if (p->mode_h == DV_TOPK && (long long)p->k_h * D.B > D.kh_max && D.h > D.kh_max) return DV_ERR_ARG;

@@ -248,7 +248,7 @@ typedef struct {
   int exact_kv; /* nonzero: also compute k and v of the UNSELECTED heads and store them at
                    slot pos (every head's cache then holds this token, as a dense model's
                    would; 2 h_unselected dh d more weight bytes); 0: only the selected
-                   heads' slots are written, the others keep what they held */
+                   heads' slots are written, the others keep what they held; h <= 1024 */
 } dv_layer_params;
 
 /* Device buffers for the selected sets and the intermediates of a layer. In

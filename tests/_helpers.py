@@ -46,6 +46,21 @@ def assert_out(got, ref, what="out"):
     assert dmax <= OUT_MAX_REL * max(inf, 1e-30), (what, "max-abs", dmax, inf)
 
 
+def assert_kv_slot(got, ref, what="KV slot"):
+    """A written K or V slot (last axis = dh channels) against the oracle's:
+    every element within one bf16 rounding of the oracle's value
+    (2^-7 |ref|) plus 2^-12 of the largest magnitude in its dh-vector. The
+    second term is the accumulation difference of a d-term fp32 dot product
+    (its absolute error scales with the vector's magnitude, not with one
+    small element); both stay far inside the layer-output bar (max-abs
+    2e-2 ||out||_inf)."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    scale = np.max(np.abs(ref), axis=-1, keepdims=True)
+    bad = np.abs(got - ref) > np.abs(ref) * 2.0 ** -7 + scale * 2.0 ** -12
+    assert not bad.any(), (what, int(bad.sum()), np.argwhere(bad)[:4].tolist())
+
+
 def oracle_layer(t, kv_round="bf16") -> O.LayerF64:
     g = lambda n: f64(t[n]) if n in t and t[n] is not None else None  # noqa: E731
     return O.LayerF64(PA=g("PA"), Wqkv=g("Wqkv"), bqkv=g("bqkv"), WOt=g("WOt"), bO=g("bO"), K=g("K"), V=g("V"),

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 from oracle import dejavu_oracle as O
-from tests._helpers import assert_out, f64
+from tests._helpers import assert_kv_slot, assert_out, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -88,7 +88,7 @@ def test_sparse_mha_q8(name, B, nsel):
         for p, i in enumerate(heads):
             for cache, r in ((t["K"], ref.k_new), (t["V"], ref.v_new)):
                 got = f64(cache[b, i, pos])
-                assert np.all(np.abs(got - r[b, p]) <= np.abs(r[b, p]) * 2.0 ** -7 + 1e-6)
+                assert_kv_slot(got, r[b, p])
     assert bd.dv_read_device_status(ws) == 0
 
 

@@ -14,7 +14,7 @@ import pytest
 import torch
 
 from oracle import dejavu_oracle as O
-from tests._helpers import assert_out, f64, oracle_layer, selected
+from tests._helpers import assert_kv_slot, assert_out, f64, oracle_layer, selected
 
 pytestmark = pytest.mark.gpu
 
@@ -39,9 +39,8 @@ def _shape(name, B):
 
 
 def _assert_slot(cache_gpu, ref_slot):
-    """Slot values within one bf16 rounding of the oracle's."""
-    got = f64(cache_gpu)
-    assert np.all(np.abs(got - ref_slot) <= np.abs(ref_slot) * 2.0 ** -7 + 1e-6)
+    """Slot values within one bf16 rounding of the oracle's (assert_kv_slot)."""
+    assert_kv_slot(f64(cache_gpu), ref_slot)
 
 
 @pytest.mark.parametrize("name,B", [("fused128", 1), ("fused128", 2), ("wide", 1), ("ragged", 1), ("opt-like", 8)])

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 from oracle import dejavu_oracle as O
-from tests._helpers import assert_out, assert_scores, f64, oracle_layer, selected, wname
+from tests._helpers import assert_kv_slot, assert_out, assert_scores, f64, oracle_layer, selected, wname
 
 pytestmark = pytest.mark.gpu
 
@@ -266,8 +266,10 @@ def test_device_status_on_bad_count_and_index():
 
 def _assert_kv_slot(cache_gpu, ref_vals, b, head, pos, is_bf16):
     got = f64(cache_gpu[b, head, pos])
-    tol = np.abs(ref_vals) * 2.0 ** -7 + 1e-6 if is_bf16 else np.abs(ref_vals) * 1e-5 + 1e-6
-    assert np.all(np.abs(got - ref_vals) <= tol)
+    if is_bf16:
+        assert_kv_slot(got, ref_vals)
+    else:
+        assert np.all(np.abs(got - ref_vals) <= np.abs(ref_vals) * 1e-5 + 1e-6)
 
 
 @pytest.mark.parametrize("name,B,pos,nsel", [("tiny", 1, 64, 2), ("tiny", 1, 0, 4), ("ragged", 2, 99, 3),

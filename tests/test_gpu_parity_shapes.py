@@ -27,7 +27,7 @@ import pytest
 import torch
 
 from oracle import dejavu_oracle as O
-from tests._helpers import assert_out, assert_scores, f64, oracle_layer, selected
+from tests._helpers import assert_kv_slot, assert_out, assert_scores, f64, oracle_layer, selected
 
 pytestmark = pytest.mark.gpu
 
@@ -101,7 +101,7 @@ def test_decode_layer_at_large_row_lengths(name, B, kf, khf):
         for j, i in enumerate(hsel):
             for cache, ref in ((t["K"], tr.mha.k_new), (t["V"], tr.mha.v_new)):
                 got = f64(cache[b, i, s.L])
-                assert np.all(np.abs(got - ref[b, j]) <= np.abs(ref[b, j]) * 2.0 ** -7 + 1e-6)
+                assert_kv_slot(got, ref[b, j])
     _no_device_errors(ws)
 
 
@@ -252,7 +252,7 @@ def test_opt175b_shaped_stack_in_bench_configuration(B):
             for j, i in enumerate(hs):
                 for cache, ref in ((t["K"], k_new), (t["V"], v_new)):
                     got = f64(cache[b, i, pos])
-                    assert np.all(np.abs(got - ref[b, j]) <= np.abs(ref[b, j]) * 2.0 ** -7 + 1e-6)
+                    assert_kv_slot(got, ref[b, j])
         xcur = xout
     assert_out(x.cpu().numpy() - f64(xin), xcur - f64(xin), "stack out - x")
     _no_device_errors(stk.ws_main)

@@ -16,7 +16,7 @@ import pytest
 import torch
 
 from oracle import dejavu_oracle as O
-from tests._helpers import assert_out, assert_scores, f64, oracle_layer, selected
+from tests._helpers import assert_kv_slot, assert_out, assert_scores, f64, oracle_layer, selected
 
 pytestmark = pytest.mark.gpu
 
@@ -129,7 +129,7 @@ def test_tc_sparse_mha(name, B, nsel):
         for p, i in enumerate(heads):
             for cache, r in ((t["K"], ref.k_new), (t["V"], ref.v_new)):
                 got = f64(cache[b, i, pos])
-                assert np.all(np.abs(got - r[b, p]) <= np.abs(r[b, p]) * 2.0 ** -7 + 1e-6)
+                assert_kv_slot(got, r[b, p])
     untouched = [i for i in range(s.h) if i not in set(heads.tolist())]
     assert torch.equal(t["K"][:, untouched], K0[:, untouched])
     _no_device_errors(ws)
