@@ -30,8 +30,8 @@ constexpr int KH_LIMIT = 1000;  // B * kh_max counters must fit the header
 struct Layout {
   size_t status, sel_ticket_h, sel_ticket_m, pa_ticket, pb_ticket, attn_ctr, hist, t1;
   size_t yA, yM, z, scores_h, bm_h, head_idx, head_count, scores, bm_m, idx, count;
-  size_t q, part, H, seg_idx, seg_a, seg_cnt, tc_act, tc_rowid, tc_tiles, total;
-  int nseg, SEG, nsplit_max, KC;
+  size_t q, part, H, seg_idx, seg_a, seg_cnt, tc_x, tc_act, tc_rowid, tc_tiles, total;
+  int nseg, SEG, nsplit_max, KC, XC;
 };
 
 bool dims_ok(const dv_dims& D) {
@@ -74,10 +74,14 @@ Layout layout(const dv_dims& D, int wbytes) {
   L.seg_idx = take(4ull * L.nseg * L.SEG);
   L.seg_a = take(4ull * L.nseg * L.SEG * B);
   L.seg_cnt = take(4ull * (L.nseg > 0 ? L.nseg : 1));
-  // tensor-core MLP: activations compacted per tile of 128 selected neurons
+  // tensor-core path: the operand split into bf16 hi / lo rows [16][XC]
+  // (LN output or the attention outputs H), and the MLP's activations
+  // compacted per tile of 128 selected neurons, hi / lo rows [16][KC]
   const int tiles = tc_tiles(D.k_max);
   L.KC = tiles * TC_M;
-  L.tc_act = take(4ull * TC_N * L.KC);
+  L.XC = D.d > D.kh_max * D.dh ? D.d : D.kh_max * D.dh;
+  L.tc_x = take(2ull * 2 * TC_N * L.XC);
+  L.tc_act = take(2ull * 2 * TC_N * (L.KC > 0 ? L.KC : 1));
   L.tc_rowid = take(4ull * (L.KC > 0 ? L.KC : 1));
   L.tc_tiles = take(4ull * (tiles > 0 ? tiles : 1));
   L.total = o;
@@ -114,6 +118,26 @@ dv_status tc_qkv(const Layout& L, void* ws, const float* y, int B, int d, int h,
 dv_status tc_wo(const Layout& L, void* ws, int B, int d, int h, int dh, const void* WOt, const float* bO,
                 const int32_t* head_idx, const int32_t* head_count, int kh_max, float* out, cudaStream_t st);
 
+// Selection of B score rows of length n: one thread-block cluster per row
+// (select_rows_kernel) up to SR_MAX_N scores per row, the one-CTA-per-row
+// select_kernel beyond. DV_SELROWS=0 keeps select_kernel for every n.
+bool sel_rows_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("DV_SELROWS");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+cudaError_t select_any(const float* scores, int nrows, int n, int k, float tau, int mode, uint32_t* bm,
+                       unsigned* ticket, int32_t* idx, int32_t* count, cudaStream_t st) {
+  if (n <= SR_MAX_N && sel_rows_enabled()) {
+    SelectRowsArgs a{scores, n, nrows, k, mode, tau, bm, ticket, idx, count};
+    return launch_cluster(select_rows_kernel, dim3(SR_CS, nrows), dim3(SR_THREADS), 0, st, SR_CS, a);
+  }
+  return run_select(scores, nrows, n, k, tau, mode, bm, ticket, idx, count, st);
+}
+
 // ---------------------------------------------------------------------------
 // Operation bodies shared by the public entry points
 // ---------------------------------------------------------------------------
@@ -124,7 +148,7 @@ dv_status do_predict_mlp(const Layout& L, void* ws, const float* y, int B, int d
   float* z = at<float>(ws, L.z);
   DV_TRY(run_gemv(dt, At, r, d, y, d, B, nullptr, z, r, st));
   DV_TRY(run_gemv(dt, Bm, N, r, z, r, B, b1, scores, N, st));
-  DV_TRY(run_select(scores, B, N, k, tau, mode, at<uint32_t>(ws, L.bm_m), at<unsigned>(ws, L.sel_ticket_m), idx, count,
+  DV_TRY(select_any(scores, B, N, k, tau, mode, at<uint32_t>(ws, L.bm_m), at<unsigned>(ws, L.sel_ticket_m), idx, count,
                     st));
   return DV_OK;
 }
@@ -133,7 +157,7 @@ dv_status do_predict_heads(const Layout& L, void* ws, const float* y, int B, int
                            int k_h, float tau, int mode, float* scores, int32_t* head_idx, int32_t* head_count,
                            cudaStream_t st) {
   DV_TRY(run_gemv(dt, PA, h, d, y, d, B, nullptr, scores, h, st));
-  DV_TRY(run_select(scores, B, h, k_h, tau, mode, at<uint32_t>(ws, L.bm_h), at<unsigned>(ws, L.sel_ticket_h), head_idx,
+  DV_TRY(select_any(scores, B, h, k_h, tau, mode, at<uint32_t>(ws, L.bm_h), at<unsigned>(ws, L.sel_ticket_h), head_idx,
                     head_count, st));
   return DV_OK;
 }
@@ -226,7 +250,6 @@ dv_status tc_mlp(const Layout& L, void* ws, const float* y, int B, int d, int N,
   a.b1 = b1;
   a.W2t = static_cast<const bf16*>(W2t);
   a.b2 = b2;
-  a.y = y;
   a.idx = idx;
   a.count = count;
   a.k_max = k_max;
@@ -234,11 +257,16 @@ dv_status tc_mlp(const Layout& L, void* ws, const float* y, int B, int d, int N,
   a.N = N;
   a.nb = B;
   a.KC = L.KC;
-  a.act_c = at<float>(ws, L.tc_act);
+  bf16* xhi = at<bf16>(ws, L.tc_x);
+  a.xhi = xhi;
+  a.xlo = xhi + (size_t)TC_N * L.XC;
+  a.act_hi = at<bf16>(ws, L.tc_act);
+  a.act_lo = a.act_hi + (size_t)TC_N * (L.KC > 0 ? L.KC : 1);
   a.rowid_c = at<int32_t>(ws, L.tc_rowid);
   a.tile_cnt = at<int32_t>(ws, L.tc_tiles);
   a.out = out;
   a.status = at<int>(ws, L.status);
+  if (k_max > 0) DV_TRY(run_tc_split(y, B, d, d, xhi, xhi + (size_t)TC_N * L.XC, d, st));
   return cuda_status(run_tc_mlp(a, st));
 }
 
@@ -248,7 +276,9 @@ dv_status tc_qkv(const Layout& L, void* ws, const float* y, int B, int d, int h,
   TcQkvArgs a = {};
   a.Wqkv = static_cast<const bf16*>(Wqkv);
   a.bqkv = bqkv;
-  a.y = y;
+  bf16* xhi = at<bf16>(ws, L.tc_x);
+  a.xhi = xhi;
+  a.xlo = xhi + (size_t)TC_N * L.XC;
   a.head_idx = head_idx;
   a.head_count = head_count;
   a.kh_max = kh_max;
@@ -262,6 +292,7 @@ dv_status tc_qkv(const Layout& L, void* ws, const float* y, int B, int d, int h,
   a.Kc = static_cast<bf16*>(Kc);
   a.Vc = static_cast<bf16*>(Vc);
   a.status = at<int>(ws, L.status);
+  DV_TRY(run_tc_split(y, B, d, d, xhi, xhi + (size_t)TC_N * L.XC, d, st));
   return cuda_status(run_tc_qkv(a, st));
 }
 
@@ -270,7 +301,9 @@ dv_status tc_wo(const Layout& L, void* ws, int B, int d, int h, int dh, const vo
   TcWoArgs a = {};
   a.WOt = static_cast<const bf16*>(WOt);
   a.bO = bO;
-  a.H = at<float>(ws, L.H);
+  bf16* hhi = at<bf16>(ws, L.tc_x);
+  a.hhi = hhi;
+  a.hlo = hhi + (size_t)TC_N * L.XC;
   a.head_idx = head_idx;
   a.head_count = head_count;
   a.kh_max = kh_max;
@@ -280,6 +313,9 @@ dv_status tc_wo(const Layout& L, void* ws, int B, int d, int h, int dh, const vo
   a.nb = B;
   a.out = out;
   a.status = at<int>(ws, L.status);
+  if (kh_max > 0)
+    DV_TRY(run_tc_split(at<float>(ws, L.H), B, kh_max * dh, (long long)kh_max * dh, hhi, hhi + (size_t)TC_N * L.XC,
+                        (long long)kh_max * dh, st));
   return cuda_status(run_tc_wo(a, st));
 }
 
@@ -315,7 +351,6 @@ bool fused_ok(const dv_dims& D, dv_dtype wdt) {
 dv_status fused_predict_rest(const Layout& L, void* ws, const dv_layer_weights* w, const dv_dims& D,
                              const dv_layer_params* p, bool heads, bool neurons, float* sh, int32_t* hidx,
                              int32_t* hcnt, float* sm, int32_t* midx, int32_t* mcnt, cudaStream_t st) {
-  const bool hist_mode = p->mode == DV_TOPK && p->k > 0 && p->k < D.N;
   if (neurons) {
     PredictBArgs b = {};
     b.z = at<float>(ws, L.z);
@@ -324,35 +359,28 @@ dv_status fused_predict_rest(const Layout& L, void* ws, const dv_layer_weights* 
     b.N = D.N;
     b.r = D.r;
     b.nb = D.B;
-    b.hist_mode = hist_mode ? 1 : 0;
+    b.hist_mode = 0;
     b.scores = sm;
     b.hist = at<unsigned>(ws, L.hist);
     DV_TRY(run_predict_b_dt(w->wdtype, b, st));
+    DV_TRY(select_any(sm, D.B, D.N, p->k, p->tau, p->mode, at<uint32_t>(ws, L.bm_m), at<unsigned>(ws, L.pb_ticket),
+                      midx, mcnt, st));
   }
-  SelectFinishArgs f = {};
-  f.scores = sm;
-  f.hist = at<unsigned>(ws, L.hist);
-  f.bitmaps = at<uint32_t>(ws, L.bm_m);
-  f.ticket = at<unsigned>(ws, L.pb_ticket);
-  f.neuron_rows = neurons ? D.B : 0;
-  f.N = D.N;
-  f.nb = D.B;
-  f.k = p->k;
-  f.mode = p->mode;
-  f.tau = p->tau;
-  f.idx = midx;
-  f.count = mcnt;
-  f.scores_h = heads ? sh : nullptr;
-  f.h = D.h;
-  f.k_h = p->k_h;
-  f.mode_h = p->mode_h;
-  f.tau_h = p->tau_h;
-  f.head_idx = hidx;
-  f.head_count = hcnt;
-  const int grid = (neurons ? D.B : 0) + (heads ? 1 : 0);
-  const size_t smem = 4ull * (neurons && hist_mode ? (D.N > D.h ? D.N : D.h) : D.h);
-  DV_TRY(allow_smem(select_finish_kernel, smem));
-  DV_TRY(launch(select_finish_kernel, dim3(grid), dim3(SEL_THREADS), smem, st, f));
+  if (heads) {
+    SelectFinishArgs f = {};
+    f.neuron_rows = 0;
+    f.nb = D.B;
+    f.scores_h = sh;
+    f.h = D.h;
+    f.k_h = p->k_h;
+    f.mode_h = p->mode_h;
+    f.tau_h = p->tau_h;
+    f.head_idx = hidx;
+    f.head_count = hcnt;
+    const size_t smem = 4ull * D.h;
+    DV_TRY(allow_smem(select_finish_kernel, smem));
+    DV_TRY(launch(select_finish_kernel, dim3(1), dim3(SEL_THREADS), smem, st, f));
+  }
   return DV_OK;
 }
 
@@ -708,7 +736,7 @@ dv_status dv_topk(const float* scores, int B, int n, int k, float tau, int mode,
   dv_dims D = {B, 8, n, 0, 0, 0, 0, (k > n ? n : (k < 0 ? 0 : k)), 0};
   const Layout L = layout(D, 2);
   DV_CHECK(check_ws(L, ws, ws_bytes));
-  return cuda_status(run_select(scores, B, n, k, tau, mode, at<uint32_t>(ws, L.bm_m), at<unsigned>(ws, L.sel_ticket_m),
+  return cuda_status(select_any(scores, B, n, k, tau, mode, at<uint32_t>(ws, L.bm_m), at<unsigned>(ws, L.sel_ticket_m),
                                 idx, count, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -897,11 +925,11 @@ dv_status dv_predict_layer_tail(const dv_layer_weights* w, const dv_dims* dims, 
                                 out->scores, out->idx, out->count, st));
   } else {
     if (heads)
-      DV_TRY(run_select(out->scores_h, D.B, D.h, p->k_h, p->tau_h, p->mode_h, at<uint32_t>(ws, L.bm_h),
+      DV_TRY(select_any(out->scores_h, D.B, D.h, p->k_h, p->tau_h, p->mode_h, at<uint32_t>(ws, L.bm_h),
                         at<unsigned>(ws, L.sel_ticket_h), out->head_idx, out->head_count, st));
     if (neurons) {
       DV_TRY(run_gemv(w->wdtype, w->Bm, D.N, D.r, at<float>(ws, L.z), D.r, D.B, w->b1, out->scores, D.N, st));
-      DV_TRY(run_select(out->scores, D.B, D.N, p->k, p->tau, p->mode, at<uint32_t>(ws, L.bm_m),
+      DV_TRY(select_any(out->scores, D.B, D.N, p->k, p->tau, p->mode, at<uint32_t>(ws, L.bm_m),
                         at<unsigned>(ws, L.sel_ticket_m), out->idx, out->count, st));
     }
   }
@@ -1046,5 +1074,5 @@ extern "C" dv_status dv_topk_static(const float* scores, int B, int n, int k, fl
   unsigned* ticket = static_cast<unsigned*>(base);
   uint32_t* bitmaps = reinterpret_cast<uint32_t*>(static_cast<char*>(base) + 256);
   DV_TRY(cudaMemsetAsync(ticket, 0, sizeof(unsigned), st));  // the last-CTA ticket starts at zero
-  return cuda_status(run_select(scores, B, n, k, tau, mode, bitmaps, ticket, idx, count, st));
+  return cuda_status(select_any(scores, B, n, k, tau, mode, bitmaps, ticket, idx, count, st));
 }

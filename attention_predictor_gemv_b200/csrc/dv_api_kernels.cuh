@@ -473,6 +473,207 @@ __global__ void __launch_bounds__(SEL_THREADS) select_finish_kernel(SelectFinish
 
 
 // ----------------------------------------------------------------------------
+// select_rows_kernel: the selected set of B score rows of length n (top-k per
+// row, ties to the lower index, or s > tau), united over the rows, as an
+// ascending index list. One thread-block cluster of SR_CS CTAs per row; CTA
+// c holds the keys of a contiguous index range of the row in registers
+// (order-preserving 32-bit keys: NaN lowest, -0 == +0), SR_KPT per thread.
+//
+// Top-k: the k-th largest key T is found exactly by four radix passes of 8
+// bits, most significant first. In each pass every warp counts the digits of
+// its keys that match the prefix found so far into its own 256-bin
+// histogram in shared memory; the CTA sums its 8 warp histograms, publishes
+// the sum, and after one cluster barrier every CTA reads the SR_CS sums
+// through distributed shared memory and picks the same digit. The keys above
+// T are taken, and of the keys equal to T the kk lowest-index ones (their
+// rank is the count of equal keys in lower-indexed words: in the warp, the
+// CTA's earlier warps, and the cluster's earlier CTAs).
+//
+// The row's bitmap: with one row each CTA writes its own indices at its
+// offset in the cluster; with several rows every cluster stores its bitmap,
+// and the last cluster to finish (ticket) ORs the rows and writes the union.
+// ----------------------------------------------------------------------------
+constexpr int SR_CS = 8;
+constexpr int SR_THREADS = 256;
+constexpr int SR_WARPS = SR_THREADS / 32;
+constexpr int SR_KPT = 24;
+constexpr int SR_MAX_N = SR_CS * SR_THREADS * SR_KPT;  // 49152
+constexpr int SR_MAX_WPC = SR_MAX_N / 32 / SR_CS;      // bitmap words per CTA
+
+struct SelectRowsArgs {
+  const float* scores;  // [nrows][n]
+  int n, nrows, k, mode;
+  float tau;
+  uint32_t* bitmaps;    // [nrows][(n + 31) / 32] (used when nrows > 1)
+  unsigned* ticket;     // zero on entry, left zero
+  int32_t* idx;
+  int32_t* count;
+};
+
+__global__ void __launch_bounds__(SR_THREADS) select_rows_kernel(SelectRowsArgs a) {
+  __shared__ unsigned s_wh[SR_WARPS][256];  // per-warp digit histograms
+  __shared__ unsigned s_cnt[2][256];        // this CTA's digit counts (read by the cluster)
+  __shared__ uint32_t s_bm[SR_MAX_WPC];     // this CTA's bitmap words
+  __shared__ unsigned s_wv[SR_WARPS];       // per-warp counts
+  __shared__ unsigned sc[SR_WARPS + 1];
+  __shared__ unsigned s_ceq, s_csel, s_digit, s_kk;  // s_ceq, s_csel: read by the cluster
+  __shared__ int s_last;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int crank = (int)cluster.block_rank();
+  const int row = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned lt = (1u << lane) - 1u;
+  griddep_launch();
+  griddep_wait();
+  const int n = a.n, nw = (n + 31) >> 5;
+  const int wpc = (nw + SR_CS - 1) / SR_CS;
+  const int cw0 = crank * wpc, cw1 = min(nw, cw0 + wpc);
+  const int wpw = (wpc + SR_WARPS - 1) / SR_WARPS;  // <= SR_KPT (n <= SR_MAX_N, checked on the host)
+  const int ww0 = cw0 + warp * wpw, ww1 = min(cw1, ww0 + wpw);
+  const float* srow = a.scores + (size_t)row * n;
+
+  uint32_t key[SR_KPT];
+  unsigned vmask = 0u;  // bit j: key j exists
+#pragma unroll
+  for (int j = 0; j < SR_KPT; ++j) {
+    const int w = ww0 + j, i = w * 32 + lane;
+    const bool v = w < ww1 && i < n;
+    key[j] = v ? ord_key(srow[i]) : 0u;
+    vmask |= (v ? 1u : 0u) << j;
+  }
+
+  const bool topk = a.mode == 0 && a.k > 0 && a.k < n;
+  uint32_t T = 0u;
+  unsigned kk = 0u;
+  if (topk) {
+    uint32_t prefix = 0u, mask = 0u;
+    kk = (unsigned)a.k;
+#pragma unroll 1
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+#pragma unroll
+      for (int w = 0; w < SR_WARPS; ++w) s_wh[w][tid] = 0u;
+      __syncthreads();
+#pragma unroll
+      for (int j = 0; j < SR_KPT; ++j)
+        if (((vmask >> j) & 1u) && (key[j] & mask) == prefix) atomicAdd(&s_wh[warp][(key[j] >> shift) & 255u], 1u);
+      __syncthreads();
+      unsigned c = 0u;
+#pragma unroll
+      for (int w = 0; w < SR_WARPS; ++w) c += s_wh[w][255 - tid];  // thread t: bin 255 - t (descending)
+      s_cnt[pass & 1][tid] = c;
+      cluster.sync();
+      unsigned tot = 0u;
+#pragma unroll
+      for (int r = 0; r < SR_CS; ++r) tot += cluster.map_shared_rank(&s_cnt[pass & 1][0], r)[tid];
+      unsigned total;
+      const unsigned above = block_exclusive_scan<SR_THREADS>(tot, sc, &total);
+      if (above < kk && kk <= above + tot) {
+        s_digit = 255u - (unsigned)tid;
+        s_kk = kk - above;
+      }
+      __syncthreads();
+      prefix |= s_digit << shift;
+      mask |= 0xffu << shift;
+      kk = s_kk;
+    }
+    T = prefix;  // the k-th largest key; kk of the keys equal to it are taken
+  }
+
+  // ---- this CTA's bitmap words ----
+  unsigned rank = 0u;  // keys equal to T in lower-indexed words of the row
+  if (topk) {
+    unsigned eq = 0u;
+#pragma unroll
+    for (int j = 0; j < SR_KPT; ++j) eq += __popc(__ballot_sync(0xffffffffu, ((vmask >> j) & 1u) && key[j] == T));
+    if (lane == 0) s_wv[warp] = eq;
+    __syncthreads();
+    unsigned ctot = 0u, wbefore = 0u;
+#pragma unroll
+    for (int w = 0; w < SR_WARPS; ++w) {
+      wbefore += w < warp ? s_wv[w] : 0u;
+      ctot += s_wv[w];
+    }
+    if (tid == 0) s_ceq = ctot;
+    cluster.sync();
+    unsigned cbefore = 0u;
+    for (int r = 0; r < crank; ++r) cbefore += *cluster.map_shared_rank(&s_ceq, r);
+    rank = cbefore + wbefore;
+  }
+  const uint32_t tau_key = ord_key(a.tau);
+  const bool tau_nan = a.tau != a.tau;
+  unsigned nsel = 0u;
+#pragma unroll
+  for (int j = 0; j < SR_KPT; ++j) {
+    const bool v = (vmask >> j) & 1u;
+    bool take;
+    if (topk) {
+      const bool e = v && key[j] == T;
+      const unsigned em = __ballot_sync(0xffffffffu, e);
+      take = v && (key[j] > T || (e && rank + __popc(em & lt) < kk));
+      rank += __popc(em);
+    } else if (a.mode == 1) {
+      take = v && !tau_nan && key[j] != 0u && key[j] > tau_key;  // NaN (key 0) never passes
+    } else {
+      take = v && a.k >= n;
+    }
+    const uint32_t word = __ballot_sync(0xffffffffu, take);
+    const int w = ww0 + j;
+    if (lane == 0 && w < ww1) s_bm[w - cw0] = word;
+    nsel += __popc(word);
+  }
+  __syncthreads();
+
+  // ---- several rows: store the bitmap; the last cluster forms the union ----
+  if (a.nrows > 1) {
+    uint32_t* bm = a.bitmaps + (size_t)row * nw;
+    for (int w = cw0 + tid; w < cw1; w += SR_THREADS) bm[w] = s_bm[w - cw0];
+    __threadfence();
+    cluster.sync();  // every CTA of the row has stored its words
+    if (crank == 0 && tid == 0) {
+      const int last = atomicAdd(a.ticket, 1u) == (unsigned)a.nrows - 1u;
+#pragma unroll
+      for (int r = 0; r < SR_CS; ++r) *cluster.map_shared_rank(&s_last, r) = last;
+    }
+    cluster.sync();
+    if (!s_last) return;
+    __threadfence();
+    nsel = 0u;
+    for (int w = cw0 + tid; w < cw1; w += SR_THREADS) {
+      uint32_t u = 0u;
+      for (int rr = 0; rr < a.nrows; ++rr) u |= __ldcg(a.bitmaps + (size_t)rr * nw + w);
+      s_bm[w - cw0] = u;
+    }
+    __syncthreads();
+    if (crank == 0 && tid == 0) *a.ticket = 0u;
+    for (int w = ww0; w < ww1; ++w) nsel += __popc(s_bm[w - cw0]) * (lane == 0 ? 1u : 0u);
+    nsel = __reduce_add_sync(0xffffffffu, nsel);
+  } else {
+    nsel = __shfl_sync(0xffffffffu, nsel, 0);
+  }
+  // ---- the index list: warp offsets in the CTA, CTA offsets in the cluster ----
+  if (lane == 0) s_wv[warp] = nsel;
+  __syncthreads();
+  unsigned ctot = 0u, wbefore = 0u;
+#pragma unroll
+  for (int w = 0; w < SR_WARPS; ++w) {
+    wbefore += w < warp ? s_wv[w] : 0u;
+    ctot += s_wv[w];
+  }
+  if (tid == 0) s_csel = ctot;
+  cluster.sync();
+  unsigned off = wbefore;
+  for (int r = 0; r < crank; ++r) off += *cluster.map_shared_rank(&s_csel, r);
+  if (crank == SR_CS - 1 && tid == 0) *a.count = (int32_t)(off - wbefore + ctot);
+  for (int w = ww0; w < ww1; ++w) {
+    const uint32_t u = s_bm[w - cw0];
+    if ((u >> lane) & 1u) a.idx[off + __popc(u & lt)] = w * 32 + lane;
+    off += __popc(u);
+  }
+  cluster.sync();  // no CTA exits while another may still read its shared memory
+}
+
+// ----------------------------------------------------------------------------
 // Gate: returns once the previous kernel on its stream has completed and its
 // writes are visible. Ends the look-ahead predictor so that a kernel on
 // another stream that depends on it through an event, and that may be

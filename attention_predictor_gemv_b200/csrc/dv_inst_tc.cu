@@ -34,6 +34,13 @@ bool tc_shape_ok(int B, int wbytes, int dh, int k_max) {
 
 int tc_tiles(int k_max) { return (k_max + TC_M - 1) / TC_M; }
 
+cudaError_t run_tc_split(const float* x, int nb, int n, long long ld_src, __nv_bfloat16* hi, __nv_bfloat16* lo,
+                         long long ld_dst, cudaStream_t st) {
+  TcSplitArgs a{x, nb, n, ld_src, hi, lo, ld_dst};
+  const int gx = (n + 255) / 256 < 64 ? (n + 255) / 256 : 64;
+  return launch_main(tc_split_kernel, dim3(gx > 0 ? gx : 1, TC_N), dim3(256), 0, st, a);
+}
+
 cudaError_t run_tc_qkv(const TcQkvArgs& a, cudaStream_t st) {
   const long long units = ((long long)a.kh_max * 3 * a.dh + TC_M - 1) / TC_M;
   if (units == 0) return cudaSuccess;

@@ -14,15 +14,18 @@
 // with M = 128 (gathered rows, or output columns), N = 16 (the batch rows,
 // zero-padded) and 64 K-elements per pipeline stage.
 //
+// The activations enter as two bf16 arrays, hi = bf16(v) and lo =
+// bf16(v - hi) (tc_split_kernel, or the W1 kernel's epilogue for the W2
+// operand), so hi + lo carries 16 significant bits of every activation:
+// D = W X_hi + W X_lo is accurate to about 2^-16 relative instead of the 2^-9
+// of one bf16 rounding, at twice the (idle) tensor work.
+//
 // Per CTA (128 threads, one CTA per SM, persistent over work units):
-//   * all threads stage the weight tile (bf16, 16 KB) and the fp32 operand
-//     block (16 x 64) of a stage with 16-byte cp.async copies, four stages
-//     ahead, into the canonical no-swizzle UMMA layout (8 x 16-byte core
-//     matrices);
-//   * at consume time the fp32 operand block is split into two bf16 blocks,
-//     hi = bf16(v) and lo = bf16(v - hi), so hi + lo carries 16 significant
-//     bits of every activation: D = W (X_hi + X_lo) is fp32-accurate to about
-//     2^-16 relative instead of the 2^-9 of one bf16 rounding;
+//   * all threads stage the weight tile (bf16, 16 KB) and the operand blocks
+//     (16 x 64, hi and lo) of a stage with 16-byte cp.async copies, six stages
+//     ahead, straight into the canonical no-swizzle UMMA layout (8 x 16-byte
+//     core matrices); each thread keeps the pointers of its 8 weight rows for
+//     the unit (rowdot) or the chunk (rowaxpy);
 //   * thread 0 issues the MMAs (tcgen05.mma kind::f16, bf16 inputs, fp32
 //     accumulator in tensor memory, 32 TMEM columns) and commits them to the
 //     stage's mbarrier, which frees the stage for its next copies;
@@ -41,16 +44,12 @@ namespace dv {
 
 constexpr int TC_THREADS = 128;
 constexpr int TC_K = 64;        // K elements per stage
-constexpr int TC_STAGES = 6;
+constexpr int TC_STAGES = 8;
 constexpr int TC_DIST = TC_STAGES - 2;  // stages in flight ahead of the one consumed
-constexpr int TC_A_BYTES = TC_M * TC_K * 2;       // 16 KB weight tile
-constexpr int TC_B_BYTES = TC_N * TC_K * 2;       // 2 KB bf16 operand (hi or lo)
-constexpr int TC_S_BYTES = TC_N * TC_K * 4;       // 4 KB fp32 operand staging
-constexpr int TC_STAGE_BYTES = TC_A_BYTES + 2 * TC_B_BYTES + TC_S_BYTES;
-// Slack after the last stage: every descriptor's reach stays inside the
-// allocation even if its two strides were read the other way round.
-constexpr int TC_SLACK = 32 * 1024;
-constexpr size_t TC_SMEM = 1024 + (size_t)TC_STAGES * TC_STAGE_BYTES + TC_SLACK;
+constexpr int TC_A_BYTES = TC_M * TC_K * 2;  // 16 KB weight tile
+constexpr int TC_B_BYTES = TC_N * TC_K * 2;  // 2 KB bf16 operand (hi or lo)
+constexpr int TC_STAGE_BYTES = TC_A_BYTES + 2 * TC_B_BYTES;
+constexpr size_t TC_SMEM = 1024 + (size_t)TC_STAGES * TC_STAGE_BYTES;
 constexpr int TC_TMEM_COLS = 32;
 constexpr int TC_TILES_PER_GROUP = 8;  // rowdot tiles per rowaxpy unit of the MLP (1024 neurons), at most
 constexpr int TC_HEADS_PER_GROUP = 4;  // heads per rowaxpy unit of W^O, at most
@@ -181,7 +180,6 @@ __host__ __device__ constexpr uint32_t tc_idesc(int M, int N, int a_mn) {
 //   A    [0, 16 KB)      weight tile, canonical no-swizzle layout
 //   Bhi  [16, 18 KB)     operand hi part, [n/8][k/8][n%8][k%8] (K-major)
 //   Blo  [18, 20 KB)     operand lo part
-//   S    [20, 24 KB)     fp32 operand staging, [n][64]
 //
 // rowdot A (K-major, 128 rows x 64 K): byte (m/8)*1024 + (k/8)*128 +
 // (m%8)*16 + (k%8)*2, so lbo = 128, sbo = 1024, and the K = 16 slice kk of
@@ -193,54 +191,56 @@ __host__ __device__ constexpr uint32_t tc_idesc(int M, int N, int a_mn) {
 // lbo = 128, sbo = 1024, slice kk at kk * 256.
 constexpr int TC_OFF_BHI = TC_A_BYTES;
 constexpr int TC_OFF_BLO = TC_A_BYTES + TC_B_BYTES;
-constexpr int TC_OFF_S = TC_A_BYTES + 2 * TC_B_BYTES;
 
-// Splits the stage's fp32 staging block into the hi / lo bf16 operand
-// blocks. Each thread converts exactly the pieces it copied itself
-// (tc_stage_operand: batch rows t/16 and t/16 + 8, 16-byte piece t%16), so
-// its own cp.async wait is all the ordering the conversion needs.
-__device__ __forceinline__ void tc_split_operand(unsigned char* stage) {
+// Copies the stage's operand blocks: batch row n (< nb, zero otherwise),
+// elements k0 .. k0+63 of hi[n * ld] and lo[n * ld], the first `valid` of
+// them (the rest zero; valid is a multiple of 8 or the tail of the row).
+// Thread t copies row t/8, 16-byte piece t%8, of both.
+__device__ __forceinline__ void tc_load_operand(unsigned char* stage, const __nv_bfloat16* hi,
+                                                const __nv_bfloat16* lo, long long ld, int nb, int k0, int valid) {
   const int t = threadIdx.x;
-  const int q = t & 15;
+  const int n = t >> 3, k8 = t & 7;
+  const bool ok = n < nb && k8 * 8 < valid;
+  const long long off = ok ? (long long)n * ld + k0 + k8 * 8 : 0;
+  const int dst = (n >> 3) * 1024 + k8 * 128 + (n & 7) * 16;
+  cp_async16_zfill(stage + TC_OFF_BHI + dst, hi + off, ok ? 16 : 0);
+  cp_async16_zfill(stage + TC_OFF_BLO + dst, lo + off, ok ? 16 : 0);
+}
+
+// This thread's 8 rows of a tile (pointers; null: a zero row). rowdot:
+// piece j of thread t is tile row (t%8) + 8 (t/64) + 16 j, column piece
+// (t/8)%8; rowaxpy: chunk row (t%8) + 8 j, column piece (t/8)%16.
+__device__ __forceinline__ int tc_rowdot_row(int j) { return (threadIdx.x & 7) + 8 * (threadIdx.x >> 6) + 16 * j; }
+__device__ __forceinline__ int tc_rowaxpy_row(int j) { return (threadIdx.x & 7) + 8 * j; }
+
+// rowdot weight tile, K-major: columns k0 .. k0+63 of the 8 rows rp[j]
+// (columns >= d zero).
+__device__ __forceinline__ void tc_load_tile_kmajor(unsigned char* stage, const __nv_bfloat16* const (&rp)[8], int k0,
+                                                    int d, const void* dummy) {
+  const int t = threadIdx.x;
+  const int k8 = (t >> 3) & 7;
+  const int col = k0 + k8 * 8;
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int n = (t >> 4) + 8 * h;
-    const float4 a = *reinterpret_cast<const float4*>(stage + TC_OFF_S + n * 256 + q * 16);
-    const float v[4] = {a.x, a.y, a.z, a.w};
-    uint32_t hi[2], lo[2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * i]), h1 = __float2bfloat16_rn(v[2 * i + 1]);
-      const __nv_bfloat16 l0 = __float2bfloat16_rn(v[2 * i] - __bfloat162float(h0));
-      const __nv_bfloat16 l1 = __float2bfloat16_rn(v[2 * i + 1] - __bfloat162float(h1));
-      hi[i] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-      lo[i] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
-    }
-    // elements k = 4q .. 4q+3 of row n: core matrix k/8 = q/2, bytes (k%8)*2 = (q%2)*8
-    const int off = (n >> 3) * 1024 + (q >> 1) * 128 + (n & 7) * 16 + (q & 1) * 8;
-    *reinterpret_cast<uint2*>(stage + TC_OFF_BHI + off) = make_uint2(hi[0], hi[1]);
-    *reinterpret_cast<uint2*>(stage + TC_OFF_BLO + off) = make_uint2(lo[0], lo[1]);
+  for (int j = 0; j < 8; ++j) {
+    const int m = tc_rowdot_row(j);
+    const bool ok = rp[j] != nullptr && col < d;
+    cp_async16_zfill(stage + (m >> 3) * 1024 + k8 * 128 + (m & 7) * 16, ok ? (const void*)(rp[j] + col) : dummy,
+                     ok ? 16 : 0);
   }
 }
 
-// Stages the fp32 operand block of a stage: batch row n (< nb, zero
-// otherwise), 64 consecutive elements from src + n * ld, the first `valid`
-// of them (the rest zero). Thread t copies rows t/16 and t/16 + 8, 16-byte
-// piece t%16 of each.
-__device__ __forceinline__ void tc_stage_operand(unsigned char* stage, const float* src, long long ld, int nb,
-                                                 int valid) {
+// rowaxpy weight tile, MN-major: columns col0 .. col0+127 of the 8 rows rp[j]
+// (columns >= d zero).
+__device__ __forceinline__ void tc_load_tile_mnmajor(unsigned char* stage, const __nv_bfloat16* const (&rp)[8],
+                                                     int col0, int d, const void* dummy) {
   const int t = threadIdx.x;
-  const int q = t & 15;
+  const int c8 = (t >> 3) & 15;
+  const int col = col0 + c8 * 8;
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int n = (t >> 4) + 8 * h;
-    int bytes = 0;
-    if (n < nb) {
-      const int rem = valid - q * 4;
-      bytes = rem >= 4 ? 16 : (rem > 0 ? rem * 4 : 0);
-    }
-    const float* p = bytes ? src + (long long)n * ld + q * 4 : src;
-    cp_async16_zfill(stage + TC_OFF_S + n * 256 + q * 16, p, bytes);
+  for (int j = 0; j < 8; ++j) {
+    const bool ok = rp[j] != nullptr && col < d;
+    cp_async16_zfill(stage + j * 2048 + c8 * 128 + (t & 7) * 16, ok ? (const void*)(rp[j] + col) : dummy,
+                     ok ? 16 : 0);
   }
 }
 
@@ -250,10 +250,12 @@ __device__ __forceinline__ void tc_stage_operand(unsigned char* stage, const flo
 //
 // A problem P provides:
 //   static constexpr int kAMajorMN;               // 0 rowdot, 1 rowaxpy
+//   static constexpr bool kRowsPerUnit;           // rows() depends on the unit only
 //   __device__ int units() const;                 // work units in total
 //   __device__ int chunks(int unit) const;        // stages of K in a unit (>= 1 for every unit)
 //   __device__ bool live(int unit, int c) const;  // false: the stage is empty (no copies, no MMA)
-//   __device__ void load(unsigned char* stage, int unit, int c) const;   // issue the stage's copies
+//   __device__ void rows(int unit, int c, const bf16* (&rp)[8]) const;  // this thread's 8 weight rows
+//   __device__ void load(unsigned char* stage, int unit, int c, const bf16* const (&rp)[8]) const;
 //   __device__ void epilogue(int unit, int m, const float (&v)[16], bool any) const;
 // The epilogue is called by all 128 threads together (it may use
 // __syncthreads); thread m holds accumulator row m. `any` is false when the
@@ -294,6 +296,7 @@ __device__ void tc_run(const P& p, int* status) {
   const int nunits = p.units();
   int prod_u = blockIdx.x, prod_c = 0;
   int issued = 0;
+  const __nv_bfloat16* rp[8];
   auto produce = [&]() {
     if (prod_u < nunits) {
       const int s = issued % TC_STAGES;
@@ -301,7 +304,10 @@ __device__ void tc_run(const P& p, int* status) {
         if (!abort_local) raise_status(status, DV_DEV_TIMEOUT_BIT);
         abort_local = 1;
       }
-      if (!abort_local && p.live(prod_u, prod_c)) p.load(smem + (size_t)s * TC_STAGE_BYTES, prod_u, prod_c);
+      if (!abort_local && p.live(prod_u, prod_c)) {
+        if (!P::kRowsPerUnit || prod_c == 0) p.rows(prod_u, prod_c, rp);
+        p.load(smem + (size_t)s * TC_STAGE_BYTES, prod_u, prod_c, rp);
+      }
       if (++prod_c >= p.chunks(prod_u)) {
         prod_c = 0;
         prod_u += gridDim.x;
@@ -321,7 +327,6 @@ __device__ void tc_run(const P& p, int* status) {
     const int s = consumed % TC_STAGES;
     unsigned char* stage = smem + (size_t)s * TC_STAGE_BYTES;
     const bool live = p.live(u, c);
-    if (live) tc_split_operand(stage);
     fence_proxy_async_smem();
     tc_fence_before();
     if (__syncthreads_or(abort_local)) break;
@@ -376,44 +381,27 @@ __device__ void tc_run(const P& p, int* status) {
 }
 
 // ---------------------------------------------------------------------------
-// Weight tiles
+// Activations split into bf16 hi / lo rows: hi[b][j] = bf16(x), lo[b][j] =
+// bf16(x - hi) for b < nb, zero for nb <= b < 16; x = src[b * ld + j].
 // ---------------------------------------------------------------------------
+struct TcSplitArgs {
+  const float* src;
+  int nb, n;
+  long long ld_src;
+  __nv_bfloat16* hi;
+  __nv_bfloat16* lo;
+  long long ld_dst;
+};
 
-// rowdot tile: 128 rows (row_of(m): pointer to row m, or null for a zero
-// row) x 64 columns from k0 (columns >= d zero). Thread t copies pieces
-// i = t + 128 j, j < 8: row (i % 8) + 8 (i / 64), 16-byte column piece
-// (i / 8) % 8, so eight consecutive threads fill one 128-byte core matrix.
-template <class RowOf>
-__device__ __forceinline__ void tc_load_rows_kmajor(unsigned char* stage, const RowOf& row_of, int k0, int d,
-                                                    const void* dummy) {
-  const int t = threadIdx.x;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int i = t + 128 * j;
-    const int m = (i & 7) + 8 * (i >> 6), k8 = (i >> 3) & 7;
-    const int col = k0 + k8 * 8;
-    const __nv_bfloat16* r = row_of(m);
-    const bool ok = r != nullptr && col < d;
-    cp_async16_zfill(stage + (m >> 3) * 1024 + k8 * 128 + (m & 7) * 16, ok ? (const void*)(r + col) : dummy,
-                     ok ? 16 : 0);
-  }
-}
-
-// rowaxpy tile: 64 rows (row_of(j), null for zero) x 128 columns from col0
-// (columns >= d zero), MN-major. Thread t copies pieces i = t + 128 j, j < 8:
-// row (i % 8) + 8 (i / 128), 16-byte column piece (i / 8) % 16.
-template <class RowOf>
-__device__ __forceinline__ void tc_load_rows_mnmajor(unsigned char* stage, const RowOf& row_of, int col0, int d,
-                                                     const void* dummy) {
-  const int t = threadIdx.x;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int i = t + 128 * j;
-    const int kr = (i & 7) + 8 * j, c8 = (i >> 3) & 15;
-    const int col = col0 + c8 * 8;
-    const __nv_bfloat16* r = row_of(kr);
-    const bool ok = r != nullptr && col < d;
-    cp_async16_zfill(stage + j * 2048 + c8 * 128 + (i & 7) * 16, ok ? (const void*)(r + col) : dummy, ok ? 16 : 0);
+__global__ void __launch_bounds__(256) tc_split_kernel(TcSplitArgs a) {
+  griddep_launch();
+  griddep_wait();
+  const int b = blockIdx.y;
+  for (int j = blockIdx.x * 256 + threadIdx.x; j < a.n; j += gridDim.x * 256) {
+    const float x = b < a.nb ? a.src[(size_t)b * a.ld_src + j] : 0.f;
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    a.hi[(size_t)b * a.ld_dst + j] = h;
+    a.lo[(size_t)b * a.ld_dst + j] = __float2bfloat16_rn(x - __bfloat162float(h));
   }
 }
 
@@ -421,25 +409,30 @@ __device__ __forceinline__ void tc_load_rows_mnmajor(unsigned char* stage, const
 // q, k, v of the selected heads (rowdot over Wqkv rows)
 // ---------------------------------------------------------------------------
 
-
 struct TcQkvProblem {
   static constexpr int kAMajorMN = 0;
+  static constexpr bool kRowsPerUnit = true;
   TcQkvArgs a;
   int nslots;  // selected heads x 3 dh
   __device__ int units() const { return (nslots + TC_M - 1) / TC_M; }
   __device__ int chunks(int) const { return (a.d + TC_K - 1) / TC_K; }
   __device__ bool live(int, int) const { return true; }
-  __device__ const __nv_bfloat16* row(int s) const {
-    if (s >= nslots) return nullptr;
+  __device__ void rows(int unit, int, const __nv_bfloat16* (&rp)[8]) const {
     const int per = 3 * a.dh;
-    const int head = a.head_idx[s / per];
-    if (head < 0 || head >= a.h) return nullptr;
-    return a.Wqkv + ((size_t)head * per + s % per) * a.d;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int s = unit * TC_M + tc_rowdot_row(j);
+      const __nv_bfloat16* r = nullptr;
+      if (s < nslots) {
+        const int head = a.head_idx[s / per];
+        if (head >= 0 && head < a.h) r = a.Wqkv + ((size_t)head * per + s % per) * a.d;
+      }
+      rp[j] = r;
+    }
   }
-  __device__ void load(unsigned char* stage, int unit, int c) const {
-    const int base = unit * TC_M;
-    tc_load_rows_kmajor(stage, [&](int m) { return row(base + m); }, c * TC_K, a.d, a.Wqkv);
-    tc_stage_operand(stage, a.y + c * TC_K, a.d, a.nb, a.d - c * TC_K);
+  __device__ void load(unsigned char* stage, int, int c, const __nv_bfloat16* const (&rp)[8]) const {
+    tc_load_tile_kmajor(stage, rp, c * TC_K, a.d, a.Wqkv);
+    tc_load_operand(stage, a.xhi, a.xlo, a.d, a.nb, c * TC_K, a.d - c * TC_K);
   }
   __device__ void epilogue(int unit, int m, const float (&v)[16], bool) const {
     const int per = 3 * a.dh;
@@ -480,10 +473,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_qkv_kernel(TcQkvArgs a) {
 
 // ---------------------------------------------------------------------------
 // The MLP: activations of the selected neurons (rowdot over W1 rows, with
-// bias, ReLU and per-tile compaction of the nonzero ones), then the
-// gather-axpy of their W2 rows (rowaxpy)
+// bias, activation and per-tile compaction of the nonzero ones, written as
+// hi / lo bf16 rows), then the gather-axpy of their W2 rows (rowaxpy)
 // ---------------------------------------------------------------------------
-
 
 __device__ __forceinline__ int tc_clamped_count(const int32_t* count, int bound, int* status) {
   int c = *count;
@@ -496,21 +488,24 @@ __device__ __forceinline__ int tc_clamped_count(const int32_t* count, int bound,
 
 struct TcW1Problem {
   static constexpr int kAMajorMN = 0;
+  static constexpr bool kRowsPerUnit = true;
   TcMlpArgs a;
   int cnt;
-  int* s_warp;  // [5] shared: per-warp nonzero counts
+  int* s_warp;  // [4] shared: per-warp nonzero counts
   __device__ int units() const { return (cnt + TC_M - 1) / TC_M; }
   __device__ int chunks(int) const { return (a.d + TC_K - 1) / TC_K; }
   __device__ bool live(int, int) const { return true; }
-  __device__ const __nv_bfloat16* row(int s) const {
-    if (s >= cnt) return nullptr;
-    const int r = a.idx[s];
-    return (r >= 0 && r < a.N) ? a.W1t + (size_t)r * a.d : nullptr;
+  __device__ void rows(int unit, int, const __nv_bfloat16* (&rp)[8]) const {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int s = unit * TC_M + tc_rowdot_row(j);
+      const int r = s < cnt ? a.idx[s] : -1;
+      rp[j] = (r >= 0 && r < a.N) ? a.W1t + (size_t)r * a.d : nullptr;
+    }
   }
-  __device__ void load(unsigned char* stage, int unit, int c) const {
-    const int base = unit * TC_M;
-    tc_load_rows_kmajor(stage, [&](int m) { return row(base + m); }, c * TC_K, a.d, a.W1t);
-    tc_stage_operand(stage, a.y + c * TC_K, a.d, a.nb, a.d - c * TC_K);
+  __device__ void load(unsigned char* stage, int, int c, const __nv_bfloat16* const (&rp)[8]) const {
+    tc_load_tile_kmajor(stage, rp, c * TC_K, a.d, a.W1t);
+    tc_load_operand(stage, a.xhi, a.xlo, a.d, a.nb, c * TC_K, a.d - c * TC_K);
   }
   __device__ void epilogue(int unit, int m, const float (&v)[16], bool) const {
     const int s = unit * TC_M + m;
@@ -539,13 +534,26 @@ struct TcW1Problem {
       total += n;
     }
     const int base = unit * TC_M;
-    if (nz) {
-      const int pos = before + __popc(bal & ((1u << lane) - 1u));
-      for (int b = 0; b < a.nb; ++b) a.act_c[(size_t)b * a.KC + base + pos] = act[b];
-      a.rowid_c[base + pos] = r;
+    if (nz) {  // the nonzero activations at their compacted slot
+      const int slot = before + __popc(bal & ((1u << lane) - 1u));
+#pragma unroll
+      for (int b = 0; b < TC_N; ++b) {
+        if (b >= a.nb) break;
+        const __nv_bfloat16 h = __float2bfloat16_rn(act[b]);
+        a.act_hi[(size_t)b * a.KC + base + slot] = h;
+        a.act_lo[(size_t)b * a.KC + base + slot] = __float2bfloat16_rn(act[b] - __bfloat162float(h));
+      }
+      a.rowid_c[base + slot] = r;
     }
-    if (m >= total)  // the slots after the tile's count hold zero activations
-      for (int b = 0; b < a.nb; ++b) a.act_c[(size_t)b * a.KC + base + m] = 0.f;
+    if (m >= total) {  // zeros after the tile's count (the W2 operand reads 8-slot pieces)
+      const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
+#pragma unroll
+      for (int b = 0; b < TC_N; ++b) {
+        if (b >= a.nb) break;
+        a.act_hi[(size_t)b * a.KC + base + m] = z;
+        a.act_lo[(size_t)b * a.KC + base + m] = z;
+      }
+    }
     if (threadIdx.x == 0) a.tile_cnt[unit] = total;
     __syncthreads();  // s_warp is reused by the next unit
   }
@@ -561,6 +569,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_w1_kernel(TcMlpArgs a) {
 
 struct TcW2Problem {
   static constexpr int kAMajorMN = 1;
+  static constexpr bool kRowsPerUnit = false;
   TcMlpArgs a;
   int ntiles, n_mt, n_groups;
   const int* s_cnt;  // shared: tile_cnt of every tile
@@ -578,17 +587,22 @@ struct TcW2Problem {
     if ((c >> 1) >= tiles_in(g)) return false;
     return s_cnt[g * a.tiles_per_group + (c >> 1)] > (c & 1) * 64;
   }
-  __device__ void load(unsigned char* stage, int unit, int c) const {
-    const int g = unit / n_mt, mt = unit % n_mt;
-    const int t = g * a.tiles_per_group + (c >> 1), half = c & 1;
-    const int n = s_cnt[t] - half * 64;  // > 0 (live)
+  __device__ void rows(int unit, int c, const __nv_bfloat16* (&rp)[8]) const {
+    const int t = (unit / n_mt) * a.tiles_per_group + (c >> 1), half = c & 1;
+    const int n = s_cnt[t] - half * 64;
     const int base = t * TC_M + half * 64;
-    tc_load_rows_mnmajor(stage,
-                         [&](int j) -> const __nv_bfloat16* {
-                           return j < n ? a.W2t + (size_t)a.rowid_c[base + j] * a.d : nullptr;
-                         },
-                         mt * TC_M, a.d, a.W2t);
-    tc_stage_operand(stage, a.act_c + base, a.KC, a.nb, n < 64 ? n : 64);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int kr = tc_rowaxpy_row(j);
+      rp[j] = kr < n ? a.W2t + (size_t)a.rowid_c[base + kr] * a.d : nullptr;
+    }
+  }
+  __device__ void load(unsigned char* stage, int unit, int c, const __nv_bfloat16* const (&rp)[8]) const {
+    const int t = (unit / n_mt) * a.tiles_per_group + (c >> 1), half = c & 1;
+    const int n = s_cnt[t] - half * 64;  // > 0 (live)
+    tc_load_tile_mnmajor(stage, rp, (unit % n_mt) * TC_M, a.d, a.W2t);
+    const int valid = n < 64 ? (n + 7) & ~7 : 64;  // the slots after the count hold zeros
+    tc_load_operand(stage, a.act_hi, a.act_lo, a.KC, a.nb, t * TC_M + half * 64, valid);
   }
   __device__ void epilogue(int unit, int m, const float (&v)[16], bool any) const {
     const int g = unit / n_mt, mt = unit % n_mt;
@@ -622,12 +636,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_w2_kernel(TcMlpArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// W^O of the selected heads (rowaxpy over WOt rows; operand H)
+// W^O of the selected heads (rowaxpy over WOt rows; operand H as hi / lo)
 // ---------------------------------------------------------------------------
-
 
 struct TcWoProblem {
   static constexpr int kAMajorMN = 1;
+  static constexpr bool kRowsPerUnit = false;
   TcWoArgs a;
   int hc, n_mt, n_groups, cph;  // cph: 64-row chunks per head
   __device__ int units() const { return n_mt * n_groups; }
@@ -640,15 +654,18 @@ struct TcWoProblem {
     return n > 0 ? n : 1;
   }
   __device__ bool live(int unit, int c) const { return c / cph < heads_in(unit / n_mt); }
-  __device__ void load(unsigned char* stage, int unit, int c) const {
-    const int g = unit / n_mt, mt = unit % n_mt;
-    const int p = g * a.heads_per_group + c / cph, part = c % cph;
+  __device__ void rows(int unit, int c, const __nv_bfloat16* (&rp)[8]) const {
+    const int p = (unit / n_mt) * a.heads_per_group + c / cph, part = c % cph;
     const int head = a.head_idx[p];
     const bool ok = head >= 0 && head < a.h;
-    const __nv_bfloat16* rows = a.WOt + ((size_t)(ok ? head : 0) * a.dh + part * 64) * a.d;
-    tc_load_rows_mnmajor(stage, [&](int j) -> const __nv_bfloat16* { return ok ? rows + (size_t)j * a.d : nullptr; },
-                         mt * TC_M, a.d, a.WOt);
-    tc_stage_operand(stage, a.H + (size_t)p * a.dh + part * 64, (long long)a.kh_max * a.dh, a.nb, ok ? 64 : 0);
+    const __nv_bfloat16* rows0 = a.WOt + ((size_t)(ok ? head : 0) * a.dh + part * 64) * a.d;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) rp[j] = ok ? rows0 + (size_t)tc_rowaxpy_row(j) * a.d : nullptr;
+  }
+  __device__ void load(unsigned char* stage, int unit, int c, const __nv_bfloat16* const (&rp)[8]) const {
+    const int p = (unit / n_mt) * a.heads_per_group + c / cph, part = c % cph;
+    tc_load_tile_mnmajor(stage, rp, (unit % n_mt) * TC_M, a.d, a.WOt);
+    tc_load_operand(stage, a.hhi, a.hlo, (long long)a.kh_max * a.dh, a.nb, p * a.dh + part * 64, 64);
   }
   __device__ void epilogue(int unit, int m, const float (&v)[16], bool any) const {
     const int g = unit / n_mt, mt = unit % n_mt;

@@ -16,7 +16,8 @@ constexpr int DV_DEV_TIMEOUT_BIT = 8;  // device status bit: a bounded wait ran 
 struct TcQkvArgs {
   const __nv_bfloat16* Wqkv;  // [h][3][dh][d]
   const float* bqkv;          // [h][3][dh] or null
-  const float* y;             // [nb][d] normalised input
+  const __nv_bfloat16* xhi;   // [16][d] normalised input, hi part (rows >= nb zero)
+  const __nv_bfloat16* xlo;   // [16][d] lo part
   const int32_t* head_idx;
   const int32_t* head_count;
   int kh_max, h, dh, d, nb, cap, pos;
@@ -31,13 +32,15 @@ struct TcMlpArgs {
   const float* b1;           // [N]
   const __nv_bfloat16* W2t;  // [N][d]
   const float* b2;           // [d] or null
-  const float* y;            // [nb][d]
+  const __nv_bfloat16* xhi;  // [16][d] normalised input, hi part
+  const __nv_bfloat16* xlo;  // [16][d] lo part
   const int32_t* idx;
   const int32_t* count;
   int k_max, d, N, nb;
   int KC;                    // slots per batch row of act_c: tiles_max x 128
   int tiles_per_group;       // rowdot tiles per rowaxpy unit
-  float* act_c;              // [16][KC] activations, compacted per tile
+  __nv_bfloat16* act_hi;     // [16][KC] activations compacted per tile, hi part
+  __nv_bfloat16* act_lo;     // [16][KC] lo part
   int32_t* rowid_c;          // [KC] the neuron of each compacted slot
   int32_t* tile_cnt;         // [tiles_max] nonzero neurons per tile
   float* out;                // [nb][d], accumulated into
@@ -48,7 +51,8 @@ struct TcMlpArgs {
 struct TcWoArgs {
   const __nv_bfloat16* WOt;  // [h][dh][d]
   const float* bO;           // [d] or null
-  const float* H;            // [nb][kh_max][dh]
+  const __nv_bfloat16* hhi;  // [16][kh_max dh] attention outputs H, hi part
+  const __nv_bfloat16* hlo;  // lo part
   const int32_t* head_idx;
   const int32_t* head_count;
   int kh_max, h, dh, d, nb;

@@ -13,6 +13,9 @@ bool tc_shape_ok(int B, int wbytes, int dh, int k_max);
 // Tiles of 128 selected neurons for a bound of k_max.
 int tc_tiles(int k_max);
 
+// hi / lo bf16 rows [16][ld_dst] of x [nb][n] (row stride ld_src); rows >= nb zero.
+cudaError_t run_tc_split(const float* x, int nb, int n, long long ld_src, __nv_bfloat16* hi, __nv_bfloat16* lo,
+                         long long ld_dst, cudaStream_t st);
 cudaError_t run_tc_qkv(const TcQkvArgs& a, cudaStream_t st);
 // W1 + bias + ReLU with per-tile compaction, then the W2 gather-axpy into out.
 cudaError_t run_tc_mlp(TcMlpArgs a, cudaStream_t st);
