@@ -20,15 +20,14 @@ namespace {
 constexpr int ATTN_S_MIN = 32;
 // Every layout starts with the same fixed header that holds the counters, so
 // calls of different operations may share one workspace: the status word at
-// 0, the selection tickets at 16, 32, 48 and 64, the attention split counters
-// [B][kh_max] from 1024, and the neuron-score histograms from 64 KB.
-constexpr size_t WS_HEADER = 192 * 1024;
-constexpr size_t WS_HIST = 64 * 1024;  // [16][2048] digit histograms of the fused neuron predictor
+// 0, the selection tickets at 16, 32, 48 and 64, and the attention split
+// counters [B][kh_max] from 1024.
+constexpr size_t WS_HEADER = 72 * 1024;
 constexpr int KH_LIMIT = 1000;  // B * kh_max counters must fit the header
 
 // Workspace layout. Offsets in bytes from the workspace base.
 struct Layout {
-  size_t status, sel_ticket_h, sel_ticket_m, pa_ticket, pb_ticket, attn_ctr, hist, t1;
+  size_t status, sel_ticket_h, sel_ticket_m, pa_ticket, pb_ticket, attn_ctr, t1;
   size_t yA, yM, z, scores_h, bm_h, head_idx, head_count, scores, bm_m, idx, count;
   size_t q, part, H, seg_idx, seg_a, seg_cnt, tc_x, tc_act, tc_rowid, tc_tiles, total;
   int nseg, SEG, nsplit_max, KC, XC;
@@ -55,7 +54,6 @@ Layout layout(const dv_dims& D, int wbytes) {
   L.pa_ticket = L.status + 48;
   L.pb_ticket = L.status + 64;
   L.attn_ctr = L.status + 1024;
-  L.hist = L.status + WS_HIST;
   L.t1 = take(4ull * B * D.d);
   L.yA = take(4ull * B * D.d);
   L.yM = take(4ull * B * D.d);
@@ -108,7 +106,7 @@ dv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DV_OK : DV_ERR_
   } while (0)
 
 // Tensor-core path for batch 5..16 (defined below)
-bool tc_ok(int B, dv_dtype wdt, int dh, int k_max);
+bool tc_ok(int B, int d, dv_dtype wdt, int dh, int k_max);
 dv_status tc_mlp(const Layout& L, void* ws, const float* y, int B, int d, int N, const void* W1t, const float* b1,
                  const void* W2t, const float* b2, const int32_t* idx, const int32_t* count, int k_max, float* out,
                  int act, cudaStream_t st);
@@ -166,7 +164,7 @@ dv_status do_sparse_mlp(const Layout& L, void* ws, const float* y, int B, int d,
                         const float* b1, const void* W2t, const float* b2, dv_dtype dt, const int32_t* idx,
                         const int32_t* count, int k_max, float* out, int accumulate, int act, cudaStream_t st) {
   if (!accumulate) DV_TRY(cudaMemsetAsync(out, 0, 4ull * B * d, st));
-  if (tc_ok(B, dt, 64, k_max)) return tc_mlp(L, ws, y, B, d, N, W1t, b1, W2t, b2, idx, count, k_max, out, act, st);
+  if (tc_ok(B, d, dt, 64, k_max)) return tc_mlp(L, ws, y, B, d, N, W1t, b1, W2t, b2, idx, count, k_max, out, act, st);
   int* status = at<int>(ws, L.status);
   int32_t* seg_idx = at<int32_t>(ws, L.seg_idx);
   float* seg_a = at<float>(ws, L.seg_a);
@@ -190,7 +188,7 @@ dv_status do_sparse_mha(const Layout& L, void* ws, const float* y, int B, int d,
                         float* out, int accumulate, cudaStream_t st) {
   if (!accumulate) DV_TRY(cudaMemsetAsync(out, 0, 4ull * B * d, st));
   int* status = at<int>(ws, L.status);
-  if (tc_ok(B, dt, dh, 0)) {
+  if (tc_ok(B, d, dt, dh, 0)) {
     if (kh_max > 0) {
       DV_CHECK(tc_qkv(L, ws, y, B, d, h, dh, Wqkv, bqkv, Kc, Vc, cap, pos, head_idx, head_count, kh_max, st));
       DV_TRY(run_attn_dt(dt, dh, at<float>(ws, L.q), Kc, Vc, B, h, cap, pos, scale, head_idx, head_count, kh_max,
@@ -237,8 +235,11 @@ bool tc_enabled() {
   return on;
 }
 
-bool tc_ok(int B, dv_dtype wdt, int dh, int k_max) {
-  return tc_enabled() && B >= TC_MIN_B && tc_shape_ok(B, wbytes_of(wdt), dh > 0 ? dh : 64, k_max);
+// Batch 5-16, and batch 3-4 when the rows are too long for the column-owner
+// kernels (d > 4096 bf16), where the CUDA-core row kernels would take them.
+bool tc_ok(int B, int d, dv_dtype wdt, int dh, int k_max) {
+  const bool batch = B >= TC_MIN_B || (B >= 3 && !co_ok(B, d, 8));
+  return tc_enabled() && batch && tc_shape_ok(B, wbytes_of(wdt), dh > 0 ? dh : 64, k_max);
 }
 
 dv_status tc_mlp(const Layout& L, void* ws, const float* y, int B, int d, int N, const void* W1t, const float* b1,
@@ -336,7 +337,7 @@ bool fused_enabled() {
 // the normalised input and the K/V tiles within shared memory.
 bool fused_ok(const dv_dims& D, dv_dtype wdt) {
   if (!fused_enabled()) return false;
-  if (tc_ok(D.B, wdt, D.dh, D.k_max)) return false;  // batch 5..16, bf16: tensor-core kernels
+  if (tc_ok(D.B, D.d, wdt, D.dh, D.k_max)) return false;  // batch 5..16, bf16: tensor-core kernels
   const int wb = wbytes_of(wdt), E = 16 / wb;
   if (D.d % (ATTN_CS * E) != 0) return false;
   if ((size_t)D.B * D.d * 4 > 160 * 1024) return false;
@@ -359,34 +360,24 @@ dv_status fused_predict_rest(const Layout& L, void* ws, const dv_layer_weights* 
     b.N = D.N;
     b.r = D.r;
     b.nb = D.B;
-    b.hist_mode = 0;
     b.scores = sm;
-    b.hist = at<unsigned>(ws, L.hist);
     DV_TRY(run_predict_b_dt(w->wdtype, b, st));
     DV_TRY(select_any(sm, D.B, D.N, p->k, p->tau, p->mode, at<uint32_t>(ws, L.bm_m), at<unsigned>(ws, L.pb_ticket),
                       midx, mcnt, st));
   }
   if (heads) {
-    SelectFinishArgs f = {};
-    f.neuron_rows = 0;
-    f.nb = D.B;
-    f.scores_h = sh;
-    f.h = D.h;
-    f.k_h = p->k_h;
-    f.mode_h = p->mode_h;
-    f.tau_h = p->tau_h;
-    f.head_idx = hidx;
-    f.head_count = hcnt;
+    SelectHeadsArgs f{sh, D.B, D.h, p->k_h, p->mode_h, p->tau_h, hidx, hcnt};
     const size_t smem = 4ull * D.h;
-    DV_TRY(allow_smem(select_finish_kernel, smem));
-    DV_TRY(launch(select_finish_kernel, dim3(1), dim3(SEL_THREADS), smem, st, f));
+    DV_TRY(allow_smem(select_heads_kernel, smem));
+    DV_TRY(launch(select_heads_kernel, dim3(1), dim3(SEL_THREADS), smem, st, f));
   }
   return DV_OK;
 }
 
 // The head set (heads) and/or the neuron set (neurons) predicted from y:
-// predict_a (head scores, z = y A), predict_b (neuron scores + first digit
-// histogram), select_finish (exact top-k / threshold of both).
+// predict_a (head scores, z = y A), predict_b (neuron scores), then the exact
+// top-k / threshold selections (select_rows_kernel for the neurons,
+// select_heads_kernel for the heads).
 dv_status fused_predict(const Layout& L, void* ws, const dv_layer_weights* w, const dv_dims& D,
                         const dv_layer_params* p, const float* y, bool heads, bool neurons, float* sh, int32_t* hidx,
                         int32_t* hcnt, float* sm, int32_t* midx, int32_t* mcnt, cudaStream_t st) {
@@ -504,7 +495,7 @@ dv_status layer_begin(const Layout& L, void* ws, const dv_layer_weights* w, cons
     DV_CHECK(do_predict_heads(L, ws, yA, D.B, D.d, D.h, w->PA, w->wdtype, p->k_h, p->tau_h, p->mode_h, r.sh, r.hidx,
                               r.hcnt, st));
   if (D.kh_max > 0) {
-    if (tc_ok(D.B, w->wdtype, D.dh, D.k_max)) {
+    if (tc_ok(D.B, D.d, w->wdtype, D.dh, D.k_max)) {
       DV_CHECK(tc_qkv(L, ws, yA, D.B, D.d, D.h, D.dh, w->Wqkv, w->bqkv, w->Kc, w->Vc, D.cap, pos, r.use_hidx,
                       r.use_hcnt, D.kh_max, st));
     } else {
@@ -577,9 +568,30 @@ dv_status layer_attn(const Layout& L, void* ws, const dv_layer_weights* w, const
     b.sets_ready = sel ? 1 : 0;
     b.scale = p->scale;
     b.status = status;
+    const int E = w->wdtype == DV_BF16 ? 8 : 4;
+    if (w->wdtype == DV_BF16 && wo_split_ok(D.B, D.d, E, wbytes_of(w->kvdtype))) {
+      b.H_out = at<float>(ws, L.H);  // attention only; then the W^O rows over every SM
+      DV_TRY(run_attn_out_dt(w->kvdtype, b, st));
+      WoStreamArgs o = {};
+      o.WOt = w->WOt;
+      o.bO = w->bO;
+      o.H = b.H_out;
+      o.head_idx = r.use_hidx;
+      o.head_count = r.use_hcnt;
+      o.kh_max = D.kh_max;
+      o.h = D.h;
+      o.dh = D.dh;
+      o.d = D.d;
+      o.nb = D.B;
+      o.sets_ready = b.sets_ready;
+      o.x = x;
+      o.t1 = b.t1;
+      o.status = status;
+      return cuda_status(run_wo_stream_dt(w->wdtype, o, st));
+    }
     return cuda_status(run_attn_out_dt(w->kvdtype, b, st));
   }
-  if (tc_ok(D.B, w->wdtype, D.dh, D.k_max)) {
+  if (tc_ok(D.B, D.d, w->wdtype, D.dh, D.k_max)) {
     if (D.kh_max > 0)
       DV_TRY(run_attn_dt(w->kvdtype, D.dh, at<float>(ws, L.q), w->Kc, w->Vc, D.B, D.h, D.cap, pos, p->scale,
                          r.use_hidx, r.use_hcnt, D.kh_max, at<float>(ws, L.part), at<unsigned>(ws, L.attn_ctr),

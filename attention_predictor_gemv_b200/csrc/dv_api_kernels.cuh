@@ -123,354 +123,72 @@ __global__ void __launch_bounds__(256) prefetch_layer_kernel(PrefetchArgs a) {
 }
 
 // ----------------------------------------------------------------------------
-// Exact selection after predict_b_kernel. CTAs 0..B-1 take one neuron score
-// row each (1024 threads, keys in shared memory): the bin of the k-th largest
-// key comes from the global histogram (which this kernel clears), the keys in
-// that bin are collected and refined by two more digit passes, and a
-// warp-ordered pass takes every key above the threshold plus the lowest-index
-// copies of the threshold key. The last neuron CTA unites the rows' bitmaps
-// and writes idx / count. CTA B (when heads are predicted) selects the heads
-// from their scores by rank (few heads: direct comparison).
+// Head selection from the head scores of B rows: the union over the rows of
+// each row's k_h best (ties to the lower index) or of its scores > tau. Few
+// heads (h <= HSEL_MAX): every thread ranks its head by direct comparison
+// with all others. One CTA.
 // ----------------------------------------------------------------------------
-// Boundary-bin keys held in shared memory. They share one array with the
-// digit histogram, which is no longer read once they are written, so that
-// static plus dynamic shared memory stays within 227 KB at N = 49152.
-constexpr int SF_CAND = 4096;
-
-struct SelectFinishArgs {
-  const float* scores;  // [B][N]
-  unsigned* hist;       // [B][2048]
-  uint32_t* bitmaps;    // [B][N/32]
-  unsigned* ticket;
-  int neuron_rows;      // B when the neuron set is selected, else 0
-  int N, nb, k, mode;
-  float tau;
-  int32_t* idx;
-  int32_t* count;
-  const float* scores_h;  // [B][h] or null
-  int h, k_h, mode_h;
+struct SelectHeadsArgs {
+  const float* scores_h;  // [B][h]
+  int nb, h, k_h, mode_h;
   float tau_h;
   int32_t* head_idx;
   int32_t* head_count;
 };
 
-__global__ void __launch_bounds__(SEL_THREADS) select_finish_kernel(SelectFinishArgs a) {
-  extern __shared__ uint32_t s_keys[];  // [N] for a neuron row, [h] for the head row
-  __shared__ uint32_t s_hc[SF_CAND > SEL_BINS ? SF_CAND : SEL_BINS];
-  unsigned* s_h = s_hc;      // [SEL_BINS] digit histogram
-  uint32_t* s_cand = s_hc;   // [SF_CAND] boundary-bin keys (after the top digit is known)
+__global__ void __launch_bounds__(SEL_THREADS) select_heads_kernel(SelectHeadsArgs a) {
+  extern __shared__ uint32_t s_keys[];  // [h]
   __shared__ uint32_t s_hsel[HSEL_MAX / 32];
-  __shared__ uint32_t s_bm[SEL_SMEM_KEYS / 32];
-  __shared__ unsigned sc[SEL_WARPS + 1];
-  __shared__ unsigned s_wcnt[SEL_WARPS];
-  __shared__ unsigned s_digit, s_kk, s_ncand, s_last;
   griddep_launch();
   griddep_wait();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
-  if ((int)blockIdx.x == a.neuron_rows) {
-    // ---- heads: the union over rows of each row's k_h best (or > tau) ----
-    const int h = a.h, nw = (h + 31) >> 5;
-    for (int w = tid; w < nw; w += SEL_THREADS) s_hsel[w] = 0u;
-    for (int b = 0; b < a.nb; ++b) {
-      __syncthreads();
-      for (int i = tid; i < h; i += SEL_THREADS) s_keys[i] = ord_key(a.scores_h[(size_t)b * h + i]);
-      __syncthreads();
-      for (int i = tid; i < h; i += SEL_THREADS) {
-        bool take;
-        if (a.mode_h == 1) {
-          take = a.scores_h[(size_t)b * h + i] > a.tau_h;
-        } else {
-          const uint32_t ki = s_keys[i];
-          int rank = 0;
-          for (int j = 0; j < h; ++j) {
-            const uint32_t kj = s_keys[j];
-            rank += (kj > ki) || (kj == ki && j < i);
-          }
-          take = rank < a.k_h;
-        }
-        if (take) atomicOr(&s_hsel[i >> 5], 1u << (i & 31));
-      }
-    }
+  const int h = a.h, nw = (h + 31) >> 5;
+  for (int w = tid; w < nw; w += SEL_THREADS) s_hsel[w] = 0u;
+  for (int b = 0; b < a.nb; ++b) {
     __syncthreads();
-    if (warp == 0) {
-      unsigned base = 0;
-      for (int w0 = 0; w0 < nw; w0 += 32) {
-        const int w = w0 + lane;
-        const uint32_t u = w < nw ? s_hsel[w] : 0u;
-        const unsigned c = __popc(u);
-        unsigned incl = c;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += t;
+    for (int i = tid; i < h; i += SEL_THREADS) s_keys[i] = ord_key(a.scores_h[(size_t)b * h + i]);
+    __syncthreads();
+    for (int i = tid; i < h; i += SEL_THREADS) {
+      bool take;
+      if (a.mode_h == 1) {
+        take = a.scores_h[(size_t)b * h + i] > a.tau_h;
+      } else {
+        const uint32_t ki = s_keys[i];
+        int rank = 0;
+        for (int j = 0; j < h; ++j) {
+          const uint32_t kj = s_keys[j];
+          rank += (kj > ki) || (kj == ki && j < i);
         }
-        unsigned off = base + incl - c;
-        uint32_t v = u;
-        while (v) {
-          const int jb = __ffs(v) - 1;
-          v &= v - 1u;
-          a.head_idx[off++] = w * 32 + jb;
-        }
-        base += __shfl_sync(0xffffffffu, incl, 31);
+        take = rank < a.k_h;
       }
-      if (lane == 0) *a.head_count = (int32_t)base;
+      if (take) atomicOr(&s_hsel[i >> 5], 1u << (i & 31));
     }
-    return;
   }
-
-  // ---- one neuron score row ----
-  const int b = blockIdx.x, n = a.N;
-  const float* row = a.scores + (size_t)b * n;
-  const int nw = (n + 31) >> 5;
-  uint32_t* bm = a.bitmaps + (size_t)b * nw;
-  const int wpw = (nw + SEL_WARPS - 1) / SEL_WARPS;  // warp w owns the words [w wpw, (w+1) wpw)
-  const int w0 = warp * wpw, w1 = min(nw, w0 + wpw);
-  const unsigned lt = (1u << lane) - 1u;
-  // exclusive offset of this warp's count among the CTA's warps, and the
-  // total: every warp scans the SEL_WARPS counts itself (no second barrier)
-  auto warp_offsets = [&](unsigned& off, unsigned& total) {
-    const unsigned v = s_wcnt[lane];
-    unsigned incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    off = __shfl_sync(0xffffffffu, incl - v, warp);
-    total = __shfl_sync(0xffffffffu, incl, 31);
-  };
-  const bool hist_mode = a.mode == 0 && a.k > 0 && a.k < n;
-  if (!hist_mode) {
-    for (int w = w0; w < w1; ++w) {
-      const int i = w * 32 + lane;
-      const bool take = i < n && (a.mode == 1 ? row[i] > a.tau : a.k > 0);
-      const unsigned word = __ballot_sync(0xffffffffu, take);
-      if (lane == 0) s_bm[w] = word;
-    }
-  } else {
-    unsigned* gh = a.hist + (size_t)b * SEL_BINS;
-    static_assert(SEL_BINS == 2 * SEL_THREADS, "two histogram bins per thread");
-    static_assert(SEL_WARPS == 32, "one count per lane of a warp");
-    const unsigned h0 = gh[tid], h1 = gh[tid + SEL_THREADS];
-    {  // keys into shared memory, 8 loads in flight per thread
-      constexpr int UNR = 8;
-      for (int i0 = tid; i0 < n; i0 += SEL_THREADS * UNR) {
-        float v[UNR];
-#pragma unroll
-        for (int u = 0; u < UNR; ++u) {
-          const int i = i0 + u * SEL_THREADS;
-          v[u] = i < n ? row[i] : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < UNR; ++u) {
-          const int i = i0 + u * SEL_THREADS;
-          if (i < n) s_keys[i] = ord_key(v[u]);
-        }
-      }
-    }
-    s_h[tid] = h0;
-    s_h[tid + SEL_THREADS] = h1;
-    gh[tid] = 0u;  // cleared for the next call
-    gh[tid + SEL_THREADS] = 0u;
-    __syncthreads();
-    // ---- top digit (bits 31..21) of the k-th largest key: warp 0 walks the
-    // histogram from the top, 64 bins per lane ----
-    if (warp == 0) {
-      const int hi = SEL_BINS - 1 - 64 * lane;  // lane's bins hi, hi-1, ..., hi-63
-      unsigned sum = 0u;
-#pragma unroll 8
-      for (int j = 0; j < 64; ++j) sum += s_h[hi - j];
-      unsigned incl = sum;
+  __syncthreads();
+  if (warp == 0) {
+    unsigned base = 0;
+    for (int w0 = 0; w0 < nw; w0 += 32) {
+      const int w = w0 + lane;
+      const uint32_t u = w < nw ? s_hsel[w] : 0u;
+      const unsigned c = __popc(u);
+      unsigned incl = c;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += t;
       }
-      const unsigned kk0 = (unsigned)a.k;
-      if (incl - sum < kk0 && kk0 <= incl) {
-        unsigned acc = incl - sum;
-        for (int j = 0; j < 64; ++j) {
-          const unsigned c = s_h[hi - j];
-          if (acc + c >= kk0) {
-            s_digit = (unsigned)(hi - j);
-            s_kk = kk0 - acc;
-            break;
-          }
-          acc += c;
-        }
+      unsigned off = base + incl - c;
+      uint32_t v = u;
+      while (v) {
+        const int jb = __ffs(v) - 1;
+        v &= v - 1u;
+        a.head_idx[off++] = w * 32 + jb;
       }
+      base += __shfl_sync(0xffffffffu, incl, 31);
     }
-    __syncthreads();
-    uint32_t prefix = s_digit << 21, mask = 0x7ffu << 21;
-    unsigned kk = s_kk;
-    bool take_all_eq = false;
-    // ---- the keys of the boundary bin, compacted in index order ----
-    {
-      unsigned cnt = 0u;
-      for (int w = w0; w < w1; ++w) {
-        const int i = w * 32 + lane;
-        cnt += __popc(__ballot_sync(0xffffffffu, i < n && (s_keys[i] & mask) == prefix));
-      }
-      if (lane == 0) s_wcnt[warp] = cnt;
-    }
-    __syncthreads();
-    unsigned off, nc;
-    warp_offsets(off, nc);
-    if (nc <= SF_CAND) {
-      for (int w = w0; w < w1; ++w) {
-        const int i = w * 32 + lane;
-        const uint32_t key = i < n ? s_keys[i] : 0u;
-        const bool c = i < n && (key & mask) == prefix;
-        const unsigned bal = __ballot_sync(0xffffffffu, c);
-        if (c) s_cand[off + __popc(bal & lt)] = key;
-        off += __popc(bal);
-      }
-      __syncthreads();
-      // ---- warp 0: the kk-th largest candidate by bisection on the low 21
-      // bits (count of candidates >= a trial key, one warp reduction each) ----
-      if (warp == 0) {
-        constexpr int KR = 16;  // candidates per lane held in registers
-        uint32_t ck[KR];
-        const bool in_regs = nc <= 32u * KR;
-#pragma unroll
-        for (int q = 0; q < KR; ++q) {
-          const unsigned i = q * 32u + lane;
-          ck[q] = (in_regs && i < nc) ? s_cand[i] : 0u;
-        }
-        auto count_ge = [&](uint32_t t) {
-          unsigned c = 0u;
-          if (in_regs) {
-#pragma unroll
-            for (int q = 0; q < KR; ++q) c += (q * 32u + lane < nc) && ck[q] >= t;
-          } else {
-            for (unsigned i = lane; i < nc; i += 32u) c += s_cand[i] >= t;
-          }
-          return __reduce_add_sync(0xffffffffu, c);
-        };
-        uint32_t T = prefix;
-#pragma unroll 1
-        for (int bit = 20; bit >= 0; --bit) {
-          const uint32_t t = T | (1u << bit);
-          if (count_ge(t) >= kk) T = t;
-        }
-        // T is the kk-th largest candidate key; c_gt keys above it
-        const unsigned c_ge = count_ge(T), c_gt = (T == 0xffffffffu) ? 0u : count_ge(T + 1u);
-        if (lane == 0) {
-          s_digit = T;
-          s_kk = kk - c_gt;
-          s_ncand = c_ge - c_gt;  // keys equal to T
-        }
-      }
-      __syncthreads();
-      prefix = s_digit;
-      mask = 0xffffffffu;
-      kk = s_kk;
-      take_all_eq = (kk == s_ncand);
-    } else {
-      // many keys in the boundary bin: two more digit passes over all keys
-#pragma unroll 1
-      for (int pass = 1; pass < 3; ++pass) {
-        const int shift = pass == 1 ? 10 : 0;
-        const unsigned dmask = pass == 2 ? 0x3ffu : 0x7ffu;
-        for (int i = tid; i < SEL_BINS; i += SEL_THREADS) s_h[i] = 0u;
-        __syncthreads();
-        for (int i0 = 0; i0 < n; i0 += SEL_THREADS) {
-          const int i = i0 + tid;
-          const uint32_t key = i < n ? s_keys[i] : 0u;
-          const bool in = i < n && (key & mask) == prefix;
-          const unsigned bin = in ? (key >> shift) & dmask : 0xffffffffu;
-          const unsigned peers = __match_any_sync(0xffffffffu, bin);
-          if (in && (__ffs(peers) - 1) == lane) atomicAdd(&s_h[bin], (unsigned)__popc(peers));
-        }
-        __syncthreads();
-        const unsigned c0 = s_h[SEL_BINS - 1 - 2 * tid], c1 = s_h[SEL_BINS - 2 - 2 * tid];
-        unsigned tot;
-        const unsigned above = block_exclusive_scan<SEL_THREADS>(c0 + c1, sc, &tot);
-        if (above < kk && kk <= above + c0 + c1) {
-          if (kk <= above + c0) {
-            s_digit = SEL_BINS - 1 - 2 * tid;
-            s_kk = kk - above;
-          } else {
-            s_digit = SEL_BINS - 2 - 2 * tid;
-            s_kk = kk - above - c0;
-          }
-        }
-        __syncthreads();
-        prefix |= s_digit << shift;
-        mask |= dmask << shift;
-        kk = s_kk;
-      }
-    }
-    // ---- the row's bitmap: keys above the threshold key T = prefix, plus the
-    // kk lowest-index keys equal to it ----
-    if (take_all_eq) {
-      for (int w = w0; w < w1; ++w) {
-        const int i = w * 32 + lane;
-        const unsigned word = __ballot_sync(0xffffffffu, i < n && s_keys[i] >= prefix);
-        if (lane == 0) s_bm[w] = word;
-      }
-    } else {
-      unsigned eq = 0u;
-      for (int w = w0; w < w1; ++w) {
-        const int i = w * 32 + lane;
-        eq += __popc(__ballot_sync(0xffffffffu, i < n && s_keys[i] == prefix));
-      }
-      __syncthreads();  // s_wcnt is rewritten
-      if (lane == 0) s_wcnt[warp] = eq;
-      __syncthreads();
-      unsigned rank, tot_eq;
-      warp_offsets(rank, tot_eq);
-      for (int w = w0; w < w1; ++w) {
-        const int i = w * 32 + lane;
-        const bool ok = i < n;
-        const uint32_t key = ok ? s_keys[i] : 0u;
-        const bool e = ok && key == prefix;
-        const unsigned em = __ballot_sync(0xffffffffu, e);
-        const unsigned rk = rank + __popc(em & lt);
-        const unsigned word = __ballot_sync(0xffffffffu, ok && (key > prefix || (e && rk < kk)));
-        if (lane == 0) s_bm[w] = word;
-        rank += __popc(em);
-      }
-    }
+    if (lane == 0) *a.head_count = (int32_t)base;
   }
-  // union over the neuron rows: with one row the CTA's own bitmap is the
-  // union; otherwise the rows' bitmaps meet in global memory and the last
-  // CTA (ticket) ORs them, loading every word at once
-  if (a.neuron_rows > 1) {
-    __syncthreads();
-    for (int w = tid; w < nw; w += SEL_THREADS) bm[w] = s_bm[w];
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = (atomicAdd(a.ticket, 1u) == (unsigned)a.neuron_rows - 1u);
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    for (int w = tid; w < nw; w += SEL_THREADS) {
-      uint32_t u = 0;
-      for (int rr = 0; rr < a.neuron_rows; ++rr) u |= __ldcg(a.bitmaps + (size_t)rr * nw + w);
-      s_bm[w] = u;
-    }
-    __syncthreads();
-    if (tid == 0) *a.ticket = 0u;
-  }
-  // idx: each warp writes the set bits of its own words in ascending order
-  __syncwarp();
-  unsigned pc = 0u;
-  for (int w = w0; w < w1; ++w) pc += __popc(s_bm[w]);
-  __syncthreads();  // s_wcnt is rewritten
-  if (lane == 0) s_wcnt[warp] = pc;
-  __syncthreads();
-  unsigned out_off, total;
-  warp_offsets(out_off, total);
-  for (int w = w0; w < w1; ++w) {
-    const uint32_t u = s_bm[w];
-    if ((u >> lane) & 1u) a.idx[out_off + __popc(u & lt)] = w * 32 + lane;
-    out_off += __popc(u);
-  }
-  if (tid == 0) *a.count = (int32_t)total;
 }
-
 
 // ----------------------------------------------------------------------------
 // select_rows_kernel: the selected set of B score rows of length n (top-k per

@@ -68,15 +68,24 @@ struct WT<__nv_bfloat16> {
 
 // Weight-only int8 rows (a per-row scale applied by the kernel): a 16-byte
 // vector holds 16 signed bytes, element i in byte i.
+//
+// Conversion without the integer-to-float unit: flipping a byte's sign bit
+// gives u = x + 128 in [0, 255]; placed in the low mantissa byte of 2^23
+// (bit pattern 0x4B0000uu, one byte permute) it is exactly the float
+// 2^23 + u, and subtracting 2^23 + 128 leaves x exactly. One permute and one
+// add per element, both at full rate.
 template <>
 struct WT<int8_t> {
   static constexpr int E = 16;
   __device__ static __forceinline__ void unpack(const uint4& u, float (&f)[16]) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    const uint32_t w[4] = {u.x ^ 0x80808080u, u.y ^ 0x80808080u, u.z ^ 0x80808080u, u.w ^ 0x80808080u};
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) f[4 * i + j] = (float)(int8_t)(w[i] >> (8 * j));
+    for (int i = 0; i < 4; ++i) {
+      f[4 * i + 0] = __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7650u)) - 8388736.f;
+      f[4 * i + 1] = __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7651u)) - 8388736.f;
+      f[4 * i + 2] = __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7652u)) - 8388736.f;
+      f[4 * i + 3] = __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7653u)) - 8388736.f;
+    }
   }
 };
 

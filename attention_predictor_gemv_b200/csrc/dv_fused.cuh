@@ -11,9 +11,10 @@
 //                     (column-owner and ring variants as above)
 // and the look-ahead predictor as kernels on side streams:
 //   predict_a_kernel  head scores and z = y A (when not carried by attn_in)
-//   predict_b_kernel  neuron scores z B^T + b1 with a digit histogram
-//   select_finish_kernel and gate_kernel (dv_api_kernels.cuh): the exact
-//                     head and neuron selections, and the ordering gate
+//   predict_b_kernel  neuron scores z B^T + b1
+//   select_rows_kernel, select_heads_kernel and gate_kernel
+//                     (dv_api_kernels.cuh): the exact neuron and head
+//                     selections, and the ordering gate
 //
 // The residual stream moves x -> t1 -> x through the three main kernels:
 // attn_in zeroes t1, attn_out adds x + MHA(yA) into t1 and zeroes x, and
@@ -504,7 +505,9 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_in_kernel(AttnInArgs a) {
 // t1. With WV > 0 the slice (WV 16-byte vectors per thread) is loaded into
 // registers before griddep_wait; with WV = 0 it is streamed afterwards. The
 // cluster of slot 0 also moves the residual: t1 += x (+ bO) on its slices,
-// then x = 0. With WV < 0 (long rows, batch 1-2) CTA c instead multiplies H
+// then x = 0. With WV = ATTN_H_ONLY the kernel stops at H, which CTA 0 of
+// the cluster stores to memory (the W^O product and the residual are then
+// wo_stream_kernel's). With WV < 0 (long rows, batch 1-2) CTA c instead multiplies H
 // by whole rows c, c + CS, ... of W_i^O (each thread -WV 16-byte vectors of a
 // row) and adds its full-width partial to t1: on B200 a CTA streaming whole
 // 16-24 KB rows reaches about three times the bandwidth of CTAs that each
@@ -526,7 +529,12 @@ struct AttnOutArgs {
   float scale;
   int* status;
   int stage_rows;  // batch rows whose K/V tiles fit in shared memory at once: nb, or 1
+  float* H_out;    // [nb][kh_max][dh]: the attention outputs (only with WV = ATTN_H_ONLY)
 };
+
+// attn_out_kernel's WV for "attention only": H goes to memory and
+// wo_stream_kernel (dv_stream.cuh) multiplies it by the W^O rows
+constexpr int ATTN_H_ONLY = 1;
 
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
@@ -552,7 +560,8 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
   constexpr int G = DH / E;    // lanes per key row
   constexpr int KPW = 32 / G;  // keys per warp step
   constexpr int PW = DH + 2;   // partial: m, l, acc[DH]
-  constexpr int RG = WV > 0 ? DH / WV : 1;  // W^O row groups (register path)
+  constexpr bool H_ONLY = WV == ATTN_H_ONLY;  // H to global memory; W^O in wo_stream_kernel
+  constexpr int RG = (WV > 0 && !H_ONLY) ? DH / WV : 1;  // W^O row groups (register path)
   extern __shared__ __align__(16) unsigned char s_dyn[];
   const int SR = a.stage_rows;
   KT* sK = reinterpret_cast<KT*>(s_dyn);                               // [SR][S][DH]
@@ -561,7 +570,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
   float* s_q = s_all + (size_t)a.nb * CS * PW;                          // [nb][DH], scaled q
   __shared__ __align__(16) float s_w[FUSED_WARPS][PW];
   __shared__ __align__(16) float s_H[NB][DH];
-  __shared__ float s_red[WV > 0 ? 1 : FUSED_THREADS * E];
+  __shared__ float s_red[WV != 0 ? 1 : FUSED_THREADS * E];
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = (int)cluster.block_rank();
   const int p = blockIdx.y;
@@ -603,7 +612,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
   const bool pos_in_chunk = a.pos >= t0 && a.pos < t0 + nk;
   // register path: thread (cgi, rg) holds rows rg + i RG of column vector cgi
   const int cgi = tid / RG, rg = tid % RG;
-  uint4 wo[WV > 0 ? WV : 1];
+  uint4 wo[(WV > 0 && !H_ONLY) ? WV : 1];
   // whole-row path: rows crank + CS u, u < WU, of W_i^O are this CTA's first
   // group; they are loaded into registers at the start, so they arrive while
   // the attention runs
@@ -611,7 +620,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
   constexpr int NVO = WV < 0 ? -WV : 1;
   uint4 wfirst[WU][NVO];
   auto load_wo = [&]() {
-    if constexpr (WV > 0) {
+    if constexpr (WV > 0 && !H_ONLY) {
       const KT* Wh = WO + (size_t)head * DH * a.d + c_lo + cgi * E;
 #pragma unroll
       for (int i = 0; i < WV; ++i) wo[i] = ld_stream(Wh + (size_t)(rg + i * RG) * a.d);
@@ -776,6 +785,12 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
     }
   }
   __syncthreads();
+  if constexpr (H_ONLY) {  // H of the head to global memory (CTA 0 of the cluster)
+    if (active && crank == 0)
+      for (int i = tid; i < a.nb * DH; i += FUSED_THREADS)
+        a.H_out[((size_t)(i / DH) * a.kh_max + p) * DH + i % DH] = s_H[i / DH][i % DH];
+    return;
+  }
   // slot 0's cluster moves the residual: every CTA on its own column slice,
   // or CTA 0 on all columns when CTAs take whole rows
   const bool residual = (p == 0) && (WV >= 0 || crank == 0);
@@ -857,7 +872,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
                    make_float4(o[b][j][4 * e4], o[b][j][4 * e4 + 1], o[b][j][4 * e4 + 2], o[b][j][4 * e4 + 3]));
       }
     }
-  } else if constexpr (WV > 0) {
+  } else if constexpr (WV > 0 && !H_ONLY) {
     // ---- W^O slice from registers; row groups reduced across RG lanes ----
     float o[NB][E];
 #pragma unroll
@@ -1019,57 +1034,60 @@ __global__ void __launch_bounds__(FUSED_THREADS) predict_a_kernel(PredictAArgs a
 
 // ----------------------------------------------------------------------------
 // Look-ahead predictor, second kernel: neuron scores s[b][i] = z[b] . Bm[i] +
-// b1[i] (rows of length r); in top-k mode each score also adds one to a
-// global histogram of the top 11 bits of its order-preserving key (the first
-// digit pass of the selection, spread over the whole grid).
+// b1[i] (rows of length r). Persistent grid: warp w of CTA c takes row
+// groups (c * FUSED_WARPS + w) RPW + k (grid size) RPW, and issues the loads
+// of its next group before it reduces the current one, so two groups per
+// warp are always in flight.
 // ----------------------------------------------------------------------------
-constexpr int PB_MAX_N = 65536;
-
 struct PredictBArgs {
   const float* z;  // [B][r]
   const void* Bm;  // [N][r]
   const float* b1; // [N]
-  int N, r, nb, hist_mode;
+  int N, r, nb;
   float* scores;   // [B][N]
-  unsigned* hist;  // [B][2048], zero on entry
 };
 
 template <typename T, int NB, int RPW, int U>
 __global__ void __launch_bounds__(FUSED_THREADS) predict_b_kernel(PredictBArgs a) {
   griddep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row0 = (blockIdx.x * FUSED_WARPS + warp) * RPW;
-  const T* rowp[RPW];
-  bool valid[RPW];
-  float bias[RPW];
+  const int nvec = a.r / WT<T>::E;
+  const int stride = gridDim.x * FUSED_WARPS * RPW;
+  const T* Bm = static_cast<const T*>(a.Bm);
+  auto setup = [&](int r0, const T* (&rowp)[RPW], bool (&valid)[RPW]) {
 #pragma unroll
-  for (int r = 0; r < RPW; ++r) {
-    valid[r] = row0 + r < a.N;
-    rowp[r] = static_cast<const T*>(a.Bm) + (size_t)(valid[r] ? row0 + r : 0) * a.r;
-    bias[r] = valid[r] ? a.b1[row0 + r] : 0.f;
-  }
+    for (int r = 0; r < RPW; ++r) {
+      valid[r] = r0 + r < a.N;
+      rowp[r] = Bm + (size_t)(valid[r] ? r0 + r : 0) * a.r;
+    }
+  };
+  int row0 = (blockIdx.x * FUSED_WARPS + warp) * RPW;
+  const T* rp[RPW];
+  bool vd[RPW];
   RowLoads<T, RPW, U> L;
-  issue_row_loads<T, RPW, U>(L, rowp, valid, a.r / WT<T>::E, lane);
-  griddep_wait();  // z comes from the previous kernel
-  float acc[RPW][NB];
-  finish_rows_dot<T, NB, RPW, U>(L, rowp, valid, a.z, a.r, a.nb, acc);
-  // lane (r * NB + b) % 32 owns score (r, b); lanes with equal histogram
-  // bins are merged before the global atomic (one per distinct bin)
-#pragma unroll
-  for (int c0 = 0; c0 < RPW * NB; c0 += 32) {
-    unsigned bin = 0xffffffffu;
+  setup(row0, rp, vd);
+  issue_row_loads<T, RPW, U>(L, rp, vd, nvec, lane);  // Bm does not depend on the previous kernel
+  griddep_wait();                                     // z does
+#pragma unroll 1
+  for (; row0 < a.N; row0 += stride) {
+    const T* rpn[RPW];
+    bool vn[RPW];
+    RowLoads<T, RPW, U> Ln;
+    setup(row0 + stride, rpn, vn);
+    issue_row_loads<T, RPW, U>(Ln, rpn, vn, nvec, lane);
+    float acc[RPW][NB];
+    finish_rows_dot<T, NB, RPW, U>(L, rp, vd, a.z, a.r, a.nb, acc);
 #pragma unroll
     for (int r = 0; r < RPW; ++r)
 #pragma unroll
       for (int b = 0; b < NB; ++b)
-        if (r * NB + b >= c0 && r * NB + b < c0 + 32 && lane == r * NB + b - c0 && valid[r] && b < a.nb) {
-          const float v = acc[r][b] + bias[r];
-          a.scores[(size_t)b * a.N + row0 + r] = v;
-          bin = (unsigned)b * SEL_BINS + (ord_key(v) >> 21);
-        }
-    if (a.hist_mode) {
-      const unsigned peers = __match_any_sync(0xffffffffu, bin);
-      if (bin != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(a.hist + bin, (unsigned)__popc(peers));
+        if (lane == ((r * NB + b) & 31) && vd[r] && b < a.nb)
+          a.scores[(size_t)b * a.N + row0 + r] = acc[r][b] + a.b1[row0 + r];
+    L = Ln;
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+      rp[r] = rpn[r];
+      vd[r] = vn[r];
     }
   }
 }

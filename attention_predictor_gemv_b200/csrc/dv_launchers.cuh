@@ -281,6 +281,7 @@ inline int attn_out_whole_rows(int d, int E, int kvbytes, int nb) {
 template <typename KT, int DH, int NB>
 cudaError_t run_attn_out_nb(const AttnOutArgs& a, cudaStream_t st) {
   if constexpr (NB <= 2 && sizeof(KT) == 2) {
+    if (a.H_out) return run_attn_out_nbw<KT, DH, NB, ATTN_H_ONLY>(a, st);  // W^O in wo_stream_kernel
     switch (attn_out_whole_rows(a.d, WT<KT>::E, sizeof(KT), a.nb)) {
       case 4: return run_attn_out_nbw<KT, DH, NB, -4>(a, st);
       case 5: return run_attn_out_nbw<KT, DH, NB, -5>(a, st);
@@ -370,7 +371,8 @@ cudaError_t run_predict_a(const PredictAArgs& a, cudaStream_t st) {
 template <typename T, int NB>
 cudaError_t run_predict_b_nb(const PredictBArgs& a, cudaStream_t st) {
   const int rpw = rpw_for(a.r, WT<T>::E), per = FUSED_WARPS * rpw;
-  const dim3 grid((a.N + per - 1) / per);
+  const int groups = (a.N + per - 1) / per;
+  const dim3 grid(groups < 2 * sm_count() ? groups : 2 * sm_count());  // persistent: two CTAs per SM
   switch (rpw) {
     case 1: return launch(predict_b_kernel<T, NB, 1, 8>, grid, FUSED_THREADS, 0, st, a);
     case 2: return launch(predict_b_kernel<T, NB, 2, 4>, grid, FUSED_THREADS, 0, st, a);
@@ -529,7 +531,23 @@ cudaError_t run_predict_a_st_nb(const PredictAArgs& a, cudaStream_t st) {
   const dim3 grid(st_grid((a.PA ? a.h : 0) + (a.At ? a.r : 0)));
   DV_ST_SWITCH(predict_a_stream_kernel, NB, grid, st, a)
 }
+template <typename T, int NB>
+cudaError_t run_wo_stream_nb(const WoStreamArgs& a, cudaStream_t st) {
+  const int nv = co_nv(a.d, WT<T>::E);
+  const dim3 grid(sm_count());
+  DV_ST_SWITCH(wo_stream_kernel, NB, grid, st, a)
+}
 #undef DV_ST_SWITCH
+
+// The W^O product in its own ring kernel after an attention-only attn_out:
+// long rows (16-24 KB, bf16), batch 1-2, and DV_WOSPLIT not 0.
+inline bool wo_split_ok(int nb, int d, int E, int kvbytes) {
+  static const bool on = [] {
+    const char* e = std::getenv("DV_WOSPLIT");
+    return !(e && e[0] == '0');
+  }();
+  return on && attn_out_whole_rows(d, E, kvbytes, nb) != 0 && st_ok(nb, d, E);
+}
 
 // Whether run_attn_in_any picks a kernel that also takes the next layer's
 // predictor rows (the column-owner and streaming kernels).
@@ -600,6 +618,7 @@ cudaError_t run_axpy_q8(const int8_t* W, int d, int nrows_w, RowsHeads src, cons
 cudaError_t run_attn_out_dt(dv_dtype kvdt, const AttnOutArgs& a, cudaStream_t st);
 cudaError_t run_attn_out_bf16(const AttnOutArgs& a, cudaStream_t st);
 cudaError_t run_attn_out_f32(const AttnOutArgs& a, cudaStream_t st);
+cudaError_t run_wo_stream_dt(dv_dtype wdt, const WoStreamArgs& a, cudaStream_t st);
 cudaError_t run_mlp_block_any_dt(dv_dtype wdt, const MlpBlockArgs& a, cudaStream_t st);
 cudaError_t run_predict_a_any_dt(dv_dtype wdt, const PredictAArgs& a, cudaStream_t st);
 cudaError_t run_predict_b_dt(dv_dtype wdt, const PredictBArgs& a, cudaStream_t st);

@@ -422,4 +422,141 @@ __global__ void __launch_bounds__(CO_THREADS, 1) mlp_stream_kernel(MlpBlockArgs 
   }
 }
 
+// ----------------------------------------------------------------------------
+// wo_stream_kernel: the W^O product of eq. (2) for long rows (16-24 KB, batch
+// 1-2), after attn_out_kernel stopped at H (ATTN_H_ONLY):
+//   t1 += sum over the selected heads' rows (p, c) of H[b][p][c] W_i^O[c][:]
+// Rows are spread evenly over one CTA per SM; each CTA streams its rows
+// through the ring into its threads' own columns (no CTA reduction) and adds
+// its full-width partial to t1 once. The first rows are issued before the
+// dependency wait when the head set is known ahead (their W^O rows do not
+// depend on the attention), so they stream while the attention runs. CTA 0
+// also moves the residual: t1 += x + bO, then x = 0.
+// ----------------------------------------------------------------------------
+struct WoStreamArgs {
+  const void* WOt;  // [h][dh][d]
+  const float* bO;  // [d] or null
+  const float* H;   // [nb][kh_max][dh]
+  const int32_t* head_idx;
+  const int32_t* head_count;
+  int kh_max, h, dh, d, nb, sets_ready;
+  float* x;
+  float* t1;
+  int* status;
+};
+
+constexpr int WO_CHUNK = 1024;  // rows whose coefficients a CTA holds at once
+
+template <typename T, int NB, int NV>
+__global__ void __launch_bounds__(CO_THREADS, 1) wo_stream_kernel(WoStreamArgs a) {
+  constexpr int E = WT<T>::E;
+  extern __shared__ __align__(16) uint4 s_ring[];
+  __shared__ float s_coef[WO_CHUNK][NB];
+  const T* WO = static_cast<const T*>(a.WOt);
+  const int nvec = a.d / E;
+  griddep_launch();
+  int r0 = 0, r1 = 0;
+  auto range = [&]() {
+    int hc = *a.head_count;
+    if (hc > a.kh_max || hc < 0) {
+      if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(a.status, 1);
+      hc = hc < 0 ? 0 : a.kh_max;
+    }
+    const long long nrows = (long long)hc * a.dh;
+    r0 = (int)(nrows * blockIdx.x / gridDim.x);
+    r1 = (int)(nrows * (blockIdx.x + 1) / gridDim.x);
+  };
+  auto head_of = [&](int i) {
+    const int head = a.head_idx[i / a.dh];
+    return (head >= 0 && head < a.h) ? head : -1;
+  };
+  auto row = [&](int i) -> const T* {
+    const int head = head_of(i);
+    return head >= 0 ? WO + ((size_t)head * a.dh + i % a.dh) * a.d : nullptr;
+  };
+  auto rowr = [&](int i) -> const T* { return row(r0 + i); };
+  if (a.sets_ready) {
+    range();
+    st_prologue<T, NV>(s_ring, 0, r1 - r0, nvec, rowr);
+  }
+  griddep_wait();
+  if (!a.sets_ready) {
+    range();
+    st_prologue<T, NV>(s_ring, 0, r1 - r0, nvec, rowr);
+  }
+  float acc[NB][NV][E];
+#pragma unroll
+  for (int b = 0; b < NB; ++b)
+#pragma unroll
+    for (int j = 0; j < NV; ++j)
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[b][j][e] = 0.f;
+  const int n = r1 - r0;
+#pragma unroll 1
+  for (int c0 = 0; c0 < n; c0 += WO_CHUNK) {
+    const int cn = min(WO_CHUNK, n - c0);
+    __syncthreads();  // the previous chunk's coefficients are consumed
+    for (int t = threadIdx.x; t < cn * NB; t += CO_THREADS) {
+      const int i = t / NB, b = t % NB, rr = r0 + c0 + i;
+      const bool ok = b < a.nb && head_of(rr) >= 0;
+      s_coef[i][b] = ok ? __ldcg(a.H + ((size_t)b * a.kh_max + rr / a.dh) * a.dh + rr % a.dh) : 0.f;
+      if (b == 0 && head_of(rr) < 0 && rr % a.dh == 0) raise_status(a.status, 2);
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int i = c0; i < c0 + cn; ++i) {
+      const int ahead = i + ST_SLOTS - 1;
+      st_issue<T, NV>(s_ring, ahead, ahead < n ? rowr(ahead) : nullptr, nvec);
+      cp_async_wait<ST_SLOTS - 1>();
+      if (head_of(r0 + i) < 0) continue;  // a skipped row: its slot holds no data (same for every thread)
+      uint4 w[NV];
+      st_read<NV>(s_ring, i, nvec, w);
+      float cb[NB];
+#pragma unroll
+      for (int b = 0; b < NB; ++b) cb[b] = s_coef[i - c0][b];
+#pragma unroll
+      for (int j = 0; j < NV; ++j) {
+        float wf[E];
+        WT<T>::unpack(w[j], wf);
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+          for (int e = 0; e < E; ++e) acc[b][j][e] = fmaf(cb[b], wf[e], acc[b][j][e]);
+      }
+    }
+  }
+  const bool residual = blockIdx.x == 0;
+  if (n == 0 && !residual) return;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int c = (j * CO_THREADS + threadIdx.x) * E;
+    if (c >= a.d) continue;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (b >= a.nb) continue;
+      float o[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) o[e] = acc[b][j][e];
+      if (residual) {
+        float* xr = a.x + (size_t)b * a.d + c;
+#pragma unroll
+        for (int e4 = 0; e4 < E / 4; ++e4) {
+          const float4 xv = __ldcg(reinterpret_cast<const float4*>(xr) + e4);
+          float4 bb = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (a.bO) bb = *(reinterpret_cast<const float4*>(a.bO + c) + e4);
+          o[4 * e4 + 0] += xv.x + bb.x;
+          o[4 * e4 + 1] += xv.y + bb.y;
+          o[4 * e4 + 2] += xv.z + bb.z;
+          o[4 * e4 + 3] += xv.w + bb.w;
+          reinterpret_cast<float4*>(xr)[e4] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int e4 = 0; e4 < E / 4; ++e4)
+        red_add4(a.t1 + (size_t)b * a.d + c + 4 * e4,
+                 make_float4(o[4 * e4], o[4 * e4 + 1], o[4 * e4 + 2], o[4 * e4 + 3]));
+    }
+  }
+}
+
 }  // namespace dv

@@ -1,6 +1,7 @@
-"""Tensor-core gathered-row path (batch 5..16, bf16 weights) vs the CPU oracle.
+"""Tensor-core gathered-row path (batch 5..16, and 3..4 for rows longer than
+4096 bf16 elements; bf16 weights) vs the CPU oracle.
 
-From five batch rows on, the layer and block calls run q/k/v, W1 (+ bias,
+From five batch rows on (three for long rows), the layer and block calls run q/k/v, W1 (+ bias,
 ReLU, compaction), W2 and W^O as tcgen05 MMAs over the gathered rows, with
 the activations split into two bf16 halves. Same bar as every parity test:
 index sets bit-exact, block outputs within relative L2 5e-3 and max-abs
@@ -49,7 +50,8 @@ def _no_device_errors(ws):
 
 @pytest.mark.parametrize("name,B,k", [("ragged", 5, 37), ("ragged", 8, 1000), ("opt-like", 8, 819),
                                       ("opt-like", 16, 4100), ("opt-like", 16, 8192), ("opt-like", 12, 129),
-                                      ("wide", 16, 2000), ("175b-slice", 8, 3001)])
+                                      ("wide", 16, 2000), ("175b-slice", 8, 3001), ("wide", 3, 1500),
+                                      ("175b-slice", 4, 615)])
 @pytest.mark.parametrize("with_b2", [False, True])
 def test_tc_sparse_mlp(name, B, k, with_b2):
     s = _shape(name, B)
@@ -145,7 +147,8 @@ def _trace_bufs(s):
 
 @pytest.mark.parametrize("name,B,kf,khf", [("opt-like", 8, 0.10, 0.25), ("opt-like", 16, 0.05, 0.25),
                                           ("ragged", 6, 0.2, 0.34), ("wide", 8, 0.1, 0.25),
-                                          ("175b-slice", 16, 0.15, 0.25), ("opt-like", 16, 1.0, 1.0)])
+                                          ("175b-slice", 16, 0.15, 0.25), ("opt-like", 16, 1.0, 1.0),
+                                          ("wide", 4, 0.1, 0.25), ("175b-slice", 3, 0.15, 0.25)])
 def test_tc_decode_layer(name, B, kf, khf):
     s = _shape(name, B)
     t = wl.make_layer(s, 61, DEV)
