@@ -78,6 +78,7 @@ Layout layout(const dv_dims& D, int wbytes) {
   const int tiles = tc_tiles(D.k_max);
   L.KC = tiles * TC_M;
   L.XC = D.d > D.kh_max * D.dh ? D.d : D.kh_max * D.dh;
+  if (L.XC < D.r) L.XC = D.r;
   L.tc_x = take(2ull * 2 * TC_N * L.XC);
   L.tc_act = take(2ull * 2 * TC_N * (L.KC > 0 ? L.KC : 1));
   L.tc_rowid = take(4ull * (L.KC > 0 ? L.KC : 1));
@@ -140,12 +141,65 @@ cudaError_t select_any(const float* scores, int nrows, int n, int k, float tau, 
 // Operation bodies shared by the public entry points
 // ---------------------------------------------------------------------------
 
+bool fused_enabled();
+bool tc_enabled();
+int wbytes_of(dv_dtype t);
+
+// A predictor GEMM at batch >= 3 on the tensor cores (tc_dense_kernel):
+// out[b][row] = W[row] . x[b] (+ bias[row]), x [B][K] split into the
+// workspace's hi / lo operand rows first.
+bool pred_tc_ok(int B, dv_dtype wdt, int nrows, int K) {
+  return tc_enabled() && B >= 3 && tc_dense_ok(B, wbytes_of(wdt), nrows, K);
+}
+
+cudaError_t pred_tc(const Layout& L, void* ws, const void* W, int nrows, int K, const float* bias, const float* x, int B,
+                    float* out, long long ldo, cudaStream_t st) {
+  bf16* xhi = at<bf16>(ws, L.tc_x);
+  bf16* xlo = xhi + (size_t)TC_N * L.XC;
+  cudaError_t e = run_tc_split(x, B, K, K, xhi, xlo, K, st);
+  if (e != cudaSuccess) return e;
+  return run_tc_dense(static_cast<const bf16*>(W), nrows, K, bias, xhi, xlo, B, out, ldo, at<int>(ws, L.status), st);
+}
+
+// The predictor's two stages: z = y A (predict_a_kernel family; rows of At
+// read once for all batch rows) and the neuron scores z B^T + b1
+// (predict_b_kernel); at batch >= 3 both on the tensor cores. DV_FUSED=0
+// runs them as plain GEMVs instead.
+cudaError_t predict_z(const Layout& L, void* ws, const float* y, int B, int d, int r, const void* At, dv_dtype dt,
+                      float* z, cudaStream_t st) {
+  if (!fused_enabled()) return run_gemv(dt, At, r, d, y, d, B, nullptr, z, r, st);
+  if (pred_tc_ok(B, dt, r, d)) return pred_tc(L, ws, At, r, d, nullptr, y, B, z, r, st);
+  PredictAArgs a = {};
+  a.y = y;
+  a.At = At;
+  a.r = r;
+  a.d = d;
+  a.nb = B;
+  a.z = z;
+  return run_predict_a_any_dt(dt, a, st);
+}
+
+cudaError_t predict_scores(const Layout& L, void* ws, const float* z, int B, int r, int N, const void* Bm,
+                           const float* b1, dv_dtype dt, float* scores, cudaStream_t st) {
+  if (!fused_enabled()) return run_gemv(dt, Bm, N, r, z, r, B, b1, scores, N, st);
+  if (pred_tc_ok(B, dt, N, r)) return pred_tc(L, ws, Bm, N, r, b1, z, B, scores, N, st);
+  PredictBArgs b = {};
+  b.z = z;
+  b.Bm = Bm;
+  b.b1 = b1;
+  b.N = N;
+  b.r = r;
+  b.nb = B;
+  b.scores = scores;
+  return run_predict_b_dt(dt, b, st);
+}
+
 dv_status do_predict_mlp(const Layout& L, void* ws, const float* y, int B, int d, int r, int N, const void* At,
                          const void* Bm, const float* b1, dv_dtype dt, int k, float tau, int mode, float* scores,
                          int32_t* idx, int32_t* count, cudaStream_t st) {
   float* z = at<float>(ws, L.z);
-  DV_TRY(run_gemv(dt, At, r, d, y, d, B, nullptr, z, r, st));
-  DV_TRY(run_gemv(dt, Bm, N, r, z, r, B, b1, scores, N, st));
+  DV_TRY(predict_z(L, ws, y, B, d, r, At, dt, z, st));
+  DV_TRY(predict_scores(L, ws, z, B, r, N, Bm, b1, dt, scores, st));
   DV_TRY(select_any(scores, B, N, k, tau, mode, at<uint32_t>(ws, L.bm_m), at<unsigned>(ws, L.sel_ticket_m), idx, count,
                     st));
   return DV_OK;
@@ -154,7 +208,20 @@ dv_status do_predict_mlp(const Layout& L, void* ws, const float* y, int B, int d
 dv_status do_predict_heads(const Layout& L, void* ws, const float* y, int B, int d, int h, const void* PA, dv_dtype dt,
                            int k_h, float tau, int mode, float* scores, int32_t* head_idx, int32_t* head_count,
                            cudaStream_t st) {
-  DV_TRY(run_gemv(dt, PA, h, d, y, d, B, nullptr, scores, h, st));
+  if (fused_enabled() && pred_tc_ok(B, dt, h, d)) {
+    DV_TRY(pred_tc(L, ws, PA, h, d, nullptr, y, B, scores, h, st));
+  } else if (fused_enabled()) {
+    PredictAArgs a = {};
+    a.y = y;
+    a.PA = PA;
+    a.h = h;
+    a.d = d;
+    a.nb = B;
+    a.scores_h = scores;
+    DV_TRY(run_predict_a_any_dt(dt, a, st));
+  } else {
+    DV_TRY(run_gemv(dt, PA, h, d, y, d, B, nullptr, scores, h, st));
+  }
   DV_TRY(select_any(scores, B, h, k_h, tau, mode, at<uint32_t>(ws, L.bm_h), at<unsigned>(ws, L.sel_ticket_h), head_idx,
                     head_count, st));
   return DV_OK;
@@ -239,7 +306,7 @@ bool tc_enabled() {
 // kernels (d > 4096 bf16), where the CUDA-core row kernels would take them.
 bool tc_ok(int B, int d, dv_dtype wdt, int dh, int k_max) {
   const bool batch = B >= TC_MIN_B || (B >= 3 && !co_ok(B, d, 8));
-  return tc_enabled() && batch && tc_shape_ok(B, wbytes_of(wdt), dh > 0 ? dh : 64, k_max);
+  return tc_enabled() && batch && tc_shape_ok(B, d, wbytes_of(wdt), dh > 0 ? dh : 64, k_max);
 }
 
 dv_status tc_mlp(const Layout& L, void* ws, const float* y, int B, int d, int N, const void* W1t, const float* b1,
@@ -444,8 +511,25 @@ dv_status layer_begin(const Layout& L, void* ws, const dv_layer_weights* w, cons
     dv_layer_io tr = trace ? *trace : dv_layer_io{};
     if (!(sel && sel->yA)) tr.yA = yA;
     DV_CHECK(layer_begin(L, ws, w, D, p, x, pos, sel, &tr, st));
-    DV_TRY(run_gemv(w->wdtype, ahead->w->PA, D.h, D.d, yA, D.d, D.B, nullptr, ahead->sh, D.h, st));
-    return cuda_status(run_gemv(w->wdtype, ahead->w->At, D.r, D.d, yA, D.d, D.B, nullptr, ahead->z, D.r, st));
+    if (!fused_enabled()) {
+      DV_TRY(run_gemv(w->wdtype, ahead->w->PA, D.h, D.d, yA, D.d, D.B, nullptr, ahead->sh, D.h, st));
+      return cuda_status(run_gemv(w->wdtype, ahead->w->At, D.r, D.d, yA, D.d, D.B, nullptr, ahead->z, D.r, st));
+    }
+    const bool tc_h = pred_tc_ok(D.B, w->wdtype, D.h, D.d), tc_z = pred_tc_ok(D.B, w->wdtype, D.r, D.d);
+    if (tc_h) DV_TRY(pred_tc(L, ws, ahead->w->PA, D.h, D.d, nullptr, yA, D.B, ahead->sh, D.h, st));
+    if (tc_z) DV_TRY(pred_tc(L, ws, ahead->w->At, D.r, D.d, nullptr, yA, D.B, ahead->z, D.r, st));
+    if (tc_h && tc_z) return DV_OK;
+    PredictAArgs pa = {};
+    pa.y = yA;
+    pa.PA = tc_h ? nullptr : ahead->w->PA;
+    pa.At = tc_z ? nullptr : ahead->w->At;
+    pa.h = D.h;
+    pa.r = D.r;
+    pa.d = D.d;
+    pa.nb = D.B;
+    pa.scores_h = ahead->sh;
+    pa.z = ahead->z;
+    return cuda_status(run_predict_a_any_dt(w->wdtype, pa, st));
   }
   if (fused_ok(D, w->wdtype)) {
     if (!sel) {
@@ -940,7 +1024,7 @@ dv_status dv_predict_layer_tail(const dv_layer_weights* w, const dv_dims* dims, 
       DV_TRY(select_any(out->scores_h, D.B, D.h, p->k_h, p->tau_h, p->mode_h, at<uint32_t>(ws, L.bm_h),
                         at<unsigned>(ws, L.sel_ticket_h), out->head_idx, out->head_count, st));
     if (neurons) {
-      DV_TRY(run_gemv(w->wdtype, w->Bm, D.N, D.r, at<float>(ws, L.z), D.r, D.B, w->b1, out->scores, D.N, st));
+      DV_TRY(predict_scores(L, ws, at<float>(ws, L.z), D.B, D.r, D.N, w->Bm, w->b1, w->wdtype, out->scores, st));
       DV_TRY(select_any(out->scores, D.B, D.N, p->k, p->tau, p->mode, at<uint32_t>(ws, L.bm_m),
                         at<unsigned>(ws, L.sel_ticket_m), out->idx, out->count, st));
     }

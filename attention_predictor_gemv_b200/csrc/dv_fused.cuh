@@ -1047,8 +1047,8 @@ struct PredictBArgs {
   float* scores;   // [B][N]
 };
 
-template <typename T, int NB, int RPW, int U>
-__global__ void __launch_bounds__(FUSED_THREADS) predict_b_kernel(PredictBArgs a) {
+template <typename T, int NB, int RPW, int U, int MINB = 1>
+__global__ void __launch_bounds__(FUSED_THREADS, MINB) predict_b_kernel(PredictBArgs a) {
   griddep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nvec = a.r / WT<T>::E;

@@ -1,4 +1,9 @@
-// Launchers of the tensor-core gathered-row kernels (dv_tc.cuh).
+// Launchers of the tensor-core gathered-row kernels (dv_tc.cuh), and the
+// TMA descriptors they read.
+#include <cudaTypedefs.h>
+
+#include <cstdlib>
+
 #include "dv_launch.cuh"
 #include "dv_tc.cuh"
 #include "dv_tc_launch.h"
@@ -7,29 +12,85 @@ namespace dv {
 
 namespace {
 
+// CTAs per SM: one with a TC_STAGES_MAX-stage ring, or two with half the
+// ring each (DV_TC_CTAS=1 / 2).
+int tc_ctas_per_sm() {
+  static const int n = [] {
+    const char* e = std::getenv("DV_TC_CTAS");
+    return (e && e[0] == '1') ? 1 : 2;
+  }();
+  return n;
+}
+int tc_stages() { return TC_STAGES_MAX / tc_ctas_per_sm(); }
+
 template <typename K, typename A>
-cudaError_t launch_tc(K kern, int grid, cudaStream_t st, const A& a) {
-  cudaError_t e = allow_smem(kern, TC_SMEM);
+cudaError_t launch_tc(K kern, int grid, cudaStream_t st, const TcMaps& m, A a) {
+  a.stages = tc_stages();
+  const size_t smem = tc_smem(a.stages);
+  cudaError_t e = allow_smem(kern, smem);
   if (e != cudaSuccess) return e;
-  return launch_main(kern, dim3(grid < 1 ? 1 : grid), dim3(TC_THREADS), TC_SMEM, st, a);
+  return launch_main(kern, dim3(grid < 1 ? 1 : grid), dim3(TC_THREADS), smem, st, m, a);
 }
 
 int clamp_grid(long long units) {
-  const long long cap = sm_count();
+  const long long cap = (long long)tc_ctas_per_sm() * sm_count();
   return (int)(units < 1 ? 1 : (units > cap ? cap : units));
 }
 
-// Rows (tiles, heads) per rowaxpy unit: as many as still give every SM two
+// Rows (tiles, heads) per rowaxpy unit: as many as still give every CTA two
 // units at the largest count, at most `most`.
 int per_group(long long items_max, long long n_mt, int most) {
-  long long g = items_max * n_mt / (2ll * sm_count());
+  long long g = items_max * n_mt / (2ll * tc_ctas_per_sm() * sm_count());
   return (int)(g < 1 ? 1 : (g > most ? most : g));
+}
+
+// cuTensorMapEncodeTiled, from the driver the runtime is bound to (no link
+// against libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// A bf16 matrix [rows][cols] with row stride ld elements, read in boxes of
+// box_cols x box_rows into the 128-byte swizzled shared layout; reads past
+// the matrix return zeros.
+cudaError_t tc_map(CUtensorMap* m, const void* base, long long cols, long long rows, long long ld, int box_cols,
+                   int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  if (!aligned16(base) || (ld * 2) % 16 != 0 || cols < 1 || rows < 1 || ld < cols) return cudaErrorInvalidValue;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// Maps of one kernel: gathered weight rows (or W^O in 64-row tiles) and the
+// operand's hi / lo rows [16][ld] of which the first `cols` are used.
+cudaError_t tc_maps(TcMaps* m, const __nv_bfloat16* W, long long w_rows, int d, int w_box_rows,
+                    const __nv_bfloat16* hi, const __nv_bfloat16* lo, long long cols, long long ld) {
+  cudaError_t e = tc_map(&m->w, W, d, w_rows, d, TC_K, w_box_rows);
+  if (e == cudaSuccess) e = tc_map(&m->hi, hi, cols, TC_N, ld, TC_K, TC_N);
+  if (e == cudaSuccess) e = tc_map(&m->lo, lo, cols, TC_N, ld, TC_K, TC_N);
+  return e;
 }
 
 }  // namespace
 
-bool tc_shape_ok(int B, int wbytes, int dh, int k_max) {
-  return wbytes == 2 && B >= 1 && B <= TC_N && dh % 64 == 0 && (k_max + TC_M - 1) / TC_M <= TC_MAX_TILES;
+bool tc_shape_ok(int B, int d, int wbytes, int dh, int k_max) {
+  return wbytes == 2 && B >= 1 && B <= TC_N && d >= TC_K && d % 8 == 0 && dh % 64 == 0 &&
+         (k_max + TC_M - 1) / TC_M <= TC_MAX_TILES && encode_fn() != nullptr;
 }
 
 int tc_tiles(int k_max) { return (k_max + TC_M - 1) / TC_M; }
@@ -44,7 +105,10 @@ cudaError_t run_tc_split(const float* x, int nb, int n, long long ld_src, __nv_b
 cudaError_t run_tc_qkv(const TcQkvArgs& a, cudaStream_t st) {
   const long long units = ((long long)a.kh_max * 3 * a.dh + TC_M - 1) / TC_M;
   if (units == 0) return cudaSuccess;
-  return launch_tc(tc_qkv_kernel, clamp_grid(units), st, a);
+  TcMaps m;
+  cudaError_t e = tc_maps(&m, a.Wqkv, (long long)a.h * 3 * a.dh, a.d, 64, a.xhi, a.xlo, a.d, a.d);
+  if (e != cudaSuccess) return e;
+  return launch_tc(tc_qkv_kernel, clamp_grid(units), st, m, a);
 }
 
 cudaError_t run_tc_mlp(TcMlpArgs a, cudaStream_t st) {
@@ -52,18 +116,59 @@ cudaError_t run_tc_mlp(TcMlpArgs a, cudaStream_t st) {
   const int n_mt = (a.d + TC_M - 1) / TC_M;
   a.tiles_per_group = per_group(tiles, n_mt, TC_TILES_PER_GROUP);
   if (tiles > 0) {
-    cudaError_t e = launch_tc(tc_w1_kernel, clamp_grid(tiles), st, a);
+    TcMaps m1;
+    cudaError_t e = tc_maps(&m1, a.W1t, a.N, a.d, 1, a.xhi, a.xlo, a.d, a.d);
+    if (e == cudaSuccess) e = launch_tc(tc_w1_kernel, clamp_grid(tiles), st, m1, a);
     if (e != cudaSuccess) return e;
   }
+  TcMaps m2;
+  cudaError_t e = tc_maps(&m2, a.W2t, a.N, a.d, 1, a.act_hi, a.act_lo, a.KC > 0 ? a.KC : TC_M, a.KC > 0 ? a.KC : TC_M);
+  if (e != cudaSuccess) return e;
   const long long groups = tiles > 0 ? (tiles + a.tiles_per_group - 1) / a.tiles_per_group : 1;
-  return launch_tc(tc_w2_kernel, clamp_grid(groups * n_mt), st, a);
+  return launch_tc(tc_w2_kernel, clamp_grid(groups * n_mt), st, m2, a);
 }
 
 cudaError_t run_tc_wo(TcWoArgs a, cudaStream_t st) {
   const int n_mt = (a.d + TC_M - 1) / TC_M;
   a.heads_per_group = per_group(a.kh_max, n_mt, TC_HEADS_PER_GROUP);
   const long long groups = a.kh_max > 0 ? (a.kh_max + a.heads_per_group - 1) / a.heads_per_group : 1;
-  return launch_tc(tc_wo_kernel, clamp_grid(groups * n_mt), st, a);
+  const long long ldh = (long long)(a.kh_max > 0 ? a.kh_max : 1) * a.dh;
+  TcMaps m;
+  cudaError_t e = tc_maps(&m, a.WOt, (long long)a.h * a.dh, a.d, 64, a.hhi, a.hlo, ldh, ldh);
+  if (e != cudaSuccess) return e;
+  return launch_tc(tc_wo_kernel, clamp_grid(groups * n_mt), st, m, a);
+}
+
+bool tc_dense_ok(int B, int wbytes, int nrows, int K) {
+  return wbytes == 2 && B >= 1 && B <= TC_N && nrows >= 64 && K >= TC_K && K % 8 == 0 && encode_fn() != nullptr;
+}
+
+cudaError_t run_tc_dense(const __nv_bfloat16* W, int nrows, int K, const float* bias, const __nv_bfloat16* xhi,
+                         const __nv_bfloat16* xlo, int nb, float* out, long long ldo, int* status, cudaStream_t st) {
+  const long long tiles = (nrows + TC_M - 1) / TC_M, C = (K + TC_K - 1) / TC_K;
+  const long long slots = (long long)tc_ctas_per_sm() * sm_count();
+  long long ks = (slots + tiles - 1) / tiles;
+  if (ks > C) ks = C;
+  if (ks < 1) ks = 1;
+  TcDenseArgs a = {};
+  a.bias = bias;
+  a.nrows = nrows;
+  a.K = K;
+  a.nb = nb;
+  a.ks = (int)ks;
+  a.out = out;
+  a.ldo = ldo;
+  a.status = status;
+  if (ks > 1) {
+    for (int b = 0; b < nb; ++b) {
+      cudaError_t e = cudaMemsetAsync(out + (size_t)b * ldo, 0, sizeof(float) * (size_t)nrows, st);
+      if (e != cudaSuccess) return e;
+    }
+  }
+  TcMaps m;
+  cudaError_t e = tc_maps(&m, W, nrows, K, 64, xhi, xlo, K, K);
+  if (e != cudaSuccess) return e;
+  return launch_tc(tc_dense_kernel, clamp_grid(tiles * ks), st, m, a);
 }
 
 }  // namespace dv

@@ -1,10 +1,11 @@
-// Tensor-core gathered-row kernels (tcgen05, sm_100a) for batch 5..16.
+// Tensor-core gathered-row kernels (tcgen05 + TMA, sm_100a) for batch 3..16.
 //
 // At batch B the selected rows of W1, W2, W^{Q,K,V} and W^O meet B input
 // vectors: a gathered row times a [d][B] block is a thin dense contraction
 // (B flop per weight byte), which the CUDA cores cannot keep up with at HBM
 // rate once B reaches 8-16, so these kernels hand the multiply-adds to the
-// 5th-generation tensor cores and keep the SMs' issue slots for the loads.
+// 5th-generation tensor cores and move the bytes with the tensor memory
+// accelerator (TMA).
 //
 // Two kernel forms share one pipeline:
 //   rowdot  D[m][b] = sum_c W[row(m)][c] X[b][c]    rows of W are K-major
@@ -20,21 +21,29 @@
 // D = W X_hi + W X_lo is accurate to about 2^-16 relative instead of the 2^-9
 // of one bf16 rounding, at twice the (idle) tensor work.
 //
-// Per CTA (128 threads, one CTA per SM, persistent over work units):
-//   * all threads stage the weight tile (bf16, 16 KB) and the operand blocks
-//     (16 x 64, hi and lo) of a stage with 16-byte cp.async copies, six stages
-//     ahead, straight into the canonical no-swizzle UMMA layout (8 x 16-byte
-//     core matrices); each thread keeps the pointers of its 8 weight rows for
-//     the unit (rowdot) or the chunk (rowaxpy);
-//   * thread 0 issues the MMAs (tcgen05.mma kind::f16, bf16 inputs, fp32
-//     accumulator in tensor memory, 32 TMEM columns) and commits them to the
-//     stage's mbarrier, which frees the stage for its next copies;
-//   * at the end of a unit the four warps read the 128 x 16 accumulator
-//     (tcgen05.ld 32x32b, warp w owns TMEM lanes 32w..32w+31) and run the
-//     unit's epilogue.
+// Per CTA (416 threads, one CTA per SM, persistent over work units), three
+// roles that meet only at mbarriers:
+//   * warps 0-7 fill a ring of `stages` stages with TMA copies, in the
+//     128-byte swizzled layout the MMA reads, completing on the stage's
+//     "full" barrier: the weight tile (16 KB) as two plain 2-D tiles of 64
+//     rows where the rows are consecutive (a head's Q/K/V or W^O rows), else
+//     by 32 tile::gather4 loads of 4 gathered rows x 64 columns (W1, W2 rows),
+//     4 per producer warp: a warp's gather copies leave it one after another
+//     at about 80 cycles each (measured), so one warp alone would cap a CTA
+//     at about 12 GB/s; and the operand blocks (16 x 64, hi and lo) as 2-D
+//     tiles;
+//   * warp 8 (one lane) issues the MMAs of each stage (tcgen05.mma kind::f16,
+//     bf16 inputs, fp32 accumulator in tensor memory) and commits them to the
+//     stage's "empty" barrier, which hands the stage back to the producers;
+//     at the end of a unit it commits the accumulator to the epilogue;
+//   * warps 9-12 read the 128 x 16 accumulator (tcgen05.ld 32x32b; warp w
+//     owns TMEM lanes 32 (w%4) ..) and run the unit's epilogue, while the
+//     MMAs of the next unit already run into the second accumulator (two
+//     16-column accumulators in 32 TMEM columns).
 // Every mbarrier wait is bounded (about 2 s of %globaltimer); on a timeout
-// the kernel sets DV_DEV_TIMEOUT in the status word, stops issuing work,
-// waits for its own copies, releases its tensor memory and returns.
+// the kernel sets DV_DEV_TIMEOUT in the status word, the other roles stop at
+// their next wait, the producers wait for their copies in flight, the MMA
+// warp for its MMAs, the tensor memory is released and the kernel returns.
 #pragma once
 
 #include "dv_common.cuh"
@@ -42,15 +51,18 @@
 
 namespace dv {
 
-constexpr int TC_THREADS = 128;
-constexpr int TC_K = 64;        // K elements per stage
-constexpr int TC_STAGES = 8;
-constexpr int TC_DIST = TC_STAGES - 2;  // stages in flight ahead of the one consumed
+constexpr int TC_PRODUCERS = 8;                    // warps that issue the copies
+constexpr int TC_MMA_WARP = TC_PRODUCERS;          // warp that issues the MMAs
+constexpr int TC_EPI_WARP0 = TC_PRODUCERS + 1;     // first of the four epilogue warps
+constexpr int TC_THREADS = (TC_PRODUCERS + 5) * 32;
+constexpr int TC_GATHERS_PER_WARP = 32 / TC_PRODUCERS;  // tile::gather4 copies per producer warp per stage
+constexpr int TC_K = 64;        // K elements per stage (128 bytes of a bf16 row: one swizzle span)
+constexpr int TC_STAGES_MAX = 10;  // ring stages with one CTA per SM (half with two)
 constexpr int TC_A_BYTES = TC_M * TC_K * 2;  // 16 KB weight tile
 constexpr int TC_B_BYTES = TC_N * TC_K * 2;  // 2 KB bf16 operand (hi or lo)
 constexpr int TC_STAGE_BYTES = TC_A_BYTES + 2 * TC_B_BYTES;
-constexpr size_t TC_SMEM = 1024 + (size_t)TC_STAGES * TC_STAGE_BYTES;
-constexpr int TC_TMEM_COLS = 32;
+__host__ __device__ constexpr size_t tc_smem(int stages) { return 1024 + (size_t)stages * TC_STAGE_BYTES; }
+constexpr int TC_TMEM_COLS = 32;       // two accumulators of TC_N columns
 constexpr int TC_TILES_PER_GROUP = 8;  // rowdot tiles per rowaxpy unit of the MLP (1024 neurons), at most
 constexpr int TC_HEADS_PER_GROUP = 4;  // heads per rowaxpy unit of W^O, at most
 
@@ -60,21 +72,6 @@ constexpr int TC_HEADS_PER_GROUP = 4;  // heads per rowaxpy unit of W^O, at most
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait_n() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_none() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
@@ -94,6 +91,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
   return ok != 0;
 }
 
+// One arrival that also announces `bytes` of asynchronous copies the phase
+// waits for.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -101,14 +107,36 @@ __device__ __forceinline__ uint64_t global_ns() {
 }
 
 // Waits for the phase with the given parity to complete, for at most about
-// two seconds; false on a timeout.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity) {
+// two seconds, or until *abort is set (by another role that gave up);
+// false in both cases.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, const volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   while (!mbar_try_wait(bar, parity)) {
+    if (abort && *abort) return false;
     if (global_ns() - t0 > 2000000000ull) return false;
   }
   return true;
+}
+
+// 2-D tensor tile load into shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Four rows r[0..3] (each one box of the map: TC_K columns from x) into
+// consecutive 128-byte rows of shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int x, const int (&r)[4],
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(smem_u32(bar))
+      : "memory");
 }
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst, int ncols) {
@@ -156,14 +184,34 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Shared-memory matrix descriptor, no swizzle (canonical layout of 8-row x
-// 16-byte core matrices): start address, the byte distance between core
-// matrices along K (lbo) and along M/N (sbo), descriptor version 1.
+// Barrier of the four epilogue warps (named barrier 1, 128 threads), and the
+// same barrier returning whether `ok` holds in all of them.
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ bool epi_all(bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)ok)
+      : "memory");
+  return r != 0;
+}
+
+// Shared-memory matrix descriptor of the 128-byte swizzled layouts (rows of
+// 128 bytes whose 16-byte pieces are permuted by the row index mod 8, in
+// atoms of 8 rows = 1024 bytes): start address, leading-dimension byte offset
+// (K-major: unused, 16; MN-major: the distance between 64-element blocks
+// along M), stride-dimension byte offset (the distance between 8-row groups),
+// descriptor version 1, layout type 2 (128-byte swizzle).
 __device__ __forceinline__ uint64_t tc_sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
   d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
   d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
   d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
   return d;
 }
 
@@ -175,74 +223,23 @@ __host__ __device__ constexpr uint32_t tc_idesc(int M, int N, int a_mn) {
 }
 
 // ---------------------------------------------------------------------------
-// Shared-memory stage layout (offsets inside one stage)
+// Shared-memory stage layout (offsets inside one 1024-aligned stage)
 // ---------------------------------------------------------------------------
-//   A    [0, 16 KB)      weight tile, canonical no-swizzle layout
-//   Bhi  [16, 18 KB)     operand hi part, [n/8][k/8][n%8][k%8] (K-major)
+//   A    [0, 16 KB)      weight tile
+//   Bhi  [16, 18 KB)     operand hi part: 16 batch rows x 64 K, K-major
 //   Blo  [18, 20 KB)     operand lo part
 //
-// rowdot A (K-major, 128 rows x 64 K): byte (m/8)*1024 + (k/8)*128 +
-// (m%8)*16 + (k%8)*2, so lbo = 128, sbo = 1024, and the K = 16 slice kk of
-// the stage starts at kk * 256.
-// rowaxpy A (MN-major, 128 columns x 64 K rows): byte (k/8)*2048 +
-// (m/8)*128 + (k%8)*16 + (m%8)*2, so sbo = 128, lbo = 2048, and the K = 16
-// slice kk starts at kk * 4096.
-// B (K-major, 16 x 64): byte (n/8)*1024 + (k/8)*128 + (n%8)*16 + (k%8)*2,
-// lbo = 128, sbo = 1024, slice kk at kk * 256.
+// rowdot A (K-major, 128 rows x 64 K): row m at m * 128 bytes (gather4 g
+// brings rows 4g..4g+3 to g * 512, a 64-row tile k to k * 8192); sbo = 1024;
+// the K = 16 slice kk of the
+// stage starts 32 kk bytes in (inside the swizzle span, as the hardware
+// applies the permutation to the address bits).
+// rowaxpy A (MN-major, 128 columns x 64 K rows): two blocks of 64 columns at
+// 0 and 8 KB, K row j of a block at j * 128 bytes; lbo = 8192, sbo = 1024;
+// the K = 16 slice kk starts at kk * 2048 (two 8-row groups).
+// B (K-major, 16 x 64): like rowdot A with 16 rows.
 constexpr int TC_OFF_BHI = TC_A_BYTES;
 constexpr int TC_OFF_BLO = TC_A_BYTES + TC_B_BYTES;
-
-// Copies the stage's operand blocks: batch row n (< nb, zero otherwise),
-// elements k0 .. k0+63 of hi[n * ld] and lo[n * ld], the first `valid` of
-// them (the rest zero; valid is a multiple of 8 or the tail of the row).
-// Thread t copies row t/8, 16-byte piece t%8, of both.
-__device__ __forceinline__ void tc_load_operand(unsigned char* stage, const __nv_bfloat16* hi,
-                                                const __nv_bfloat16* lo, long long ld, int nb, int k0, int valid) {
-  const int t = threadIdx.x;
-  const int n = t >> 3, k8 = t & 7;
-  const bool ok = n < nb && k8 * 8 < valid;
-  const long long off = ok ? (long long)n * ld + k0 + k8 * 8 : 0;
-  const int dst = (n >> 3) * 1024 + k8 * 128 + (n & 7) * 16;
-  cp_async16_zfill(stage + TC_OFF_BHI + dst, hi + off, ok ? 16 : 0);
-  cp_async16_zfill(stage + TC_OFF_BLO + dst, lo + off, ok ? 16 : 0);
-}
-
-// This thread's 8 rows of a tile (pointers; null: a zero row). rowdot:
-// piece j of thread t is tile row (t%8) + 8 (t/64) + 16 j, column piece
-// (t/8)%8; rowaxpy: chunk row (t%8) + 8 j, column piece (t/8)%16.
-__device__ __forceinline__ int tc_rowdot_row(int j) { return (threadIdx.x & 7) + 8 * (threadIdx.x >> 6) + 16 * j; }
-__device__ __forceinline__ int tc_rowaxpy_row(int j) { return (threadIdx.x & 7) + 8 * j; }
-
-// rowdot weight tile, K-major: columns k0 .. k0+63 of the 8 rows rp[j]
-// (columns >= d zero).
-__device__ __forceinline__ void tc_load_tile_kmajor(unsigned char* stage, const __nv_bfloat16* const (&rp)[8], int k0,
-                                                    int d, const void* dummy) {
-  const int t = threadIdx.x;
-  const int k8 = (t >> 3) & 7;
-  const int col = k0 + k8 * 8;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int m = tc_rowdot_row(j);
-    const bool ok = rp[j] != nullptr && col < d;
-    cp_async16_zfill(stage + (m >> 3) * 1024 + k8 * 128 + (m & 7) * 16, ok ? (const void*)(rp[j] + col) : dummy,
-                     ok ? 16 : 0);
-  }
-}
-
-// rowaxpy weight tile, MN-major: columns col0 .. col0+127 of the 8 rows rp[j]
-// (columns >= d zero).
-__device__ __forceinline__ void tc_load_tile_mnmajor(unsigned char* stage, const __nv_bfloat16* const (&rp)[8],
-                                                     int col0, int d, const void* dummy) {
-  const int t = threadIdx.x;
-  const int c8 = (t >> 3) & 15;
-  const int col = col0 + c8 * 8;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const bool ok = rp[j] != nullptr && col < d;
-    cp_async16_zfill(stage + j * 2048 + c8 * 128 + (t & 7) * 16, ok ? (const void*)(rp[j] + col) : dummy,
-                     ok ? 16 : 0);
-  }
-}
 
 // ---------------------------------------------------------------------------
 // The pipeline (shared by both forms)
@@ -250,131 +247,185 @@ __device__ __forceinline__ void tc_load_tile_mnmajor(unsigned char* stage, const
 //
 // A problem P provides:
 //   static constexpr int kAMajorMN;               // 0 rowdot, 1 rowaxpy
+//   static constexpr bool kGather;                // weight rows by gather4 (else by the first producer thread)
 //   static constexpr bool kRowsPerUnit;           // rows() depends on the unit only
 //   __device__ int units() const;                 // work units in total
 //   __device__ int chunks(int unit) const;        // stages of K in a unit (>= 1 for every unit)
-//   __device__ bool live(int unit, int c) const;  // false: the stage is empty (no copies, no MMA)
-//   __device__ void rows(int unit, int c, const bf16* (&rp)[8]) const;  // this thread's 8 weight rows
-//   __device__ void load(unsigned char* stage, int unit, int c, const bf16* const (&rp)[8]) const;
-//   __device__ void epilogue(int unit, int m, const float (&v)[16], bool any) const;
-// The epilogue is called by all 128 threads together (it may use
-// __syncthreads); thread m holds accumulator row m. `any` is false when the
-// unit issued no MMA (its accumulator is then taken as zero).
-//
-// Timeouts are agreed on with __syncthreads_or, so every thread leaves the
-// loop at the same barrier.
+//   __device__ bool live(int unit, int c) const;  // false: the stage is skipped (no copies, no MMA)
+//   __device__ bool any(int unit) const;          // some stage of the unit is live
+//   __device__ void rows(int unit, int c, int g, int (&r)[4]) const;   // gather g's 4 rows (kGather)
+//   __device__ void issue(uint32_t stage, uint64_t* full, int unit, int c, int g, const int (&r)[4]) const;
+//                                                 // gather g's copy (kGather), and with g = 0 the rest of the
+//                                                 // stage's copies (TC_STAGE_BYTES in all)
+//   __device__ void epilogue(int unit, int m, int q, const float (&v)[16], bool any) const;
+// The epilogue runs in the four epilogue warps together (it may use
+// epi_sync()); thread m holds accumulator row m (epilogue warp q = m / 32).
+// `any` is false when the unit issued no MMA (its accumulator is then zero).
 
 template <class P>
-__device__ void tc_run(const P& p, int* status) {
+__device__ void tc_run(const P& p, int* status, int stages) {
   extern __shared__ __align__(1024) unsigned char tc_smem_raw[];
-  __shared__ __align__(8) uint64_t bar_free[TC_STAGES];
-  __shared__ __align__(8) uint64_t bar_done;
+  __shared__ __align__(8) uint64_t bar_full[TC_STAGES_MAX];
+  __shared__ __align__(8) uint64_t bar_empty[TC_STAGES_MAX];
+  __shared__ __align__(8) uint64_t bar_acc_full[2];
+  __shared__ __align__(8) uint64_t bar_acc_empty[2];
+  __shared__ __align__(8) uint64_t bar_final;
   __shared__ uint32_t s_tmem;
+  __shared__ volatile int s_abort;
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t smem0 = smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  if (warp == 0) {
+  if (warp == TC_MMA_WARP) {
     tmem_alloc(&s_tmem, TC_TMEM_COLS);
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int s = 0; s < TC_STAGES; ++s) mbar_init(&bar_free[s], 1);
-    mbar_init(&bar_done, 1);
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&bar_full[s], 1);
+      mbar_init(&bar_empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&bar_acc_full[a], 1);
+      mbar_init(&bar_acc_empty[a], 4);
+    }
+    mbar_init(&bar_final, 1);
+    s_abort = 0;
     fence_mbar_init();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  constexpr uint32_t idesc = tc_idesc(TC_M, TC_N, P::kAMajorMN);
-  int abort_local = 0;
-
-  // this CTA's units are blockIdx.x, + gridDim.x, ...; its chunk sequence is
-  // the concatenation of their chunks, walked by the producer TC_DIST
-  // chunks ahead of the consumer
   const int nunits = p.units();
-  int prod_u = blockIdx.x, prod_c = 0;
-  int issued = 0;
-  const __nv_bfloat16* rp[8];
-  auto produce = [&]() {
-    if (prod_u < nunits) {
-      const int s = issued % TC_STAGES;
-      if (issued >= TC_STAGES && !mbar_wait_bounded(&bar_free[s], ((issued / TC_STAGES) - 1) & 1)) {
-        if (!abort_local) raise_status(status, DV_DEV_TIMEOUT_BIT);
-        abort_local = 1;
-      }
-      if (!abort_local && p.live(prod_u, prod_c)) {
-        if (!P::kRowsPerUnit || prod_c == 0) p.rows(prod_u, prod_c, rp);
-        p.load(smem + (size_t)s * TC_STAGE_BYTES, prod_u, prod_c, rp);
-      }
-      if (++prod_c >= p.chunks(prod_u)) {
-        prod_c = 0;
-        prod_u += gridDim.x;
-      }
-      ++issued;
-    }
-    cp_async_commit();
+  auto give_up = [&]() {
+    if (!s_abort) raise_status(status, DV_DEV_TIMEOUT_BIT);
+    s_abort = 1;
   };
-  for (int i = 0; i < TC_DIST; ++i) produce();
 
-  int u = blockIdx.x, c = 0;
-  int consumed = 0, units_done = 0;
-  bool unit_any = false;  // the current unit issued an MMA
-  while (u < nunits) {
-    produce();
-    cp_async_wait_n<TC_DIST>();
-    const int s = consumed % TC_STAGES;
-    unsigned char* stage = smem + (size_t)s * TC_STAGE_BYTES;
-    const bool live = p.live(u, c);
-    fence_proxy_async_smem();
-    tc_fence_before();
-    if (__syncthreads_or(abort_local)) break;
-    const bool last = c + 1 >= p.chunks(u);
-    if (tid == 0) {
-      tc_fence_after();
-      if (live) {
-        const uint32_t a0 = smem_u32(stage), b0 = smem_u32(stage + TC_OFF_BHI), l0 = smem_u32(stage + TC_OFF_BLO);
-#pragma unroll
-        for (int kk = 0; kk < TC_K / 16; ++kk) {
-          const uint64_t ad = P::kAMajorMN ? tc_sdesc(a0 + kk * 4096, 2048, 128) : tc_sdesc(a0 + kk * 256, 128, 1024);
-          tc_mma(tmem, ad, tc_sdesc(b0 + kk * 256, 128, 1024), idesc, (unit_any || kk > 0) ? 1u : 0u);
-          tc_mma(tmem, ad, tc_sdesc(l0 + kk * 256, 128, 1024), idesc, 1u);
+  if (warp < TC_PRODUCERS) {
+    // ---- producers: the CTA's live stages in order (units blockIdx.x,
+    // + gridDim.x, ...); every producer warp waits for a slot, lanes
+    // 0..TC_GATHERS_PER_WARP-1 issue one gather each (gather index g), and
+    // thread 0 also announces the stage's bytes and issues the rest. The
+    // gather rows of the next stage are loaded while waiting for its slot. ----
+    if (P::kGather || warp == 0) {
+      const int g = warp * TC_GATHERS_PER_WARP + lane;
+      const bool active = P::kGather ? lane < TC_GATHERS_PER_WARP : lane == 0;
+      auto next_live = [&](int& u, int& c) {
+        while (u < nunits) {
+          if (++c >= p.chunks(u)) {
+            u += gridDim.x;
+            c = -1;
+            continue;
+          }
+          if (p.live(u, c)) return;
+        }
+      };
+      int u = blockIdx.x, c = -1;
+      next_live(u, c);
+      int r[4] = {0, 0, 0, 0};
+      int ru = -1;
+      if (u < nunits && active && P::kGather) {
+        p.rows(u, c, g, r);
+        ru = u;
+      }
+      int issued = 0;
+      bool ok = true;
+      while (u < nunits) {
+        const int s = issued % stages;
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar_empty[s], ((issued / stages) & 1) ^ 1, &s_abort));
+        if (!ok) break;
+        if (tid == 0) mbar_expect_tx(&bar_full[s], TC_STAGE_BYTES);
+        if (active) p.issue(smem0 + (uint32_t)s * TC_STAGE_BYTES, &bar_full[s], u, c, g, r);
+        ++issued;
+        next_live(u, c);
+        if (u < nunits && active && P::kGather && (!P::kRowsPerUnit || u != ru)) {
+          p.rows(u, c, g, r);
+          ru = u;
         }
       }
-      tc_commit(&bar_free[s]);
-      if (last) tc_commit(&bar_done);
+      if (!ok && lane == 0) give_up();
+      // the copies of the last stages issued have landed before the CTA may
+      // exit (at once when the MMA warp consumed them)
+      if (lane == 0)
+        for (int i = issued > stages ? issued - stages : 0; i < issued; ++i)
+          mbar_wait(&bar_full[i % stages], (i / stages) & 1, nullptr);
     }
-    unit_any = unit_any || live;
-    ++consumed;
-    if (last) {
-      if (!mbar_wait_bounded(&bar_done, units_done & 1)) {
-        if (!abort_local) raise_status(status, DV_DEV_TIMEOUT_BIT);
-        abort_local = 1;
+  } else if (warp == TC_MMA_WARP) {
+    if (lane == 0) {
+      // ---- MMA issuer ----
+      constexpr uint32_t idesc = tc_idesc(TC_M, TC_N, P::kAMajorMN);
+      int consumed = 0, n = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++n) {
+        const int acc = n & 1;
+        if (!mbar_wait(&bar_acc_empty[acc], ((n >> 1) & 1) ^ 1, &s_abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dt = tmem + (uint32_t)(acc * TC_N);
+        bool first = true;
+        const int nc = p.chunks(u);
+        for (int c = 0; c < nc; ++c) {
+          if (!p.live(u, c)) continue;
+          const int s = consumed % stages;
+          if (!mbar_wait(&bar_full[s], (consumed / stages) & 1, &s_abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem0 + (uint32_t)s * TC_STAGE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < TC_K / 16; ++kk) {
+            const uint64_t ad =
+                P::kAMajorMN ? tc_sdesc(a0 + kk * 2048, 8192, 1024) : tc_sdesc(a0 + kk * 32, 16, 1024);
+            tc_mma(dt, ad, tc_sdesc(a0 + TC_OFF_BHI + kk * 32, 16, 1024), idesc, (!first || kk > 0) ? 1u : 0u);
+            tc_mma(dt, ad, tc_sdesc(a0 + TC_OFF_BLO + kk * 32, 16, 1024), idesc, 1u);
+          }
+          tc_commit(&bar_empty[s]);
+          ++consumed;
+          first = false;
+        }
+        if (!ok) break;
+        tc_commit(&bar_acc_full[acc]);
       }
-      if (__syncthreads_or(abort_local)) break;
+      if (!ok) give_up();
+      // every MMA issued has completed before the tensor memory is released
+      tc_commit(&bar_final);
+      mbar_wait(&bar_final, 0, nullptr);
+    }
+  } else {
+    // ---- epilogue warps: accumulator quarter q = warp % 4 ----
+    const int q = warp & 3;
+    int n = 0;
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++n) {
+      const int acc = n & 1;
+      const bool ok = epi_all(mbar_wait(&bar_acc_full[acc], (n >> 1) & 1, &s_abort));
+      if (!ok) {
+        if (warp == TC_EPI_WARP0 && lane == 0) give_up();
+        break;
+      }
       tc_fence_after();
+      const bool any = p.any(u);
       float v[16];
-      if (unit_any) {
-        tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16), v);
+      if (any) {
+        tmem_ld16(tmem + (uint32_t)(acc * TC_N) + ((uint32_t)(q * 32) << 16), v);
       } else {
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[i] = 0.f;
       }
-      p.epilogue(u, warp * 32 + lane, v, unit_any);
       tc_fence_before();
-      ++units_done;
-      unit_any = false;
-    }
-    if (++c >= p.chunks(u)) {
-      c = 0;
-      u += gridDim.x;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_acc_empty[acc]);
+      p.epilogue(u, q * 32 + lane, q, v, any);
     }
   }
-  cp_async_wait_none();
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == TC_MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, TC_TMEM_COLS);
   }
@@ -405,38 +456,49 @@ __global__ void __launch_bounds__(256) tc_split_kernel(TcSplitArgs a) {
   }
 }
 
+// The operand blocks of a stage: columns x .. x+63 of the 16 hi and lo rows.
+__device__ __forceinline__ void tc_issue_operand(const TcMaps& m, uint32_t stage, uint64_t* full, int x) {
+  tma_load_2d(stage + TC_OFF_BHI, &m.hi, x, 0, full);
+  tma_load_2d(stage + TC_OFF_BLO, &m.lo, x, 0, full);
+}
+
 // ---------------------------------------------------------------------------
 // q, k, v of the selected heads (rowdot over Wqkv rows)
 // ---------------------------------------------------------------------------
 
 struct TcQkvProblem {
   static constexpr int kAMajorMN = 0;
+  static constexpr bool kGather = false;
   static constexpr bool kRowsPerUnit = true;
+  const TcMaps& m;
   TcQkvArgs a;
   int nslots;  // selected heads x 3 dh
   __device__ int units() const { return (nslots + TC_M - 1) / TC_M; }
   __device__ int chunks(int) const { return (a.d + TC_K - 1) / TC_K; }
   __device__ bool live(int, int) const { return true; }
-  __device__ void rows(int unit, int, const __nv_bfloat16* (&rp)[8]) const {
+  __device__ bool any(int) const { return true; }
+  __device__ void rows(int, int, int, int (&)[4]) const {}
+  // the unit's 128 slots as two tiles of 64 consecutive Wqkv rows (3 dh is a
+  // multiple of 64, so a tile never spans two heads); slots past the
+  // selected ones, and invalid heads, read rows 0.. (their accumulator rows
+  // are not used)
+  __device__ void issue(uint32_t st, uint64_t* full, int unit, int c, int, const int (&)[4]) const {
     const int per = 3 * a.dh;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int s = unit * TC_M + tc_rowdot_row(j);
-      const __nv_bfloat16* r = nullptr;
-      if (s < nslots) {
-        const int head = a.head_idx[s / per];
-        if (head >= 0 && head < a.h) r = a.Wqkv + ((size_t)head * per + s % per) * a.d;
+    for (int k = 0; k < 2; ++k) {
+      const int s0 = unit * TC_M + 64 * k;
+      int y = 0;
+      if (s0 < nslots) {
+        const int head = a.head_idx[s0 / per];
+        if (head >= 0 && head < a.h) y = head * per + s0 % per;
       }
-      rp[j] = r;
+      tma_load_2d(st + k * 8192, &m.w, c * TC_K, y, full);
     }
+    tc_issue_operand(m, st, full, c * TC_K);
   }
-  __device__ void load(unsigned char* stage, int, int c, const __nv_bfloat16* const (&rp)[8]) const {
-    tc_load_tile_kmajor(stage, rp, c * TC_K, a.d, a.Wqkv);
-    tc_load_operand(stage, a.xhi, a.xlo, a.d, a.nb, c * TC_K, a.d - c * TC_K);
-  }
-  __device__ void epilogue(int unit, int m, const float (&v)[16], bool) const {
+  __device__ void epilogue(int unit, int mrow, int, const float (&v)[16], bool) const {
     const int per = 3 * a.dh;
-    const int s = unit * TC_M + m;
+    const int s = unit * TC_M + mrow;
     if (s >= nslots) return;
     const int p = s / per, rem = s % per, which = rem / a.dh, c = rem % a.dh;
     const int head = a.head_idx[p];
@@ -459,7 +521,7 @@ struct TcQkvProblem {
   }
 };
 
-__global__ void __launch_bounds__(TC_THREADS, 1) tc_qkv_kernel(TcQkvArgs a) {
+__global__ void __launch_bounds__(TC_THREADS, 2) tc_qkv_kernel(const __grid_constant__ TcMaps m, TcQkvArgs a) {
   griddep_launch();
   griddep_wait();
   int hc = *a.head_count;
@@ -467,8 +529,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_qkv_kernel(TcQkvArgs a) {
     if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(a.status, 1);
     hc = hc < 0 ? 0 : a.kh_max;
   }
-  TcQkvProblem p{a, hc * 3 * a.dh};
-  tc_run(p, a.status);
+  TcQkvProblem p{m, a, hc * 3 * a.dh};
+  tc_run(p, a.status, a.stages);
 }
 
 // ---------------------------------------------------------------------------
@@ -488,27 +550,31 @@ __device__ __forceinline__ int tc_clamped_count(const int32_t* count, int bound,
 
 struct TcW1Problem {
   static constexpr int kAMajorMN = 0;
+  static constexpr bool kGather = true;
   static constexpr bool kRowsPerUnit = true;
+  const TcMaps& m;
   TcMlpArgs a;
   int cnt;
-  int* s_warp;  // [4] shared: per-warp nonzero counts
+  int* s_warp;  // [4] shared: nonzero counts of the epilogue warps
   __device__ int units() const { return (cnt + TC_M - 1) / TC_M; }
   __device__ int chunks(int) const { return (a.d + TC_K - 1) / TC_K; }
   __device__ bool live(int, int) const { return true; }
-  __device__ void rows(int unit, int, const __nv_bfloat16* (&rp)[8]) const {
+  __device__ bool any(int) const { return true; }
+  // gather g: tile rows 4g .. 4g+3 (slots past the count read row 0)
+  __device__ void rows(int unit, int, int g, int (&r)[4]) const {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int s = unit * TC_M + tc_rowdot_row(j);
-      const int r = s < cnt ? a.idx[s] : -1;
-      rp[j] = (r >= 0 && r < a.N) ? a.W1t + (size_t)r * a.d : nullptr;
+    for (int i = 0; i < 4; ++i) {
+      const int s = unit * TC_M + 4 * g + i;
+      const int v = s < cnt ? a.idx[s] : 0;
+      r[i] = (v >= 0 && v < a.N) ? v : 0;
     }
   }
-  __device__ void load(unsigned char* stage, int, int c, const __nv_bfloat16* const (&rp)[8]) const {
-    tc_load_tile_kmajor(stage, rp, c * TC_K, a.d, a.W1t);
-    tc_load_operand(stage, a.xhi, a.xlo, a.d, a.nb, c * TC_K, a.d - c * TC_K);
+  __device__ void issue(uint32_t st, uint64_t* full, int, int c, int g, const int (&r)[4]) const {
+    tma_gather4(st + g * 512, &m.w, c * TC_K, r, full);
+    if (g == 0) tc_issue_operand(m, st, full, c * TC_K);
   }
-  __device__ void epilogue(int unit, int m, const float (&v)[16], bool) const {
-    const int s = unit * TC_M + m;
+  __device__ void epilogue(int unit, int mrow, int q, const float (&v)[16], bool) const {
+    const int s = unit * TC_M + mrow;
     int r = s < cnt ? a.idx[s] : -1;
     if (s < cnt && (r < 0 || r >= a.N)) {
       raise_status(a.status, 2);
@@ -522,54 +588,56 @@ struct TcW1Problem {
       act[b] = (r >= 0 && b < a.nb) ? activate(v[b] + bias, a.act) : 0.f;
       nz = nz || act[b] != 0.f;
     }
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
     const unsigned bal = __ballot_sync(0xffffffffu, nz);
-    if (lane == 0) s_warp[warp] = __popc(bal);
-    __syncthreads();
+    if (lane == 0) s_warp[q] = __popc(bal);
+    epi_sync();
     int before = 0, total = 0;
 #pragma unroll
-    for (int w = 0; w < TC_THREADS / 32; ++w) {
+    for (int w = 0; w < 4; ++w) {
       const int n = s_warp[w];
-      before += w < warp ? n : 0;
+      before += w < q ? n : 0;
       total += n;
     }
     const int base = unit * TC_M;
+    // all 16 rows are written (rows >= nb zero): the W2 operand loads read
+    // whole 16-row blocks
     if (nz) {  // the nonzero activations at their compacted slot
       const int slot = before + __popc(bal & ((1u << lane) - 1u));
 #pragma unroll
       for (int b = 0; b < TC_N; ++b) {
-        if (b >= a.nb) break;
         const __nv_bfloat16 h = __float2bfloat16_rn(act[b]);
         a.act_hi[(size_t)b * a.KC + base + slot] = h;
         a.act_lo[(size_t)b * a.KC + base + slot] = __float2bfloat16_rn(act[b] - __bfloat162float(h));
       }
       a.rowid_c[base + slot] = r;
     }
-    if (m >= total) {  // zeros after the tile's count (the W2 operand reads 8-slot pieces)
+    if (mrow >= total) {  // zeros after the tile's count (the W2 operand reads 64-slot pieces)
       const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
 #pragma unroll
       for (int b = 0; b < TC_N; ++b) {
-        if (b >= a.nb) break;
-        a.act_hi[(size_t)b * a.KC + base + m] = z;
-        a.act_lo[(size_t)b * a.KC + base + m] = z;
+        a.act_hi[(size_t)b * a.KC + base + mrow] = z;
+        a.act_lo[(size_t)b * a.KC + base + mrow] = z;
       }
     }
-    if (threadIdx.x == 0) a.tile_cnt[unit] = total;
-    __syncthreads();  // s_warp is reused by the next unit
+    if (mrow == 0) a.tile_cnt[unit] = total;
+    epi_sync();  // s_warp is reused by the next unit
   }
 };
 
-__global__ void __launch_bounds__(TC_THREADS, 1) tc_w1_kernel(TcMlpArgs a) {
-  __shared__ int s_warp[TC_THREADS / 32];
+__global__ void __launch_bounds__(TC_THREADS, 2) tc_w1_kernel(const __grid_constant__ TcMaps m, TcMlpArgs a) {
+  __shared__ int s_warp[4];
   griddep_launch();
   griddep_wait();
-  TcW1Problem p{a, tc_clamped_count(a.count, a.k_max, a.status), s_warp};
-  tc_run(p, a.status);
+  TcW1Problem p{m, a, tc_clamped_count(a.count, a.k_max, a.status), s_warp};
+  tc_run(p, a.status, a.stages);
 }
 
 struct TcW2Problem {
   static constexpr int kAMajorMN = 1;
+  static constexpr bool kGather = true;
   static constexpr bool kRowsPerUnit = false;
+  const TcMaps& m;
   TcMlpArgs a;
   int ntiles, n_mt, n_groups;
   const int* s_cnt;  // shared: tile_cnt of every tile
@@ -587,26 +655,34 @@ struct TcW2Problem {
     if ((c >> 1) >= tiles_in(g)) return false;
     return s_cnt[g * a.tiles_per_group + (c >> 1)] > (c & 1) * 64;
   }
-  __device__ void rows(int unit, int c, const __nv_bfloat16* (&rp)[8]) const {
+  __device__ bool any(int unit) const {
+    const int g = unit / n_mt, nt = tiles_in(g);
+    for (int t = 0; t < nt; ++t)
+      if (s_cnt[g * a.tiles_per_group + t] > 0) return true;
+    return false;
+  }
+  // gather g: K rows 4 (g % 16) .. +3 of the stage (the stage's 64
+  // compacted slots; slots past the tile's count read row 0, against zero
+  // activations), output columns 64 (g / 16) .. +63 of the unit's 128
+  __device__ void rows(int unit, int c, int g, int (&r)[4]) const {
     const int t = (unit / n_mt) * a.tiles_per_group + (c >> 1), half = c & 1;
     const int n = s_cnt[t] - half * 64;
-    const int base = t * TC_M + half * 64;
+    const int base = t * TC_M + half * 64, kr = 4 * (g & 15);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int kr = tc_rowaxpy_row(j);
-      rp[j] = kr < n ? a.W2t + (size_t)a.rowid_c[base + kr] * a.d : nullptr;
+    for (int i = 0; i < 4; ++i) {
+      const int v = kr + i < n ? a.rowid_c[base + kr + i] : 0;
+      r[i] = (v >= 0 && v < a.N) ? v : 0;
     }
   }
-  __device__ void load(unsigned char* stage, int unit, int c, const __nv_bfloat16* const (&rp)[8]) const {
+  __device__ void issue(uint32_t st, uint64_t* full, int unit, int c, int g, const int (&r)[4]) const {
     const int t = (unit / n_mt) * a.tiles_per_group + (c >> 1), half = c & 1;
-    const int n = s_cnt[t] - half * 64;  // > 0 (live)
-    tc_load_tile_mnmajor(stage, rp, (unit % n_mt) * TC_M, a.d, a.W2t);
-    const int valid = n < 64 ? (n + 7) & ~7 : 64;  // the slots after the count hold zeros
-    tc_load_operand(stage, a.act_hi, a.act_lo, a.KC, a.nb, t * TC_M + half * 64, valid);
+    const int mh = g >> 4;
+    tma_gather4(st + mh * 8192 + (g & 15) * 512, &m.w, (unit % n_mt) * TC_M + mh * 64, r, full);
+    if (g == 0) tc_issue_operand(m, st, full, t * TC_M + half * 64);
   }
-  __device__ void epilogue(int unit, int m, const float (&v)[16], bool any) const {
+  __device__ void epilogue(int unit, int mrow, int, const float (&v)[16], bool any) const {
     const int g = unit / n_mt, mt = unit % n_mt;
-    const int col = mt * TC_M + m;
+    const int col = mt * TC_M + mrow;
     if (col >= a.d) return;
     const float bias = (g == 0 && a.b2) ? a.b2[col] : 0.f;
     if (!any && bias == 0.f) return;
@@ -618,7 +694,7 @@ struct TcW2Problem {
   }
 };
 
-__global__ void __launch_bounds__(TC_THREADS, 1) tc_w2_kernel(TcMlpArgs a) {
+__global__ void __launch_bounds__(TC_THREADS, 2) tc_w2_kernel(const __grid_constant__ TcMaps m, TcMlpArgs a) {
   __shared__ int s_cnt[TC_MAX_TILES];
   griddep_launch();
   griddep_wait();
@@ -631,17 +707,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1) tc_w2_kernel(TcMlpArgs a) {
   __syncthreads();
   const int n_mt = (a.d + TC_M - 1) / TC_M;
   const int n_groups = ntiles > 0 ? (ntiles + a.tiles_per_group - 1) / a.tiles_per_group : 1;
-  TcW2Problem p{a, ntiles, n_mt, n_groups, s_cnt};
-  tc_run(p, a.status);
+  TcW2Problem p{m, a, ntiles, n_mt, n_groups, s_cnt};
+  tc_run(p, a.status, a.stages);
 }
 
 // ---------------------------------------------------------------------------
-// W^O of the selected heads (rowaxpy over WOt rows; operand H as hi / lo)
+// W^O of the selected heads (rowaxpy over WOt rows; operand H as hi / lo).
+// A head's dh rows are consecutive, so a stage's 64 K rows x 128 columns are
+// two plain 64 x 64 tiles.
 // ---------------------------------------------------------------------------
 
 struct TcWoProblem {
   static constexpr int kAMajorMN = 1;
-  static constexpr bool kRowsPerUnit = false;
+  static constexpr bool kGather = false;
+  static constexpr bool kRowsPerUnit = true;
+  const TcMaps& m;
   TcWoArgs a;
   int hc, n_mt, n_groups, cph;  // cph: 64-row chunks per head
   __device__ int units() const { return n_mt * n_groups; }
@@ -653,23 +733,31 @@ struct TcWoProblem {
     const int n = cph * heads_in(unit / n_mt);
     return n > 0 ? n : 1;
   }
-  __device__ bool live(int unit, int c) const { return c / cph < heads_in(unit / n_mt); }
-  __device__ void rows(int unit, int c, const __nv_bfloat16* (&rp)[8]) const {
-    const int p = (unit / n_mt) * a.heads_per_group + c / cph, part = c % cph;
+  __device__ bool head_ok(int p) const {
     const int head = a.head_idx[p];
-    const bool ok = head >= 0 && head < a.h;
-    const __nv_bfloat16* rows0 = a.WOt + ((size_t)(ok ? head : 0) * a.dh + part * 64) * a.d;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) rp[j] = ok ? rows0 + (size_t)tc_rowaxpy_row(j) * a.d : nullptr;
+    return head >= 0 && head < a.h;
   }
-  __device__ void load(unsigned char* stage, int unit, int c, const __nv_bfloat16* const (&rp)[8]) const {
+  __device__ bool live(int unit, int c) const {
+    const int g = unit / n_mt, j = c / cph;
+    return j < heads_in(g) && head_ok(g * a.heads_per_group + j);
+  }
+  __device__ bool any(int unit) const {
+    const int g = unit / n_mt, nh = heads_in(g);
+    for (int j = 0; j < nh; ++j)
+      if (head_ok(g * a.heads_per_group + j)) return true;
+    return false;
+  }
+  __device__ void rows(int, int, int, int (&)[4]) const {}
+  __device__ void issue(uint32_t st, uint64_t* full, int unit, int c, int, const int (&)[4]) const {
     const int p = (unit / n_mt) * a.heads_per_group + c / cph, part = c % cph;
-    tc_load_tile_mnmajor(stage, rp, (unit % n_mt) * TC_M, a.d, a.WOt);
-    tc_load_operand(stage, a.hhi, a.hlo, (long long)a.kh_max * a.dh, a.nb, p * a.dh + part * 64, 64);
+    const int y = a.head_idx[p] * a.dh + part * 64, x = (unit % n_mt) * TC_M;
+    tma_load_2d(st, &m.w, x, y, full);
+    tma_load_2d(st + 8192, &m.w, x + 64, y, full);
+    tc_issue_operand(m, st, full, p * a.dh + part * 64);
   }
-  __device__ void epilogue(int unit, int m, const float (&v)[16], bool any) const {
+  __device__ void epilogue(int unit, int mrow, int, const float (&v)[16], bool any) const {
     const int g = unit / n_mt, mt = unit % n_mt;
-    const int col = mt * TC_M + m;
+    const int col = mt * TC_M + mrow;
     if (col >= a.d) return;
     const float bias = (g == 0 && a.bO) ? a.bO[col] : 0.f;
     if (!any && bias == 0.f) return;
@@ -681,14 +769,62 @@ struct TcWoProblem {
   }
 };
 
-__global__ void __launch_bounds__(TC_THREADS, 1) tc_wo_kernel(TcWoArgs a) {
+__global__ void __launch_bounds__(TC_THREADS, 2) tc_wo_kernel(const __grid_constant__ TcMaps m, TcWoArgs a) {
   griddep_launch();
   griddep_wait();
   const int hc = tc_clamped_count(a.head_count, a.kh_max, a.status);
   const int n_mt = (a.d + TC_M - 1) / TC_M;
   const int n_groups = hc > 0 ? (hc + a.heads_per_group - 1) / a.heads_per_group : 1;
-  TcWoProblem p{a, hc, n_mt, n_groups, a.dh / 64};
-  tc_run(p, a.status);
+  TcWoProblem p{m, a, hc, n_mt, n_groups, a.dh / 64};
+  tc_run(p, a.status, a.stages);
+}
+
+// ---------------------------------------------------------------------------
+// Dense rowdot (rows of W consecutive, two 64-row tiles per stage), with the
+// K range of a 128-row tile split ks ways: unit u is tile u / ks, part u % ks
+// ---------------------------------------------------------------------------
+
+struct TcDenseProblem {
+  static constexpr int kAMajorMN = 0;
+  static constexpr bool kGather = false;
+  static constexpr bool kRowsPerUnit = true;
+  const TcMaps& m;
+  TcDenseArgs a;
+  int C;  // 64-column chunks of K
+  __device__ int units() const { return ((a.nrows + TC_M - 1) / TC_M) * a.ks; }
+  __device__ int c0(int unit) const { return (int)((long long)(unit % a.ks) * C / a.ks); }
+  __device__ int chunks(int unit) const { return (int)((long long)(unit % a.ks + 1) * C / a.ks) - c0(unit); }
+  __device__ bool live(int, int) const { return true; }
+  __device__ bool any(int) const { return true; }
+  __device__ void rows(int, int, int, int (&)[4]) const {}
+  __device__ void issue(uint32_t st, uint64_t* full, int unit, int c, int, const int (&)[4]) const {
+    const int y = (unit / a.ks) * TC_M, x = (c0(unit) + c) * TC_K;
+    tma_load_2d(st, &m.w, x, y, full);
+    tma_load_2d(st + 8192, &m.w, x, y + 64, full);
+    tc_issue_operand(m, st, full, x);
+  }
+  __device__ void epilogue(int unit, int mrow, int, const float (&v)[16], bool) const {
+    const int row = (unit / a.ks) * TC_M + mrow;
+    if (row >= a.nrows) return;
+    const float bias = (unit % a.ks == 0 && a.bias) ? a.bias[row] : 0.f;
+#pragma unroll
+    for (int b = 0; b < TC_N; ++b) {
+      if (b >= a.nb) break;
+      float* o = a.out + (size_t)b * a.ldo + row;
+      if (a.ks > 1) {
+        atomicAdd(o, v[b] + bias);
+      } else {
+        *o = v[b] + bias;
+      }
+    }
+  }
+};
+
+__global__ void __launch_bounds__(TC_THREADS, 2) tc_dense_kernel(const __grid_constant__ TcMaps m, TcDenseArgs a) {
+  griddep_launch();
+  griddep_wait();
+  TcDenseProblem p{m, a, (a.K + TC_K - 1) / TC_K};
+  tc_run(p, a.status, a.stages);
 }
 
 }  // namespace dv

@@ -2,6 +2,7 @@
 // (dv_tc.cuh), shared by the kernels and the host code that launches them.
 #pragma once
 
+#include <cuda.h>  // CUtensorMap
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -12,6 +13,13 @@ constexpr int TC_N = 16;          // batch rows, zero-padded
 constexpr int TC_MIN_B = 5;       // batch rows from which the layer calls use the tensor-core kernels
 constexpr int TC_MAX_TILES = 1024;  // tiles of 128 selected neurons (k_max <= 131072)
 constexpr int DV_DEV_TIMEOUT_BIT = 8;  // device status bit: a bounded wait ran out
+
+// TMA descriptors of one kernel (128-byte swizzle, bf16): the weight rows
+// (boxes of 64 columns x 1 row for gathered rows, 64 x 64 for W^O) and the
+// operand's hi and lo rows [16][ld] (boxes of 64 x 16).
+struct TcMaps {
+  CUtensorMap w, hi, lo;
+};
 
 struct TcQkvArgs {
   const __nv_bfloat16* Wqkv;  // [h][3][dh][d]
@@ -25,6 +33,7 @@ struct TcQkvArgs {
   __nv_bfloat16* Kc;          // [nb][h][cap][dh]
   __nv_bfloat16* Vc;
   int* status;
+  int stages;                 // ring stages (set by the launcher)
 };
 
 struct TcMlpArgs {
@@ -46,6 +55,7 @@ struct TcMlpArgs {
   float* out;                // [nb][d], accumulated into
   int* status;
   int act;                   // ACT_RELU or ACT_GELU
+  int stages;                // ring stages (set by the launcher)
 };
 
 struct TcWoArgs {
@@ -59,6 +69,19 @@ struct TcWoArgs {
   int heads_per_group;
   float* out;                // [nb][d], accumulated into
   int* status;
+  int stages;                // ring stages (set by the launcher)
+};
+
+// Dense rowdot over consecutive rows: out[b][row] (+)= W[row] . X[b] (+
+// bias[row]) for row < nrows, b < nb (the predictor's GEMMs at batch >= 3).
+struct TcDenseArgs {
+  const float* bias;  // [nrows] or null
+  int nrows, K, nb;
+  int ks;             // K splits per 128-row tile (> 1: out zeroed, partials added)
+  float* out;         // [nb][ldo]
+  long long ldo;
+  int* status;
+  int stages;         // ring stages (set by the launcher)
 };
 
 }  // namespace dv

@@ -8,8 +8,9 @@
 namespace dv {
 
 // Shapes the tensor-core path takes: bf16 weights, at most 16 batch rows,
-// dh a multiple of 64, at most 1024 tiles of 128 selected neurons.
-bool tc_shape_ok(int B, int wbytes, int dh, int k_max);
+// d >= 64 and a multiple of 8, dh a multiple of 64, at most 1024 tiles of 128
+// selected neurons; and a driver that encodes TMA descriptors.
+bool tc_shape_ok(int B, int d, int wbytes, int dh, int k_max);
 // Tiles of 128 selected neurons for a bound of k_max.
 int tc_tiles(int k_max);
 
@@ -20,5 +21,13 @@ cudaError_t run_tc_qkv(const TcQkvArgs& a, cudaStream_t st);
 // W1 + bias + ReLU with per-tile compaction, then the W2 gather-axpy into out.
 cudaError_t run_tc_mlp(TcMlpArgs a, cudaStream_t st);
 cudaError_t run_tc_wo(TcWoArgs a, cudaStream_t st);
+
+// The dense rowdot: out[b][row] (+)= W[row] . x[b] (+ bias[row]) for the
+// rows of W [nrows][K] (bf16) and the operand split into xhi / xlo [16][K];
+// out [nb][ldo] is written (or zeroed and accumulated into, when the K range
+// is split across CTAs).
+bool tc_dense_ok(int B, int wbytes, int nrows, int K);
+cudaError_t run_tc_dense(const __nv_bfloat16* W, int nrows, int K, const float* bias, const __nv_bfloat16* xhi,
+                         const __nv_bfloat16* xlo, int nb, float* out, long long ldo, int* status, cudaStream_t st);
 
 }  // namespace dv
