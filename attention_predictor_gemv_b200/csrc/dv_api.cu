@@ -29,7 +29,7 @@ constexpr int KH_LIMIT = 1000;  // B * kh_max counters must fit the header
 struct Layout {
   size_t status, sel_ticket_h, sel_ticket_m, pa_ticket, pb_ticket, attn_ctr, t1;
   size_t yA, yM, z, scores_h, bm_h, head_idx, head_count, scores, bm_m, idx, count;
-  size_t q, part, H, seg_idx, seg_a, seg_cnt, tc_x, tc_act, tc_rowid, tc_tiles, total;
+  size_t q, part, H, seg_idx, seg_a, seg_cnt, tc_x, tc_act, tc_rowid, tc_tiles, tc_red, tc_tick, total;
   int nseg, SEG, nsplit_max, KC, XC;
 };
 
@@ -83,6 +83,15 @@ Layout layout(const dv_dims& D, int wbytes) {
   L.tc_act = take(2ull * 2 * TC_N * (L.KC > 0 ? L.KC : 1));
   L.tc_rowid = take(4ull * (L.KC > 0 ? L.KC : 1));
   L.tc_tiles = take(4ull * (tiles > 0 ? tiles : 1));
+  // split-K partial sums (one [16][128] slot per unit) and tickets of the
+  // rowdot kernels: Q/K/V and W1 (up to 4 parts per tile), the predictor's
+  // dense GEMMs (up to TC_DENSE_PARTS units)
+  const long long qkv_tiles = ((long long)D.kh_max * 3 * D.dh + TC_M - 1) / TC_M;
+  long long red_tiles = qkv_tiles > tiles ? qkv_tiles : tiles;
+  const long long red_units = 4 * red_tiles > TC_DENSE_PARTS ? 4 * red_tiles : TC_DENSE_PARTS;
+  if (red_tiles < TC_DENSE_PARTS) red_tiles = TC_DENSE_PARTS;
+  L.tc_red = take(4ull * TC_N * TC_M * red_units);
+  L.tc_tick = take(4ull * red_tiles);
   L.total = o;
   return L;
 }
@@ -158,7 +167,8 @@ cudaError_t pred_tc(const Layout& L, void* ws, const void* W, int nrows, int K, 
   bf16* xlo = xhi + (size_t)TC_N * L.XC;
   cudaError_t e = run_tc_split(x, B, K, K, xhi, xlo, K, st);
   if (e != cudaSuccess) return e;
-  return run_tc_dense(static_cast<const bf16*>(W), nrows, K, bias, xhi, xlo, B, out, ldo, at<int>(ws, L.status), st);
+  return run_tc_dense(static_cast<const bf16*>(W), nrows, K, bias, xhi, xlo, B, out, ldo, at<float>(ws, L.tc_red),
+                      at<unsigned>(ws, L.tc_tick), at<int>(ws, L.status), st);
 }
 
 // The predictor's two stages: z = y A (predict_a_kernel family; rows of At
@@ -332,6 +342,8 @@ dv_status tc_mlp(const Layout& L, void* ws, const float* y, int B, int d, int N,
   a.act_lo = a.act_hi + (size_t)TC_N * (L.KC > 0 ? L.KC : 1);
   a.rowid_c = at<int32_t>(ws, L.tc_rowid);
   a.tile_cnt = at<int32_t>(ws, L.tc_tiles);
+  a.red = at<float>(ws, L.tc_red);
+  a.tick = at<unsigned>(ws, L.tc_tick);
   a.out = out;
   a.status = at<int>(ws, L.status);
   if (k_max > 0) DV_TRY(run_tc_split(y, B, d, d, xhi, xhi + (size_t)TC_N * L.XC, d, st));
@@ -360,6 +372,8 @@ dv_status tc_qkv(const Layout& L, void* ws, const float* y, int B, int d, int h,
   a.Kc = static_cast<bf16*>(Kc);
   a.Vc = static_cast<bf16*>(Vc);
   a.status = at<int>(ws, L.status);
+  a.red = at<float>(ws, L.tc_red);
+  a.tick = at<unsigned>(ws, L.tc_tick);
   DV_TRY(run_tc_split(y, B, d, d, xhi, xhi + (size_t)TC_N * L.XC, d, st));
   return cuda_status(run_tc_qkv(a, st));
 }

@@ -102,13 +102,16 @@ cudaError_t run_tc_split(const float* x, int nb, int n, long long ld_src, __nv_b
   return launch_main(tc_split_kernel, dim3(gx > 0 ? gx : 1, TC_N), dim3(256), 0, st, a);
 }
 
-cudaError_t run_tc_qkv(const TcQkvArgs& a, cudaStream_t st) {
-  const long long units = ((long long)a.kh_max * 3 * a.dh + TC_M - 1) / TC_M;
-  if (units == 0) return cudaSuccess;
+// The rowdot kernels split K on the device (tc_pick_ks, up to 4 parts): the
+// grid covers up to four units per tile.
+cudaError_t run_tc_qkv(TcQkvArgs a, cudaStream_t st) {
+  const long long tiles = ((long long)a.kh_max * 3 * a.dh + TC_M - 1) / TC_M;
+  if (tiles == 0) return cudaSuccess;
+  a.sms = sm_count();
   TcMaps m;
   cudaError_t e = tc_maps(&m, a.Wqkv, (long long)a.h * 3 * a.dh, a.d, 64, a.xhi, a.xlo, a.d, a.d);
   if (e != cudaSuccess) return e;
-  return launch_tc(tc_qkv_kernel, clamp_grid(units), st, m, a);
+  return launch_tc(tc_qkv_kernel, clamp_grid(tiles * 4), st, m, a);
 }
 
 cudaError_t run_tc_mlp(TcMlpArgs a, cudaStream_t st) {
@@ -117,8 +120,9 @@ cudaError_t run_tc_mlp(TcMlpArgs a, cudaStream_t st) {
   a.tiles_per_group = per_group(tiles, n_mt, TC_TILES_PER_GROUP);
   if (tiles > 0) {
     TcMaps m1;
+    a.sms = sm_count();
     cudaError_t e = tc_maps(&m1, a.W1t, a.N, a.d, 1, a.xhi, a.xlo, a.d, a.d);
-    if (e == cudaSuccess) e = launch_tc(tc_w1_kernel, clamp_grid(tiles), st, m1, a);
+    if (e == cudaSuccess) e = launch_tc(tc_w1_kernel, clamp_grid(4ll * tiles), st, m1, a);
     if (e != cudaSuccess) return e;
   }
   TcMaps m2;
@@ -144,27 +148,27 @@ bool tc_dense_ok(int B, int wbytes, int nrows, int K) {
 }
 
 cudaError_t run_tc_dense(const __nv_bfloat16* W, int nrows, int K, const float* bias, const __nv_bfloat16* xhi,
-                         const __nv_bfloat16* xlo, int nb, float* out, long long ldo, int* status, cudaStream_t st) {
+                         const __nv_bfloat16* xlo, int nb, float* out, long long ldo, float* red, unsigned* tick,
+                         int* status, cudaStream_t st) {
   const long long tiles = (nrows + TC_M - 1) / TC_M, C = (K + TC_K - 1) / TC_K;
   const long long slots = (long long)tc_ctas_per_sm() * sm_count();
-  long long ks = (slots + tiles - 1) / tiles;
-  if (ks > C) ks = C;
-  if (ks < 1) ks = 1;
+  long long want = (slots + tiles - 1) / tiles;
+  if (want > C) want = C;
+  if (want > TC_DENSE_PARTS / tiles) want = TC_DENSE_PARTS / tiles;
+  int kslog = 0;  // the largest power of two not above want
+  while ((2ll << kslog) <= want) ++kslog;
+  const long long ks = 1ll << kslog;
   TcDenseArgs a = {};
   a.bias = bias;
   a.nrows = nrows;
   a.K = K;
   a.nb = nb;
-  a.ks = (int)ks;
+  a.kslog = kslog;
   a.out = out;
   a.ldo = ldo;
   a.status = status;
-  if (ks > 1) {
-    for (int b = 0; b < nb; ++b) {
-      cudaError_t e = cudaMemsetAsync(out + (size_t)b * ldo, 0, sizeof(float) * (size_t)nrows, st);
-      if (e != cudaSuccess) return e;
-    }
-  }
+  a.red = red;
+  a.tick = tick;
   TcMaps m;
   cudaError_t e = tc_maps(&m, W, nrows, K, 64, xhi, xlo, K, K);
   if (e != cudaSuccess) return e;

@@ -313,17 +313,18 @@ __device__ void tc_run(const P& p, int* status, int stages) {
     if (P::kGather || warp == 0) {
       const int g = warp * TC_GATHERS_PER_WARP + lane;
       const bool active = P::kGather ? lane < TC_GATHERS_PER_WARP : lane == 0;
+      int u = blockIdx.x, c = -1, nc = u < nunits ? p.chunks(u) : 0;
       auto next_live = [&](int& u, int& c) {
         while (u < nunits) {
-          if (++c >= p.chunks(u)) {
+          if (++c >= nc) {
             u += gridDim.x;
             c = -1;
+            nc = u < nunits ? p.chunks(u) : 0;
             continue;
           }
           if (p.live(u, c)) return;
         }
       };
-      int u = blockIdx.x, c = -1;
       next_live(u, c);
       int r[4] = {0, 0, 0, 0};
       int ru = -1;
@@ -463,6 +464,68 @@ __device__ __forceinline__ void tc_issue_operand(const TcMaps& m, uint32_t stage
 }
 
 // ---------------------------------------------------------------------------
+// Split K for the rowdot kernels. A 128-row tile's K range is cut into ks
+// parts (units tile * ks + part), so that a tile count that does not fill the
+// CTAs evenly still keeps every SM streaming. ks is the same in every CTA:
+// chosen from the tile count on the device, for the grid's CTAs dealt
+// round-robin with CTAs c and c + sms on one SM, as the value of ks (1, 2, 4, at
+// most the chunks of K; a power of two, so that the unit arithmetic is
+// shifts) with the least per-SM work (3% added per extra part for the
+// reduction).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int tc_pick_kslog(int tiles, int C, int sms) {
+  const int G = gridDim.x;
+  int best_log = 0;
+  float best = 3.0e38f;
+  for (int lg = 0; lg <= 2 && (1 << lg) <= C; ++lg) {
+    const int ks = 1 << lg, units = tiles * ks, q = units / G, rem = units % G;
+    const int load = (q + (rem > 0 ? 1 : 0)) + (sms < G ? q + (rem > sms ? 1 : 0) : 0);
+    const float t = (float)load / (float)ks * (1.0f + 0.03f * (float)(ks - 1));
+    if (t < best) {
+      best = t;
+      best_log = lg;
+    }
+  }
+  return best_log;
+}
+
+// The epilogue threads' partial sums of `tile` (thread m: row m, v[b] for b <
+// nb) go into this part's own slot of red; the part that finishes the tile
+// last (ticket) sums the ks slots in part order into v, resets the ticket and
+// returns true in all 128 threads; the other parts return false. The sum is
+// the same whichever part arrives last, so results do not depend on timing
+// (the selections downstream compare scores exactly). With ks == 1 v is
+// already complete.
+__device__ __forceinline__ bool tc_reduce_parts(float* red, unsigned* tick, int tile, int part, int ks, int nb, int m,
+                                                float (&v)[16], int* s_flag) {
+  if (ks == 1) return true;
+  float* slot = red + ((size_t)tile * ks + part) * TC_N * TC_M;
+#pragma unroll
+  for (int b = 0; b < TC_N; ++b)
+    if (b < nb) slot[b * TC_M + m] = v[b];
+  __threadfence();
+  epi_sync();
+  if (m == 0) *s_flag = atomicAdd(tick + tile, 1u) == (unsigned)(ks - 1) ? 1 : 0;
+  epi_sync();
+  const bool last = *s_flag != 0;
+  if (last) {
+    __threadfence();
+    const float* t0 = red + (size_t)tile * ks * TC_N * TC_M;
+#pragma unroll
+    for (int b = 0; b < TC_N; ++b) {
+      if (b < nb) {
+        float sum = 0.f;
+        for (int p = 0; p < ks; ++p) sum += __ldcg(t0 + ((size_t)p * TC_N + b) * TC_M + m);
+        v[b] = sum;
+      }
+    }
+    if (m == 0) tick[tile] = 0u;
+  }
+  epi_sync();  // s_flag is reused by the next unit
+  return last;
+}
+
+// ---------------------------------------------------------------------------
 // q, k, v of the selected heads (rowdot over Wqkv rows)
 // ---------------------------------------------------------------------------
 
@@ -472,33 +535,41 @@ struct TcQkvProblem {
   static constexpr bool kRowsPerUnit = true;
   const TcMaps& m;
   TcQkvArgs a;
-  int nslots;  // selected heads x 3 dh
-  __device__ int units() const { return (nslots + TC_M - 1) / TC_M; }
-  __device__ int chunks(int) const { return (a.d + TC_K - 1) / TC_K; }
+  int nslots;      // selected heads x 3 dh
+  int C, kslog;    // 64-column chunks of d; log2 of the K parts per tile
+  int* s_flag;
+  __device__ int units() const { return ((nslots + TC_M - 1) / TC_M) << kslog; }
+  __device__ int c0(int unit) const { return ((unit & ((1 << kslog) - 1)) * C) >> kslog; }
+  __device__ int chunks(int unit) const { return ((((unit & ((1 << kslog) - 1)) + 1) * C) >> kslog) - c0(unit); }
   __device__ bool live(int, int) const { return true; }
   __device__ bool any(int) const { return true; }
   __device__ void rows(int, int, int, int (&)[4]) const {}
-  // the unit's 128 slots as two tiles of 64 consecutive Wqkv rows (3 dh is a
+  // the tile's 128 slots as two tiles of 64 consecutive Wqkv rows (3 dh is a
   // multiple of 64, so a tile never spans two heads); slots past the
   // selected ones, and invalid heads, read rows 0.. (their accumulator rows
   // are not used)
   __device__ void issue(uint32_t st, uint64_t* full, int unit, int c, int, const int (&)[4]) const {
-    const int per = 3 * a.dh;
+    const int per = 3 * a.dh, x = (c0(unit) + c) * TC_K;
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-      const int s0 = unit * TC_M + 64 * k;
+      const int s0 = (unit >> kslog) * TC_M + 64 * k;
       int y = 0;
       if (s0 < nslots) {
         const int head = a.head_idx[s0 / per];
         if (head >= 0 && head < a.h) y = head * per + s0 % per;
       }
-      tma_load_2d(st + k * 8192, &m.w, c * TC_K, y, full);
+      tma_load_2d(st + k * 8192, &m.w, x, y, full);
     }
-    tc_issue_operand(m, st, full, c * TC_K);
+    tc_issue_operand(m, st, full, x);
   }
-  __device__ void epilogue(int unit, int mrow, int, const float (&v)[16], bool) const {
+  __device__ void epilogue(int unit, int mrow, int, const float (&v0)[16], bool) const {
+    float v[16];
+#pragma unroll
+    for (int b = 0; b < 16; ++b) v[b] = v0[b];
+    const int tile = unit >> kslog;
+    if (!tc_reduce_parts(a.red, a.tick, tile, unit & ((1 << kslog) - 1), 1 << kslog, a.nb, mrow, v, s_flag)) return;
     const int per = 3 * a.dh;
-    const int s = unit * TC_M + mrow;
+    const int s = tile * TC_M + mrow;
     if (s >= nslots) return;
     const int p = s / per, rem = s % per, which = rem / a.dh, c = rem % a.dh;
     const int head = a.head_idx[p];
@@ -522,6 +593,7 @@ struct TcQkvProblem {
 };
 
 __global__ void __launch_bounds__(TC_THREADS, 2) tc_qkv_kernel(const __grid_constant__ TcMaps m, TcQkvArgs a) {
+  __shared__ int s_flag;
   griddep_launch();
   griddep_wait();
   int hc = *a.head_count;
@@ -529,7 +601,8 @@ __global__ void __launch_bounds__(TC_THREADS, 2) tc_qkv_kernel(const __grid_cons
     if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(a.status, 1);
     hc = hc < 0 ? 0 : a.kh_max;
   }
-  TcQkvProblem p{m, a, hc * 3 * a.dh};
+  const int nslots = hc * 3 * a.dh, C = (a.d + TC_K - 1) / TC_K;
+  TcQkvProblem p{m, a, nslots, C, tc_pick_kslog((nslots + TC_M - 1) / TC_M, C, a.sms), &s_flag};
   tc_run(p, a.status, a.stages);
 }
 
@@ -555,26 +628,35 @@ struct TcW1Problem {
   const TcMaps& m;
   TcMlpArgs a;
   int cnt;
-  int* s_warp;  // [4] shared: nonzero counts of the epilogue warps
-  __device__ int units() const { return (cnt + TC_M - 1) / TC_M; }
-  __device__ int chunks(int) const { return (a.d + TC_K - 1) / TC_K; }
+  int C, kslog;  // 64-column chunks of d; log2 of the K parts per tile
+  int* s_warp;   // [4] shared: nonzero counts of the epilogue warps
+  int* s_flag;
+  __device__ int units() const { return ((cnt + TC_M - 1) / TC_M) << kslog; }
+  __device__ int c0(int unit) const { return ((unit & ((1 << kslog) - 1)) * C) >> kslog; }
+  __device__ int chunks(int unit) const { return ((((unit & ((1 << kslog) - 1)) + 1) * C) >> kslog) - c0(unit); }
   __device__ bool live(int, int) const { return true; }
   __device__ bool any(int) const { return true; }
   // gather g: tile rows 4g .. 4g+3 (slots past the count read row 0)
   __device__ void rows(int unit, int, int g, int (&r)[4]) const {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int s = unit * TC_M + 4 * g + i;
+      const int s = (unit >> kslog) * TC_M + 4 * g + i;
       const int v = s < cnt ? a.idx[s] : 0;
       r[i] = (v >= 0 && v < a.N) ? v : 0;
     }
   }
-  __device__ void issue(uint32_t st, uint64_t* full, int, int c, int g, const int (&r)[4]) const {
-    tma_gather4(st + g * 512, &m.w, c * TC_K, r, full);
-    if (g == 0) tc_issue_operand(m, st, full, c * TC_K);
+  __device__ void issue(uint32_t st, uint64_t* full, int unit, int c, int g, const int (&r)[4]) const {
+    const int x = (c0(unit) + c) * TC_K;
+    tma_gather4(st + g * 512, &m.w, x, r, full);
+    if (g == 0) tc_issue_operand(m, st, full, x);
   }
-  __device__ void epilogue(int unit, int mrow, int q, const float (&v)[16], bool) const {
-    const int s = unit * TC_M + mrow;
+  __device__ void epilogue(int unit, int mrow, int q, const float (&v0)[16], bool) const {
+    float v[16];
+#pragma unroll
+    for (int b = 0; b < 16; ++b) v[b] = v0[b];
+    const int tile = unit >> kslog;
+    if (!tc_reduce_parts(a.red, a.tick, tile, unit & ((1 << kslog) - 1), 1 << kslog, a.nb, mrow, v, s_flag)) return;
+    const int s = tile * TC_M + mrow;
     int r = s < cnt ? a.idx[s] : -1;
     if (s < cnt && (r < 0 || r >= a.N)) {
       raise_status(a.status, 2);
@@ -599,7 +681,7 @@ struct TcW1Problem {
       before += w < q ? n : 0;
       total += n;
     }
-    const int base = unit * TC_M;
+    const int base = tile * TC_M;
     // all 16 rows are written (rows >= nb zero): the W2 operand loads read
     // whole 16-row blocks
     if (nz) {  // the nonzero activations at their compacted slot
@@ -620,16 +702,18 @@ struct TcW1Problem {
         a.act_lo[(size_t)b * a.KC + base + mrow] = z;
       }
     }
-    if (mrow == 0) a.tile_cnt[unit] = total;
+    if (mrow == 0) a.tile_cnt[tile] = total;
     epi_sync();  // s_warp is reused by the next unit
   }
 };
 
 __global__ void __launch_bounds__(TC_THREADS, 2) tc_w1_kernel(const __grid_constant__ TcMaps m, TcMlpArgs a) {
   __shared__ int s_warp[4];
+  __shared__ int s_flag;
   griddep_launch();
   griddep_wait();
-  TcW1Problem p{m, a, tc_clamped_count(a.count, a.k_max, a.status), s_warp};
+  const int cnt = tc_clamped_count(a.count, a.k_max, a.status), C = (a.d + TC_K - 1) / TC_K;
+  TcW1Problem p{m, a, cnt, C, tc_pick_kslog((cnt + TC_M - 1) / TC_M, C, a.sms), s_warp, &s_flag};
   tc_run(p, a.status, a.stages);
 }
 
@@ -781,7 +865,9 @@ __global__ void __launch_bounds__(TC_THREADS, 2) tc_wo_kernel(const __grid_const
 
 // ---------------------------------------------------------------------------
 // Dense rowdot (rows of W consecutive, two 64-row tiles per stage), with the
-// K range of a 128-row tile split ks ways: unit u is tile u / ks, part u % ks
+// K range of a 128-row tile split ks = 2^kslog ways: unit u is tile u / ks,
+// part u % ks
+// (the parts reduced in order by tc_reduce_parts)
 // ---------------------------------------------------------------------------
 
 struct TcDenseProblem {
@@ -791,39 +877,44 @@ struct TcDenseProblem {
   const TcMaps& m;
   TcDenseArgs a;
   int C;  // 64-column chunks of K
-  __device__ int units() const { return ((a.nrows + TC_M - 1) / TC_M) * a.ks; }
-  __device__ int c0(int unit) const { return (int)((long long)(unit % a.ks) * C / a.ks); }
-  __device__ int chunks(int unit) const { return (int)((long long)(unit % a.ks + 1) * C / a.ks) - c0(unit); }
+  int* s_flag;
+  __device__ int units() const { return ((a.nrows + TC_M - 1) / TC_M) << a.kslog; }
+  __device__ int c0(int unit) const { return ((unit & ((1 << a.kslog) - 1)) * C) >> a.kslog; }
+  __device__ int chunks(int unit) const {
+    return ((((unit & ((1 << a.kslog) - 1)) + 1) * C) >> a.kslog) - c0(unit);
+  }
   __device__ bool live(int, int) const { return true; }
   __device__ bool any(int) const { return true; }
   __device__ void rows(int, int, int, int (&)[4]) const {}
   __device__ void issue(uint32_t st, uint64_t* full, int unit, int c, int, const int (&)[4]) const {
-    const int y = (unit / a.ks) * TC_M, x = (c0(unit) + c) * TC_K;
+    const int y = (unit >> a.kslog) * TC_M, x = (c0(unit) + c) * TC_K;
     tma_load_2d(st, &m.w, x, y, full);
     tma_load_2d(st + 8192, &m.w, x, y + 64, full);
     tc_issue_operand(m, st, full, x);
   }
-  __device__ void epilogue(int unit, int mrow, int, const float (&v)[16], bool) const {
-    const int row = (unit / a.ks) * TC_M + mrow;
+  __device__ void epilogue(int unit, int mrow, int, const float (&v0)[16], bool) const {
+    float v[16];
+#pragma unroll
+    for (int b = 0; b < 16; ++b) v[b] = v0[b];
+    const int tile = unit >> a.kslog;
+    if (!tc_reduce_parts(a.red, a.tick, tile, unit & ((1 << a.kslog) - 1), 1 << a.kslog, a.nb, mrow, v, s_flag))
+      return;
+    const int row = tile * TC_M + mrow;
     if (row >= a.nrows) return;
-    const float bias = (unit % a.ks == 0 && a.bias) ? a.bias[row] : 0.f;
+    const float bias = a.bias ? a.bias[row] : 0.f;
 #pragma unroll
     for (int b = 0; b < TC_N; ++b) {
       if (b >= a.nb) break;
-      float* o = a.out + (size_t)b * a.ldo + row;
-      if (a.ks > 1) {
-        atomicAdd(o, v[b] + bias);
-      } else {
-        *o = v[b] + bias;
-      }
+      a.out[(size_t)b * a.ldo + row] = v[b] + bias;
     }
   }
 };
 
 __global__ void __launch_bounds__(TC_THREADS, 2) tc_dense_kernel(const __grid_constant__ TcMaps m, TcDenseArgs a) {
+  __shared__ int s_flag;
   griddep_launch();
   griddep_wait();
-  TcDenseProblem p{m, a, (a.K + TC_K - 1) / TC_K};
+  TcDenseProblem p{m, a, (a.K + TC_K - 1) / TC_K, &s_flag};
   tc_run(p, a.status, a.stages);
 }
 

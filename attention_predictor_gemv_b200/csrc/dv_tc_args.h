@@ -33,7 +33,10 @@ struct TcQkvArgs {
   __nv_bfloat16* Kc;          // [nb][h][cap][dh]
   __nv_bfloat16* Vc;
   int* status;
+  float* red;                 // [tiles][4][16][128] split-K partial sums
+  unsigned* tick;             // [tiles] parts finished per tile, zero between calls
   int stages;                 // ring stages (set by the launcher)
+  int sms;                    // SMs of the device (set by the launcher)
 };
 
 struct TcMlpArgs {
@@ -55,7 +58,10 @@ struct TcMlpArgs {
   float* out;                // [nb][d], accumulated into
   int* status;
   int act;                   // ACT_RELU or ACT_GELU
+  float* red;                // [tiles][4][16][128] split-K partial sums of W1
+  unsigned* tick;            // [tiles] parts finished per tile, zero between calls
   int stages;                // ring stages (set by the launcher)
+  int sms;                   // SMs of the device (set by the launcher)
 };
 
 struct TcWoArgs {
@@ -77,10 +83,12 @@ struct TcWoArgs {
 struct TcDenseArgs {
   const float* bias;  // [nrows] or null
   int nrows, K, nb;
-  int ks;             // K splits per 128-row tile (> 1: out zeroed, partials added)
+  int kslog;          // log2 of the K splits per 128-row tile
   float* out;         // [nb][ldo]
   long long ldo;
   int* status;
+  float* red;         // [tiles][2^kslog][16][128] split-K partial sums
+  unsigned* tick;     // [tiles] parts finished per tile, zero between calls
   int stages;         // ring stages (set by the launcher)
 };
 

@@ -17,17 +17,20 @@ int tc_tiles(int k_max);
 // hi / lo bf16 rows [16][ld_dst] of x [nb][n] (row stride ld_src); rows >= nb zero.
 cudaError_t run_tc_split(const float* x, int nb, int n, long long ld_src, __nv_bfloat16* hi, __nv_bfloat16* lo,
                          long long ld_dst, cudaStream_t st);
-cudaError_t run_tc_qkv(const TcQkvArgs& a, cudaStream_t st);
+cudaError_t run_tc_qkv(TcQkvArgs a, cudaStream_t st);
 // W1 + bias + ReLU with per-tile compaction, then the W2 gather-axpy into out.
 cudaError_t run_tc_mlp(TcMlpArgs a, cudaStream_t st);
 cudaError_t run_tc_wo(TcWoArgs a, cudaStream_t st);
 
-// The dense rowdot: out[b][row] (+)= W[row] . x[b] (+ bias[row]) for the
-// rows of W [nrows][K] (bf16) and the operand split into xhi / xlo [16][K];
-// out [nb][ldo] is written (or zeroed and accumulated into, when the K range
-// is split across CTAs).
+// The dense rowdot: out[b][row] = W[row] . x[b] (+ bias[row]) for the rows
+// of W [nrows][K] (bf16) and the operand split into xhi / xlo [16][K]; out
+// [nb][ldo]. When the K range is split across CTAs (at most TC_DENSE_PARTS
+// units of tiles x parts) the partial sums go through red [units][16][128]
+// and the per-tile tickets tick [tiles] (zero between calls).
+constexpr int TC_DENSE_PARTS = 512;
 bool tc_dense_ok(int B, int wbytes, int nrows, int K);
 cudaError_t run_tc_dense(const __nv_bfloat16* W, int nrows, int K, const float* bias, const __nv_bfloat16* xhi,
-                         const __nv_bfloat16* xlo, int nb, float* out, long long ldo, int* status, cudaStream_t st);
+                         const __nv_bfloat16* xlo, int nb, float* out, long long ldo, float* red, unsigned* tick,
+                         int* status, cudaStream_t st);
 
 }  // namespace dv
