@@ -29,7 +29,7 @@ constexpr int KH_LIMIT = 1000;  // B * kh_max counters must fit the header
 struct Layout {
   size_t status, sel_ticket_h, sel_ticket_m, pa_ticket, pb_ticket, attn_ctr, t1;
   size_t yA, yM, z, scores_h, bm_h, head_idx, head_count, scores, bm_m, idx, count;
-  size_t q, part, H, seg_idx, seg_a, seg_cnt, tc_x, tc_act, tc_rowid, tc_tiles, tc_red, tc_tick, total;
+  size_t q, part, H, seg_idx, seg_a, seg_cnt, tc_x, tc_act, tc_rowid, tc_tiles, tc_red, tc_tick, tc_acc, total;
   int nseg, SEG, nsplit_max, KC, XC;
 };
 
@@ -83,15 +83,13 @@ Layout layout(const dv_dims& D, int wbytes) {
   L.tc_act = take(2ull * 2 * TC_N * (L.KC > 0 ? L.KC : 1));
   L.tc_rowid = take(4ull * (L.KC > 0 ? L.KC : 1));
   L.tc_tiles = take(4ull * (tiles > 0 ? tiles : 1));
-  // split-K partial sums (one [16][128] slot per unit) and tickets of the
-  // rowdot kernels: Q/K/V and W1 (up to 4 parts per tile), the predictor's
-  // dense GEMMs (up to TC_DENSE_PARTS units)
-  const long long qkv_tiles = ((long long)D.kh_max * 3 * D.dh + TC_M - 1) / TC_M;
-  long long red_tiles = qkv_tiles > tiles ? qkv_tiles : tiles;
-  const long long red_units = 4 * red_tiles > TC_DENSE_PARTS ? 4 * red_tiles : TC_DENSE_PARTS;
-  if (red_tiles < TC_DENSE_PARTS) red_tiles = TC_DENSE_PARTS;
-  L.tc_red = take(4ull * TC_N * TC_M * red_units);
-  L.tc_tick = take(4ull * red_tiles);
+  // partial-sum slots ([16][128] each) and tickets of the tensor-core
+  // reductions: split K of Q/K/V, W1 and the predictor's dense GEMMs, and the
+  // row groups of W2 and W^O
+  L.tc_red = take(4ull * tc_red_floats(D.k_max, D.kh_max, D.dh, D.d));
+  L.tc_tick = take(4ull * tc_tick_count(D.k_max, D.kh_max, D.dh, D.d));
+  // fixed-point accumulator of the W2 and W^O partial sums [16][d]
+  L.tc_acc = take(8ull * TC_N * D.d);
   L.total = o;
   return L;
 }
@@ -344,6 +342,7 @@ dv_status tc_mlp(const Layout& L, void* ws, const float* y, int B, int d, int N,
   a.tile_cnt = at<int32_t>(ws, L.tc_tiles);
   a.red = at<float>(ws, L.tc_red);
   a.tick = at<unsigned>(ws, L.tc_tick);
+  a.acc = at<unsigned long long>(ws, L.tc_acc);
   a.out = out;
   a.status = at<int>(ws, L.status);
   if (k_max > 0) DV_TRY(run_tc_split(y, B, d, d, xhi, xhi + (size_t)TC_N * L.XC, d, st));
@@ -395,6 +394,7 @@ dv_status tc_wo(const Layout& L, void* ws, int B, int d, int h, int dh, const vo
   a.nb = B;
   a.out = out;
   a.status = at<int>(ws, L.status);
+  a.acc = at<unsigned long long>(ws, L.tc_acc);
   if (kh_max > 0)
     DV_TRY(run_tc_split(at<float>(ws, L.H), B, kh_max * dh, (long long)kh_max * dh, hhi, hhi + (size_t)TC_N * L.XC,
                         (long long)kh_max * dh, st));

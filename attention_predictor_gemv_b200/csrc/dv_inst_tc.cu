@@ -37,12 +37,6 @@ int clamp_grid(long long units) {
   return (int)(units < 1 ? 1 : (units > cap ? cap : units));
 }
 
-// Rows (tiles, heads) per rowaxpy unit: as many as still give every CTA two
-// units at the largest count, at most `most`.
-int per_group(long long items_max, long long n_mt, int most) {
-  long long g = items_max * n_mt / (2ll * tc_ctas_per_sm() * sm_count());
-  return (int)(g < 1 ? 1 : (g > most ? most : g));
-}
 
 // cuTensorMapEncodeTiled, from the driver the runtime is bound to (no link
 // against libcuda).
@@ -95,6 +89,39 @@ bool tc_shape_ok(int B, int d, int wbytes, int dh, int k_max) {
 
 int tc_tiles(int k_max) { return (k_max + TC_M - 1) / TC_M; }
 
+int tc_axpy_group(int items_max, int d, int most) {
+  const long long n_mt = (d + TC_M - 1) / TC_M;
+  const long long g = (long long)items_max * n_mt / (2ll * tc_ctas_per_sm() * sm_count());
+  return (int)(g < 1 ? 1 : (g > most ? most : g));
+}
+
+size_t tc_red_floats(int k_max, int kh_max, int dh, int d) {
+  const long long tiles = tc_tiles(k_max), qkv = ((long long)kh_max * 3 * dh + TC_M - 1) / TC_M;
+  long long slots = TC_DENSE_PARTS;
+  if (8 * tiles > slots) slots = 8 * tiles;
+  if (8 * qkv > slots) slots = 8 * qkv;
+  (void)d;
+  return (size_t)slots * TC_N * TC_M;
+}
+
+size_t tc_tick_count(int k_max, int kh_max, int dh, int d) {
+  long long n = TC_DENSE_PARTS;
+  const long long cand[2] = {tc_tiles(k_max), ((long long)kh_max * 3 * dh + TC_M - 1) / TC_M};
+  for (long long c : cand) n = c > n ? c : n;
+  (void)d;
+  return (size_t)n;
+}
+
+namespace {
+// out[b][:] += the fixed-point totals in acc (+ bias); acc back to zero
+cudaError_t run_tc_finalize(unsigned long long* acc, const float* bias, float* out, int nb, int d, cudaStream_t st) {
+  TcFinalizeArgs f{acc, bias, out, nb, d};
+  const long long n = (long long)nb * d, cap = 2ll * sm_count();
+  const long long g = (n + 255) / 256;
+  return launch_main(tc_finalize_kernel, dim3((unsigned)(g < 1 ? 1 : (g > cap ? cap : g))), dim3(256), 0, st, f);
+}
+}  // namespace
+
 cudaError_t run_tc_split(const float* x, int nb, int n, long long ld_src, __nv_bfloat16* hi, __nv_bfloat16* lo,
                          long long ld_dst, cudaStream_t st) {
   TcSplitArgs a{x, nb, n, ld_src, hi, lo, ld_dst};
@@ -102,45 +129,47 @@ cudaError_t run_tc_split(const float* x, int nb, int n, long long ld_src, __nv_b
   return launch_main(tc_split_kernel, dim3(gx > 0 ? gx : 1, TC_N), dim3(256), 0, st, a);
 }
 
-// The rowdot kernels split K on the device (tc_pick_ks, up to 4 parts): the
-// grid covers up to four units per tile.
+// The rowdot kernels split K on the device (tc_pick_kslog, up to 8 parts):
+// the grid covers up to eight units per tile.
 cudaError_t run_tc_qkv(TcQkvArgs a, cudaStream_t st) {
   const long long tiles = ((long long)a.kh_max * 3 * a.dh + TC_M - 1) / TC_M;
   if (tiles == 0) return cudaSuccess;
-  a.sms = sm_count();
   TcMaps m;
   cudaError_t e = tc_maps(&m, a.Wqkv, (long long)a.h * 3 * a.dh, a.d, 64, a.xhi, a.xlo, a.d, a.d);
   if (e != cudaSuccess) return e;
-  return launch_tc(tc_qkv_kernel, clamp_grid(tiles * 4), st, m, a);
+  return launch_tc(tc_qkv_kernel, clamp_grid(tiles * 8), st, m, a);
 }
 
 cudaError_t run_tc_mlp(TcMlpArgs a, cudaStream_t st) {
   const int tiles = tc_tiles(a.k_max);
   const int n_mt = (a.d + TC_M - 1) / TC_M;
-  a.tiles_per_group = per_group(tiles, n_mt, TC_TILES_PER_GROUP);
+  a.tiles_per_group = tc_axpy_group(tiles, a.d, 8);
   if (tiles > 0) {
     TcMaps m1;
-    a.sms = sm_count();
     cudaError_t e = tc_maps(&m1, a.W1t, a.N, a.d, 1, a.xhi, a.xlo, a.d, a.d);
-    if (e == cudaSuccess) e = launch_tc(tc_w1_kernel, clamp_grid(4ll * tiles), st, m1, a);
+    if (e == cudaSuccess) e = launch_tc(tc_w1_kernel, clamp_grid(8ll * tiles), st, m1, a);
     if (e != cudaSuccess) return e;
   }
   TcMaps m2;
   cudaError_t e = tc_maps(&m2, a.W2t, a.N, a.d, 1, a.act_hi, a.act_lo, a.KC > 0 ? a.KC : TC_M, a.KC > 0 ? a.KC : TC_M);
   if (e != cudaSuccess) return e;
   const long long groups = tiles > 0 ? (tiles + a.tiles_per_group - 1) / a.tiles_per_group : 1;
-  return launch_tc(tc_w2_kernel, clamp_grid(groups * n_mt), st, m2, a);
+  e = launch_tc(tc_w2_kernel, clamp_grid(groups * n_mt), st, m2, a);
+  if (e != cudaSuccess) return e;
+  return run_tc_finalize(a.acc, a.b2, a.out, a.nb, a.d, st);
 }
 
 cudaError_t run_tc_wo(TcWoArgs a, cudaStream_t st) {
   const int n_mt = (a.d + TC_M - 1) / TC_M;
-  a.heads_per_group = per_group(a.kh_max, n_mt, TC_HEADS_PER_GROUP);
+  a.heads_per_group = tc_axpy_group(a.kh_max, a.d, 4);
   const long long groups = a.kh_max > 0 ? (a.kh_max + a.heads_per_group - 1) / a.heads_per_group : 1;
   const long long ldh = (long long)(a.kh_max > 0 ? a.kh_max : 1) * a.dh;
   TcMaps m;
   cudaError_t e = tc_maps(&m, a.WOt, (long long)a.h * a.dh, a.d, 64, a.hhi, a.hlo, ldh, ldh);
   if (e != cudaSuccess) return e;
-  return launch_tc(tc_wo_kernel, clamp_grid(groups * n_mt), st, m, a);
+  e = launch_tc(tc_wo_kernel, clamp_grid(groups * n_mt), st, m, a);
+  if (e != cudaSuccess) return e;
+  return run_tc_finalize(a.acc, a.bO, a.out, a.nb, a.d, st);
 }
 
 bool tc_dense_ok(int B, int wbytes, int nrows, int K) {

@@ -11,7 +11,11 @@
 //   rowdot  D[m][b] = sum_c W[row(m)][c] X[b][c]    rows of W are K-major
 //           (q, k, v of the selected heads; the MLP's first layer)
 //   rowaxpy D[c][b] = sum_j W[row(j)][c] S[b][j]    rows of W are MN-major
-//           (W^O of the selected heads; the MLP's second layer)
+//           (W^O of the selected heads; the MLP's second layer); a unit is a
+//           group of rows times 128 output columns, and the groups' partials
+//           are summed as 64-bit fixed-point integers (exact, so the sum does
+//           not depend on the order in which CTAs finish; tc_acc_fixed) and
+//           added into the output once by tc_finalize_kernel
 // with M = 128 (gathered rows, or output columns), N = 16 (the batch rows,
 // zero-padded) and 64 K-elements per pipeline stage.
 //
@@ -23,15 +27,16 @@
 //
 // Per CTA (416 threads, one CTA per SM, persistent over work units), three
 // roles that meet only at mbarriers:
-//   * warps 0-7 fill a ring of `stages` stages with TMA copies, in the
-//     128-byte swizzled layout the MMA reads, completing on the stage's
-//     "full" barrier: the weight tile (16 KB) as two plain 2-D tiles of 64
-//     rows where the rows are consecutive (a head's Q/K/V or W^O rows), else
-//     by 32 tile::gather4 loads of 4 gathered rows x 64 columns (W1, W2 rows),
-//     4 per producer warp: a warp's gather copies leave it one after another
-//     at about 80 cycles each (measured), so one warp alone would cap a CTA
-//     at about 12 GB/s; and the operand blocks (16 x 64, hi and lo) as 2-D
-//     tiles;
+//   * warps 0-7 fill a ring of `stages` stages, in the 128-byte swizzled
+//     layout the MMA reads, completing on the stage's "full" barrier: the
+//     weight tile (16 KB) as two TMA 2-D tiles of 64 rows where the rows are
+//     consecutive (a head's Q/K/V or W^O rows), else (gathered W1, W2 rows)
+//     by 16-byte cp.async copies of all 256 producer threads into their
+//     swizzled places, each thread's completion counted on the barrier
+//     (cp.async.mbarrier.arrive); and the operand blocks (16 x 64, hi and
+//     lo) as TMA 2-D tiles. TMA tile::gather4 for the gathered rows was
+//     measured at about 25 GB/s per SM (about 40 cycles per 4-row copy
+//     however many warps issue them), below the SM's share of HBM;
 //   * warp 8 (one lane) issues the MMAs of each stage (tcgen05.mma kind::f16,
 //     bf16 inputs, fp32 accumulator in tensor memory) and commits them to the
 //     stage's "empty" barrier, which hands the stage back to the producers;
@@ -55,7 +60,7 @@ constexpr int TC_PRODUCERS = 8;                    // warps that issue the copie
 constexpr int TC_MMA_WARP = TC_PRODUCERS;          // warp that issues the MMAs
 constexpr int TC_EPI_WARP0 = TC_PRODUCERS + 1;     // first of the four epilogue warps
 constexpr int TC_THREADS = (TC_PRODUCERS + 5) * 32;
-constexpr int TC_GATHERS_PER_WARP = 32 / TC_PRODUCERS;  // tile::gather4 copies per producer warp per stage
+constexpr int TC_PRODUCER_THREADS = TC_PRODUCERS * 32;
 constexpr int TC_K = 64;        // K elements per stage (128 bytes of a bf16 row: one swizzle span)
 constexpr int TC_STAGES_MAX = 10;  // ring stages with one CTA per SM (half with two)
 constexpr int TC_A_BYTES = TC_M * TC_K * 2;  // 16 KB weight tile
@@ -63,8 +68,6 @@ constexpr int TC_B_BYTES = TC_N * TC_K * 2;  // 2 KB bf16 operand (hi or lo)
 constexpr int TC_STAGE_BYTES = TC_A_BYTES + 2 * TC_B_BYTES;
 __host__ __device__ constexpr size_t tc_smem(int stages) { return 1024 + (size_t)stages * TC_STAGE_BYTES; }
 constexpr int TC_TMEM_COLS = 32;       // two accumulators of TC_N columns
-constexpr int TC_TILES_PER_GROUP = 8;  // rowdot tiles per rowaxpy unit of the MLP (1024 neurons), at most
-constexpr int TC_HEADS_PER_GROUP = 4;  // heads per rowaxpy unit of W^O, at most
 
 // ---------------------------------------------------------------------------
 // PTX wrappers
@@ -128,15 +131,23 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// Four rows r[0..3] (each one box of the map: TC_K columns from x) into
-// consecutive 128-byte rows of shared memory, completing on `bar`.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int x, const int (&r)[4],
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(smem_u32(bar))
-      : "memory");
+// 16-byte copy global -> shared through L2 (cp.async), the first src_bytes
+// of it read and the rest zero (src_bytes 0: nothing is read).
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+// One arrival on `bar` (counted in its expected arrivals) once every
+// cp.async this thread issued before has landed.
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// The MMA reads shared memory through the async proxy; the copies above
+// wrote it through the generic one.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst, int ncols) {
@@ -247,16 +258,18 @@ constexpr int TC_OFF_BLO = TC_A_BYTES + TC_B_BYTES;
 //
 // A problem P provides:
 //   static constexpr int kAMajorMN;               // 0 rowdot, 1 rowaxpy
-//   static constexpr bool kGather;                // weight rows by gather4 (else by the first producer thread)
+//   static constexpr bool kGather;                // weight rows by the producers' cp.async (else TMA tiles
+//                                                 // issued by producer thread 0)
 //   static constexpr bool kRowsPerUnit;           // rows() depends on the unit only
 //   __device__ int units() const;                 // work units in total
 //   __device__ int chunks(int unit) const;        // stages of K in a unit (>= 1 for every unit)
 //   __device__ bool live(int unit, int c) const;  // false: the stage is skipped (no copies, no MMA)
 //   __device__ bool any(int unit) const;          // some stage of the unit is live
-//   __device__ void rows(int unit, int c, int g, int (&r)[4]) const;   // gather g's 4 rows (kGather)
-//   __device__ void issue(uint32_t stage, uint64_t* full, int unit, int c, int g, const int (&r)[4]) const;
-//                                                 // gather g's copy (kGather), and with g = 0 the rest of the
-//                                                 // stage's copies (TC_STAGE_BYTES in all)
+//   __device__ void rows(int unit, int c, int t, int (&r)[4]) const;   // producer thread t's rows (kGather;
+//                                                 // -1: zero-filled)
+//   __device__ void issue(uint32_t stage, uint64_t* full, int unit, int c, int t, const int (&r)[4]) const;
+//                                                 // thread t's copies (kGather), and with t = 0 the stage's
+//                                                 // TMA copies (tiles and operands)
 //   __device__ void epilogue(int unit, int m, int q, const float (&v)[16], bool any) const;
 // The epilogue runs in the four epilogue warps together (it may use
 // epi_sync()); thread m holds accumulator row m (epilogue warp q = m / 32).
@@ -283,7 +296,7 @@ __device__ void tc_run(const P& p, int* status, int stages) {
   }
   if (tid == 0) {
     for (int s = 0; s < stages; ++s) {
-      mbar_init(&bar_full[s], 1);
+      mbar_init(&bar_full[s], P::kGather ? TC_PRODUCER_THREADS + 1 : 1);
       mbar_init(&bar_empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -306,13 +319,14 @@ __device__ void tc_run(const P& p, int* status, int stages) {
 
   if (warp < TC_PRODUCERS) {
     // ---- producers: the CTA's live stages in order (units blockIdx.x,
-    // + gridDim.x, ...); every producer warp waits for a slot, lanes
-    // 0..TC_GATHERS_PER_WARP-1 issue one gather each (gather index g), and
-    // thread 0 also announces the stage's bytes and issues the rest. The
-    // gather rows of the next stage are loaded while waiting for its slot. ----
+    // + gridDim.x, ...); every producer warp waits for a slot; with gathered
+    // rows all 256 producer threads copy (thread t), otherwise thread 0
+    // alone; thread 0 also announces the stage's TMA bytes and issues those
+    // copies. The rows of the next stage are loaded while waiting for its
+    // slot. ----
     if (P::kGather || warp == 0) {
-      const int g = warp * TC_GATHERS_PER_WARP + lane;
-      const bool active = P::kGather ? lane < TC_GATHERS_PER_WARP : lane == 0;
+      const int t = tid;
+      const bool active = P::kGather || lane == 0;
       int u = blockIdx.x, c = -1, nc = u < nunits ? p.chunks(u) : 0;
       auto next_live = [&](int& u, int& c) {
         while (u < nunits) {
@@ -326,10 +340,10 @@ __device__ void tc_run(const P& p, int* status, int stages) {
         }
       };
       next_live(u, c);
-      int r[4] = {0, 0, 0, 0};
+      int r[4] = {-1, -1, -1, -1};
       int ru = -1;
-      if (u < nunits && active && P::kGather) {
-        p.rows(u, c, g, r);
+      if (u < nunits && P::kGather) {
+        p.rows(u, c, t, r);
         ru = u;
       }
       int issued = 0;
@@ -338,18 +352,20 @@ __device__ void tc_run(const P& p, int* status, int stages) {
         const int s = issued % stages;
         ok = __all_sync(0xffffffffu, mbar_wait(&bar_empty[s], ((issued / stages) & 1) ^ 1, &s_abort));
         if (!ok) break;
-        if (tid == 0) mbar_expect_tx(&bar_full[s], TC_STAGE_BYTES);
-        if (active) p.issue(smem0 + (uint32_t)s * TC_STAGE_BYTES, &bar_full[s], u, c, g, r);
+        if (tid == 0) mbar_expect_tx(&bar_full[s], P::kGather ? 2 * TC_B_BYTES : TC_STAGE_BYTES);
+        if (active) p.issue(smem0 + (uint32_t)s * TC_STAGE_BYTES, &bar_full[s], u, c, t, r);
+        if (P::kGather) cp_async_arrive(&bar_full[s]);
         ++issued;
         next_live(u, c);
-        if (u < nunits && active && P::kGather && (!P::kRowsPerUnit || u != ru)) {
-          p.rows(u, c, g, r);
+        if (u < nunits && P::kGather && (!P::kRowsPerUnit || u != ru)) {
+          p.rows(u, c, t, r);
           ru = u;
         }
       }
       if (!ok && lane == 0) give_up();
       // the copies of the last stages issued have landed before the CTA may
       // exit (at once when the MMA warp consumed them)
+      if (P::kGather) cp_async_wait_all();
       if (lane == 0)
         for (int i = issued > stages ? issued - stages : 0; i < issued; ++i)
           mbar_wait(&bar_full[i % stages], (i / stages) & 1, nullptr);
@@ -377,6 +393,7 @@ __device__ void tc_run(const P& p, int* status, int stages) {
             ok = false;
             break;
           }
+          if (P::kGather) fence_proxy_async_smem();
           tc_fence_after();
           const uint32_t a0 = smem0 + (uint32_t)s * TC_STAGE_BYTES;
 #pragma unroll
@@ -466,21 +483,19 @@ __device__ __forceinline__ void tc_issue_operand(const TcMaps& m, uint32_t stage
 // ---------------------------------------------------------------------------
 // Split K for the rowdot kernels. A 128-row tile's K range is cut into ks
 // parts (units tile * ks + part), so that a tile count that does not fill the
-// CTAs evenly still keeps every SM streaming. ks is the same in every CTA:
-// chosen from the tile count on the device, for the grid's CTAs dealt
-// round-robin with CTAs c and c + sms on one SM, as the value of ks (1, 2, 4, at
-// most the chunks of K; a power of two, so that the unit arithmetic is
-// shifts) with the least per-SM work (3% added per extra part for the
-// reduction).
+// CTAs evenly still keeps them all streaming. A CTA streams at a rate of its
+// own (its producers' copies in flight), so the step takes about as long as
+// the most units any CTA holds: ceil(tiles * ks / grid) / ks tiles' time. ks
+// is the power of two (1, 2, 4, 8, at most the chunks of K) that minimises it,
+// with 3% added per extra part for the reduction; the same in every CTA.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ int tc_pick_kslog(int tiles, int C, int sms) {
+__device__ __forceinline__ int tc_pick_kslog(int tiles, int C) {
   const int G = gridDim.x;
   int best_log = 0;
   float best = 3.0e38f;
-  for (int lg = 0; lg <= 2 && (1 << lg) <= C; ++lg) {
-    const int ks = 1 << lg, units = tiles * ks, q = units / G, rem = units % G;
-    const int load = (q + (rem > 0 ? 1 : 0)) + (sms < G ? q + (rem > sms ? 1 : 0) : 0);
-    const float t = (float)load / (float)ks * (1.0f + 0.03f * (float)(ks - 1));
+  for (int lg = 0; lg <= 3 && (1 << lg) <= C; ++lg) {
+    const int ks = 1 << lg, per_cta = (tiles * ks + G - 1) / G;
+    const float t = (float)per_cta / (float)ks * (1.0f + 0.03f * (float)(ks - 1));
     if (t < best) {
       best = t;
       best_log = lg;
@@ -523,6 +538,44 @@ __device__ __forceinline__ bool tc_reduce_parts(float* red, unsigned* tick, int 
   }
   epi_sync();  // s_flag is reused by the next unit
   return last;
+}
+
+// ---------------------------------------------------------------------------
+// Order-independent sums of the rowaxpy partials: each partial is rounded to
+// a multiple of 2^-32 and added as a 64-bit integer (two's complement, so an
+// unsigned atomic add), which is exact and associative; tc_finalize_kernel
+// converts each total once (to fp64, exactly, then fp32), adds it and the bias
+// into the output, and zeroes the accumulator. Partials stay far inside the
+// range (|v| < 2^31).
+// ---------------------------------------------------------------------------
+constexpr double TC_FIXED_SCALE = 4294967296.0;  // 2^32
+
+__device__ __forceinline__ void tc_acc_fixed(unsigned long long* acc, int d, int nb, int col, const float (&v)[16]) {
+#pragma unroll
+  for (int b = 0; b < TC_N; ++b) {
+    if (b >= nb) break;
+    const long long q = __double2ll_rn((double)v[b] * TC_FIXED_SCALE);
+    atomicAdd(acc + (size_t)b * d + col, (unsigned long long)q);
+  }
+}
+
+struct TcFinalizeArgs {
+  unsigned long long* acc;  // [nb][d], zero on exit
+  const float* bias;        // [d] or null
+  float* out;               // [nb][d], accumulated into
+  int nb, d;
+};
+
+__global__ void __launch_bounds__(256) tc_finalize_kernel(TcFinalizeArgs a) {
+  griddep_launch();
+  griddep_wait();
+  const int n = a.nb * a.d;
+  for (int i = blockIdx.x * 256 + threadIdx.x; i < n; i += gridDim.x * 256) {
+    const long long q = (long long)a.acc[i];
+    a.acc[i] = 0ull;
+    const int col = i % a.d;
+    a.out[i] += (float)((double)q / TC_FIXED_SCALE) + (a.bias ? a.bias[col] : 0.f);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -602,7 +655,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2) tc_qkv_kernel(const __grid_cons
     hc = hc < 0 ? 0 : a.kh_max;
   }
   const int nslots = hc * 3 * a.dh, C = (a.d + TC_K - 1) / TC_K;
-  TcQkvProblem p{m, a, nslots, C, tc_pick_kslog((nslots + TC_M - 1) / TC_M, C, a.sms), &s_flag};
+  TcQkvProblem p{m, a, nslots, C, tc_pick_kslog((nslots + TC_M - 1) / TC_M, C), &s_flag};
   tc_run(p, a.status, a.stages);
 }
 
@@ -636,19 +689,26 @@ struct TcW1Problem {
   __device__ int chunks(int unit) const { return ((((unit & ((1 << kslog) - 1)) + 1) * C) >> kslog) - c0(unit); }
   __device__ bool live(int, int) const { return true; }
   __device__ bool any(int) const { return true; }
-  // gather g: tile rows 4g .. 4g+3 (slots past the count read row 0)
-  __device__ void rows(int unit, int, int g, int (&r)[4]) const {
+  // thread t copies 16-byte piece t % 8 of tile rows t / 8 + 32 j (j < 4);
+  // slots past the count (and invalid indices) are zero-filled
+  __device__ void rows(int unit, int, int t, int (&r)[4]) const {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int s = (unit >> kslog) * TC_M + 4 * g + i;
-      const int v = s < cnt ? a.idx[s] : 0;
-      r[i] = (v >= 0 && v < a.N) ? v : 0;
+    for (int j = 0; j < 4; ++j) {
+      const int s = (unit >> kslog) * TC_M + (t >> 3) + 32 * j;
+      const int v = s < cnt ? a.idx[s] : -1;
+      r[j] = (v >= 0 && v < a.N) ? v : -1;
     }
   }
-  __device__ void issue(uint32_t st, uint64_t* full, int unit, int c, int g, const int (&r)[4]) const {
-    const int x = (c0(unit) + c) * TC_K;
-    tma_gather4(st + g * 512, &m.w, x, r, full);
-    if (g == 0) tc_issue_operand(m, st, full, x);
+  __device__ void issue(uint32_t st, uint64_t* full, int unit, int c, int t, const int (&r)[4]) const {
+    const int x = (c0(unit) + c) * TC_K, g = t & 7, row0 = t >> 3, col = x + 8 * g;
+    const uint32_t dst0 = st + (uint32_t)(row0 * 128) + (uint32_t)((g ^ (row0 & 7)) << 4);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const bool ok = r[j] >= 0 && col < a.d;
+      cp_async16_zfill(dst0 + 32 * 128 * j, ok ? (const void*)(a.W1t + (size_t)r[j] * a.d + col) : (const void*)a.W1t,
+                       ok ? 16 : 0);
+    }
+    if (t == 0) tc_issue_operand(m, st, full, x);
   }
   __device__ void epilogue(int unit, int mrow, int q, const float (&v0)[16], bool) const {
     float v[16];
@@ -713,7 +773,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2) tc_w1_kernel(const __grid_const
   griddep_launch();
   griddep_wait();
   const int cnt = tc_clamped_count(a.count, a.k_max, a.status), C = (a.d + TC_K - 1) / TC_K;
-  TcW1Problem p{m, a, cnt, C, tc_pick_kslog((cnt + TC_M - 1) / TC_M, C, a.sms), s_warp, &s_flag};
+  TcW1Problem p{m, a, cnt, C, tc_pick_kslog((cnt + TC_M - 1) / TC_M, C), s_warp, &s_flag};
   tc_run(p, a.status, a.stages);
 }
 
@@ -745,36 +805,36 @@ struct TcW2Problem {
       if (s_cnt[g * a.tiles_per_group + t] > 0) return true;
     return false;
   }
-  // gather g: K rows 4 (g % 16) .. +3 of the stage (the stage's 64
-  // compacted slots; slots past the tile's count read row 0, against zero
-  // activations), output columns 64 (g / 16) .. +63 of the unit's 128
-  __device__ void rows(int unit, int c, int g, int (&r)[4]) const {
-    const int t = (unit / n_mt) * a.tiles_per_group + (c >> 1), half = c & 1;
-    const int n = s_cnt[t] - half * 64;
-    const int base = t * TC_M + half * 64, kr = 4 * (g & 15);
+  // thread t copies 16-byte piece t % 8 of K rows t / 8 and t / 8 + 32 of
+  // the stage (its 64 compacted slots), output columns col0 .. col0+63 and
+  // col0+64 .. col0+127; slots past the tile's count are zero-filled
+  __device__ void rows(int unit, int c, int t, int (&r)[4]) const {
+    const int tl = (unit / n_mt) * a.tiles_per_group + (c >> 1), half = c & 1;
+    const int n = s_cnt[tl] - half * 64;
+    const int base = tl * TC_M + half * 64, j0 = t >> 3;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int j = j0 + 32 * i;
+      const int v = j < n ? a.rowid_c[base + j] : -1;
+      r[i] = (v >= 0 && v < a.N) ? v : -1;
+    }
+  }
+  __device__ void issue(uint32_t st, uint64_t* full, int unit, int c, int t, const int (&r)[4]) const {
+    const int tl = (unit / n_mt) * a.tiles_per_group + (c >> 1), half = c & 1;
+    const int g = t & 7, j0 = t >> 3, col0 = (unit % n_mt) * TC_M + 8 * g;
+    const uint32_t sw = (uint32_t)((g ^ (j0 & 7)) << 4);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int v = kr + i < n ? a.rowid_c[base + kr + i] : 0;
-      r[i] = (v >= 0 && v < a.N) ? v : 0;
+      const int h = i >> 1, j = j0 + 32 * (i & 1), rid = r[i & 1], col = col0 + 64 * h;
+      const bool ok = rid >= 0 && col < a.d;
+      cp_async16_zfill(st + (uint32_t)(h * 8192 + j * 128) + sw,
+                       ok ? (const void*)(a.W2t + (size_t)rid * a.d + col) : (const void*)a.W2t, ok ? 16 : 0);
     }
-  }
-  __device__ void issue(uint32_t st, uint64_t* full, int unit, int c, int g, const int (&r)[4]) const {
-    const int t = (unit / n_mt) * a.tiles_per_group + (c >> 1), half = c & 1;
-    const int mh = g >> 4;
-    tma_gather4(st + mh * 8192 + (g & 15) * 512, &m.w, (unit % n_mt) * TC_M + mh * 64, r, full);
-    if (g == 0) tc_issue_operand(m, st, full, t * TC_M + half * 64);
+    if (t == 0) tc_issue_operand(m, st, full, tl * TC_M + half * 64);
   }
   __device__ void epilogue(int unit, int mrow, int, const float (&v)[16], bool any) const {
-    const int g = unit / n_mt, mt = unit % n_mt;
-    const int col = mt * TC_M + mrow;
-    if (col >= a.d) return;
-    const float bias = (g == 0 && a.b2) ? a.b2[col] : 0.f;
-    if (!any && bias == 0.f) return;
-#pragma unroll
-    for (int b = 0; b < TC_N; ++b) {
-      if (b >= a.nb) break;
-      atomicAdd(a.out + (size_t)b * a.d + col, v[b] + bias);
-    }
+    const int col = (unit % n_mt) * TC_M + mrow;
+    if (any && col < a.d) tc_acc_fixed(a.acc, a.d, a.nb, col, v);
   }
 };
 
@@ -840,16 +900,8 @@ struct TcWoProblem {
     tc_issue_operand(m, st, full, p * a.dh + part * 64);
   }
   __device__ void epilogue(int unit, int mrow, int, const float (&v)[16], bool any) const {
-    const int g = unit / n_mt, mt = unit % n_mt;
-    const int col = mt * TC_M + mrow;
-    if (col >= a.d) return;
-    const float bias = (g == 0 && a.bO) ? a.bO[col] : 0.f;
-    if (!any && bias == 0.f) return;
-#pragma unroll
-    for (int b = 0; b < TC_N; ++b) {
-      if (b >= a.nb) break;
-      atomicAdd(a.out + (size_t)b * a.d + col, v[b] + bias);
-    }
+    const int col = (unit % n_mt) * TC_M + mrow;
+    if (any && col < a.d) tc_acc_fixed(a.acc, a.d, a.nb, col, v);
   }
 };
 

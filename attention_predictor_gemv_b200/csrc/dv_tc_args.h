@@ -33,10 +33,9 @@ struct TcQkvArgs {
   __nv_bfloat16* Kc;          // [nb][h][cap][dh]
   __nv_bfloat16* Vc;
   int* status;
-  float* red;                 // [tiles][4][16][128] split-K partial sums
+  float* red;                 // [tiles][parts][16][128] split-K partial sums (parts <= 8)
   unsigned* tick;             // [tiles] parts finished per tile, zero between calls
   int stages;                 // ring stages (set by the launcher)
-  int sms;                    // SMs of the device (set by the launcher)
 };
 
 struct TcMlpArgs {
@@ -58,10 +57,10 @@ struct TcMlpArgs {
   float* out;                // [nb][d], accumulated into
   int* status;
   int act;                   // ACT_RELU or ACT_GELU
-  float* red;                // [tiles][4][16][128] split-K partial sums of W1
+  float* red;                // [tiles][parts][16][128] split-K partial sums of W1 (parts <= 8)
   unsigned* tick;            // [tiles] parts finished per tile, zero between calls
+  unsigned long long* acc;   // [nb][d] fixed-point partial sums of W2, zero between calls
   int stages;                // ring stages (set by the launcher)
-  int sms;                   // SMs of the device (set by the launcher)
 };
 
 struct TcWoArgs {
@@ -75,6 +74,7 @@ struct TcWoArgs {
   int heads_per_group;
   float* out;                // [nb][d], accumulated into
   int* status;
+  unsigned long long* acc;   // [nb][d] fixed-point partial sums, zero between calls
   int stages;                // ring stages (set by the launcher)
 };
 
