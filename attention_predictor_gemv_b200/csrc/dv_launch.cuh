@@ -167,6 +167,16 @@ inline int sm_count() {
   return n;
 }
 
+// CTAs of the batch-1 neuron-score kernel (predict_b_kernel, one row per
+// warp): four per SM unless DV_PB_CTAS gives the count.
+inline int pb_ctas() {
+  static const int n = [] {
+    const char* e = std::getenv("DV_PB_CTAS");
+    return e ? std::atoi(e) : 0;
+  }();
+  return n > 0 ? n : 4 * sm_count();
+}
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
 inline bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }

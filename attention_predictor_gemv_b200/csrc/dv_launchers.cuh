@@ -377,8 +377,8 @@ cudaError_t run_predict_b_nb(const PredictBArgs& a, cudaStream_t st) {
     // the warps of the two-rows-per-warp form, which the memory pipe needs
     // to keep enough 16-byte loads in flight for rows of 4 vectors per lane
     if (a.r / WT<T>::E == 128) {
-      const int g1 = (a.N + FUSED_WARPS - 1) / FUSED_WARPS;
-      const dim3 grid1(g1 < 4 * sm_count() ? g1 : 4 * sm_count());
+      const int g1 = (a.N + FUSED_WARPS - 1) / FUSED_WARPS, cap = pb_ctas();
+      const dim3 grid1(g1 < cap ? g1 : cap);
       return launch(predict_b_kernel<T, 1, 1, 4, 4>, grid1, FUSED_THREADS, 0, st, a);
     }
   }

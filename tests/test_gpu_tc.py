@@ -227,3 +227,39 @@ def test_tc_lookahead_stack_and_graph_replay(name, B):
     _no_device_errors(stk.ws_main)
     _no_device_errors(stk.ws_side)
     del g
+
+
+@pytest.mark.parametrize("name,B", [("opt-like", 8), ("opt-like", 16), ("175b-slice", 4)])
+def test_tc_stack_is_bitwise_reproducible(name, B):
+    """The tensor-core layer path sums its partials in a fixed order (split-K
+    parts in part order, W2 / W^O groups as exact fixed-point integers, the
+    attention splits in split order), so two runs of the same step from the
+    same state give the same bits: outputs, scores, selected sets and the
+    appended KV slots. Without that, a score within rounding of the top-k
+    boundary could select a different neuron on a rerun."""
+    nL = 3
+    s = _shape(name, B)
+    layers = [wl.make_layer(s, 700 + l, DEV) for l in range(nL)]
+    K0 = [(t["K"].clone(), t["V"].clone()) for t in layers]
+    k, k_h = wl.k_for(0.1, s.N), 2
+    stk = DecoderStack(layers, B, k, k_h, 1.0 / np.sqrt(s.dh), lookahead=True)
+    xin = wl.make_input(s, 71, DEV)
+    runs = []
+    for _ in range(2):
+        for (Kc, Vc), t in zip(K0, layers):
+            t["K"].copy_(Kc)
+            t["V"].copy_(Vc)
+        x = xin.clone()
+        stk.step(x, s.L)
+        torch.cuda.synchronize()
+        runs.append(dict(x=x.clone(), sm=[v.clone() for v in stk.scores], sh=[v.clone() for v in stk.scores_h],
+                         idx=[selected(stk.idx[l], stk.count[l]) for l in range(nL)],
+                         K=[t["K"][:, :, s.L].clone() for t in layers]))
+    a, b = runs
+    assert torch.equal(a["x"], b["x"])
+    for l in range(nL):
+        assert torch.equal(a["sm"][l], b["sm"][l]), l
+        assert torch.equal(a["sh"][l], b["sh"][l]), l
+        assert np.array_equal(a["idx"][l], b["idx"][l]), l
+        assert torch.equal(a["K"][l], b["K"][l]), l
+    _no_device_errors(stk.ws_main)
