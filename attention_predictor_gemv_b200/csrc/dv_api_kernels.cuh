@@ -272,18 +272,13 @@ __global__ void __launch_bounds__(SR_THREADS) select_rows_kernel(SelectRowsArgs 
 #pragma unroll
       for (int w = 0; w < SR_WARPS; ++w) s_wh[w][tid] = 0u;
       __syncthreads();
-      // one shared-memory add per distinct digit of the warp's 32 keys: scores
-      // share few exponents, so in the first pass most keys of a warp hold the
-      // same digit and per-key adds to one address would serialise
+      // per-key adds; grouping a warp's equal digits first (__match_any_sync)
+      // made the whole look-ahead step 20 us per layer slower when this kernel
+      // ran beside the main-stream kernels (measured at N = 49152), though it
+      // was not slower alone
 #pragma unroll
-      for (int j = 0; j < SR_KPT; ++j) {
-        const bool part = ((vmask >> j) & 1u) && (key[j] & mask) == prefix;
-        if (__any_sync(0xffffffffu, part)) {
-          const unsigned dg = part ? (key[j] >> shift) & 255u : 256u;
-          const unsigned peers = __match_any_sync(0xffffffffu, dg);
-          if (part && (peers & lt) == 0u) atomicAdd(&s_wh[warp][dg], (unsigned)__popc(peers));
-        }
-      }
+      for (int j = 0; j < SR_KPT; ++j)
+        if (((vmask >> j) & 1u) && (key[j] & mask) == prefix) atomicAdd(&s_wh[warp][(key[j] >> shift) & 255u], 1u);
       __syncthreads();
       unsigned c = 0u;
 #pragma unroll

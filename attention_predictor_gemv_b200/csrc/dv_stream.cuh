@@ -560,4 +560,3 @@ __global__ void __launch_bounds__(CO_THREADS, 1) wo_stream_kernel(WoStreamArgs a
 }
 
 }  // namespace dv
-
