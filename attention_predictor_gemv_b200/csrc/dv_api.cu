@@ -160,13 +160,15 @@ bool pred_tc_ok(int B, dv_dtype wdt, int nrows, int K) {
 }
 
 cudaError_t pred_tc(const Layout& L, void* ws, const void* W, int nrows, int K, const float* bias, const float* x, int B,
-                    float* out, long long ldo, cudaStream_t st) {
+                    float* out, long long ldo, cudaStream_t st, bool split = true) {
   bf16* xhi = at<bf16>(ws, L.tc_x);
   bf16* xlo = xhi + (size_t)TC_N * L.XC;
-  cudaError_t e = run_tc_split(x, B, K, K, xhi, xlo, K, st);
-  if (e != cudaSuccess) return e;
-  return run_tc_dense(static_cast<const bf16*>(W), nrows, K, bias, xhi, xlo, B, out, ldo, at<float>(ws, L.tc_red),
-                      at<unsigned>(ws, L.tc_tick), at<int>(ws, L.status), st);
+  if (split) {  // (not when the previous call split the same x)
+    cudaError_t e = run_tc_split(x, B, K, K, xhi, xlo, K, st);
+    if (e != cudaSuccess) return e;
+  }
+  return run_tc_dense(nullptr, 0, nullptr, nullptr, 0, static_cast<const bf16*>(W), nrows, bias, out, ldo, K, xhi, xlo,
+                      B, at<float>(ws, L.tc_red), at<unsigned>(ws, L.tc_tick), at<int>(ws, L.status), st);
 }
 
 // The predictor's two stages: z = y A (predict_a_kernel family; rows of At
@@ -530,9 +532,16 @@ dv_status layer_begin(const Layout& L, void* ws, const dv_layer_weights* w, cons
       return cuda_status(run_gemv(w->wdtype, ahead->w->At, D.r, D.d, yA, D.d, D.B, nullptr, ahead->z, D.r, st));
     }
     const bool tc_h = pred_tc_ok(D.B, w->wdtype, D.h, D.d), tc_z = pred_tc_ok(D.B, w->wdtype, D.r, D.d);
+    if (tc_h && tc_z) {  // head scores and z in one launch: rows of P_A, then rows of A^T
+      bf16* xhi = at<bf16>(ws, L.tc_x);
+      bf16* xlo = xhi + (size_t)TC_N * L.XC;
+      DV_TRY(run_tc_split(yA, D.B, D.d, D.d, xhi, xlo, D.d, st));
+      return cuda_status(run_tc_dense(static_cast<const bf16*>(ahead->w->PA), D.h, nullptr, ahead->sh, D.h,
+                                      static_cast<const bf16*>(ahead->w->At), D.r, nullptr, ahead->z, D.r, D.d, xhi,
+                                      xlo, D.B, at<float>(ws, L.tc_red), at<unsigned>(ws, L.tc_tick), status, st));
+    }
     if (tc_h) DV_TRY(pred_tc(L, ws, ahead->w->PA, D.h, D.d, nullptr, yA, D.B, ahead->sh, D.h, st));
-    if (tc_z) DV_TRY(pred_tc(L, ws, ahead->w->At, D.r, D.d, nullptr, yA, D.B, ahead->z, D.r, st));
-    if (tc_h && tc_z) return DV_OK;
+    if (tc_z) DV_TRY(pred_tc(L, ws, ahead->w->At, D.r, D.d, nullptr, yA, D.B, ahead->z, D.r, st, !tc_h));
     PredictAArgs pa = {};
     pa.y = yA;
     pa.PA = tc_h ? nullptr : ahead->w->PA;

@@ -176,31 +176,45 @@ bool tc_dense_ok(int B, int wbytes, int nrows, int K) {
   return wbytes == 2 && B >= 1 && B <= TC_N && nrows >= 64 && K >= TC_K && K % 8 == 0 && encode_fn() != nullptr;
 }
 
-cudaError_t run_tc_dense(const __nv_bfloat16* W, int nrows, int K, const float* bias, const __nv_bfloat16* xhi,
-                         const __nv_bfloat16* xlo, int nb, float* out, long long ldo, float* red, unsigned* tick,
+
+cudaError_t run_tc_dense(const __nv_bfloat16* W1, int n1, const float* bias1, float* out1, long long ldo1,
+                         const __nv_bfloat16* W2, int n2, const float* bias2, float* out2, long long ldo2, int K,
+                         const __nv_bfloat16* xhi, const __nv_bfloat16* xlo, int nb, float* red, unsigned* tick,
                          int* status, cudaStream_t st) {
-  const long long tiles = (nrows + TC_M - 1) / TC_M, C = (K + TC_K - 1) / TC_K;
+  if (n1 < 0 || n2 < 1) return cudaErrorInvalidValue;
+  const long long p1 = (n1 + 63) / 64 * 64;
+  const long long tiles = (p1 + n2 + TC_M - 1) / TC_M, C = (K + TC_K - 1) / TC_K;
   const long long slots = (long long)tc_ctas_per_sm() * sm_count();
   long long want = (slots + tiles - 1) / tiles;
   if (want > C) want = C;
   if (want > TC_DENSE_PARTS / tiles) want = TC_DENSE_PARTS / tiles;
+  if (want > TC_DENSE_MAX_KS) want = TC_DENSE_MAX_KS;
   int kslog = 0;  // the largest power of two not above want
   while ((2ll << kslog) <= want) ++kslog;
   const long long ks = 1ll << kslog;
   TcDenseArgs a = {};
-  a.bias = bias;
-  a.nrows = nrows;
+  a.bias1 = bias1;
+  a.bias2 = bias2;
+  a.n1 = n1;
+  a.n2 = n2;
   a.K = K;
   a.nb = nb;
   a.kslog = kslog;
-  a.out = out;
-  a.ldo = ldo;
+  a.out1 = out1;
+  a.out2 = out2;
+  a.ldo1 = ldo1;
+  a.ldo2 = ldo2;
   a.status = status;
   a.red = red;
   a.tick = tick;
   TcMaps m;
-  cudaError_t e = tc_maps(&m, W, nrows, K, 64, xhi, xlo, K, K);
+  cudaError_t e = tc_maps(&m, W2, n2, K, 64, xhi, xlo, K, K);
   if (e != cudaSuccess) return e;
+  m.w2 = m.w;
+  if (n1 > 0) {
+    e = tc_map(&m.w, W1, K, n1, K, TC_K, 64);
+    if (e != cudaSuccess) return e;
+  }
   return launch_tc(tc_dense_kernel, clamp_grid(tiles * ks), st, m, a);
 }
 

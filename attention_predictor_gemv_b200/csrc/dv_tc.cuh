@@ -505,19 +505,22 @@ __device__ __forceinline__ int tc_pick_kslog(int tiles, int C) {
 }
 
 // The epilogue threads' partial sums of `tile` (thread m: row m, v[b] for b <
-// nb) go into this part's own slot of red; the part that finishes the tile
-// last (ticket) sums the ks slots in part order into v, resets the ticket and
-// returns true in all 128 threads; the other parts return false. The sum is
-// the same whichever part arrives last, so results do not depend on timing
-// (the selections downstream compare scores exactly). With ks == 1 v is
-// already complete.
+// nb) go into this part's own slot of red ([128][16] floats, so a thread's
+// values are four float4); the part that finishes the tile last (ticket)
+// sums the ks slots in part order into v, resets the ticket and returns true
+// in all 128 threads; the other parts return false. The sum is the same
+// whichever part arrives last, so results do not depend on timing (the
+// selections downstream compare scores exactly). With ks == 1 v is already
+// complete.
 __device__ __forceinline__ bool tc_reduce_parts(float* red, unsigned* tick, int tile, int part, int ks, int nb, int m,
                                                 float (&v)[16], int* s_flag) {
   if (ks == 1) return true;
-  float* slot = red + ((size_t)tile * ks + part) * TC_N * TC_M;
+  constexpr int SLOT4 = TC_N * TC_M / 4;  // float4 per slot
+  const int nq = (nb + 3) >> 2;
+  float4* slot = reinterpret_cast<float4*>(red) + ((size_t)tile * ks + part) * SLOT4 + m * 4;
 #pragma unroll
-  for (int b = 0; b < TC_N; ++b)
-    if (b < nb) slot[b * TC_M + m] = v[b];
+  for (int q = 0; q < 4; ++q)
+    if (q < nq) slot[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
   __threadfence();
   epi_sync();
   if (m == 0) *s_flag = atomicAdd(tick + tile, 1u) == (unsigned)(ks - 1) ? 1 : 0;
@@ -525,14 +528,29 @@ __device__ __forceinline__ bool tc_reduce_parts(float* red, unsigned* tick, int 
   const bool last = *s_flag != 0;
   if (last) {
     __threadfence();
-    const float* t0 = red + (size_t)tile * ks * TC_N * TC_M;
+    const float4* t0 = reinterpret_cast<const float4*>(red) + (size_t)tile * ks * SLOT4 + m * 4;
+    float4 sum[4];
 #pragma unroll
-    for (int b = 0; b < TC_N; ++b) {
-      if (b < nb) {
-        float sum = 0.f;
-        for (int p = 0; p < ks; ++p) sum += __ldcg(t0 + ((size_t)p * TC_N + b) * TC_M + m);
-        v[b] = sum;
+    for (int q = 0; q < 4; ++q) sum[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int p = 0; p < ks; ++p) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (q < nq) {
+          const float4 w = __ldcg(t0 + (size_t)p * SLOT4 + q);
+          sum[q].x += w.x;
+          sum[q].y += w.y;
+          sum[q].z += w.z;
+          sum[q].w += w.w;
+        }
       }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      v[4 * q] = sum[q].x;
+      v[4 * q + 1] = sum[q].y;
+      v[4 * q + 2] = sum[q].z;
+      v[4 * q + 3] = sum[q].w;
     }
     if (m == 0) tick[tile] = 0u;
   }
@@ -916,10 +934,9 @@ __global__ void __launch_bounds__(TC_THREADS, 2) tc_wo_kernel(const __grid_const
 }
 
 // ---------------------------------------------------------------------------
-// Dense rowdot (rows of W consecutive, two 64-row tiles per stage), with the
-// K range of a 128-row tile split ks = 2^kslog ways: unit u is tile u / ks,
-// part u % ks
-// (the parts reduced in order by tc_reduce_parts)
+// Dense rowdot (rows of one or two matrices, two 64-row tiles per stage),
+// with the K range of a 128-row tile split ks = 2^kslog ways: unit u is tile
+// u / ks, part u % ks (the parts reduced in order by tc_reduce_parts)
 // ---------------------------------------------------------------------------
 
 struct TcDenseProblem {
@@ -928,9 +945,10 @@ struct TcDenseProblem {
   static constexpr bool kRowsPerUnit = true;
   const TcMaps& m;
   TcDenseArgs a;
-  int C;  // 64-column chunks of K
+  int C;   // 64-column chunks of K
+  int p1;  // rows of the first block, padded to 64
   int* s_flag;
-  __device__ int units() const { return ((a.nrows + TC_M - 1) / TC_M) << a.kslog; }
+  __device__ int units() const { return ((p1 + a.n2 + TC_M - 1) / TC_M) << a.kslog; }
   __device__ int c0(int unit) const { return ((unit & ((1 << a.kslog) - 1)) * C) >> a.kslog; }
   __device__ int chunks(int unit) const {
     return ((((unit & ((1 << a.kslog) - 1)) + 1) * C) >> a.kslog) - c0(unit);
@@ -940,8 +958,12 @@ struct TcDenseProblem {
   __device__ void rows(int, int, int, int (&)[4]) const {}
   __device__ void issue(uint32_t st, uint64_t* full, int unit, int c, int, const int (&)[4]) const {
     const int y = (unit >> a.kslog) * TC_M, x = (c0(unit) + c) * TC_K;
-    tma_load_2d(st, &m.w, x, y, full);
-    tma_load_2d(st + 8192, &m.w, x, y + 64, full);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int yv = y + 64 * k;  // rows past both blocks read zeros
+      if (yv < p1) tma_load_2d(st + k * 8192, &m.w, x, yv, full);
+      else tma_load_2d(st + k * 8192, &m.w2, x, yv - p1, full);
+    }
     tc_issue_operand(m, st, full, x);
   }
   __device__ void epilogue(int unit, int mrow, int, const float (&v0)[16], bool) const {
@@ -952,12 +974,27 @@ struct TcDenseProblem {
     if (!tc_reduce_parts(a.red, a.tick, tile, unit & ((1 << a.kslog) - 1), 1 << a.kslog, a.nb, mrow, v, s_flag))
       return;
     const int row = tile * TC_M + mrow;
-    if (row >= a.nrows) return;
-    const float bias = a.bias ? a.bias[row] : 0.f;
+    float* out;
+    long long ld;
+    float bias = 0.f;
+    int i;
+    if (row < p1) {
+      if (row >= a.n1) return;
+      i = row;
+      out = a.out1;
+      ld = a.ldo1;
+      if (a.bias1) bias = a.bias1[i];
+    } else {
+      i = row - p1;
+      if (i >= a.n2) return;
+      out = a.out2;
+      ld = a.ldo2;
+      if (a.bias2) bias = a.bias2[i];
+    }
 #pragma unroll
     for (int b = 0; b < TC_N; ++b) {
       if (b >= a.nb) break;
-      a.out[(size_t)b * a.ldo + row] = v[b] + bias;
+      out[(size_t)b * ld + i] = v[b] + bias;
     }
   }
 };
@@ -966,7 +1003,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2) tc_dense_kernel(const __grid_co
   __shared__ int s_flag;
   griddep_launch();
   griddep_wait();
-  TcDenseProblem p{m, a, (a.K + TC_K - 1) / TC_K, &s_flag};
+  TcDenseProblem p{m, a, (a.K + TC_K - 1) / TC_K, (a.n1 + 63) / 64 * 64, &s_flag};
   tc_run(p, a.status, a.stages);
 }
 

@@ -19,6 +19,7 @@ constexpr int DV_DEV_TIMEOUT_BIT = 8;  // device status bit: a bounded wait ran 
 // operand's hi and lo rows [16][ld] (boxes of 64 x 16).
 struct TcMaps {
   CUtensorMap w, hi, lo;
+  CUtensorMap w2;  // a second weight matrix (the dense rowdot's second row block)
 };
 
 struct TcQkvArgs {
@@ -78,14 +79,19 @@ struct TcWoArgs {
   int stages;                // ring stages (set by the launcher)
 };
 
-// Dense rowdot over consecutive rows: out[b][row] (+)= W[row] . X[b] (+
-// bias[row]) for row < nrows, b < nb (the predictor's GEMMs at batch >= 3).
+// Dense rowdot over consecutive rows of up to two matrices sharing the
+// operand (the predictor's GEMMs at batch >= 3): out1[b][i] = W1[i] . X[b]
+// (+ bias1[i]) for i < n1 (maps.w), then out2[b][i] = W2[i] . X[b] (+
+// bias2[i]) for i < n2 (maps.w2); the first block is padded to p1 =
+// ceil(n1 / 64) 64 rows, so a 64-row tile never spans both.
 struct TcDenseArgs {
-  const float* bias;  // [nrows] or null
-  int nrows, K, nb;
-  int kslog;          // log2 of the K splits per 128-row tile
-  float* out;         // [nb][ldo]
-  long long ldo;
+  const float* bias1;  // [n1] or null
+  const float* bias2;  // [n2] or null
+  int n1, n2, K, nb;
+  int kslog;           // log2 of the K splits per 128-row tile
+  float* out1;         // [nb][ldo1]
+  float* out2;         // [nb][ldo2]
+  long long ldo1, ldo2;
   int* status;
   float* red;         // [tiles][2^kslog][16][128] split-K partial sums
   unsigned* tick;     // [tiles] parts finished per tile, zero between calls

@@ -8,6 +8,7 @@
 namespace dv {
 
 constexpr int TC_DENSE_PARTS = 512;  // dense rowdot units (tiles x K parts) with partial-sum slots, at most
+constexpr int TC_DENSE_MAX_KS = 32;  // K parts per dense tile, at most (the last part sums them)
 
 // Shapes the tensor-core path takes: bf16 weights, at most 16 batch rows,
 // d >= 64 and a multiple of 8, dh a multiple of 64, at most 1024 tiles of 128
@@ -32,14 +33,17 @@ cudaError_t run_tc_qkv(TcQkvArgs a, cudaStream_t st);
 cudaError_t run_tc_mlp(TcMlpArgs a, cudaStream_t st);
 cudaError_t run_tc_wo(TcWoArgs a, cudaStream_t st);
 
-// The dense rowdot: out[b][row] = W[row] . x[b] (+ bias[row]) for the rows
-// of W [nrows][K] (bf16) and the operand split into xhi / xlo [16][K]; out
-// [nb][ldo]. When the K range is split across CTAs (at most TC_DENSE_PARTS
-// units of tiles x parts) the partial sums go through red [units][16][128]
-// and the per-tile tickets tick [tiles] (zero between calls).
+// The dense rowdot over one or two matrices sharing the operand x (split
+// into xhi / xlo [16][K]): out1[b][i] = W1[i] . x[b] (+ bias1[i]) for the n1
+// rows of W1 [n1][K] (n1 = 0: none), and out2[b][i] = W2[i] . x[b] (+
+// bias2[i]) for the n2 rows of W2, bf16. When the K range is split across
+// CTAs (at most TC_DENSE_PARTS units of tiles x parts) the partial sums go
+// through red [units][128][16] and the per-tile tickets tick (zero between
+// calls).
 bool tc_dense_ok(int B, int wbytes, int nrows, int K);
-cudaError_t run_tc_dense(const __nv_bfloat16* W, int nrows, int K, const float* bias, const __nv_bfloat16* xhi,
-                         const __nv_bfloat16* xlo, int nb, float* out, long long ldo, float* red, unsigned* tick,
+cudaError_t run_tc_dense(const __nv_bfloat16* W1, int n1, const float* bias1, float* out1, long long ldo1,
+                         const __nv_bfloat16* W2, int n2, const float* bias2, float* out2, long long ldo2, int K,
+                         const __nv_bfloat16* xhi, const __nv_bfloat16* xlo, int nb, float* red, unsigned* tick,
                          int* status, cudaStream_t st);
 
 }  // namespace dv
