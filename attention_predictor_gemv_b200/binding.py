@@ -319,7 +319,25 @@ class Layer:
         W1t, Wqkv, K = t["W1t"], t["Wqkv"], t["K"]
         N, d = W1t.shape
         h, _, dh, _ = Wqkv.shape
-        self.dims = Dims(B, d, N, t["At"].shape[0], h, dh, K.shape[2], k_max, kh_max)
+        r, cap = t["At"].shape[0], K.shape[2]
+        # every tensor's extent against the dims the library will index with
+        # (the C ABI sees pointers only, so a short tensor would be read past
+        # its end)
+        want = {"W1t": (N, d), "W2t": (N, d), "PA": (h, d), "Wqkv": (h, 3, dh, d), "WOt": (h, dh, d),
+                "K": (B, h, cap, dh), "V": (B, h, cap, dh), "At": (r, d), "Bm": (N, r), "b1": (N,), "b2": (d,),
+                "bqkv": (h, 3, dh), "bO": (d,), "ln1_g": (d,), "ln1_b": (d,), "ln2_g": (d,), "ln2_b": (d,)}
+        for n, shp in want.items():
+            v = t.get(n)
+            if v is None:
+                continue
+            got = tuple(v.shape)
+            if n in ("K", "V"):  # a cache with more batch rows than B: its first B rows are used
+                ok = len(got) == 4 and got[0] >= B and got[1:] == shp[1:]
+            else:
+                ok = got == shp
+            if not ok or not v.is_contiguous():
+                raise ValueError(f"{n}: shape {got}, expected {shp} (contiguous) for batch {B}")
+        self.dims = Dims(B, d, N, r, h, dh, cap, k_max, kh_max)
         g = lambda n, dt=None: _ptr(t.get(n), dt, n)  # noqa: E731
         self.c = LayerWeightsC(_wdt(W1t), _wdt(K), g("ln1_g", torch.float32), g("ln1_b", torch.float32), g("PA"),
                                g("Wqkv"), g("bqkv", torch.float32), g("WOt"), g("bO", torch.float32), g("K"), g("V"),

@@ -372,14 +372,14 @@ template <typename T, int NB>
 cudaError_t run_predict_b_nb(const PredictBArgs& a, cudaStream_t st) {
   const int rpw = rpw_for(a.r, WT<T>::E), per = FUSED_WARPS * rpw;
   const int groups = (a.N + per - 1) / per;
-  if constexpr (NB == 1) {
+  if constexpr (NB <= 2) {
     // one row per warp and four CTAs per SM (registers capped at 64): twice
     // the warps of the two-rows-per-warp form, which the memory pipe needs
     // to keep enough 16-byte loads in flight for rows of 4 vectors per lane
     if (a.r / WT<T>::E == 128) {
       const int g1 = (a.N + FUSED_WARPS - 1) / FUSED_WARPS, cap = pb_ctas();
       const dim3 grid1(g1 < cap ? g1 : cap);
-      return launch(predict_b_kernel<T, 1, 1, 4, 4>, grid1, FUSED_THREADS, 0, st, a);
+      return launch(predict_b_kernel<T, NB, 1, 4, 4>, grid1, FUSED_THREADS, 0, st, a);
     }
   }
   const dim3 grid(groups < 2 * sm_count() ? groups : 2 * sm_count());  // persistent: two CTAs per SM

@@ -282,7 +282,7 @@ def point(layers, shape, B, sparsity, steps, warmup, dist, lookahead=True, kv_se
 KERNEL_HEADERS = {
     "attn_in": ("dv_common.cuh", "dv_fused.cuh", "dv_colowner.cuh", "dv_stream.cuh"),
     "mlp_block": ("dv_common.cuh", "dv_fused.cuh", "dv_colowner.cuh", "dv_stream.cuh"),
-    "attn_out": ("dv_common.cuh", "dv_kernels.cuh", "dv_fused.cuh"),
+    "attn_out": ("dv_common.cuh", "dv_kernels.cuh", "dv_fused.cuh", "dv_stream.cuh"),
     "predict_neurons": ("dv_common.cuh", "dv_fused.cuh", "dv_api_kernels.cuh"),
 }
 

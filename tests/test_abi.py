@@ -185,3 +185,24 @@ def test_q8_block_calls_check_arguments_on_the_host():
     bad = list(args)
     bad[14] = 8
     assert g(*bad) == bd.DV_ERR_ARG  # pos >= cap
+
+
+def test_layer_rejects_tensors_shorter_than_the_dims():
+    """The binding checks every tensor's extent against the dims the library
+    indexes with: a KV cache made for batch 1 cannot back a batch-2 layer."""
+    from attention_predictor_gemv_b200 import binding as bd
+    from attention_predictor_gemv_b200 import workload as wl
+
+    s = wl.LayerShape(B=1, d=256, N=1024, r=32, h=4, dh=64, L=64, cap=65, wdtype="f32", kvdtype="f32",
+                      p_active=0.1)
+    t = wl.make_layer(s, 0, "cpu")
+    # shapes that match pass the check and stop at the device check (CPU tensors here)
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        bd.Layer(t, 1, 64, 2)
+    with pytest.raises(ValueError, match="^K: shape"):
+        bd.Layer(t, 2, 64, 2)
+    K3, V3 = wl.make_kv(s, 3, 1, "cpu")
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):  # more cache rows than B is fine
+        bd.Layer(dict(t, K=K3, V=V3), 2, 64, 2)
+    with pytest.raises(ValueError, match="^Bm: shape"):
+        bd.Layer(dict(t, Bm=t["Bm"][:, :16].contiguous()), 1, 64, 2)
