@@ -698,27 +698,42 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
       float m = -INFINITY, l = 0.f, acc[E];
 #pragma unroll
       for (int e = 0; e < E; ++e) acc[e] = 0.f;
-      for (int tb = kw0; tb < kw1; tb += KPW) {  // warp-uniform trip count
-        const int t = tb + kq;
-        const bool ok = t < kw1;
-        float dot = 0.f;
-        if (ok) {
-          float kf[E];
-          WT<KT>::unpack(*reinterpret_cast<const uint4*>(tK + t * DH + g * E), kf);
+      // two key groups per trip (warp-uniform trip count): both dot products
+      // and their shuffle reductions are independent, so their latencies
+      // overlap; the running-max updates then follow in key order
+      for (int tb = kw0; tb < kw1; tb += 2 * KPW) {
+        float dot[2];
+        bool ok[2];
 #pragma unroll
-          for (int e = 0; e < E; ++e) dot = fmaf(qv[e], kf[e], dot);
+        for (int u = 0; u < 2; ++u) {
+          const int t = tb + u * KPW + kq;
+          ok[u] = t < kw1;
+          dot[u] = 0.f;
+          if (ok[u]) {
+            float kf[E];
+            WT<KT>::unpack(*reinterpret_cast<const uint4*>(tK + t * DH + g * E), kf);
+#pragma unroll
+            for (int e = 0; e < E; ++e) dot[u] = fmaf(qv[e], kf[e], dot[u]);
+          }
         }
 #pragma unroll
-        for (int o = G / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-        if (ok) {
-          float vf[E];
-          WT<KT>::unpack(*reinterpret_cast<const uint4*>(tV + t * DH + g * E), vf);
-          const float mn = fmaxf(m, dot);
-          const float c = __expf(m - mn), pe = __expf(dot - mn);
-          l = l * c + pe;
+        for (int o = G / 2; o > 0; o >>= 1) {
+          dot[0] += __shfl_xor_sync(0xffffffffu, dot[0], o);
+          dot[1] += __shfl_xor_sync(0xffffffffu, dot[1], o);
+        }
 #pragma unroll
-          for (int e = 0; e < E; ++e) acc[e] = fmaf(pe, vf[e], acc[e] * c);
-          m = mn;
+        for (int u = 0; u < 2; ++u) {
+          if (ok[u]) {
+            const int t = tb + u * KPW + kq;
+            float vf[E];
+            WT<KT>::unpack(*reinterpret_cast<const uint4*>(tV + t * DH + g * E), vf);
+            const float mn = fmaxf(m, dot[u]);
+            const float c = __expf(m - mn), pe = __expf(dot[u] - mn);
+            l = l * c + pe;
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc[e] = fmaf(pe, vf[e], acc[e] * c);
+            m = mn;
+          }
         }
       }
       // merge the warp's KPW key groups (lanes g, g + G, ... hold the same dims)

@@ -203,10 +203,22 @@ cudaError_t run_attn(int dh, const float* q, const void* Kc, const void* Vc, int
 
 constexpr int ATTN_CS = 8;  // CTAs per cluster (per selected head) in attn_out_kernel
 
-inline int attn_out_S(int pos) { return (pos + 1 + ATTN_CS - 1) / ATTN_CS; }
+inline int attn_out_S(int pos, int cs = ATTN_CS) { return (pos + 1 + cs - 1) / cs; }
 // K/V tiles of S keys, the cluster's partials (m, l, acc[dh]) and q of nb rows.
-inline size_t attn_out_smem(int S, int dh, int kvbytes, int nb) {
-  return 2ull * S * dh * kvbytes + 4ull * nb * ATTN_CS * (dh + 2) + 4ull * nb * dh;
+inline size_t attn_out_smem(int S, int dh, int kvbytes, int nb, int cs = ATTN_CS) {
+  return 2ull * S * dh * kvbytes + 4ull * nb * cs * (dh + 2) + 4ull * nb * dh;
+}
+// CTAs per cluster (per selected head) of the attention-only form: 8 at
+// batch 1, 16 (a non-portable cluster size, half the keys per CTA) at batch
+// 2, where each CTA holds two rows' K/V tiles (measured at the OPT-175B
+// shape: 249 against 259 us per layer at batch 2, 119 against 118 at batch
+// 1). DV_ATTN_CS=8 or 16 overrides.
+inline int attn_h_cs(int nb) {
+  static const int env = [] {
+    const char* e = std::getenv("DV_ATTN_CS");
+    return !e ? 0 : (e[0] == '1' && e[1] == '6' ? 16 : 8);
+  }();
+  return env ? env : (nb >= 2 ? 16 : 8);
 }
 constexpr size_t ATTN_SMEM_MAX = 204 * 1024;  // dynamic part; the static part stays below 21 KB
 
@@ -253,21 +265,26 @@ cudaError_t run_attn_in(const AttnInArgs& a, cudaStream_t st) {
   }
 }
 
-template <typename KT, int DH, int NB, int WV>
+template <typename KT, int DH, int NB, int WV, int CS = ATTN_CS>
 cudaError_t run_attn_out_nbw(AttnOutArgs a, cudaStream_t st) {
   // K/V tiles of every batch row at once when they fit, else row by row; and
   // row by row too when the grid is larger than the SMs and holding every
   // row would leave one CTA per SM (a second wave costs more than staging
   // the rows one after the other)
+  a.S = attn_out_S(a.pos, CS);
   const size_t tiles = 2ull * a.S * DH * sizeof(KT);
-  const size_t all_rows = attn_out_smem(a.S, DH, sizeof(KT), a.nb) + (a.nb - 1) * tiles;
-  const bool waves = (long long)ATTN_CS * (a.kh_max > 0 ? a.kh_max : 1) > sm_count();
+  const size_t all_rows = attn_out_smem(a.S, DH, sizeof(KT), a.nb, CS) + (a.nb - 1) * tiles;
+  const bool waves = (long long)CS * (a.kh_max > 0 ? a.kh_max : 1) > sm_count();
   a.stage_rows = (all_rows <= ATTN_SMEM_MAX && !(waves && all_rows > 110 * 1024)) ? a.nb : 1;
-  const size_t smem = attn_out_smem(a.S, DH, sizeof(KT), a.nb) + (a.stage_rows - 1) * tiles;
-  auto kern = attn_out_kernel<KT, DH, ATTN_CS, NB, WV>;
+  const size_t smem = attn_out_smem(a.S, DH, sizeof(KT), a.nb, CS) + (a.stage_rows - 1) * tiles;
+  auto kern = attn_out_kernel<KT, DH, CS, NB, WV>;
   cudaError_t e = allow_smem(kern, smem);
   if (e != cudaSuccess) return e;
-  return launch_cluster(kern, dim3(ATTN_CS, a.kh_max > 0 ? a.kh_max : 1), FUSED_THREADS, smem, st, ATTN_CS, a);
+  if constexpr (CS > 8) {
+    static const cudaError_t np = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (np != cudaSuccess) return np;
+  }
+  return launch_cluster(kern, dim3(CS, a.kh_max > 0 ? a.kh_max : 1), FUSED_THREADS, smem, st, CS, a);
 }
 
 // Whole-row W^O (long rows, bf16, batch 1-2): 16-byte vectors per thread
@@ -281,7 +298,10 @@ inline int attn_out_whole_rows(int d, int E, int kvbytes, int nb) {
 template <typename KT, int DH, int NB>
 cudaError_t run_attn_out_nb(const AttnOutArgs& a, cudaStream_t st) {
   if constexpr (NB <= 2 && sizeof(KT) == 2) {
-    if (a.H_out) return run_attn_out_nbw<KT, DH, NB, ATTN_H_ONLY>(a, st);  // W^O in wo_stream_kernel
+    if (a.H_out) {  // W^O in wo_stream_kernel
+      if (attn_h_cs(a.nb) == 16) return run_attn_out_nbw<KT, DH, NB, ATTN_H_ONLY, 16>(a, st);
+      return run_attn_out_nbw<KT, DH, NB, ATTN_H_ONLY>(a, st);
+    }
     switch (attn_out_whole_rows(a.d, WT<KT>::E, sizeof(KT), a.nb)) {
       case 4: return run_attn_out_nbw<KT, DH, NB, -4>(a, st);
       case 5: return run_attn_out_nbw<KT, DH, NB, -5>(a, st);
