@@ -565,7 +565,30 @@ template <typename T, int NB>
 cudaError_t run_wo_stream_nb(const WoStreamArgs& a, cudaStream_t st) {
   const int nv = co_nv(a.d, WT<T>::E);
   const dim3 grid(sm_count());
-  DV_ST_SWITCH(wo_stream_kernel, NB, grid, st, a)
+  // ring slots: 4 at batch 1, 8 at batch 2 (DV_WO_SLOTS = 4 or 8
+  // overrides; 5 and 6 measured no better). At the OPT-175B shape the smaller ring made the look-ahead
+  // step faster at batch 1 (117.0-117.4 against 118.1-118.2 us per layer,
+  // two runs each) although the kernel alone is slower (20.5 against 19.1
+  // us with the attention); at batch 2 it was slower (250.5 against 248.9).
+  static const int env_slots = [] {
+    const char* e = std::getenv("DV_WO_SLOTS");
+    const int v = e ? std::atoi(e) : 0;
+    return (v == 4 || v == 8) ? v : 0;
+  }();
+  const int slots = env_slots ? env_slots : (a.nb == 1 ? 4 : 8);
+  auto go = [&](auto kern, int s) {
+    return launch_fused_co(kern, grid, (size_t)s * nv * CO_THREADS * 16, st, a);
+  };
+#define DV_WO_CASE(S)                                                      \
+  if (slots == S) switch (nv) {                                           \
+      case 4: return go(wo_stream_kernel<T, NB, 4, S>, S);                 \
+      case 5: return go(wo_stream_kernel<T, NB, 5, S>, S);                 \
+      default: return go(wo_stream_kernel<T, NB, 6, S>, S);                \
+    }
+  DV_WO_CASE(4)
+  DV_WO_CASE(8)
+#undef DV_WO_CASE
+  return cudaErrorInvalidValue;
 }
 #undef DV_ST_SWITCH
 

@@ -27,42 +27,43 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Ring layout: [ST_SLOTS][NV][CO_THREADS] 16-byte vectors.
-template <int NV>
+// Ring layout: [S][NV][CO_THREADS] 16-byte vectors (S slots, ST_SLOTS by
+// default).
+template <int NV, int S = ST_SLOTS>
 __device__ __forceinline__ uint4* st_vec(uint4* ring, int slot, int j) {
-  return ring + ((size_t)(slot % ST_SLOTS) * NV + j) * CO_THREADS + threadIdx.x;
+  return ring + ((size_t)(slot % S) * NV + j) * CO_THREADS + threadIdx.x;
 }
 
 // Copies this thread's vectors of `row` (null: nothing) into `slot` and
 // closes one cp.async group (empty when row is null).
-template <typename T, int NV>
+template <typename T, int NV, int S = ST_SLOTS>
 __device__ __forceinline__ void st_issue(uint4* ring, int slot, const T* row, int nvec) {
   constexpr int E = WT<T>::E;
   if (row) {
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
       const int v = j * CO_THREADS + threadIdx.x;
-      if (v < nvec) cp_async16(st_vec<NV>(ring, slot, j), row + (size_t)v * E);
+      if (v < nvec) cp_async16(st_vec<NV, S>(ring, slot, j), row + (size_t)v * E);
     }
   }
   cp_async_commit();
 }
 
 // This thread's vectors of the row in `slot` (zero past the row's end).
-template <int NV>
+template <int NV, int S = ST_SLOTS>
 __device__ __forceinline__ void st_read(uint4* ring, int slot, int nvec, uint4 (&w)[NV]) {
 #pragma unroll
   for (int j = 0; j < NV; ++j) {
     const int v = j * CO_THREADS + threadIdx.x;
-    w[j] = v < nvec ? *st_vec<NV>(ring, slot, j) : make_uint4(0u, 0u, 0u, 0u);
+    w[j] = v < nvec ? *st_vec<NV, S>(ring, slot, j) : make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
-// Issues the first ST_SLOTS - 1 rows of [r0, r1) (always ST_SLOTS - 1 groups).
-template <typename T, int NV, class RowFn>
+// Issues the first S - 1 rows of [r0, r1) (always S - 1 groups).
+template <typename T, int NV, class RowFn, int S = ST_SLOTS>
 __device__ __forceinline__ void st_prologue(uint4* ring, int r0, int r1, int nvec, RowFn row) {
 #pragma unroll 1
-  for (int s = 0; s < ST_SLOTS - 1; ++s) st_issue<T, NV>(ring, s, r0 + s < r1 ? row(r0 + s) : nullptr, nvec);
+  for (int s = 0; s < S - 1; ++s) st_issue<T, NV, S>(ring, s, r0 + s < r1 ? row(r0 + s) : nullptr, nvec);
 }
 
 // Streams rows [r0, r1) whose first ST_SLOTS - 1 were issued by st_prologue;
@@ -447,7 +448,7 @@ struct WoStreamArgs {
 
 constexpr int WO_CHUNK = 1024;  // rows whose coefficients a CTA holds at once
 
-template <typename T, int NB, int NV>
+template <typename T, int NB, int NV, int S = ST_SLOTS>
 __global__ void __launch_bounds__(CO_THREADS, 1) wo_stream_kernel(WoStreamArgs a) {
   constexpr int E = WT<T>::E;
   extern __shared__ __align__(16) uint4 s_ring[];
@@ -477,12 +478,12 @@ __global__ void __launch_bounds__(CO_THREADS, 1) wo_stream_kernel(WoStreamArgs a
   auto rowr = [&](int i) -> const T* { return row(r0 + i); };
   if (a.sets_ready) {
     range();
-    st_prologue<T, NV>(s_ring, 0, r1 - r0, nvec, rowr);
+    st_prologue<T, NV, decltype(rowr), S>(s_ring, 0, r1 - r0, nvec, rowr);
   }
   griddep_wait();
   if (!a.sets_ready) {
     range();
-    st_prologue<T, NV>(s_ring, 0, r1 - r0, nvec, rowr);
+    st_prologue<T, NV, decltype(rowr), S>(s_ring, 0, r1 - r0, nvec, rowr);
   }
   float acc[NB][NV][E];
 #pragma unroll
@@ -505,12 +506,12 @@ __global__ void __launch_bounds__(CO_THREADS, 1) wo_stream_kernel(WoStreamArgs a
     __syncthreads();
 #pragma unroll 1
     for (int i = c0; i < c0 + cn; ++i) {
-      const int ahead = i + ST_SLOTS - 1;
-      st_issue<T, NV>(s_ring, ahead, ahead < n ? rowr(ahead) : nullptr, nvec);
-      cp_async_wait<ST_SLOTS - 1>();
+      const int ahead = i + S - 1;
+      st_issue<T, NV, S>(s_ring, ahead, ahead < n ? rowr(ahead) : nullptr, nvec);
+      cp_async_wait<S - 1>();
       if (head_of(r0 + i) < 0) continue;  // a skipped row: its slot holds no data (same for every thread)
       uint4 w[NV];
-      st_read<NV>(s_ring, i, nvec, w);
+      st_read<NV, S>(s_ring, i, nvec, w);
       float cb[NB];
 #pragma unroll
       for (int b = 0; b < NB; ++b) cb[b] = s_coef[i - c0][b];
