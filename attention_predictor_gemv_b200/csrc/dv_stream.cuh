@@ -60,7 +60,7 @@ __device__ __forceinline__ void st_read(uint4* ring, int slot, int nvec, uint4 (
 }
 
 // Issues the first S - 1 rows of [r0, r1) (always S - 1 groups).
-template <typename T, int NV, class RowFn, int S = ST_SLOTS>
+template <typename T, int NV, int S = ST_SLOTS, class RowFn>
 __device__ __forceinline__ void st_prologue(uint4* ring, int r0, int r1, int nvec, RowFn row) {
 #pragma unroll 1
   for (int s = 0; s < S - 1; ++s) st_issue<T, NV, S>(ring, s, r0 + s < r1 ? row(r0 + s) : nullptr, nvec);
@@ -70,7 +70,7 @@ __device__ __forceinline__ void st_prologue(uint4* ring, int r0, int r1, int nve
 // row(i) gives row i's pointer (null: skipped). For every row and batch row
 // out(i, b, s) receives the CTA-wide dot product s of the row with the input
 // slices xr, called by one thread. red: [2][ST_RB][NB][CO_WARPS].
-template <typename T, int NB, int NV, class RowFn, class OutFn>
+template <typename T, int NB, int NV, int S = ST_SLOTS, class RowFn, class OutFn>
 __device__ __forceinline__ void st_rows_dot(uint4* ring, int r0, int r1, int nvec,
                                             const float (&xr)[NB][NV][WT<T>::E], float* red, RowFn row,
                                             OutFn out) {
@@ -79,11 +79,11 @@ __device__ __forceinline__ void st_rows_dot(uint4* ring, int r0, int r1, int nve
   const int n = r1 - r0;
 #pragma unroll 1
   for (int i = 0; i < n; ++i) {
-    const int ahead = i + ST_SLOTS - 1;
-    st_issue<T, NV>(ring, ahead, ahead < n ? row(r0 + ahead) : nullptr, nvec);
-    cp_async_wait<ST_SLOTS - 1>();
+    const int ahead = i + S - 1;
+    st_issue<T, NV, S>(ring, ahead, ahead < n ? row(r0 + ahead) : nullptr, nvec);
+    cp_async_wait<S - 1>();
     uint4 w[NV];
-    st_read<NV>(ring, i, nvec, w);
+    st_read<NV, S>(ring, i, nvec, w);
     float acc[NB];
 #pragma unroll
     for (int b = 0; b < NB; ++b) acc[b] = 0.f;
@@ -123,7 +123,7 @@ __device__ __forceinline__ void st_rows_dot(uint4* ring, int r0, int r1, int nve
 // [g n / G, (g + 1) n / G) of the n = |S_A| * 3 dh selected Q/K/V rows
 // followed by the optional rows of the next layer's predictor.
 // ----------------------------------------------------------------------------
-template <typename T, int NB, int NV>
+template <typename T, int NB, int NV, int S = ST_SLOTS>
 __global__ void __launch_bounds__(CO_THREADS, 1) attn_in_stream_kernel(AttnInArgs a) {
   constexpr int E = WT<T>::E;
   extern __shared__ __align__(16) uint4 s_ring[];
@@ -159,12 +159,12 @@ __global__ void __launch_bounds__(CO_THREADS, 1) attn_in_stream_kernel(AttnInArg
   };
   if (a.sets_ready) {
     setup();
-    st_prologue<T, NV>(s_ring, r0, r1, nvec, row);
+    st_prologue<T, NV, S>(s_ring, r0, r1, nvec, row);
   }
   griddep_wait();
   if (!a.sets_ready) {
     setup();
-    st_prologue<T, NV>(s_ring, r0, r1, nvec, row);
+    st_prologue<T, NV, S>(s_ring, r0, r1, nvec, row);
   }
   float xr[NB][NV][E];
   x_slice_load<T, NB, NV>(a.x, a.d, a.nb, xr);
@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(CO_THREADS, 1) attn_in_stream_kernel(AttnInArg
   }
   T* Kc = static_cast<T*>(a.Kc);
   T* Vc = static_cast<T*>(a.Vc);
-  st_rows_dot<T, NB, NV>(s_ring, r0, r1, nvec, xr, red, row, [&](int slot, int b, float v) {
+  st_rows_dot<T, NB, NV, S>(s_ring, r0, r1, nvec, xr, red, row, [&](int slot, int b, float v) {
     if (b >= a.nb) return;
     if (slot >= nq) {
       const int i2 = slot - nq;
@@ -238,7 +238,7 @@ __global__ void __launch_bounds__(CO_THREADS, 1) predict_a_stream_kernel(Predict
 // rows stream through the ring into the thread's own output columns, which
 // are added to x once at the end (CTA 0 also adds t1 and b2).
 // ----------------------------------------------------------------------------
-template <typename T, int NB, int NV>
+template <typename T, int NB, int NV, int S = ST_SLOTS>
 __global__ void __launch_bounds__(CO_THREADS, 1) mlp_stream_kernel(MlpBlockArgs a) {
   constexpr int E = WT<T>::E;
   extern __shared__ __align__(16) uint4 s_ring[];
@@ -276,7 +276,7 @@ __global__ void __launch_bounds__(CO_THREADS, 1) mlp_stream_kernel(MlpBlockArgs 
       s_bias[threadIdx.x] = rw >= 0 ? a.b1[rw] : 0.f;
     }
     __syncthreads();
-    st_prologue<T, NV>(s_ring, 0, cn, nvec, [&](int i) -> const T* {
+    st_prologue<T, NV, S>(s_ring, 0, cn, nvec, [&](int i) -> const T* {
       const int rw = s_row[i];
       return rw >= 0 ? W1t + (size_t)rw * a.d : nullptr;
     });
@@ -309,12 +309,12 @@ __global__ void __launch_bounds__(CO_THREADS, 1) mlp_stream_kernel(MlpBlockArgs 
     // ---- W1: partial dots of the chunk's rows ----
 #pragma unroll 1
     for (int i = 0; i < cn; ++i) {
-      const int ahead = i + ST_SLOTS - 1;
+      const int ahead = i + S - 1;
       const int rw = ahead < cn ? s_row[ahead] : -1;
-      st_issue<T, NV>(s_ring, ahead, rw >= 0 ? W1t + (size_t)rw * a.d : nullptr, nvec);
-      cp_async_wait<ST_SLOTS - 1>();
+      st_issue<T, NV, S>(s_ring, ahead, rw >= 0 ? W1t + (size_t)rw * a.d : nullptr, nvec);
+      cp_async_wait<S - 1>();
       uint4 w[NV];
-      st_read<NV>(s_ring, i, nvec, w);
+      st_read<NV, S>(s_ring, i, nvec, w);
       float d1[NB];
 #pragma unroll
       for (int b = 0; b < NB; ++b) d1[b] = 0.f;
@@ -368,14 +368,14 @@ __global__ void __launch_bounds__(CO_THREADS, 1) mlp_stream_kernel(MlpBlockArgs 
     // ---- W2: the nonzero rows into this thread's columns ----
     const int nl = s_nz;
     auto row2 = [&](int i) -> const T* { return W2t + (size_t)s_row2[i] * a.d; };
-    st_prologue<T, NV>(s_ring, 0, nl, nvec, row2);
+    st_prologue<T, NV, S>(s_ring, 0, nl, nvec, row2);
 #pragma unroll 1
     for (int i = 0; i < nl; ++i) {
-      const int ahead = i + ST_SLOTS - 1;
-      st_issue<T, NV>(s_ring, ahead, ahead < nl ? row2(ahead) : nullptr, nvec);
-      cp_async_wait<ST_SLOTS - 1>();
+      const int ahead = i + S - 1;
+      st_issue<T, NV, S>(s_ring, ahead, ahead < nl ? row2(ahead) : nullptr, nvec);
+      cp_async_wait<S - 1>();
       uint4 w[NV];
-      st_read<NV>(s_ring, i, nvec, w);
+      st_read<NV, S>(s_ring, i, nvec, w);
       float cb[NB];
 #pragma unroll
       for (int b = 0; b < NB; ++b) cb[b] = s_act2[i][b];
@@ -478,12 +478,12 @@ __global__ void __launch_bounds__(CO_THREADS, 1) wo_stream_kernel(WoStreamArgs a
   auto rowr = [&](int i) -> const T* { return row(r0 + i); };
   if (a.sets_ready) {
     range();
-    st_prologue<T, NV, decltype(rowr), S>(s_ring, 0, r1 - r0, nvec, rowr);
+    st_prologue<T, NV, S>(s_ring, 0, r1 - r0, nvec, rowr);
   }
   griddep_wait();
   if (!a.sets_ready) {
     range();
-    st_prologue<T, NV, decltype(rowr), S>(s_ring, 0, r1 - r0, nvec, rowr);
+    st_prologue<T, NV, S>(s_ring, 0, r1 - r0, nvec, rowr);
   }
   float acc[NB][NV][E];
 #pragma unroll
