@@ -540,6 +540,26 @@ cudaError_t launch_fused_co(K kern, dim3 grid, size_t smem, cudaStream_t st, con
   return launch_main(kern, grid, CO_THREADS, smem, st, a);
 }
 
+// Whether the MLP ring kernel fills its ring by bulk copies instead of
+// per-thread cp.async: at batch 1 (DV_BULK=0 or 1 overrides). Measured at the
+// OPT-175B shape: the MLP kernel alone 36.1 against 40.7 us at batch 1, but
+// 74.1 against 71.6 at batch 2; the Q/K/V kernel was slower with bulk copies
+// at both batches (30.0 against 25.2 us at batch 1), so it keeps cp.async.
+inline bool st_bulk(int nb) {
+  static const int env = [] {
+    const char* e = std::getenv("DV_BULK");
+    return !e ? -1 : (e[0] == '1' ? 1 : 0);
+  }();
+  return env >= 0 ? env == 1 : nb == 1;
+}
+
+#define DV_ST_SWITCH_BULK(KERN, NB, grid, st, a)                                              \
+  switch (nv) {                                                                              \
+    case 4: return launch_fused_co(KERN<T, NB, 4, ST_SLOTS, true>, grid, st_smem(4), st, a);  \
+    case 5: return launch_fused_co(KERN<T, NB, 5, ST_SLOTS, true>, grid, st_smem(5), st, a);  \
+    default: return launch_fused_co(KERN<T, NB, 6, ST_SLOTS, true>, grid, st_smem(6), st, a); \
+  }
+
 template <typename T, int NB>
 cudaError_t run_attn_in_st_nb(const AttnInArgs& a, cudaStream_t st) {
   const int nv = co_nv(a.d, WT<T>::E);
@@ -552,8 +572,10 @@ cudaError_t run_mlp_block_st_nb(MlpBlockArgs a, cudaStream_t st) {
   const int nv = co_nv(a.d, WT<T>::E);
   a.G = st_grid(a.k_max);
   const dim3 grid(a.G);
+  if (st_bulk(a.nb)) DV_ST_SWITCH_BULK(mlp_stream_kernel, NB, grid, st, a)
   DV_ST_SWITCH(mlp_stream_kernel, NB, grid, st, a)
 }
+#undef DV_ST_SWITCH_BULK
 
 template <typename T, int NB>
 cudaError_t run_predict_a_st_nb(const PredictAArgs& a, cudaStream_t st) {

@@ -66,6 +66,101 @@ __device__ __forceinline__ void st_prologue(uint4* ring, int r0, int r1, int nve
   for (int s = 0; s < S - 1; ++s) st_issue<T, NV, S>(ring, s, r0 + s < r1 ? row(r0 + s) : nullptr, nvec);
 }
 
+// ---- the ring filled by bulk copies (the TMA engine) ----
+// One thread issues each row as one cp.async.bulk into its slot, completing
+// on the slot's "full" barrier (count 1, transaction bytes); every warp
+// releases a slot on its "empty" barrier (count CO_WARPS) once it has read its
+// vectors, and the issuing thread waits on that before reusing the slot. The
+// slot layout is the row itself (vector v of the row at v * 16 bytes), which
+// is the per-thread layout above, so st_read serves both forms. Every wait is
+// bounded (about 2 s, DV_DEV_TIMEOUT); after a timeout the ring's waits
+// return at once, so the kernel ends with incomplete outputs.
+__device__ __forceinline__ uint32_t rb_smem(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ uint64_t rb_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ bool rb_try(uint64_t* bar, unsigned parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(rb_smem(bar)), "r"(parity)
+      : "memory");
+  return ok != 0u;
+}
+
+template <typename T, int NV, int S>
+struct BulkRing {
+  uint4* ring;      // [S][NV][CO_THREADS] 16-byte vectors
+  uint64_t* full;   // [S]
+  uint64_t* empty;  // [S]
+  int* abort;       // shared: a wait timed out
+  int* status;
+  unsigned bytes;   // bytes of a row
+  unsigned fp;      // this thread's parity of each slot's next "full" phase
+  unsigned ep;      // the issuing thread's parity of each slot's next "empty" wait
+
+  __device__ void init() {  // the caller synchronises the CTA afterwards
+    fp = 0u;
+    ep = ~0u;  // the first wait on a slot's "empty" barrier passes at once
+    if (threadIdx.x == 0) {
+      for (int s = 0; s < S; ++s) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(rb_smem(&full[s])) : "memory");
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(rb_smem(&empty[s])), "r"(CO_WARPS) : "memory");
+      }
+      *abort = 0;
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+  }
+  __device__ bool wait_bar(uint64_t* bar, unsigned parity) {
+    if (rb_try(bar, parity)) return true;
+    const uint64_t t0 = rb_ns();
+    while (!rb_try(bar, parity)) {
+      if (*reinterpret_cast<volatile int*>(abort)) return false;
+      if (rb_ns() - t0 > 2000000000ull) {
+        *reinterpret_cast<volatile int*>(abort) = 1;
+        raise_status(status, 8);
+        return false;
+      }
+    }
+    return true;
+  }
+  // Thread 0: the row of position p (null: a row with no data, which still
+  // completes the slot's phase). Every position issued is consumed once.
+  __device__ void issue(int p, const T* row) {
+    if (threadIdx.x != 0) return;
+    const int s = p % S;
+    wait_bar(&empty[s], (ep >> s) & 1u);
+    ep ^= 1u << s;
+    if (row) {
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(rb_smem(&full[s])), "r"(bytes)
+                   : "memory");
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+              rb_smem(ring + (size_t)s * NV * CO_THREADS)),
+          "l"(row), "r"(bytes), "r"(rb_smem(&full[s]))
+          : "memory");
+    } else {
+      asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(rb_smem(&full[s])) : "memory");
+    }
+  }
+  __device__ void wait(int p) {  // every thread, in position order
+    const int s = p % S;
+    wait_bar(&full[s], (fp >> s) & 1u);
+    fp ^= 1u << s;
+  }
+  __device__ void release(int p) {  // every thread, after reading position p
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(rb_smem(&empty[p % S])) : "memory");
+  }
+  template <class RowFn>
+  __device__ void prologue(int r0, int r1, RowFn row) {  // positions 0 .. S - 2 of [r0, r1)
+    for (int q = 0; q < S - 1 && r0 + q < r1; ++q) issue(q, row(r0 + q));
+  }
+};
+
 // Streams rows [r0, r1) whose first ST_SLOTS - 1 were issued by st_prologue;
 // row(i) gives row i's pointer (null: skipped). For every row and batch row
 // out(i, b, s) receives the CTA-wide dot product s of the row with the input
@@ -117,6 +212,7 @@ __device__ __forceinline__ void st_rows_dot(uint4* ring, int r0, int r1, int nve
     }
   }
 }
+
 
 // ----------------------------------------------------------------------------
 // attn_in_stream_kernel: attn_in_kernel for long rows. CTA g streams the rows
@@ -177,7 +273,7 @@ __global__ void __launch_bounds__(CO_THREADS, 1) attn_in_stream_kernel(AttnInArg
   }
   T* Kc = static_cast<T*>(a.Kc);
   T* Vc = static_cast<T*>(a.Vc);
-  st_rows_dot<T, NB, NV, S>(s_ring, r0, r1, nvec, xr, red, row, [&](int slot, int b, float v) {
+  auto out = [&](int slot, int b, float v) {
     if (b >= a.nb) return;
     if (slot >= nq) {
       const int i2 = slot - nq;
@@ -198,7 +294,8 @@ __global__ void __launch_bounds__(CO_THREADS, 1) attn_in_stream_kernel(AttnInArg
       T* cache = (m == 1) ? Kc : Vc;
       cache[(((size_t)b * a.h + head) * a.cap + a.pos) * a.dh + c] = WT<T>::store_cvt(v);
     }
-  });
+  };
+  st_rows_dot<T, NB, NV, S>(s_ring, r0, r1, nvec, xr, red, row, out);
 }
 
 // ----------------------------------------------------------------------------
@@ -238,7 +335,7 @@ __global__ void __launch_bounds__(CO_THREADS, 1) predict_a_stream_kernel(Predict
 // rows stream through the ring into the thread's own output columns, which
 // are added to x once at the end (CTA 0 also adds t1 and b2).
 // ----------------------------------------------------------------------------
-template <typename T, int NB, int NV, int S = ST_SLOTS>
+template <typename T, int NB, int NV, int S = ST_SLOTS, bool BULK = false>
 __global__ void __launch_bounds__(CO_THREADS, 1) mlp_stream_kernel(MlpBlockArgs a) {
   constexpr int E = WT<T>::E;
   extern __shared__ __align__(16) uint4 s_ring[];
@@ -253,6 +350,13 @@ __global__ void __launch_bounds__(CO_THREADS, 1) mlp_stream_kernel(MlpBlockArgs 
   const T* W2t = static_cast<const T*>(a.W2t);
   const int nvec = a.d / E;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __shared__ uint64_t s_full[BULK ? S : 1], s_empty[BULK ? S : 1];
+  __shared__ int s_abort;
+  BulkRing<T, NV, S> rb{s_ring, s_full, s_empty, &s_abort, a.status, (unsigned)nvec * 16u, 0u, 0u};
+  if constexpr (BULK) {
+    rb.init();
+    __syncthreads();
+  }
   griddep_launch();
   int j0 = 0, j1 = 0;
   auto slot_range = [&]() {
@@ -276,10 +380,12 @@ __global__ void __launch_bounds__(CO_THREADS, 1) mlp_stream_kernel(MlpBlockArgs 
       s_bias[threadIdx.x] = rw >= 0 ? a.b1[rw] : 0.f;
     }
     __syncthreads();
-    st_prologue<T, NV, S>(s_ring, 0, cn, nvec, [&](int i) -> const T* {
+    auto row1 = [&](int i) -> const T* {
       const int rw = s_row[i];
       return rw >= 0 ? W1t + (size_t)rw * a.d : nullptr;
-    });
+    };
+    if constexpr (BULK) rb.prologue(0, cn, row1);
+    else st_prologue<T, NV, S>(s_ring, 0, cn, nvec, row1);
   };
   if (a.sets_ready) {
     slot_range();
@@ -311,10 +417,17 @@ __global__ void __launch_bounds__(CO_THREADS, 1) mlp_stream_kernel(MlpBlockArgs 
     for (int i = 0; i < cn; ++i) {
       const int ahead = i + S - 1;
       const int rw = ahead < cn ? s_row[ahead] : -1;
-      st_issue<T, NV, S>(s_ring, ahead, rw >= 0 ? W1t + (size_t)rw * a.d : nullptr, nvec);
-      cp_async_wait<S - 1>();
       uint4 w[NV];
-      st_read<NV, S>(s_ring, i, nvec, w);
+      if constexpr (BULK) {
+        if (ahead < cn) rb.issue(ahead, rw >= 0 ? W1t + (size_t)rw * a.d : nullptr);
+        rb.wait(i);
+        st_read<NV, S>(s_ring, i, nvec, w);
+        rb.release(i);
+      } else {
+        st_issue<T, NV, S>(s_ring, ahead, rw >= 0 ? W1t + (size_t)rw * a.d : nullptr, nvec);
+        cp_async_wait<S - 1>();
+        st_read<NV, S>(s_ring, i, nvec, w);
+      }
       float d1[NB];
 #pragma unroll
       for (int b = 0; b < NB; ++b) d1[b] = 0.f;
@@ -368,14 +481,22 @@ __global__ void __launch_bounds__(CO_THREADS, 1) mlp_stream_kernel(MlpBlockArgs 
     // ---- W2: the nonzero rows into this thread's columns ----
     const int nl = s_nz;
     auto row2 = [&](int i) -> const T* { return W2t + (size_t)s_row2[i] * a.d; };
-    st_prologue<T, NV, S>(s_ring, 0, nl, nvec, row2);
+    if constexpr (BULK) rb.prologue(0, nl, row2);
+    else st_prologue<T, NV, S>(s_ring, 0, nl, nvec, row2);
 #pragma unroll 1
     for (int i = 0; i < nl; ++i) {
       const int ahead = i + S - 1;
-      st_issue<T, NV, S>(s_ring, ahead, ahead < nl ? row2(ahead) : nullptr, nvec);
-      cp_async_wait<S - 1>();
       uint4 w[NV];
-      st_read<NV, S>(s_ring, i, nvec, w);
+      if constexpr (BULK) {
+        if (ahead < nl) rb.issue(ahead, row2(ahead));
+        rb.wait(i);
+        st_read<NV, S>(s_ring, i, nvec, w);
+        rb.release(i);
+      } else {
+        st_issue<T, NV, S>(s_ring, ahead, ahead < nl ? row2(ahead) : nullptr, nvec);
+        cp_async_wait<S - 1>();
+        st_read<NV, S>(s_ring, i, nvec, w);
+      }
       float cb[NB];
 #pragma unroll
       for (int b = 0; b < NB; ++b) cb[b] = s_act2[i][b];
