@@ -554,8 +554,9 @@ __device__ __forceinline__ void softmax_merge(float& m, float& l, float (&acc)[E
   m = M;
 }
 
-template <typename KT, int DH, int CS, int NB, int WV>
-__global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) {
+template <typename KT, int DH, int CS, int NB, int WV, int NT = FUSED_THREADS>
+__global__ void __launch_bounds__(NT) attn_out_kernel(AttnOutArgs a) {
+  constexpr int NW = NT / 32;  // warps
   constexpr int E = WT<KT>::E;
   constexpr int G = DH / E;    // lanes per key row
   constexpr int KPW = 32 / G;  // keys per warp step
@@ -568,9 +569,9 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
   KT* sV = sK + (size_t)SR * a.S * DH;                                 // [SR][S][DH]
   float* s_all = reinterpret_cast<float*>(sV + (size_t)SR * a.S * DH);  // [nb][CS][PW]
   float* s_q = s_all + (size_t)a.nb * CS * PW;                          // [nb][DH], scaled q
-  __shared__ __align__(16) float s_w[FUSED_WARPS][PW];
+  __shared__ __align__(16) float s_w[NW][PW];
   __shared__ __align__(16) float s_H[NB][DH];
-  __shared__ float s_red[WV != 0 ? 1 : FUSED_THREADS * E];
+  __shared__ float s_red[WV != 0 ? 1 : NT * E];
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = (int)cluster.block_rank();
   const int p = blockIdx.y;
@@ -604,7 +605,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
     const size_t base = (((size_t)b * a.h + head) * a.cap + t0) * DH;
     const size_t tile = (size_t)(b % SR) * a.S * DH;
     const int v0 = lo * DH / E, v1 = hi * DH / E;
-    for (int v = v0 + tid; v < v1; v += FUSED_THREADS) {
+    for (int v = v0 + tid; v < v1; v += NT) {
       cp_async16(sK + tile + v * E, Kc + base + (size_t)v * E);
       cp_async16(sV + tile + v * E, Vc + base + (size_t)v * E);
     }
@@ -630,7 +631,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
       for (int u = 0; u < WU; ++u)
 #pragma unroll
         for (int j = 0; j < NVO; ++j) {
-          const int r = crank + u * CS, v = tid + j * FUSED_THREADS;
+          const int r = crank + u * CS, v = tid + j * NT;
           wfirst[u][j] = (r < DH && v * E < a.d) ? ld_stream(Wh + (size_t)r * a.d + (size_t)v * E)
                                                  : make_uint4(0u, 0u, 0u, 0u);
         }
@@ -639,10 +640,10 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
   auto prefetch_wo = [&]() {
     if constexpr (WV == 0) {
       const char* base = reinterpret_cast<const char*>(WO + (size_t)head * DH * a.d + c_lo);
-      for (int i = tid; i < DH; i += FUSED_THREADS) prefetch_l2(base + (size_t)i * a.d * sizeof(KT), cols * sizeof(KT));
+      for (int i = tid; i < DH; i += NT) prefetch_l2(base + (size_t)i * a.d * sizeof(KT), cols * sizeof(KT));
     } else if constexpr (WV < 0) {
       const char* base = reinterpret_cast<const char*>(WO + (size_t)head * DH * a.d);
-      for (int i = crank + tid * CS; i < DH; i += FUSED_THREADS * CS)
+      for (int i = crank + tid * CS; i < DH; i += NT * CS)
         prefetch_l2(base + (size_t)i * a.d * sizeof(KT), a.d * sizeof(KT));
     }
   };
@@ -671,12 +672,12 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
   // ---- partial attention over this CTA's keys, per batch row ----
   if (active) {
     const int g = lane % G, kq = lane / G;
-    const int KW = (nk + FUSED_WARPS - 1) / FUSED_WARPS;
+    const int KW = (nk + NW - 1) / NW;
     const int kw0 = min(nk, warp * KW), kw1 = min(nk, kw0 + KW);
     if (SR == a.nb && pos_in_chunk)
       for (int b = 0; b < a.nb; ++b) stage(b, false, true);  // slot pos of every row, written by attn_in
     // q of every batch row (written by attn_in) in one round of loads
-    for (int i = tid; i < a.nb * DH / 4; i += FUSED_THREADS) {
+    for (int i = tid; i < a.nb * DH / 4; i += NT) {
       const int b = i / (DH / 4), c4 = i % (DH / 4);
       const float4 v = __ldcg(reinterpret_cast<const float4*>(a.q + ((size_t)b * a.kh_max + p) * DH) + c4);
       reinterpret_cast<float4*>(s_q + (size_t)b * DH)[c4] =
@@ -755,17 +756,17 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
       }
       __syncthreads();
       // this CTA's partial, stored into every CTA of the cluster
-      for (int c = tid; c < PW; c += FUSED_THREADS) {
+      for (int c = tid; c < PW; c += NT) {
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < FUSED_WARPS; ++w) M = fmaxf(M, s_w[w][0]);
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, s_w[w][0]);
         float v = 0.f;
         if (M != -INFINITY) {
           if (c == 0) {
             v = M;
           } else {
 #pragma unroll
-            for (int w = 0; w < FUSED_WARPS; ++w) {
+            for (int w = 0; w < NW; ++w) {
               const float mw = s_w[w][0];
               v += (mw == -INFINITY) ? 0.f : __expf(mw - M) * s_w[w][c];
             }
@@ -782,7 +783,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
   cluster.sync();  // every partial has reached every CTA
   if (active) {
     // ---- combine the CS partials of each batch row (local shared memory) ----
-    for (int i = tid; i < a.nb * DH; i += FUSED_THREADS) {
+    for (int i = tid; i < a.nb * DH; i += NT) {
       const int b = i / DH, c = i % DH;
       const float* pb = s_all + (size_t)b * CS * PW;
       float M = -INFINITY;
@@ -802,7 +803,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
   __syncthreads();
   if constexpr (H_ONLY) {  // H of the head to global memory (CTA 0 of the cluster)
     if (active && crank == 0)
-      for (int i = tid; i < a.nb * DH; i += FUSED_THREADS)
+      for (int i = tid; i < a.nb * DH; i += NT)
         a.H_out[((size_t)(i / DH) * a.kh_max + p) * DH + i % DH] = s_H[i / DH][i % DH];
     return;
   }
@@ -866,7 +867,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
         for (int u = 0; u < U; ++u)
 #pragma unroll
           for (int j = 0; j < NVO; ++j) {
-            const int r = r0 + u * CS, v = tid + j * FUSED_THREADS;
+            const int r = r0 + u * CS, v = tid + j * NT;
             w[u][j] = (r < DH && v * E < a.d) ? ld_stream(Wh + (size_t)r * a.d + (size_t)v * E)
                                               : make_uint4(0u, 0u, 0u, 0u);
           }
@@ -875,7 +876,7 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
     }
 #pragma unroll
     for (int j = 0; j < NVO; ++j) {
-      const int c = (tid + j * FUSED_THREADS) * E;
+      const int c = (tid + j * NT) * E;
       if (c >= a.d) continue;
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
@@ -928,9 +929,9 @@ __global__ void __launch_bounds__(FUSED_THREADS) attn_out_kernel(AttnOutArgs a) 
   } else {
     // ---- W^O slice streamed: columns [c_lo, c_lo + cols) ----
     const int ncg = cols / E;
-    for (int cg0 = 0; cg0 < ncg; cg0 += FUSED_THREADS) {
-      const int ngrp = min(FUSED_THREADS, ncg - cg0);
-      const int nrg = max(1, FUSED_THREADS / ngrp);  // row groups
+    for (int cg0 = 0; cg0 < ncg; cg0 += NT) {
+      const int ngrp = min(NT, ncg - cg0);
+      const int nrg = max(1, NT / ngrp);  // row groups
       const int cgj = tid % ngrp, rgj = tid / ngrp;
       const bool thr_ok = rgj < nrg && tid < ngrp * nrg;
       const int c = c_lo + (cg0 + cgj) * E;

@@ -265,7 +265,7 @@ cudaError_t run_attn_in(const AttnInArgs& a, cudaStream_t st) {
   }
 }
 
-template <typename KT, int DH, int NB, int WV, int CS = ATTN_CS>
+template <typename KT, int DH, int NB, int WV, int CS = ATTN_CS, int NT = FUSED_THREADS>
 cudaError_t run_attn_out_nbw(AttnOutArgs a, cudaStream_t st) {
   // K/V tiles of every batch row at once when they fit, else row by row; and
   // row by row too when the grid is larger than the SMs and holding every
@@ -277,14 +277,14 @@ cudaError_t run_attn_out_nbw(AttnOutArgs a, cudaStream_t st) {
   const bool waves = (long long)CS * (a.kh_max > 0 ? a.kh_max : 1) > sm_count();
   a.stage_rows = (all_rows <= ATTN_SMEM_MAX && !(waves && all_rows > 110 * 1024)) ? a.nb : 1;
   const size_t smem = attn_out_smem(a.S, DH, sizeof(KT), a.nb, CS) + (a.stage_rows - 1) * tiles;
-  auto kern = attn_out_kernel<KT, DH, CS, NB, WV>;
+  auto kern = attn_out_kernel<KT, DH, CS, NB, WV, NT>;
   cudaError_t e = allow_smem(kern, smem);
   if (e != cudaSuccess) return e;
   if constexpr (CS > 8) {
     static const cudaError_t np = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (np != cudaSuccess) return np;
   }
-  return launch_cluster(kern, dim3(CS, a.kh_max > 0 ? a.kh_max : 1), FUSED_THREADS, smem, st, CS, a);
+  return launch_cluster(kern, dim3(CS, a.kh_max > 0 ? a.kh_max : 1), NT, smem, st, CS, a);
 }
 
 // Whole-row W^O (long rows, bf16, batch 1-2): 16-byte vectors per thread
@@ -300,6 +300,16 @@ cudaError_t run_attn_out_nb(const AttnOutArgs& a, cudaStream_t st) {
   if constexpr (NB <= 2 && sizeof(KT) == 2) {
     if (a.H_out) {  // W^O in wo_stream_kernel
       if (attn_h_cs(a.nb) == 16) return run_attn_out_nbw<KT, DH, NB, ATTN_H_ONLY, 16>(a, st);
+      // batch 1: 512 threads per CTA (16 warps over the CTA's keys: the
+      // attention is bound by issue latency at 8 warps per SM); measured at
+      // the OPT-175B shape 109.6-110.0 against 111.2 us per layer-step.
+      // DV_ATTN_NT=256 or 512 overrides.
+      static const int nt_env = [] {
+        const char* e = std::getenv("DV_ATTN_NT");
+        return !e ? 0 : (e[0] == '5' ? 512 : 256);
+      }();
+      const int nt = nt_env ? nt_env : (a.nb == 1 ? 512 : 256);
+      if (nt == 512) return run_attn_out_nbw<KT, DH, NB, ATTN_H_ONLY, ATTN_CS, 512>(a, st);
       return run_attn_out_nbw<KT, DH, NB, ATTN_H_ONLY>(a, st);
     }
     switch (attn_out_whole_rows(a.d, WT<KT>::E, sizeof(KT), a.nb)) {
