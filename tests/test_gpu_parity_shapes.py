@@ -258,3 +258,24 @@ def test_opt175b_shaped_stack_in_bench_configuration(B):
     _no_device_errors(stk.ws_main)
     _no_device_errors(stk.ws_side)
     del g
+
+
+def test_other_kernel_forms_via_environment():
+    """The kernel forms the launchers do not pick by default at these shapes,
+    chosen by their environment switches (read once per process, so in a
+    child process): the per-thread cp.async MLP ring at batch 1, the
+    256-thread attention at batch 1, the 8-slot W^O ring at batch 1 and 8-CTA
+    attention clusters at batch 2. The large-row parity tests above must pass
+    with all of them."""
+    import os
+    import subprocess
+    import sys
+
+    env = dict(os.environ, DV_BULK="0", DV_ATTN_NT="256", DV_WO_SLOTS="8", DV_ATTN_CS="8")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-m", "pytest", os.path.join(root, "tests", "test_gpu_parity_shapes.py"),
+                        "-m", "gpu", "-q", "-x", "-p", "no:cacheprovider",
+                        "-k", "large_row_lengths and 175b"],
+                       cwd=root, env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
+    assert "4 passed" in r.stdout, r.stdout[-3000:]
