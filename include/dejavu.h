@@ -352,6 +352,25 @@ DV_API dv_status dv_predict_layer_tail(const dv_layer_weights* w, const dv_dims*
                                        const dv_layer_io* out, int sets, void* ws, size_t ws_bytes,
                                        dv_stream_t stream);
 
+/* Environment switches. Each is read once per process, at the first call
+ * that needs it. The defaults are the forms measured fastest on B200; the
+ * switches exist for comparison and tuning, and every form gives the same
+ * results up to float rounding.
+ *   DV_FUSED=0     kernel-per-step layer path instead of the fused kernels
+ *   DV_TC=0        no tensor-core (tcgen05) kernels at batch >= 3
+ *   DV_TC_CTAS=1   one tensor-core CTA per SM with a 10-stage ring (default 2 x 5)
+ *   DV_STREAM=0    no shared-memory ring kernels for 16-24 KB rows
+ *   DV_WOSPLIT=0   attention and W^O in one kernel for long rows at batch 1-2
+ *   DV_BULK=0|1    MLP ring filled by per-thread cp.async (0) or bulk copies (1);
+ *                  default: bulk copies at batch 1 only
+ *   DV_WO_SLOTS=4|8  W^O ring slots (default 4 at batch 1, 8 at batch 2)
+ *   DV_ATTN_CS=8|16  CTAs per attention cluster (default 8 at batch 1, 16 at batch 2)
+ *   DV_ATTN_NT=256|512  threads per attention CTA (default 512 at batch 1)
+ *   DV_PB_CTAS=n   CTAs of the batch-1/2 neuron-score kernel (default 4 per SM)
+ *   DV_SELROWS=0   one-CTA-per-row selection instead of the cluster selection
+ *   DV_PDL=0       no programmatic dependent launch
+ *   DV_PRIO=0      no launch priority for the critical-path kernels */
+
 /* L2 prefetch of one layer's selected parameters (§1: for the next layer
  * the look-ahead predictor picks the heads / neurons and only those
  * parameters are loaded). Given the sets `sel` (head_idx/head_count and
