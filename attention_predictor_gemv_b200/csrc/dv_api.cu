@@ -432,19 +432,43 @@ bool fused_ok(const dv_dims& D, dv_dtype wdt) {
 
 // Second half of the fused predictor: neuron scores from z (in ws) and the
 // selections; the head scores sh must be complete when heads is set.
+// The smallest batch whose look-ahead neuron scores z B^T + b1 run on the
+// tensor cores (tc_dense_kernel) in the fused path; below it predict_b_kernel
+// (DV_PB_TC_MIN_B overrides; 17 keeps predict_b_kernel at every batch). At
+// the OPT-175B shape the tensor-core form made the look-ahead step faster at
+// batch 1 (106.2 against 110.0 us per layer) and batch 2 (212.2 against
+// 247.2), although alone it is no faster at batch 1 (49.7 against 46.9 us
+// with the selection): its CTAs share the SMs with the main kernels better.
+int pb_tc_min_batch() {
+  static const int b = [] {
+    const char* e = std::getenv("DV_PB_TC_MIN_B");
+    const int v = e ? std::atoi(e) : 0;
+    return v > 0 ? v : 1;
+  }();
+  return b;
+}
+
 dv_status fused_predict_rest(const Layout& L, void* ws, const dv_layer_weights* w, const dv_dims& D,
                              const dv_layer_params* p, bool heads, bool neurons, float* sh, int32_t* hidx,
                              int32_t* hcnt, float* sm, int32_t* midx, int32_t* mcnt, cudaStream_t st) {
   if (neurons) {
-    PredictBArgs b = {};
-    b.z = at<float>(ws, L.z);
-    b.Bm = w->Bm;
-    b.b1 = w->b1;
-    b.N = D.N;
-    b.r = D.r;
-    b.nb = D.B;
-    b.scores = sm;
-    DV_TRY(run_predict_b_dt(w->wdtype, b, st));
+    // large predictors only: at the OPT-1.3B and OPT-6.7B shapes (B of 4 and
+    // 17 MB) the tensor-core form made the step slower (by 2-6 and 1 us per
+    // layer); from the OPT-66B shape (75 MB) on it made it faster
+    const bool large = (long long)D.N * D.r >= (16ll << 20);
+    if (large && D.B >= pb_tc_min_batch() && tc_enabled() && tc_dense_ok(D.B, wbytes_of(w->wdtype), D.N, D.r)) {
+      DV_TRY(pred_tc(L, ws, w->Bm, D.N, D.r, w->b1, at<float>(ws, L.z), D.B, sm, D.N, st));
+    } else {
+      PredictBArgs b = {};
+      b.z = at<float>(ws, L.z);
+      b.Bm = w->Bm;
+      b.b1 = w->b1;
+      b.N = D.N;
+      b.r = D.r;
+      b.nb = D.B;
+      b.scores = sm;
+      DV_TRY(run_predict_b_dt(w->wdtype, b, st));
+    }
     DV_TRY(select_any(sm, D.B, D.N, p->k, p->tau, p->mode, at<uint32_t>(ws, L.bm_m), at<unsigned>(ws, L.pb_ticket),
                       midx, mcnt, st));
   }
