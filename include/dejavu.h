@@ -367,6 +367,9 @@ DV_API dv_status dv_predict_layer_tail(const dv_layer_weights* w, const dv_dims*
  *   DV_ATTN_CS=8|16  CTAs per attention cluster (default 8 at batch 1, 16 at batch 2)
  *   DV_ATTN_NT=256|512  threads per attention CTA (default 512 at batch 1)
  *   DV_PB_CTAS=n   CTAs of the batch-1/2 neuron-score kernel (default 4 per SM)
+ *   DV_PB_TC_MIN_B=n  smallest batch whose look-ahead neuron scores of a large
+ *                  predictor (N r >= 16M) run on the tensor cores (default 1;
+ *                  17: never)
  *   DV_SELROWS=0   one-CTA-per-row selection instead of the cluster selection
  *   DV_PDL=0       no programmatic dependent launch
  *   DV_PRIO=0      no launch priority for the critical-path kernels */
